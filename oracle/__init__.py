@@ -1,0 +1,16 @@
+"""fp64 CPU oracle of the Mamba selective scan and selective state update.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
+benchmark's CPU-baseline leg, never by the product package. It shares no code
+with the CUDA path. See ``mamba_oracle.c`` for what it computes and which
+passage of the Mamba pages each step follows.
+"""
+from .oracle import (  # noqa: F401
+    build_oracle,
+    load_oracle,
+    scan,
+    scan_mt,
+    state_update,
+    softplus,
+    silu,
+)

@@ -1,0 +1,264 @@
+/*
+ * mamba_oracle.c -- fp64 CPU oracle of the Mamba selective scan and of the
+ * single-token selective state update.
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may link, load or call
+ * this file: only the tests, the smoke check and the benchmark's CPU-baseline
+ * leg use it. It shares no code, header, table or constant with the CUDA path.
+ *
+ * What it computes (sources are the web pages on Mamba this project follows):
+ *  - "Mamba (deep learning)" wiki page, paragraph on state space models: the
+ *    discretised transition is A_bar = exp(Delta*A), applied per state.
+ *  - "Mamba-1/2/3 Markdown図解" blog, section 1 (数式で見ると): the recurrence
+ *    h_t = A_bar_t h_{t-1} + B_bar_t x_t and the readout y_t = C_t h_t.
+ *  - Same blog, section 2 (Mamba-1): Delta_t, B_t, C_t are per-token inputs
+ *    (selectivity); the block gates the SSM output with a second branch.
+ *  - The input term B_bar_t x_t is taken as Delta_t * B_t * u_t (Euler form of
+ *    the input; the pages lost that equation), Delta_t = softplus(delta_t +
+ *    bias_d) when the softplus flag is set, the D skip sits inside the gate,
+ *    and the gate is silu(z) = z * sigmoid(z). These are the readings this
+ *    project fixes for steps the pages leave open.
+ *  - Generation is the same recurrence taken one token at a time from a stored
+ *    state (blog, section 2, "1トークン生成 → recurrent update").
+ *
+ * Layouts (all arrays dense, row-major, fp64):
+ *   u, delta, z, y      [batch][dim][seqlen]
+ *   A                   [dim][dstate]
+ *   B, C                [batch][dstate][seqlen]   (one group shared by all dim)
+ *   D, delta_bias       [dim]
+ *   h0, last_state      [batch][dim][dstate]
+ *   decode: x, delta, z, y [batch][dim]; B, C [batch][dstate]; state [batch][dim][dstate]
+ * Nullable: D, z, delta_bias, h0 (zero initial state), last_state.
+ *
+ * Built with -O2 and no fast-math; exp/log1p are the C library's.
+ * ORACLE_MUTANT (compile-time, tests only) plants one known mistake so that a
+ * test can show the pins catch it; the default build plants none.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <pthread.h>
+
+#ifndef ORACLE_MUTANT
+#define ORACLE_MUTANT 0
+#endif
+
+/* softplus(x) = log(1 + e^x), written so that neither branch overflows. */
+double oracle_softplus(double x)
+{
+    double ax = fabs(x);
+    return (x > 0.0 ? x : 0.0) + log1p(exp(-ax));
+}
+
+/* silu(z) = z * sigmoid(z) = z / (1 + e^-z). */
+double oracle_silu(double z)
+{
+#if ORACLE_MUTANT == 8
+    return 1.0 / (1.0 + exp(-z)); /* mutant: sigmoid gate instead of silu */
+#else
+    return z / (1.0 + exp(-z));
+#endif
+}
+
+/* Delta_t from the raw per-token value: bias added first, then softplus. */
+static double step_size(double raw, double bias, int softplus_flag)
+{
+#if ORACLE_MUTANT == 7
+    (void)bias;
+    double v = raw; /* mutant: bias dropped */
+#else
+    double v = raw + bias;
+#endif
+#if ORACLE_MUTANT == 6
+    (void)softplus_flag;
+    return v; /* mutant: softplus never applied */
+#else
+    return softplus_flag ? oracle_softplus(v) : v;
+#endif
+}
+
+/*
+ * One channel (b, d) over tokens [0, L): the recurrence of the blog's
+ * section 1 with A_bar = exp(Delta*A) (wiki page) per state n, readout C.h,
+ * D skip, then the silu(z) gate. h (length N) is the running state: on entry
+ * the initial state, on exit the state after token L-1.
+ * Strides: u/delta/z/y step 1 per token; B/C: element (n, t) at n*bc_sn + t.
+ */
+static void scan_channel(int64_t N, int64_t L,
+                         const double *u, const double *delta, const double *A_d,
+                         const double *B, const double *C, int64_t bc_sn,
+                         const double *D_d, const double *z, const double *bias_d,
+                         int softplus_flag, double *h, double *y)
+{
+    for (int64_t t = 0; t < L; ++t) {
+        double dt = step_size(delta[t], bias_d ? *bias_d : 0.0, softplus_flag);
+        double acc = 0.0;
+        for (int64_t n = 0; n < N; ++n) {
+#if ORACLE_MUTANT == 10
+            double A_n = A_d[N - 1 - n]; /* mutant: state index reversed in A */
+#else
+            double A_n = A_d[n];
+#endif
+#if ORACLE_MUTANT == 2
+            double abar = exp(-dt * A_n); /* mutant: wrong sign in the exponent */
+#else
+            double abar = exp(dt * A_n);
+#endif
+#if ORACLE_MUTANT == 3
+            double bx = u[t] * B[n * bc_sn + t]; /* mutant: Delta dropped from the input term */
+#elif ORACLE_MUTANT == 5
+            double bx = dt * u[t] * C[n * bc_sn + t]; /* mutant: B and C swapped */
+#elif ORACLE_MUTANT == 9
+            double bx = dt * u[t] * (t > 0 ? B[n * bc_sn + t - 1] : 0.0); /* mutant: B one token late */
+#else
+            double bx = dt * u[t] * B[n * bc_sn + t];
+#endif
+#if ORACLE_MUTANT == 4
+            acc += (ORACLE_MUTANT == 5 ? B : C)[n * bc_sn + t] * h[n]; /* mutant: readout before update */
+            h[n] = abar * h[n] + bx;
+#else
+            h[n] = abar * h[n] + bx;
+#if ORACLE_MUTANT == 5
+            acc += B[n * bc_sn + t] * h[n];
+#else
+            acc += C[n * bc_sn + t] * h[n];
+#endif
+#endif
+        }
+#if ORACLE_MUTANT == 1
+        double yv = acc; /* mutant: D skip dropped */
+#else
+        double yv = acc + (D_d ? *D_d : 0.0) * u[t];
+#endif
+        if (z) yv *= oracle_silu(z[t]);
+        y[t] = yv;
+    }
+}
+
+/* Scan over channels [c0, c1) of the flattened (batch, dim) range. */
+static void scan_range(int64_t c0, int64_t c1, int64_t batch, int64_t dim, int64_t N, int64_t L,
+                       const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *z, const double *delta_bias, int softplus_flag,
+                       const double *h0, double *y, double *last_state)
+{
+    (void)batch;
+    double *h = (double *)malloc((size_t)N * sizeof(double));
+    if (!h) return;
+    for (int64_t c = c0; c < c1; ++c) {
+        int64_t b = c / dim, d = c % dim;
+        for (int64_t n = 0; n < N; ++n) h[n] = h0 ? h0[c * N + n] : 0.0;
+        const int64_t row = c * L;
+        scan_channel(N, L, u + row, delta + row, A + d * N,
+                     B + b * N * L, C + b * N * L, L,
+                     D ? D + d : NULL, z ? z + row : NULL,
+                     delta_bias ? delta_bias + d : NULL, softplus_flag, h, y + row);
+#if ORACLE_MUTANT == 12
+        (void)last_state; /* mutant: final state never written */
+#else
+        if (last_state)
+            for (int64_t n = 0; n < N; ++n) last_state[c * N + n] = h[n];
+#endif
+    }
+    free(h);
+}
+
+/*
+ * Selective scan over a whole batch. Returns 0, or -1 on a bad size or a
+ * missing required array.
+ */
+int oracle_scan_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                    const double *u, const double *delta, const double *A,
+                    const double *B, const double *C, const double *D,
+                    const double *z, const double *delta_bias, int softplus_flag,
+                    const double *h0, double *y, double *last_state)
+{
+    if (batch < 0 || dim < 0 || dstate < 1 || seqlen < 0) return -1;
+    if (batch * dim * seqlen > 0 && (!u || !delta || !A || !B || !C || !y)) return -1;
+    scan_range(0, batch * dim, batch, dim, dstate, seqlen, u, delta, A, B, C, D, z,
+               delta_bias, softplus_flag, h0, y, last_state);
+    return 0;
+}
+
+struct mt_job {
+    int64_t c0, c1, batch, dim, N, L;
+    const double *u, *delta, *A, *B, *C, *D, *z, *bias, *h0;
+    int flag;
+    double *y, *last;
+};
+
+static void *mt_worker(void *p)
+{
+    struct mt_job *j = (struct mt_job *)p;
+    scan_range(j->c0, j->c1, j->batch, j->dim, j->N, j->L, j->u, j->delta, j->A, j->B,
+               j->C, j->D, j->z, j->bias, j->flag, j->h0, j->y, j->last);
+    return NULL;
+}
+
+/*
+ * Same result as oracle_scan_f64; the independent (batch, dim) channels are
+ * split over nthreads POSIX threads. The per-channel arithmetic is unchanged.
+ */
+int oracle_scan_f64_mt(int nthreads, int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                       const double *u, const double *delta, const double *A,
+                       const double *B, const double *C, const double *D,
+                       const double *z, const double *delta_bias, int softplus_flag,
+                       const double *h0, double *y, double *last_state)
+{
+    if (nthreads <= 1)
+        return oracle_scan_f64(batch, dim, dstate, seqlen, u, delta, A, B, C, D, z,
+                               delta_bias, softplus_flag, h0, y, last_state);
+    if (batch < 0 || dim < 0 || dstate < 1 || seqlen < 0) return -1;
+    int64_t nch = batch * dim;
+    if (nch * seqlen > 0 && (!u || !delta || !A || !B || !C || !y)) return -1;
+    if (nthreads > 256) nthreads = 256;
+    pthread_t th[256];
+    struct mt_job jobs[256];
+    int started = 0;
+    for (int i = 0; i < nthreads; ++i) {
+        struct mt_job j = {nch * i / nthreads, nch * (i + 1) / nthreads, batch, dim, dstate, seqlen,
+                           u, delta, A, B, C, D, z, delta_bias, h0, softplus_flag, y, last_state};
+        jobs[i] = j;
+        if (pthread_create(&th[i], NULL, mt_worker, &jobs[i]) == 0) {
+            ++started;
+        } else {
+            mt_worker(&jobs[i]); /* could not start a thread: do this share here */
+            th[i] = 0;
+        }
+    }
+    for (int i = 0; i < nthreads; ++i)
+        if (th[i]) pthread_join(th[i], NULL);
+    (void)started;
+    return 0;
+}
+
+/*
+ * Single-token selective state update for a batch: for every (b, d) one step
+ * of the recurrence from the stored state, which is read and overwritten.
+ * x is the token input (u in the scan's notation).
+ */
+int oracle_state_update_f64(int64_t batch, int64_t dim, int64_t dstate,
+                            double *state, const double *x, const double *delta,
+                            const double *A, const double *B, const double *C,
+                            const double *D, const double *z, const double *delta_bias,
+                            int softplus_flag, double *y)
+{
+    if (batch < 0 || dim < 0 || dstate < 1) return -1;
+    if (batch * dim > 0 && (!state || !x || !delta || !A || !B || !C || !y)) return -1;
+    const int64_t N = dstate;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            int64_t c = b * dim + d;
+#if ORACLE_MUTANT == 11
+            for (int64_t n = 0; n < N; ++n) state[c * N + n] = 0.0; /* mutant: stored state ignored */
+#endif
+            /* One token: the same per-channel step as the scan with L = 1; B/C
+               for this batch row hold one value per state (stride 1 in n). */
+            scan_channel(N, 1, x + c, delta + c, A + d * N, B + b * N, C + b * N, 1,
+                         D ? D + d : NULL, z ? z + c : NULL,
+                         delta_bias ? delta_bias + d : NULL, softplus_flag,
+                         state + c * N, y + c);
+        }
+    }
+    return 0;
+}

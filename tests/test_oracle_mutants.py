@@ -1,0 +1,48 @@
+"""The pins must catch plausible oracle mistakes.
+
+Each mutant build of the oracle (compiled with ORACLE_MUTANT=k into a
+temporary directory) plants one mistake: a dropped term, a wrong sign, a
+wrong or shifted index, swapped operands, a missing step. For every mutant at
+least one pin of ``test_oracle_pins`` must fail; the real oracle passes them
+all (checked there).
+"""
+import numpy as np
+import pytest
+
+import oracle.oracle as ow
+from test_oracle_pins import PINS, TOL
+
+MUTANTS = {
+    1: "D skip dropped",
+    2: "wrong sign in exp(Delta*A)",
+    3: "Delta dropped from the input term",
+    4: "readout taken before the state update",
+    5: "B and C swapped",
+    6: "softplus never applied",
+    7: "delta bias dropped",
+    8: "sigmoid gate instead of silu",
+    9: "B read one token late",
+    10: "state index reversed in A",
+    11: "decode ignores the stored state",
+    12: "final state never written",
+}
+
+
+@pytest.fixture(scope="module")
+def mutant_dir(tmp_path_factory):
+    return str(tmp_path_factory.mktemp("oracle_mutants"))
+
+
+@pytest.mark.parametrize("mutant", sorted(MUTANTS))
+def test_some_pin_catches_mutant(mutant, mutant_dir):
+    lib = ow.mutant_library(mutant, mutant_dir)
+    caught = []
+    for name, pin in PINS.items():
+        with np.errstate(all="ignore"):
+            try:
+                err = pin(lib)
+            except Exception:  # a crash or an assertion inside a pin also counts
+                err = float("inf")
+        if not (err <= TOL):
+            caught.append(name)
+    assert caught, f"no pin caught mutant {mutant} ({MUTANTS[mutant]})"

@@ -1,0 +1,300 @@
+"""Pins of the fp64 oracle to facts that do not come from the oracle itself.
+
+Each pin is an independent formulation of something the Mamba pages (or plain
+mathematics) fix, written without the oracle's code:
+
+* time-invariant case == one long convolution ('Mamba (deep learning)' wiki
+  page, state-space paragraph: constant A, B, C, Delta make the model an LTI
+  convolution), kernel K_k = sum_n C_n A_bar_n^k Delta B_n, by direct O(L^2) sum;
+* d_state = 1 closed form with cumulative step sums S_t (A_bar = exp(Delta*A),
+  same paragraph, composed over tokens);
+* zero input: the state only decays, h_k = h_0 * exp(A * sum_j Delta_j);
+* brute force: h_T = sum_s (prod_{r>s} A_bar_r) B_bar_s u_s with explicit
+  products, against the recurrence of the 'Mamba-1/2/3 Markdown図解' blog,
+  section 1;
+* decode == scan (blog, section 2: train/prefill by scan and one-token
+  generation by recurrent update are the same model) and split/resume (only
+  the state is carried between tokens);
+* degenerate cases: B = 0, and Delta = 0 (A_bar = 1);
+* softplus / silu special values and library routines (numpy logaddexp,
+  scipy expit);
+* the hand-worked cases in tests/golden/hand_worked.json.
+
+``test_oracle_mutants.py`` plants known mistakes in the oracle and checks
+that at least one of these pins fails for each.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+from scipy.special import expit
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+TOL = 1e-12
+
+
+def _rel(a, b):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    scale = max(np.max(np.abs(b)), 1e-300)
+    return float(np.max(np.abs(a - b)) / scale)
+
+
+def _softplus_ref(x):
+    return np.logaddexp(0.0, x)
+
+
+def _silu_ref(z):
+    return z * expit(z)
+
+
+# ---------------------------------------------------------------- pins ----
+
+def pin_softplus_silu(lib):
+    errs = []
+    errs.append(abs(oracle.softplus(0.0, lib) - math.log(2.0)))
+    for x in (-30.0, -3.5, -0.25, 0.7, 4.0, 19.0, 40.0):
+        errs.append(abs(oracle.softplus(x, lib) - oracle.softplus(-x, lib) - x) / max(1.0, abs(x)))
+        errs.append(abs(oracle.softplus(x, lib) - _softplus_ref(x)) / _softplus_ref(x))
+        errs.append(abs(oracle.silu(x, lib) - oracle.silu(-x, lib) - x) / max(1.0, abs(x)))
+        errs.append(abs(oracle.silu(x, lib) - _silu_ref(x)) / max(abs(_silu_ref(x)), 1e-300))
+    errs.append(abs(oracle.silu(0.0, lib)))
+    return max(errs)
+
+
+def pin_lti_convolution(lib):
+    rng = np.random.default_rng(11)
+    b, d, N, L = 2, 3, 5, 40
+    A = -rng.uniform(0.2, 3.0, size=(d, N))
+    Bc = rng.standard_normal((b, N))
+    Cc = rng.standard_normal((b, N))
+    dt = rng.uniform(0.05, 0.5, size=(b, d))
+    u = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    D = rng.standard_normal(d)
+    delta = np.repeat(dt[:, :, None], L, axis=2)
+    B = np.repeat(Bc[:, :, None], L, axis=2)
+    C = np.repeat(Cc[:, :, None], L, axis=2)
+    worst = 0.0
+    for with_gate in (False, True):
+        y, _ = oracle.scan(u, delta, A, B, C, D if with_gate else None, z if with_gate else None,
+                           np.zeros(d), False, lib=lib)
+        ref = np.empty_like(y)
+        for bi in range(b):
+            for di in range(d):
+                k = np.arange(L)
+                K = np.zeros(L)
+                for n in range(N):
+                    K += Cc[bi, n] * np.exp(dt[bi, di] * A[di, n]) ** k * dt[bi, di] * Bc[bi, n]
+                conv = np.convolve(u[bi, di], K)[:L]
+                if with_gate:
+                    conv = (conv + D[di] * u[bi, di]) * _silu_ref(z[bi, di])
+                ref[bi, di] = conv
+        worst = max(worst, _rel(y, ref))
+    return worst
+
+
+def pin_n1_closed_form(lib):
+    rng = np.random.default_rng(12)
+    b, d, L = 2, 3, 50
+    A = -rng.uniform(0.3, 2.0, size=(d, 1))
+    u = rng.standard_normal((b, d, L))
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    B = rng.standard_normal((b, 1, L))
+    C = rng.standard_normal((b, 1, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-2.0, 0.5, size=d)
+    y, last = oracle.scan(u, raw, A, B, C, D, z, bias, True, lib=lib)
+    ref = np.empty_like(y)
+    ref_last = np.empty_like(last)
+    for bi in range(b):
+        for di in range(d):
+            dt = _softplus_ref(raw[bi, di] + bias[di])
+            S = np.cumsum(dt)
+            for t in range(L):
+                s = np.arange(t + 1)
+                h = np.sum(np.exp(A[di, 0] * (S[t] - S[s])) * dt[s] * B[bi, 0, s] * u[bi, di, s])
+                ref[bi, di, t] = (C[bi, 0, t] * h + D[di] * u[bi, di, t]) * _silu_ref(z[bi, di, t])
+                if t == L - 1:
+                    ref_last[bi, di, 0] = h
+    return max(_rel(y, ref), _rel(last, ref_last))
+
+
+def pin_zero_input_decay(lib):
+    rng = np.random.default_rng(13)
+    b, d, N, K = 2, 4, 6, 25
+    A = -rng.uniform(0.1, 4.0, size=(d, N))
+    h0 = rng.standard_normal((b, d, N))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-3.0, 0.0, size=d)
+    h = h0.copy()
+    S = np.zeros((b, d))
+    worst = 0.0
+    for k in range(K):
+        raw = rng.standard_normal((b, d))
+        z = rng.standard_normal((b, d))
+        B = rng.standard_normal((b, N))
+        C = rng.standard_normal((b, N))
+        y, h = oracle.state_update(h, np.zeros((b, d)), raw, A, B, C, D, z, bias, True, lib=lib)
+        S += _softplus_ref(raw + bias)
+        h_ref = h0 * np.exp(A[None, :, :] * S[:, :, None])
+        y_ref = np.einsum("bn,bdn->bd", C, h_ref) * _silu_ref(z)
+        worst = max(worst, _rel(h, h_ref), _rel(y, y_ref))
+    return worst
+
+
+def pin_brute_force_products(lib):
+    rng = np.random.default_rng(14)
+    b, d, N, L = 1, 2, 3, 12
+    A = -rng.uniform(0.1, 2.5, size=(d, N))
+    u = rng.standard_normal((b, d, L))
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    B = rng.standard_normal((b, N, L))
+    C = rng.standard_normal((b, N, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-1.0, 1.0, size=d)
+    y, last = oracle.scan(u, raw, A, B, C, D, z, bias, True, lib=lib)
+    ref = np.zeros_like(y)
+    ref_last = np.zeros_like(last)
+    for di in range(d):
+        dt = [math.log1p(math.exp(raw[0, di, t] + bias[di])) for t in range(L)]
+        for T in range(L):
+            acc = 0.0
+            for n in range(N):
+                hT = 0.0
+                for s in range(T + 1):
+                    prod = 1.0
+                    for r in range(s + 1, T + 1):
+                        prod *= math.exp(dt[r] * A[di, n])
+                    hT += prod * dt[s] * B[0, n, s] * u[0, di, s]
+                acc += C[0, n, T] * hT
+                if T == L - 1:
+                    ref_last[0, di, n] = hT
+            zz = z[0, di, T]
+            ref[0, di, T] = (acc + D[di] * u[0, di, T]) * zz / (1.0 + math.exp(-zz))
+    return max(_rel(y, ref), _rel(last, ref_last))
+
+
+def pin_scan_equals_decode(lib):
+    rng = np.random.default_rng(15)
+    b, d, N, L = 2, 3, 4, 30
+    A = -rng.uniform(0.1, 3.0, size=(d, N))
+    u = rng.standard_normal((b, d, L))
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    B = rng.standard_normal((b, N, L))
+    C = rng.standard_normal((b, N, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-2.0, 0.0, size=d)
+    y, last = oracle.scan(u, raw, A, B, C, D, z, bias, True, lib=lib)
+    h = np.zeros((b, d, N))
+    ys = []
+    for t in range(L):
+        yt, h = oracle.state_update(h, u[:, :, t], raw[:, :, t], A, B[:, :, t], C[:, :, t], D,
+                                    z[:, :, t], bias, True, lib=lib)
+        ys.append(yt)
+    return max(_rel(np.stack(ys, axis=2), y), _rel(h, last))
+
+
+def pin_split_resume(lib):
+    rng = np.random.default_rng(16)
+    b, d, N, L, m = 2, 3, 4, 40, 17
+    A = -rng.uniform(0.1, 3.0, size=(d, N))
+    u = rng.standard_normal((b, d, L))
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    B = rng.standard_normal((b, N, L))
+    C = rng.standard_normal((b, N, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-2.0, 0.0, size=d)
+    y, last = oracle.scan(u, raw, A, B, C, D, z, bias, True, lib=lib)
+    y1, h1 = oracle.scan(u[:, :, :m], raw[:, :, :m], A, B[:, :, :m], C[:, :, :m], D, z[:, :, :m],
+                         bias, True, lib=lib)
+    y2, h2 = oracle.scan(u[:, :, m:], raw[:, :, m:], A, B[:, :, m:], C[:, :, m:], D, z[:, :, m:],
+                         bias, True, h0=h1, lib=lib)
+    return max(_rel(np.concatenate([y1, y2], axis=2), y), _rel(h2, last))
+
+
+def pin_degenerate(lib):
+    rng = np.random.default_rng(17)
+    b, d, N, L = 2, 3, 4, 20
+    A = -rng.uniform(0.1, 3.0, size=(d, N))
+    u = rng.standard_normal((b, d, L))
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    C = rng.standard_normal((b, N, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-2.0, 0.0, size=d)
+    # B = 0: nothing is written into the state.
+    y, last = oracle.scan(u, raw, A, np.zeros((b, N, L)), C, D, z, bias, True, lib=lib)
+    e1 = max(_rel(y, D[None, :, None] * u * _silu_ref(z)), float(np.max(np.abs(last))))
+    # Delta = 0 (softplus off, raw = -bias): A_bar = 1 and the input term is 0,
+    # so the state keeps h0 and y_t = C_t . h0 + D u_t, gated.
+    h0 = rng.standard_normal((b, d, N))
+    Bn = rng.standard_normal((b, N, L))
+    raw0 = np.repeat(-bias[None, :, None], b, axis=0).repeat(L, axis=2)
+    y, last = oracle.scan(u, raw0, A, Bn, C, D, z, bias, False, h0=h0, lib=lib)
+    y_ref = (np.einsum("bnt,bdn->bdt", C, h0) + D[None, :, None] * u) * _silu_ref(z)
+    e2 = max(_rel(y, y_ref), _rel(last, h0))
+    return max(e1, e2)
+
+
+def pin_hand_worked(lib):
+    with open(os.path.join(HERE, "golden", "hand_worked.json")) as f:
+        cases = json.load(f)["cases"]
+    worst = 0.0
+    for c in cases:
+        arr = {k: (None if c[k] is None else np.array(c[k], dtype=np.float64))
+               for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")}
+        y, last = oracle.scan(arr["u"], arr["delta"], arr["A"], arr["B"], arr["C"], arr["D"],
+                              arr["z"], arr["delta_bias"], c["softplus"], lib=lib)
+        if "y_over_ln2" in c:
+            y_ref = np.array(c["y_over_ln2"]) * math.log(2.0)
+        else:
+            y_ref = np.array(c["y_over_ln3"]) * math.log(3.0)
+        last_ref = np.array(c["last_state_over_ln2"]) * math.log(2.0)
+        worst = max(worst, float(np.max(np.abs(y - y_ref))), float(np.max(np.abs(last - last_ref))))
+    return worst
+
+
+PINS = {
+    "softplus_silu": pin_softplus_silu,
+    "lti_convolution": pin_lti_convolution,
+    "n1_closed_form": pin_n1_closed_form,
+    "zero_input_decay": pin_zero_input_decay,
+    "brute_force_products": pin_brute_force_products,
+    "scan_equals_decode": pin_scan_equals_decode,
+    "split_resume": pin_split_resume,
+    "degenerate": pin_degenerate,
+    "hand_worked": pin_hand_worked,
+}
+
+
+@pytest.mark.parametrize("name", sorted(PINS))
+def test_pin(name, oracle_lib):
+    err = PINS[name](oracle_lib)
+    assert err <= TOL, f"pin {name}: error {err:.3e} > {TOL:.0e}"
+
+
+def test_multithreaded_oracle_is_identical(oracle_lib):
+    rng = np.random.default_rng(21)
+    b, d, N, L = 3, 7, 5, 33
+    args = (rng.standard_normal((b, d, L)), rng.standard_normal((b, d, L)),
+            -rng.uniform(0.1, 3, (d, N)), rng.standard_normal((b, N, L)),
+            rng.standard_normal((b, N, L)), rng.standard_normal(d),
+            rng.standard_normal((b, d, L)), rng.uniform(-2, 0, d))
+    y1, h1 = oracle.scan(*args, lib=oracle_lib)
+    y4, h4 = oracle.scan_mt(4, *args, lib=oracle_lib)
+    assert np.array_equal(y1, y4) and np.array_equal(h1, h4)
+
+
+def test_oracle_rejects_bad_sizes(oracle_lib):
+    dp = None
+    assert oracle_lib.oracle_scan_f64(1, 1, 0, 4, *([dp] * 8), 1, dp, dp, dp) == -1
+    assert oracle_lib.oracle_scan_f64(1, 1, 4, 4, *([dp] * 8), 1, dp, dp, dp) == -1

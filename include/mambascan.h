@@ -1,0 +1,188 @@
+/*
+ * mambascan.h -- C ABI of libmambascan.so: the Mamba selective scan (forward)
+ * and the single-token selective state update, as hand-written CUDA for
+ * NVIDIA B200 (sm_100a).
+ *
+ * What is computed. For every batch row b and channel d, with Delta_t the step
+ * size of token t:
+ *     Delta_t = softplus(delta[b,d,t] + delta_bias[d])   (plain sum when the
+ *                                                         softplus flag is 0)
+ *     A_bar   = exp(Delta_t * A[d,n])                     per state n
+ *     h_t[n]  = A_bar * h_{t-1}[n] + Delta_t * B[b,n,t] * u[b,d,t]
+ *     y[b,d,t] = (sum_n C[b,n,t] * h_t[n] + D[d] * u[b,d,t]) * silu(z[b,d,t])
+ * with silu(z) = z * sigmoid(z). Sources: the 'Mamba (deep learning)' wiki
+ * page, paragraph on state space models (A_bar = exp(Delta*A); Delta, B, C made
+ * functions of the input), and the 'Mamba-1/2/3 Markdown図解' blog, section 1
+ * (h_t = A_bar_t h_{t-1} + B_bar_t x_t, y_t = C_t h_t) and section 2 (the block
+ * gates the SSM output with a second branch; training/prefill runs the scan
+ * while one-token generation runs the recurrent update of the same model).
+ * The input term B_bar_t x_t is read as Delta_t * B_t * u_t, the bias is added
+ * before softplus, and D is applied inside the gate: the pages leave those
+ * steps open and this library fixes that reading.
+ *
+ * Conventions common to every entry point:
+ *  - All array pointers are device pointers owned by the caller. The library
+ *    keeps no global mutable state; calls are re-entrant and asynchronous on
+ *    the given stream (NULL = the legacy default stream).
+ *  - Strides are in ELEMENTS, and the innermost stride is always 1.
+ *  - Arguments are checked on the host before anything touches the GPU; a
+ *    failed check returns its MS_ERR_* code and launches nothing.
+ *  - dev_status (optional device int): the kernels OR device-detected error
+ *    codes into it; the caller zeroes it before the call.
+ *  - There is no CPU fallback: without a usable sm_100 device a call returns
+ *    MS_ERR_CUDA or MS_ERR_DEVICE.
+ */
+#ifndef MAMBASCAN_H
+#define MAMBASCAN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *ms_stream_t;
+
+/* Element types of the token-indexed arrays. A, D, delta_bias and every state
+   array are always fp32. */
+enum { MS_F32 = 0, MS_BF16 = 1 };
+
+/* Status codes. */
+enum {
+    MS_OK = 0,
+    MS_ERR_NULL = 1,      /* a required pointer is NULL                          */
+    MS_ERR_DTYPE = 2,     /* in_dtype / out_dtype not MS_F32 or MS_BF16          */
+    MS_ERR_SHAPE = 3,     /* negative size, dstate outside [1, 16], or a size    */
+                          /* whose element offsets overflow int64                */
+    MS_ERR_STRIDE = 4,    /* negative stride                                     */
+    MS_ERR_ALIGN = 5,     /* pointer not aligned to its element size             */
+    MS_ERR_WORKSPACE = 6, /* workspace argument inconsistent                     */
+    MS_ERR_CUDA = 7,      /* a CUDA runtime call failed (no device, launch error)*/
+    MS_ERR_TIMEOUT = 8,   /* device: a bounded wait gave up                      */
+    MS_ERR_DEVICE = 9     /* device is not compute capability 10.0 (B200)        */
+};
+
+/* Maximum d_state the kernels support (Mamba-1 layers use 16). */
+#define MS_MAX_DSTATE 16
+
+/*
+ * Sizes and strides of one selective-scan call.
+ *   u, delta, z, y : [batch, dim, seqlen]   element (b,d,t) at b*x_sb + d*x_sd + t
+ *   B, C           : [batch, dstate, seqlen] element (b,n,t) at b*x_sb + n*x_sn + t
+ *                    (one group: every channel of a batch row shares B and C)
+ *   A              : [dim, dstate] dense;  D, delta_bias : [dim] dense
+ *   initial_state, last_state : [batch, dim, dstate] dense fp32
+ */
+typedef struct {
+    int64_t batch, dim, dstate, seqlen;
+    int64_t u_sb, u_sd;
+    int64_t delta_sb, delta_sd;
+    int64_t z_sb, z_sd;
+    int64_t y_sb, y_sd;
+    int64_t B_sb, B_sn;
+    int64_t C_sb, C_sn;
+    int32_t in_dtype;  /* u, delta, z, B, C */
+    int32_t out_dtype; /* y */
+} ms_scan_dims;
+
+/*
+ * Workspace bytes mamba_scan_fwd needs for these dims (0 when it needs none).
+ * Returns 0 also for dims that mamba_scan_fwd would reject.
+ */
+size_t mamba_scan_workspace_size(const ms_scan_dims *dims);
+
+/*
+ * Selective scan forward over whole sequences (prefill / training forward).
+ *   u, delta, B, C   required; delta is the raw step before bias and softplus.
+ *   A                required, fp32 [dim, dstate]; real diagonal transition
+ *                    (Mamba-1), usually negative.
+ *   D, delta_bias    optional fp32 [dim] (NULL = 0).
+ *   z                optional gate input (NULL = no gate).
+ *   softplus_flag    nonzero: Delta = softplus(delta + bias); zero: delta + bias.
+ *   initial_state    optional fp32 [batch, dim, dstate] (NULL = zero state):
+ *                    the state before token 0, so that a sequence can be scanned
+ *                    in pieces (the state is the only thing carried).
+ *   y                required output [batch, dim, seqlen] in out_dtype.
+ *   last_state       optional fp32 [batch, dim, dstate] output: the state after
+ *                    token seqlen-1 (equal to initial_state, or 0, if seqlen = 0).
+ *   workspace        device scratch of mamba_scan_workspace_size() bytes, or
+ *                    NULL with workspace_bytes = 0 when that size is 0.
+ * Returns MS_OK or an MS_ERR_* code.
+ */
+int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
+                   const void *C, const float *D, const void *z, const float *delta_bias,
+                   int softplus_flag, const float *initial_state, void *y, float *last_state,
+                   const ms_scan_dims *dims, void *workspace, size_t workspace_bytes,
+                   int *dev_status, ms_stream_t stream);
+
+/*
+ * Launch shape of the scan kernel. mamba_scan_fwd picks one from the sizes;
+ * mamba_scan_fwd_plan takes it from the caller (tuning and tests). Any valid
+ * plan gives the same result up to fp32 rounding order.
+ *   seg_per_warp  1, 2, 4 or 8: time segments a warp splits each tile into
+ *                 (the warp then holds 32/seg_per_warp channels).
+ *   poly_pairs    0, 2, 4 or 8: how many of the 8 state pairs evaluate
+ *                 exp on the FMA pipe (the rest use the MUFU unit).
+ */
+typedef struct {
+    int32_t seg_per_warp;
+    int32_t poly_pairs;
+} ms_scan_plan;
+
+/* mamba_scan_fwd with an explicit plan (NULL = choose automatically).
+   Returns MS_ERR_SHAPE for a plan value outside the lists above. */
+int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B,
+                        const void *C, const float *D, const void *z, const float *delta_bias,
+                        int softplus_flag, const float *initial_state, void *y, float *last_state,
+                        const ms_scan_dims *dims, void *workspace, size_t workspace_bytes,
+                        int *dev_status, ms_stream_t stream, const ms_scan_plan *plan);
+
+/* The plan mamba_scan_fwd would choose for these dims on the current device
+   (written to *plan). Returns MS_OK or the code mamba_scan_fwd would return
+   for invalid dims. */
+int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan);
+
+/*
+ * Sizes and strides of one decode step.
+ *   x, delta, z, y : [batch, dim]     element (b,d) at b*x_sb + d
+ *   B, C           : [batch, dstate]  element (b,n) at b*x_sb + n
+ *   state          : [batch, dim, dstate] fp32, element (b,d,n) at
+ *                    b*state_sb + d*state_sd + n
+ *   A [dim, dstate], D [dim], delta_bias [dim] dense fp32.
+ */
+typedef struct {
+    int64_t batch, dim, dstate;
+    int64_t x_sb, delta_sb, z_sb, y_sb;
+    int64_t B_sb, C_sb;
+    int64_t state_sb, state_sd;
+    int32_t in_dtype;  /* x, delta, z, B, C */
+    int32_t out_dtype; /* y */
+} ms_update_dims;
+
+/*
+ * Selective state update: one token for every (b, d), the recurrent form used
+ * for generation (blog, section 2). Reads the fp32 state, applies the same
+ * step as the scan, writes the new state in place and y.
+ *   state            required, read and overwritten.
+ *   x, delta, A, B, C, y required; D, delta_bias, z optional as in the scan.
+ * Returns MS_OK or an MS_ERR_* code.
+ */
+int mamba_state_update(float *state, const void *x, const void *delta, const float *A,
+                       const void *B, const void *C, const float *D, const void *z,
+                       const float *delta_bias, int softplus_flag, void *y,
+                       const ms_update_dims *dims, int *dev_status, ms_stream_t stream);
+
+/* Static English text for a status code (never NULL). */
+const char *mamba_status_string(int code);
+
+/* MS_OK when the current CUDA device is usable (compute capability 10.0);
+   MS_ERR_CUDA when there is no device, MS_ERR_DEVICE for another GPU. */
+int mamba_device_check(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MAMBASCAN_H */

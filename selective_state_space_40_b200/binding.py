@@ -1,0 +1,219 @@
+"""Thin ctypes binding of libmambascan.so (declared in include/mambascan.h).
+
+The raw functions keep the C names and take plain integers (device addresses,
+sizes, a stream handle). ``scan_fwd`` and ``state_update`` are conveniences
+that read the addresses, strides and dtypes off torch CUDA tensors; they do
+argument marshalling only, every step of the computation runs in the CUDA
+library. A missing library raises: there is no CPU fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmambascan.so")
+
+MS_F32, MS_BF16 = 0, 1
+MS_OK, MS_ERR_NULL, MS_ERR_DTYPE, MS_ERR_SHAPE, MS_ERR_STRIDE = 0, 1, 2, 3, 4
+MS_ERR_ALIGN, MS_ERR_WORKSPACE, MS_ERR_CUDA, MS_ERR_TIMEOUT, MS_ERR_DEVICE = 5, 6, 7, 8, 9
+MS_MAX_DSTATE = 16
+
+
+class ScanDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "dim", "dstate", "seqlen", "u_sb", "u_sd", "delta_sb", "delta_sd",
+        "z_sb", "z_sd", "y_sb", "y_sd", "B_sb", "B_sn", "C_sb", "C_sn")] + [
+        ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+class UpdateDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "dim", "dstate", "x_sb", "delta_sb", "z_sb", "y_sb", "B_sb", "C_sb",
+        "state_sb", "state_sd")] + [("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+class ScanPlan(ctypes.Structure):
+    _fields_ = [("seg_per_warp", ctypes.c_int32), ("poly_pairs", ctypes.c_int32)]
+
+
+class MambaScanError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: status {code} ({mamba_status_string(code)})")
+        self.code = code
+
+
+_lib = None
+_vp = ctypes.c_void_p
+
+
+def library() -> ctypes.CDLL:
+    """Load libmambascan.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with `python -m selective_state_space_40_b200.build`")
+        lib = ctypes.CDLL(LIB_PATH)
+        lib.mamba_scan_workspace_size.argtypes = [ctypes.POINTER(ScanDims)]
+        lib.mamba_scan_workspace_size.restype = ctypes.c_size_t
+        scan_args = [_vp] * 8 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(ScanDims), _vp,
+                                 ctypes.c_size_t, _vp, _vp]
+        lib.mamba_scan_fwd.argtypes = scan_args
+        lib.mamba_scan_fwd.restype = ctypes.c_int
+        lib.mamba_scan_fwd_plan.argtypes = scan_args + [ctypes.POINTER(ScanPlan)]
+        lib.mamba_scan_fwd_plan.restype = ctypes.c_int
+        lib.mamba_scan_choose_plan.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ScanPlan)]
+        lib.mamba_scan_choose_plan.restype = ctypes.c_int
+        lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
+                                                       _vp, _vp]
+        lib.mamba_state_update.restype = ctypes.c_int
+        lib.mamba_status_string.argtypes = [ctypes.c_int]
+        lib.mamba_status_string.restype = ctypes.c_char_p
+        lib.mamba_device_check.argtypes = []
+        lib.mamba_device_check.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+# ------------------------------------------------------------ raw C entry ----
+
+def mamba_status_string(code: int) -> str:
+    return library().mamba_status_string(int(code)).decode()
+
+
+def mamba_device_check() -> int:
+    return library().mamba_device_check()
+
+
+def mamba_scan_workspace_size(dims: ScanDims) -> int:
+    return library().mamba_scan_workspace_size(ctypes.byref(dims))
+
+
+def mamba_scan_choose_plan(dims: ScanDims) -> Tuple[int, ScanPlan]:
+    plan = ScanPlan()
+    rc = library().mamba_scan_choose_plan(ctypes.byref(dims), ctypes.byref(plan))
+    return rc, plan
+
+
+def mamba_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                   dims: ScanDims, workspace, workspace_bytes, dev_status, stream,
+                   plan: Optional[ScanPlan] = None) -> int:
+    lib = library()
+    args = (u, delta, A, B, C, D, z, delta_bias, int(softplus_flag), initial_state, y, last_state,
+            ctypes.byref(dims), workspace, int(workspace_bytes), dev_status, stream)
+    if plan is None:
+        return lib.mamba_scan_fwd(*args)
+    return lib.mamba_scan_fwd_plan(*args, ctypes.byref(plan))
+
+
+def mamba_state_update(state, x, delta, A, B, C, D, z, delta_bias, softplus_flag, y,
+                       dims: UpdateDims, dev_status, stream) -> int:
+    return library().mamba_state_update(state, x, delta, A, B, C, D, z, delta_bias,
+                                        int(softplus_flag), y, ctypes.byref(dims), dev_status, stream)
+
+
+# ----------------------------------------------------- torch conveniences ----
+
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.float32:
+        return MS_F32
+    if t.dtype == torch.bfloat16:
+        return MS_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    return None if t is None else t.data_ptr()
+
+
+def _stream_handle(stream) -> Optional[int]:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _inner_contiguous(t, name):
+    if t is not None and t.numel() > 0 and t.stride(-1) != 1:
+        raise ValueError(f"{name} must have unit stride along its last dimension")
+
+
+def scan_dims_for(u, delta, B, C, z, y) -> ScanDims:
+    """ScanDims read off tensors u/delta/z/y [b, d, L] and B/C [b, N, L]."""
+    for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z"), (y, "y")):
+        _inner_contiguous(t, n)
+    batch, dim, L = u.shape
+    N = B.shape[1]
+    zz = z if z is not None else u
+    return ScanDims(batch, dim, N, L, u.stride(0), u.stride(1), delta.stride(0), delta.stride(1),
+                    zz.stride(0), zz.stride(1), y.stride(0), y.stride(1), B.stride(0), B.stride(1),
+                    C.stride(0), C.stride(1), _dtype_code(u), _dtype_code(y))
+
+
+def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+             initial_state=None, out_dtype=None, y=None, last_state=None,
+             return_last_state: bool = True, stream=None, plan: Optional[Tuple[int, int]] = None,
+             dev_status=None):
+    """Selective scan forward on torch CUDA tensors (see include/mambascan.h).
+    Returns (y, last_state or None)."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=out_dtype, device=u.device)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
+    for t, n in ((A, "A"), (D, "D"), (delta_bias, "delta_bias"), (initial_state, "initial_state"),
+                 (last_state, "last_state")):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous fp32 tensor")
+    dims = scan_dims_for(u, delta, B, C, z, y)
+    ws_bytes = mamba_scan_workspace_size(dims)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=u.device) if ws_bytes else None
+    pl = ScanPlan(*plan) if plan is not None else None
+    rc = mamba_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                        _ptr(delta_bias), softplus, _ptr(initial_state), _ptr(y), _ptr(last_state),
+                        dims, _ptr(ws), ws_bytes, _ptr(dev_status), _stream_handle(stream), pl)
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_scan_fwd")
+    return y, last_state
+
+
+def update_dims_for(state, x, delta, B, C, z, y) -> UpdateDims:
+    for t, n in ((x, "x"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z"), (y, "y"), (state, "state")):
+        _inner_contiguous(t, n)
+    batch, dim, N = state.shape
+    zz = z if z is not None else x
+    return UpdateDims(batch, dim, N, x.stride(0), delta.stride(0), zz.stride(0), y.stride(0),
+                      B.stride(0), C.stride(0), state.stride(0), state.stride(1),
+                      _dtype_code(x), _dtype_code(y))
+
+
+def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+                 out_dtype=None, y=None, stream=None, dev_status=None):
+    """One decode step on torch CUDA tensors; ``state`` [b, d, N] fp32 is
+    updated in place. Returns y [b, d]."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    if state.dtype != torch.float32:
+        raise ValueError("state must be fp32")
+    batch, dim, N = state.shape
+    if y is None:
+        y = torch.empty((batch, dim), dtype=out_dtype, device=state.device)
+    dims = update_dims_for(state, x, delta, B, C, z, y)
+    rc = mamba_state_update(_ptr(state), _ptr(x), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                            _ptr(z), _ptr(delta_bias), softplus, _ptr(y), dims, _ptr(dev_status),
+                            _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_state_update")
+    return y

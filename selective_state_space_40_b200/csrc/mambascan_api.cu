@@ -1,0 +1,233 @@
+// mambascan_api.cu -- the extern "C" entry points of libmambascan.so: host-side
+// argument checks, launch planning and status codes. The operations are
+// described in include/mambascan.h.
+
+#include <climits>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "mambascan.h"
+#include "ms_internal.h"
+
+namespace {
+
+bool aligned(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+// Largest element offset b*sb + d*sd + t for the given extents, or -1 on
+// int64 overflow (extents are >= 1 here, strides >= 0).
+int64_t max_offset3(int64_t n0, int64_t s0, int64_t n1, int64_t s1, int64_t n2) {
+    __int128 o = (__int128)(n0 - 1) * s0 + (__int128)(n1 - 1) * s1 + (n2 - 1);
+    if (o > (__int128)INT64_MAX / 4) return -1;
+    return (int64_t)o;
+}
+
+int elem_bytes(int32_t dt) { return dt == MS_BF16 ? 2 : 4; }
+
+int num_sms_current() {
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    return sms > 0 ? sms : 148;
+}
+
+bool vec_ok(const void *p, int64_t sb, int64_t sd, int es) {
+    return p == nullptr || (aligned(p, 16) && (sb * es) % 16 == 0 && (sd * es) % 16 == 0);
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *mamba_status_string(int code) {
+    switch (code) {
+        case MS_OK: return "ok";
+        case MS_ERR_NULL: return "a required pointer is NULL";
+        case MS_ERR_DTYPE: return "unsupported dtype code";
+        case MS_ERR_SHAPE: return "invalid sizes (negative, dstate outside [1,16], or offset overflow)";
+        case MS_ERR_STRIDE: return "negative stride";
+        case MS_ERR_ALIGN: return "pointer not aligned to its element size";
+        case MS_ERR_WORKSPACE: return "workspace argument inconsistent";
+        case MS_ERR_CUDA: return "CUDA runtime error (no device or launch failure)";
+        case MS_ERR_TIMEOUT: return "device wait timed out";
+        case MS_ERR_DEVICE: return "device is not compute capability 10.0";
+        default: return "unknown status code";
+    }
+}
+
+int mamba_device_check(void) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return (major == 10 && minor == 0) ? MS_OK : MS_ERR_DEVICE;
+}
+
+static int check_scan(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                      const float *D, const void *z, const float *delta_bias, const float *h0, void *y,
+                      float *last, const ms_scan_dims *dm) {
+    if (!dm) return MS_ERR_NULL;
+    if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) ||
+        (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
+        return MS_ERR_DTYPE;
+    if (dm->batch < 0 || dm->dim < 0 || dm->seqlen < 0 || dm->dstate < 1 || dm->dstate > MS_MAX_DSTATE)
+        return MS_ERR_SHAPE;
+    if (dm->u_sb < 0 || dm->u_sd < 0 || dm->delta_sb < 0 || dm->delta_sd < 0 || dm->z_sb < 0 ||
+        dm->z_sd < 0 || dm->y_sb < 0 || dm->y_sd < 0 || dm->B_sb < 0 || dm->B_sn < 0 || dm->C_sb < 0 ||
+        dm->C_sn < 0)
+        return MS_ERR_STRIDE;
+    const bool channels = dm->batch > 0 && dm->dim > 0;
+    if (!channels) return MS_OK;
+    if (!A) return MS_ERR_NULL;
+    if (dm->seqlen > 0 && (!u || !delta || !B || !C || !y)) return MS_ERR_NULL;
+    const int ei = elem_bytes(dm->in_dtype), eo = elem_bytes(dm->out_dtype);
+    if (!aligned(u, ei) || !aligned(delta, ei) || !aligned(B, ei) || !aligned(C, ei) ||
+        (z && !aligned(z, ei)) || !aligned(y, eo) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+        (delta_bias && !aligned(delta_bias, 4)) || (h0 && !aligned(h0, 4)) || (last && !aligned(last, 4)))
+        return MS_ERR_ALIGN;
+    if (dm->seqlen > 0) {
+        const int64_t L = dm->seqlen;
+        if (max_offset3(dm->batch, dm->u_sb, dm->dim, dm->u_sd, L) < 0 ||
+            max_offset3(dm->batch, dm->delta_sb, dm->dim, dm->delta_sd, L) < 0 ||
+            max_offset3(dm->batch, dm->z_sb, dm->dim, dm->z_sd, L) < 0 ||
+            max_offset3(dm->batch, dm->y_sb, dm->dim, dm->y_sd, L) < 0 ||
+            max_offset3(dm->batch, dm->B_sb, dm->dstate, dm->B_sn, L) < 0 ||
+            max_offset3(dm->batch, dm->C_sb, dm->dstate, dm->C_sn, L) < 0)
+            return MS_ERR_SHAPE;
+    }
+    if (max_offset3(dm->batch, dm->dim * dm->dstate, dm->dim, dm->dstate, dm->dstate) < 0)
+        return MS_ERR_SHAPE;
+    return MS_OK;
+}
+
+size_t mamba_scan_workspace_size(const ms_scan_dims *dims) {
+    (void)dims;
+    return 0;
+}
+
+static bool plan_valid(const ms_scan_plan *p) {
+    const int s = p->seg_per_warp, q = p->poly_pairs;
+    return (s == 1 || s == 2 || s == 4 || s == 8) && (q == 0 || q == 2 || q == 4 || q == 8);
+}
+
+static ms::ScanPlan auto_plan(const ms_scan_dims *dims) {
+    ms::ScanArgs a{};
+    a.batch = dims->batch;
+    a.dim = dims->dim;
+    a.L = dims->seqlen;
+    a.N = (int)dims->dstate;
+    return ms::plan_scan(a, dims->in_dtype == MS_BF16, num_sms_current());
+}
+
+int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan) {
+    if (!dims || !plan) return MS_ERR_NULL;
+    int rc = check_scan(nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        nullptr, nullptr, dims);
+    if (rc != MS_OK && rc != MS_ERR_NULL) return rc;
+    const ms::ScanPlan p = auto_plan(dims);
+    plan->seg_per_warp = p.seg_per_warp;
+    plan->poly_pairs = p.poly_pairs;
+    return MS_OK;
+}
+
+int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                   const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
+                   void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream) {
+    return mamba_scan_fwd_plan(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y,
+                               last_state, dims, workspace, workspace_bytes, dev_status, stream, nullptr);
+}
+
+int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                        const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
+                        void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream,
+                        const ms_scan_plan *plan) {
+    if (plan && !plan_valid(plan)) return MS_ERR_SHAPE;
+    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
+    if (rc != MS_OK) return rc;
+    if (workspace_bytes < mamba_scan_workspace_size(dims) || (workspace_bytes > 0 && !workspace))
+        return MS_ERR_WORKSPACE;
+    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
+    if (dims->seqlen == 0 && !last_state) return MS_OK;
+
+    ms::ScanArgs a{};
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.A = A; a.D = D; a.bias = delta_bias; a.h0 = initial_state;
+    a.y = y; a.last = last_state; a.status = dev_status;
+    a.batch = dims->batch; a.dim = dims->dim; a.L = dims->seqlen; a.N = (int)dims->dstate;
+    a.u_sb = dims->u_sb; a.u_sd = dims->u_sd;
+    a.dl_sb = dims->delta_sb; a.dl_sd = dims->delta_sd;
+    a.z_sb = dims->z_sb; a.z_sd = dims->z_sd;
+    a.y_sb = dims->y_sb; a.y_sd = dims->y_sd;
+    a.B_sb = dims->B_sb; a.B_sn = dims->B_sn; a.C_sb = dims->C_sb; a.C_sn = dims->C_sn;
+    a.softplus = softplus_flag ? 1 : 0;
+    const int ei = elem_bytes(dims->in_dtype), eo = elem_bytes(dims->out_dtype);
+    a.vec_in = vec_ok(u, dims->u_sb, dims->u_sd, ei) && vec_ok(delta, dims->delta_sb, dims->delta_sd, ei) &&
+               vec_ok(z, dims->z_sb, dims->z_sd, ei);
+    a.vec_out = vec_ok(y, dims->y_sb, dims->y_sd, eo);
+
+    const bool in_bf16 = dims->in_dtype == MS_BF16, out_bf16 = dims->out_dtype == MS_BF16;
+    ms::ScanPlan pl = auto_plan(dims);
+    if (plan) {
+        pl.seg_per_warp = plan->seg_per_warp;
+        pl.tokens_per_seg = plan->seg_per_warp == 1 ? 16 : 8;
+        pl.poly_pairs = plan->poly_pairs;
+    }
+    cudaError_t e = ms::launch_scan_fwd(a, pl, in_bf16, out_bf16, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
+int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,
+                       const void *C, const float *D, const void *z, const float *delta_bias,
+                       int softplus_flag, void *y, const ms_update_dims *dm, int *dev_status,
+                       ms_stream_t stream) {
+    if (!dm) return MS_ERR_NULL;
+    if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) ||
+        (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
+        return MS_ERR_DTYPE;
+    if (dm->batch < 0 || dm->dim < 0 || dm->dstate < 1 || dm->dstate > MS_MAX_DSTATE) return MS_ERR_SHAPE;
+    if (dm->x_sb < 0 || dm->delta_sb < 0 || dm->z_sb < 0 || dm->y_sb < 0 || dm->B_sb < 0 || dm->C_sb < 0 ||
+        dm->state_sb < 0 || dm->state_sd < 0)
+        return MS_ERR_STRIDE;
+    if (dm->batch == 0 || dm->dim == 0) return MS_OK;
+    if (!state || !x || !delta || !A || !B || !C || !y) return MS_ERR_NULL;
+    const int ei = elem_bytes(dm->in_dtype), eo = elem_bytes(dm->out_dtype);
+    if (!aligned(state, 4) || !aligned(x, ei) || !aligned(delta, ei) || !aligned(B, ei) || !aligned(C, ei) ||
+        (z && !aligned(z, ei)) || !aligned(y, eo) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+        (delta_bias && !aligned(delta_bias, 4)))
+        return MS_ERR_ALIGN;
+    if (max_offset3(dm->batch, dm->x_sb, 1, 0, dm->dim) < 0 || max_offset3(dm->batch, dm->delta_sb, 1, 0, dm->dim) < 0 ||
+        max_offset3(dm->batch, dm->z_sb, 1, 0, dm->dim) < 0 || max_offset3(dm->batch, dm->y_sb, 1, 0, dm->dim) < 0 ||
+        max_offset3(dm->batch, dm->B_sb, 1, 0, dm->dstate) < 0 || max_offset3(dm->batch, dm->C_sb, 1, 0, dm->dstate) < 0 ||
+        max_offset3(dm->batch, dm->state_sb, dm->dim, dm->state_sd, dm->dstate) < 0)
+        return MS_ERR_SHAPE;
+
+    ms::UpdateArgs a{};
+    a.state = state; a.x = x; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.A = A; a.D = D; a.bias = delta_bias; a.y = y; a.status = dev_status;
+    a.batch = dm->batch; a.dim = dm->dim; a.N = (int)dm->dstate;
+    a.x_sb = dm->x_sb; a.dl_sb = dm->delta_sb; a.z_sb = dm->z_sb; a.y_sb = dm->y_sb;
+    a.B_sb = dm->B_sb; a.C_sb = dm->C_sb; a.st_sb = dm->state_sb; a.st_sd = dm->state_sd;
+    a.softplus = softplus_flag ? 1 : 0;
+    a.vec_state = aligned(state, 16) && (dm->state_sb % 4) == 0 && (dm->state_sd % 4) == 0;
+    cudaError_t e = ms::launch_state_update(a, dm->in_dtype == MS_BF16, dm->out_dtype == MS_BF16,
+                                            (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,55 @@
+// ms_internal.h -- argument blocks passed from the C-ABI layer to the kernel
+// launchers (not part of the public ABI).
+#pragma once
+
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace ms {
+
+struct ScanArgs {
+    const void *u, *delta, *z, *B, *C;
+    const float *A, *D, *bias, *h0;
+    void *y;
+    float *last;
+    int *status;
+    int64_t batch, dim, L;
+    int N;
+    int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, y_sb, y_sd;
+    int64_t B_sb, B_sn, C_sb, C_sn;
+    int softplus;
+    int vec_in;   // u/delta/z rows 16-byte aligned: vector loads allowed
+    int vec_out;  // y rows 16-byte aligned: vector stores allowed
+};
+
+// Launch shape chosen on the host for one scan call.
+struct ScanPlan {
+    int seg_per_warp;   // S_W: time segments per warp (1, 2, 4, 8)
+    int tokens_per_seg; // T
+    int poly_pairs;     // state pairs whose exp runs on the FMA pipe
+    int warps_per_cta;
+};
+
+struct UpdateArgs {
+    float *state;
+    const void *x, *delta, *z, *B, *C;
+    const float *A, *D, *bias;
+    void *y;
+    int *status;
+    int64_t batch, dim;
+    int N;
+    int64_t x_sb, dl_sb, z_sb, y_sb, B_sb, C_sb, st_sb, st_sd;
+    int softplus;
+    int vec_state;  // state rows of 16 fp32 at 16-byte aligned addresses
+};
+
+// in_bf16/out_bf16 select the element types. Return a cudaError_t.
+cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16,
+                            cudaStream_t stream);
+cudaError_t launch_state_update(const UpdateArgs &a, bool in_bf16, bool out_bf16,
+                                cudaStream_t stream);
+
+// Plan for a call (host heuristic from sizes and dtypes).
+ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms);
+
+}  // namespace ms

@@ -1,0 +1,161 @@
+"""The C-ABI library: builds, loads without a GPU, exports every function the
+headers declare, and rejects bad arguments on the host (no GPU involved)."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+from selective_state_space_40_b200 import binding as mb
+from selective_state_space_40_b200 import build as mbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mbuild.build()
+    return mb.library()
+
+
+def declared_functions():
+    names = set()
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(mamba_\w+)\s*\(", text, flags=re.M):
+            names.add(m.group(1))
+    return sorted(names)
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    for n in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size",
+              "mamba_status_string", "mamba_device_check", "mamba_scan_fwd_plan",
+              "mamba_scan_choose_plan"):
+        assert n in names
+
+
+@pytest.mark.parametrize("name", declared_functions())
+def test_library_exports(lib, name):
+    assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+
+
+def test_no_cpu_fallback_symbols(lib):
+    # the product library never links the oracle
+    for sym in ("oracle_scan_f64", "oracle_state_update_f64"):
+        with pytest.raises(AttributeError):
+            getattr(lib, sym)
+
+
+def test_status_strings(lib):
+    for code in range(0, 10):
+        s = mb.mamba_status_string(code)
+        assert isinstance(s, str) and s
+    assert mb.mamba_status_string(0) == "ok"
+    assert "unknown" in mb.mamba_status_string(12345)
+
+
+def _dims(**kw):
+    d = dict(batch=2, dim=8, dstate=16, seqlen=32, u_sb=256, u_sd=32, delta_sb=256, delta_sd=32,
+             z_sb=256, z_sd=32, y_sb=256, y_sd=32, B_sb=512, B_sn=32, C_sb=512, C_sn=32,
+             in_dtype=mb.MS_F32, out_dtype=mb.MS_F32)
+    d.update(kw)
+    return mb.ScanDims(**d)
+
+
+FAKE = 1 << 20  # never dereferenced: every call below fails its host checks
+
+
+def _scan(dims, u=FAKE, delta=FAKE, A=FAKE, B=FAKE, C=FAKE, y=FAKE, ws=None, ws_bytes=0, plan=None):
+    return mb.mamba_scan_fwd(u, delta, A, B, C, None, None, None, 1, None, y, None, dims,
+                             ws, ws_bytes, None, None, plan)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(in_dtype=7), mb.MS_ERR_DTYPE),
+    (dict(out_dtype=-1), mb.MS_ERR_DTYPE),
+    (dict(dstate=0), mb.MS_ERR_SHAPE),
+    (dict(dstate=17), mb.MS_ERR_SHAPE),
+    (dict(batch=-1), mb.MS_ERR_SHAPE),
+    (dict(seqlen=-5), mb.MS_ERR_SHAPE),
+    (dict(u_sd=-1), mb.MS_ERR_STRIDE),
+    (dict(B_sn=-2), mb.MS_ERR_STRIDE),
+    (dict(u_sb=1 << 61, batch=1 << 4), mb.MS_ERR_SHAPE),
+])
+def test_scan_rejects_bad_dims(lib, kw, code):
+    assert _scan(_dims(**kw)) == code
+
+
+def test_scan_rejects_null_and_misaligned(lib):
+    assert mb.library().mamba_scan_fwd(*([None] * 8), 1, None, None, None, None, None, 0, None, None) \
+        == mb.MS_ERR_NULL
+    assert _scan(_dims(), u=None) == mb.MS_ERR_NULL
+    assert _scan(_dims(), y=None) == mb.MS_ERR_NULL
+    assert _scan(_dims(), A=None) == mb.MS_ERR_NULL
+    assert _scan(_dims(), u=FAKE + 2) == mb.MS_ERR_ALIGN       # fp32 needs 4-byte alignment
+    assert _scan(_dims(in_dtype=mb.MS_BF16), u=FAKE + 1) == mb.MS_ERR_ALIGN
+    assert _scan(_dims(), A=FAKE + 1) == mb.MS_ERR_ALIGN
+
+
+def test_scan_rejects_bad_plan_and_workspace(lib):
+    assert _scan(_dims(), plan=mb.ScanPlan(3, 0)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(4, 5)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), ws=None, ws_bytes=64) == mb.MS_ERR_WORKSPACE
+
+
+def test_empty_scan_is_a_noop(lib):
+    # nothing to compute: no launch, so this is safe without a GPU
+    assert _scan(_dims(batch=0)) == mb.MS_OK
+    assert _scan(_dims(dim=0), u=None, y=None) == mb.MS_OK
+    assert mb.mamba_scan_workspace_size(_dims()) == 0
+
+
+def test_choose_plan(lib):
+    rc, plan = mb.mamba_scan_choose_plan(_dims(batch=8, dim=1536, seqlen=2048, in_dtype=mb.MS_BF16))
+    assert rc == mb.MS_OK and plan.seg_per_warp in (1, 2, 4, 8) and plan.poly_pairs in (0, 2, 4, 8)
+    rc, _ = mb.mamba_scan_choose_plan(_dims(dstate=40))
+    assert rc == mb.MS_ERR_SHAPE
+
+
+def _udims(**kw):
+    d = dict(batch=4, dim=8, dstate=16, x_sb=8, delta_sb=8, z_sb=8, y_sb=8, B_sb=16, C_sb=16,
+             state_sb=128, state_sd=16, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)
+    d.update(kw)
+    return mb.UpdateDims(**d)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(in_dtype=3), mb.MS_ERR_DTYPE),
+    (dict(dstate=0), mb.MS_ERR_SHAPE),
+    (dict(dstate=32), mb.MS_ERR_SHAPE),
+    (dict(state_sd=-16), mb.MS_ERR_STRIDE),
+])
+def test_update_rejects_bad_dims(lib, kw, code):
+    rc = mb.mamba_state_update(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE,
+                               _udims(**kw), None, None)
+    assert rc == code
+
+
+def test_update_rejects_null_and_misaligned(lib):
+    assert mb.mamba_state_update(None, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE,
+                                 _udims(), None, None) == mb.MS_ERR_NULL
+    assert mb.mamba_state_update(FAKE + 2, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE,
+                                 _udims(), None, None) == mb.MS_ERR_ALIGN
+    assert mb.mamba_state_update(FAKE, FAKE + 1, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, FAKE,
+                                 _udims(), None, None) == mb.MS_ERR_ALIGN
+
+
+def test_device_check_without_gpu(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; this checks the no-device answer")
+    assert mb.mamba_device_check() == mb.MS_ERR_CUDA
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(mb, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(mb, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        mb.library()

@@ -1,0 +1,135 @@
+"""GPU parity of mamba_state_update (decode) against the fp64 oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_40_b200 import binding as mb
+from selective_state_space_40_b200 import synthetic as syn
+from parity_util import check, check_bf16, check_fp32, f64
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    mb.library()
+
+
+def _step_gpu(state, inp, params, use_z=True, use_D=True, use_bias=True, softplus=True):
+    return mb.state_update(state, inp["x"].to(DEV), inp["delta"].to(DEV), params["A"],
+                           inp["B"].to(DEV), inp["C"].to(DEV), params["D"] if use_D else None,
+                           inp["z"].to(DEV) if use_z else None,
+                           params["delta_bias"] if use_bias else None, softplus)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("N", [1, 3, 4, 5, 16])
+def test_small_steps_full(dtype, N):
+    w = syn.DecodeWorkload("small", batch=3, dim=37, dstate=N, steps=20, in_dtype=dtype)
+    p = syn.decode_params(w)
+    params = {k: v.to(DEV) for k, v in p.items()}
+    state = params["state0"].clone()
+    h = f64(p["state0"])
+    for k in range(w.steps):
+        inp = syn.decode_step_inputs(w, k)
+        y = _step_gpu(state, inp, params)
+        yr, h = oracle.state_update(h, f64(inp["x"]), f64(inp["delta"]), f64(p["A"]), f64(inp["B"]),
+                                    f64(inp["C"]), f64(p["D"]), f64(inp["z"]), f64(p["delta_bias"]), True)
+        torch.cuda.synchronize()
+        check(f64(y), yr, dtype, f"step {k} y")
+    check(f64(state), h, dtype, "final state")
+
+
+@pytest.mark.parametrize("flags", [dict(use_z=False), dict(use_D=False), dict(use_bias=False)])
+def test_optional_inputs(flags):
+    w = syn.DecodeWorkload("small", batch=4, dim=64, dstate=16, steps=5, in_dtype=torch.float32)
+    p = syn.decode_params(w)
+    params = {k: v.to(DEV) for k, v in p.items()}
+    state = params["state0"].clone()
+    h = f64(p["state0"])
+    for k in range(w.steps):
+        inp = syn.decode_step_inputs(w, k)
+        y = _step_gpu(state, inp, params, **flags)
+        yr, h = oracle.state_update(
+            h, f64(inp["x"]), f64(inp["delta"]), f64(p["A"]), f64(inp["B"]), f64(inp["C"]),
+            None if not flags.get("use_D", True) else f64(p["D"]),
+            None if not flags.get("use_z", True) else f64(inp["z"]),
+            None if not flags.get("use_bias", True) else f64(p["delta_bias"]), True)
+        torch.cuda.synchronize()
+        check_fp32(f64(y), yr, f"{flags} y")
+    check_fp32(f64(state), h, f"{flags} state")
+
+
+def test_strided_state():
+    """State rows padded (d stride 20 instead of 16): scalar path."""
+    w = syn.DecodeWorkload("small", batch=2, dim=16, dstate=16, steps=3, in_dtype=torch.float32)
+    p = syn.decode_params(w)
+    params = {k: v.to(DEV) for k, v in p.items()}
+    big = torch.zeros(2, 16, 20, device=DEV)
+    big[:, :, 2:18] = params["state0"]
+    state = big[:, :, 2:18]
+    h = f64(p["state0"])
+    for k in range(w.steps):
+        inp = syn.decode_step_inputs(w, k)
+        y = _step_gpu(state, inp, params)
+        yr, h = oracle.state_update(h, f64(inp["x"]), f64(inp["delta"]), f64(p["A"]), f64(inp["B"]),
+                                    f64(inp["C"]), f64(p["D"]), f64(inp["z"]), f64(p["delta_bias"]), True)
+        torch.cuda.synchronize()
+        check_fp32(f64(y), yr, "strided y")
+    check_fp32(f64(state), h, "strided state")
+    assert float(big[:, :, :2].abs().max()) == 0.0 and float(big[:, :, 18:].abs().max()) == 0.0
+
+
+def test_scan_equals_decode_on_gpu():
+    """L decode steps from zero give the scan's y and last_state."""
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=50, in_dtype=torch.float32, seed=8)
+    inp = syn.scan_inputs(w)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    y_scan, last = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                               g["delta_bias"], True)
+    state = torch.zeros(2, 40, 16, device=DEV)
+    ys = []
+    for t in range(w.seqlen):
+        ys.append(mb.state_update(state, g["u"][:, :, t].contiguous(), g["delta"][:, :, t].contiguous(),
+                                  g["A"], g["B"][:, :, t].contiguous(), g["C"][:, :, t].contiguous(),
+                                  g["D"], g["z"][:, :, t].contiguous(), g["delta_bias"], True))
+    torch.cuda.synchronize()
+    yr, lr = oracle.scan(f64(inp["u"]), f64(inp["delta"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
+                         f64(inp["D"]), f64(inp["z"]), f64(inp["delta_bias"]), True)
+    check_fp32(f64(torch.stack(ys, dim=2)), yr, "decode-as-scan y")
+    check_fp32(f64(state), lr, "decode-as-scan state")
+    check_fp32(f64(y_scan), yr, "scan y")
+
+
+@pytest.mark.slow
+def test_full_decode_1000_steps_sampled():
+    """b256 d5120 N16, 1000 steps on the GPU at full size; a seeded sample of
+    channels is followed by the oracle through every step (every y) and the
+    final state."""
+    w = syn.DECODE
+    p = syn.decode_params(w)
+    params = {k: v.to(DEV) for k, v in p.items()}
+    state = params["state0"].clone()
+    rng = np.random.default_rng(99)
+    nb = 24
+    bs = np.sort(rng.choice(w.batch, nb, replace=False))
+    ds = np.sort(rng.choice(w.dim, 48, replace=False))
+    h = f64(p["state0"][bs][:, ds])
+    A, D, bias = f64(p["A"][ds]), f64(p["D"][ds]), f64(p["delta_bias"][ds])
+    y_all, yr_all = [], []
+    for k in range(w.steps):
+        inp = syn.decode_step_inputs(w, k)
+        y = _step_gpu(state, inp, params)
+        sel = lambda t: f64(t[bs][:, ds])  # noqa: E731
+        yr, h = oracle.state_update(h, sel(inp["x"]), sel(inp["delta"]), A, f64(inp["B"][bs]),
+                                    f64(inp["C"][bs]), D, sel(inp["z"]), bias, True)
+        y_all.append(f64(y[torch.as_tensor(bs)][:, torch.as_tensor(ds)]))
+        yr_all.append(yr)
+    torch.cuda.synchronize()
+    assert torch.isfinite(state).all()
+    check_bf16(np.stack(y_all), np.stack(yr_all), "decode every y (sampled channels)")
+    check_bf16(f64(state[torch.as_tensor(bs)][:, torch.as_tensor(ds)]), h, "decode final state (sampled)")

@@ -1,0 +1,418 @@
+"""Benchmark of the selective scan forward (and the decode step) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one selective-scan forward (mamba_scan_fwd through the C ABI) over
+the 130M-class layer: batch 8, d_inner 1536, d_state 16, L 2048, bf16 inputs,
+fp32 y and last_state. Inputs are synthetic, seeded, resident in HBM; two
+copies of them are rotated so that every step reads inputs not touched by the
+previous step (254 MB per set, above the 126 MB L2). Rank 0 prints one JSON
+line. Under torchrun every rank runs its own layer (weak scaling, no
+collective on the data path); the device time is the max over ranks.
+
+`--impl reference` times the fp64 CPU oracle on the host cores instead, on a
+bounded sample of the same workload per step.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import glob
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "selective-scan fwd achieved HBM GB/s and Gchannel-tokens/s vs HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_HBM_GBS = 6650.0
+
+
+# ------------------------------------------------------------ byte models ----
+
+def scan_bytes(batch, dim, dstate, seqlen, in_bytes, out_bytes):
+    """Minimum HBM bytes of one scan: u, delta, z read and y written per
+    channel-token; B, C read once per (batch, token); A read, D and bias read,
+    last_state written."""
+    ct = batch * dim * seqlen
+    return (ct * (3 * in_bytes + out_bytes) + batch * seqlen * 2 * dstate * in_bytes
+            + batch * dim * dstate * 4 + dim * dstate * 4 + 2 * dim * 4)
+
+
+def decode_bytes(batch, dim, dstate, in_bytes, out_bytes):
+    """Minimum HBM bytes of one decode step: the fp32 state read and written,
+    x, delta, z read and y written per channel, B and C per batch row, A, D,
+    bias."""
+    return (batch * dim * dstate * 8 + batch * dim * (3 * in_bytes + out_bytes)
+            + batch * dstate * 2 * in_bytes + dim * dstate * 4 + 2 * dim * 4)
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_digest():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "selective_state_space_40_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel):
+    """DRAM bytes per launch from the committed ncu capture, if it was taken
+    on the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None
+    if not rec or rec.get("csrc_sha") != csrc_digest():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------- clock sampler ----
+
+class ClockSampler:
+    """Samples the SM clock and the clock-event reasons through NVML while the
+    timed region runs (reads only; changes no setting)."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period=0.02):
+        self.period = period
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                r = self._nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self._ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._ok:
+            self._t.join()
+
+    def summary(self):
+        if not self._ok or not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["nvml unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons - {"gpu_idle"}), "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------- dist plumbing --
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        import datetime
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(value, world, device=None):
+    """Max of a per-rank float over all ranks (identity for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------- CPU baseline ----
+
+def oracle_sample_time(inp, n_batch_rows, nthreads):
+    """Run the fp64 oracle (as it stands) on the first n_batch_rows batch rows
+    of the workload; returns (channel_tokens, seconds)."""
+    import oracle
+
+    def f64(t):
+        return t.to("cpu").to(__import__("torch").float64).numpy()
+
+    sl = slice(0, n_batch_rows)
+    args = (f64(inp["u"][sl]), f64(inp["delta"][sl]), f64(inp["A"]), f64(inp["B"][sl]),
+            f64(inp["C"][sl]), f64(inp["D"]), f64(inp["z"][sl]), f64(inp["delta_bias"]))
+    lib = oracle.load_oracle()
+    t = time.perf_counter()
+    oracle.scan(*args, softplus_flag=True, lib=lib, nthreads=nthreads)
+    dt = time.perf_counter() - t
+    b, d, L = inp["u"][sl].shape
+    return b * d * L, dt
+
+
+def cpu_threads():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------- main ----
+
+def run_reference(args, w, world, rank):
+    """The oracle on the host cores, each step a bounded sample (one batch
+    row) of the same workload."""
+    if rank != 0:
+        return 0
+    import torch
+    from selective_state_space_40_b200 import synthetic as syn
+    torch.set_num_threads(max(1, cpu_threads()))
+    inp = syn.scan_inputs(w)
+    es = 2 if w.in_dtype == torch.bfloat16 else 4
+    threads = cpu_threads()
+    rows = 1
+    for _ in range(args.warmup):
+        oracle_sample_time(inp, rows, threads)
+    total_ct, total_s = 0, 0.0
+    for _ in range(args.steps):
+        ct, s = oracle_sample_time(inp, rows, threads)
+        total_ct += ct
+        total_s += s
+    ct_s = total_ct / total_s
+    bytes_per_ct = scan_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4) / w.channel_tokens
+    gbs = ct_s * bytes_per_ct / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s",
+        "gct_per_s": ct_s / 1e9, "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                   "seqlen": w.seqlen, "in_dtype": "bf16", "out_dtype": "f64",
+                   "sample": f"{rows} of {w.batch} batch rows per step"},
+        "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{rows} of {w.batch} batch rows ({rows * w.dim * w.seqlen} channel-tokens) per step"},
+        "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world, rank, local = dist_env()
+    from selective_state_space_40_b200 import synthetic as syn
+    w = syn.M130
+
+    if args.impl == "reference":
+        return run_reference(args, w, world, rank)
+
+    import torch
+    from selective_state_space_40_b200 import binding as mb
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    init_dist(world, "nccl")
+    if mb.mamba_device_check() != mb.MS_OK:
+        raise SystemExit("libmambascan: " + mb.mamba_status_string(mb.mamba_device_check()))
+
+    es = 2 if w.in_dtype == torch.bfloat16 else 4
+    host = syn.scan_inputs(w)
+    sets = [{k: v.to(dev) for k, v in host.items()} for _ in range(2)]
+    y = torch.empty(w.batch, w.dim, w.seqlen, dtype=torch.float32, device=dev)
+    last = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        g = sets[i & 1]
+        mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                    True, y=y, last_state=last, stream=stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # ---- timed region: K steps, per-launch events on the launching stream
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        t0.record(stream)
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
+        t1.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), world, dev)
+    kernel_ms = statistics.fmean(a.elapsed_time(b) for a, b in ev)
+    kernel_ms = max_over_ranks(kernel_ms, world, dev)
+
+    nbytes = scan_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4)
+    ct = w.channel_tokens
+    value = world * nbytes * args.steps / (elapsed_ms * 1e-3) / 1e9
+    gct = world * ct * args.steps / (elapsed_ms * 1e-3) / 1e9
+    peak, peak_kind = measured_peaks()
+    achieved = nbytes / (kernel_ms * 1e-3) / 1e9
+    traffic = recorded_traffic("scan_fwd_130m")
+
+    # ---- end to end through the public API with host buffers
+    pinned = {k: v.pin_memory() for k, v in host.items()}
+    y_host = torch.empty(y.shape, dtype=y.dtype, pin_memory=True)
+    last_host = torch.empty(last.shape, dtype=last.dtype, pin_memory=True)
+    dev_in = sets[0]
+    h2d = sum(v.numel() * v.element_size() for v in pinned.values())
+    d2h = y_host.numel() * 4 + last_host.numel() * 4
+    e2e_steps = max(3, min(20, args.steps // 20))
+
+    def e2e_step():
+        for k, v in pinned.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        mb.scan_fwd(dev_in["u"], dev_in["delta"], dev_in["A"], dev_in["B"], dev_in["C"], dev_in["D"],
+                    dev_in["z"], dev_in["delta_bias"], True, y=y, last_state=last, stream=stream)
+        y_host.copy_(y, non_blocking=True)
+        last_host.copy_(last, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    e2e_gbs = world * nbytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
+
+    # ---- decode step (selective state update) at b256 d5120 N16, L2 flushed
+    dw = syn.DECODE
+    dp = {k: v.to(dev) for k, v in syn.decode_params(dw).items()}
+    ds = {k: v.to(dev) for k, v in syn.decode_step_inputs(dw, 0).items()}
+    state = dp["state0"].clone()
+    yd = torch.empty(dw.batch, dw.dim, dtype=torch.float32, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    dec_times = []
+    for i in range(40):
+        flush.fill_(i & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        mb.state_update(state, ds["x"], ds["delta"], dp["A"], ds["B"], ds["C"], dp["D"], ds["z"],
+                        dp["delta_bias"], True, y=yd, stream=stream)
+        b.record(stream)
+        dec_times.append((a, b))
+    torch.cuda.synchronize()
+    dec_ms = statistics.fmean(a.elapsed_time(b) for a, b in dec_times[5:])
+    dec_ms = max_over_ranks(dec_ms, world, dev)
+    dbytes = decode_bytes(dw.batch, dw.dim, dw.dstate, 2, 4)
+    dec_gbs = dbytes / (dec_ms * 1e-3) / 1e9
+    del flush
+
+    # ---- CPU baseline: the oracle on this host's cores, one batch row
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = cpu_threads()
+        cts, secs = oracle_sample_time(host, 1, threads)
+        ct_s = cts / secs
+        cpu = {"value": ct_s * nbytes / ct / 1e9, "unit": "GB/s", "gct_per_s": ct_s / 1e9,
+               "cores": threads, "kind": "oracle",
+               "sample": f"1 of {w.batch} batch rows ({cts} channel-tokens), {secs:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "gct_per_s": gct,
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": elapsed_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
+                       "seqlen": w.seqlen, "in_dtype": "bf16", "out_dtype": "f32",
+                       "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": "two rotating input sets of 254 MB each (> 126 MB L2), no flush"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": traffic,
+                         "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
+                         "kernel": "scan_fwd_kernel", "bytes_per_launch": nbytes,
+                         "kernel_ms": kernel_ms},
+            "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "decode_step": {"workload": dw.name, "value": dec_gbs, "unit": "GB/s",
+                            "ms": dec_ms, "bytes": dbytes, "frac": dec_gbs / peak,
+                            "l2": "2x L2 buffer written before every timed launch"},
+            "gpu_launches": args.steps,
+            "clocks": clk.summary(),
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

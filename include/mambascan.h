@@ -120,15 +120,15 @@ int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void 
 /*
  * Launch shape of the scan kernel. mamba_scan_fwd picks one from the sizes;
  * mamba_scan_fwd_plan takes it from the caller (tuning and tests). Any valid
- * plan gives the same result up to fp32 rounding order.
- *   seg_per_warp  1, 2, 4 or 8: time segments a warp splits each tile into
- *                 (the warp then holds 32/seg_per_warp channels).
- *   poly_pairs    0, 2, 4 or 8: how many of the 8 state pairs evaluate
- *                 exp on the FMA pipe (the rest use the MUFU unit).
+ * plan gives the same result up to fp32 rounding.
+ *   lanes_per_channel  2, 4 or 8: lanes sharing one channel, each holding
+ *                      16/lanes_per_channel of its states.
+ *   poly8              0, 2, 3, 4 or 8: eighths of the exponentials computed
+ *                      by a polynomial on the FMA pipe instead of the MUFU unit.
  */
 typedef struct {
-    int32_t seg_per_warp;
-    int32_t poly_pairs;
+    int32_t lanes_per_channel;
+    int32_t poly8;
 } ms_scan_plan;
 
 /* mamba_scan_fwd with an explicit plan (NULL = choose automatically).

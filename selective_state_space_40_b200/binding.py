@@ -35,7 +35,7 @@ class UpdateDims(ctypes.Structure):
 
 
 class ScanPlan(ctypes.Structure):
-    _fields_ = [("seg_per_warp", ctypes.c_int32), ("poly_pairs", ctypes.c_int32)]
+    _fields_ = [("lanes_per_channel", ctypes.c_int32), ("poly8", ctypes.c_int32)]
 
 
 class MambaScanError(RuntimeError):

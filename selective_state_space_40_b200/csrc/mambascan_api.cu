@@ -112,8 +112,8 @@ size_t mamba_scan_workspace_size(const ms_scan_dims *dims) {
 }
 
 static bool plan_valid(const ms_scan_plan *p) {
-    const int s = p->seg_per_warp, q = p->poly_pairs;
-    return (s == 1 || s == 2 || s == 4 || s == 8) && (q == 0 || q == 2 || q == 4 || q == 8);
+    const int g = p->lanes_per_channel, q = p->poly8;
+    return (g == 2 || g == 4 || g == 8) && (q == 0 || q == 2 || q == 3 || q == 4 || q == 8);
 }
 
 static ms::ScanPlan auto_plan(const ms_scan_dims *dims) {
@@ -131,8 +131,8 @@ int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan) {
                         nullptr, nullptr, dims);
     if (rc != MS_OK && rc != MS_ERR_NULL) return rc;
     const ms::ScanPlan p = auto_plan(dims);
-    plan->seg_per_warp = p.seg_per_warp;
-    plan->poly_pairs = p.poly_pairs;
+    plan->lanes_per_channel = p.lanes_per_channel;
+    plan->poly8 = p.poly8;
     return MS_OK;
 }
 
@@ -176,9 +176,8 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
     const bool in_bf16 = dims->in_dtype == MS_BF16, out_bf16 = dims->out_dtype == MS_BF16;
     ms::ScanPlan pl = auto_plan(dims);
     if (plan) {
-        pl.seg_per_warp = plan->seg_per_warp;
-        pl.tokens_per_seg = plan->seg_per_warp == 1 ? 16 : 8;
-        pl.poly_pairs = plan->poly_pairs;
+        pl.lanes_per_channel = plan->lanes_per_channel;
+        pl.poly8 = plan->poly8;
     }
     cudaError_t e = ms::launch_scan_fwd(a, pl, in_bf16, out_bf16, (cudaStream_t)stream);
     if (e != cudaSuccess) {
@@ -197,6 +196,7 @@ int mamba_state_update(float *state, const void *x, const void *delta, const flo
         (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
         return MS_ERR_DTYPE;
     if (dm->batch < 0 || dm->dim < 0 || dm->dstate < 1 || dm->dstate > MS_MAX_DSTATE) return MS_ERR_SHAPE;
+    if (dm->batch > 65535 || dm->dim > (int64_t)(INT32_MAX / 4)) return MS_ERR_SHAPE;
     if (dm->x_sb < 0 || dm->delta_sb < 0 || dm->z_sb < 0 || dm->y_sb < 0 || dm->B_sb < 0 || dm->C_sb < 0 ||
         dm->state_sb < 0 || dm->state_sd < 0)
         return MS_ERR_STRIDE;
@@ -221,6 +221,8 @@ int mamba_state_update(float *state, const void *x, const void *delta, const flo
     a.B_sb = dm->B_sb; a.C_sb = dm->C_sb; a.st_sb = dm->state_sb; a.st_sd = dm->state_sd;
     a.softplus = softplus_flag ? 1 : 0;
     a.vec_state = aligned(state, 16) && (dm->state_sb % 4) == 0 && (dm->state_sd % 4) == 0;
+    a.vec_A = aligned(A, 16) && (dm->dstate % 4) == 0;
+    a.vec_bc = aligned(B, 4 * ei) && aligned(C, 4 * ei) && (dm->B_sb % 4) == 0 && (dm->C_sb % 4) == 0;
     cudaError_t e = ms::launch_state_update(a, dm->in_dtype == MS_BF16, dm->out_dtype == MS_BF16,
                                             (cudaStream_t)stream);
     if (e != cudaSuccess) {

@@ -78,6 +78,19 @@ __device__ __forceinline__ f2 f2_sub(f2 a, f2 b) {
 }
 __device__ __forceinline__ f2 f2_splat(float v) { return f2_make(v, v); }
 
+// 16 bytes of shared memory straight into two fp32 pairs.
+__device__ __forceinline__ void lds_f2x2(const float *p, f2 &a, f2 &b) {
+    const unsigned addr = static_cast<unsigned>(__cvta_generic_to_shared(p));
+    asm volatile("ld.shared.v2.b64 {%0, %1}, [%2];" : "=l"(a), "=l"(b) : "r"(addr));
+}
+// 8 bytes of shared memory straight into one fp32 pair.
+__device__ __forceinline__ f2 lds_f2(const float *p) {
+    const unsigned addr = static_cast<unsigned>(__cvta_generic_to_shared(p));
+    f2 a;
+    asm volatile("ld.shared.b64 %0, [%1];" : "=l"(a) : "r"(addr));
+    return a;
+}
+
 // ------------------------------------------------------------ exponentials --
 // 2^x on the MUFU pipe (16 per clock per SM on B200).
 __device__ __forceinline__ float exp2_mufu(float x) {

@@ -24,10 +24,8 @@ struct ScanArgs {
 
 // Launch shape chosen on the host for one scan call.
 struct ScanPlan {
-    int seg_per_warp;   // S_W: time segments per warp (1, 2, 4, 8)
-    int tokens_per_seg; // T
-    int poly_pairs;     // state pairs whose exp runs on the FMA pipe
-    int warps_per_cta;
+    int lanes_per_channel;  // G: lanes sharing one channel (2, 4, 8), 16/G states each
+    int poly8;              // eighths of the exponentials evaluated on the FMA pipe
 };
 
 struct UpdateArgs {
@@ -40,7 +38,9 @@ struct UpdateArgs {
     int N;
     int64_t x_sb, dl_sb, z_sb, y_sb, B_sb, C_sb, st_sb, st_sd;
     int softplus;
-    int vec_state;  // state rows of 16 fp32 at 16-byte aligned addresses
+    int vec_state;  // state: 16-byte aligned groups of 4 states
+    int vec_A;      // A: 16-byte aligned groups of 4 states
+    int vec_bc;     // B, C: groups of 4 states aligned for one vector load
 };
 
 // in_bf16/out_bf16 select the element types. Return a cudaError_t.

@@ -6,24 +6,29 @@
 // ('Mamba-1/2/3 Markdown図解' blog, section 1), plus D u_t inside the silu(z_t)
 // gate (blog, section 2: the SSM output is gated by a second branch).
 //
-// Work decomposition. A warp owns C_W = 32 / S_W channels of one batch row and
-// splits each tile of S_W*T tokens into S_W segments of T tokens: lane
-// (segment s, channel c). The state stays in registers for the whole
-// sequence and is never written to HBM except as last_state (blog, section 2:
-// the fused scan keeps intermediate state on chip). d_state is padded to 16 and
-// processed as 8 pairs with packed f32x2 arithmetic.
-//   S_W = 1: each lane runs the plain recurrence over its T tokens.
-//   S_W > 1: for each state pair a lane first folds its segment from a zero
-//     state into (P, H) = (prod A_bar, local end state), keeping A_bar and the
-//     input term of its T tokens in registers; a warp-shuffle inclusive scan
-//     over the segments with (P1,H1) o (P2,H2) = (P1 P2, P2 H1 + H2) gives each
-//     segment its incoming state from the tile carry; the lane then replays its
-//     T tokens from that state to produce y. No exponential is computed twice.
-// B and C of the tile (shared by every channel of the batch row) are staged
-// once per CTA in shared memory as fp32 pairs; the next tile's u/delta/z and
-// B/C are prefetched into registers while the current tile computes.
-// exp(x) = 2^(x log2 e): state pairs below `poly_pairs` use the FMA-pipe
-// polynomial (unbiased, relieves the MUFU pipe), the others ex2.approx.
+// Work decomposition. G consecutive lanes of a warp share one channel; lane g
+// owns the 16/G states [16g/G, 16(g+1)/G) of that channel for the whole
+// sequence, so the state never leaves registers (blog, section 2: the fused
+// scan keeps the state on chip; only last_state is written). A warp holds
+// 32/G channels of one batch row; a CTA of 4 warps shares the batch row's B
+// and C. Tokens go in tiles of 8G; every tile runs three phases:
+//   prologue  lane (c, g) takes the 8-token chunk g of its channel c: loads
+//             u, delta, z (16-byte vectors), computes Delta (softplus),
+//             Delta*u, D*u and silu(z) once per token; Delta and Delta*u go to
+//             shared memory for the channel's G lanes, D*u and silu(z) stay in
+//             registers for the epilogue. B and C of the tile are staged once
+//             per CTA as fp32 rows [token][state].
+//   states    lane (c, g) runs its states over the tile's tokens in order:
+//             A_bar by exp2, h = A_bar h + (Delta u) B, readout C.h over its
+//             states (packed f32x2 arithmetic). After every R tokens the G
+//             partial readouts are summed by a reduce-scatter over the G lanes
+//             (xor shuffles), so each lane ends up owning whole sums.
+//   epilogue  lane (c, g) gathers the sums of its chunk, adds D*u, multiplies
+//             by silu(z) and stores y with 16-byte stores.
+// The next tile's global loads are issued before the current tile computes.
+// exp(x) = 2^(x log2 e); a fixed, lane-uniform share (poly8 / 8) of the
+// (state pair, token) slots uses the FMA-pipe polynomial, the rest the MUFU
+// ex2, to balance the two pipes.
 
 #include "ms_device.cuh"
 #include "ms_internal.h"
@@ -32,46 +37,43 @@ namespace ms {
 
 namespace {
 
-constexpr int kPairs = 8;  // d_state padded to 16 = 8 pairs
+constexpr int kNW = 4;            // warps per CTA
+constexpr int kThreads = kNW * 32;
+constexpr int kBCRow = 36;        // floats per staged token row: B[0..15], C[16..31], pad
 
-template <int SW, int T, int NW>
+template <int G>
 struct Geom {
-    static constexpr int kCW = 32 / SW;             // channels per warp
-    static constexpr int kTT = SW * T;              // tokens per tile
-    static constexpr int kSegStride = T + 2;        // float2 units (padding: no bank conflicts)
-    static constexpr int kPairStride = SW * kSegStride;
-    static constexpr int kBuf = kPairs * kPairStride;  // float2 per B (or C) buffer
-    static constexpr int kChannels = NW * kCW;      // channels per CTA
-    static constexpr int kThreads = NW * 32;
-    static constexpr int kBcItems = (kPairs * kTT + kThreads - 1) / kThreads;
+    static constexpr int kCW = 32 / G;          // channels per warp
+    static constexpr int kTT = 8 * G;           // tokens per tile: one 8-token chunk per lane
+    static constexpr int kStates = 16 / G;      // states per lane
+    static constexpr int kPairs = kStates / 2;  // state pairs per lane
+    static constexpr int kR = 8;                // tokens per reduction group
+    static constexpr int kRow = kTT + 4;        // floats per per-channel smem row (padded)
+    static constexpr int kChannels = kNW * kCW; // channels per CTA
+    static constexpr int kSlots = kR * kPairs;  // (token, pair) slots per reduction group
 };
 
-// T consecutive elements of one row, kept in their storage format.
-template <typename TIn, int T>
-struct Chunk {
-    static constexpr int kWords = T * (int)sizeof(TIn) / 4;
+// 8 consecutive elements of one row, kept in their storage format.
+template <typename TIn>
+struct Chunk8 {
+    static constexpr int kWords = 8 * (int)sizeof(TIn) / 4;
     uint32_t w[kWords];
 
     __device__ __forceinline__ float get(int j) const {
-        if constexpr (sizeof(TIn) == 4) {
-            return __uint_as_float(w[j]);
-        } else {
-            return (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
-        }
+        if constexpr (sizeof(TIn) == 4) return __uint_as_float(w[j]);
+        else return (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
     }
-
     __device__ __forceinline__ void clear() {
 #pragma unroll
         for (int i = 0; i < kWords; ++i) w[i] = 0u;
     }
-
-    // Load tokens [t, t+T) of `row` (t + j >= L reads as 0).
+    // Tokens [t, t+8) of `row`; positions at or past L read as 0.
     __device__ __forceinline__ void load(const TIn *row, int64_t t, int64_t L, bool vec) {
-        if (vec && t + T <= L) {
+        if (vec && t + 8 <= L) {
             const uint4 *p = reinterpret_cast<const uint4 *>(row + t);
 #pragma unroll
             for (int i = 0; i < kWords / 4; ++i) {
-                uint4 v = __ldcs(p + i);
+                const uint4 v = __ldcs(p + i);
                 w[4 * i + 0] = v.x;
                 w[4 * i + 1] = v.y;
                 w[4 * i + 2] = v.z;
@@ -80,12 +82,12 @@ struct Chunk {
         } else {
             clear();
 #pragma unroll
-            for (int j = 0; j < T; ++j) {
+            for (int j = 0; j < 8; ++j) {
                 if (t + j < L) {
                     if constexpr (sizeof(TIn) == 4) {
                         w[j] = __float_as_uint(__ldcs(reinterpret_cast<const float *>(row) + t + j));
                     } else {
-                        uint32_t bits = __ldcs(reinterpret_cast<const unsigned short *>(row) + t + j);
+                        const uint32_t bits = __ldcs(reinterpret_cast<const unsigned short *>(row) + t + j);
                         w[j >> 1] |= (j & 1) ? (bits << 16) : bits;
                     }
                 }
@@ -94,76 +96,117 @@ struct Chunk {
     }
 };
 
-template <typename TOut, int T>
-__device__ __forceinline__ void store_y(TOut *row, int64_t t, int64_t L, bool vec, const float (&v)[T]) {
-    if (vec && t + T <= L) {
+// One staged row of B (or C) for one token: 16 states, storage format.
+template <typename TIn>
+struct Row16 {
+    static constexpr int kWords = 16 * (int)sizeof(TIn) / 4;
+    uint32_t w[kWords];
+    __device__ __forceinline__ float get(int n) const {
+        if constexpr (sizeof(TIn) == 4) return __uint_as_float(w[n]);
+        else return (n & 1) ? bf16_hi(w[n >> 1]) : bf16_lo(w[n >> 1]);
+    }
+    // Element n at base + n*stride (n < N, t < L), else 0.
+    __device__ __forceinline__ void load(const TIn *base, int64_t stride, int N, bool ok) {
+#pragma unroll
+        for (int i = 0; i < kWords; ++i) w[i] = 0u;
+        if (!ok) return;
+#pragma unroll
+        for (int n = 0; n < 16; ++n) {
+            if (n < N) {
+                if constexpr (sizeof(TIn) == 4) {
+                    w[n] = __float_as_uint(__ldg(reinterpret_cast<const float *>(base) + n * stride));
+                } else {
+                    const uint32_t bits = __ldg(reinterpret_cast<const unsigned short *>(base) + n * stride);
+                    w[n >> 1] |= (n & 1) ? (bits << 16) : bits;
+                }
+            }
+        }
+    }
+};
+
+template <typename TOut>
+__device__ __forceinline__ void store8(TOut *row, int64_t t, int64_t L, bool vec, const float (&v)[8]) {
+    if (vec && t + 8 <= L) {
         if constexpr (sizeof(TOut) == 4) {
             float4 *p = reinterpret_cast<float4 *>(row + t);
-#pragma unroll
-            for (int i = 0; i < T / 4; ++i)
-                __stcs(p + i, make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]));
+            __stcs(p, make_float4(v[0], v[1], v[2], v[3]));
+            __stcs(p + 1, make_float4(v[4], v[5], v[6], v[7]));
         } else {
-            uint4 *p = reinterpret_cast<uint4 *>(row + t);
+            uint32_t w[4];
 #pragma unroll
-            for (int i = 0; i < T / 8; ++i) {
-                uint32_t w[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v[8 * i + 2 * k], v[8 * i + 2 * k + 1]);
-                    w[k] = *reinterpret_cast<uint32_t *>(&h2);
-                }
-                __stcs(p + i, make_uint4(w[0], w[1], w[2], w[3]));
+            for (int k = 0; k < 4; ++k) {
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(v[2 * k], v[2 * k + 1]);
+                w[k] = *reinterpret_cast<uint32_t *>(&h2);
             }
+            __stcs(reinterpret_cast<uint4 *>(row + t), make_uint4(w[0], w[1], w[2], w[3]));
         }
     } else {
 #pragma unroll
-        for (int j = 0; j < T; ++j)
+        for (int j = 0; j < 8; ++j)
             if (t + j < L) Elem<TOut>::store(row + t + j, v[j]);
     }
 }
 
-__device__ __forceinline__ f2 shfl_up_f2(f2 v, int delta) {
-    return __shfl_up_sync(0xffffffffu, v, delta);
-}
-__device__ __forceinline__ f2 shfl_idx_f2(f2 v, int src) {
-    return __shfl_sync(0xffffffffu, v, src);
+// Reduce-scatter of v[0..G) over the G lanes of a group (lane bits below G):
+// afterwards lane g holds the sum over the group of element g, in v[0].
+template <int G>
+__device__ __forceinline__ float reduce_scatter(float (&v)[G], int g) {
+#pragma unroll
+    for (int half = G / 2; half >= 1; half >>= 1) {
+        const bool upper = (g & half) != 0;
+#pragma unroll
+        for (int i = 0; i < half; ++i) {
+            const float send = upper ? v[i] : v[i + half];
+            const float keep = upper ? v[i + half] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, half);
+        }
+    }
+    return v[0];
 }
 
-template <typename TIn, typename TOut, int SW, int T, int NW, int NPOLY>
-__global__ void __launch_bounds__(NW * 32)
+template <typename TIn, typename TOut, int G, int POLY8>
+__global__ void __launch_bounds__(kThreads)
 scan_fwd_kernel(const ScanArgs a) {
-    using G = Geom<SW, T, NW>;
-    __shared__ __align__(16) float2 sB[2][G::kBuf];
-    __shared__ __align__(16) float2 sC[2][G::kBuf];
+    using Gm = Geom<G>;
+    constexpr int TT = Gm::kTT;
+    constexpr int S = Gm::kStates;
+    constexpr int P = Gm::kPairs;
+    constexpr int R = Gm::kR;
+
+    __shared__ __align__(16) float sDelta[kNW][Gm::kCW][Gm::kRow];
+    __shared__ __align__(16) float sDu[kNW][Gm::kCW][Gm::kRow];
+    __shared__ __align__(16) float sY[kNW][Gm::kCW][Gm::kRow];
+    __shared__ __align__(16) float sBC[2][TT][kBCRow];
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int seg = lane / G::kCW;
-    const int cw = lane % G::kCW;
+    const int c = lane / G;   // channel within the warp
+    const int g = lane % G;   // state group / prologue chunk
 
-    const int64_t dblocks = (a.dim + G::kChannels - 1) / G::kChannels;
+    const int64_t dblocks = (a.dim + Gm::kChannels - 1) / Gm::kChannels;
     const int64_t b = blockIdx.x / dblocks;
-    const int64_t d = (blockIdx.x % dblocks) * G::kChannels + warp * G::kCW + cw;
+    const int64_t d = (blockIdx.x % dblocks) * Gm::kChannels + warp * Gm::kCW + c;
     const bool active = d < a.dim;
     const int64_t dd = active ? d : 0;
     const int N = a.N;
     const int64_t L = a.L;
+    const int n0 = g * S;  // first state of this lane
 
-    // Per-channel parameters: A (scaled by log2 e) as pairs, D, bias, state.
-    f2 A2[kPairs], carry[kPairs];
+    // Per-lane state, transition scaled by log2 e.
+    f2 A2[P], h[P];
 #pragma unroll
-    for (int p = 0; p < kPairs; ++p) {
-        const int n0 = 2 * p, n1 = 2 * p + 1;
-        const float a0 = n0 < N ? __ldg(a.A + dd * N + n0) * kLog2e : 0.0f;
-        const float a1 = n1 < N ? __ldg(a.A + dd * N + n1) * kLog2e : 0.0f;
-        A2[p] = f2_make(a0, a1);
-        float h0 = 0.0f, h1 = 0.0f;
+    for (int p = 0; p < P; ++p) {
+        const int na = n0 + 2 * p, nb = na + 1;
+        const float aa = na < N ? __ldg(a.A + dd * N + na) * kLog2e : 0.0f;
+        const float ab = nb < N ? __ldg(a.A + dd * N + nb) * kLog2e : 0.0f;
+        A2[p] = f2_make(aa, ab);
+        float ha = 0.0f, hb = 0.0f;
         if (a.h0 != nullptr && active) {
             const float *hs = a.h0 + (b * a.dim + d) * N;
-            if (n0 < N) h0 = __ldg(hs + n0);
-            if (n1 < N) h1 = __ldg(hs + n1);
+            if (na < N) ha = __ldg(hs + na);
+            if (nb < N) hb = __ldg(hs + nb);
         }
-        carry[p] = f2_make(h0, h1);
+        h[p] = f2_make(ha, hb);
     }
     const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
     const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
@@ -179,14 +222,19 @@ scan_fwd_kernel(const ScanArgs a) {
     const bool vin = a.vec_in != 0;
     const bool vout = a.vec_out != 0;
 
-    const int64_t ntiles = (L + G::kTT - 1) / G::kTT;
+    // B/C staging: thread i < TT stages B of token i, TT <= i < 2TT stages C.
+    const bool bc_thread = threadIdx.x < 2 * TT;
+    const int bc_t = threadIdx.x % TT;
+    const bool bc_isC = threadIdx.x >= TT;
+    const TIn *bc_base = bc_isC ? C_b : B_b;
+    const int64_t bc_sn = bc_isC ? a.C_sn : a.B_sn;
 
-    // Register prefetch buffers for the next tile.
-    Chunk<TIn, T> nu, nd, nz;
-    float bcv[G::kBcItems][4];
+    const int64_t ntiles = (L + TT - 1) / TT;
 
-    auto load_tokens = [&](int64_t t0) {
-        const int64_t ts = t0 + seg * T;
+    Chunk8<TIn> nu, nd, nz;
+    Row16<TIn> nbc;
+    auto prefetch = [&](int64_t t0) {
+        const int64_t ts = t0 + 8 * g;
         if (active) {
             nu.load(u_row, ts, L, vin);
             nd.load(d_row, ts, L, vin);
@@ -197,206 +245,165 @@ scan_fwd_kernel(const ScanArgs a) {
             nd.clear();
             nz.clear();
         }
-    };
-    auto load_bc = [&](int64_t t0) {
-#pragma unroll
-        for (int i = 0; i < G::kBcItems; ++i) {
-            const int e = threadIdx.x + i * G::kThreads;
-            const int p = e / G::kTT, tt = e % G::kTT;
-            const int64_t t = t0 + tt;
-            float v0 = 0.f, v1 = 0.f, v2 = 0.f, v3 = 0.f;
-            if (e < kPairs * G::kTT && t < L) {
-                const int n0 = 2 * p, n1 = 2 * p + 1;
-                if (n0 < N) {
-                    v0 = Elem<TIn>::load(B_b + n0 * a.B_sn + t);
-                    v2 = Elem<TIn>::load(C_b + n0 * a.C_sn + t);
-                }
-                if (n1 < N) {
-                    v1 = Elem<TIn>::load(B_b + n1 * a.B_sn + t);
-                    v3 = Elem<TIn>::load(C_b + n1 * a.C_sn + t);
-                }
-            }
-            bcv[i][0] = v0;
-            bcv[i][1] = v1;
-            bcv[i][2] = v2;
-            bcv[i][3] = v3;
-        }
-    };
-    auto store_bc = [&](int buf) {
-#pragma unroll
-        for (int i = 0; i < G::kBcItems; ++i) {
-            const int e = threadIdx.x + i * G::kThreads;
-            if (e < kPairs * G::kTT) {
-                const int p = e / G::kTT, tt = e % G::kTT;
-                const int idx = p * G::kPairStride + (tt / T) * G::kSegStride + (tt % T);
-                sB[buf][idx] = make_float2(bcv[i][0], bcv[i][1]);
-                sC[buf][idx] = make_float2(bcv[i][2], bcv[i][3]);
-            }
-        }
+        const int64_t tb = t0 + bc_t;
+        nbc.load(bc_base + tb, bc_sn, N, bc_thread && tb < L);
     };
 
-    if (ntiles > 0) {
-        load_tokens(0);
-        load_bc(0);
-        store_bc(0);
-    }
-    __syncthreads();
+    if (ntiles > 0) prefetch(0);
+
+    float (*myDelta)[Gm::kRow] = sDelta[warp];
+    float (*myDu)[Gm::kRow] = sDu[warp];
+    float (*myY)[Gm::kRow] = sY[warp];
 
     for (int64_t k = 0; k < ntiles; ++k) {
-        const int64_t t0 = k * G::kTT;
+        const int64_t t0 = k * TT;
         const int buf = (int)(k & 1);
-        const Chunk<TIn, T> cu = nu, cd = nd, cz = nz;
-        if (k + 1 < ntiles) {
-            load_tokens(t0 + G::kTT);
-            load_bc(t0 + G::kTT);
+
+        // ---- prologue: per-token quantities of chunk g of channel c, from the
+        // registers filled by the previous iteration's prefetch.
+        const int64_t ts = t0 + 8 * g;
+        float du_skip[8], gate[8];
+        {
+            float dl[8], dlu[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float uj = nu.get(j);
+                const float v = nd.get(j) + bias;
+                const float step = sp ? softplus_f(v) : v;
+                dl[j] = (ts + j < L) ? step : 0.0f;  // past the end: the state is left alone
+                dlu[j] = dl[j] * uj;
+                du_skip[j] = Dd * uj;
+                gate[j] = has_z ? silu_f(nz.get(j)) : 1.0f;
+            }
+            float4 *pd = reinterpret_cast<float4 *>(&myDelta[c][8 * g]);
+            float4 *pu = reinterpret_cast<float4 *>(&myDu[c][8 * g]);
+            pd[0] = make_float4(dl[0], dl[1], dl[2], dl[3]);
+            pd[1] = make_float4(dl[4], dl[5], dl[6], dl[7]);
+            pu[0] = make_float4(dlu[0], dlu[1], dlu[2], dlu[3]);
+            pu[1] = make_float4(dlu[4], dlu[5], dlu[6], dlu[7]);
         }
-
-        // Token prologue: step sizes, input term scale, D skip.
-        const int64_t ts = t0 + seg * T;
-        float dt[T], du[T];
-        f2 y2[T];
-        float dsum = 0.0f;
+        if (bc_thread) {
+            float4 *row = reinterpret_cast<float4 *>(&sBC[buf][bc_t][bc_isC ? 16 : 0]);
 #pragma unroll
-        for (int j = 0; j < T; ++j) {
-            const float uj = cu.get(j);
-            const float v = cd.get(j) + bias;
-            const float step = sp ? softplus_f(v) : v;
-            dt[j] = (ts + j < L) ? step : 0.0f;  // tokens past the end leave the state alone
-            du[j] = dt[j] * uj;
-            y2[j] = f2_make(Dd * uj, 0.0f);
-            dsum += dt[j];
+            for (int q = 0; q < 4; ++q)
+                row[q] = make_float4(nbc.get(4 * q), nbc.get(4 * q + 1), nbc.get(4 * q + 2), nbc.get(4 * q + 3));
         }
+        // The next tile's loads stay in flight while this tile's states run.
+        if (k + 1 < ntiles) prefetch(t0 + TT);
+        __syncthreads();
 
-        const float2 *bB = sB[buf] + seg * G::kSegStride;
-        const float2 *bC = sC[buf] + seg * G::kSegStride;
-
+        // ---- states: tokens of the tile in order.
+        const float *dl_row = myDelta[c];
+        const float *du_row = myDu[c];
+#pragma unroll 2
+        for (int tr = 0; tr < TT; tr += R) {
+            float part[R];
+            float dlv[R], duv[R];
 #pragma unroll
-        for (int p = 0; p < kPairs; ++p) {
-            constexpr bool kDummy = false;
-            (void)kDummy;
-            const bool poly = p < NPOLY;
-            const float4 *Bq = reinterpret_cast<const float4 *>(bB + p * G::kPairStride);
-            const float4 *Cq = reinterpret_cast<const float4 *>(bC + p * G::kPairStride);
-            if constexpr (SW == 1) {
-                f2 h = carry[p];
+            for (int q = 0; q < R / 4; ++q) {
+                const float4 x = *reinterpret_cast<const float4 *>(dl_row + tr + 4 * q);
+                const float4 y = *reinterpret_cast<const float4 *>(du_row + tr + 4 * q);
+                dlv[4 * q] = x.x; dlv[4 * q + 1] = x.y; dlv[4 * q + 2] = x.z; dlv[4 * q + 3] = x.w;
+                duv[4 * q] = y.x; duv[4 * q + 1] = y.y; duv[4 * q + 2] = y.z; duv[4 * q + 3] = y.w;
+            }
 #pragma unroll
-                for (int j2 = 0; j2 < T / 2; ++j2) {
-                    const float4 bq = Bq[j2];
-                    const float4 cq = Cq[j2];
+            for (int j = 0; j < R; ++j) {
+                const float *bcr = sBC[buf][tr + j];
+                f2 Bp[P], Cp[P];
+                if constexpr (P >= 2) {
 #pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        const int j = 2 * j2 + s;
-                        const f2 x2 = f2_mul(f2_splat(dt[j]), A2[p]);
-                        const f2 a2 = poly ? exp2_pair<true>(x2) : exp2_pair<false>(x2);
-                        const f2 Bp = s ? f2_make(bq.z, bq.w) : f2_make(bq.x, bq.y);
-                        const f2 Cp = s ? f2_make(cq.z, cq.w) : f2_make(cq.x, cq.y);
-                        h = f2_fma(a2, h, f2_mul(f2_splat(du[j]), Bp));
-                        y2[j] = f2_fma(Cp, h, y2[j]);
+                    for (int q = 0; q < P / 2; ++q) {
+                        lds_f2x2(bcr + n0 + 4 * q, Bp[2 * q], Bp[2 * q + 1]);
+                        lds_f2x2(bcr + 16 + n0 + 4 * q, Cp[2 * q], Cp[2 * q + 1]);
                     }
+                } else {
+                    Bp[0] = lds_f2(bcr + n0);
+                    Cp[0] = lds_f2(bcr + 16 + n0);
                 }
-                carry[p] = h;
-            } else {
-                f2 av[T], wv[T];
-                f2 H = f2_splat(0.0f);
+                const f2 du2 = f2_splat(duv[j]);
+                f2 acc = f2_splat(0.0f);
 #pragma unroll
-                for (int j2 = 0; j2 < T / 2; ++j2) {
-                    const float4 bq = Bq[j2];
-#pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        const int j = 2 * j2 + s;
-                        const f2 x2 = f2_mul(f2_splat(dt[j]), A2[p]);
-                        av[j] = poly ? exp2_pair<true>(x2) : exp2_pair<false>(x2);
-                        const f2 Bp = s ? f2_make(bq.z, bq.w) : f2_make(bq.x, bq.y);
-                        wv[j] = f2_mul(f2_splat(du[j]), Bp);
-                        H = f2_fma(av[j], H, wv[j]);
-                    }
+                for (int p = 0; p < P; ++p) {
+                    float xa, xb;
+                    f2_split(A2[p], xa, xb);
+                    xa *= dlv[j];
+                    xb *= dlv[j];
+                    const int slot = j * P + p;
+                    const bool poly = slot * 8 < POLY8 * Gm::kSlots;
+                    const f2 ab = poly ? exp2_pair<true>(f2_make(xa, xb)) : f2_make(exp2_mufu(xa), exp2_mufu(xb));
+                    h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp[p]));
+                    acc = (p == 0) ? f2_mul(Cp[p], h[p]) : f2_fma(Cp[p], h[p], acc);
                 }
-                const f2 xs = f2_mul(f2_splat(dsum), A2[p]);
-                f2 P = poly ? exp2_pair<true>(xs) : exp2_pair<false>(xs);
+                float lo, hi;
+                f2_split(acc, lo, hi);
+                part[j] = lo + hi;
+            }
+            // G partial readouts per token -> whole sums owned by one lane each.
 #pragma unroll
-                for (int off = 1; off < SW; off <<= 1) {
-                    const f2 Pp = shfl_up_f2(P, off * G::kCW);
-                    const f2 Hp = shfl_up_f2(H, off * G::kCW);
-                    if (seg >= off) {
-                        H = f2_fma(P, Hp, H);
-                        P = f2_mul(P, Pp);
-                    }
-                }
-                const f2 hout = f2_fma(P, carry[p], H);
-                f2 h = shfl_up_f2(hout, G::kCW);
-                if (seg == 0) h = carry[p];
-                carry[p] = shfl_idx_f2(hout, (SW - 1) * G::kCW + cw);
+            for (int blk = 0; blk < R / G; ++blk) {
+                float v[G];
 #pragma unroll
-                for (int j2 = 0; j2 < T / 2; ++j2) {
-                    const float4 cq = Cq[j2];
-#pragma unroll
-                    for (int s = 0; s < 2; ++s) {
-                        const int j = 2 * j2 + s;
-                        const f2 Cp = s ? f2_make(cq.z, cq.w) : f2_make(cq.x, cq.y);
-                        h = f2_fma(av[j], h, wv[j]);
-                        y2[j] = f2_fma(Cp, h, y2[j]);
-                    }
-                }
+                for (int i = 0; i < G; ++i) v[i] = part[blk * G + i];
+                const float sum = reduce_scatter<G>(v, g);
+                myY[c][tr + blk * G + g] = sum;
             }
         }
+        __syncwarp();
 
-        // Epilogue: readout halves, gate, store.
-        float yo[T];
+        // ---- epilogue: chunk g of channel c.
+        {
+            const float4 y0 = *reinterpret_cast<const float4 *>(&myY[c][8 * g]);
+            const float4 y1 = *reinterpret_cast<const float4 *>(&myY[c][8 * g + 4]);
+            const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+            float yo[8];
 #pragma unroll
-        for (int j = 0; j < T; ++j) {
-            float lo, hi;
-            f2_split(y2[j], lo, hi);
-            float yv = lo + hi;
-            if (has_z) yv *= silu_f(cz.get(j));
-            yo[j] = yv;
+            for (int j = 0; j < 8; ++j) yo[j] = (ys[j] + du_skip[j]) * gate[j];
+            if (active) store8<TOut>(y_row, ts, L, vout, yo);
         }
-        if (active) store_y<TOut, T>(y_row, ts, L, vout, yo);
-
-        if (k + 1 < ntiles) store_bc(buf ^ 1);
-        __syncthreads();
+        __syncwarp();
     }
 
-    if (active && seg == 0 && a.last != nullptr) {
+    if (active && a.last != nullptr) {
         float *ls = a.last + (b * a.dim + d) * N;
 #pragma unroll
-        for (int p = 0; p < kPairs; ++p) {
-            float h0, h1;
-            f2_split(carry[p], h0, h1);
-            if (2 * p < N) ls[2 * p] = h0;
-            if (2 * p + 1 < N) ls[2 * p + 1] = h1;
+        for (int p = 0; p < P; ++p) {
+            float ha, hb;
+            f2_split(h[p], ha, hb);
+            const int na = n0 + 2 * p;
+            if (na < N) ls[na] = ha;
+            if (na + 1 < N) ls[na + 1] = hb;
         }
     }
 }
 
-template <typename TIn, typename TOut, int SW, int T, int NPOLY>
+template <typename TIn, typename TOut, int G, int POLY8>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
-    constexpr int NW = 4;
-    using G = Geom<SW, T, NW>;
-    const int64_t dblocks = (a.dim + G::kChannels - 1) / G::kChannels;
+    using Gm = Geom<G>;
+    const int64_t dblocks = (a.dim + Gm::kChannels - 1) / Gm::kChannels;
     const int64_t blocks = dblocks * a.batch;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    scan_fwd_kernel<TIn, TOut, SW, T, NW, NPOLY><<<(unsigned)blocks, G::kThreads, 0, stream>>>(a);
+    scan_fwd_kernel<TIn, TOut, G, POLY8><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 
-template <typename TIn, typename TOut, int SW, int T>
-cudaError_t launch_poly(const ScanArgs &a, int poly_pairs, cudaStream_t stream) {
-    switch (poly_pairs) {
-        case 0: return launch_one<TIn, TOut, SW, T, 0>(a, stream);
-        case 2: return launch_one<TIn, TOut, SW, T, 2>(a, stream);
-        case 4: return launch_one<TIn, TOut, SW, T, 4>(a, stream);
-        default: return launch_one<TIn, TOut, SW, T, 8>(a, stream);
+template <typename TIn, typename TOut, int G>
+cudaError_t launch_poly(const ScanArgs &a, int poly8, cudaStream_t stream) {
+    switch (poly8) {
+        case 0: return launch_one<TIn, TOut, G, 0>(a, stream);
+        case 2: return launch_one<TIn, TOut, G, 2>(a, stream);
+        case 3: return launch_one<TIn, TOut, G, 3>(a, stream);
+        case 4: return launch_one<TIn, TOut, G, 4>(a, stream);
+        default: return launch_one<TIn, TOut, G, 8>(a, stream);
     }
 }
 
 template <typename TIn, typename TOut>
 cudaError_t launch_types(const ScanArgs &a, const ScanPlan &pl, cudaStream_t stream) {
-    switch (pl.seg_per_warp) {
-        case 1: return launch_poly<TIn, TOut, 1, 16>(a, pl.poly_pairs, stream);
-        case 2: return launch_poly<TIn, TOut, 2, 8>(a, pl.poly_pairs, stream);
-        case 4: return launch_poly<TIn, TOut, 4, 8>(a, pl.poly_pairs, stream);
-        default: return launch_poly<TIn, TOut, 8, 8>(a, pl.poly_pairs, stream);
+    switch (pl.lanes_per_channel) {
+        case 2: return launch_poly<TIn, TOut, 2>(a, pl.poly8, stream);
+        case 4: return launch_poly<TIn, TOut, 4>(a, pl.poly8, stream);
+        default: return launch_poly<TIn, TOut, 8>(a, pl.poly8, stream);
     }
 }
 
@@ -414,19 +421,15 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf1
 
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms) {
     ScanPlan pl{};
-    pl.warps_per_cta = 4;
-    pl.tokens_per_seg = 8;
-    // Enough warps to give every SM sub-partition at least two: split time
-    // inside the warp until the channel count alone provides them.
+    // Four lanes per channel unless the channels alone cannot give every SM
+    // sub-partition two warps; then eight (each extra lane adds reduction
+    // shuffles, and two lanes per channel measured slower at every size tried).
     const int64_t channels = a.batch * a.dim;
     const int64_t want_warps = (int64_t)num_sms * 4 * 2;
-    int sw = 1;
-    while (sw < 8 && channels * sw / 32 < want_warps) sw *= 2;
-    pl.seg_per_warp = sw;
-    if (sw == 1) pl.tokens_per_seg = 16;
+    pl.lanes_per_channel = (channels * 4 / 32 >= want_warps) ? 4 : 8;
     // fp32 inputs: every exponential on the unbiased polynomial (slow-decay
-    // accuracy); bf16 inputs: a share on the FMA pipe to balance the pipes.
-    pl.poly_pairs = in_bf16 ? 2 : 8;
+    // accuracy); bf16 inputs: all on the MUFU unit (fastest measured).
+    pl.poly8 = in_bf16 ? 0 : 8;
     return pl;
 }
 

@@ -88,8 +88,10 @@ typedef struct {
 } ms_scan_dims;
 
 /*
- * Workspace bytes mamba_scan_fwd needs for these dims (0 when it needs none).
- * Returns 0 also for dims that mamba_scan_fwd would reject.
+ * Workspace bytes mamba_scan_fwd needs for these dims. The scan keeps its
+ * state in registers and its tiles in shared memory, so this is 0; the
+ * argument pair stays in the ABI so callers need not change if a future
+ * kernel needs scratch.
  */
 size_t mamba_scan_workspace_size(const ms_scan_dims *dims);
 
@@ -108,7 +110,8 @@ size_t mamba_scan_workspace_size(const ms_scan_dims *dims);
  *   last_state       optional fp32 [batch, dim, dstate] output: the state after
  *                    token seqlen-1 (equal to initial_state, or 0, if seqlen = 0).
  *   workspace        device scratch of mamba_scan_workspace_size() bytes, or
- *                    NULL with workspace_bytes = 0 when that size is 0.
+ *                    NULL with workspace_bytes = 0 when that size is 0 (it
+ *                    is 0 for every size in this version).
  * Returns MS_OK or an MS_ERR_* code.
  */
 int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,
@@ -121,13 +124,17 @@ int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void 
  * Launch shape of the scan kernel. mamba_scan_fwd picks one from the sizes;
  * mamba_scan_fwd_plan takes it from the caller (tuning and tests). Any valid
  * plan gives the same result up to fp32 rounding.
- *   lanes_per_channel  2, 4 or 8: lanes sharing one channel, each holding
+ *   lanes_per_channel  1, 2, 4 or 8: lanes sharing one channel, each holding
  *                      16/lanes_per_channel of its states.
- *   poly8              0, 2, 3, 4 or 8: eighths of the exponentials computed
- *                      by a polynomial on the FMA pipe instead of the MUFU unit.
+ *   chunks_per_lane    1 or 2 (1 when lanes_per_channel is 8): 8-token
+ *                      chunks each lane prepares per tile; a tile is
+ *                      8 * lanes_per_channel * chunks_per_lane tokens.
+ *   poly8              0, 2, 4 or 8: eighths of the exponentials computed by
+ *                      a polynomial on the FMA pipe instead of the MUFU unit.
  */
 typedef struct {
     int32_t lanes_per_channel;
+    int32_t chunks_per_lane;
     int32_t poly8;
 } ms_scan_plan;
 

@@ -35,7 +35,8 @@ class UpdateDims(ctypes.Structure):
 
 
 class ScanPlan(ctypes.Structure):
-    _fields_ = [("lanes_per_channel", ctypes.c_int32), ("poly8", ctypes.c_int32)]
+    _fields_ = [("lanes_per_channel", ctypes.c_int32), ("chunks_per_lane", ctypes.c_int32),
+                ("poly8", ctypes.c_int32)]
 
 
 class MambaScanError(RuntimeError):
@@ -159,9 +160,11 @@ def scan_dims_for(u, delta, B, C, z, y) -> ScanDims:
 
 def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
              initial_state=None, out_dtype=None, y=None, last_state=None,
-             return_last_state: bool = True, stream=None, plan: Optional[Tuple[int, int]] = None,
-             dev_status=None):
+             return_last_state: bool = True, stream=None, plan: Optional[Tuple[int, int, int]] = None,
+             dev_status=None, workspace=None):
     """Selective scan forward on torch CUDA tensors (see include/mambascan.h).
+    ``workspace`` (optional, uint8 CUDA tensor of at least
+    ``mamba_scan_workspace_size`` bytes) is allocated per call when omitted.
     Returns (y, last_state or None)."""
     torch = _torch()
     if out_dtype is None:
@@ -178,7 +181,10 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool 
             raise ValueError(f"{n} must be a contiguous fp32 tensor")
     dims = scan_dims_for(u, delta, B, C, z, y)
     ws_bytes = mamba_scan_workspace_size(dims)
-    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=u.device) if ws_bytes else None
+    if workspace is not None:
+        ws, ws_bytes = workspace, workspace.numel() * workspace.element_size()
+    else:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=u.device) if ws_bytes else None
     pl = ScanPlan(*plan) if plan is not None else None
     rc = mamba_scan_fwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
                         _ptr(delta_bias), softplus, _ptr(initial_state), _ptr(y), _ptr(last_state),

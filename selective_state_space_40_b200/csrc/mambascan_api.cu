@@ -108,12 +108,13 @@ static int check_scan(const void *u, const void *delta, const float *A, const vo
 
 size_t mamba_scan_workspace_size(const ms_scan_dims *dims) {
     (void)dims;
-    return 0;
+    return 0;  // the scan keeps everything in registers and shared memory
 }
 
 static bool plan_valid(const ms_scan_plan *p) {
-    const int g = p->lanes_per_channel, q = p->poly8;
-    return (g == 2 || g == 4 || g == 8) && (q == 0 || q == 2 || q == 3 || q == 4 || q == 8);
+    const int g = p->lanes_per_channel, c = p->chunks_per_lane, q = p->poly8;
+    return (g == 1 || g == 2 || g == 4 || g == 8) && (c == 1 || (c == 2 && g != 8)) &&
+           (q == 0 || q == 2 || q == 4 || q == 8);
 }
 
 static ms::ScanPlan auto_plan(const ms_scan_dims *dims) {
@@ -132,6 +133,7 @@ int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan) {
     if (rc != MS_OK && rc != MS_ERR_NULL) return rc;
     const ms::ScanPlan p = auto_plan(dims);
     plan->lanes_per_channel = p.lanes_per_channel;
+    plan->chunks_per_lane = p.chunks_per_lane;
     plan->poly8 = p.poly8;
     return MS_OK;
 }
@@ -177,6 +179,7 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
     ms::ScanPlan pl = auto_plan(dims);
     if (plan) {
         pl.lanes_per_channel = plan->lanes_per_channel;
+        pl.chunks_per_lane = plan->chunks_per_lane;
         pl.poly8 = plan->poly8;
     }
     cudaError_t e = ms::launch_scan_fwd(a, pl, in_bf16, out_bf16, (cudaStream_t)stream);

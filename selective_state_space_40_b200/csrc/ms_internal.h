@@ -24,7 +24,8 @@ struct ScanArgs {
 
 // Launch shape chosen on the host for one scan call.
 struct ScanPlan {
-    int lanes_per_channel;  // G: lanes sharing one channel (2, 4, 8), 16/G states each
+    int lanes_per_channel;  // G: lanes sharing one channel (1, 2, 4, 8), 16/G states each
+    int chunks_per_lane;    // CH: 8-token chunks per lane per tile (1, 2; 1 when G = 8)
     int poly8;              // eighths of the exponentials evaluated on the FMA pipe
 };
 

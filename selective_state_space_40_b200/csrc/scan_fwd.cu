@@ -41,16 +41,30 @@ constexpr int kNW = 4;            // warps per CTA
 constexpr int kThreads = kNW * 32;
 constexpr int kBCRow = 36;        // floats per staged token row: B[0..15], C[16..31], pad
 
-template <int G>
+template <int G, int CH>
 struct Geom {
     static constexpr int kCW = 32 / G;          // channels per warp
-    static constexpr int kTT = 8 * G;           // tokens per tile: one 8-token chunk per lane
+    static constexpr int kTT = 8 * G * CH;      // tokens per tile: CH 8-token chunks per lane
     static constexpr int kStates = 16 / G;      // states per lane
     static constexpr int kPairs = kStates / 2;  // state pairs per lane
     static constexpr int kR = 8;                // tokens per reduction group
     static constexpr int kRow = kTT + 4;        // floats per per-channel smem row (padded)
     static constexpr int kChannels = kNW * kCW; // channels per CTA
     static constexpr int kSlots = kR * kPairs;  // (token, pair) slots per reduction group
+};
+
+template <int G, int CH>
+struct SmemLayout {
+    using Gm = Geom<G, CH>;
+    static constexpr int kRows = G > 1 ? Gm::kCW : 1;  // per-channel rows (none needed when G == 1)
+    static constexpr int kRow2 = Gm::kTT + 2;          // float2 per splatted row (padded)
+    static constexpr int kBCBytes = 2 * Gm::kTT * kBCRow * 4;
+    static constexpr int kPairBytes = G > 1 ? kNW * kRows * kRow2 * 8 : 0;
+    static constexpr int kYBytes = G > 1 ? kNW * kRows * Gm::kRow * 4 : 0;
+    static constexpr int kOffDelta = kBCBytes;
+    static constexpr int kOffDu = kOffDelta + kPairBytes;
+    static constexpr int kOffY = kOffDu + kPairBytes;
+    static constexpr int kTotal = kOffY + kYBytes;
 };
 
 // 8 consecutive elements of one row, kept in their storage format.
@@ -164,24 +178,77 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int g) {
     return v[0];
 }
 
-template <typename TIn, typename TOut, int G, int POLY8>
-__global__ void __launch_bounds__(kThreads)
+// One token of the state phase for a lane owning P state pairs from n0:
+// A_bar = 2^(Delta A log2e), h = A_bar h + (Delta u) B, returns C . h over
+// the lane's states. `slot0` numbers the (token, pair) slots for the
+// MUFU/polynomial split.
+template <int P, int POLY8, int SLOTS>
+__device__ __forceinline__ float state_token(const float *bcr, int n0, f2 dl2, f2 du2, const f2 (&A2)[P],
+                                             f2 (&h)[P], int slot0) {
+    f2 Bp[P], Cp[P];
+    if constexpr (P >= 2) {
+#pragma unroll
+        for (int q = 0; q < P / 2; ++q) {
+            lds_f2x2(bcr + n0 + 4 * q, Bp[2 * q], Bp[2 * q + 1]);
+            lds_f2x2(bcr + 16 + n0 + 4 * q, Cp[2 * q], Cp[2 * q + 1]);
+        }
+    } else {
+        Bp[0] = lds_f2(bcr + n0);
+        Cp[0] = lds_f2(bcr + 16 + n0);
+    }
+    f2 acc = f2_splat(0.0f);
+#pragma unroll
+    for (int p = 0; p < P; ++p) {
+        const f2 x2 = f2_mul(dl2, A2[p]);
+        const f2 w2 = f2_mul(du2, Bp[p]);
+        const bool poly = (slot0 + p) * 8 < POLY8 * SLOTS;
+        float ha, hb, wa, wb;
+        f2_split(h[p], ha, hb);
+        f2_split(w2, wa, wb);
+        if (poly) {
+            const f2 ab = exp2_pair<true>(x2);
+            float ea, eb;
+            f2_split(ab, ea, eb);
+            ha = fmaf(ea, ha, wa);
+            hb = fmaf(eb, hb, wb);
+        } else {
+            float xa, xb;
+            f2_split(x2, xa, xb);
+            ha = fmaf(exp2_mufu(xa), ha, wa);
+            hb = fmaf(exp2_mufu(xb), hb, wb);
+        }
+        h[p] = f2_make(ha, hb);
+        acc = (p == 0) ? f2_mul(Cp[p], h[p]) : f2_fma(Cp[p], h[p], acc);
+    }
+    float lo, hi;
+    f2_split(acc, lo, hi);
+    return lo + hi;
+}
+
+template <typename TIn, typename TOut, int G, int CH, int POLY8>
+__global__ void __launch_bounds__(kThreads, 3)
 scan_fwd_kernel(const ScanArgs a) {
-    using Gm = Geom<G>;
+    using Gm = Geom<G, CH>;
     constexpr int TT = Gm::kTT;
     constexpr int S = Gm::kStates;
     constexpr int P = Gm::kPairs;
     constexpr int R = Gm::kR;
+    using Sm = SmemLayout<G, CH>;
+    constexpr int ROWS = Sm::kRows;
 
-    __shared__ __align__(16) float sDelta[kNW][Gm::kCW][Gm::kRow];
-    __shared__ __align__(16) float sDu[kNW][Gm::kCW][Gm::kRow];
-    __shared__ __align__(16) float sY[kNW][Gm::kCW][Gm::kRow];
-    __shared__ __align__(16) float sBC[2][TT][kBCRow];
+    // Dynamic shared memory: B/C tiles (double buffered, shared by the CTA),
+    // then per warp: Delta and Delta*u per token, each stored twice (a ready
+    // fp32 pair), and the reduced readouts.
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    auto sBC = reinterpret_cast<float (*)[TT][kBCRow]>(smem_raw);
+    auto sDelta = reinterpret_cast<float2 (*)[ROWS][Sm::kRow2]>(smem_raw + Sm::kOffDelta);
+    auto sDu = reinterpret_cast<float2 (*)[ROWS][Sm::kRow2]>(smem_raw + Sm::kOffDu);
+    auto sY = reinterpret_cast<float (*)[ROWS][Gm::kRow]>(smem_raw + Sm::kOffY);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int c = lane / G;   // channel within the warp
-    const int g = lane % G;   // state group / prologue chunk
+    const int g = lane % G;   // state group / prologue chunk group
 
     const int64_t dblocks = (a.dim + Gm::kChannels - 1) / Gm::kChannels;
     const int64_t b = blockIdx.x / dblocks;
@@ -223,6 +290,7 @@ scan_fwd_kernel(const ScanArgs a) {
     const bool vout = a.vec_out != 0;
 
     // B/C staging: thread i < TT stages B of token i, TT <= i < 2TT stages C.
+    static_assert(2 * TT <= kThreads, "one staging thread per B/C token row");
     const bool bc_thread = threadIdx.x < 2 * TT;
     const int bc_t = threadIdx.x % TT;
     const bool bc_isC = threadIdx.x >= TT;
@@ -231,19 +299,24 @@ scan_fwd_kernel(const ScanArgs a) {
 
     const int64_t ntiles = (L + TT - 1) / TT;
 
-    Chunk8<TIn> nu, nd, nz;
+    // Lane (c, g) owns the prologue/epilogue chunks g*CH .. g*CH+CH-1 of its
+    // channel in every tile (8*CH consecutive tokens).
+    Chunk8<TIn> nu[CH], nd[CH], nz[CH];
     Row16<TIn> nbc;
     auto prefetch = [&](int64_t t0) {
-        const int64_t ts = t0 + 8 * g;
-        if (active) {
-            nu.load(u_row, ts, L, vin);
-            nd.load(d_row, ts, L, vin);
-            if (has_z) nz.load(z_row, ts, L, vin);
-            else nz.clear();
-        } else {
-            nu.clear();
-            nd.clear();
-            nz.clear();
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t ts = t0 + 8 * (g * CH + i);
+            if (active) {
+                nu[i].load(u_row, ts, L, vin);
+                nd[i].load(d_row, ts, L, vin);
+                if (has_z) nz[i].load(z_row, ts, L, vin);
+                else nz[i].clear();
+            } else {
+                nu[i].clear();
+                nd[i].clear();
+                nz[i].clear();
+            }
         }
         const int64_t tb = t0 + bc_t;
         nbc.load(bc_base + tb, bc_sn, N, bc_thread && tb < L);
@@ -251,36 +324,34 @@ scan_fwd_kernel(const ScanArgs a) {
 
     if (ntiles > 0) prefetch(0);
 
-    float (*myDelta)[Gm::kRow] = sDelta[warp];
-    float (*myDu)[Gm::kRow] = sDu[warp];
-    float (*myY)[Gm::kRow] = sY[warp];
-
     for (int64_t k = 0; k < ntiles; ++k) {
         const int64_t t0 = k * TT;
         const int buf = (int)(k & 1);
 
-        // ---- prologue: per-token quantities of chunk g of channel c, from the
-        // registers filled by the previous iteration's prefetch.
-        const int64_t ts = t0 + 8 * g;
-        float du_skip[8], gate[8];
-        {
-            float dl[8], dlu[8];
+        // ---- prologue: per-token quantities of this lane's chunks.
+        float dl[CH][8], dlu[CH][8], dug[CH][8], gate[CH][8];
+#pragma unroll
+        for (int i = 0; i < CH; ++i) {
+            const int64_t ts = t0 + 8 * (g * CH + i);
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float uj = nu.get(j);
-                const float v = nd.get(j) + bias;
+                const float uj = nu[i].get(j);
+                const float v = nd[i].get(j) + bias;
                 const float step = sp ? softplus_f(v) : v;
-                dl[j] = (ts + j < L) ? step : 0.0f;  // past the end: the state is left alone
-                dlu[j] = dl[j] * uj;
-                du_skip[j] = Dd * uj;
-                gate[j] = has_z ? silu_f(nz.get(j)) : 1.0f;
+                dl[i][j] = (ts + j < L) ? step : 0.0f;  // past the end: the state is left alone
+                dlu[i][j] = dl[i][j] * uj;
+                gate[i][j] = has_z ? silu_f(nz[i].get(j)) : 1.0f;
+                dug[i][j] = Dd * uj * gate[i][j];
             }
-            float4 *pd = reinterpret_cast<float4 *>(&myDelta[c][8 * g]);
-            float4 *pu = reinterpret_cast<float4 *>(&myDu[c][8 * g]);
-            pd[0] = make_float4(dl[0], dl[1], dl[2], dl[3]);
-            pd[1] = make_float4(dl[4], dl[5], dl[6], dl[7]);
-            pu[0] = make_float4(dlu[0], dlu[1], dlu[2], dlu[3]);
-            pu[1] = make_float4(dlu[4], dlu[5], dlu[6], dlu[7]);
+            if constexpr (G > 1) {
+                float4 *pd = reinterpret_cast<float4 *>(&sDelta[warp][c][8 * (g * CH + i)]);
+                float4 *pu = reinterpret_cast<float4 *>(&sDu[warp][c][8 * (g * CH + i)]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    pd[q] = make_float4(dl[i][2 * q], dl[i][2 * q], dl[i][2 * q + 1], dl[i][2 * q + 1]);
+                    pu[q] = make_float4(dlu[i][2 * q], dlu[i][2 * q], dlu[i][2 * q + 1], dlu[i][2 * q + 1]);
+                }
+            }
         }
         if (bc_thread) {
             float4 *row = reinterpret_cast<float4 *>(&sBC[buf][bc_t][bc_isC ? 16 : 0]);
@@ -292,75 +363,63 @@ scan_fwd_kernel(const ScanArgs a) {
         if (k + 1 < ntiles) prefetch(t0 + TT);
         __syncthreads();
 
-        // ---- states: tokens of the tile in order.
-        const float *dl_row = myDelta[c];
-        const float *du_row = myDu[c];
+        if constexpr (G == 1) {
+            // ---- one lane per channel: states, readout and gate in registers.
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+                float yo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float *bcr = sBC[buf][8 * i + j];
+                    const float yv = state_token<P, POLY8, Gm::kSlots>(bcr, 0, f2_splat(dl[i][j]),
+                                                                        f2_splat(dlu[i][j]), A2, h, j * P);
+                    yo[j] = fmaf(yv, gate[i][j], dug[i][j]);
+                }
+                if (active) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
+            }
+        } else {
+            __syncwarp();
+            // ---- states: tokens of the tile in order.
+            const float *dl_row = reinterpret_cast<const float *>(&sDelta[warp][c][0]);
+            const float *du_row = reinterpret_cast<const float *>(&sDu[warp][c][0]);
 #pragma unroll 2
-        for (int tr = 0; tr < TT; tr += R) {
-            float part[R];
-            float dlv[R], duv[R];
+            for (int tr = 0; tr < TT; tr += R) {
+                float part[R];
+                f2 dlv[R], duv[R];
 #pragma unroll
-            for (int q = 0; q < R / 4; ++q) {
-                const float4 x = *reinterpret_cast<const float4 *>(dl_row + tr + 4 * q);
-                const float4 y = *reinterpret_cast<const float4 *>(du_row + tr + 4 * q);
-                dlv[4 * q] = x.x; dlv[4 * q + 1] = x.y; dlv[4 * q + 2] = x.z; dlv[4 * q + 3] = x.w;
-                duv[4 * q] = y.x; duv[4 * q + 1] = y.y; duv[4 * q + 2] = y.z; duv[4 * q + 3] = y.w;
-            }
-#pragma unroll
-            for (int j = 0; j < R; ++j) {
-                const float *bcr = sBC[buf][tr + j];
-                f2 Bp[P], Cp[P];
-                if constexpr (P >= 2) {
-#pragma unroll
-                    for (int q = 0; q < P / 2; ++q) {
-                        lds_f2x2(bcr + n0 + 4 * q, Bp[2 * q], Bp[2 * q + 1]);
-                        lds_f2x2(bcr + 16 + n0 + 4 * q, Cp[2 * q], Cp[2 * q + 1]);
-                    }
-                } else {
-                    Bp[0] = lds_f2(bcr + n0);
-                    Cp[0] = lds_f2(bcr + 16 + n0);
+                for (int q = 0; q < R / 2; ++q) {
+                    lds_f2x2(dl_row + 2 * (tr + 2 * q), dlv[2 * q], dlv[2 * q + 1]);
+                    lds_f2x2(du_row + 2 * (tr + 2 * q), duv[2 * q], duv[2 * q + 1]);
                 }
-                const f2 du2 = f2_splat(duv[j]);
-                f2 acc = f2_splat(0.0f);
 #pragma unroll
-                for (int p = 0; p < P; ++p) {
-                    float xa, xb;
-                    f2_split(A2[p], xa, xb);
-                    xa *= dlv[j];
-                    xb *= dlv[j];
-                    const int slot = j * P + p;
-                    const bool poly = slot * 8 < POLY8 * Gm::kSlots;
-                    const f2 ab = poly ? exp2_pair<true>(f2_make(xa, xb)) : f2_make(exp2_mufu(xa), exp2_mufu(xb));
-                    h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp[p]));
-                    acc = (p == 0) ? f2_mul(Cp[p], h[p]) : f2_fma(Cp[p], h[p], acc);
+                for (int j = 0; j < R; ++j)
+                    part[j] = state_token<P, POLY8, Gm::kSlots>(sBC[buf][tr + j], n0, dlv[j], duv[j], A2, h,
+                                                                 j * P);
+                // G partial readouts per token -> whole sums owned by one lane each.
+#pragma unroll
+                for (int blk = 0; blk < R / G; ++blk) {
+                    float v[G];
+#pragma unroll
+                    for (int q = 0; q < G; ++q) v[q] = part[blk * G + q];
+                    sY[warp][c][tr + blk * G + g] = reduce_scatter<G>(v, g);
                 }
-                float lo, hi;
-                f2_split(acc, lo, hi);
-                part[j] = lo + hi;
             }
-            // G partial readouts per token -> whole sums owned by one lane each.
-#pragma unroll
-            for (int blk = 0; blk < R / G; ++blk) {
-                float v[G];
-#pragma unroll
-                for (int i = 0; i < G; ++i) v[i] = part[blk * G + i];
-                const float sum = reduce_scatter<G>(v, g);
-                myY[c][tr + blk * G + g] = sum;
-            }
-        }
-        __syncwarp();
+            __syncwarp();
 
-        // ---- epilogue: chunk g of channel c.
-        {
-            const float4 y0 = *reinterpret_cast<const float4 *>(&myY[c][8 * g]);
-            const float4 y1 = *reinterpret_cast<const float4 *>(&myY[c][8 * g + 4]);
-            const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
-            float yo[8];
+            // ---- epilogue: this lane's chunks.
 #pragma unroll
-            for (int j = 0; j < 8; ++j) yo[j] = (ys[j] + du_skip[j]) * gate[j];
-            if (active) store8<TOut>(y_row, ts, L, vout, yo);
+            for (int i = 0; i < CH; ++i) {
+                const int off = 8 * (g * CH + i);
+                const float4 y0 = *reinterpret_cast<const float4 *>(&sY[warp][c][off]);
+                const float4 y1 = *reinterpret_cast<const float4 *>(&sY[warp][c][off + 4]);
+                const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+                float yo[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) yo[j] = fmaf(ys[j], gate[i][j], dug[i][j]);
+                if (active) store8<TOut>(y_row, t0 + off, L, vout, yo);
+            }
+            __syncwarp();
         }
-        __syncwarp();
     }
 
     if (active && a.last != nullptr) {
@@ -376,34 +435,51 @@ scan_fwd_kernel(const ScanArgs a) {
     }
 }
 
-template <typename TIn, typename TOut, int G, int POLY8>
+template <typename TIn, typename TOut, int G, int CH, int POLY8>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
-    using Gm = Geom<G>;
+    using Gm = Geom<G, CH>;
+    using Sm = SmemLayout<G, CH>;
     const int64_t dblocks = (a.dim + Gm::kChannels - 1) / Gm::kChannels;
     const int64_t blocks = dblocks * a.batch;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    scan_fwd_kernel<TIn, TOut, G, POLY8><<<(unsigned)blocks, kThreads, 0, stream>>>(a);
+    // Opt in to more than 48 KB of dynamic shared memory once per device and
+    // instantiation (idempotent, so a race between host threads is harmless).
+    static bool opted[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !opted[dev]) {
+        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) opted[dev] = true;
+    }
+    scan_fwd_kernel<TIn, TOut, G, CH, POLY8><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
     return cudaGetLastError();
 }
 
-template <typename TIn, typename TOut, int G>
+template <typename TIn, typename TOut, int G, int CH>
 cudaError_t launch_poly(const ScanArgs &a, int poly8, cudaStream_t stream) {
     switch (poly8) {
-        case 0: return launch_one<TIn, TOut, G, 0>(a, stream);
-        case 2: return launch_one<TIn, TOut, G, 2>(a, stream);
-        case 3: return launch_one<TIn, TOut, G, 3>(a, stream);
-        case 4: return launch_one<TIn, TOut, G, 4>(a, stream);
-        default: return launch_one<TIn, TOut, G, 8>(a, stream);
+        case 0: return launch_one<TIn, TOut, G, CH, 0>(a, stream);
+        case 2: return launch_one<TIn, TOut, G, CH, 2>(a, stream);
+        case 4: return launch_one<TIn, TOut, G, CH, 4>(a, stream);
+        default: return launch_one<TIn, TOut, G, CH, 8>(a, stream);
     }
 }
 
 template <typename TIn, typename TOut>
 cudaError_t launch_types(const ScanArgs &a, const ScanPlan &pl, cudaStream_t stream) {
+    const int ch = pl.chunks_per_lane;
     switch (pl.lanes_per_channel) {
-        case 2: return launch_poly<TIn, TOut, 2>(a, pl.poly8, stream);
-        case 4: return launch_poly<TIn, TOut, 4>(a, pl.poly8, stream);
-        default: return launch_poly<TIn, TOut, 8>(a, pl.poly8, stream);
+        case 1: return ch == 1 ? launch_poly<TIn, TOut, 1, 1>(a, pl.poly8, stream)
+                               : launch_poly<TIn, TOut, 1, 2>(a, pl.poly8, stream);
+        case 2: return ch == 1 ? launch_poly<TIn, TOut, 2, 1>(a, pl.poly8, stream)
+                               : launch_poly<TIn, TOut, 2, 2>(a, pl.poly8, stream);
+        case 4: return ch == 1 ? launch_poly<TIn, TOut, 4, 1>(a, pl.poly8, stream)
+                               : launch_poly<TIn, TOut, 4, 2>(a, pl.poly8, stream);
+        default: return launch_poly<TIn, TOut, 8, 1>(a, pl.poly8, stream);
     }
 }
 
@@ -421,14 +497,10 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf1
 
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms) {
     ScanPlan pl{};
-    // Four lanes per channel unless the channels alone cannot give every SM
-    // sub-partition two warps; then eight (each extra lane adds reduction
-    // shuffles, and two lanes per channel measured slower at every size tried).
     const int64_t channels = a.batch * a.dim;
     const int64_t want_warps = (int64_t)num_sms * 4 * 2;
     pl.lanes_per_channel = (channels * 4 / 32 >= want_warps) ? 4 : 8;
-    // fp32 inputs: every exponential on the unbiased polynomial (slow-decay
-    // accuracy); bf16 inputs: all on the MUFU unit (fastest measured).
+    pl.chunks_per_lane = 1;
     pl.poly8 = in_bf16 ? 0 : 8;
     return pl;
 }

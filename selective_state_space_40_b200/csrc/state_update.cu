@@ -9,8 +9,7 @@
 // The fp32 state (64 bytes per channel at d_state 16) dominates the traffic:
 // it is read and written once per step, so the kernel is an HBM stream. Four
 // lanes share a channel, each owning four consecutive states (one 16-byte
-// vector), so a warp moves 8 channels x 64 contiguous bytes per access; the
-// readout is summed over the four lanes with two xor-shuffles. The
+// vector); the readout is summed over the quad with xor-shuffles. The
 // exponentials use the MUFU unit: the arithmetic per channel must stay well
 // below the time its 128 state bytes take to stream.
 
@@ -21,7 +20,15 @@ namespace ms {
 
 namespace {
 
-constexpr int kThreads = 256;
+// Threads per block and channels per lane quad (state vectors in flight per
+// lane). Compile-time constants; the defaults are the measured best on B200.
+#ifndef MS_DECODE_THREADS
+#define MS_DECODE_THREADS 256
+#endif
+#ifndef MS_DECODE_U
+#define MS_DECODE_U 1
+#endif
+constexpr int kThreads = MS_DECODE_THREADS;
 
 template <typename TIn>
 __device__ __forceinline__ void load4(const TIn *p, bool vec, int valid, float (&v)[4]) {
@@ -39,75 +46,95 @@ __device__ __forceinline__ void load4(const TIn *p, bool vec, int valid, float (
     }
 }
 
-// grid: x covers the channels of one batch row (4 lanes each), y = batch row
-template <typename TIn, typename TOut>
+// grid: x covers the channels of one batch row, y = batch row. Lane i of a
+// warp is quad lane q = i % 4 (states 4q..4q+3) of channel slot s = i / 4;
+// the warp owns 8U consecutive channels and lane (s, q) serves channels
+// s, s + 8, ..., s + 8(U-1) of them, so for each u the warp's 16-byte state
+// accesses cover 512 contiguous bytes, and each lane has U vectors in flight.
+template <typename TIn, typename TOut, int U>
 __global__ void __launch_bounds__(kThreads)
 state_update_kernel(const UpdateArgs a) {
     const int64_t b = blockIdx.y;
-    const int tid = blockIdx.x * kThreads + threadIdx.x;
-    const int q = tid & 3;
-    const int64_t d = tid >> 2;
-    const bool act = d < a.dim;
-    const int64_t dd = act ? d : 0;
+    const int lane = threadIdx.x & 31;
+    const int q = lane & 3;
+    const int64_t dwarp = ((int64_t)blockIdx.x * (kThreads / 32) + (threadIdx.x >> 5)) * (8 * U);
     const int N = a.N;
     const int n0 = 4 * q;
-    const int nv = act ? (N - n0 < 0 ? 0 : (N - n0 > 4 ? 4 : N - n0)) : 0;  // states this lane owns
 
-    float h[4], A[4], Bv[4], Cv[4];
-    float *st = a.state + b * a.st_sb + dd * a.st_sd + n0;
-    if (a.vec_state && nv == 4) {
-        const float4 v = __ldcs(reinterpret_cast<const float4 *>(st));
-        h[0] = v.x; h[1] = v.y; h[2] = v.z; h[3] = v.w;
-    } else {
+    float h[U][4], A[U][4], Bv[4], Cv[4];
+    float x[U], raw[U], zv[U], bias[U], Dd[U];
+    bool act[U];
+    int64_t dd[U];
+    int nvs[U];
+    const int nq = N - n0 < 0 ? 0 : (N - n0 > 4 ? 4 : N - n0);  // states of this quad lane
+    // B and C depend only on the batch row: load once.
+    load4<TIn>(static_cast<const TIn *>(a.B) + b * a.B_sb + n0, a.vec_bc != 0, nq, Bv);
+    load4<TIn>(static_cast<const TIn *>(a.C) + b * a.C_sb + n0, a.vec_bc != 0, nq, Cv);
 #pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = i < nv ? __ldcs(st + i) : 0.0f;
+    for (int u = 0; u < U; ++u) {
+        const int64_t d = dwarp + (lane >> 2) + 8 * u;
+        act[u] = d < a.dim;
+        dd[u] = act[u] ? d : 0;
+        nvs[u] = act[u] ? nq : 0;
+        const float *st = a.state + b * a.st_sb + dd[u] * a.st_sd + n0;
+        if (a.vec_state && nvs[u] == 4) {
+            const float4 t = __ldcs(reinterpret_cast<const float4 *>(st));
+            h[u][0] = t.x; h[u][1] = t.y; h[u][2] = t.z; h[u][3] = t.w;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) h[u][i] = i < nvs[u] ? __ldcs(st + i) : 0.0f;
+        }
+        x[u] = raw[u] = zv[u] = 0.0f;
+        if (act[u]) {
+            x[u] = Elem<TIn>::load(static_cast<const TIn *>(a.x) + b * a.x_sb + dd[u]);
+            raw[u] = Elem<TIn>::load(static_cast<const TIn *>(a.delta) + b * a.dl_sb + dd[u]);
+            if (a.z) zv[u] = Elem<TIn>::load(static_cast<const TIn *>(a.z) + b * a.z_sb + dd[u]);
+        }
+        load4<float>(a.A + dd[u] * N + n0, a.vec_A != 0, nvs[u], A[u]);
+        bias[u] = (a.bias && act[u]) ? __ldg(a.bias + dd[u]) : 0.0f;
+        Dd[u] = (a.D && act[u]) ? __ldg(a.D + dd[u]) : 0.0f;
     }
-    float x = 0.f, raw = 0.f, zv = 0.f;
-    if (act) {
-        x = Elem<TIn>::load(static_cast<const TIn *>(a.x) + b * a.x_sb + dd);
-        raw = Elem<TIn>::load(static_cast<const TIn *>(a.delta) + b * a.dl_sb + dd);
-        if (a.z) zv = Elem<TIn>::load(static_cast<const TIn *>(a.z) + b * a.z_sb + dd);
-    }
-    load4<float>(a.A + dd * N + n0, a.vec_A != 0, nv, A);
-    load4<TIn>(static_cast<const TIn *>(a.B) + b * a.B_sb + n0, a.vec_bc != 0, nv, Bv);
-    load4<TIn>(static_cast<const TIn *>(a.C) + b * a.C_sb + n0, a.vec_bc != 0, nv, Cv);
-    const float bias = (a.bias && act) ? __ldg(a.bias + dd) : 0.0f;
-    const float Dd = (a.D && act) ? __ldg(a.D + dd) : 0.0f;
 
-    const float v = raw + bias;
-    const float dt = a.softplus ? softplus_f(v) : v;
-    const float dx = dt * x;
-    const float dtl = dt * kLog2e;
-    float acc = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const float abar = exp2_mufu(dtl * A[i]);
-        h[i] = fmaf(abar, h[i], dx * Bv[i]);
-        acc = fmaf(Cv[i], h[i], acc);
-    }
-    acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-    acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+    for (int u = 0; u < U; ++u) {
+        const float v = raw[u] + bias[u];
+        const float dt = a.softplus ? softplus_f(v) : v;
+        const float dx = dt * x[u];
+        const float dtl = dt * kLog2e;
+        float acc = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float abar = exp2_mufu(dtl * A[u][i]);
+            h[u][i] = fmaf(abar, h[u][i], dx * Bv[i]);
+            acc = fmaf(Cv[i], h[u][i], acc);
+        }
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
 
-    if (a.vec_state && nv == 4) {
-        __stcs(reinterpret_cast<float4 *>(st), make_float4(h[0], h[1], h[2], h[3]));
-    } else {
+        float *st = a.state + b * a.st_sb + dd[u] * a.st_sd + n0;
+        if (a.vec_state && nvs[u] == 4) {
+            __stcs(reinterpret_cast<float4 *>(st), make_float4(h[u][0], h[u][1], h[u][2], h[u][3]));
+        } else {
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (i < nv) __stcs(st + i, h[i]);
-    }
-    if (act && q == 0) {
-        float yv = acc + Dd * x;
-        if (a.z) yv *= silu_f(zv);
-        Elem<TOut>::store(static_cast<TOut *>(a.y) + b * a.y_sb + dd, yv);
+            for (int i = 0; i < 4; ++i)
+                if (i < nvs[u]) __stcs(st + i, h[u][i]);
+        }
+        if (act[u] && q == 0) {
+            float yv = acc + Dd[u] * x[u];
+            if (a.z) yv *= silu_f(zv[u]);
+            Elem<TOut>::store(static_cast<TOut *>(a.y) + b * a.y_sb + dd[u], yv);
+        }
     }
 }
 
 template <typename TIn, typename TOut>
 cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
+    constexpr int U = MS_DECODE_U;
     if (a.batch <= 0 || a.dim <= 0) return cudaSuccess;
-    const int64_t bx = (a.dim * 4 + kThreads - 1) / kThreads;
-    if (bx > 0x7fffffffLL / kThreads || a.batch > 65535) return cudaErrorInvalidConfiguration;
-    state_update_kernel<TIn, TOut><<<dim3((unsigned)bx, (unsigned)a.batch), kThreads, 0, stream>>>(a);
+    if (a.batch > 65535) return cudaErrorInvalidConfiguration;
+    const int64_t per_block = (int64_t)(kThreads / 32) * 8 * U;  // channels per block
+    const int64_t bx = (a.dim + per_block - 1) / per_block;
+    state_update_kernel<TIn, TOut, U><<<dim3((unsigned)bx, (unsigned)a.batch), kThreads, 0, stream>>>(a);
     return cudaGetLastError();
 }
 

@@ -100,9 +100,10 @@ def test_scan_rejects_null_and_misaligned(lib):
 
 
 def test_scan_rejects_bad_plan_and_workspace(lib):
-    assert _scan(_dims(), plan=mb.ScanPlan(3, 0)) == mb.MS_ERR_SHAPE
-    assert _scan(_dims(), plan=mb.ScanPlan(1, 0)) == mb.MS_ERR_SHAPE
-    assert _scan(_dims(), plan=mb.ScanPlan(4, 5)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(3, 1, 0)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(4, 3, 0)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(8, 2, 0)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(4, 1, 5)) == mb.MS_ERR_SHAPE
     assert _scan(_dims(), ws=None, ws_bytes=64) == mb.MS_ERR_WORKSPACE
 
 
@@ -115,7 +116,8 @@ def test_empty_scan_is_a_noop(lib):
 
 def test_choose_plan(lib):
     rc, plan = mb.mamba_scan_choose_plan(_dims(batch=8, dim=1536, seqlen=2048, in_dtype=mb.MS_BF16))
-    assert rc == mb.MS_OK and plan.lanes_per_channel in (2, 4, 8) and plan.poly8 in (0, 2, 3, 4, 8)
+    assert rc == mb.MS_OK and plan.lanes_per_channel in (1, 2, 4, 8) and plan.poly8 in (0, 2, 4, 8)
+    assert plan.chunks_per_lane in (1, 2)
     rc, _ = mb.mamba_scan_choose_plan(_dims(dstate=40))
     assert rc == mb.MS_ERR_SHAPE
 

@@ -85,11 +85,11 @@ def test_dstate(N):
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
-@pytest.mark.parametrize("lanes", [2, 4, 8])
-@pytest.mark.parametrize("poly", [0, 2, 3, 4, 8])
-def test_every_plan(dtype, lanes, poly):
-    w = syn.scaled(syn.M130, batch=3, dim=72, seqlen=517, in_dtype=dtype, seed=7)
-    compare_full(syn.scan_inputs(w), f"plan {lanes}/{poly} {dtype}", plan=(lanes, poly))
+@pytest.mark.parametrize("lanes,chunks", [(1, 1), (1, 2), (2, 1), (2, 2), (4, 1), (4, 2), (8, 1)])
+@pytest.mark.parametrize("poly", [0, 2, 4, 8])
+def test_every_plan(dtype, lanes, chunks, poly):
+    w = syn.scaled(syn.M130, batch=3, dim=136, seqlen=517, in_dtype=dtype, seed=7)
+    compare_full(syn.scan_inputs(w), f"plan {lanes}/{chunks}/{poly} {dtype}", plan=(lanes, chunks, poly))
 
 
 @pytest.mark.parametrize("flags", [

@@ -226,8 +226,10 @@ int mamba_state_update(float *state, const void *x, const void *delta, const flo
     a.vec_state = aligned(state, 16) && (dm->state_sb % 4) == 0 && (dm->state_sd % 4) == 0;
     a.vec_A = aligned(A, 16) && (dm->dstate % 4) == 0;
     a.vec_bc = aligned(B, 4 * ei) && aligned(C, 4 * ei) && (dm->B_sb % 4) == 0 && (dm->C_sb % 4) == 0;
-    cudaError_t e = ms::launch_state_update(a, dm->in_dtype == MS_BF16, dm->out_dtype == MS_BF16,
-                                            (cudaStream_t)stream);
+    const bool ib = dm->in_dtype == MS_BF16, ob = dm->out_dtype == MS_BF16;
+    cudaError_t e = ms::state_update_stream_applies(a, ei, eo)
+                        ? ms::launch_state_update_stream(a, ib, ob, (cudaStream_t)stream)
+                        : ms::launch_state_update(a, ib, ob, (cudaStream_t)stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return MS_ERR_CUDA;

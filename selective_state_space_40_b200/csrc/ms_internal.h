@@ -50,6 +50,11 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf1
 cudaError_t launch_state_update(const UpdateArgs &a, bool in_bf16, bool out_bf16,
                                 cudaStream_t stream);
 
+// Bulk-copy stream variant of the decode step (dense 16-state rows, dim a
+// multiple of 128, 16-byte aligned rows).
+bool state_update_stream_applies(const UpdateArgs &a, int in_bytes, int out_bytes);
+cudaError_t launch_state_update_stream(const UpdateArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
+
 // Plan for a call (host heuristic from sizes and dtypes).
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms);
 

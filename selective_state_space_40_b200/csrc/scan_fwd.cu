@@ -57,9 +57,8 @@ template <int G, int CH>
 struct SmemLayout {
     using Gm = Geom<G, CH>;
     static constexpr int kRows = G > 1 ? Gm::kCW : 1;  // per-channel rows (none needed when G == 1)
-    static constexpr int kRow2 = Gm::kTT + 2;          // float2 per splatted row (padded)
     static constexpr int kBCBytes = 2 * Gm::kTT * kBCRow * 4;
-    static constexpr int kPairBytes = G > 1 ? kNW * kRows * kRow2 * 8 : 0;
+    static constexpr int kPairBytes = G > 1 ? kNW * kRows * Gm::kRow * 4 : 0;
     static constexpr int kYBytes = G > 1 ? kNW * kRows * Gm::kRow * 4 : 0;
     static constexpr int kOffDelta = kBCBytes;
     static constexpr int kOffDu = kOffDelta + kPairBytes;
@@ -183,7 +182,7 @@ __device__ __forceinline__ float reduce_scatter(float (&v)[G], int g) {
 // the lane's states. `slot0` numbers the (token, pair) slots for the
 // MUFU/polynomial split.
 template <int P, int POLY8, int SLOTS>
-__device__ __forceinline__ float state_token(const float *bcr, int n0, f2 dl2, f2 du2, const f2 (&A2)[P],
+__device__ __forceinline__ float state_token(const float *bcr, int n0, float dl, float du, const f2 (&A2)[P],
                                              f2 (&h)[P], int slot0) {
     f2 Bp[P], Cp[P];
     if constexpr (P >= 2) {
@@ -196,28 +195,17 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, f2 dl2, f
         Bp[0] = lds_f2(bcr + n0);
         Cp[0] = lds_f2(bcr + 16 + n0);
     }
+    const f2 du2 = f2_splat(du);
     f2 acc = f2_splat(0.0f);
 #pragma unroll
     for (int p = 0; p < P; ++p) {
-        const f2 x2 = f2_mul(dl2, A2[p]);
-        const f2 w2 = f2_mul(du2, Bp[p]);
+        float xa, xb;
+        f2_split(A2[p], xa, xb);
+        xa *= dl;
+        xb *= dl;
         const bool poly = (slot0 + p) * 8 < POLY8 * SLOTS;
-        float ha, hb, wa, wb;
-        f2_split(h[p], ha, hb);
-        f2_split(w2, wa, wb);
-        if (poly) {
-            const f2 ab = exp2_pair<true>(x2);
-            float ea, eb;
-            f2_split(ab, ea, eb);
-            ha = fmaf(ea, ha, wa);
-            hb = fmaf(eb, hb, wb);
-        } else {
-            float xa, xb;
-            f2_split(x2, xa, xb);
-            ha = fmaf(exp2_mufu(xa), ha, wa);
-            hb = fmaf(exp2_mufu(xb), hb, wb);
-        }
-        h[p] = f2_make(ha, hb);
+        const f2 ab = poly ? exp2_pair<true>(f2_make(xa, xb)) : f2_make(exp2_mufu(xa), exp2_mufu(xb));
+        h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp[p]));
         acc = (p == 0) ? f2_mul(Cp[p], h[p]) : f2_fma(Cp[p], h[p], acc);
     }
     float lo, hi;
@@ -226,7 +214,7 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, f2 dl2, f
 }
 
 template <typename TIn, typename TOut, int G, int CH, int POLY8>
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads)
 scan_fwd_kernel(const ScanArgs a) {
     using Gm = Geom<G, CH>;
     constexpr int TT = Gm::kTT;
@@ -237,12 +225,11 @@ scan_fwd_kernel(const ScanArgs a) {
     constexpr int ROWS = Sm::kRows;
 
     // Dynamic shared memory: B/C tiles (double buffered, shared by the CTA),
-    // then per warp: Delta and Delta*u per token, each stored twice (a ready
-    // fp32 pair), and the reduced readouts.
+    // then per warp: Delta, Delta*u and the reduced readout per token.
     extern __shared__ __align__(16) unsigned char smem_raw[];
     auto sBC = reinterpret_cast<float (*)[TT][kBCRow]>(smem_raw);
-    auto sDelta = reinterpret_cast<float2 (*)[ROWS][Sm::kRow2]>(smem_raw + Sm::kOffDelta);
-    auto sDu = reinterpret_cast<float2 (*)[ROWS][Sm::kRow2]>(smem_raw + Sm::kOffDu);
+    auto sDelta = reinterpret_cast<float (*)[ROWS][Gm::kRow]>(smem_raw + Sm::kOffDelta);
+    auto sDu = reinterpret_cast<float (*)[ROWS][Gm::kRow]>(smem_raw + Sm::kOffDu);
     auto sY = reinterpret_cast<float (*)[ROWS][Gm::kRow]>(smem_raw + Sm::kOffY);
 
     const int warp = threadIdx.x >> 5;
@@ -346,11 +333,10 @@ scan_fwd_kernel(const ScanArgs a) {
             if constexpr (G > 1) {
                 float4 *pd = reinterpret_cast<float4 *>(&sDelta[warp][c][8 * (g * CH + i)]);
                 float4 *pu = reinterpret_cast<float4 *>(&sDu[warp][c][8 * (g * CH + i)]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    pd[q] = make_float4(dl[i][2 * q], dl[i][2 * q], dl[i][2 * q + 1], dl[i][2 * q + 1]);
-                    pu[q] = make_float4(dlu[i][2 * q], dlu[i][2 * q], dlu[i][2 * q + 1], dlu[i][2 * q + 1]);
-                }
+                pd[0] = make_float4(dl[i][0], dl[i][1], dl[i][2], dl[i][3]);
+                pd[1] = make_float4(dl[i][4], dl[i][5], dl[i][6], dl[i][7]);
+                pu[0] = make_float4(dlu[i][0], dlu[i][1], dlu[i][2], dlu[i][3]);
+                pu[1] = make_float4(dlu[i][4], dlu[i][5], dlu[i][6], dlu[i][7]);
             }
         }
         if (bc_thread) {
@@ -371,8 +357,8 @@ scan_fwd_kernel(const ScanArgs a) {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float *bcr = sBC[buf][8 * i + j];
-                    const float yv = state_token<P, POLY8, Gm::kSlots>(bcr, 0, f2_splat(dl[i][j]),
-                                                                        f2_splat(dlu[i][j]), A2, h, j * P);
+                    const float yv = state_token<P, POLY8, Gm::kSlots>(bcr, 0, dl[i][j], dlu[i][j], A2, h,
+                                                                        j * P);
                     yo[j] = fmaf(yv, gate[i][j], dug[i][j]);
                 }
                 if (active) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
@@ -385,11 +371,13 @@ scan_fwd_kernel(const ScanArgs a) {
 #pragma unroll 2
             for (int tr = 0; tr < TT; tr += R) {
                 float part[R];
-                f2 dlv[R], duv[R];
+                float dlv[R], duv[R];
 #pragma unroll
-                for (int q = 0; q < R / 2; ++q) {
-                    lds_f2x2(dl_row + 2 * (tr + 2 * q), dlv[2 * q], dlv[2 * q + 1]);
-                    lds_f2x2(du_row + 2 * (tr + 2 * q), duv[2 * q], duv[2 * q + 1]);
+                for (int q = 0; q < R / 4; ++q) {
+                    const float4 x = *reinterpret_cast<const float4 *>(dl_row + tr + 4 * q);
+                    const float4 y = *reinterpret_cast<const float4 *>(du_row + tr + 4 * q);
+                    dlv[4 * q] = x.x; dlv[4 * q + 1] = x.y; dlv[4 * q + 2] = x.z; dlv[4 * q + 3] = x.w;
+                    duv[4 * q] = y.x; duv[4 * q + 1] = y.y; duv[4 * q + 2] = y.z; duv[4 * q + 3] = y.w;
                 }
 #pragma unroll
                 for (int j = 0; j < R; ++j)

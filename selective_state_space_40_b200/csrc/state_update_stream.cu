@@ -1,0 +1,275 @@
+// state_update_stream.cu -- selective state update (decode) as a bulk-copy
+// stream on sm_100a.
+//
+// Same step as state_update.cu (one token from the stored fp32 state; blog
+// 'Mamba-1/2/3 Markdown図解', section 2: generation is the recurrent update of
+// the same model), organised for HBM streaming: a persistent CTA walks tiles
+// of kTC consecutive channels of one batch row. The tile's state rows (kTC x 64
+// bytes) and its x, delta, z values arrive by bulk copies (TMA engine) into a
+// ring of kStages shared-memory stages tracked by mbarriers; the threads update
+// the state in place in shared memory; bulk copies write the state and y back.
+// Loads run up to kStages - 1 tiles ahead, so the copy engine, not the
+// threads, keeps the HBM requests in flight. No cluster multicast is used.
+//
+// Used when the state rows are dense (16 fp32 per channel, 16-byte aligned),
+// d_state is 16, dim is a multiple of kTC and every row start is 16-byte
+// aligned; otherwise state_update.cu runs.
+
+#include <cstdint>
+
+#include "mambascan.h"
+#include "ms_device.cuh"
+#include "ms_internal.h"
+
+namespace ms {
+
+namespace {
+
+constexpr int kTC = 128;                   // channels per tile
+constexpr int kThreads = 256;              // 4 lanes per channel, 2 channels per lane
+constexpr int kStages = 4;
+constexpr uint32_t kSpinLimit = 1u << 20;  // try_wait rounds before giving up
+
+__device__ __forceinline__ uint32_t saddr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+    const uint32_t a = saddr(bar);
+    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            saddr(dst)),
+        "l"(src), "r"(bytes), "r"(saddr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void bulk_store(void *dst, const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(saddr(src)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// Wait until at most N committed store groups still read shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+template <typename TIn, typename TOut>
+struct StreamSmem {
+    static constexpr int kStateBytes = kTC * 16 * 4;
+    static constexpr int kInBytes = kTC * (int)sizeof(TIn);
+    static constexpr int kYBytes = kTC * (int)sizeof(TOut);
+    static constexpr int kStageBytes = kStateBytes + 3 * kInBytes + ((kYBytes + 15) & ~15);
+    static constexpr int kOffStages = 128;  // mbarriers first
+    static constexpr int kTotal = kOffStages + kStages * kStageBytes;
+};
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kThreads)
+state_update_stream_kernel(const UpdateArgs a) {
+    using Sm = StreamSmem<TIn, TOut>;
+    extern __shared__ __align__(128) unsigned char smem[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    auto stage = [&](int s) { return smem + Sm::kOffStages + s * Sm::kStageBytes; };
+
+    const int64_t tiles_per_row = a.dim / kTC;
+    const int64_t ntiles = a.batch * tiles_per_row;
+    const bool has_z = a.z != nullptr;
+    const int lane = threadIdx.x & 31;
+    const int q = lane & 3;        // states 4q..4q+3
+    const int n0 = 4 * q;
+
+    // Bytes of one tile's loads (state + x + delta [+ z]).
+    const uint32_t tile_bytes = Sm::kStateBytes + (has_z ? 3 : 2) * Sm::kInBytes;
+
+    auto issue = [&](int s, int64_t tile) {
+        const int64_t b = tile / tiles_per_row;
+        const int64_t d0 = (tile % tiles_per_row) * kTC;
+        unsigned char *st = stage(s);
+        mbar_arrive_expect_tx(&full[s], tile_bytes);
+        bulk_load(st, a.state + b * a.st_sb + d0 * 16, Sm::kStateBytes, &full[s]);
+        bulk_load(st + Sm::kStateBytes, static_cast<const TIn *>(a.x) + b * a.x_sb + d0, Sm::kInBytes, &full[s]);
+        bulk_load(st + Sm::kStateBytes + Sm::kInBytes, static_cast<const TIn *>(a.delta) + b * a.dl_sb + d0,
+                  Sm::kInBytes, &full[s]);
+        if (has_z)
+            bulk_load(st + Sm::kStateBytes + 2 * Sm::kInBytes, static_cast<const TIn *>(a.z) + b * a.z_sb + d0,
+                      Sm::kInBytes, &full[s]);
+    };
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    // Prologue: the first kStages - 1 tiles of this CTA.
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kStages - 1; ++s) {
+            const int64_t tile = blockIdx.x + (int64_t)s * gridDim.x;
+            if (tile < ntiles) issue(s, tile);
+        }
+    }
+
+    bool failed = false;
+    int64_t i = 0;
+    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+        const int s = (int)(i % kStages);
+        const bool ok = mbar_wait(&full[s], (uint32_t)((i / kStages) & 1));
+        if (__syncthreads_or(!ok)) {  // one decision for the whole CTA
+            failed = true;
+            break;
+        }
+        const int64_t b = tile / tiles_per_row;
+        const int64_t d0 = (tile % tiles_per_row) * kTC;
+        unsigned char *st = stage(s);
+        float *sstate = reinterpret_cast<float *>(st);
+        const TIn *sx = reinterpret_cast<const TIn *>(st + Sm::kStateBytes);
+        const TIn *sdl = sx + kTC;
+        const TIn *sz = sdl + kTC;
+        TOut *sy = reinterpret_cast<TOut *>(st + Sm::kStateBytes + 3 * Sm::kInBytes);
+
+        // B and C of this batch row (4 states of this quad lane).
+        float Bv[4], Cv[4];
+        {
+            const TIn *Bb = static_cast<const TIn *>(a.B) + b * a.B_sb + n0;
+            const TIn *Cb = static_cast<const TIn *>(a.C) + b * a.C_sb + n0;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                Bv[k] = Elem<TIn>::load(Bb + k);
+                Cv[k] = Elem<TIn>::load(Cb + k);
+            }
+        }
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            const int cl = (threadIdx.x >> 2) + half * (kThreads / 4);  // channel within the tile
+            const int64_t d = d0 + cl;
+            float4 hv = *reinterpret_cast<const float4 *>(sstate + cl * 16 + n0);
+            float h[4] = {hv.x, hv.y, hv.z, hv.w};
+            const float4 Av = __ldg(reinterpret_cast<const float4 *>(a.A + d * 16 + n0));
+            const float A[4] = {Av.x, Av.y, Av.z, Av.w};
+            const float x = to_f32(sx[cl]);
+            const float v = to_f32(sdl[cl]) + (a.bias ? __ldg(a.bias + d) : 0.0f);
+            const float dt = a.softplus ? softplus_f(v) : v;
+            const float dx = dt * x;
+            const float dtl = dt * kLog2e;
+            float acc = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                h[k] = fmaf(exp2_mufu(dtl * A[k]), h[k], dx * Bv[k]);
+                acc = fmaf(Cv[k], h[k], acc);
+            }
+            acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+            acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+            *reinterpret_cast<float4 *>(sstate + cl * 16 + n0) = make_float4(h[0], h[1], h[2], h[3]);
+            if (q == 0) {
+                float yv = acc + (a.D ? __ldg(a.D + d) : 0.0f) * x;
+                if (has_z) yv *= silu_f(to_f32(sz[cl]));
+                Elem<TOut>::store(sy + cl, yv);
+            }
+        }
+        fence_proxy_async();  // this thread's shared writes -> visible to the copy engine
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            bulk_store(a.state + b * a.st_sb + d0 * 16, sstate, Sm::kStateBytes);
+            bulk_store(static_cast<TOut *>(a.y) + b * a.y_sb + d0, sy, Sm::kYBytes);
+            bulk_commit();
+            // Refill the stage freed by the previous tile once its stores
+            // have finished reading it.
+            const int64_t next = tile + (int64_t)(kStages - 1) * gridDim.x;
+            if (next < ntiles) {
+                bulk_wait_read<1>();
+                issue((int)((i + kStages - 1) % kStages), next);
+            }
+        }
+    }
+
+    if (threadIdx.x == 0) {
+        if (failed) {
+            if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+            // Drain (bounded) the loads this CTA may still have in flight.
+            for (int k = 1; k < kStages; ++k) {
+                const int64_t tile = blockIdx.x + (i + k - 1) * (int64_t)gridDim.x;
+                if (tile < ntiles) mbar_wait(&full[(i + k - 1) % kStages], (uint32_t)(((i + k - 1) / kStages) & 1));
+            }
+        }
+        bulk_wait_all();
+    }
+}
+
+template <typename TIn, typename TOut>
+cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
+    using Sm = StreamSmem<TIn, TOut>;
+    static bool opted[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !opted[dev]) {
+        e = cudaFuncSetAttribute(state_update_stream_kernel<TIn, TOut>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
+        if (e != cudaSuccess) return e;
+        if (dev < 64) opted[dev] = true;
+    }
+    int sms = 148, per_sm = 1;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, state_update_stream_kernel<TIn, TOut>, kThreads,
+                                                  Sm::kTotal);
+    if (per_sm < 1) per_sm = 1;
+    const int64_t ntiles = a.batch * (a.dim / kTC);
+    const int64_t grid = ntiles < (int64_t)sms * per_sm ? ntiles : (int64_t)sms * per_sm;
+    if (grid <= 0) return cudaSuccess;
+    state_update_stream_kernel<TIn, TOut><<<(unsigned)grid, kThreads, Sm::kTotal, stream>>>(a);
+    return cudaGetLastError();
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+}  // namespace
+
+bool state_update_stream_applies(const UpdateArgs &a, int in_bytes, int out_bytes) {
+    if (a.N != 16 || a.st_sd != 16 || a.dim % kTC != 0) return false;
+    if (!aligned16(a.state) || (a.st_sb * 4) % 16 != 0) return false;
+    const void *rows[4] = {a.x, a.delta, a.z, a.y};
+    const int64_t sbs[4] = {a.x_sb, a.dl_sb, a.z_sb, a.y_sb};
+    const int es[4] = {in_bytes, in_bytes, in_bytes, out_bytes};
+    for (int k = 0; k < 4; ++k) {
+        if (rows[k] == nullptr) continue;
+        if (!aligned16(rows[k]) || (sbs[k] * es[k]) % 16 != 0) return false;
+    }
+    return aligned16(a.A);
+}
+
+cudaError_t launch_state_update_stream(const UpdateArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream) {
+    if (in_bf16) {
+        return out_bf16 ? launch_t<__nv_bfloat16, __nv_bfloat16>(a, stream)
+                        : launch_t<__nv_bfloat16, float>(a, stream);
+    }
+    return out_bf16 ? launch_t<float, __nv_bfloat16>(a, stream) : launch_t<float, float>(a, stream);
+}
+
+}  // namespace ms

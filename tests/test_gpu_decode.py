@@ -6,7 +6,7 @@ import torch
 import oracle
 from selective_state_space_40_b200 import binding as mb
 from selective_state_space_40_b200 import synthetic as syn
-from parity_util import check, check_bf16, check_fp32, f64
+from parity_util import check, check_bf16, check_fp32, check_out_bf16, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -133,3 +133,30 @@ def test_full_decode_1000_steps_sampled():
     assert torch.isfinite(state).all()
     check_bf16(np.stack(y_all), np.stack(yr_all), "decode every y (sampled channels)")
     check_bf16(f64(state[torch.as_tensor(bs)][:, torch.as_tensor(ds)]), h, "decode final state (sampled)")
+
+
+@pytest.mark.parametrize("dtype,out_dtype,use_z", [
+    (torch.float32, torch.float32, True), (torch.bfloat16, torch.float32, True),
+    (torch.bfloat16, torch.bfloat16, True), (torch.bfloat16, torch.float32, False)])
+def test_stream_path_small(dtype, out_dtype, use_z):
+    """dim a multiple of 128 with dense 16-state rows: the bulk-copy stream
+    kernel runs (several tiles per CTA, every step checked)."""
+    w = syn.DecodeWorkload("stream", batch=5, dim=384, dstate=16, steps=12, in_dtype=dtype)
+    p = syn.decode_params(w)
+    params = {k: v.to(DEV) for k, v in p.items()}
+    state = params["state0"].clone()
+    h = f64(p["state0"])
+    for k in range(w.steps):
+        inp = syn.decode_step_inputs(w, k)
+        y = mb.state_update(state, inp["x"].to(DEV), inp["delta"].to(DEV), params["A"], inp["B"].to(DEV),
+                            inp["C"].to(DEV), params["D"], inp["z"].to(DEV) if use_z else None,
+                            params["delta_bias"], True, out_dtype=out_dtype)
+        yr, h = oracle.state_update(h, f64(inp["x"]), f64(inp["delta"]), f64(p["A"]), f64(inp["B"]),
+                                    f64(inp["C"]), f64(p["D"]), f64(inp["z"]) if use_z else None,
+                                    f64(p["delta_bias"]), True)
+        torch.cuda.synchronize()
+        if out_dtype == torch.bfloat16:
+            check_out_bf16(f64(y), yr, f"stream step {k} y")
+        else:
+            check(f64(y), yr, dtype, f"stream step {k} y")
+    check(f64(state), h, dtype, "stream final state")

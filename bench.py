@@ -350,38 +350,51 @@ def main(argv=None):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
     e2e_gbs = world * nbytes * e2e_steps / (e2e_ms * 1e-3) / 1e9
 
-    # ---- decode step (selective state update) at b256 d5120 N16, L2 flushed
+    # ---- decode step (selective state update) at b256 d5120 N16: back-to-back
+    # steps over three rotating state buffers (3 x 84 MB > 126 MB L2), the
+    # steady state of generation where each layer's state is cold when its
+    # next token comes.
     dw = syn.DECODE
     dp = {k: v.to(dev) for k, v in syn.decode_params(dw).items()}
     ds = {k: v.to(dev) for k, v in syn.decode_step_inputs(dw, 0).items()}
-    state = dp["state0"].clone()
+    states = [dp["state0"].clone() for _ in range(3)]
     yd = torch.empty(dw.batch, dw.dim, dtype=torch.float32, device=dev)
-    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
-    dec_times = []
-    for i in range(40):
-        flush.fill_(i & 0xff)
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        mb.state_update(state, ds["x"], ds["delta"], dp["A"], ds["B"], ds["C"], dp["D"], ds["z"],
+
+    def dec(i):
+        mb.state_update(states[i % 3], ds["x"], ds["delta"], dp["A"], ds["B"], ds["C"], dp["D"], ds["z"],
                         dp["delta_bias"], True, y=yd, stream=stream)
-        b.record(stream)
-        dec_times.append((a, b))
+
+    for i in range(6):
+        dec(i)
+    dec_steps = 60
+    dev_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(dec_steps)]
     torch.cuda.synchronize()
-    dec_ms = statistics.fmean(a.elapsed_time(b) for a, b in dec_times[5:])
+    for i in range(dec_steps):
+        dev_ev[i][0].record(stream)
+        dec(i)
+        dev_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    dec_ms = statistics.fmean(a.elapsed_time(b) for a, b in dev_ev)
     dec_ms = max_over_ranks(dec_ms, world, dev)
     dbytes = decode_bytes(dw.batch, dw.dim, dw.dstate, 2, 4)
     dec_gbs = dbytes / (dec_ms * 1e-3) / 1e9
-    del flush
+    del states
 
-    # ---- CPU baseline: the oracle on this host's cores, one batch row
+    # ---- CPU baseline: the oracle on this host's cores, whole passes over the
+    # workload repeated until about ten seconds of wall time have gone by
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = cpu_threads()
-        cts, secs = oracle_sample_time(host, 1, threads)
+        cts, secs, passes = 0, 0.0, 0
+        while secs < 10.0 and passes < 50:
+            c, s_ = oracle_sample_time(host, w.batch, threads)
+            cts, secs, passes = cts + c, secs + s_, passes + 1
         ct_s = cts / secs
         cpu = {"value": ct_s * nbytes / ct / 1e9, "unit": "GB/s", "gct_per_s": ct_s / 1e9,
                "cores": threads, "kind": "oracle",
-               "sample": f"1 of {w.batch} batch rows ({cts} channel-tokens), {secs:.1f} s"}
+               "sample": f"{passes} full passes over the workload ({cts} channel-tokens), "
+                         f"{secs:.1f} s wall on {threads} threads"}
 
     if rank == 0:
         line = {
@@ -402,7 +415,8 @@ def main(argv=None):
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps},
             "decode_step": {"workload": dw.name, "value": dec_gbs, "unit": "GB/s",
                             "ms": dec_ms, "bytes": dbytes, "frac": dec_gbs / peak,
-                            "l2": "2x L2 buffer written before every timed launch"},
+                            "l2": "back-to-back steps over 3 rotating 84 MB states (> 126 MB L2)",
+                            "traffic": recorded_traffic("decode_step")},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

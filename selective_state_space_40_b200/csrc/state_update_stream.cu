@@ -25,9 +25,20 @@ namespace ms {
 
 namespace {
 
-constexpr int kTC = 128;                   // channels per tile
-constexpr int kThreads = 256;              // 4 lanes per channel, 2 channels per lane
-constexpr int kStages = 4;
+// Tile size, block size and ring depth (compile-time; defaults measured best).
+#ifndef MS_STREAM_TC
+#define MS_STREAM_TC 128
+#endif
+#ifndef MS_STREAM_THREADS
+#define MS_STREAM_THREADS 256
+#endif
+#ifndef MS_STREAM_STAGES
+#define MS_STREAM_STAGES 4
+#endif
+constexpr int kTC = MS_STREAM_TC;            // channels per tile
+constexpr int kThreads = MS_STREAM_THREADS;  // 4 lanes per channel
+constexpr int kStages = MS_STREAM_STAGES;
+static_assert(kTC * 4 % kThreads == 0, "whole channels per pass");
 constexpr uint32_t kSpinLimit = 1u << 20;  // try_wait rounds before giving up
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
@@ -166,7 +177,7 @@ state_update_stream_kernel(const UpdateArgs a) {
             }
         }
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
+        for (int half = 0; half < kTC * 4 / kThreads; ++half) {
             const int cl = (threadIdx.x >> 2) + half * (kThreads / 4);  // channel within the tile
             const int64_t d = d0 + cl;
             float4 hv = *reinterpret_cast<const float4 *>(sstate + cl * 16 + n0);

@@ -37,7 +37,24 @@ namespace ms {
 
 namespace {
 
-constexpr int kNW = 4;            // warps per CTA
+// Tuning (measured on the 130M-class layer: 2 warps per CTA, the reduction
+// pipelined against the next group and a register cap that keeps 6 CTAs per
+// SM resident gave 221 us against 238 us for 4-warp CTAs without either;
+// the packed Delta*A multiply took another 1 %).
+#ifndef MS_SCAN_NW
+#define MS_SCAN_NW 2              // warps per CTA
+#endif
+#ifndef MS_SCAN_MINB
+#define MS_SCAN_MINB 6            // resident CTAs per SM the one-chunk kernels are capped for
+#endif
+#ifndef MS_SCAN_PIPE
+#define MS_SCAN_PIPE 1            // 1: reduce a token group while the next group's states run
+#endif
+#ifndef MS_SCAN_PACKED_DA
+#define MS_SCAN_PACKED_DA 1       // 1: Delta*A for a state pair as one packed multiply
+#endif
+
+constexpr int kNW = MS_SCAN_NW;
 constexpr int kThreads = kNW * 32;
 constexpr int kBCRow = 36;        // floats per staged token row: B[0..15], C[16..31], pad
 
@@ -196,13 +213,20 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, float dl,
         Cp[0] = lds_f2(bcr + 16 + n0);
     }
     const f2 du2 = f2_splat(du);
+#if MS_SCAN_PACKED_DA
+    const f2 dl2 = f2_splat(dl);
+#endif
     f2 acc = f2_splat(0.0f);
 #pragma unroll
     for (int p = 0; p < P; ++p) {
         float xa, xb;
+#if MS_SCAN_PACKED_DA
+        f2_split(f2_mul(A2[p], dl2), xa, xb);
+#else
         f2_split(A2[p], xa, xb);
         xa *= dl;
         xb *= dl;
+#endif
         const bool poly = (slot0 + p) * 8 < POLY8 * SLOTS;
         const f2 ab = poly ? exp2_pair<true>(f2_make(xa, xb)) : f2_make(exp2_mufu(xa), exp2_mufu(xb));
         h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp[p]));
@@ -214,7 +238,7 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, float dl,
 }
 
 template <typename TIn, typename TOut, int G, int CH, int POLY8>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, CH == 1 ? MS_SCAN_MINB : 1)
 scan_fwd_kernel(const ScanArgs a) {
     using Gm = Geom<G, CH>;
     constexpr int TT = Gm::kTT;
@@ -276,20 +300,16 @@ scan_fwd_kernel(const ScanArgs a) {
     const bool vin = a.vec_in != 0;
     const bool vout = a.vec_out != 0;
 
-    // B/C staging: thread i < TT stages B of token i, TT <= i < 2TT stages C.
-    static_assert(2 * TT <= kThreads, "one staging thread per B/C token row");
-    const bool bc_thread = threadIdx.x < 2 * TT;
-    const int bc_t = threadIdx.x % TT;
-    const bool bc_isC = threadIdx.x >= TT;
-    const TIn *bc_base = bc_isC ? C_b : B_b;
-    const int64_t bc_sn = bc_isC ? a.C_sn : a.B_sn;
+    // B/C staging: staged row r < TT is B of token r, TT <= r < 2TT is C of
+    // token r - TT; thread i stages rows i, i + kThreads, ...
+    constexpr int kBCPer = (2 * TT + kThreads - 1) / kThreads;
 
     const int64_t ntiles = (L + TT - 1) / TT;
 
     // Lane (c, g) owns the prologue/epilogue chunks g*CH .. g*CH+CH-1 of its
     // channel in every tile (8*CH consecutive tokens).
     Chunk8<TIn> nu[CH], nd[CH], nz[CH];
-    Row16<TIn> nbc;
+    Row16<TIn> nbc[kBCPer];
     auto prefetch = [&](int64_t t0) {
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
@@ -305,8 +325,13 @@ scan_fwd_kernel(const ScanArgs a) {
                 nz[i].clear();
             }
         }
-        const int64_t tb = t0 + bc_t;
-        nbc.load(bc_base + tb, bc_sn, N, bc_thread && tb < L);
+#pragma unroll
+        for (int r = 0; r < kBCPer; ++r) {
+            const int row = threadIdx.x + r * kThreads;
+            const bool isC = row >= TT;
+            const int64_t tb = t0 + (row % TT);
+            nbc[r].load((isC ? C_b : B_b) + tb, isC ? a.C_sn : a.B_sn, N, row < 2 * TT && tb < L);
+        }
     };
 
     if (ntiles > 0) prefetch(0);
@@ -339,11 +364,16 @@ scan_fwd_kernel(const ScanArgs a) {
                 pu[1] = make_float4(dlu[i][4], dlu[i][5], dlu[i][6], dlu[i][7]);
             }
         }
-        if (bc_thread) {
-            float4 *row = reinterpret_cast<float4 *>(&sBC[buf][bc_t][bc_isC ? 16 : 0]);
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-                row[q] = make_float4(nbc.get(4 * q), nbc.get(4 * q + 1), nbc.get(4 * q + 2), nbc.get(4 * q + 3));
+        for (int r = 0; r < kBCPer; ++r) {
+            const int rr = threadIdx.x + r * kThreads;
+            if (rr < 2 * TT) {
+                float4 *row = reinterpret_cast<float4 *>(&sBC[buf][rr % TT][rr >= TT ? 16 : 0]);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    row[q] = make_float4(nbc[r].get(4 * q), nbc[r].get(4 * q + 1), nbc[r].get(4 * q + 2),
+                                         nbc[r].get(4 * q + 3));
+            }
         }
         // The next tile's loads stay in flight while this tile's states run.
         if (k + 1 < ntiles) prefetch(t0 + TT);
@@ -368,9 +398,17 @@ scan_fwd_kernel(const ScanArgs a) {
             // ---- states: tokens of the tile in order.
             const float *dl_row = reinterpret_cast<const float *>(&sDelta[warp][c][0]);
             const float *du_row = reinterpret_cast<const float *>(&sDu[warp][c][0]);
-#pragma unroll 2
-            for (int tr = 0; tr < TT; tr += R) {
-                float part[R];
+            // G partial readouts per token -> whole sums owned by one lane each.
+            auto reduce_group = [&](const float (&part)[R], int tr) {
+#pragma unroll
+                for (int blk = 0; blk < R / G; ++blk) {
+                    float v[G];
+#pragma unroll
+                    for (int q = 0; q < G; ++q) v[q] = part[blk * G + q];
+                    sY[warp][c][tr + blk * G + g] = reduce_scatter<G>(v, g);
+                }
+            };
+            auto state_group = [&](float (&part)[R], int tr) {
                 float dlv[R], duv[R];
 #pragma unroll
                 for (int q = 0; q < R / 4; ++q) {
@@ -383,15 +421,29 @@ scan_fwd_kernel(const ScanArgs a) {
                 for (int j = 0; j < R; ++j)
                     part[j] = state_token<P, POLY8, Gm::kSlots>(sBC[buf][tr + j], n0, dlv[j], duv[j], A2, h,
                                                                  j * P);
-                // G partial readouts per token -> whole sums owned by one lane each.
+            };
+#if MS_SCAN_PIPE
+            // The reduction of group k-1 sits in the same block as the state
+            // work of group k, so its shuffles fill the state chain's stalls.
+            float prev[R];
+            state_group(prev, 0);
 #pragma unroll
-                for (int blk = 0; blk < R / G; ++blk) {
-                    float v[G];
+            for (int tr = R; tr < TT; tr += R) {
+                float part[R];
+                state_group(part, tr);
+                reduce_group(prev, tr - R);
 #pragma unroll
-                    for (int q = 0; q < G; ++q) v[q] = part[blk * G + q];
-                    sY[warp][c][tr + blk * G + g] = reduce_scatter<G>(v, g);
-                }
+                for (int j = 0; j < R; ++j) prev[j] = part[j];
             }
+            reduce_group(prev, TT - R);
+#else
+#pragma unroll 2
+            for (int tr = 0; tr < TT; tr += R) {
+                float part[R];
+                state_group(part, tr);
+                reduce_group(part, tr);
+            }
+#endif
             __syncwarp();
 
             // ---- epilogue: this lane's chunks.

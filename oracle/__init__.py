@@ -1,4 +1,5 @@
-"""fp64 CPU oracle of the Mamba selective scan and selective state update.
+"""fp64 CPU oracle of the Mamba selective scan, the selective state update and
+the causal conv front-end of the block's input path.
 
 TEST INFRASTRUCTURE ONLY: imported by the tests, by the smoke check and by the
 benchmark's CPU-baseline leg, never by the product package. It shares no code
@@ -7,6 +8,8 @@ passage of the Mamba pages each step follows.
 """
 from .oracle import (  # noqa: F401
     build_oracle,
+    causal_conv,
+    conv_scan,
     load_oracle,
     scan,
     scan_mt,

@@ -20,6 +20,11 @@
  *    project fixes for steps the pages leave open.
  *  - Generation is the same recurrence taken one token at a time from a stored
  *    state (blog, section 2, "1トークン生成 → recurrent update").
+ *  - The block's input path (blog, section 2, block diagram): the projected
+ *    input passes a short causal convolution along the tokens, one filter per
+ *    channel, then silu, and the result is the SSM's input u. Read here as
+ *    u_t = silu(bias_d + sum_{k<W} w[d][k] * x_{t-(W-1)+k}), with the W-1
+ *    tokens before t = 0 taken from a given history or zero.
  *
  * Layouts (all arrays dense, row-major, fp64):
  *   u, delta, z, y      [batch][dim][seqlen]
@@ -29,6 +34,8 @@
  *   h0, last_state      [batch][dim][dstate]
  *   decode: x, delta, z, y [batch][dim]; B, C [batch][dstate]; state [batch][dim][dstate]
  * Nullable: D, z, delta_bias, h0 (zero initial state), last_state.
+ *   conv: x, u [batch][dim][seqlen]; w [dim][W]; bias [dim]; x0 [batch][dim][W-1]
+ *   (x0[b][d][j] is x_{-(W-1)+j}); bias and x0 nullable.
  *
  * Built with -O2 and no fast-math; exp/log1p are the C library's.
  * ORACLE_MUTANT (compile-time, tests only) plants one known mistake so that a
@@ -258,6 +265,57 @@ int oracle_state_update_f64(int64_t batch, int64_t dim, int64_t dstate,
                          D ? D + d : NULL, z ? z + c : NULL,
                          delta_bias ? delta_bias + d : NULL, softplus_flag,
                          state + c * N, y + c);
+        }
+    }
+    return 0;
+}
+
+/*
+ * Causal depthwise convolution of the block's input path, then silu (when
+ * silu_flag): for every (b, d) and token t,
+ *   u_t = act(bias_d + sum_{k=0}^{W-1} w[d][k] * x_{t-(W-1)+k}),
+ * where x_s for s < 0 is x0[b][d][s + W - 1] (zero when x0 is NULL). The
+ * filter's last tap w[d][W-1] weights the current token. Returns 0, or -1 on
+ * a bad size or a missing required array.
+ */
+int oracle_causal_conv_f64(int64_t batch, int64_t dim, int64_t seqlen, int64_t width,
+                           const double *x, const double *w, const double *bias,
+                           const double *x0, int silu_flag, double *u)
+{
+    if (batch < 0 || dim < 0 || seqlen < 0 || width < 1) return -1;
+    if (batch * dim * seqlen > 0 && (!x || !w || !u)) return -1;
+    const int64_t W = width;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t c = b * dim + d;
+            const double *xr = x + c * seqlen;
+            for (int64_t t = 0; t < seqlen; ++t) {
+                double acc = bias ? bias[d] : 0.0;
+                for (int64_t k = 0; k < W; ++k) {
+                    const int64_t s = t - (W - 1) + k; /* token under tap k */
+                    double xs;
+                    if (s >= 0) {
+                        xs = xr[s];
+                    } else {
+#if ORACLE_MUTANT == 15
+                        xs = 0.0; /* mutant: history before token 0 ignored */
+#else
+                        xs = x0 ? x0[c * (W - 1) + (s + W - 1)] : 0.0;
+#endif
+                    }
+#if ORACLE_MUTANT == 13
+                    acc += w[d * W + (W - 1 - k)] * xs; /* mutant: filter taps reversed */
+#else
+                    acc += w[d * W + k] * xs;
+#endif
+                }
+#if ORACLE_MUTANT == 14
+                (void)silu_flag;
+                u[c * seqlen + t] = acc; /* mutant: activation dropped */
+#else
+                u[c * seqlen + t] = silu_flag ? oracle_silu(acc) : acc;
+#endif
+            }
         }
     }
     return 0;

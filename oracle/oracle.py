@@ -50,6 +50,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_scan_f64_mt.restype = ctypes.c_int
     lib.oracle_state_update_f64.argtypes = [i64, i64, i64] + [_dp] * 9 + [ctypes.c_int, _dp]
     lib.oracle_state_update_f64.restype = ctypes.c_int
+    lib.oracle_causal_conv_f64.argtypes = [i64, i64, i64, i64] + [_dp] * 4 + [ctypes.c_int, _dp]
+    lib.oracle_causal_conv_f64.restype = ctypes.c_int
     return lib
 
 
@@ -143,6 +145,34 @@ def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise ValueError(f"oracle_state_update_f64 rejected its arguments (rc={rc})")
     return y, st
+
+
+def causal_conv(x, w, bias=None, x0=None, silu_flag=True, lib=None):
+    """Causal depthwise convolution + silu of the block's input path, fp64.
+    x [batch, dim, L]; w [dim, W]; bias [dim]; x0 [batch, dim, W-1] (the W-1
+    tokens before token 0; zero if None). Returns u [batch, dim, L]."""
+    lib = lib or load_oracle()
+    x, w, bias, x0 = (_f64(a) for a in (x, w, bias, x0))
+    batch, dim, L = x.shape
+    W = w.shape[1]
+    assert w.shape == (dim, W) and (bias is None or bias.shape == (dim,))
+    assert x0 is None or x0.shape == (batch, dim, W - 1)
+    u = np.full((batch, dim, L), np.nan, dtype=np.float64)
+    rc = lib.oracle_causal_conv_f64(batch, dim, L, W, _ptr(x), _ptr(w), _ptr(bias), _ptr(x0),
+                                    int(bool(silu_flag)), _ptr(u))
+    if rc != 0:
+        raise ValueError(f"oracle_causal_conv_f64 rejected its arguments (rc={rc})")
+    return u
+
+
+def conv_scan(x, conv_w, conv_b, conv_x0, conv_silu, delta, A, B, C, D=None, z=None,
+              delta_bias=None, softplus_flag=True, h0=None, lib=None, nthreads: int = 1):
+    """The scan fed by the block's causal conv front-end: u = causal_conv(x),
+    then the selective scan of u. Returns (y, last_state, u)."""
+    lib = lib or load_oracle()
+    u = causal_conv(x, conv_w, conv_b, conv_x0, conv_silu, lib=lib)
+    y, last = scan(u, delta, A, B, C, D, z, delta_bias, softplus_flag, h0, lib=lib, nthreads=nthreads)
+    return y, last, u
 
 
 def mutant_library(mutant: int, directory: Optional[str] = None) -> ctypes.CDLL:

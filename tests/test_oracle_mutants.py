@@ -25,6 +25,9 @@ MUTANTS = {
     10: "state index reversed in A",
     11: "decode ignores the stored state",
     12: "final state never written",
+    13: "conv filter taps reversed",
+    14: "conv activation dropped",
+    15: "conv history before token 0 ignored",
 }
 
 

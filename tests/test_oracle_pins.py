@@ -18,7 +18,12 @@ mathematics) fix, written without the oracle's code:
 * degenerate cases: B = 0, and Delta = 0 (A_bar = 1);
 * softplus / silu special values and library routines (numpy logaddexp,
   scipy expit);
-* the hand-worked cases in tests/golden/hand_worked.json.
+* the hand-worked cases in tests/golden/hand_worked.json;
+* the block's causal conv front-end (blog, section 2, block diagram: a short
+  causal convolution per channel, then silu, feeds the SSM) against numpy's
+  full convolution with the history prepended, one-hot filters as explicit
+  token shifts, and split/resume of conv + scan with the conv history and the
+  state carried.
 
 ``test_oracle_mutants.py`` plants known mistakes in the oracle and checks
 that at least one of these pins fails for each.
@@ -263,6 +268,76 @@ def pin_hand_worked(lib):
     return worst
 
 
+def _conv_ref(x, w, bias, x0, silu_flag):
+    """u_t = act(bias + sum_k w_k x_{t-(W-1)+k}) from numpy's full convolution
+    of the history-prepended row with the reversed filter."""
+    b, d, L = x.shape
+    W = w.shape[1]
+    u = np.empty((b, d, L))
+    for bi in range(b):
+        for di in range(d):
+            hist = np.zeros(W - 1) if x0 is None else x0[bi, di]
+            full = np.convolve(np.concatenate([hist, x[bi, di]]), w[di, ::-1])
+            v = full[W - 1:W - 1 + L] + (0.0 if bias is None else bias[di])
+            u[bi, di] = _silu_ref(v) if silu_flag else v
+    return u
+
+
+def pin_conv_numpy(lib):
+    rng = np.random.default_rng(18)
+    worst = 0.0
+    for W in (1, 2, 3, 4):
+        b, d, L = 2, 3, 29
+        x = rng.standard_normal((b, d, L))
+        w = rng.standard_normal((d, W))
+        bias = rng.standard_normal(d)
+        x0 = rng.standard_normal((b, d, W - 1))
+        for silu_flag in (False, True):
+            for hist in (None, x0):
+                u = oracle.causal_conv(x, w, bias, hist, silu_flag, lib=lib)
+                worst = max(worst, _rel(u, _conv_ref(x, w, bias, hist, silu_flag)))
+    return worst
+
+
+def pin_conv_shift(lib):
+    rng = np.random.default_rng(19)
+    b, d, L, W = 1, 2, 15, 4
+    x = rng.standard_normal((b, d, L))
+    x0 = rng.standard_normal((b, d, W - 1))
+    ext = np.concatenate([x0, x], axis=2)  # ext[..., s + W - 1] = x_s
+    worst = 0.0
+    for k in range(W):
+        w = np.zeros((d, W))
+        w[:, k] = 1.0
+        u = oracle.causal_conv(x, w, None, x0, False, lib=lib)
+        # tap k alone picks token t - (W-1) + k
+        ref = np.stack([ext[:, :, t + k] for t in range(L)], axis=2)
+        worst = max(worst, float(np.max(np.abs(u - ref))))
+    return worst
+
+
+def pin_conv_scan_split(lib):
+    rng = np.random.default_rng(20)
+    b, d, N, L, m, W = 2, 3, 4, 36, 13, 4
+    A = -rng.uniform(0.1, 3.0, size=(d, N))
+    x = rng.standard_normal((b, d, L))
+    w = rng.standard_normal((d, W))
+    cb = rng.standard_normal(d)
+    raw = rng.standard_normal((b, d, L))
+    z = rng.standard_normal((b, d, L))
+    B = rng.standard_normal((b, N, L))
+    C = rng.standard_normal((b, N, L))
+    D = rng.standard_normal(d)
+    bias = rng.uniform(-2.0, 0.0, size=d)
+    y, last, u = oracle.conv_scan(x, w, cb, None, True, raw, A, B, C, D, z, bias, True, lib=lib)
+    y1, h1, u1 = oracle.conv_scan(x[:, :, :m], w, cb, None, True, raw[:, :, :m], A, B[:, :, :m],
+                                  C[:, :, :m], D, z[:, :, :m], bias, True, lib=lib)
+    y2, h2, u2 = oracle.conv_scan(x[:, :, m:], w, cb, x[:, :, m - W + 1:m], True, raw[:, :, m:], A,
+                                  B[:, :, m:], C[:, :, m:], D, z[:, :, m:], bias, True, h0=h1, lib=lib)
+    return max(_rel(np.concatenate([y1, y2], axis=2), y), _rel(h2, last),
+               _rel(np.concatenate([u1, u2], axis=2), u))
+
+
 PINS = {
     "softplus_silu": pin_softplus_silu,
     "lti_convolution": pin_lti_convolution,
@@ -273,6 +348,9 @@ PINS = {
     "split_resume": pin_split_resume,
     "degenerate": pin_degenerate,
     "hand_worked": pin_hand_worked,
+    "conv_numpy": pin_conv_numpy,
+    "conv_shift": pin_conv_shift,
+    "conv_scan_split": pin_conv_scan_split,
 }
 
 

@@ -152,6 +152,45 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
 int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan);
 
 /*
+ * Scan with the block's causal conv front-end. In the Mamba-1 block (blog,
+ * section 2, block diagram) the projected input passes a short causal
+ * convolution along the tokens, one filter per channel, and silu before the
+ * selective SSM. This entry point takes that convolution's input x and forms
+ * the SSM input inside the scan's load stage (u never goes through HBM):
+ *     u[b,d,t] = act(conv_b[d] + sum_{k=0}^{W-1} conv_w[d,k] * x[b,d,t-(W-1)+k])
+ * with act = silu when silu is nonzero (identity otherwise) and x at t < 0
+ * taken from conv_x0[b,d,t+W-1] (zero when conv_x0 is NULL). A sequence
+ * scanned in pieces passes the previous piece's last W-1 inputs as conv_x0
+ * and its last_state as initial_state. Everything after u is mamba_scan_fwd.
+ */
+typedef struct {
+    int64_t width;            /* W: filter taps, 1..4 (conv_w[d, W-1] weights token t) */
+    int64_t uout_sb, uout_sd; /* strides of u_out; inner stride 1 */
+    int32_t silu;             /* nonzero: act = silu */
+} ms_conv_dims;
+
+/*
+ *   x          required input of the convolution, [batch, dim, seqlen] in
+ *              dims->in_dtype, strides dims->u_sb / dims->u_sd.
+ *   conv_w     required fp32 [dim, W], dense.
+ *   conv_b     optional fp32 [dim] (NULL = 0).
+ *   conv_x0    optional [batch, dim, W-1] dense, in_dtype: inputs before token 0.
+ *   u_out      optional output [batch, dim, seqlen], in_dtype: the computed u
+ *              (rounded to in_dtype; the scan itself uses fp32 u).
+ *   plan       NULL = automatic; a given plan must have chunks_per_lane 1 and
+ *              poly8 0 or 8.
+ * The other arguments are those of mamba_scan_fwd; no workspace is needed.
+ * Returns MS_OK or an MS_ERR_* code (MS_ERR_SHAPE for W outside [1, 4] or a
+ * plan outside the list above).
+ */
+int mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b, const void *conv_x0,
+                        void *u_out, const ms_conv_dims *cdims, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D, const void *z,
+                        const float *delta_bias, int softplus_flag, const float *initial_state,
+                        void *y, float *last_state, const ms_scan_dims *dims,
+                        const ms_scan_plan *plan, int *dev_status, ms_stream_t stream);
+
+/*
  * Sizes and strides of one decode step.
  *   x, delta, z, y : [batch, dim]     element (b,d) at b*x_sb + d
  *   B, C           : [batch, dstate]  element (b,n) at b*x_sb + n

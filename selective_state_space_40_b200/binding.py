@@ -39,6 +39,11 @@ class ScanPlan(ctypes.Structure):
                 ("poly8", ctypes.c_int32)]
 
 
+class ConvDims(ctypes.Structure):
+    _fields_ = [("width", ctypes.c_int64), ("uout_sb", ctypes.c_int64), ("uout_sd", ctypes.c_int64),
+                ("silu", ctypes.c_int32)]
+
+
 class MambaScanError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: status {code} ({mamba_status_string(code)})")
@@ -67,6 +72,10 @@ def library() -> ctypes.CDLL:
         lib.mamba_scan_fwd_plan.restype = ctypes.c_int
         lib.mamba_scan_choose_plan.argtypes = [ctypes.POINTER(ScanDims), ctypes.POINTER(ScanPlan)]
         lib.mamba_scan_choose_plan.restype = ctypes.c_int
+        lib.mamba_conv_scan_fwd.argtypes = ([_vp] * 5 + [ctypes.POINTER(ConvDims)] + [_vp] * 7 +
+                                            [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(ScanDims),
+                                             ctypes.POINTER(ScanPlan), _vp, _vp])
+        lib.mamba_conv_scan_fwd.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
                                                        _vp, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
@@ -107,6 +116,15 @@ def mamba_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_s
     if plan is None:
         return lib.mamba_scan_fwd(*args)
     return lib.mamba_scan_fwd_plan(*args, ctypes.byref(plan))
+
+
+def mamba_conv_scan_fwd(x, conv_w, conv_b, conv_x0, u_out, cdims: ConvDims, delta, A, B, C, D, z,
+                        delta_bias, softplus_flag, initial_state, y, last_state, dims: ScanDims,
+                        plan: Optional[ScanPlan], dev_status, stream) -> int:
+    return library().mamba_conv_scan_fwd(
+        x, conv_w, conv_b, conv_x0, u_out, ctypes.byref(cdims), delta, A, B, C, D, z, delta_bias,
+        int(softplus_flag), initial_state, y, last_state, ctypes.byref(dims),
+        None if plan is None else ctypes.byref(plan), dev_status, stream)
 
 
 def mamba_state_update(state, x, delta, A, B, C, D, z, delta_bias, softplus_flag, y,
@@ -192,6 +210,45 @@ def scan_fwd(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool 
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba_scan_fwd")
     return y, last_state
+
+
+def conv_scan_fwd(x, conv_w, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+                  conv_b=None, conv_x0=None, conv_silu: bool = True, return_u: bool = False,
+                  initial_state=None, out_dtype=None, y=None, last_state=None, u_out=None,
+                  return_last_state: bool = True, stream=None,
+                  plan: Optional[Tuple[int, int, int]] = None, dev_status=None):
+    """Scan with the causal conv front-end on torch CUDA tensors (see
+    include/mambascan.h, mamba_conv_scan_fwd): x [b, d, L] is the conv input,
+    conv_w [d, W] fp32. Returns (y, last_state or None, u or None)."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    batch, dim, L = x.shape
+    N = A.shape[1]
+    if y is None:
+        y = torch.empty((batch, dim, L), dtype=out_dtype, device=x.device)
+    if last_state is None and return_last_state:
+        last_state = torch.empty((batch, dim, N), dtype=torch.float32, device=x.device)
+    if u_out is None and return_u:
+        u_out = torch.empty((batch, dim, L), dtype=x.dtype, device=x.device)
+    for t, n in ((A, "A"), (D, "D"), (delta_bias, "delta_bias"), (initial_state, "initial_state"),
+                 (last_state, "last_state"), (conv_w, "conv_w"), (conv_b, "conv_b")):
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous fp32 tensor")
+    if conv_x0 is not None and (conv_x0.dtype != x.dtype or not conv_x0.is_contiguous()):
+        raise ValueError("conv_x0 must be contiguous with the dtype of x")
+    _inner_contiguous(u_out, "u_out")
+    dims = scan_dims_for(x, delta, B, C, z, y)
+    uo = u_out if u_out is not None else x
+    cdims = ConvDims(conv_w.shape[1], uo.stride(0), uo.stride(1), int(bool(conv_silu)))
+    pl = ScanPlan(*plan) if plan is not None else None
+    rc = mamba_conv_scan_fwd(_ptr(x), _ptr(conv_w), _ptr(conv_b), _ptr(conv_x0), _ptr(u_out), cdims,
+                             _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                             softplus, _ptr(initial_state), _ptr(y), _ptr(last_state), dims, pl,
+                             _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_conv_scan_fwd")
+    return y, last_state, u_out
 
 
 def update_dims_for(state, x, delta, B, C, z, y) -> UpdateDims:

@@ -146,19 +146,36 @@ int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void 
                                last_state, dims, workspace, workspace_bytes, dev_status, stream, nullptr);
 }
 
-int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B, const void *C,
-                        const float *D, const void *z, const float *delta_bias, int softplus_flag,
-                        const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
-                        void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream,
-                        const ms_scan_plan *plan) {
-    if (plan && !plan_valid(plan)) return MS_ERR_SHAPE;
-    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
-    if (rc != MS_OK) return rc;
-    if (workspace_bytes < mamba_scan_workspace_size(dims) || (workspace_bytes > 0 && !workspace))
-        return MS_ERR_WORKSPACE;
-    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
-    if (dims->seqlen == 0 && !last_state) return MS_OK;
+// Conv front-end arguments of mamba_conv_scan_fwd (all null for the plain scan).
+struct ConvIn {
+    const float *w, *b;
+    const void *x0;
+    void *u_out;
+    const ms_conv_dims *cd;
+};
 
+static int check_conv(const ConvIn &cv, const ms_scan_dims *dm) {
+    if (!cv.cd) return MS_ERR_NULL;
+    const ms_conv_dims *cd = cv.cd;
+    if (cd->width < 1 || cd->width > 4) return MS_ERR_SHAPE;
+    if (cd->uout_sb < 0 || cd->uout_sd < 0) return MS_ERR_STRIDE;
+    if (dm->batch == 0 || dm->dim == 0) return MS_OK;
+    if (!cv.w) return MS_ERR_NULL;
+    const int ei = elem_bytes(dm->in_dtype);
+    if (!aligned(cv.w, 4) || (cv.b && !aligned(cv.b, 4)) || (cv.x0 && !aligned(cv.x0, ei)) ||
+        (cv.u_out && !aligned(cv.u_out, ei)))
+        return MS_ERR_ALIGN;
+    if (dm->seqlen > 0 && cv.u_out &&
+        max_offset3(dm->batch, cd->uout_sb, dm->dim, cd->uout_sd, dm->seqlen) < 0)
+        return MS_ERR_SHAPE;
+    if (max_offset3(dm->batch, dm->dim * cd->width, dm->dim, cd->width, cd->width) < 0) return MS_ERR_SHAPE;
+    return MS_OK;
+}
+
+static int scan_common(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                       const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                       const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
+                       int *dev_status, ms_stream_t stream, const ms_scan_plan *plan, const ConvIn *cv) {
     ms::ScanArgs a{};
     a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
     a.A = A; a.D = D; a.bias = delta_bias; a.h0 = initial_state;
@@ -174,6 +191,17 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
     a.vec_in = vec_ok(u, dims->u_sb, dims->u_sd, ei) && vec_ok(delta, dims->delta_sb, dims->delta_sd, ei) &&
                vec_ok(z, dims->z_sb, dims->z_sd, ei);
     a.vec_out = vec_ok(y, dims->y_sb, dims->y_sd, eo);
+    if (cv) {
+        a.conv_w = cv->w;
+        a.conv_b = cv->b;
+        a.conv_x0 = cv->x0;
+        a.u_out = cv->u_out;
+        a.uo_sb = cv->cd->uout_sb;
+        a.uo_sd = cv->cd->uout_sd;
+        a.conv_width = (int)cv->cd->width;
+        a.conv_silu = cv->cd->silu ? 1 : 0;
+        a.vec_uout = vec_ok(cv->u_out, a.uo_sb, a.uo_sd, ei);
+    }
 
     const bool in_bf16 = dims->in_dtype == MS_BF16, out_bf16 = dims->out_dtype == MS_BF16;
     ms::ScanPlan pl = auto_plan(dims);
@@ -188,6 +216,41 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
         return MS_ERR_CUDA;
     }
     return MS_OK;
+}
+
+int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                        const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                        const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
+                        void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream,
+                        const ms_scan_plan *plan) {
+    if (plan && !plan_valid(plan)) return MS_ERR_SHAPE;
+    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
+    if (rc != MS_OK) return rc;
+    if (workspace_bytes < mamba_scan_workspace_size(dims) || (workspace_bytes > 0 && !workspace))
+        return MS_ERR_WORKSPACE;
+    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
+    if (dims->seqlen == 0 && !last_state) return MS_OK;
+    return scan_common(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                       dims, dev_status, stream, plan, nullptr);
+}
+
+int mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b, const void *conv_x0,
+                        void *u_out, const ms_conv_dims *cdims, const void *delta, const float *A,
+                        const void *B, const void *C, const float *D, const void *z,
+                        const float *delta_bias, int softplus_flag, const float *initial_state,
+                        void *y, float *last_state, const ms_scan_dims *dims,
+                        const ms_scan_plan *plan, int *dev_status, ms_stream_t stream) {
+    if (plan && (!plan_valid(plan) || plan->chunks_per_lane != 1 || (plan->poly8 != 0 && plan->poly8 != 8)))
+        return MS_ERR_SHAPE;
+    int rc = check_scan(x, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
+    if (rc != MS_OK) return rc;
+    const ConvIn cv{conv_w, conv_b, conv_x0, u_out, cdims};
+    rc = check_conv(cv, dims);
+    if (rc != MS_OK) return rc;
+    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
+    if (dims->seqlen == 0 && !last_state) return MS_OK;
+    return scan_common(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                       dims, dev_status, stream, plan, &cv);
 }
 
 int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,

@@ -20,6 +20,15 @@ struct ScanArgs {
     int softplus;
     int vec_in;   // u/delta/z rows 16-byte aligned: vector loads allowed
     int vec_out;  // y rows 16-byte aligned: vector stores allowed
+    // Causal conv front-end (conv_w == nullptr: u is read as given). With the
+    // front-end, `u` points at the conv input x.
+    const float *conv_w, *conv_b;  // [dim, conv_width], [dim]
+    const void *conv_x0;           // [batch, dim, conv_width - 1] in the input dtype, or null
+    void *u_out;                   // [batch, dim, L] in the input dtype, or null
+    int64_t uo_sb, uo_sd;
+    int conv_width;                // 1..4
+    int conv_silu;
+    int vec_uout;                  // u_out rows 16-byte aligned
 };
 
 // Launch shape chosen on the host for one scan call.

@@ -29,6 +29,15 @@
 // exp(x) = 2^(x log2 e); a fixed, lane-uniform share (poly8 / 8) of the
 // (state pair, token) slots uses the FMA-pipe polynomial, the rest the MUFU
 // ex2, to balance the two pipes.
+//
+// Conv front-end (CONV): the block's input path (blog, section 2, block
+// diagram) runs a short causal convolution per channel and silu before the
+// SSM. With CONV the kernel reads that convolution's input x instead of u and
+// forms u_t = silu(bias_d + sum_k w[d,k] x_{t-(W-1)+k}) in the prologue, so u
+// never makes an HBM round trip. The 3 tokens before a lane's chunk come from
+// the previous lane of the channel by shuffle (lane 0 takes the last lane's
+// chunk of the previous tile, kept in registers; before token 0 the given
+// history or zeros).
 
 #include "ms_device.cuh"
 #include "ms_internal.h"
@@ -237,9 +246,10 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, float dl,
     return lo + hi;
 }
 
-template <typename TIn, typename TOut, int G, int CH, int POLY8>
+template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV>
 __global__ void __launch_bounds__(kThreads, CH == 1 ? MS_SCAN_MINB : 1)
 scan_fwd_kernel(const ScanArgs a) {
+    static_assert(!CONV || CH == 1, "the conv front-end runs with one chunk per lane");
     using Gm = Geom<G, CH>;
     constexpr int TT = Gm::kTT;
     constexpr int S = Gm::kStates;
@@ -291,10 +301,32 @@ scan_fwd_kernel(const ScanArgs a) {
     const bool has_z = a.z != nullptr;
     const bool sp = a.softplus != 0;
 
+    // Conv taps right-aligned in cw (cw[3] weights the current token) and the
+    // 3 inputs before this lane's next chunk (only the channel's last lane's
+    // copy is read: it feeds lane 0 of the next tile).
+    float cw[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cb = 0.0f;
+    float keep[3] = {0.0f, 0.0f, 0.0f};
+    if constexpr (CONV) {
+        const int W = a.conv_width;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int src = k - (4 - W);
+            if (src >= 0) cw[k] = __ldg(a.conv_w + dd * W + src);
+        }
+        cb = a.conv_b ? __ldg(a.conv_b + dd) : 0.0f;
+        if (a.conv_x0 != nullptr && active) {
+            const TIn *x0 = static_cast<const TIn *>(a.conv_x0) + (b * a.dim + d) * (W - 1);
+#pragma unroll
+            for (int j = 1; j <= 3; ++j)
+                if (W - 1 - j >= 0) keep[3 - j] = Elem<TIn>::load(x0 + (W - 1 - j));
+        }
+    }
+
     const TIn *u_row = static_cast<const TIn *>(a.u) + b * a.u_sb + dd * a.u_sd;
     const TIn *d_row = static_cast<const TIn *>(a.delta) + b * a.dl_sb + dd * a.dl_sd;
     const TIn *z_row = has_z ? static_cast<const TIn *>(a.z) + b * a.z_sb + dd * a.z_sd : u_row;
     TOut *y_row = static_cast<TOut *>(a.y) + b * a.y_sb + dd * a.y_sd;
+    TIn *uo_row = CONV && a.u_out ? static_cast<TIn *>(a.u_out) + b * a.uo_sb + dd * a.uo_sd : nullptr;
     const TIn *B_b = static_cast<const TIn *>(a.B) + b * a.B_sb;
     const TIn *C_b = static_cast<const TIn *>(a.C) + b * a.C_sb;
     const bool vin = a.vec_in != 0;
@@ -345,9 +377,41 @@ scan_fwd_kernel(const ScanArgs a) {
 #pragma unroll
         for (int i = 0; i < CH; ++i) {
             const int64_t ts = t0 + 8 * (g * CH + i);
+            float uv[8];
+            if constexpr (CONV) {
+                // Halo x_{ts-3..ts-1}: the previous lane's chunk tail, or for
+                // lane 0 the last lane's tail from the previous tile.
+                const float t5 = nu[i].get(5), t6 = nu[i].get(6), t7 = nu[i].get(7);
+                const bool last_lane = g == G - 1;
+                const int src = g == 0 ? lane + G - 1 : lane - 1;
+                const float h0 = __shfl_sync(0xffffffffu, last_lane ? keep[0] : t5, src);
+                const float h1 = __shfl_sync(0xffffffffu, last_lane ? keep[1] : t6, src);
+                const float h2 = __shfl_sync(0xffffffffu, last_lane ? keep[2] : t7, src);
+                keep[0] = t5;
+                keep[1] = t6;
+                keep[2] = t7;
+                float xs[11];
+                xs[0] = h0;
+                xs[1] = h1;
+                xs[2] = h2;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) xs[3 + j] = nu[i].get(j);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float v = fmaf(cw[0], xs[j], cb);
+                    v = fmaf(cw[1], xs[j + 1], v);
+                    v = fmaf(cw[2], xs[j + 2], v);
+                    v = fmaf(cw[3], xs[j + 3], v);
+                    uv[j] = a.conv_silu ? silu_f(v) : v;
+                }
+                if (uo_row != nullptr && active) store8<TIn>(uo_row, ts, L, a.vec_uout != 0, uv);
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) uv[j] = nu[i].get(j);
+            }
 #pragma unroll
             for (int j = 0; j < 8; ++j) {
-                const float uj = nu[i].get(j);
+                const float uj = uv[j];
                 const float v = nd[i].get(j) + bias;
                 const float step = sp ? softplus_f(v) : v;
                 dl[i][j] = (ts + j < L) ? step : 0.0f;  // past the end: the state is left alone
@@ -475,7 +539,7 @@ scan_fwd_kernel(const ScanArgs a) {
     }
 }
 
-template <typename TIn, typename TOut, int G, int CH, int POLY8>
+template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV = false>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     using Gm = Geom<G, CH>;
     using Sm = SmemLayout<G, CH>;
@@ -490,12 +554,12 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !opted[dev]) {
-        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8>,
+        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
         if (e != cudaSuccess) return e;
         if (dev < 64) opted[dev] = true;
     }
-    scan_fwd_kernel<TIn, TOut, G, CH, POLY8><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
+    scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -523,10 +587,35 @@ cudaError_t launch_types(const ScanArgs &a, const ScanPlan &pl, cudaStream_t str
     }
 }
 
+// Conv front-end: one chunk per lane, exponentials all on MUFU or all on the
+// polynomial.
+template <typename TIn, typename TOut>
+cudaError_t launch_types_conv(const ScanArgs &a, const ScanPlan &pl, cudaStream_t stream) {
+    const bool poly = pl.poly8 != 0;
+    switch (pl.lanes_per_channel) {
+        case 1: return poly ? launch_one<TIn, TOut, 1, 1, 8, true>(a, stream)
+                            : launch_one<TIn, TOut, 1, 1, 0, true>(a, stream);
+        case 2: return poly ? launch_one<TIn, TOut, 2, 1, 8, true>(a, stream)
+                            : launch_one<TIn, TOut, 2, 1, 0, true>(a, stream);
+        case 4: return poly ? launch_one<TIn, TOut, 4, 1, 8, true>(a, stream)
+                            : launch_one<TIn, TOut, 4, 1, 0, true>(a, stream);
+        default: return poly ? launch_one<TIn, TOut, 8, 1, 8, true>(a, stream)
+                             : launch_one<TIn, TOut, 8, 1, 0, true>(a, stream);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16,
                             cudaStream_t stream) {
+    if (a.conv_w != nullptr) {
+        if (in_bf16) {
+            return out_bf16 ? launch_types_conv<__nv_bfloat16, __nv_bfloat16>(a, plan, stream)
+                            : launch_types_conv<__nv_bfloat16, float>(a, plan, stream);
+        }
+        return out_bf16 ? launch_types_conv<float, __nv_bfloat16>(a, plan, stream)
+                        : launch_types_conv<float, float>(a, plan, stream);
+    }
     if (in_bf16) {
         return out_bf16 ? launch_types<__nv_bfloat16, __nv_bfloat16>(a, plan, stream)
                         : launch_types<__nv_bfloat16, float>(a, plan, stream);

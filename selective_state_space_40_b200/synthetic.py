@@ -111,6 +111,20 @@ def scan_inputs(w: ScanWorkload, seed: Optional[int] = None) -> Dict[str, torch.
     return dict(u=u, delta=delta, z=z, B=B, C=C, A=a_matrix(d, n), D=D, delta_bias=bias)
 
 
+def conv_params(w: ScanWorkload, width: int = 4, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """Parameters of the causal conv front-end for a scan workload (whose ``u``
+    draw serves as the conv input x): conv_w [d, width] and conv_b [d] fp32
+    ~ Uniform(-1/sqrt(width), 1/sqrt(width)) (a depthwise conv's fan-in is
+    its width), and a history conv_x0 [b, d, width-1] ~ N(0, 1) in
+    ``w.in_dtype``; drawn in that order from seed + 1000."""
+    g = torch.Generator().manual_seed((w.seed if seed is None else seed) + 1000)
+    lim = 1.0 / math.sqrt(width)
+    conv_w = (torch.rand(w.dim, width, generator=g, dtype=torch.float32) * 2.0 - 1.0) * lim
+    conv_b = (torch.rand(w.dim, generator=g, dtype=torch.float32) * 2.0 - 1.0) * lim
+    conv_x0 = _normal(g, (w.batch, w.dim, width - 1), w.in_dtype)
+    return dict(conv_w=conv_w, conv_b=conv_b, conv_x0=conv_x0)
+
+
 def decode_params(w: DecodeWorkload) -> Dict[str, torch.Tensor]:
     """state0 [b, d, N] fp32 ~ N(0, 0.1); A, D, delta_bias as the 130M-class layer."""
     g = torch.Generator().manual_seed(w.seed)

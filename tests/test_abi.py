@@ -33,7 +33,7 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size",
               "mamba_status_string", "mamba_device_check", "mamba_scan_fwd_plan",
-              "mamba_scan_choose_plan"):
+              "mamba_scan_choose_plan", "mamba_conv_scan_fwd"):
         assert n in names
 
 
@@ -44,7 +44,7 @@ def test_library_exports(lib, name):
 
 def test_no_cpu_fallback_symbols(lib):
     # the product library never links the oracle
-    for sym in ("oracle_scan_f64", "oracle_state_update_f64"):
+    for sym in ("oracle_scan_f64", "oracle_state_update_f64", "oracle_causal_conv_f64"):
         with pytest.raises(AttributeError):
             getattr(lib, sym)
 
@@ -120,6 +120,41 @@ def test_choose_plan(lib):
     assert plan.chunks_per_lane in (1, 2)
     rc, _ = mb.mamba_scan_choose_plan(_dims(dstate=40))
     assert rc == mb.MS_ERR_SHAPE
+
+
+def _conv(dims, width=4, silu=1, uout_sb=256, uout_sd=32, w=FAKE, b=None, x0=None, u_out=None,
+          x=FAKE, y=FAKE, plan=None):
+    cd = mb.ConvDims(width, uout_sb, uout_sd, silu)
+    return mb.mamba_conv_scan_fwd(x, w, b, x0, u_out, cd, FAKE, FAKE, FAKE, FAKE, None, None, None, 1,
+                                  None, y, None, dims, plan, None, None)
+
+
+def test_conv_scan_rejects_bad_arguments(lib):
+    assert _conv(_dims(), width=0) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(), width=5) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(), uout_sd=-1) == mb.MS_ERR_STRIDE
+    assert _conv(_dims(), w=None) == mb.MS_ERR_NULL
+    assert _conv(_dims(), x=None) == mb.MS_ERR_NULL
+    assert _conv(_dims(), w=FAKE + 2) == mb.MS_ERR_ALIGN
+    assert _conv(_dims(), b=FAKE + 1) == mb.MS_ERR_ALIGN
+    assert _conv(_dims(in_dtype=mb.MS_BF16), x0=FAKE + 1) == mb.MS_ERR_ALIGN
+    assert _conv(_dims(), u_out=FAKE + 2) == mb.MS_ERR_ALIGN
+    assert _conv(_dims(), u_out=FAKE, uout_sb=1 << 61, uout_sd=1) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(in_dtype=9)) == mb.MS_ERR_DTYPE
+    # the conv front-end runs one chunk per lane, exponentials all MUFU or all polynomial
+    assert _conv(_dims(), plan=mb.ScanPlan(4, 2, 0)) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(), plan=mb.ScanPlan(4, 1, 2)) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(), plan=mb.ScanPlan(3, 1, 0)) == mb.MS_ERR_SHAPE
+    cd = mb.ConvDims(4, 0, 0, 1)
+    assert mb.library().mamba_conv_scan_fwd(FAKE, FAKE, None, None, None, None, FAKE, FAKE, FAKE, FAKE,
+                                            None, None, None, 1, None, FAKE, None, ctypes.byref(_dims()),
+                                            None, None, None) == mb.MS_ERR_NULL
+    del cd
+
+
+def test_conv_scan_empty_is_a_noop(lib):
+    assert _conv(_dims(batch=0)) == mb.MS_OK
+    assert _conv(_dims(dim=0), w=None, x=None, y=None) == mb.MS_OK
 
 
 def _udims(**kw):

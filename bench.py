@@ -379,6 +379,31 @@ def main(argv=None):
     dec_gbs = dbytes / (dec_ms * 1e-3) / 1e9
     del states
 
+    # ---- scan with the causal conv front-end (width 4) on the same layer: u is
+    # formed from the conv input x in the load stage, so the bytes are the
+    # scan's plus the filter.
+    cp = {k: v.to(dev) for k, v in syn.conv_params(w, 4).items()}
+    conv_steps = 40
+
+    def conv_step(i):
+        g = sets[i & 1]
+        mb.conv_scan_fwd(g["u"], cp["conv_w"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"],
+                         g["delta_bias"], True, conv_b=cp["conv_b"], y=y, last_state=last, stream=stream)
+
+    for i in range(4):
+        conv_step(i)
+    cev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(conv_steps)]
+    torch.cuda.synchronize()
+    for i in range(conv_steps):
+        cev[i][0].record(stream)
+        conv_step(i)
+        cev[i][1].record(stream)
+    torch.cuda.synchronize()
+    conv_ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in cev), world, dev)
+    conv_bytes = nbytes + w.dim * 5 * 4
+    conv_gbs = conv_bytes / (conv_ms * 1e-3) / 1e9
+
     # ---- CPU baseline: the oracle on this host's cores, whole passes over the
     # workload repeated until about ten seconds of wall time have gone by
     cpu = None
@@ -416,6 +441,10 @@ def main(argv=None):
                             "l2": "back-to-back steps over 3 rotating 84 MB states (> 126 MB L2)",
                             "timing": f"one event pair around {dec_steps} back-to-back launches",
                             "traffic": recorded_traffic("decode_step")},
+            "conv_scan": {"workload": w.name + " + causal conv width 4", "value": conv_gbs, "unit": "GB/s",
+                          "ms": conv_ms, "bytes": conv_bytes, "frac": conv_gbs / peak,
+                          "l2": "two rotating input sets", "timing": "mean of per-launch event pairs",
+                          "traffic": recorded_traffic("conv_scan_130m")},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

@@ -12,6 +12,7 @@ from .oracle import (  # noqa: F401
     conv_scan,
     load_oracle,
     scan,
+    scan_bwd,
     scan_mt,
     state_update,
     softplus,

@@ -320,3 +320,125 @@ int oracle_causal_conv_f64(int64_t batch, int64_t dim, int64_t seqlen, int64_t w
     }
     return 0;
 }
+
+/*
+ * Gradients of the selective scan (reverse mode of the recurrence above; the
+ * blog's section 2 notes the same model is trained through the scan). For a
+ * scalar loss with dL/dy = dout [batch][dim][seqlen] on the gated output and
+ * dL/dlast_state = dlast [batch][dim][dstate] (nullable = 0), per channel:
+ *   forward, kept per token: Delta_t, A_bar_t[n], h_t[n], the pre-gate output
+ *     q_t = sum_n C_t[n] h_t[n] + D u_t, and the gate g_t = silu(z_t) (1 without z);
+ *   backward over t = L-1 .. 0, with lam the adjoint of h_t:
+ *     dq_t = dout_t g_t;  dz_t = dout_t q_t silu'(z_t);  dD += dq_t u_t;  du_t = D dq_t
+ *     lam[n] = C_t[n] dq_t + carry[n]           (carry = dlast at t = L-1)
+ *     dC_t[n] += dq_t h_t[n]
+ *     dh_{t-1}[n] through A_bar: dAbar = lam[n] h_{t-1}[n]
+ *     dA[n] += dAbar A_bar_t[n] Delta_t;  dDelta_t += dAbar A_bar_t[n] A[n]
+ *     input term Delta_t u_t B_t[n]: dDelta_t += lam u_t B_t[n]; du_t += lam Delta_t B_t[n];
+ *                                    dB_t[n] += lam Delta_t u_t
+ *     carry[n] = A_bar_t[n] lam[n]
+ *   ddelta_t = dDelta_t * sigmoid(delta_t + bias) (softplus' ; 1 without the flag),
+ *   dbias += ddelta_t, dh0 = carry after t = 0.
+ * dB, dC, dA, dD, dbias are sums over channels/tokens/batch and are
+ * ACCUMULATED into (callers zero them); du, ddelta, dz, dh0 are written.
+ * Nullable outputs: dz (needs z), dD, dbias, dh0; nullable inputs as the scan.
+ */
+static double silu_grad(double z)
+{
+    double s = 1.0 / (1.0 + exp(-z));
+#if ORACLE_MUTANT == 16
+    return s; /* mutant: derivative of silu missing the z*s*(1-s) term */
+#else
+    return s * (1.0 + z * (1.0 - s));
+#endif
+}
+
+int oracle_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seqlen,
+                        const double *u, const double *delta, const double *A,
+                        const double *B, const double *C, const double *D,
+                        const double *z, const double *delta_bias, int softplus_flag,
+                        const double *h0, const double *dout, const double *dlast,
+                        double *du, double *ddelta, double *dA, double *dB, double *dC,
+                        double *dD, double *dz, double *dbias, double *dh0)
+{
+    if (batch < 0 || dim < 0 || dstate < 1 || seqlen < 0) return -1;
+    if (batch * dim * seqlen > 0 &&
+        (!u || !delta || !A || !B || !C || !dout || !du || !ddelta || !dA || !dB || !dC)) return -1;
+    const int64_t N = dstate, L = seqlen;
+    double *hs = (double *)malloc((size_t)((L + 1) * N) * sizeof(double)); /* h_{-1..L-1} */
+    double *ab = (double *)malloc((size_t)((L > 0 ? L : 1) * N) * sizeof(double));
+    double *dts = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    double *q = (double *)malloc((size_t)(L > 0 ? L : 1) * sizeof(double));
+    double *lam = (double *)malloc((size_t)N * sizeof(double));
+    double *carry = (double *)malloc((size_t)N * sizeof(double));
+    if (!hs || !ab || !dts || !q || !lam || !carry) {
+        free(hs); free(ab); free(dts); free(q); free(lam); free(carry);
+        return -1;
+    }
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t d = 0; d < dim; ++d) {
+            const int64_t c = b * dim + d, row = c * L;
+            const double *Bb = B + b * N * L, *Cb = C + b * N * L;
+            const double Dd = D ? D[d] : 0.0, bias = delta_bias ? delta_bias[d] : 0.0;
+            /* forward, keeping what the backward needs */
+            for (int64_t n = 0; n < N; ++n) hs[n] = h0 ? h0[c * N + n] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const double dt = step_size(delta[row + t], bias, softplus_flag);
+                dts[t] = dt;
+                double acc = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double a = exp(dt * A[d * N + n]);
+                    ab[t * N + n] = a;
+                    const double h = a * hs[t * N + n] + dt * u[row + t] * Bb[n * L + t];
+                    hs[(t + 1) * N + n] = h;
+                    acc += Cb[n * L + t] * h;
+                }
+                q[t] = acc + Dd * u[row + t];
+            }
+            /* backward */
+            for (int64_t n = 0; n < N; ++n) carry[n] = dlast ? dlast[c * N + n] : 0.0;
+            double dDacc = 0.0, dbacc = 0.0;
+            for (int64_t t = L - 1; t >= 0; --t) {
+                const double ut = u[row + t], dt = dts[t];
+                const double g = z ? oracle_silu(z[row + t]) : 1.0;
+                const double dq = dout[row + t] * g;
+                if (z && dz) dz[row + t] = dout[row + t] * q[t] * silu_grad(z[row + t]);
+                dDacc += dq * ut;
+                double dut = Dd * dq, ddt = 0.0;
+                for (int64_t n = 0; n < N; ++n) {
+                    const double Bt = Bb[n * L + t], Ct = Cb[n * L + t];
+                    const double ht = hs[(t + 1) * N + n], hprev = hs[t * N + n];
+                    const double a = ab[t * N + n];
+#if ORACLE_MUTANT == 17
+                    lam[n] = Ct * dq + a * carry[n]; /* mutant: adjoint decayed by this token's A_bar */
+#else
+                    lam[n] = Ct * dq + carry[n];
+#endif
+                    dC[b * N * L + n * L + t] += dq * ht;
+                    const double dab = lam[n] * hprev;
+                    dA[d * N + n] += dab * a * dt;
+#if ORACLE_MUTANT == 18
+                    (void)0; /* mutant: Delta's path through A_bar dropped */
+#else
+                    ddt += dab * a * A[d * N + n];
+#endif
+                    ddt += lam[n] * ut * Bt;
+                    dut += lam[n] * dt * Bt;
+                    dB[b * N * L + n * L + t] += lam[n] * dt * ut;
+                    carry[n] = a * lam[n];
+                }
+                const double v = delta[row + t] + bias;
+                const double dv = softplus_flag ? ddt / (1.0 + exp(-v)) : ddt;
+                du[row + t] = dut;
+                ddelta[row + t] = dv;
+                dbacc += dv;
+            }
+            if (dD) dD[d] += dDacc;
+            if (dbias) dbias[d] += dbacc;
+            if (dh0)
+                for (int64_t n = 0; n < N; ++n) dh0[c * N + n] = carry[n];
+        }
+    }
+    free(hs); free(ab); free(dts); free(q); free(lam); free(carry);
+    return 0;
+}

@@ -52,6 +52,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_state_update_f64.restype = ctypes.c_int
     lib.oracle_causal_conv_f64.argtypes = [i64, i64, i64, i64] + [_dp] * 4 + [ctypes.c_int, _dp]
     lib.oracle_causal_conv_f64.restype = ctypes.c_int
+    lib.oracle_scan_bwd_f64.argtypes = [i64, i64, i64, i64] + [_dp] * 8 + [ctypes.c_int] + [_dp] * 12
+    lib.oracle_scan_bwd_f64.restype = ctypes.c_int
     return lib
 
 
@@ -145,6 +147,30 @@ def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None,
     if rc != 0:
         raise ValueError(f"oracle_state_update_f64 rejected its arguments (rc={rc})")
     return y, st
+
+
+def scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, dout, h0=None, dlast=None, lib=None):
+    """Gradients of the selective scan in fp64 for dL/dy = dout (and
+    dL/dlast_state = dlast). Returns a dict du, ddelta, dA, dB, dC, dD, dz,
+    ddelta_bias, dh0 (dD/dz/ddelta_bias None when D/z/delta_bias are None)."""
+    lib = lib or load_oracle()
+    u, delta, A, B, C, D, z, delta_bias, h0, batch, dim, N, L = _scan_args(
+        u, delta, A, B, C, D, z, delta_bias, h0)
+    dout, dlast = _f64(dout), _f64(dlast)
+    assert dout.shape == u.shape and (dlast is None or dlast.shape == (batch, dim, N))
+    g = {"du": np.full(u.shape, np.nan), "ddelta": np.full(u.shape, np.nan),
+         "dA": np.zeros((dim, N)), "dB": np.zeros((batch, N, L)), "dC": np.zeros((batch, N, L)),
+         "dD": None if D is None else np.zeros(dim), "dz": None if z is None else np.full(u.shape, np.nan),
+         "ddelta_bias": None if delta_bias is None else np.zeros(dim),
+         "dh0": np.full((batch, dim, N), np.nan)}
+    rc = lib.oracle_scan_bwd_f64(batch, dim, N, L, _ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                 _ptr(z), _ptr(delta_bias), int(bool(softplus_flag)), _ptr(h0), _ptr(dout),
+                                 _ptr(dlast), _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]),
+                                 _ptr(g["dC"]), _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]),
+                                 _ptr(g["dh0"]))
+    if rc != 0:
+        raise ValueError(f"oracle_scan_bwd_f64 rejected its arguments (rc={rc})")
+    return g
 
 
 def causal_conv(x, w, bias=None, x0=None, silu_flag=True, lib=None):

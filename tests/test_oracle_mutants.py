@@ -10,7 +10,7 @@ import numpy as np
 import pytest
 
 import oracle.oracle as ow
-from test_oracle_pins import PINS, TOL
+from test_oracle_pins import PINS, pin_tol
 
 MUTANTS = {
     1: "D skip dropped",
@@ -28,6 +28,9 @@ MUTANTS = {
     13: "conv filter taps reversed",
     14: "conv activation dropped",
     15: "conv history before token 0 ignored",
+    16: "gradient of silu missing its z*s*(1-s) term",
+    17: "adjoint state decayed by its own token's A_bar",
+    18: "gradient of Delta through A_bar dropped",
 }
 
 
@@ -46,6 +49,6 @@ def test_some_pin_catches_mutant(mutant, mutant_dir):
                 err = pin(lib)
             except Exception:  # a crash or an assertion inside a pin also counts
                 err = float("inf")
-        if not (err <= TOL):
+        if not (err <= pin_tol(name)):
             caught.append(name)
     assert caught, f"no pin caught mutant {mutant} ({MUTANTS[mutant]})"

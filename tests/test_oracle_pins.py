@@ -19,6 +19,9 @@ mathematics) fix, written without the oracle's code:
 * softplus / silu special values and library routines (numpy logaddexp,
   scipy expit);
 * the hand-worked cases in tests/golden/hand_worked.json;
+* the gradients of the scan (reverse mode) against central finite differences
+  of the forward oracle along random directions, for every input (u, delta,
+  A, B, C, D, z, delta_bias, h0) with a loss on both y and last_state;
 * the block's causal conv front-end (blog, section 2, block diagram: a short
   causal convolution per channel, then silu, feeds the SSM) against numpy's
   full convolution with the history prepended, one-hot filters as explicit
@@ -338,6 +341,41 @@ def pin_conv_scan_split(lib):
                _rel(np.concatenate([u1, u2], axis=2), u))
 
 
+def pin_backward_finite_differences(lib):
+    """Every gradient of oracle.scan_bwd against (L(x + eV) - L(x - eV)) / 2e
+    with L = <dout, y> + <dlast, last_state>; returns the worst relative
+    mismatch (central differences in fp64 reach ~1e-9 here)."""
+    rng = np.random.default_rng(22)
+    b, d, N, L = 2, 3, 4, 9
+    x = dict(u=rng.standard_normal((b, d, L)), delta=rng.standard_normal((b, d, L)),
+             A=-rng.uniform(0.2, 2.0, (d, N)), B=rng.standard_normal((b, N, L)),
+             C=rng.standard_normal((b, N, L)), D=rng.standard_normal(d), z=rng.standard_normal((b, d, L)),
+             delta_bias=rng.uniform(-1.5, 0.5, d), h0=rng.standard_normal((b, d, N)))
+    dout = rng.standard_normal((b, d, L))
+    dlast = rng.standard_normal((b, d, N))
+
+    def loss(v):
+        y, last = oracle.scan(v["u"], v["delta"], v["A"], v["B"], v["C"], v["D"], v["z"], v["delta_bias"],
+                              True, h0=v["h0"], lib=lib)
+        return float(np.sum(y * dout) + np.sum(last * dlast))
+
+    g = oracle.scan_bwd(x["u"], x["delta"], x["A"], x["B"], x["C"], x["D"], x["z"], x["delta_bias"], True,
+                        dout, h0=x["h0"], dlast=dlast, lib=lib)
+    names = dict(u="du", delta="ddelta", A="dA", B="dB", C="dC", D="dD", z="dz", delta_bias="ddelta_bias",
+                 h0="dh0")
+    eps = 1e-5
+    worst = 0.0
+    for k, gk in names.items():
+        for _ in range(2):
+            V = rng.standard_normal(x[k].shape)
+            xp = dict(x); xp[k] = x[k] + eps * V
+            xm = dict(x); xm[k] = x[k] - eps * V
+            fd = (loss(xp) - loss(xm)) / (2 * eps)
+            an = float(np.sum(g[gk] * V))
+            worst = max(worst, abs(fd - an) / max(abs(an), 1e-3))
+    return worst
+
+
 PINS = {
     "softplus_silu": pin_softplus_silu,
     "lti_convolution": pin_lti_convolution,
@@ -351,13 +389,21 @@ PINS = {
     "conv_numpy": pin_conv_numpy,
     "conv_shift": pin_conv_shift,
     "conv_scan_split": pin_conv_scan_split,
+    "backward_finite_differences": pin_backward_finite_differences,
 }
+
+# Pins that compare against a numerical approximation carry their own bound.
+PIN_TOL = {"backward_finite_differences": 1e-7}
+
+
+def pin_tol(name):
+    return PIN_TOL.get(name, TOL)
 
 
 @pytest.mark.parametrize("name", sorted(PINS))
 def test_pin(name, oracle_lib):
     err = PINS[name](oracle_lib)
-    assert err <= TOL, f"pin {name}: error {err:.3e} > {TOL:.0e}"
+    assert err <= pin_tol(name), f"pin {name}: error {err:.3e} > {pin_tol(name):.0e}"
 
 
 def test_multithreaded_oracle_is_identical(oracle_lib):

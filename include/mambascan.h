@@ -191,6 +191,55 @@ int mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
                         const ms_scan_plan *plan, int *dev_status, ms_stream_t stream);
 
 /*
+ * Training. The forward of a training step also saves the state before every
+ * MS_CKPT_TOKENS-token block (fp32 [batch, dim, ceil(seqlen/64), dstate],
+ * mamba_scan_ckpt_size() bytes); the backward recomputes each block from it.
+ * The blog's section 2 describes training as running the same model through
+ * the scan; the gradients are the reverse mode of the recurrence above.
+ */
+#define MS_CKPT_TOKENS 64
+
+/* Bytes of the saved-state array for these dims (0 when seqlen is 0). */
+size_t mamba_scan_ckpt_size(const ms_scan_dims *dims);
+
+/*
+ * mamba_scan_fwd that also writes the saved states into ckpt (required,
+ * caller-owned, mamba_scan_ckpt_size() bytes, 4-byte aligned).
+ */
+int mamba_scan_fwd_train(const void *u, const void *delta, const float *A, const void *B,
+                         const void *C, const float *D, const void *z, const float *delta_bias,
+                         int softplus_flag, const float *initial_state, void *y, float *last_state,
+                         float *ckpt, const ms_scan_dims *dims, int *dev_status, ms_stream_t stream);
+
+/* Workspace bytes mamba_scan_bwd needs when it is given no saved states
+   (it then recomputes them); 0 is enough when ckpt is given. */
+size_t mamba_scan_bwd_workspace_size(const ms_scan_dims *dims);
+
+/*
+ * Gradients of the selective scan for a loss with dL/dy = dout and
+ * dL/dlast_state = dlast. Inputs are those of the forward (same dims; dout
+ * has y's dtype and strides). Gradients are fp32 and dense:
+ *   du, ddelta, dz           [batch, dim, seqlen]   (dz only with z; NULL = skip)
+ *   dB, dC                   [batch, dstate, seqlen]
+ *   dA                       [dim, dstate]
+ *   dD, ddelta_bias          [dim]                  (NULL = skip)
+ *   dinitial_state           [batch, dim, dstate]   (NULL = skip): dL/d initial_state
+ * dA, dB, dC, dD, ddelta_bias are sums over channels, batch rows or tokens,
+ * accumulated with fp32 atomics (the library zeroes them first on the
+ * stream), so their last bits may differ between runs; the others are
+ * written directly. ckpt: the saved states of mamba_scan_fwd_train for the
+ * same inputs, or NULL to have them recomputed into the workspace
+ * (mamba_scan_bwd_workspace_size() bytes). dlast NULL = 0.
+ * Returns MS_OK or an MS_ERR_* code (also MS_ERR_SHAPE for dstate > 16).
+ */
+int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                   const float *initial_state, const float *ckpt, const void *dout, const float *dlast,
+                   float *du, float *ddelta, float *dA, float *dB, float *dC, float *dD, float *dz,
+                   float *ddelta_bias, float *dinitial_state, const ms_scan_dims *dims,
+                   void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream);
+
+/*
  * Sizes and strides of one decode step.
  *   x, delta, z, y : [batch, dim]     element (b,d) at b*x_sb + d
  *   B, C           : [batch, dstate]  element (b,n) at b*x_sb + n

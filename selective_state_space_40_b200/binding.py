@@ -76,6 +76,16 @@ def library() -> ctypes.CDLL:
                                             [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(ScanDims),
                                              ctypes.POINTER(ScanPlan), _vp, _vp])
         lib.mamba_conv_scan_fwd.restype = ctypes.c_int
+        lib.mamba_scan_ckpt_size.argtypes = [ctypes.POINTER(ScanDims)]
+        lib.mamba_scan_ckpt_size.restype = ctypes.c_size_t
+        lib.mamba_scan_bwd_workspace_size.argtypes = [ctypes.POINTER(ScanDims)]
+        lib.mamba_scan_bwd_workspace_size.restype = ctypes.c_size_t
+        lib.mamba_scan_fwd_train.argtypes = [_vp] * 8 + [ctypes.c_int, _vp, _vp, _vp, _vp,
+                                                         ctypes.POINTER(ScanDims), _vp, _vp]
+        lib.mamba_scan_fwd_train.restype = ctypes.c_int
+        lib.mamba_scan_bwd.argtypes = ([_vp] * 8 + [ctypes.c_int] + [_vp] * 13 +
+                                       [ctypes.POINTER(ScanDims), _vp, ctypes.c_size_t, _vp, _vp])
+        lib.mamba_scan_bwd.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
                                                        _vp, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
@@ -116,6 +126,30 @@ def mamba_scan_fwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_s
     if plan is None:
         return lib.mamba_scan_fwd(*args)
     return lib.mamba_scan_fwd_plan(*args, ctypes.byref(plan))
+
+
+def mamba_scan_ckpt_size(dims: ScanDims) -> int:
+    return library().mamba_scan_ckpt_size(ctypes.byref(dims))
+
+
+def mamba_scan_bwd_workspace_size(dims: ScanDims) -> int:
+    return library().mamba_scan_bwd_workspace_size(ctypes.byref(dims))
+
+
+def mamba_scan_fwd_train(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                         ckpt, dims: ScanDims, dev_status, stream) -> int:
+    return library().mamba_scan_fwd_train(u, delta, A, B, C, D, z, delta_bias, int(softplus_flag),
+                                          initial_state, y, last_state, ckpt, ctypes.byref(dims),
+                                          dev_status, stream)
+
+
+def mamba_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, ckpt, dout, dlast,
+                   du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dinitial_state, dims: ScanDims,
+                   workspace, workspace_bytes, dev_status, stream) -> int:
+    return library().mamba_scan_bwd(u, delta, A, B, C, D, z, delta_bias, int(softplus_flag), initial_state,
+                                    ckpt, dout, dlast, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
+                                    dinitial_state, ctypes.byref(dims), workspace, int(workspace_bytes),
+                                    dev_status, stream)
 
 
 def mamba_conv_scan_fwd(x, conv_w, conv_b, conv_x0, u_out, cdims: ConvDims, delta, A, B, C, D, z,
@@ -249,6 +283,60 @@ def conv_scan_fwd(x, conv_w, delta, A, B, C, D=None, z=None, delta_bias=None, so
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba_conv_scan_fwd")
     return y, last_state, u_out
+
+
+def scan_fwd_train(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus: bool = True,
+                   initial_state=None, out_dtype=None, stream=None, dev_status=None):
+    """Training forward: (y, last_state, ckpt), ckpt the saved states the
+    backward recomputes from (fp32 [b, d, ceil(L/64), N])."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    y = torch.empty((batch, dim, L), dtype=out_dtype, device=u.device)
+    last = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
+    ckpt = torch.empty((batch, dim, (L + 63) // 64, N), dtype=torch.float32, device=u.device)
+    dims = scan_dims_for(u, delta, B, C, z, y)
+    rc = mamba_scan_fwd_train(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                              _ptr(delta_bias), softplus, _ptr(initial_state), _ptr(y), _ptr(last), _ptr(ckpt),
+                              dims, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_scan_fwd_train")
+    return y, last, ckpt
+
+
+def scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, dlast=None, initial_state=None,
+             ckpt=None, want_dinitial: bool = True, stream=None, dev_status=None, workspace=None):
+    """Gradients of the scan on torch CUDA tensors. dout has y's shape and
+    dtype. Returns a dict du, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
+    dinitial_state (fp32; None where the input is None)."""
+    torch = _torch()
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    dev = u.device
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = {"du": torch.empty((batch, dim, L), **f32), "ddelta": torch.empty((batch, dim, L), **f32),
+         "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
+         "dC": torch.empty((batch, N, L), **f32),
+         "dD": torch.empty(dim, **f32) if D is not None else None,
+         "dz": torch.empty((batch, dim, L), **f32) if z is not None else None,
+         "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None,
+         "dinitial_state": torch.empty((batch, dim, N), **f32) if want_dinitial else None}
+    dims = scan_dims_for(u, delta, B, C, z, dout)
+    ws_bytes = 0 if ckpt is not None else mamba_scan_bwd_workspace_size(dims)
+    if workspace is not None:
+        ws, ws_bytes = workspace, workspace.numel() * workspace.element_size()
+    else:
+        ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev) if ws_bytes else None
+    rc = mamba_scan_bwd(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z), _ptr(delta_bias),
+                        softplus, _ptr(initial_state), _ptr(ckpt), _ptr(dout), _ptr(dlast), _ptr(g["du"]),
+                        _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]), _ptr(g["dD"]),
+                        _ptr(g["dz"]), _ptr(g["ddelta_bias"]), _ptr(g["dinitial_state"]), dims, _ptr(ws),
+                        ws_bytes, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_scan_bwd")
+    return g
 
 
 def update_dims_for(state, x, delta, B, C, z, y) -> UpdateDims:

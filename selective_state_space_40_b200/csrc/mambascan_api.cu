@@ -9,6 +9,8 @@
 #include "mambascan.h"
 #include "ms_internal.h"
 
+static_assert(MS_CKPT_TOKENS == ms::kCkptTokens, "saved-state interval of the ABI and the kernels");
+
 namespace {
 
 bool aligned(const void *p, size_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
@@ -175,8 +177,10 @@ static int check_conv(const ConvIn &cv, const ms_scan_dims *dm) {
 static int scan_common(const void *u, const void *delta, const float *A, const void *B, const void *C,
                        const float *D, const void *z, const float *delta_bias, int softplus_flag,
                        const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
-                       int *dev_status, ms_stream_t stream, const ms_scan_plan *plan, const ConvIn *cv) {
+                       int *dev_status, ms_stream_t stream, const ms_scan_plan *plan, const ConvIn *cv,
+                       float *ckpt = nullptr) {
     ms::ScanArgs a{};
+    a.ckpt = ckpt;
     a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
     a.A = A; a.D = D; a.bias = delta_bias; a.h0 = initial_state;
     a.y = y; a.last = last_state; a.status = dev_status;
@@ -251,6 +255,88 @@ int mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
     if (dims->seqlen == 0 && !last_state) return MS_OK;
     return scan_common(x, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
                        dims, dev_status, stream, plan, &cv);
+}
+
+size_t mamba_scan_ckpt_size(const ms_scan_dims *dims) {
+    if (!dims || dims->batch <= 0 || dims->dim <= 0 || dims->seqlen <= 0 || dims->dstate <= 0) return 0;
+    const int64_t nck = (dims->seqlen + ms::kCkptTokens - 1) / ms::kCkptTokens;
+    return (size_t)dims->batch * (size_t)dims->dim * (size_t)nck * (size_t)dims->dstate * sizeof(float);
+}
+
+int mamba_scan_fwd_train(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                         const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                         const float *initial_state, void *y, float *last_state, float *ckpt,
+                         const ms_scan_dims *dims, int *dev_status, ms_stream_t stream) {
+    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
+    if (rc != MS_OK) return rc;
+    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
+    if (dims->seqlen > 0 && !ckpt) return MS_ERR_NULL;
+    if (ckpt && !aligned(ckpt, 4)) return MS_ERR_ALIGN;
+    if (dims->seqlen == 0 && !last_state) return MS_OK;
+    return scan_common(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
+                       dims, dev_status, stream, nullptr, nullptr, ckpt);
+}
+
+size_t mamba_scan_bwd_workspace_size(const ms_scan_dims *dims) { return mamba_scan_ckpt_size(dims); }
+
+int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                   const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                   const float *initial_state, const float *ckpt, const void *dout, const float *dlast,
+                   float *du, float *ddelta, float *dA, float *dB, float *dC, float *dD, float *dz,
+                   float *ddelta_bias, float *dinitial_state, const ms_scan_dims *dims, void *workspace,
+                   size_t workspace_bytes, int *dev_status, ms_stream_t stream) {
+    // dout takes y's place in the forward checks (its dtype and strides).
+    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, const_cast<void *>(dout), nullptr,
+                        dims);
+    if (rc != MS_OK) return rc;
+    const int64_t nb = dims->batch, nd = dims->dim, N = dims->dstate, L = dims->seqlen;
+    if (nb == 0 || nd == 0) return MS_OK;
+    if (!dA || (L > 0 && (!du || !ddelta || !dB || !dC))) return MS_ERR_NULL;
+    const float *outs[] = {du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dinitial_state, ckpt, dlast};
+    for (const float *p : outs)
+        if (p && !aligned(p, 4)) return MS_ERR_ALIGN;
+    if (max_offset3(nb, nd * L, nd, L, L > 0 ? L : 1) < 0 || max_offset3(nb, N * L, N, L, L > 0 ? L : 1) < 0)
+        return MS_ERR_SHAPE;
+    const size_t ck_bytes = mamba_scan_ckpt_size(dims);
+    if (!ckpt && L > 0 && (workspace_bytes < ck_bytes || !workspace)) return MS_ERR_WORKSPACE;
+    if (!ckpt && L > 0 && !aligned(workspace, 4)) return MS_ERR_ALIGN;
+
+    const cudaStream_t st = (cudaStream_t)stream;
+    // sums are accumulated: start from zero
+    const size_t fl = sizeof(float);
+    cudaError_t e = cudaMemsetAsync(dA, 0, (size_t)(nd * N) * fl, st);
+    if (e == cudaSuccess && L > 0) e = cudaMemsetAsync(dB, 0, (size_t)(nb * N * L) * fl, st);
+    if (e == cudaSuccess && L > 0) e = cudaMemsetAsync(dC, 0, (size_t)(nb * N * L) * fl, st);
+    if (e == cudaSuccess && dD) e = cudaMemsetAsync(dD, 0, (size_t)nd * fl, st);
+    if (e == cudaSuccess && ddelta_bias) e = cudaMemsetAsync(ddelta_bias, 0, (size_t)nd * fl, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    if (L > 0 && !ckpt) {
+        // recompute the saved states: the forward without y
+        float *wck = static_cast<float *>(workspace);
+        rc = scan_common(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, nullptr, nullptr,
+                         dims, dev_status, stream, nullptr, nullptr, wck);
+        if (rc != MS_OK) return rc;
+        ckpt = wck;
+    }
+    ms::BwdArgs a{};
+    a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
+    a.A = A; a.D = D; a.bias = delta_bias; a.ckpt = ckpt; a.dlast = dlast; a.dout = dout;
+    a.du = du; a.ddelta = ddelta; a.dz = z ? dz : nullptr; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD;
+    a.dbias = ddelta_bias; a.dh0 = dinitial_state;
+    a.batch = nb; a.dim = nd; a.L = L; a.N = (int)N;
+    a.u_sb = dims->u_sb; a.u_sd = dims->u_sd; a.dl_sb = dims->delta_sb; a.dl_sd = dims->delta_sd;
+    a.z_sb = dims->z_sb; a.z_sd = dims->z_sd; a.y_sb = dims->y_sb; a.y_sd = dims->y_sd;
+    a.B_sb = dims->B_sb; a.B_sn = dims->B_sn; a.C_sb = dims->C_sb; a.C_sn = dims->C_sn;
+    a.softplus = softplus_flag ? 1 : 0;
+    e = ms::launch_scan_bwd(a, dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, st);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
 }
 
 int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,

@@ -29,6 +29,26 @@ struct ScanArgs {
     int conv_width;                // 1..4
     int conv_silu;
     int vec_uout;                  // u_out rows 16-byte aligned
+    // Training: the state before every kCkptTokens-token block, [batch, dim,
+    // ceil(L / kCkptTokens), N] fp32 (null: not written). y may be null then.
+    float *ckpt;
+};
+
+// Tokens between two saved states of the forward (the backward recomputes
+// each block from its saved state).
+constexpr int kCkptTokens = 64;
+
+// Arguments of the backward kernel (gradients are fp32, dense).
+struct BwdArgs {
+    const void *u, *delta, *z, *B, *C;  // input dtype
+    const float *A, *D, *bias, *ckpt, *dlast;
+    const void *dout;                   // output dtype, strides y_sb / y_sd
+    float *du, *ddelta, *dz, *dA, *dB, *dC, *dD, *dbias, *dh0;
+    int64_t batch, dim, L;
+    int N;
+    int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, y_sb, y_sd;
+    int64_t B_sb, B_sn, C_sb, C_sn;
+    int softplus;
 };
 
 // Launch shape chosen on the host for one scan call.
@@ -63,6 +83,8 @@ cudaError_t launch_state_update(const UpdateArgs &a, bool in_bf16, bool out_bf16
 // multiple of 128, 16-byte aligned rows).
 bool state_update_stream_applies(const UpdateArgs &a, int in_bytes, int out_bytes);
 cudaError_t launch_state_update_stream(const UpdateArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
+
+cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
 
 // Plan for a call (host heuristic from sizes and dtypes).
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms);

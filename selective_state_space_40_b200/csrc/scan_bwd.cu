@@ -1,0 +1,353 @@
+// scan_bwd.cu -- gradients of the selective scan on sm_100a.
+//
+// Reverse mode of the forward recurrence ('Mamba (deep learning)' wiki page,
+// state-space paragraph: A_bar = exp(Delta*A); 'Mamba-1/2/3 Markdown図解'
+// blog, section 1: h_t = A_bar_t h_{t-1} + B_bar_t x_t, y_t = C_t h_t;
+// section 2: the same model is trained through the scan). With q_t the
+// pre-gate output and lam the adjoint of h_t, per channel from the last token
+// back:
+//   dq_t = dout_t silu(z_t), dz_t = dout_t q_t silu'(z_t)
+//   lam = C_t dq_t + A_bar_{t+1} lam_{t+1}          (dL/dlast_state at the end)
+//   dA += lam h_{t-1} A_bar_t Delta_t,  dDelta_t = sum_n lam (h_{t-1} A_bar_t A + u_t B_t)
+//   du_t = D dq_t + sum_n lam Delta_t B_t,  dB_t += lam Delta_t u_t,  dC_t += dq_t h_t
+//   ddelta_t = dDelta_t softplus'(delta_t + bias)
+//
+// The forward saved the state before every 64-token block. This kernel walks
+// the blocks from the last: it recomputes the block forward from its saved
+// state, keeping the state at every 8-token boundary in shared memory; then
+// for each 8-token sub-chunk from the last it recomputes A_bar and h into
+// registers and runs the adjoint back over those 8 tokens. Work split as in
+// the forward: 4 lanes per channel, 4 states each; a CTA holds 32 channels of
+// one batch row. B_t and C_t of the block are staged once per CTA as fp32
+// token rows. Sums over channels (dB, dC) are reduced within the warp by
+// reduce-scatter shuffles, across the CTA's warps in shared memory, then
+// added to global memory with fp32 atomics (run-to-run order of those adds
+// varies, so dB/dC/dA/dD/dbias can differ in the last bits between runs).
+
+#include "ms_device.cuh"
+#include "ms_internal.h"
+
+namespace ms {
+
+namespace {
+
+constexpr int kBNW = 4;                  // warps per CTA
+constexpr int kBThreads = kBNW * 32;
+constexpr int kG = 4;                    // lanes per channel
+constexpr int kCW = 32 / kG;             // channels per warp
+constexpr int kBCh = kBNW * kCW;         // channels per CTA
+constexpr int kBlk = kCkptTokens;        // tokens per saved-state block
+constexpr int kSub = 8;                  // tokens per sub-chunk
+constexpr int kNSub = kBlk / kSub;
+static_assert(kBlk % kSub == 0, "whole sub-chunks per block");
+static_assert(2 * kBlk <= kBThreads, "one staging thread per B/C row");
+
+struct BwdSmem {
+    float bc[kBlk][36];               // token rows: B[0..15], C[16..31], pad
+    float sub[kBNW][kNSub][4][32];    // state at each sub-chunk start [warp][s][state][lane]
+    float red[kBNW][kSub][32];        // warp sums of dB/dC per token [warp][j][value]
+};
+
+template <typename T>
+__device__ __forceinline__ float ld_elem(const T *p) {
+    if constexpr (sizeof(T) == 4) return __ldg(reinterpret_cast<const float *>(p));
+    else return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)));
+}
+
+// 8 tokens [t, t+8) of a row as fp32 (0 past L), read through the read-only
+// cache (the 4 lanes of a channel read the same chunk).
+template <typename T>
+__device__ __forceinline__ void load8(const T *row, int64_t t, int64_t L, float (&v)[8]) {
+#pragma unroll
+    for (int j = 0; j < 8; ++j) v[j] = (t + j < L) ? ld_elem(row + t + j) : 0.0f;
+}
+
+// Reduce-scatter of v[0..8) over the 8 channel lanes of a warp (lane bits 2..4):
+// afterwards lane (c, g) holds the sum over channels of v[c].
+__device__ __forceinline__ float reduce_scatter_channels(float (&v)[8], int c) {
+    // step over lane bit 4 (channel bit 2): keep half 4*c2 .. 4*c2+3
+    const bool u2 = (c & 4) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = u2 ? v[i] : v[i + 4];
+        const float keep = u2 ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 16);
+    }
+    const bool u1 = (c & 2) != 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = u1 ? v[i] : v[i + 2];
+        const float keep = u1 ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 8);
+    }
+    const bool u0 = (c & 1) != 0;
+    const float send = u0 ? v[0] : v[1];
+    const float keep = u0 ? v[1] : v[0];
+    return keep + __shfl_xor_sync(0xffffffffu, send, 4);
+}
+
+// Reduce-scatter of v[0..8) over the 4 lanes of a channel (lane bits 0..1):
+// afterwards lane g holds the sums of tokens 2g and 2g+1 in v[0], v[1].
+__device__ __forceinline__ void reduce_scatter_lanes(float (&v)[8], int g) {
+    const bool u1 = (g & 2) != 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const float send = u1 ? v[i] : v[i + 4];
+        const float keep = u1 ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 2);
+    }
+    const bool u0 = (g & 1) != 0;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const float send = u0 ? v[i] : v[i + 2];
+        const float keep = u0 ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(0xffffffffu, send, 1);
+    }
+}
+
+// Softplus and its derivative (the logistic function) from one exponential.
+__device__ __forceinline__ void softplus_and_grad(float v, float &sp, float &sig) {
+    sp = softplus_f(v);
+    const float e = exp2_mufu(-fabsf(v) * kLog2e);  // e^{-|v|}
+    const float r = rcp_mufu(1.0f + e);
+    sig = v >= 0.0f ? r : e * r;
+}
+
+template <typename TIn, typename TOut>
+__global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a) {
+    __shared__ __align__(16) BwdSmem sm;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int c = lane / kG, g = lane % kG;
+    const int64_t dblocks = (a.dim + kBCh - 1) / kBCh;
+    const int64_t b = blockIdx.x / dblocks;
+    const int64_t d = (blockIdx.x % dblocks) * kBCh + warp * kCW + c;
+    const bool active = d < a.dim;
+    const int64_t dd = active ? d : 0;
+    const int N = a.N;
+    const int64_t L = a.L;
+    const int n0 = g * 4;
+
+    float A2[4], An[4], carry[4], dAacc[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int n = n0 + i;
+        An[i] = n < N ? __ldg(a.A + dd * N + n) : 0.0f;
+        A2[i] = An[i] * kLog2e;
+        carry[i] = (a.dlast != nullptr && active && n < N) ? __ldg(a.dlast + (b * a.dim + d) * N + n) : 0.0f;
+        dAacc[i] = 0.0f;
+    }
+    const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
+    const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
+    const bool has_z = a.z != nullptr;
+    const bool sp = a.softplus != 0;
+    float dDacc = 0.0f, dbacc = 0.0f;
+
+    const TIn *u_row = static_cast<const TIn *>(a.u) + b * a.u_sb + dd * a.u_sd;
+    const TIn *d_row = static_cast<const TIn *>(a.delta) + b * a.dl_sb + dd * a.dl_sd;
+    const TIn *z_row = has_z ? static_cast<const TIn *>(a.z) + b * a.z_sb + dd * a.z_sd : nullptr;
+    const TOut *o_row = static_cast<const TOut *>(a.dout) + b * a.y_sb + dd * a.y_sd;
+    const TIn *B_b = static_cast<const TIn *>(a.B) + b * a.B_sb;
+    const TIn *C_b = static_cast<const TIn *>(a.C) + b * a.C_sb;
+    const int64_t grow = (b * a.dim + dd) * L;  // dense gradient row
+
+    const int64_t nblk = (L + kBlk - 1) / kBlk;
+    for (int64_t kb = nblk - 1; kb >= 0; --kb) {
+        const int64_t tb = kb * kBlk;
+
+        // ---- stage B and C of the block as fp32 token rows
+        __syncthreads();
+        if (threadIdx.x < 2 * kBlk) {
+            const int r = threadIdx.x;
+            const bool isC = r >= kBlk;
+            const int64_t t = tb + (r % kBlk);
+            const TIn *base = (isC ? C_b : B_b) + t;
+            const int64_t sn = isC ? a.C_sn : a.B_sn;
+            float *row = &sm.bc[r % kBlk][isC ? 16 : 0];
+#pragma unroll
+            for (int n = 0; n < 16; ++n) row[n] = (n < N && t < L) ? ld_elem(base + n * sn) : 0.0f;
+        }
+        __syncthreads();
+
+        // ---- pass A: the block forward from its saved state; keep the state
+        // at every sub-chunk start.
+        float h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            h[i] = (active && n0 + i < N) ? __ldg(a.ckpt + ((b * a.dim + d) * nblk + kb) * N + n0 + i) : 0.0f;
+        for (int s = 0; s < kNSub; ++s) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) sm.sub[warp][s][i][lane] = h[i];
+            const int64_t ts = tb + s * kSub;
+            float uv[8], dv[8];
+            load8(u_row, ts, L, uv);
+            load8(d_row, ts, L, dv);
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                const float v = dv[j] + bias;
+                const float dl = (ts + j < L) ? (sp ? softplus_f(v) : v) : 0.0f;
+                const float du = dl * uv[j];
+                const float *bcr = sm.bc[s * kSub + j];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) h[i] = fmaf(exp2_mufu(dl * A2[i]), h[i], du * bcr[n0 + i]);
+            }
+        }
+
+        // ---- sub-chunks from the last: recompute, then the adjoint
+        for (int s = kNSub - 1; s >= 0; --s) {
+            const int64_t ts = tb + s * kSub;
+            float uv[8], dv[8], zv[8], ov[8];
+            load8(u_row, ts, L, uv);
+            load8(d_row, ts, L, dv);
+            if (has_z) load8(z_row, ts, L, zv);
+            // an idle lane (channel past dim) gets dout = 0: with its zero
+            // starting adjoint every contribution to the channel sums is 0
+            if (active) load8(o_row, ts, L, ov);
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) ov[j] = active ? ov[j] : 0.0f;
+            float dl[8], sig[8], gate[8], gprime[8];
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                const float v = dv[j] + bias;
+                float spv = v, sgv = 1.0f;
+                if (sp) softplus_and_grad(v, spv, sgv);
+                const bool in = ts + j < L;
+                dl[j] = in ? spv : 0.0f;
+                sig[j] = sgv;
+                if (has_z) {
+                    const float zz = zv[j];
+                    const float sz = rcp_mufu(1.0f + exp2_mufu(-zz * kLog2e));
+                    gate[j] = zz * sz;
+                    gprime[j] = sz * (1.0f + zz * (1.0f - sz));
+                } else {
+                    gate[j] = 1.0f;
+                    gprime[j] = 0.0f;
+                }
+            }
+            // recompute A_bar and h of the sub-chunk, and the pre-gate output q
+            float hs[4], ab[kSub][4], hh[kSub][4], dq[kSub], dzv[kSub];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) hs[i] = sm.sub[warp][s][i][lane];
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                const float du = dl[j] * uv[j];
+                const float *bcr = sm.bc[s * kSub + j];
+                float part = 0.0f;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ab[j][i] = exp2_mufu(dl[j] * A2[i]);
+                    const float hp = j == 0 ? hs[i] : hh[j - 1][i];
+                    hh[j][i] = fmaf(ab[j][i], hp, du * bcr[n0 + i]);
+                    part = fmaf(bcr[16 + n0 + i], hh[j][i], part);
+                }
+                part += __shfl_xor_sync(0xffffffffu, part, 1);
+                part += __shfl_xor_sync(0xffffffffu, part, 2);
+                const float q = part + Dd * uv[j];
+                dq[j] = ov[j] * gate[j];
+                dzv[j] = ov[j] * q * gprime[j];
+            }
+            // adjoint over the sub-chunk, last token first
+            float ddt[kSub], dus[kSub];
+#pragma unroll
+            for (int j = kSub - 1; j >= 0; --j) {
+                const float dqj = dq[j];
+                const float *bcr = sm.bc[s * kSub + j];
+                const float du = dl[j] * uv[j];
+                float pdt = 0.0f, pdu = 0.0f, v8[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float Bn = bcr[n0 + i], Cn = bcr[16 + n0 + i];
+                    const float lam = fmaf(Cn, dqj, carry[i]);
+                    const float hp = j == 0 ? hs[i] : hh[j - 1][i];
+                    const float dab = lam * hp * ab[j][i];
+                    dAacc[i] = fmaf(dab, dl[j], dAacc[i]);
+                    pdt = fmaf(dab, An[i], pdt);
+                    pdt = fmaf(lam * Bn, uv[j], pdt);
+                    pdu = fmaf(lam * Bn, dl[j], pdu);
+                    v8[i] = lam * du;          // dB
+                    v8[4 + i] = dqj * hh[j][i]; // dC
+                    carry[i] = ab[j][i] * lam;
+                }
+                ddt[j] = pdt;
+                dus[j] = pdu;
+                sm.red[warp][j][lane] = reduce_scatter_channels(v8, c);
+            }
+            // per-token sums over the channel's 4 lanes; lane g owns tokens 2g, 2g+1
+            reduce_scatter_lanes(ddt, g);
+            reduce_scatter_lanes(dus, g);
+#pragma unroll
+            for (int j = 0; j < kSub; ++j) {
+                // compile-time indices; the lane owning token j acts
+                const int k = j & 1;
+                const int64_t t = ts + j;
+                if ((j >> 1) == g && active && t < L) {
+                    const float ddv = sp ? ddt[k] * sig[j] : ddt[k];
+                    a.ddelta[grow + t] = ddv;
+                    a.du[grow + t] = fmaf(Dd, dq[j], dus[k]);
+                    if (has_z && a.dz != nullptr) a.dz[grow + t] = dzv[j];
+                    dDacc = fmaf(dq[j], uv[j], dDacc);
+                    dbacc += ddv;
+                }
+            }
+            // dB / dC: sum the warps' partial sums, then one atomic per output
+            __syncthreads();
+            {
+                const int col = threadIdx.x & 31;        // value column: lane that held it
+                const int jp = threadIdx.x >> 5;         // token pair
+                const int cg = col / kG, gg = col % kG;  // channel slot -> value, lane group -> states
+                const bool isC = cg >= 4;
+                const int n = gg * 4 + (cg & 3);
+#pragma unroll
+                for (int k = 0; k < 2; ++k) {
+                    const int j = 2 * jp + k;
+                    const int64_t t = ts + j;
+                    float sum = 0.0f;
+#pragma unroll
+                    for (int w = 0; w < kBNW; ++w) sum += sm.red[w][j][col];
+                    if (n < N && t < L) atomicAdd((isC ? a.dC : a.dB) + (b * N + n) * L + t, sum);
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    // ---- per-channel results
+    if (active) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const int n = n0 + i;
+            if (n < N) {
+                if (a.dh0 != nullptr) a.dh0[(b * a.dim + d) * N + n] = carry[i];
+                atomicAdd(a.dA + d * N + n, dAacc[i]);
+            }
+        }
+    }
+    dDacc += __shfl_xor_sync(0xffffffffu, dDacc, 1);
+    dDacc += __shfl_xor_sync(0xffffffffu, dDacc, 2);
+    dbacc += __shfl_xor_sync(0xffffffffu, dbacc, 1);
+    dbacc += __shfl_xor_sync(0xffffffffu, dbacc, 2);
+    if (active && g == 0) {
+        if (a.dD != nullptr) atomicAdd(a.dD + d, dDacc);
+        if (a.dbias != nullptr) atomicAdd(a.dbias + d, dbacc);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream) {
+    const int64_t dblocks = (a.dim + kBCh - 1) / kBCh;
+    const int64_t blocks = dblocks * a.batch;
+    if (blocks <= 0) return cudaSuccess;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const unsigned grid = (unsigned)blocks;
+    if (in_bf16) {
+        if (out_bf16) scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kBThreads, 0, stream>>>(a);
+        else scan_bwd_kernel<__nv_bfloat16, float><<<grid, kBThreads, 0, stream>>>(a);
+    } else {
+        if (out_bf16) scan_bwd_kernel<float, __nv_bfloat16><<<grid, kBThreads, 0, stream>>>(a);
+        else scan_bwd_kernel<float, float><<<grid, kBThreads, 0, stream>>>(a);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace ms

@@ -250,6 +250,7 @@ template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV>
 __global__ void __launch_bounds__(kThreads, CH == 1 ? MS_SCAN_MINB : 1)
 scan_fwd_kernel(const ScanArgs a) {
     static_assert(!CONV || CH == 1, "the conv front-end runs with one chunk per lane");
+    static_assert(kCkptTokens % Geom<G, CH>::kTT == 0, "saved states fall on tile starts");
     using Gm = Geom<G, CH>;
     constexpr int TT = Gm::kTT;
     constexpr int S = Gm::kStates;
@@ -368,9 +369,22 @@ scan_fwd_kernel(const ScanArgs a) {
 
     if (ntiles > 0) prefetch(0);
 
+    const int64_t nck = (L + kCkptTokens - 1) / kCkptTokens;
     for (int64_t k = 0; k < ntiles; ++k) {
         const int64_t t0 = k * TT;
         const int buf = (int)(k & 1);
+        if (a.ckpt != nullptr && active && t0 % kCkptTokens == 0) {
+            // Training: the state before this block, for the backward's recompute.
+            float *cs = a.ckpt + ((b * a.dim + d) * nck + t0 / kCkptTokens) * N;
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+                float ha, hb;
+                f2_split(h[p], ha, hb);
+                const int na = n0 + 2 * p;
+                if (na < N) cs[na] = ha;
+                if (na + 1 < N) cs[na + 1] = hb;
+            }
+        }
 
         // ---- prologue: per-token quantities of this lane's chunks.
         float dl[CH][8], dlu[CH][8], dug[CH][8], gate[CH][8];
@@ -455,7 +469,7 @@ scan_fwd_kernel(const ScanArgs a) {
                                                                         j * P);
                     yo[j] = fmaf(yv, gate[i][j], dug[i][j]);
                 }
-                if (active) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
+                if (active && a.y != nullptr) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
             }
         } else {
             __syncwarp();
@@ -520,7 +534,7 @@ scan_fwd_kernel(const ScanArgs a) {
                 float yo[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) yo[j] = fmaf(ys[j], gate[i][j], dug[i][j]);
-                if (active) store8<TOut>(y_row, t0 + off, L, vout, yo);
+                if (active && a.y != nullptr) store8<TOut>(y_row, t0 + off, L, vout, yo);
             }
             __syncwarp();
         }

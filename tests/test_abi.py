@@ -157,6 +157,35 @@ def test_conv_scan_empty_is_a_noop(lib):
     assert _conv(_dims(dim=0), w=None, x=None, y=None) == mb.MS_OK
 
 
+def _bwd(dims, ckpt=FAKE, dout=FAKE, du=FAKE, ddelta=FAKE, dA=FAKE, dB=FAKE, dC=FAKE, ws=None, ws_bytes=0):
+    return mb.mamba_scan_bwd(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, ckpt, dout, None,
+                             du, ddelta, dA, dB, dC, None, None, None, None, dims, ws, ws_bytes, None, None)
+
+
+def test_scan_bwd_rejects_bad_arguments(lib):
+    assert _bwd(_dims(dstate=17)) == mb.MS_ERR_SHAPE
+    assert _bwd(_dims(in_dtype=5)) == mb.MS_ERR_DTYPE
+    assert _bwd(_dims(), dout=None) == mb.MS_ERR_NULL
+    assert _bwd(_dims(), dA=None) == mb.MS_ERR_NULL
+    assert _bwd(_dims(), dB=None) == mb.MS_ERR_NULL
+    assert _bwd(_dims(), du=FAKE + 2) == mb.MS_ERR_ALIGN
+    assert _bwd(_dims(), ckpt=FAKE + 1) == mb.MS_ERR_ALIGN
+    # no saved states and no workspace for recomputing them
+    assert _bwd(_dims(), ckpt=None) == mb.MS_ERR_WORKSPACE
+    assert _bwd(_dims(), ckpt=None, ws=FAKE, ws_bytes=16) == mb.MS_ERR_WORKSPACE
+    assert _bwd(_dims(batch=0)) == mb.MS_OK
+
+
+def test_ckpt_sizes(lib):
+    d = _dims(batch=2, dim=8, dstate=16, seqlen=130)
+    assert mb.mamba_scan_ckpt_size(d) == 2 * 8 * 3 * 16 * 4
+    assert mb.mamba_scan_bwd_workspace_size(d) == mb.mamba_scan_ckpt_size(d)
+    assert mb.mamba_scan_ckpt_size(_dims(seqlen=0)) == 0
+    rc = mb.mamba_scan_fwd_train(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, FAKE, None, None,
+                                 _dims(), None, None)
+    assert rc == mb.MS_ERR_NULL  # training forward without its saved-state array
+
+
 def _udims(**kw):
     d = dict(batch=4, dim=8, dstate=16, x_sb=8, delta_sb=8, z_sb=8, y_sb=8, B_sb=16, C_sb=16,
              state_sb=128, state_sd=16, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)

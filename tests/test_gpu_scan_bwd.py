@@ -1,0 +1,178 @@
+"""GPU parity of the scan's training forward (saved states) and backward
+(mamba_scan_fwd_train, mamba_scan_bwd) against the fp64 oracle's gradients,
+through the C ABI.
+
+Tolerances are the forward's (tests/parity_util.py) applied to every gradient
+tensor separately: the oracle is fed the same stored input values, so the
+differences come only from fp32 arithmetic, the fast exponential and the
+order of the fp32 atomic sums.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from selective_state_space_40_b200 import binding as mb
+from selective_state_space_40_b200 import synthetic as syn
+from parity_util import check, f64
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+GRADS = ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    assert mb.mamba_device_check() == mb.MS_OK
+    mb.library()
+
+
+def _grads_inputs(w, seed, out_dtype=torch.float32, with_dlast=True, with_h0=False):
+    inp = syn.scan_inputs(w)
+    g = torch.Generator().manual_seed(seed)
+    dout = torch.randn(w.batch, w.dim, w.seqlen, generator=g).to(out_dtype)
+    dlast = torch.randn(w.batch, w.dim, w.dstate, generator=g) if with_dlast else None
+    h0 = 0.3 * torch.randn(w.batch, w.dim, w.dstate, generator=g) if with_h0 else None
+    return inp, dout, dlast, h0
+
+
+def run_gpu(inp, dout, dlast, h0, use_ckpt=True, use_z=True, use_D=True, use_bias=True, softplus=True):
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    D = g["D"] if use_D else None
+    z = g["z"] if use_z else None
+    bias = g["delta_bias"] if use_bias else None
+    h0d = None if h0 is None else h0.to(DEV)
+    ckpt = None
+    if use_ckpt:
+        _, _, ckpt = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], D, z, bias, softplus,
+                                       initial_state=h0d, out_dtype=dout.dtype)
+    return mb.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], D, z, bias, softplus, dout.to(DEV),
+                       dlast=None if dlast is None else dlast.to(DEV), initial_state=h0d, ckpt=ckpt)
+
+
+def run_oracle(inp, dout, dlast, h0, use_z=True, use_D=True, use_bias=True, softplus=True):
+    return oracle.scan_bwd(f64(inp["u"]), f64(inp["delta"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
+                           f64(inp["D"]) if use_D else None, f64(inp["z"]) if use_z else None,
+                           f64(inp["delta_bias"]) if use_bias else None, softplus, f64(dout),
+                           h0=None if h0 is None else f64(h0), dlast=None if dlast is None else f64(dlast))
+
+
+def compare(gg, rr, dtype, what):
+    torch.cuda.synchronize()
+    for k in GRADS:
+        if rr[k] is None:
+            assert gg[k] is None, f"{what}: {k} returned for a missing input"
+            continue
+        check(f64(gg[k]), rr[k], dtype, f"{what} {k}")
+    if gg["dinitial_state"] is not None:
+        check(f64(gg["dinitial_state"]), rr["dh0"], dtype, f"{what} dinitial_state")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("L", [1, 8, 63, 64, 65, 200])
+def test_lengths(dtype, L):
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=L, in_dtype=dtype, seed=100 + L)
+    inp, dout, dlast, h0 = _grads_inputs(w, 7 + L, with_h0=(L % 2 == 1))
+    compare(run_gpu(inp, dout, dlast, h0), run_oracle(inp, dout, dlast, h0), dtype, f"L={L} {dtype}")
+
+
+@pytest.mark.parametrize("N", [1, 4, 5, 16])
+def test_dstate(N):
+    w = syn.scaled(syn.M130, batch=2, dim=36, seqlen=130, dstate=N, in_dtype=torch.float32, seed=200 + N)
+    inp, dout, dlast, h0 = _grads_inputs(w, 11, with_h0=True)
+    compare(run_gpu(inp, dout, dlast, h0), run_oracle(inp, dout, dlast, h0), torch.float32, f"N={N}")
+
+
+@pytest.mark.parametrize("flags", [dict(use_z=False), dict(use_D=False), dict(use_bias=False),
+                                   dict(softplus=False)])
+def test_optional_inputs(flags):
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=150, in_dtype=torch.float32, seed=300)
+    inp, dout, dlast, h0 = _grads_inputs(w, 13)
+    if flags.get("softplus") is False:
+        inp["delta"] = (0.05 * torch.rand(inp["delta"].shape)).to(inp["delta"].dtype)  # positive steps
+        inp["delta_bias"] = torch.zeros_like(inp["delta_bias"])
+    compare(run_gpu(inp, dout, dlast, h0, **flags), run_oracle(inp, dout, dlast, h0, **flags),
+            torch.float32, f"{flags}")
+
+
+def test_bf16_dout():
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=100, in_dtype=torch.bfloat16, seed=400)
+    inp, dout, dlast, h0 = _grads_inputs(w, 17, out_dtype=torch.bfloat16)
+    compare(run_gpu(inp, dout, dlast, h0), run_oracle(inp, dout, dlast, h0), torch.bfloat16, "bf16 dout")
+
+
+def test_recomputed_states_match_saved():
+    """No saved states: the backward recomputes them into its workspace; the
+    directly written gradients are then bit-identical, and the training
+    forward's y is the plain forward's."""
+    w = syn.scaled(syn.M130, batch=3, dim=64, seqlen=333, in_dtype=torch.bfloat16, seed=500)
+    inp, dout, dlast, h0 = _grads_inputs(w, 19, with_h0=True)
+    g1 = run_gpu(inp, dout, dlast, h0, use_ckpt=True)
+    g2 = run_gpu(inp, dout, dlast, h0, use_ckpt=False)
+    torch.cuda.synchronize()
+    for k in ("du", "ddelta", "dz", "dinitial_state"):
+        assert torch.equal(g1[k], g2[k]), k
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    y1, l1, _ = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                  True, initial_state=h0.to(DEV))
+    y0, l0 = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                         initial_state=h0.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(y1, y0) and torch.equal(l1, l0)
+
+
+def test_saved_states_are_block_states():
+    """ckpt[:, :, k] is the state before token 64 k (the oracle's last_state
+    of the prefix)."""
+    w = syn.scaled(syn.M130, batch=2, dim=24, seqlen=200, in_dtype=torch.float32, seed=600)
+    inp = syn.scan_inputs(w)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    _, _, ck = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                 True)
+    torch.cuda.synchronize()
+    assert ck.shape == (2, 24, 4, 16)
+    assert float(ck[:, :, 0].abs().max()) == 0.0
+    for k in (1, 2, 3):
+        t = 64 * k
+        pre = {n: (v[:, :, :t] if n in ("u", "delta", "z", "B", "C") else v) for n, v in inp.items()}
+        _, lr = oracle.scan(f64(pre["u"]), f64(pre["delta"]), f64(pre["A"]), f64(pre["B"]), f64(pre["C"]),
+                            f64(pre["D"]), f64(pre["z"]), f64(pre["delta_bias"]), True)
+        check(f64(ck[:, :, k]), lr, torch.float32, f"saved state {k}")
+
+
+def test_no_dinitial_requested():
+    w = syn.scaled(syn.M130, batch=1, dim=32, seqlen=70, in_dtype=torch.float32, seed=700)
+    inp, dout, dlast, h0 = _grads_inputs(w, 23)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    out = mb.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                      dout.to(DEV), dlast=dlast.to(DEV), want_dinitial=False)
+    compare(out, run_oracle(inp, dout, dlast, None), torch.float32, "no dinitial")
+
+
+@pytest.mark.slow
+def test_full_130m_batch_row_and_channel_sums():
+    """130M-class layer at full size: one whole batch row is recomputed by the
+    oracle (every per-token gradient of that row and dB, dC, which sum over
+    all its channels); dA, dD, ddelta_bias (sums over batch rows and tokens)
+    on a seeded sample of channels over all batch rows."""
+    w = syn.M130
+    inp, dout, dlast, h0 = _grads_inputs(w, 29)
+    gg = run_gpu(inp, dout, dlast, h0)
+    torch.cuda.synchronize()
+    br = 5
+    row = {k: (v[br:br + 1] if k in ("u", "delta", "z", "B", "C") else v) for k, v in inp.items()}
+    rr = run_oracle(row, dout[br:br + 1], dlast[br:br + 1], None)
+    for k in ("du", "ddelta", "dz", "dB", "dC"):
+        check(f64(gg[k][br:br + 1]), rr[k], w.in_dtype, f"130M row {br} {k}")
+    check(f64(gg["dinitial_state"][br:br + 1]), rr["dh0"], w.in_dtype, f"130M row {br} dinitial_state")
+    ds = np.sort(np.random.default_rng(3).choice(w.dim, 16, replace=False))
+    idx = torch.as_tensor(ds)
+    sub = {k: (v[:, idx] if k in ("u", "delta", "z") else (v[idx] if k in ("A", "D", "delta_bias") else v))
+           for k, v in inp.items()}
+    rs = run_oracle(sub, dout[:, idx], dlast[:, idx], None)
+    check(f64(gg["dA"][idx]), rs["dA"], w.in_dtype, "130M dA (sampled channels)")
+    check(f64(gg["dD"][idx]), rs["dD"], w.in_dtype, "130M dD (sampled channels)")
+    check(f64(gg["ddelta_bias"][idx]), rs["ddelta_bias"], w.in_dtype, "130M ddelta_bias (sampled channels)")

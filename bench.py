@@ -53,6 +53,17 @@ def decode_bytes(batch, dim, dstate, in_bytes, out_bytes):
             + batch * dstate * 2 * in_bytes + dim * dstate * 4 + 2 * dim * 4)
 
 
+def bwd_bytes(batch, dim, dstate, seqlen, in_bytes, out_bytes):
+    """Minimum HBM bytes of one backward: u, delta, z and dout read and du,
+    ddelta, dz (fp32) written per channel-token; B, C read and dB, dC (fp32)
+    written per (batch, token); the saved states read; A, D, bias read and
+    their gradients and dinitial_state written."""
+    ct = batch * dim * seqlen
+    nck = (seqlen + 63) // 64
+    return (ct * (3 * in_bytes + out_bytes + 3 * 4) + batch * seqlen * 2 * dstate * (in_bytes + 4)
+            + batch * dim * nck * dstate * 4 + batch * dim * dstate * 4 + 2 * (dim * dstate * 4 + 2 * dim * 4))
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -404,6 +415,31 @@ def main(argv=None):
     conv_bytes = nbytes + w.dim * 5 * 4
     conv_gbs = conv_bytes / (conv_ms * 1e-3) / 1e9
 
+    # ---- training step of the scan on the same layer: forward with saved
+    # states, then the backward from them (dout N(0,1) fp32)
+    gdo = torch.Generator().manual_seed(77)
+    dout = torch.randn(w.batch, w.dim, w.seqlen, generator=gdo).to(dev)
+    g0 = sets[0]
+    bwd_steps = 10
+    tr = {}
+    for i in range(2 + bwd_steps):
+        f0, f1, b1 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        f0.record(stream)
+        _, _, ck = mb.scan_fwd_train(g0["u"], g0["delta"], g0["A"], g0["B"], g0["C"], g0["D"], g0["z"],
+                                     g0["delta_bias"], True, stream=stream)
+        f1.record(stream)
+        mb.scan_bwd(g0["u"], g0["delta"], g0["A"], g0["B"], g0["C"], g0["D"], g0["z"], g0["delta_bias"], True,
+                    dout, ckpt=ck, stream=stream)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        if i >= 2:
+            tr.setdefault("fwd", []).append(f0.elapsed_time(f1))
+            tr.setdefault("bwd", []).append(f1.elapsed_time(b1))
+    fwd_train_ms = max_over_ranks(statistics.fmean(tr["fwd"]), world, dev)
+    bwd_ms = max_over_ranks(statistics.fmean(tr["bwd"]), world, dev)
+    bbytes = bwd_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4)
+    del dout
+
     # ---- CPU baseline: the oracle on this host's cores, whole passes over the
     # workload repeated until about ten seconds of wall time have gone by
     cpu = None
@@ -445,6 +481,10 @@ def main(argv=None):
                           "ms": conv_ms, "bytes": conv_bytes, "frac": conv_gbs / peak,
                           "l2": "two rotating input sets", "timing": "mean of per-launch event pairs",
                           "traffic": recorded_traffic("conv_scan_130m")},
+            "backward": {"workload": w.name + ", dout N(0,1) fp32", "fwd_train_ms": fwd_train_ms,
+                         "bwd_ms": bwd_ms, "bwd_bytes": bbytes, "value": bbytes / (bwd_ms * 1e-3) / 1e9,
+                         "unit": "GB/s", "frac": bbytes / (bwd_ms * 1e-3) / 1e9 / peak,
+                         "timing": f"mean of {bwd_steps} event-timed (forward with saved states, backward) pairs"},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

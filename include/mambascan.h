@@ -61,7 +61,8 @@ enum {
     MS_ERR_WORKSPACE = 6, /* workspace argument inconsistent                     */
     MS_ERR_CUDA = 7,      /* a CUDA runtime call failed (no device, launch error)*/
     MS_ERR_TIMEOUT = 8,   /* device: a bounded wait gave up                      */
-    MS_ERR_DEVICE = 9     /* device is not compute capability 10.0 (B200)        */
+    MS_ERR_DEVICE = 9,    /* device is not compute capability 10.0 (B200)        */
+    MS_ERR_SCRATCH = 10   /* needs more scratch than the library's fixed buffer  */
 };
 
 /* Maximum d_state the kernels support (Mamba-1 layers use 16). */
@@ -238,6 +239,33 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
                    float *du, float *ddelta, float *dA, float *dB, float *dC, float *dD, float *dz,
                    float *ddelta_bias, float *dinitial_state, const ms_scan_dims *dims,
                    void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream);
+
+/*
+ * mamba_scan_bwd without saved states and without any allocation or caller
+ * workspace. The pages have no counterpart: this is a packaging of
+ * mamba_scan_bwd for callers that may not allocate (e.g. inside a captured
+ * CUDA graph). The recomputed saved states go to a fixed scratch buffer of
+ * MS_BWD_NOALLOC_MAX_BYTES compiled into the library (one per device, set up
+ * by the first call on that device); nothing is allocated, ever.
+ *  - Calls needing more than MS_BWD_NOALLOC_MAX_BYTES of saved states
+ *    (mamba_scan_bwd_workspace_size()) return MS_ERR_SCRATCH and do nothing.
+ *  - The buffer is shared by all calls on a device: two calls that run at the
+ *    same time on one device (different streams or host threads without
+ *    ordering) overwrite each other's scratch. Order them (one stream, or
+ *    events); calls on one stream are safe.
+ *  - The first call on a device looks the buffer up and may load the module:
+ *    make it before any stream capture on that device; later calls only
+ *    launch kernels and memsets and can be captured.
+ * Arguments and results are those of mamba_scan_bwd with ckpt = NULL.
+ */
+#define MS_BWD_NOALLOC_MAX_BYTES ((size_t)96 << 20)
+
+int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                           const float *initial_state, const void *dout, const float *dlast, float *du,
+                           float *ddelta, float *dA, float *dB, float *dC, float *dD, float *dz,
+                           float *ddelta_bias, float *dinitial_state, const ms_scan_dims *dims,
+                           int *dev_status, ms_stream_t stream);
 
 /*
  * Sizes and strides of one decode step.

@@ -18,6 +18,8 @@ LIB_PATH = os.path.join(_PKG, "libmambascan.so")
 MS_F32, MS_BF16 = 0, 1
 MS_OK, MS_ERR_NULL, MS_ERR_DTYPE, MS_ERR_SHAPE, MS_ERR_STRIDE = 0, 1, 2, 3, 4
 MS_ERR_ALIGN, MS_ERR_WORKSPACE, MS_ERR_CUDA, MS_ERR_TIMEOUT, MS_ERR_DEVICE = 5, 6, 7, 8, 9
+MS_ERR_SCRATCH = 10
+MS_BWD_NOALLOC_MAX_BYTES = 96 << 20
 MS_MAX_DSTATE = 16
 
 
@@ -86,6 +88,9 @@ def library() -> ctypes.CDLL:
         lib.mamba_scan_bwd.argtypes = ([_vp] * 8 + [ctypes.c_int] + [_vp] * 13 +
                                        [ctypes.POINTER(ScanDims), _vp, ctypes.c_size_t, _vp, _vp])
         lib.mamba_scan_bwd.restype = ctypes.c_int
+        lib.mamba_scan_bwd_noalloc.argtypes = ([_vp] * 8 + [ctypes.c_int] + [_vp] * 12 +
+                                               [ctypes.POINTER(ScanDims), _vp, _vp])
+        lib.mamba_scan_bwd_noalloc.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
                                                        _vp, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
@@ -150,6 +155,14 @@ def mamba_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_s
                                     ckpt, dout, dlast, du, ddelta, dA, dB, dC, dD, dz, ddelta_bias,
                                     dinitial_state, ctypes.byref(dims), workspace, int(workspace_bytes),
                                     dev_status, stream)
+
+
+def mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, dout, dlast,
+                           du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dinitial_state, dims: ScanDims,
+                           dev_status, stream) -> int:
+    return library().mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, int(softplus_flag),
+                                            initial_state, dout, dlast, du, ddelta, dA, dB, dC, dD, dz,
+                                            ddelta_bias, dinitial_state, ctypes.byref(dims), dev_status, stream)
 
 
 def mamba_conv_scan_fwd(x, conv_w, conv_b, conv_x0, u_out, cdims: ConvDims, delta, A, B, C, D, z,
@@ -336,6 +349,33 @@ def scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, dlast=No
                         ws_bytes, _ptr(dev_status), _stream_handle(stream))
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba_scan_bwd")
+    return g
+
+
+def scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, dlast=None,
+                     initial_state=None, stream=None, dev_status=None):
+    """scan_bwd through mamba_scan_bwd_noalloc (no saved states, no
+    workspace: the library's fixed scratch). Output tensors are created here
+    by torch; the library call itself allocates nothing."""
+    torch = _torch()
+    batch, dim, L = u.shape
+    N = A.shape[1]
+    f32 = dict(dtype=torch.float32, device=u.device)
+    g = {"du": torch.empty((batch, dim, L), **f32), "ddelta": torch.empty((batch, dim, L), **f32),
+         "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
+         "dC": torch.empty((batch, N, L), **f32),
+         "dD": torch.empty(dim, **f32) if D is not None else None,
+         "dz": torch.empty((batch, dim, L), **f32) if z is not None else None,
+         "ddelta_bias": torch.empty(dim, **f32) if delta_bias is not None else None,
+         "dinitial_state": torch.empty((batch, dim, N), **f32)}
+    dims = scan_dims_for(u, delta, B, C, z, dout)
+    rc = mamba_scan_bwd_noalloc(_ptr(u), _ptr(delta), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(z),
+                                _ptr(delta_bias), softplus, _ptr(initial_state), _ptr(dout), _ptr(dlast),
+                                _ptr(g["du"]), _ptr(g["ddelta"]), _ptr(g["dA"]), _ptr(g["dB"]), _ptr(g["dC"]),
+                                _ptr(g["dD"]), _ptr(g["dz"]), _ptr(g["ddelta_bias"]), _ptr(g["dinitial_state"]),
+                                dims, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba_scan_bwd_noalloc")
     return g
 
 

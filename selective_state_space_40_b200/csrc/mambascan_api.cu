@@ -4,12 +4,17 @@
 
 #include <climits>
 #include <cstdint>
+#include <mutex>
 #include <cuda_runtime.h>
 
 #include "mambascan.h"
 #include "ms_internal.h"
 
 static_assert(MS_CKPT_TOKENS == ms::kCkptTokens, "saved-state interval of the ABI and the kernels");
+
+// Fixed scratch of mamba_scan_bwd_noalloc: saved states recomputed by the
+// backward (one copy per device, placed by the module loader; never freed).
+static __device__ __align__(256) unsigned char g_bwd_scratch[MS_BWD_NOALLOC_MAX_BYTES];
 
 namespace {
 
@@ -52,6 +57,7 @@ const char *mamba_status_string(int code) {
         case MS_ERR_CUDA: return "CUDA runtime error (no device or launch failure)";
         case MS_ERR_TIMEOUT: return "device wait timed out";
         case MS_ERR_DEVICE: return "device is not compute capability 10.0";
+        case MS_ERR_SCRATCH: return "needs more scratch than the library's fixed buffer holds";
         default: return "unknown status code";
     }
 }
@@ -337,6 +343,51 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
         return MS_ERR_CUDA;
     }
     return MS_OK;
+}
+
+// Device address of g_bwd_scratch on the current device, looked up once per
+// device (the lookup may load the module, so it must not happen in capture).
+static int bwd_scratch(void **p) {
+    static std::mutex mtx;
+    static void *addr[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(mtx);
+    if (addr[dev] == nullptr) {
+        void *a = nullptr;
+        if (cudaGetSymbolAddress(&a, g_bwd_scratch) != cudaSuccess || a == nullptr) {
+            cudaGetLastError();
+            return MS_ERR_CUDA;
+        }
+        addr[dev] = a;
+    }
+    *p = addr[dev];
+    return MS_OK;
+}
+
+int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                           const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                           const float *initial_state, const void *dout, const float *dlast, float *du,
+                           float *ddelta, float *dA, float *dB, float *dC, float *dD, float *dz,
+                           float *ddelta_bias, float *dinitial_state, const ms_scan_dims *dims,
+                           int *dev_status, ms_stream_t stream) {
+    int rc = check_scan(u, delta, A, B, C, D, z, delta_bias, initial_state, const_cast<void *>(dout), nullptr,
+                        dims);
+    if (rc != MS_OK) return rc;
+    if (dims->batch == 0 || dims->dim == 0) return MS_OK;
+    const size_t need = mamba_scan_bwd_workspace_size(dims);
+    if (need > MS_BWD_NOALLOC_MAX_BYTES) return MS_ERR_SCRATCH;
+    void *scratch = nullptr;
+    if (need > 0) {
+        rc = bwd_scratch(&scratch);
+        if (rc != MS_OK) return rc;
+    }
+    return mamba_scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, nullptr, dout, dlast,
+                          du, ddelta, dA, dB, dC, dD, dz, ddelta_bias, dinitial_state, dims, scratch,
+                          need > 0 ? MS_BWD_NOALLOC_MAX_BYTES : 0, dev_status, stream);
 }
 
 int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,

@@ -50,7 +50,7 @@ def test_no_cpu_fallback_symbols(lib):
 
 
 def test_status_strings(lib):
-    for code in range(0, 10):
+    for code in range(0, 11):
         s = mb.mamba_status_string(code)
         assert isinstance(s, str) and s
     assert mb.mamba_status_string(0) == "ok"
@@ -184,6 +184,22 @@ def test_ckpt_sizes(lib):
     rc = mb.mamba_scan_fwd_train(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, FAKE, None, None,
                                  _dims(), None, None)
     assert rc == mb.MS_ERR_NULL  # training forward without its saved-state array
+
+
+def test_bwd_noalloc_rejects_oversize_and_bad_arguments(lib):
+    def call(dims, dout=FAKE):
+        return mb.mamba_scan_bwd_noalloc(FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, 1, None, dout, None,
+                                         FAKE, FAKE, FAKE, FAKE, FAKE, None, None, None, None, dims, None, None)
+    # 4 x 5120 x 65536 tokens needs 1024 blocks of saved states: 1.3 GB > the fixed 96 MiB
+    big = _dims(batch=4, dim=5120, seqlen=65536, u_sb=5120 * 65536, u_sd=65536, delta_sb=5120 * 65536,
+                delta_sd=65536, z_sb=5120 * 65536, z_sd=65536, y_sb=5120 * 65536, y_sd=65536,
+                B_sb=16 * 65536, B_sn=65536, C_sb=16 * 65536, C_sn=65536)
+    assert mb.mamba_scan_bwd_workspace_size(big) > mb.MS_BWD_NOALLOC_MAX_BYTES
+    assert call(big) == mb.MS_ERR_SCRATCH
+    assert "fixed buffer" in mb.mamba_status_string(mb.MS_ERR_SCRATCH)
+    assert call(_dims(dstate=0)) == mb.MS_ERR_SHAPE
+    assert call(_dims(), dout=None) == mb.MS_ERR_NULL
+    assert call(_dims(batch=0)) == mb.MS_OK
 
 
 def _udims(**kw):

@@ -337,6 +337,13 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
     a.z_sb = dims->z_sb; a.z_sd = dims->z_sd; a.y_sb = dims->y_sb; a.y_sd = dims->y_sd;
     a.B_sb = dims->B_sb; a.B_sn = dims->B_sn; a.C_sb = dims->C_sb; a.C_sn = dims->C_sn;
     a.softplus = softplus_flag ? 1 : 0;
+    {
+        const int ei = elem_bytes(dims->in_dtype), eo = elem_bytes(dims->out_dtype);
+        a.vec_in = vec_ok(u, dims->u_sb, dims->u_sd, ei) && vec_ok(delta, dims->delta_sb, dims->delta_sd, ei) &&
+                   vec_ok(z, dims->z_sb, dims->z_sd, ei);
+        a.vec_out = vec_ok(dout, dims->y_sb, dims->y_sd, eo);
+        a.vec_bc = aligned(dB, 16) && aligned(dC, 16) && (L % 4) == 0;
+    }
     e = ms::launch_scan_bwd(a, dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, st);
     if (e != cudaSuccess) {
         cudaGetLastError();

@@ -49,6 +49,9 @@ struct BwdArgs {
     int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, y_sb, y_sd;
     int64_t B_sb, B_sn, C_sb, C_sn;
     int softplus;
+    int vec_in;   // u/delta/z rows 16-byte aligned
+    int vec_out;  // dout rows 16-byte aligned
+    int vec_bc;   // dB/dC rows allow 16-byte atomics (L % 4 == 0, aligned base)
 };
 
 // Launch shape chosen on the host for one scan call.

@@ -41,12 +41,15 @@ constexpr int kSub = 8;                  // tokens per sub-chunk
 constexpr int kNSub = kBlk / kSub;
 static_assert(kBlk % kSub == 0, "whole sub-chunks per block");
 static_assert(2 * kBlk <= kBThreads, "one staging thread per B/C row");
+static_assert(kBlk == 16 * kG, "each lane prepares 16 tokens of its channel's block");
 
 struct BwdSmem {
-    float bc[kBlk][36];               // token rows: B[0..15], C[16..31], pad
-    float sub[kBNW][kNSub][4][32];    // state at each sub-chunk start [warp][s][state][lane]
-    float red[kBNW][kSub][32];        // warp sums of dB/dC per token [warp][j][value]
+    float bc[kBlk][36];                  // token rows: B[0..15], C[16..31], pad
+    float sub[kBNW][kNSub][4][32];       // state at each sub-chunk start [warp][s][state][lane]
+    float red[2][kBNW][kSub][32];        // warp sums of dB/dC per token, two sub-chunks in turn
+    float tok[4][kBNW][kCW][kBlk + 4];   // per channel and token: Delta, softplus', gate, gate'
 };
+enum { kTokDelta = 0, kTokSig = 1, kTokGate = 2, kTokGateGrad = 3 };
 
 template <typename T>
 __device__ __forceinline__ float ld_elem(const T *p) {
@@ -54,18 +57,30 @@ __device__ __forceinline__ float ld_elem(const T *p) {
     else return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)));
 }
 
-// 8 tokens [t, t+8) of a row as fp32 (0 past L), read through the read-only
-// cache (the 4 lanes of a channel read the same chunk).
+// 8 tokens [t, t+8) of a row as fp32 (0 past L): one or two 16-byte loads
+// when the row allows, else element loads.
 template <typename T>
-__device__ __forceinline__ void load8(const T *row, int64_t t, int64_t L, float (&v)[8]) {
+__device__ __forceinline__ void load8(const T *row, int64_t t, int64_t L, bool vec, float (&v)[8]) {
+    if (vec && t + 8 <= L) {
+        if constexpr (sizeof(T) == 4) {
+            const float4 a = __ldg(reinterpret_cast<const float4 *>(row + t));
+            const float4 b = __ldg(reinterpret_cast<const float4 *>(row + t) + 1);
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+            v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+        } else {
+            const uint4 w = __ldg(reinterpret_cast<const uint4 *>(row + t));
+            v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+            v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
+        }
+    } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) v[j] = (t + j < L) ? ld_elem(row + t + j) : 0.0f;
+        for (int j = 0; j < 8; ++j) v[j] = (t + j < L) ? ld_elem(row + t + j) : 0.0f;
+    }
 }
 
 // Reduce-scatter of v[0..8) over the 8 channel lanes of a warp (lane bits 2..4):
 // afterwards lane (c, g) holds the sum over channels of v[c].
 __device__ __forceinline__ float reduce_scatter_channels(float (&v)[8], int c) {
-    // step over lane bit 4 (channel bit 2): keep half 4*c2 .. 4*c2+3
     const bool u2 = (c & 4) != 0;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -105,17 +120,31 @@ __device__ __forceinline__ void reduce_scatter_lanes(float (&v)[8], int g) {
     }
 }
 
-// Softplus and its derivative (the logistic function) from one exponential.
+// softplus(v) and its derivative, the logistic function, from one e^{-|v|}
+// (same series / logarithm split as the forward's softplus).
 __device__ __forceinline__ void softplus_and_grad(float v, float &sp, float &sig) {
-    sp = softplus_f(v);
-    const float e = exp2_mufu(-fabsf(v) * kLog2e);  // e^{-|v|}
+    const float e = exp2_mufu(-fabsf(v) * kLog2e);
+    float s = fmaf(e, -1.0f / 6.0f, 0.2f);
+    s = fmaf(e, s, -0.25f);
+    s = fmaf(e, s, 1.0f / 3.0f);
+    s = fmaf(e, s, -0.5f);
+    s = fmaf(e, s, 1.0f);
+    const float lp = e < 0.0625f ? e * s : log2_mufu(1.0f + e) * kLn2;
+    sp = fmaxf(v, 0.0f) + lp;
     const float r = rcp_mufu(1.0f + e);
     sig = v >= 0.0f ? r : e * r;
 }
 
+struct F4 { float v[4]; };
+__device__ __forceinline__ F4 lds4(const float *p) {
+    const float4 x = *reinterpret_cast<const float4 *>(p);
+    return F4{{x.x, x.y, x.z, x.w}};
+}
+
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a) {
-    __shared__ __align__(16) BwdSmem sm;
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    BwdSmem &sm = *reinterpret_cast<BwdSmem *>(smem_raw);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int c = lane / kG, g = lane % kG;
@@ -141,6 +170,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
     const bool has_z = a.z != nullptr;
     const bool sp = a.softplus != 0;
+    const bool vin = a.vec_in != 0, vout = a.vec_out != 0;
     float dDacc = 0.0f, dbacc = 0.0f;
 
     const TIn *u_row = static_cast<const TIn *>(a.u) + b * a.u_sb + dd * a.u_sd;
@@ -150,13 +180,17 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     const TIn *B_b = static_cast<const TIn *>(a.B) + b * a.B_sb;
     const TIn *C_b = static_cast<const TIn *>(a.C) + b * a.C_sb;
     const int64_t grow = (b * a.dim + dd) * L;  // dense gradient row
+    const float *tk_dl = sm.tok[kTokDelta][warp][c];
+    const float *tk_sig = sm.tok[kTokSig][warp][c];
+    const float *tk_gate = sm.tok[kTokGate][warp][c];
+    const float *tk_gp = sm.tok[kTokGateGrad][warp][c];
 
     const int64_t nblk = (L + kBlk - 1) / kBlk;
     for (int64_t kb = nblk - 1; kb >= 0; --kb) {
         const int64_t tb = kb * kBlk;
+        __syncthreads();  // the previous block is done with bc and tok
 
-        // ---- stage B and C of the block as fp32 token rows
-        __syncthreads();
+        // ---- B and C of the block as fp32 token rows
         if (threadIdx.x < 2 * kBlk) {
             const int r = threadIdx.x;
             const bool isC = r >= kBlk;
@@ -166,6 +200,32 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
             float *row = &sm.bc[r % kBlk][isC ? 16 : 0];
 #pragma unroll
             for (int n = 0; n < 16; ++n) row[n] = (n < N && t < L) ? ld_elem(base + n * sn) : 0.0f;
+        }
+        // ---- per-token quantities of the channel, once: lane g takes 16 tokens
+#pragma unroll
+        for (int h8 = 0; h8 < 2; ++h8) {
+            const int off = 16 * g + 8 * h8;
+            const int64_t ts = tb + off;
+            float dv[8], zv[8];
+            load8(d_row, ts, L, vin, dv);
+            if (has_z) load8(z_row, ts, L, vin, zv);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                const float v = dv[j] + bias;
+                float spv = v, sgv = 1.0f;
+                if (sp) softplus_and_grad(v, spv, sgv);
+                float gt = 1.0f, gp = 0.0f;
+                if (has_z) {
+                    const float zz = zv[j];
+                    const float sz = rcp_mufu(1.0f + exp2_mufu(-zz * kLog2e));
+                    gt = zz * sz;
+                    gp = sz * (1.0f + zz * (1.0f - sz));
+                }
+                sm.tok[kTokDelta][warp][c][off + j] = (ts + j < L) ? spv : 0.0f;
+                sm.tok[kTokSig][warp][c][off + j] = sgv;
+                sm.tok[kTokGate][warp][c][off + j] = gt;
+                sm.tok[kTokGateGrad][warp][c][off + j] = gp;
+            }
         }
         __syncthreads();
 
@@ -178,99 +238,88 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
         for (int s = 0; s < kNSub; ++s) {
 #pragma unroll
             for (int i = 0; i < 4; ++i) sm.sub[warp][s][i][lane] = h[i];
-            const int64_t ts = tb + s * kSub;
-            float uv[8], dv[8];
-            load8(u_row, ts, L, uv);
-            load8(d_row, ts, L, dv);
+            float uv[8];
+            load8(u_row, tb + s * kSub, L, vin, uv);
+            const F4 dl0 = lds4(tk_dl + s * kSub), dl1 = lds4(tk_dl + s * kSub + 4);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
-                const float v = dv[j] + bias;
-                const float dl = (ts + j < L) ? (sp ? softplus_f(v) : v) : 0.0f;
+                const float dl = j < 4 ? dl0.v[j & 3] : dl1.v[j & 3];
                 const float du = dl * uv[j];
-                const float *bcr = sm.bc[s * kSub + j];
+                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) h[i] = fmaf(exp2_mufu(dl * A2[i]), h[i], du * bcr[n0 + i]);
+                for (int i = 0; i < 4; ++i) h[i] = fmaf(exp2_mufu(dl * A2[i]), h[i], du * Bn.v[i]);
             }
         }
 
         // ---- sub-chunks from the last: recompute, then the adjoint
         for (int s = kNSub - 1; s >= 0; --s) {
             const int64_t ts = tb + s * kSub;
-            float uv[8], dv[8], zv[8], ov[8];
-            load8(u_row, ts, L, uv);
-            load8(d_row, ts, L, dv);
-            if (has_z) load8(z_row, ts, L, zv);
+            const int rb = s & 1;
+            float uv[8], ov[8];
+            load8(u_row, ts, L, vin, uv);
             // an idle lane (channel past dim) gets dout = 0: with its zero
             // starting adjoint every contribution to the channel sums is 0
-            if (active) load8(o_row, ts, L, ov);
+            if (active) load8(o_row, ts, L, vout, ov);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) ov[j] = active ? ov[j] : 0.0f;
-            float dl[8], sig[8], gate[8], gprime[8];
+            float dl[8], gate[8];
+            {
+                const F4 a0 = lds4(tk_dl + s * kSub), a1 = lds4(tk_dl + s * kSub + 4);
+                const F4 g0 = lds4(tk_gate + s * kSub), g1 = lds4(tk_gate + s * kSub + 4);
 #pragma unroll
-            for (int j = 0; j < kSub; ++j) {
-                const float v = dv[j] + bias;
-                float spv = v, sgv = 1.0f;
-                if (sp) softplus_and_grad(v, spv, sgv);
-                const bool in = ts + j < L;
-                dl[j] = in ? spv : 0.0f;
-                sig[j] = sgv;
-                if (has_z) {
-                    const float zz = zv[j];
-                    const float sz = rcp_mufu(1.0f + exp2_mufu(-zz * kLog2e));
-                    gate[j] = zz * sz;
-                    gprime[j] = sz * (1.0f + zz * (1.0f - sz));
-                } else {
-                    gate[j] = 1.0f;
-                    gprime[j] = 0.0f;
+                for (int j = 0; j < 4; ++j) {
+                    dl[j] = a0.v[j]; dl[4 + j] = a1.v[j];
+                    gate[j] = g0.v[j]; gate[4 + j] = g1.v[j];
                 }
             }
             // recompute A_bar and h of the sub-chunk, and the pre-gate output q
-            float hs[4], ab[kSub][4], hh[kSub][4], dq[kSub], dzv[kSub];
+            float hs[4], ab[kSub][4], hh[kSub][4], dq[kSub], qv[kSub];
 #pragma unroll
             for (int i = 0; i < 4; ++i) hs[i] = sm.sub[warp][s][i][lane];
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
                 const float du = dl[j] * uv[j];
-                const float *bcr = sm.bc[s * kSub + j];
+                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
+                const F4 Cn = lds4(sm.bc[s * kSub + j] + 16 + n0);
                 float part = 0.0f;
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     ab[j][i] = exp2_mufu(dl[j] * A2[i]);
                     const float hp = j == 0 ? hs[i] : hh[j - 1][i];
-                    hh[j][i] = fmaf(ab[j][i], hp, du * bcr[n0 + i]);
-                    part = fmaf(bcr[16 + n0 + i], hh[j][i], part);
+                    hh[j][i] = fmaf(ab[j][i], hp, du * Bn.v[i]);
+                    part = fmaf(Cn.v[i], hh[j][i], part);
                 }
                 part += __shfl_xor_sync(0xffffffffu, part, 1);
                 part += __shfl_xor_sync(0xffffffffu, part, 2);
-                const float q = part + Dd * uv[j];
+                qv[j] = part + Dd * uv[j];
                 dq[j] = ov[j] * gate[j];
-                dzv[j] = ov[j] * q * gprime[j];
             }
             // adjoint over the sub-chunk, last token first
             float ddt[kSub], dus[kSub];
 #pragma unroll
             for (int j = kSub - 1; j >= 0; --j) {
                 const float dqj = dq[j];
-                const float *bcr = sm.bc[s * kSub + j];
                 const float du = dl[j] * uv[j];
+                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
+                const F4 Cn = lds4(sm.bc[s * kSub + j] + 16 + n0);
                 float pdt = 0.0f, pdu = 0.0f, v8[8];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
-                    const float Bn = bcr[n0 + i], Cn = bcr[16 + n0 + i];
-                    const float lam = fmaf(Cn, dqj, carry[i]);
+                    const float lam = fmaf(Cn.v[i], dqj, carry[i]);
                     const float hp = j == 0 ? hs[i] : hh[j - 1][i];
                     const float dab = lam * hp * ab[j][i];
                     dAacc[i] = fmaf(dab, dl[j], dAacc[i]);
                     pdt = fmaf(dab, An[i], pdt);
-                    pdt = fmaf(lam * Bn, uv[j], pdt);
-                    pdu = fmaf(lam * Bn, dl[j], pdu);
-                    v8[i] = lam * du;          // dB
+                    const float lb = lam * Bn.v[i];
+                    pdt = fmaf(lb, uv[j], pdt);
+                    pdu = fmaf(lb, dl[j], pdu);
+                    v8[i] = lam * du;           // dB
                     v8[4 + i] = dqj * hh[j][i]; // dC
                     carry[i] = ab[j][i] * lam;
                 }
                 ddt[j] = pdt;
                 dus[j] = pdu;
-                sm.red[warp][j][lane] = reduce_scatter_channels(v8, c);
+                sm.red[rb][warp][j][lane] = reduce_scatter_channels(v8, c);
             }
             // per-token sums over the channel's 4 lanes; lane g owns tokens 2g, 2g+1
             reduce_scatter_lanes(ddt, g);
@@ -281,33 +330,44 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 const int k = j & 1;
                 const int64_t t = ts + j;
                 if ((j >> 1) == g && active && t < L) {
-                    const float ddv = sp ? ddt[k] * sig[j] : ddt[k];
+                    const float ddv = ddt[k] * tk_sig[s * kSub + j];
                     a.ddelta[grow + t] = ddv;
                     a.du[grow + t] = fmaf(Dd, dq[j], dus[k]);
-                    if (has_z && a.dz != nullptr) a.dz[grow + t] = dzv[j];
+                    if (has_z && a.dz != nullptr) a.dz[grow + t] = ov[j] * qv[j] * tk_gp[s * kSub + j];
                     dDacc = fmaf(dq[j], uv[j], dDacc);
                     dbacc += ddv;
                 }
             }
-            // dB / dC: sum the warps' partial sums, then one atomic per output
+            // dB / dC: sum the warps' partial sums (this sub-chunk's buffer;
+            // the other buffer is being filled by the next sub-chunk), then
+            // one 4-token atomic per output row segment
             __syncthreads();
-            {
+            if (threadIdx.x < 64) {
                 const int col = threadIdx.x & 31;        // value column: lane that held it
-                const int jp = threadIdx.x >> 5;         // token pair
+                const int qd = threadIdx.x >> 5;         // token quad
                 const int cg = col / kG, gg = col % kG;  // channel slot -> value, lane group -> states
                 const bool isC = cg >= 4;
                 const int n = gg * 4 + (cg & 3);
+                float sum[4];
 #pragma unroll
-                for (int k = 0; k < 2; ++k) {
-                    const int j = 2 * jp + k;
-                    const int64_t t = ts + j;
-                    float sum = 0.0f;
+                for (int k = 0; k < 4; ++k) {
+                    const int j = 4 * qd + k;
+                    sum[k] = 0.0f;
 #pragma unroll
-                    for (int w = 0; w < kBNW; ++w) sum += sm.red[w][j][col];
-                    if (n < N && t < L) atomicAdd((isC ? a.dC : a.dB) + (b * N + n) * L + t, sum);
+                    for (int w = 0; w < kBNW; ++w) sum[k] += sm.red[rb][w][j][col];
+                }
+                const int64_t t = ts + 4 * qd;
+                if (n < N) {
+                    float *dst = (isC ? a.dC : a.dB) + (b * N + n) * L + t;
+                    if (a.vec_bc && t + 4 <= L) {
+                        atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(sum[0], sum[1], sum[2], sum[3]));
+                    } else {
+#pragma unroll
+                        for (int k = 0; k < 4; ++k)
+                            if (t + k < L) atomicAdd(dst + k, sum[k]);
+                    }
                 }
             }
-            __syncthreads();
         }
     }
 
@@ -332,6 +392,23 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     }
 }
 
+template <typename TIn, typename TOut>
+cudaError_t launch_bwd(const BwdArgs &a, unsigned grid, cudaStream_t stream) {
+    // more than 48 KB of shared memory: opt in once per device
+    static bool opted[64] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev >= 64 || !opted[dev]) {
+        e = cudaFuncSetAttribute(scan_bwd_kernel<TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)sizeof(BwdSmem));
+        if (e != cudaSuccess) return e;
+        if (dev < 64) opted[dev] = true;
+    }
+    scan_bwd_kernel<TIn, TOut><<<grid, kBThreads, sizeof(BwdSmem), stream>>>(a);
+    return cudaGetLastError();
+}
+
 }  // namespace
 
 cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream) {
@@ -341,13 +418,10 @@ cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaS
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     const unsigned grid = (unsigned)blocks;
     if (in_bf16) {
-        if (out_bf16) scan_bwd_kernel<__nv_bfloat16, __nv_bfloat16><<<grid, kBThreads, 0, stream>>>(a);
-        else scan_bwd_kernel<__nv_bfloat16, float><<<grid, kBThreads, 0, stream>>>(a);
-    } else {
-        if (out_bf16) scan_bwd_kernel<float, __nv_bfloat16><<<grid, kBThreads, 0, stream>>>(a);
-        else scan_bwd_kernel<float, float><<<grid, kBThreads, 0, stream>>>(a);
+        return out_bf16 ? launch_bwd<__nv_bfloat16, __nv_bfloat16>(a, grid, stream)
+                        : launch_bwd<__nv_bfloat16, float>(a, grid, stream);
     }
-    return cudaGetLastError();
+    return out_bf16 ? launch_bwd<float, __nv_bfloat16>(a, grid, stream) : launch_bwd<float, float>(a, grid, stream);
 }
 
 }  // namespace ms

@@ -157,14 +157,21 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     const int64_t L = a.L;
     const int n0 = g * 4;
 
-    float A2[4], An[4], carry[4], dAacc[4];
+    // the lane's 4 states as 2 packed pairs (states n0+2p, n0+2p+1)
+    f2 A2[2], An[2], carry[2], dAacc[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const int n = n0 + i;
-        An[i] = n < N ? __ldg(a.A + dd * N + n) : 0.0f;
-        A2[i] = An[i] * kLog2e;
-        carry[i] = (a.dlast != nullptr && active && n < N) ? __ldg(a.dlast + (b * a.dim + d) * N + n) : 0.0f;
-        dAacc[i] = 0.0f;
+    for (int p = 0; p < 2; ++p) {
+        float an[2], cr[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int n = n0 + 2 * p + k;
+            an[k] = n < N ? __ldg(a.A + dd * N + n) : 0.0f;
+            cr[k] = (a.dlast != nullptr && active && n < N) ? __ldg(a.dlast + (b * a.dim + d) * N + n) : 0.0f;
+        }
+        An[p] = f2_make(an[0], an[1]);
+        A2[p] = f2_make(an[0] * kLog2e, an[1] * kLog2e);
+        carry[p] = f2_make(cr[0], cr[1]);
+        dAacc[p] = f2_splat(0.0f);
     }
     const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
     const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
@@ -231,23 +238,34 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
 
         // ---- pass A: the block forward from its saved state; keep the state
         // at every sub-chunk start.
-        float h[4];
+        f2 h[2];
+        {
+            float hv[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
-            h[i] = (active && n0 + i < N) ? __ldg(a.ckpt + ((b * a.dim + d) * nblk + kb) * N + n0 + i) : 0.0f;
+            for (int i = 0; i < 4; ++i)
+                hv[i] = (active && n0 + i < N) ? __ldg(a.ckpt + ((b * a.dim + d) * nblk + kb) * N + n0 + i) : 0.0f;
+            h[0] = f2_make(hv[0], hv[1]);
+            h[1] = f2_make(hv[2], hv[3]);
+        }
         for (int s = 0; s < kNSub; ++s) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sm.sub[warp][s][i][lane] = h[i];
+            for (int p = 0; p < 2; ++p) {
+                float lo, hi;
+                f2_split(h[p], lo, hi);
+                sm.sub[warp][s][2 * p][lane] = lo;
+                sm.sub[warp][s][2 * p + 1][lane] = hi;
+            }
             float uv[8];
             load8(u_row, tb + s * kSub, L, vin, uv);
             const F4 dl0 = lds4(tk_dl + s * kSub), dl1 = lds4(tk_dl + s * kSub + 4);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
                 const float dl = j < 4 ? dl0.v[j & 3] : dl1.v[j & 3];
-                const float du = dl * uv[j];
-                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
+                const f2 dl2 = f2_splat(dl), du2 = f2_splat(dl * uv[j]);
+                f2 Bp[2];
+                lds_f2x2(sm.bc[s * kSub + j] + n0, Bp[0], Bp[1]);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) h[i] = fmaf(exp2_mufu(dl * A2[i]), h[i], du * Bn.v[i]);
+                for (int p = 0; p < 2; ++p) h[p] = f2_fma(exp2_mufu2(f2_mul(dl2, A2[p])), h[p], f2_mul(du2, Bp[p]));
             }
         }
 
@@ -273,22 +291,27 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 }
             }
             // recompute A_bar and h of the sub-chunk, and the pre-gate output q
-            float hs[4], ab[kSub][4], hh[kSub][4], dq[kSub], qv[kSub];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) hs[i] = sm.sub[warp][s][i][lane];
+            f2 hs[2], ab[kSub][2], hh[kSub][2];
+            float dq[kSub], qv[kSub];
+            hs[0] = f2_make(sm.sub[warp][s][0][lane], sm.sub[warp][s][1][lane]);
+            hs[1] = f2_make(sm.sub[warp][s][2][lane], sm.sub[warp][s][3][lane]);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
-                const float du = dl[j] * uv[j];
-                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
-                const F4 Cn = lds4(sm.bc[s * kSub + j] + 16 + n0);
-                float part = 0.0f;
+                const f2 dl2 = f2_splat(dl[j]), du2 = f2_splat(dl[j] * uv[j]);
+                f2 Bp[2], Cp[2];
+                lds_f2x2(sm.bc[s * kSub + j] + n0, Bp[0], Bp[1]);
+                lds_f2x2(sm.bc[s * kSub + j] + 16 + n0, Cp[0], Cp[1]);
+                f2 acc = f2_splat(0.0f);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    ab[j][i] = exp2_mufu(dl[j] * A2[i]);
-                    const float hp = j == 0 ? hs[i] : hh[j - 1][i];
-                    hh[j][i] = fmaf(ab[j][i], hp, du * Bn.v[i]);
-                    part = fmaf(Cn.v[i], hh[j][i], part);
+                for (int p = 0; p < 2; ++p) {
+                    ab[j][p] = exp2_mufu2(f2_mul(dl2, A2[p]));
+                    const f2 hp = j == 0 ? hs[p] : hh[j - 1][p];
+                    hh[j][p] = f2_fma(ab[j][p], hp, f2_mul(du2, Bp[p]));
+                    acc = f2_fma(Cp[p], hh[j][p], acc);
                 }
+                float plo, phi;
+                f2_split(acc, plo, phi);
+                float part = plo + phi;
                 part += __shfl_xor_sync(0xffffffffu, part, 1);
                 part += __shfl_xor_sync(0xffffffffu, part, 2);
                 qv[j] = part + Dd * uv[j];
@@ -298,27 +321,36 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
             float ddt[kSub], dus[kSub];
 #pragma unroll
             for (int j = kSub - 1; j >= 0; --j) {
-                const float dqj = dq[j];
-                const float du = dl[j] * uv[j];
-                const F4 Bn = lds4(sm.bc[s * kSub + j] + n0);
-                const F4 Cn = lds4(sm.bc[s * kSub + j] + 16 + n0);
-                float pdt = 0.0f, pdu = 0.0f, v8[8];
+                const f2 dq2 = f2_splat(dq[j]), dl2 = f2_splat(dl[j]), u2 = f2_splat(uv[j]);
+                const f2 du2 = f2_splat(dl[j] * uv[j]);
+                f2 Bp[2], Cp[2];
+                lds_f2x2(sm.bc[s * kSub + j] + n0, Bp[0], Bp[1]);
+                lds_f2x2(sm.bc[s * kSub + j] + 16 + n0, Cp[0], Cp[1]);
+                f2 pdt = f2_splat(0.0f), pdu = f2_splat(0.0f), vB[2], vC[2];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const float lam = fmaf(Cn.v[i], dqj, carry[i]);
-                    const float hp = j == 0 ? hs[i] : hh[j - 1][i];
-                    const float dab = lam * hp * ab[j][i];
-                    dAacc[i] = fmaf(dab, dl[j], dAacc[i]);
-                    pdt = fmaf(dab, An[i], pdt);
-                    const float lb = lam * Bn.v[i];
-                    pdt = fmaf(lb, uv[j], pdt);
-                    pdu = fmaf(lb, dl[j], pdu);
-                    v8[i] = lam * du;           // dB
-                    v8[4 + i] = dqj * hh[j][i]; // dC
-                    carry[i] = ab[j][i] * lam;
+                for (int p = 0; p < 2; ++p) {
+                    const f2 lam = f2_fma(Cp[p], dq2, carry[p]);
+                    const f2 hp = j == 0 ? hs[p] : hh[j - 1][p];
+                    const f2 dab = f2_mul(lam, f2_mul(hp, ab[j][p]));
+                    dAacc[p] = f2_fma(dab, dl2, dAacc[p]);
+                    pdt = f2_fma(dab, An[p], pdt);
+                    const f2 lb = f2_mul(lam, Bp[p]);
+                    pdt = f2_fma(lb, u2, pdt);
+                    pdu = f2_fma(lb, dl2, pdu);
+                    vB[p] = f2_mul(lam, du2);        // dB
+                    vC[p] = f2_mul(dq2, hh[j][p]);   // dC
+                    carry[p] = f2_mul(ab[j][p], lam);
                 }
-                ddt[j] = pdt;
-                dus[j] = pdu;
+                float x0, x1;
+                f2_split(pdt, x0, x1);
+                ddt[j] = x0 + x1;
+                f2_split(pdu, x0, x1);
+                dus[j] = x0 + x1;
+                float v8[8];
+                f2_split(vB[0], v8[0], v8[1]);
+                f2_split(vB[1], v8[2], v8[3]);
+                f2_split(vC[0], v8[4], v8[5]);
+                f2_split(vC[1], v8[6], v8[7]);
                 sm.red[rb][warp][j][lane] = reduce_scatter_channels(v8, c);
             }
             // per-token sums over the channel's 4 lanes; lane g owns tokens 2g, 2g+1
@@ -373,12 +405,17 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
 
     // ---- per-channel results
     if (active) {
+        float cv[4], av[4];
+        f2_split(carry[0], cv[0], cv[1]);
+        f2_split(carry[1], cv[2], cv[3]);
+        f2_split(dAacc[0], av[0], av[1]);
+        f2_split(dAacc[1], av[2], av[3]);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int n = n0 + i;
             if (n < N) {
-                if (a.dh0 != nullptr) a.dh0[(b * a.dim + d) * N + n] = carry[i];
-                atomicAdd(a.dA + d * N + n, dAacc[i]);
+                if (a.dh0 != nullptr) a.dh0[(b * a.dim + d) * N + n] = cv[i];
+                atomicAdd(a.dA + d * N + n, av[i]);
             }
         }
     }

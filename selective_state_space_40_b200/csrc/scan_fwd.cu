@@ -246,7 +246,7 @@ __device__ __forceinline__ float state_token(const float *bcr, int n0, float dl,
     return lo + hi;
 }
 
-template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV>
+template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV, bool CKPT>
 __global__ void __launch_bounds__(kThreads, CH == 1 ? MS_SCAN_MINB : 1)
 scan_fwd_kernel(const ScanArgs a) {
     static_assert(!CONV || CH == 1, "the conv front-end runs with one chunk per lane");
@@ -373,7 +373,7 @@ scan_fwd_kernel(const ScanArgs a) {
     for (int64_t k = 0; k < ntiles; ++k) {
         const int64_t t0 = k * TT;
         const int buf = (int)(k & 1);
-        if (a.ckpt != nullptr && active && t0 % kCkptTokens == 0) {
+        if (CKPT && active && t0 % kCkptTokens == 0) {
             // Training: the state before this block, for the backward's recompute.
             float *cs = a.ckpt + ((b * a.dim + d) * nck + t0 / kCkptTokens) * N;
 #pragma unroll
@@ -469,7 +469,7 @@ scan_fwd_kernel(const ScanArgs a) {
                                                                         j * P);
                     yo[j] = fmaf(yv, gate[i][j], dug[i][j]);
                 }
-                if (active && a.y != nullptr) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
+                if (active && (!CKPT || a.y != nullptr)) store8<TOut>(y_row, t0 + 8 * i, L, vout, yo);
             }
         } else {
             __syncwarp();
@@ -534,7 +534,7 @@ scan_fwd_kernel(const ScanArgs a) {
                 float yo[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) yo[j] = fmaf(ys[j], gate[i][j], dug[i][j]);
-                if (active && a.y != nullptr) store8<TOut>(y_row, t0 + off, L, vout, yo);
+                if (active && (!CKPT || a.y != nullptr)) store8<TOut>(y_row, t0 + off, L, vout, yo);
             }
             __syncwarp();
         }
@@ -553,7 +553,7 @@ scan_fwd_kernel(const ScanArgs a) {
     }
 }
 
-template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV = false>
+template <typename TIn, typename TOut, int G, int CH, int POLY8, bool CONV = false, bool CKPT = false>
 cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     using Gm = Geom<G, CH>;
     using Sm = SmemLayout<G, CH>;
@@ -568,12 +568,12 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev >= 64 || !opted[dev]) {
-        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV>,
+        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
         if (e != cudaSuccess) return e;
         if (dev < 64) opted[dev] = true;
     }
-    scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
+    scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
     return cudaGetLastError();
 }
 
@@ -618,10 +618,36 @@ cudaError_t launch_types_conv(const ScanArgs &a, const ScanPlan &pl, cudaStream_
     }
 }
 
+// Training forward (saved states, y optional): one chunk per lane,
+// exponentials all on MUFU or all on the polynomial (the automatic plans).
+template <typename TIn, typename TOut>
+cudaError_t launch_types_ckpt(const ScanArgs &a, const ScanPlan &pl, cudaStream_t stream) {
+    const bool poly = pl.poly8 != 0;
+    switch (pl.lanes_per_channel) {
+        case 1: return poly ? launch_one<TIn, TOut, 1, 1, 8, false, true>(a, stream)
+                            : launch_one<TIn, TOut, 1, 1, 0, false, true>(a, stream);
+        case 2: return poly ? launch_one<TIn, TOut, 2, 1, 8, false, true>(a, stream)
+                            : launch_one<TIn, TOut, 2, 1, 0, false, true>(a, stream);
+        case 4: return poly ? launch_one<TIn, TOut, 4, 1, 8, false, true>(a, stream)
+                            : launch_one<TIn, TOut, 4, 1, 0, false, true>(a, stream);
+        default: return poly ? launch_one<TIn, TOut, 8, 1, 8, false, true>(a, stream)
+                             : launch_one<TIn, TOut, 8, 1, 0, false, true>(a, stream);
+    }
+}
+
 }  // namespace
 
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16,
                             cudaStream_t stream) {
+    if (a.ckpt != nullptr) {
+        if (plan.chunks_per_lane != 1 || (plan.poly8 != 0 && plan.poly8 != 8)) return cudaErrorInvalidValue;
+        if (in_bf16) {
+            return out_bf16 ? launch_types_ckpt<__nv_bfloat16, __nv_bfloat16>(a, plan, stream)
+                            : launch_types_ckpt<__nv_bfloat16, float>(a, plan, stream);
+        }
+        return out_bf16 ? launch_types_ckpt<float, __nv_bfloat16>(a, plan, stream)
+                        : launch_types_ckpt<float, float>(a, plan, stream);
+    }
     if (a.conv_w != nullptr) {
         if (in_bf16) {
             return out_bf16 ? launch_types_conv<__nv_bfloat16, __nv_bfloat16>(a, plan, stream)

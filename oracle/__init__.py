@@ -14,6 +14,7 @@ from .oracle import (  # noqa: F401
     scan,
     scan_bwd,
     scan_mt,
+    ssd,
     state_update,
     softplus,
     silu,

@@ -442,3 +442,65 @@ int oracle_scan_bwd_f64(int64_t batch, int64_t dim, int64_t dstate, int64_t seql
     free(hs); free(ab); free(dts); free(q); free(lam); free(carry);
     return 0;
 }
+
+/*
+ * Mamba-2 state space duality layer ('Mamba-1/2/3 Markdown図解' blog,
+ * section 3: one model with a recurrent view, used for decoding, and a
+ * matrix view computed chunk by chunk for training and prefill; the
+ * transition is a scalar times the identity within a head). This oracle is
+ * the recurrent view. For batch b, head h (head dim P, state N, group
+ * g = h / (H / G) sharing B and C):
+ *   Delta_t = softplus(dt[b,t,h] + dt_bias[h])  (plain sum without the flag)
+ *   S_t[p][n] = exp(Delta_t A[h]) S_{t-1}[p][n] + Delta_t B[b,t,g,n] x[b,t,h,p]
+ *   y[b,t,h,p] = sum_n C[b,t,g,n] S_t[p][n] + D[h] x[b,t,h,p]
+ * Layouts (dense, fp64): x, y [b][L][H][P]; dt [b][L][H]; B, C [b][L][G][N];
+ * A, D, dt_bias [H]; s0, s_last [b][H][P][N]. Nullable: D, dt_bias, s0 (zero),
+ * s_last.
+ */
+int oracle_ssd_f64(int64_t batch, int64_t seqlen, int64_t nheads, int64_t headdim, int64_t dstate,
+                   int64_t ngroups, const double *x, const double *dt, const double *A,
+                   const double *B, const double *C, const double *D, const double *dt_bias,
+                   int softplus_flag, const double *s0, double *y, double *s_last)
+{
+    const int64_t H = nheads, P = headdim, N = dstate, G = ngroups, L = seqlen;
+    if (batch < 0 || L < 0 || H < 1 || P < 1 || N < 1 || G < 1 || H % G != 0) return -1;
+    if (batch * L > 0 && (!x || !dt || !A || !B || !C || !y)) return -1;
+    double *S = (double *)malloc((size_t)(P * N) * sizeof(double));
+    if (!S) return -1;
+    for (int64_t b = 0; b < batch; ++b) {
+        for (int64_t h = 0; h < H; ++h) {
+#if ORACLE_MUTANT == 19
+            const int64_t g = h % G; /* mutant: heads assigned to groups round-robin */
+#else
+            const int64_t g = h / (H / G);
+#endif
+            for (int64_t i = 0; i < P * N; ++i) S[i] = s0 ? s0[(b * H + h) * P * N + i] : 0.0;
+            for (int64_t t = 0; t < L; ++t) {
+                const double dlt = step_size(dt[(b * L + t) * H + h], dt_bias ? dt_bias[h] : 0.0, softplus_flag);
+                const double a = exp(dlt * A[h]);
+                const double *Bt = B + ((b * L + t) * G + g) * N;
+                const double *Ct = C + ((b * L + t) * G + g) * N;
+                const double *xt = x + ((b * L + t) * H + h) * P;
+                double *yt = y + ((b * L + t) * H + h) * P;
+                for (int64_t p = 0; p < P; ++p) {
+                    double acc = 0.0;
+                    for (int64_t n = 0; n < N; ++n) {
+#if ORACLE_MUTANT == 20
+                        S[p * N + n] = a * (S[p * N + n] + dlt * Bt[n] * xt[p]); /* mutant: input decayed too */
+#elif ORACLE_MUTANT == 21
+                        S[p * N + n] = a * S[p * N + n] + Bt[n] * xt[p]; /* mutant: Delta dropped from the input */
+#else
+                        S[p * N + n] = a * S[p * N + n] + dlt * Bt[n] * xt[p];
+#endif
+                        acc += Ct[n] * S[p * N + n];
+                    }
+                    yt[p] = acc + (D ? D[h] : 0.0) * xt[p];
+                }
+            }
+            if (s_last)
+                for (int64_t i = 0; i < P * N; ++i) s_last[(b * H + h) * P * N + i] = S[i];
+        }
+    }
+    free(S);
+    return 0;
+}

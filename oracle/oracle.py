@@ -54,6 +54,8 @@ def _declare(lib: ctypes.CDLL) -> ctypes.CDLL:
     lib.oracle_causal_conv_f64.restype = ctypes.c_int
     lib.oracle_scan_bwd_f64.argtypes = [i64, i64, i64, i64] + [_dp] * 8 + [ctypes.c_int] + [_dp] * 12
     lib.oracle_scan_bwd_f64.restype = ctypes.c_int
+    lib.oracle_ssd_f64.argtypes = [i64] * 6 + [_dp] * 7 + [ctypes.c_int, _dp, _dp, _dp]
+    lib.oracle_ssd_f64.restype = ctypes.c_int
     return lib
 
 
@@ -171,6 +173,25 @@ def scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus_flag, dout, h0=None, 
     if rc != 0:
         raise ValueError(f"oracle_scan_bwd_f64 rejected its arguments (rc={rc})")
     return g
+
+
+def ssd(x, dt, A, B, C, D=None, dt_bias=None, softplus_flag=True, s0=None, lib=None):
+    """Mamba-2 SSD layer, recurrent view, fp64. x [b, L, H, P]; dt [b, L, H];
+    A, D, dt_bias [H]; B, C [b, L, G, N]; s0 [b, H, P, N] (zero if None).
+    Returns (y [b, L, H, P], s_last [b, H, P, N])."""
+    lib = lib or load_oracle()
+    x, dt, A, B, C, D, dt_bias, s0 = (_f64(a) for a in (x, dt, A, B, C, D, dt_bias, s0))
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    assert dt.shape == (batch, L, H) and A.shape == (H,) and B.shape == (batch, L, G, N) and C.shape == B.shape
+    assert s0 is None or s0.shape == (batch, H, P, N)
+    y = np.full(x.shape, np.nan)
+    last = np.full((batch, H, P, N), np.nan)
+    rc = lib.oracle_ssd_f64(batch, L, H, P, N, G, _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                            _ptr(dt_bias), int(bool(softplus_flag)), _ptr(s0), _ptr(y), _ptr(last))
+    if rc != 0:
+        raise ValueError(f"oracle_ssd_f64 rejected its arguments (rc={rc})")
+    return y, last
 
 
 def causal_conv(x, w, bias=None, x0=None, silu_flag=True, lib=None):

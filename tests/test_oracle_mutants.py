@@ -31,6 +31,9 @@ MUTANTS = {
     16: "gradient of silu missing its z*s*(1-s) term",
     17: "adjoint state decayed by its own token's A_bar",
     18: "gradient of Delta through A_bar dropped",
+    19: "SSD heads assigned to groups round-robin",
+    20: "SSD input term decayed by its own token",
+    21: "SSD Delta dropped from the input term",
 }
 
 

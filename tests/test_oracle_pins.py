@@ -22,6 +22,12 @@ mathematics) fix, written without the oracle's code:
 * the gradients of the scan (reverse mode) against central finite differences
   of the forward oracle along random directions, for every input (u, delta,
   A, B, C, D, z, delta_bias, h0) with a loss on both y and last_state;
+* the Mamba-2 SSD layer (blog, section 3: one model, a recurrent view and a
+  matrix view): the matrix view written out directly, y_t = sum_{s<=t}
+  (C_t . B_s) exp(A sum_{r=s+1..t} Delta_r) Delta_s x_s (+ initial state
+  and D terms), O(L^2); the reduction of a scalar-per-head transition to the
+  Mamba-1 oracle (every (head, p) a Mamba-1 channel whose A row is A_h); and
+  split/resume (the state is what passes between chunks);
 * the block's causal conv front-end (blog, section 2, block diagram: a short
   causal convolution per channel, then silu, feeds the SSM) against numpy's
   full convolution with the history prepended, one-hot filters as explicit
@@ -376,6 +382,72 @@ def pin_backward_finite_differences(lib):
     return worst
 
 
+def _ssd_case(rng, b=2, L=23, H=4, P=3, N=5, G=2):
+    return dict(x=rng.standard_normal((b, L, H, P)), dt=rng.standard_normal((b, L, H)),
+                A=-rng.uniform(0.3, 2.5, H), B=rng.standard_normal((b, L, G, N)),
+                C=rng.standard_normal((b, L, G, N)), D=rng.standard_normal(H), dt_bias=rng.uniform(-2.0, 0.0, H),
+                s0=rng.standard_normal((b, H, P, N)))
+
+
+def pin_ssd_matrix_view(lib):
+    rng = np.random.default_rng(23)
+    c = _ssd_case(rng)
+    y, last = oracle.ssd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["dt_bias"], True, c["s0"], lib=lib)
+    b, L, H, P = c["x"].shape
+    G = c["B"].shape[2]
+    ref = np.zeros_like(y)
+    ref_last = np.zeros_like(last)
+    for bi in range(b):
+        for h in range(H):
+            g = h // (H // G)
+            dlt = _softplus_ref(c["dt"][bi, :, h] + c["dt_bias"][h])
+            S = np.concatenate([[0.0], np.cumsum(dlt)])  # S[t+1] = sum_{r<=t} Delta_r
+            for t in range(L):
+                acc = np.exp(c["A"][h] * S[t + 1]) * (c["s0"][bi, h] @ c["C"][bi, t, g])  # initial state
+                for s_ in range(t + 1):
+                    w = (c["C"][bi, t, g] @ c["B"][bi, s_, g]) * np.exp(c["A"][h] * (S[t + 1] - S[s_ + 1])) * dlt[s_]
+                    acc = acc + w * c["x"][bi, s_, h]
+                ref[bi, t, h] = acc + c["D"][h] * c["x"][bi, t, h]
+            st = np.exp(c["A"][h] * S[L]) * c["s0"][bi, h]
+            for s_ in range(L):
+                st = st + np.exp(c["A"][h] * (S[L] - S[s_ + 1])) * dlt[s_] * np.outer(c["x"][bi, s_, h], c["B"][bi, s_, g])
+            ref_last[bi, h] = st
+    return max(_rel(y, ref), _rel(last, ref_last))
+
+
+def pin_ssd_is_mamba1_with_scalar_heads(lib):
+    rng = np.random.default_rng(24)
+    c = _ssd_case(rng)
+    y, last = oracle.ssd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["dt_bias"], True, c["s0"], lib=lib)
+    b, L, H, P = c["x"].shape
+    G, N = c["B"].shape[2], c["B"].shape[3]
+    worst = 0.0
+    for h in range(H):
+        g = h // (H // G)
+        u = np.transpose(c["x"][:, :, h, :], (0, 2, 1))               # [b, P, L]
+        delta = np.repeat(c["dt"][:, None, :, h], P, axis=1)           # [b, P, L]
+        A1 = np.full((P, N), c["A"][h])
+        B1 = np.transpose(c["B"][:, :, g, :], (0, 2, 1))               # [b, N, L]
+        C1 = np.transpose(c["C"][:, :, g, :], (0, 2, 1))
+        y1, l1 = oracle.scan(u, delta, A1, B1, C1, np.full(P, c["D"][h]), None, np.full(P, c["dt_bias"][h]),
+                             True, h0=c["s0"][:, h], lib=lib)
+        worst = max(worst, _rel(np.transpose(y[:, :, h, :], (0, 2, 1)), y1), _rel(last[:, h], l1))
+    return worst
+
+
+def pin_ssd_split_resume(lib):
+    rng = np.random.default_rng(25)
+    c = _ssd_case(rng, L=40)
+    m = 17
+    y, last = oracle.ssd(c["x"], c["dt"], c["A"], c["B"], c["C"], c["D"], c["dt_bias"], True, c["s0"], lib=lib)
+    sl = lambda k, a, z: c[k][:, a:z]  # noqa: E731
+    y1, l1 = oracle.ssd(sl("x", 0, m), sl("dt", 0, m), c["A"], sl("B", 0, m), sl("C", 0, m), c["D"], c["dt_bias"],
+                        True, c["s0"], lib=lib)
+    y2, l2 = oracle.ssd(sl("x", m, 40), sl("dt", m, 40), c["A"], sl("B", m, 40), sl("C", m, 40), c["D"],
+                        c["dt_bias"], True, l1, lib=lib)
+    return max(_rel(np.concatenate([y1, y2], axis=1), y), _rel(l2, last))
+
+
 PINS = {
     "softplus_silu": pin_softplus_silu,
     "lti_convolution": pin_lti_convolution,
@@ -390,6 +462,9 @@ PINS = {
     "conv_shift": pin_conv_shift,
     "conv_scan_split": pin_conv_scan_split,
     "backward_finite_differences": pin_backward_finite_differences,
+    "ssd_matrix_view": pin_ssd_matrix_view,
+    "ssd_is_mamba1_with_scalar_heads": pin_ssd_is_mamba1_with_scalar_heads,
+    "ssd_split_resume": pin_ssd_split_resume,
 }
 
 # Pins that compare against a numerical approximation carry their own bound.

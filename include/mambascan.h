@@ -268,6 +268,41 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
                            int *dev_status, ms_stream_t stream);
 
 /*
+ * Mamba-2 state space duality (SSD) layer, forward ('Mamba-1/2/3 Markdown図解'
+ * blog, section 3: the same model has a recurrent view and a matrix view
+ * computed chunk by chunk, matrix products inside a chunk and the state
+ * passed between chunks; the transition is a scalar times the identity in a
+ * head). For batch b, head h with head dim P and state N, and group
+ * g = h / (nheads / ngroups) whose B and C it uses:
+ *     Delta_t = softplus(dt[b,t,h] + dt_bias[h])   (plain sum when the flag is 0)
+ *     S_t[p][n] = exp(Delta_t A[h]) S_{t-1}[p][n] + Delta_t x[b,t,h,p] B[b,t,g,n]
+ *     y[b,t,h,p] = sum_n C[b,t,g,n] S_t[p][n] + D[h] x[b,t,h,p]
+ * Layouts (element strides; the last dimension of each array is dense):
+ *   x, y [batch, seqlen, nheads, headdim]; dt [batch, seqlen, nheads];
+ *   B, C [batch, seqlen, ngroups, dstate]; A, D, dt_bias [nheads] fp32;
+ *   initial_state, final_state [batch, nheads, headdim, dstate] fp32, dense.
+ * This version runs headdim 64 and dstate 128 (the Mamba-2 layer sizes) with
+ * bf16 x, dt, B, C (MS_ERR_SHAPE / MS_ERR_DTYPE otherwise); x, B, C rows must
+ * be 16-byte aligned and y rows aligned to two elements (MS_ERR_ALIGN).
+ * y is fp32 or bf16 (out_dtype). D, dt_bias, initial_state, final_state may
+ * be NULL.
+ */
+typedef struct {
+    int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
+    int64_t x_sb, x_sl, x_sh;
+    int64_t dt_sb, dt_sl;
+    int64_t B_sb, B_sl, B_sg;
+    int64_t C_sb, C_sl, C_sg;
+    int64_t y_sb, y_sl, y_sh;
+    int32_t in_dtype, out_dtype;
+} ms_ssd_dims;
+
+int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
+                   const float *D, const float *dt_bias, int softplus_flag, const float *initial_state,
+                   void *y, float *final_state, const ms_ssd_dims *dims, int *dev_status,
+                   ms_stream_t stream);
+
+/*
  * Sizes and strides of one decode step.
  *   x, delta, z, y : [batch, dim]     element (b,d) at b*x_sb + d
  *   B, C           : [batch, dstate]  element (b,n) at b*x_sb + n

@@ -46,6 +46,13 @@ class ConvDims(ctypes.Structure):
                 ("silu", ctypes.c_int32)]
 
 
+class SsdDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "seqlen", "nheads", "headdim", "dstate", "ngroups", "x_sb", "x_sl", "x_sh", "dt_sb", "dt_sl",
+        "B_sb", "B_sl", "B_sg", "C_sb", "C_sl", "C_sg", "y_sb", "y_sl", "y_sh")] + [
+        ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
 class MambaScanError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: status {code} ({mamba_status_string(code)})")
@@ -91,6 +98,8 @@ def library() -> ctypes.CDLL:
         lib.mamba_scan_bwd_noalloc.argtypes = ([_vp] * 8 + [ctypes.c_int] + [_vp] * 12 +
                                                [ctypes.POINTER(ScanDims), _vp, _vp])
         lib.mamba_scan_bwd_noalloc.restype = ctypes.c_int
+        lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
+        lib.mamba2_ssd_fwd.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
                                                        _vp, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
@@ -163,6 +172,12 @@ def mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus_flag, i
     return library().mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, int(softplus_flag),
                                             initial_state, dout, dlast, du, ddelta, dA, dB, dC, dD, dz,
                                             ddelta_bias, dinitial_state, ctypes.byref(dims), dev_status, stream)
+
+
+def mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, softplus_flag, initial_state, y, final_state, dims: SsdDims,
+                   dev_status, stream) -> int:
+    return library().mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, int(softplus_flag), initial_state, y, final_state,
+                                    ctypes.byref(dims), dev_status, stream)
 
 
 def mamba_conv_scan_fwd(x, conv_w, conv_b, conv_x0, u_out, cdims: ConvDims, delta, A, B, C, D, z,
@@ -377,6 +392,31 @@ def scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, 
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba_scan_bwd_noalloc")
     return g
+
+
+def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial_state=None,
+            out_dtype=None, return_final_state: bool = True, y=None, stream=None, dev_status=None):
+    """Mamba-2 SSD layer forward on torch CUDA tensors: x [b, L, H, P], dt
+    [b, L, H], B/C [b, L, G, N] (bf16), A/D/dt_bias [H] fp32. Returns (y,
+    final_state [b, H, P, N] or None)."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    batch, L, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    for t, n in ((x, "x"), (dt, "dt"), (B, "B"), (C, "C")):
+        _inner_contiguous(t, n)
+    if y is None:
+        y = torch.empty((batch, L, H, P), dtype=out_dtype, device=x.device)
+    fs = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device) if return_final_state else None
+    dims = SsdDims(batch, L, H, P, N, G, x.stride(0), x.stride(1), x.stride(2), dt.stride(0), dt.stride(1),
+                   B.stride(0), B.stride(1), B.stride(2), C.stride(0), C.stride(1), C.stride(2),
+                   y.stride(0), y.stride(1), y.stride(2), _dtype_code(x), _dtype_code(y))
+    rc = mamba2_ssd_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias), softplus,
+                        _ptr(initial_state), _ptr(y), _ptr(fs), dims, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba2_ssd_fwd")
+    return y, fs
 
 
 def update_dims_for(state, x, delta, B, C, z, y) -> UpdateDims:

@@ -397,6 +397,61 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
                           need > 0 ? MS_BWD_NOALLOC_MAX_BYTES : 0, dev_status, stream);
 }
 
+int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
+                   const float *dt_bias, int softplus_flag, const float *initial_state, void *y, float *final_state,
+                   const ms_ssd_dims *dm, int *dev_status, ms_stream_t stream) {
+    (void)dev_status;
+    if (!dm) return MS_ERR_NULL;
+    if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) || (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
+        return MS_ERR_DTYPE;
+    if (dm->batch < 0 || dm->seqlen < 0 || dm->nheads < 1 || dm->ngroups < 1 || dm->nheads % dm->ngroups != 0 ||
+        dm->headdim < 1 || dm->dstate < 1)
+        return MS_ERR_SHAPE;
+    if (dm->x_sb < 0 || dm->x_sl < 0 || dm->x_sh < 0 || dm->dt_sb < 0 || dm->dt_sl < 0 || dm->B_sb < 0 ||
+        dm->B_sl < 0 || dm->B_sg < 0 || dm->C_sb < 0 || dm->C_sl < 0 || dm->C_sg < 0 || dm->y_sb < 0 ||
+        dm->y_sl < 0 || dm->y_sh < 0)
+        return MS_ERR_STRIDE;
+    if (!ms::ssd_shape_supported(dm->headdim, dm->dstate)) return MS_ERR_SHAPE;
+    if (dm->in_dtype != MS_BF16) return MS_ERR_DTYPE;
+    if (dm->batch == 0) return MS_OK;
+    if (!A) return MS_ERR_NULL;
+    if (dm->seqlen > 0 && (!x || !dt || !B || !C || !y)) return MS_ERR_NULL;
+    const int eo = elem_bytes(dm->out_dtype);
+    auto rows16 = [](const void *p, int64_t s1, int64_t s2, int64_t s3) {
+        return p == nullptr || (aligned(p, 16) && (s1 * 2) % 16 == 0 && (s2 * 2) % 16 == 0 && (s3 * 2) % 16 == 0);
+    };
+    if (!rows16(x, dm->x_sb, dm->x_sl, dm->x_sh) || !rows16(B, dm->B_sb, dm->B_sl, dm->B_sg) ||
+        !rows16(C, dm->C_sb, dm->C_sl, dm->C_sg) || (dt && !aligned(dt, 2)) || !aligned(A, 4) ||
+        (D && !aligned(D, 4)) || (dt_bias && !aligned(dt_bias, 4)) || (initial_state && !aligned(initial_state, 4)) ||
+        (final_state && !aligned(final_state, 4)) ||
+        (y && (!aligned(y, 2 * eo) || dm->y_sb % 2 || dm->y_sl % 2 || dm->y_sh % 2)))
+        return MS_ERR_ALIGN;
+    if (dm->seqlen > 0) {
+        const int64_t L = dm->seqlen, H = dm->nheads, G = dm->ngroups;
+        if (max_offset3(dm->batch, dm->x_sb, L, dm->x_sl, 1) < 0 || max_offset3(H, dm->x_sh, 1, 0, 64) < 0 ||
+            max_offset3(dm->batch, dm->y_sb, L, dm->y_sl, 1) < 0 || max_offset3(H, dm->y_sh, 1, 0, 64) < 0 ||
+            max_offset3(dm->batch, dm->dt_sb, L, dm->dt_sl, H) < 0 ||
+            max_offset3(dm->batch, dm->B_sb, L, dm->B_sl, 1) < 0 || max_offset3(G, dm->B_sg, 1, 0, 128) < 0 ||
+            max_offset3(dm->batch, dm->C_sb, L, dm->C_sl, 1) < 0 || max_offset3(G, dm->C_sg, 1, 0, 128) < 0)
+            return MS_ERR_SHAPE;
+    }
+    if (dm->seqlen == 0 && !final_state) return MS_OK;
+    ms::SsdArgs a{};
+    a.x = x; a.dt = dt; a.B = B; a.C = C; a.A = A; a.D = D; a.dt_bias = dt_bias; a.s0 = initial_state;
+    a.y = y; a.s_last = final_state;
+    a.batch = dm->batch; a.L = dm->seqlen; a.H = dm->nheads; a.G = dm->ngroups;
+    a.x_sb = dm->x_sb; a.x_sl = dm->x_sl; a.x_sh = dm->x_sh; a.dt_sb = dm->dt_sb; a.dt_sl = dm->dt_sl;
+    a.B_sb = dm->B_sb; a.B_sl = dm->B_sl; a.B_sg = dm->B_sg; a.C_sb = dm->C_sb; a.C_sl = dm->C_sl;
+    a.C_sg = dm->C_sg; a.y_sb = dm->y_sb; a.y_sl = dm->y_sl; a.y_sh = dm->y_sh;
+    a.softplus = softplus_flag ? 1 : 0;
+    cudaError_t e = ms::launch_ssd_fwd(a, dm->out_dtype == MS_BF16, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
 int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,
                        const void *C, const float *D, const void *z, const float *delta_bias,
                        int softplus_flag, void *y, const ms_update_dims *dm, int *dev_status,

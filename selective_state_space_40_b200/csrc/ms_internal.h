@@ -54,6 +54,20 @@ struct BwdArgs {
     int vec_bc;   // dB/dC rows allow 16-byte atomics (L % 4 == 0, aligned base)
 };
 
+// Arguments of the Mamba-2 SSD forward (bf16 x, dt, B, C; fp32 A, D, dt_bias,
+// states). Element strides; the innermost dimension of every array is dense.
+struct SsdArgs {
+    const void *x, *dt, *B, *C;
+    const float *A, *D, *dt_bias, *s0;
+    void *y;
+    float *s_last;
+    int64_t batch, L, H, G;
+    int64_t x_sb, x_sl, x_sh, dt_sb, dt_sl, B_sb, B_sl, B_sg, C_sb, C_sl, C_sg, y_sb, y_sl, y_sh;
+    int softplus;
+};
+bool ssd_shape_supported(int64_t headdim, int64_t dstate);
+cudaError_t launch_ssd_fwd(const SsdArgs &a, bool out_bf16, cudaStream_t stream);
+
 // Launch shape chosen on the host for one scan call.
 struct ScanPlan {
     int lanes_per_channel;  // G: lanes sharing one channel (1, 2, 4, 8), 16/G states each

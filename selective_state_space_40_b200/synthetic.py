@@ -125,6 +125,40 @@ def conv_params(w: ScanWorkload, width: int = 4, seed: Optional[int] = None) -> 
     return dict(conv_w=conv_w, conv_b=conv_b, conv_x0=conv_x0)
 
 
+@dataclass(frozen=True)
+class SsdWorkload:
+    """A Mamba-2 SSD layer: x [b, L, H, P], dt [b, L, H], B/C [b, L, G, N]."""
+    name: str
+    batch: int
+    seqlen: int
+    nheads: int
+    headdim: int
+    dstate: int
+    ngroups: int
+    in_dtype: torch.dtype = torch.bfloat16
+    seed: int = 0
+
+
+# Mamba-2 2.7B-class layer: d_model 2560, expand 2 -> 80 heads of 64, d_state 128.
+SSD_2P7B = SsdWorkload("mamba2-2.7b-class b4 L2048 H80 P64 N128 G1 bf16", 4, 2048, 80, 64, 128, 1)
+
+
+def ssd_inputs(w: SsdWorkload, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
+    """CPU tensors drawn in the order x, dt, B, C (N(0,1), stored in
+    ``w.in_dtype``), then A = -U[1, 16] per head, dt_bias = log(expm1(U)) with
+    U ~ U[1e-3, 0.1], D ~ N(1, 0.1) (fp32)."""
+    g = torch.Generator().manual_seed(w.seed if seed is None else seed)
+    b, L, H, P, N, G = w.batch, w.seqlen, w.nheads, w.headdim, w.dstate, w.ngroups
+    x = _normal(g, (b, L, H, P), w.in_dtype)
+    dt = _normal(g, (b, L, H), w.in_dtype)
+    B = _normal(g, (b, L, G, N), w.in_dtype)
+    C = _normal(g, (b, L, G, N), w.in_dtype)
+    A = -(1.0 + 15.0 * torch.rand(H, generator=g, dtype=torch.float32))
+    dt_bias = _inv_softplus_uniform(g, H, 1e-3, 0.1)
+    D = _normal(g, (H,), torch.float32, std=0.1, mean=1.0)
+    return dict(x=x, dt=dt, B=B, C=C, A=A, dt_bias=dt_bias, D=D)
+
+
 def decode_params(w: DecodeWorkload) -> Dict[str, torch.Tensor]:
     """state0 [b, d, N] fp32 ~ N(0, 0.1); A, D, delta_bias as the 130M-class layer."""
     g = torch.Generator().manual_seed(w.seed)

@@ -202,6 +202,30 @@ def test_bwd_noalloc_rejects_oversize_and_bad_arguments(lib):
     assert call(_dims(batch=0)) == mb.MS_OK
 
 
+def _sdims(**kw):
+    d = dict(batch=2, seqlen=64, nheads=4, headdim=64, dstate=128, ngroups=1, x_sb=64 * 256, x_sl=256, x_sh=64,
+             dt_sb=256, dt_sl=4, B_sb=64 * 128, B_sl=128, B_sg=128, C_sb=64 * 128, C_sl=128, C_sg=128,
+             y_sb=64 * 256, y_sl=256, y_sh=64, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)
+    d.update(kw)
+    return mb.SsdDims(**d)
+
+
+def test_ssd_rejects_bad_arguments(lib):
+    def call(dims, x=FAKE, y=FAKE, B=FAKE):
+        return mb.mamba2_ssd_fwd(x, FAKE, FAKE, B, FAKE, None, None, 1, None, y, None, dims, None, None)
+    assert call(_sdims(headdim=32)) == mb.MS_ERR_SHAPE
+    assert call(_sdims(dstate=64)) == mb.MS_ERR_SHAPE
+    assert call(_sdims(nheads=5, ngroups=2)) == mb.MS_ERR_SHAPE
+    assert call(_sdims(in_dtype=mb.MS_F32)) == mb.MS_ERR_DTYPE
+    assert call(_sdims(out_dtype=4)) == mb.MS_ERR_DTYPE
+    assert call(_sdims(x_sl=-1)) == mb.MS_ERR_STRIDE
+    assert call(_sdims(), x=None) == mb.MS_ERR_NULL
+    assert call(_sdims(), x=FAKE + 2) == mb.MS_ERR_ALIGN      # rows need 16-byte alignment
+    assert call(_sdims(B_sl=132)) == mb.MS_ERR_ALIGN         # row stride not a multiple of 8 elements
+    assert call(_sdims(), y=FAKE + 4) == mb.MS_ERR_ALIGN      # fp32 pairs need 8-byte alignment
+    assert call(_sdims(batch=0)) == mb.MS_OK
+
+
 def _udims(**kw):
     d = dict(batch=4, dim=8, dstate=16, x_sb=8, delta_sb=8, z_sb=8, y_sb=8, B_sb=16, C_sb=16,
              state_sb=128, state_sd=16, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)

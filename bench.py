@@ -64,6 +64,23 @@ def bwd_bytes(batch, dim, dstate, seqlen, in_bytes, out_bytes):
             + batch * dim * nck * dstate * 4 + batch * dim * dstate * 4 + 2 * (dim * dstate * 4 + 2 * dim * 4))
 
 
+def ssd_bytes(batch, seqlen, nheads, headdim, dstate, ngroups, in_bytes, out_bytes):
+    """Minimum HBM bytes of one SSD layer forward: x and dt read, y written,
+    B and C read once per (batch, token, group), A/D/dt_bias read and the
+    final state written."""
+    return (batch * seqlen * nheads * (headdim * (in_bytes + out_bytes) + in_bytes)
+            + batch * seqlen * ngroups * 2 * dstate * in_bytes + 3 * nheads * 4
+            + batch * nheads * headdim * dstate * 4)
+
+
+def ssd_flops(batch, seqlen, nheads, headdim, dstate, chunk=32):
+    """Multiply-adds x 2 of the chunked matrix view per (batch, head, chunk):
+    C S_in (Q N P), C B^T (Q Q N), G' X (Q Q P), B'^T X (N Q P)."""
+    nch = (seqlen + chunk - 1) // chunk
+    per = 2 * (chunk * dstate * headdim + chunk * chunk * dstate + chunk * chunk * headdim + dstate * chunk * headdim)
+    return batch * nheads * nch * per
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -72,6 +89,14 @@ def measured_peaks():
         return float(p["hbm_gbs"]), "measured"
     except Exception:
         return FALLBACK_HBM_GBS, "fallback"
+
+
+def measured_bf16_tflops():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"])
+    except Exception:
+        return 1590.0
 
 
 def csrc_digest():
@@ -440,6 +465,32 @@ def main(argv=None):
     bbytes = bwd_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4)
     del dout
 
+    # ---- Mamba-2 SSD layer (2.7B-class): chunked matrix view on the tensor cores
+    sw = syn.SSD_2P7B
+    ssd_in = [{k: v.to(dev) for k, v in syn.ssd_inputs(sw).items()} for _ in range(2)]
+    ssd_y = torch.empty(sw.batch, sw.seqlen, sw.nheads, sw.headdim, dtype=torch.float32, device=dev)
+    ssd_steps = 20
+
+    def ssd_step(i):
+        g = ssd_in[i & 1]
+        mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True, y=ssd_y,
+                   return_final_state=False, stream=stream)
+
+    for i in range(3):
+        ssd_step(i)
+    sev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(ssd_steps)]
+    torch.cuda.synchronize()
+    for i in range(ssd_steps):
+        sev[i][0].record(stream)
+        ssd_step(i)
+        sev[i][1].record(stream)
+    torch.cuda.synchronize()
+    ssd_ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in sev), world, dev)
+    sbytes = ssd_bytes(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate, sw.ngroups, 2, 4) \
+        - sw.batch * sw.nheads * sw.headdim * sw.dstate * 4  # no final state requested
+    sflops = ssd_flops(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate)
+    del ssd_in
+
     # ---- CPU baseline: the oracle on this host's cores, whole passes over the
     # workload repeated until about ten seconds of wall time have gone by
     cpu = None
@@ -485,6 +536,13 @@ def main(argv=None):
                          "bwd_ms": bwd_ms, "bwd_bytes": bbytes, "value": bbytes / (bwd_ms * 1e-3) / 1e9,
                          "unit": "GB/s", "frac": bbytes / (bwd_ms * 1e-3) / 1e9 / peak,
                          "timing": f"mean of {bwd_steps} event-timed (forward with saved states, backward) pairs"},
+            "ssd": {"workload": sw.name, "ms": ssd_ms, "bytes": sbytes,
+                    "value": sbytes / (ssd_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "frac_hbm": sbytes / (ssd_ms * 1e-3) / 1e9 / peak,
+                    "tflops": sflops / (ssd_ms * 1e-3) / 1e12, "algorithmic_flops": sflops,
+                    "frac_tensor": sflops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops(),
+                    "bound": "hbm (bytes / 6443 GB/s exceed flops / bf16 peak)",
+                    "timing": "mean of per-launch event pairs, two rotating input sets"},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

@@ -14,12 +14,17 @@
 // i.e. four products per chunk: Y = C S_in (scaled by row), G = C B^T (masked
 // and scaled), Y += G' X, S_out = exp(cs_Q) S_in + B'^T X.
 //
-// One CTA of 4 warps walks the chunks of one (b, h) in order; the state lives
-// in the warps' tensor-core accumulators (fp32) for the whole sequence. The
-// products run on the tensor cores as bf16 x bf16 -> fp32 (mma.sync
-// m16n8k16). Operands that are not bf16 inputs (the scaled G', B' and the
-// state) are split into a high and a low bf16 part, v = hi + lo, and both
-// parts are multiplied, which keeps about 16 significant bits.
+// One CTA of 4 warps walks the chunks of one (b, h) in order. Everything is
+// computed transposed, S^T [P x N] and Y^T [P x Q]: warp w owns rows
+// p in [16w, 16w+16) of both, so the state stays in its tensor-core
+// accumulators (fp32) for the whole sequence and feeds the next chunk's
+// S^T C^T product directly as register operands (an m16n8 accumulator pair
+// has the layout of an m16n8k16 A operand). The products run on the tensor
+// cores as bf16 x bf16 -> fp32 (mma.sync m16n8k16). Operands that are not
+// bf16 inputs (the scaled G', B' and the state) are split into a high and a
+// low bf16 part, v = hi + lo, and both parts are multiplied, which keeps
+// about 16 significant bits. The next chunk's inputs are copied in
+// asynchronously while the current one computes.
 
 #include <cstdint>
 
@@ -39,17 +44,36 @@ constexpr int kST = kSW * 32;     // threads
 // words of one fragment load fall in 32 distinct banks.
 constexpr int kLdN = kN + 8;      // rows of K = N
 constexpr int kLdQ = kQ + 8;      // rows of K = Q
+static_assert(kQ == 32, "warp 0 handles one token of the chunk per lane");
 
 struct SsdSmem {
-    __nv_bfloat16 C[kQ][kLdN];        // C_t [t][n]
-    __nv_bfloat16 B[kQ][kLdN];        // B_s [s][n]
+    __nv_bfloat16 C[2][kQ][kLdN];     // C_t [t][n], this chunk and the next (copies in flight)
+    __nv_bfloat16 B[2][kQ][kLdN];     // B_s [s][n]
+    __nv_bfloat16 X[2][kQ][kP];       // x [s][p] as loaded
     __nv_bfloat16 Xt[kP][kLdQ];       // x^T [p][s]
     __nv_bfloat16 G[2][kQ][kLdQ];     // G' hi / lo [t][s]
     __nv_bfloat16 Bt[2][kN][kLdQ];    // B'^T hi / lo [n][s]
-    __nv_bfloat16 S[2][kP][kLdN];     // state^T hi / lo [p][n]
     float dl[kQ];                     // Delta_t
     float cs[kQ];                     // A sum_{r<=t} Delta_r
+    float wq[kQ];                     // exp(cs_Q - cs_s) Delta_s
+    float ecs[kQ];                    // exp(cs_t)
 };
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// hi and lo bf16 pairs of (x, y): x ~ hi.x + lo.x
+__device__ __forceinline__ void split_pair(float x, float y, uint32_t &hi, uint32_t &lo) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(x, y);
+    hi = *reinterpret_cast<uint32_t *>(&h);
+    lo = pack_bf16(x - __low2float(h), y - __high2float(h));
+}
+
+__device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc, int src_bytes) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(gsrc), "r"(src_bytes) : "memory");
+}
 
 __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -83,7 +107,7 @@ __device__ __forceinline__ float ld1(const TIn *p) {
 }
 
 template <typename TOut>
-__global__ void __launch_bounds__(kST, 2) ssd_fwd_kernel(const SsdArgs a) {
+__global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SsdSmem &sm = *reinterpret_cast<SsdSmem *>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -102,100 +126,114 @@ __global__ void __launch_bounds__(kST, 2) ssd_fwd_kernel(const SsdArgs a) {
     const __nv_bfloat16 *Cb = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
     TOut *yb = static_cast<TOut *>(a.y) + b * a.y_sb + h * a.y_sh;
 
-    // State accumulators: warp w holds rows n in [32w, 32w+32) (two m-tiles)
-    // and all 64 columns p (eight n-tiles): element (n, p) of S^T... i.e.
-    // S[p][n] sits at n = 32w + 16mt + gid (+8), p = 8nt + 2tig (+1).
-    float sacc[2][8][4];
+    // S^T accumulators: warp w holds rows p in [16w, 16w+16) and all 128
+    // columns n (16 n-tiles): sacc[j][e] is S[p][n] with p = 16w + gid (+8
+    // for e >= 2), n = 8j + 2tig (+1 for odd e).
+    const int pw = 16 * warp;
+    float sacc[16][4];
     const float *s0 = a.s0 ? a.s0 + (b * a.H + h) * kP * kN : nullptr;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int j = 0; j < 16; ++j)
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int n = 32 * warp + 16 * mt + gid + (e >= 2 ? 8 : 0);
-                const int p = 8 * nt + 2 * tig + (e & 1);
-                sacc[mt][nt][e] = s0 ? __ldg(s0 + p * kN + n) : 0.0f;
-            }
-    // state^T into shared memory as hi/lo bf16 [p][n]
-    auto store_state = [&]() {
-#pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int n = 32 * warp + 16 * mt + gid + (e >= 2 ? 8 : 0);
-                    const int p = 8 * nt + 2 * tig + (e & 1);
-                    split_bf16(sacc[mt][nt][e], sm.S[0][p][n], sm.S[1][p][n]);
-                }
-    };
-    store_state();
+        for (int e = 0; e < 4; ++e) {
+            const int p = pw + gid + (e >= 2 ? 8 : 0);
+            const int n = 8 * j + 2 * tig + (e & 1);
+            sacc[j][e] = s0 ? __ldg(s0 + p * kN + n) : 0.0f;
+        }
 
     const int64_t nch = (L + kQ - 1) / kQ;
-    for (int64_t ck = 0; ck < nch; ++ck) {
+    // Chunk inputs arrive by asynchronous copies one chunk ahead (rows past L
+    // are zero-filled); dt goes through a register, one token per thread of
+    // warp 0.
+    auto issue_chunk = [&](int64_t ck, int buf) {
         const int64_t t0 = ck * kQ;
-        __syncthreads();  // everyone is done with the previous chunk's tiles
-        // ---- load the chunk: C, B rows (16-byte pieces), x transposed, Delta
         for (int i = tid; i < kQ * (kN / 8); i += kST) {
             const int t = i / (kN / 8), q = i % (kN / 8);
-            uint4 vc = make_uint4(0u, 0u, 0u, 0u), vb = vc;
-            if (t0 + t < L) {
-                vc = __ldg(reinterpret_cast<const uint4 *>(Cb + (t0 + t) * a.C_sl) + q);
-                vb = __ldg(reinterpret_cast<const uint4 *>(Bb + (t0 + t) * a.B_sl) + q);
-            }
-            *reinterpret_cast<uint4 *>(&sm.C[t][8 * q]) = vc;
-            *reinterpret_cast<uint4 *>(&sm.B[t][8 * q]) = vb;
+            const bool in = t0 + t < L;
+            const int64_t tt = in ? t0 + t : 0;
+            cp_async16(&sm.C[buf][t][8 * q], Cb + tt * a.C_sl + 8 * q, in ? 16 : 0);
+            cp_async16(&sm.B[buf][t][8 * q], Bb + tt * a.B_sl + 8 * q, in ? 16 : 0);
         }
         for (int i = tid; i < kQ * (kP / 8); i += kST) {
             const int t = i / (kP / 8), q = i % (kP / 8);
-            uint4 vx = make_uint4(0u, 0u, 0u, 0u);
-            if (t0 + t < L) vx = __ldg(reinterpret_cast<const uint4 *>(xb + (t0 + t) * a.x_sl) + q);
-            const __nv_bfloat16 *e = reinterpret_cast<const __nv_bfloat16 *>(&vx);
-#pragma unroll
-            for (int k = 0; k < 8; ++k) sm.Xt[8 * q + k][t] = e[k];
+            const bool in = t0 + t < L;
+            const int64_t tt = in ? t0 + t : 0;
+            cp_async16(&sm.X[buf][t][8 * q], xb + tt * a.x_sl + 8 * q, in ? 16 : 0);
         }
-        if (tid < kQ) {
-            const int64_t t = t0 + tid;
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    float dt_next = 0.0f;
+    auto load_dt = [&](int64_t ck) {
+        const int64_t t = ck * kQ + lane;
+        dt_next = (warp == 0 && t < L) ? ld1(dtb + t * a.dt_sl) : 0.0f;
+    };
+    if (nch > 0) {
+        issue_chunk(0, 0);
+        load_dt(0);
+    }
+    for (int64_t ck = 0; ck < nch; ++ck) {
+        const int64_t t0 = ck * kQ;
+        const int buf = (int)(ck & 1);
+        asm volatile("cp.async.wait_group 0;" ::: "memory");
+        __syncthreads();  // chunk ck in buf for everyone; the previous chunk's tiles are free
+        // ---- x^T for the products; warp 0: Delta, its decay prefix and weights
+        for (int i = tid; i < kQ * kP; i += kST) {
+            const int t = i / kP, p = i % kP;
+            sm.Xt[p][t] = sm.X[buf][t][p];
+        }
+        if (warp == 0) {
             float d = 0.0f;
-            if (t < L) {
-                const float v = ld1(dtb + t * a.dt_sl) + bias;
+            if (t0 + lane < L) {
+                const float v = dt_next + bias;
                 d = sp ? softplus_f(v) : v;
             }
-            sm.dl[tid] = d;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            float c = 0.0f;
-            for (int t = 0; t < kQ; ++t) {
-                c = fmaf(Ah, sm.dl[t], c);
-                sm.cs[t] = c;
+            float c = Ah * d;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, c, off);
+                if (lane >= off) c += o;
             }
+            const float cend = __shfl_sync(0xffffffffu, c, kQ - 1);
+            sm.dl[lane] = d;
+            sm.cs[lane] = c;
+            sm.wq[lane] = __expf(cend - c) * d;
+            sm.ecs[lane] = __expf(c);
+        }
+        // next chunk's copies run under this chunk's products
+        if (ck + 1 < nch) {
+            issue_chunk(ck + 1, buf ^ 1);
+            load_dt(ck + 1);
         }
         __syncthreads();
         const float cs_end = sm.cs[kQ - 1];
 
-        // ---- Y = exp(cs_t) C_t . S_in  (warp: rows 16(w%2).., cols 32(w/2)..)
-        const int ym = 16 * (warp & 1), yn = 32 * (warp >> 1);
+        // ---- Y^T = S_in^T C^T, columns scaled by exp(cs_t): the state
+        // accumulators are the A operand (hi and lo parts), C rows the B operand
         float yacc[4][4];
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) yacc[nt][e] = 0.0f;
 #pragma unroll
-        for (int k0 = 0; k0 < kN; k0 += 16)
-#pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-                    mma_tile(yacc[nt], &sm.C[0][0], kLdN, ym, &sm.S[part][0][0], kLdN, yn + 8 * nt, k0, gid, tig);
-        {
-            const float e0 = __expf(sm.cs[ym + gid]), e1 = __expf(sm.cs[ym + gid + 8]);
+        for (int kk = 0; kk < kN / 16; ++kk) {
+            uint32_t ah[4], al[4];
+            split_pair(sacc[2 * kk][0], sacc[2 * kk][1], ah[0], al[0]);
+            split_pair(sacc[2 * kk][2], sacc[2 * kk][3], ah[1], al[1]);
+            split_pair(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1], ah[2], al[2]);
+            split_pair(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3], ah[3], al[3]);
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-                yacc[nt][0] *= e0; yacc[nt][1] *= e0;
-                yacc[nt][2] *= e1; yacc[nt][3] *= e1;
+                const __nv_bfloat16 *br = &sm.C[buf][8 * nt + gid][16 * kk + 2 * tig];
+                const uint32_t b0 = ld32(br), b1 = ld32(br + 8);
+                mma_bf16(yacc[nt], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                mma_bf16(yacc[nt], al[0], al[1], al[2], al[3], b0, b1);
             }
+        }
+#pragma unroll
+        for (int nt = 0; nt < 4; ++nt) {
+            const float e0 = sm.ecs[8 * nt + 2 * tig], e1 = sm.ecs[8 * nt + 2 * tig + 1];
+            yacc[nt][0] *= e0; yacc[nt][1] *= e1;
+            yacc[nt][2] *= e0; yacc[nt][3] *= e1;
         }
 
         // ---- G = C B^T, masked and scaled: G'_ts = G exp(cs_t - cs_s) Delta_s, s <= t
@@ -211,7 +249,7 @@ __global__ void __launch_bounds__(kST, 2) ssd_fwd_kernel(const SsdArgs a) {
                 for (int k0 = 0; k0 < kN; k0 += 16)
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
-                        mma_tile(gacc[nt], &sm.C[0][0], kLdN, gm, &sm.B[0][0], kLdN, gn + 8 * nt, k0, gid, tig);
+                        mma_tile(gacc[nt], &sm.C[buf][0][0], kLdN, gm, &sm.B[buf][0][0], kLdN, gn + 8 * nt, k0, gid, tig);
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -232,76 +270,63 @@ __global__ void __launch_bounds__(kST, 2) ssd_fwd_kernel(const SsdArgs a) {
         }
         __syncthreads();
 
-        // ---- Y += G' X over the causal part, then y = Y + D x
+        // ---- Y^T += X^T G'^T over the causal part, then y = Y + D x
 #pragma unroll
-        for (int k0 = 0; k0 < kQ; k0 += 16) {
-            if (k0 > ym + 15) continue;
+        for (int k0 = 0; k0 < kQ; k0 += 16)
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt)
+            for (int nt = 0; nt < 4; ++nt) {
+                if (k0 > 8 * nt + 7) continue;  // s > t for the whole tile
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
-                    mma_tile(yacc[nt], &sm.G[part][0][0], kLdQ, ym, &sm.Xt[0][0], kLdQ, yn + 8 * nt, k0, gid, tig);
-        }
+                    mma_tile(yacc[nt], &sm.Xt[0][0], kLdQ, pw, &sm.G[part][0][0], kLdQ, 8 * nt, k0, gid, tig);
+            }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
-            for (int r = 0; r < 2; ++r) {
-                const int t = ym + gid + 8 * r;
-                const int p = yn + 8 * nt + 2 * tig;
+            for (int e = 0; e < 4; ++e) {
+                const int p = pw + gid + (e >= 2 ? 8 : 0);
+                const int t = 8 * nt + 2 * tig + (e & 1);
                 if (t0 + t < L) {
-                    const float v0 = yacc[nt][2 * r] + Dh * __bfloat162float(sm.Xt[p][t]);
-                    const float v1 = yacc[nt][2 * r + 1] + Dh * __bfloat162float(sm.Xt[p + 1][t]);
+                    const float v = yacc[nt][e] + Dh * __bfloat162float(sm.Xt[p][t]);
                     TOut *dst = yb + (t0 + t) * a.y_sl + p;
-                    if constexpr (sizeof(TOut) == 4) {
-                        *reinterpret_cast<float2 *>(dst) = make_float2(v0, v1);
-                    } else {
-                        *reinterpret_cast<__nv_bfloat162 *>(dst) = __floats2bfloat162_rn(v0, v1);
-                    }
+                    if constexpr (sizeof(TOut) == 4) *dst = v;
+                    else *dst = __float2bfloat16_rn(v);
                 }
             }
 
         // ---- B'^T [n][s] = exp(cs_Q - cs_s) Delta_s B_s[n], hi / lo
         for (int i = tid; i < kN * kQ; i += kST) {
             const int n = i / kQ, s = i % kQ;
-            const float v = __bfloat162float(sm.B[s][n]) * __expf(cs_end - sm.cs[s]) * sm.dl[s];
+            const float v = __bfloat162float(sm.B[buf][s][n]) * sm.wq[s];
             split_bf16(v, sm.Bt[0][n][s], sm.Bt[1][n][s]);
         }
         __syncthreads();
 
-        // ---- S_out = exp(cs_Q) S_in + B'^T X  (rows n, columns p)
+        // ---- S_out^T = exp(cs_Q) S_in^T + X^T B'  (rows p, columns n)
         const float decay = __expf(cs_end);
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int j = 0; j < 16; ++j)
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) sacc[mt][nt][e] *= decay;
+            for (int e = 0; e < 4; ++e) sacc[j][e] *= decay;
 #pragma unroll
         for (int k0 = 0; k0 < kQ; k0 += 16)
 #pragma unroll
-            for (int mt = 0; mt < 2; ++mt)
+            for (int j = 0; j < 16; ++j)
 #pragma unroll
-                for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                    for (int part = 0; part < 2; ++part)
-                        mma_tile(sacc[mt][nt], &sm.Bt[part][0][0], kLdQ, 32 * warp + 16 * mt, &sm.Xt[0][0], kLdQ,
-                                 8 * nt, k0, gid, tig);
-        __syncthreads();  // the state's old copy is no longer read (Y above)
-        store_state();
+                for (int part = 0; part < 2; ++part)
+                    mma_tile(sacc[j], &sm.Xt[0][0], kLdQ, pw, &sm.Bt[part][0][0], kLdQ, 8 * j, k0, gid, tig);
     }
 
     if (a.s_last != nullptr) {
         float *sl = a.s_last + (b * a.H + h) * kP * kN;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+        for (int j = 0; j < 16; ++j)
 #pragma unroll
-            for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int n = 32 * warp + 16 * mt + gid + (e >= 2 ? 8 : 0);
-                    const int p = 8 * nt + 2 * tig + (e & 1);
-                    sl[p * kN + n] = sacc[mt][nt][e];
-                }
+            for (int r = 0; r < 2; ++r) {
+                const int p = pw + gid + 8 * r;
+                const int n = 8 * j + 2 * tig;
+                *reinterpret_cast<float2 *>(sl + p * kN + n) = make_float2(sacc[j][2 * r], sacc[j][2 * r + 1]);
+            }
     }
 }
 

@@ -27,6 +27,25 @@ def test_decode_bytes():
     assert abs(n / 1e6 - 181.3) < 0.1
 
 
+def test_bwd_bytes_130m():
+    # per channel-token: u, delta, z (bf16) + dout (fp32) read, du, ddelta, dz (fp32) written
+    n = bench.bwd_bytes(8, 1536, 16, 2048, 2, 4)
+    ct = 8 * 1536 * 2048
+    assert n == (ct * (3 * 2 + 4 + 12) + 8 * 2048 * 32 * (2 + 4) + 8 * 1536 * 32 * 16 * 4
+                 + 8 * 1536 * 16 * 4 + 2 * (1536 * 16 * 4 + 2 * 1536 * 4))
+    assert abs(n / 1e6 - 583.0) < 0.1
+
+
+def test_ssd_models():
+    # x bf16 in, y fp32 out per (token, head, p); dt per (token, head); B, C per (token, group)
+    n = bench.ssd_bytes(4, 2048, 80, 64, 128, 1, 2, 4)
+    assert n == 4 * 2048 * 80 * (64 * 6 + 2) + 4 * 2048 * 2 * 128 * 2 + 3 * 80 * 4 + 4 * 80 * 64 * 128 * 4
+    # per (b, h, 32-token chunk): C S (Q N P) + C B^T (Q Q N) + G' X (Q Q P) + B'^T X (N Q P), x2
+    f = bench.ssd_flops(4, 2048, 80, 64, 128)
+    per = 2 * (32 * 128 * 64 + 32 * 32 * 128 + 32 * 32 * 64 + 128 * 32 * 64)
+    assert f == 4 * 80 * 64 * per
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))

@@ -535,14 +535,16 @@ def main(argv=None):
             "backward": {"workload": w.name + ", dout N(0,1) fp32", "fwd_train_ms": fwd_train_ms,
                          "bwd_ms": bwd_ms, "bwd_bytes": bbytes, "value": bbytes / (bwd_ms * 1e-3) / 1e9,
                          "unit": "GB/s", "frac": bbytes / (bwd_ms * 1e-3) / 1e9 / peak,
-                         "timing": f"mean of {bwd_steps} event-timed (forward with saved states, backward) pairs"},
+                         "timing": f"mean of {bwd_steps} event-timed (forward with saved states, backward) pairs",
+                         "traffic": recorded_traffic("scan_bwd_130m")},
             "ssd": {"workload": sw.name, "ms": ssd_ms, "bytes": sbytes,
                     "value": sbytes / (ssd_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "frac_hbm": sbytes / (ssd_ms * 1e-3) / 1e9 / peak,
                     "tflops": sflops / (ssd_ms * 1e-3) / 1e12, "algorithmic_flops": sflops,
                     "frac_tensor": sflops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops(),
                     "bound": "hbm (bytes / 6443 GB/s exceed flops / bf16 peak)",
-                    "timing": "mean of per-launch event pairs, two rotating input sets"},
+                    "timing": "mean of per-launch event pairs, two rotating input sets",
+                    "traffic": recorded_traffic("ssd_2p7b")},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

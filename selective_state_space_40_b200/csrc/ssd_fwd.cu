@@ -52,12 +52,24 @@ struct SsdSmem {
     __nv_bfloat16 X[2][kQ][kP];       // x [s][p] as loaded
     __nv_bfloat16 Xt[kP][kLdQ];       // x^T [p][s]
     __nv_bfloat16 G[2][kQ][kLdQ];     // G' hi / lo [t][s]
-    __nv_bfloat16 Bt[2][kN][kLdQ];    // B'^T hi / lo [n][s]
-    float dl[kQ];                     // Delta_t
-    float cs[kQ];                     // A sum_{r<=t} Delta_r
-    float wq[kQ];                     // exp(cs_Q - cs_s) Delta_s
-    float ecs[kQ];                    // exp(cs_t)
+    __nv_bfloat16 Xw[2][kP][kLdQ];    // (x_s w_s)^T hi / lo [p][s], w_s = exp(cs_Q - cs_s) Delta_s
+    // per-token chunk parameters, for this chunk and the next
+    float dl[2][kQ];                  // Delta_t
+    float cs[2][kQ];                  // A sum_{r<=t} Delta_r
+    float wq[2][kQ];                  // exp(cs_Q - cs_s) Delta_s
+    float ecs[2][kQ];                 // exp(cs_t)
 };
+
+// B operand fragments of two adjacent 8-column tiles from a row-major [k][n]
+// bf16 tile (k rows 16 bytes apart per 8 columns): ldmatrix with transpose
+// hands each thread the (k = 2tig, 2tig+1) pairs of its column.
+__device__ __forceinline__ void ldsm_x4_trans(const __nv_bfloat16 *row_addr, uint32_t &r0, uint32_t &r1,
+                                              uint32_t &r2, uint32_t &r3) {
+    const unsigned a = static_cast<unsigned>(__cvta_generic_to_shared(row_addr));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(a));
+}
 
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
@@ -167,37 +179,44 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
         const int64_t t = ck * kQ + lane;
         dt_next = (warp == 0 && t < L) ? ld1(dtb + t * a.dt_sl) : 0.0f;
     };
+    // warp 0: Delta, the decay prefix and the per-token weights of chunk ck
+    // (its dt already in dt_next) into parameter buffer pb
+    auto chunk_params = [&](int64_t ck, int pb) {
+        if (warp != 0) return;
+        float d = 0.0f;
+        if (ck * kQ + lane < L) {
+            const float v = dt_next + bias;
+            d = sp ? softplus_f(v) : v;
+        }
+        float c = Ah * d;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, c, off);
+            if (lane >= off) c += o;
+        }
+        const float cend = __shfl_sync(0xffffffffu, c, kQ - 1);
+        sm.dl[pb][lane] = d;
+        sm.cs[pb][lane] = c;
+        sm.wq[pb][lane] = __expf(cend - c) * d;
+        sm.ecs[pb][lane] = __expf(c);
+    };
     if (nch > 0) {
         issue_chunk(0, 0);
         load_dt(0);
+        chunk_params(0, 0);
     }
     for (int64_t ck = 0; ck < nch; ++ck) {
         const int64_t t0 = ck * kQ;
         const int buf = (int)(ck & 1);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
         __syncthreads();  // chunk ck in buf for everyone; the previous chunk's tiles are free
-        // ---- x^T for the products; warp 0: Delta, its decay prefix and weights
+        // ---- x^T and (x w)^T (hi / lo) for the products
+        const float *pcs = sm.cs[buf], *pdl = sm.dl[buf], *pwq = sm.wq[buf], *pecs = sm.ecs[buf];
         for (int i = tid; i < kQ * kP; i += kST) {
             const int t = i / kP, p = i % kP;
-            sm.Xt[p][t] = sm.X[buf][t][p];
-        }
-        if (warp == 0) {
-            float d = 0.0f;
-            if (t0 + lane < L) {
-                const float v = dt_next + bias;
-                d = sp ? softplus_f(v) : v;
-            }
-            float c = Ah * d;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, c, off);
-                if (lane >= off) c += o;
-            }
-            const float cend = __shfl_sync(0xffffffffu, c, kQ - 1);
-            sm.dl[lane] = d;
-            sm.cs[lane] = c;
-            sm.wq[lane] = __expf(cend - c) * d;
-            sm.ecs[lane] = __expf(c);
+            const __nv_bfloat16 xv = sm.X[buf][t][p];
+            sm.Xt[p][t] = xv;
+            split_bf16(__bfloat162float(xv) * pwq[t], sm.Xw[0][p][t], sm.Xw[1][p][t]);
         }
         // next chunk's copies run under this chunk's products
         if (ck + 1 < nch) {
@@ -205,7 +224,7 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
             load_dt(ck + 1);
         }
         __syncthreads();
-        const float cs_end = sm.cs[kQ - 1];
+        const float cs_end = pcs[kQ - 1];
 
         // ---- Y^T = S_in^T C^T, columns scaled by exp(cs_t): the state
         // accumulators are the A operand (hi and lo parts), C rows the B operand
@@ -231,7 +250,7 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
         }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt) {
-            const float e0 = sm.ecs[8 * nt + 2 * tig], e1 = sm.ecs[8 * nt + 2 * tig + 1];
+            const float e0 = pecs[8 * nt + 2 * tig], e1 = pecs[8 * nt + 2 * tig + 1];
             yacc[nt][0] *= e0; yacc[nt][1] *= e1;
             yacc[nt][2] *= e0; yacc[nt][3] *= e1;
         }
@@ -256,7 +275,7 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
                     for (int e = 0; e < 4; ++e) {
                         const int t = gm + gid + (e >= 2 ? 8 : 0);
                         const int s = gn + 8 * nt + 2 * tig + (e & 1);
-                        const float v = s <= t ? gacc[nt][e] * __expf(sm.cs[t] - sm.cs[s]) * sm.dl[s] : 0.0f;
+                        const float v = s <= t ? gacc[nt][e] * __expf(pcs[t] - pcs[s]) * pdl[s] : 0.0f;
                         split_bf16(v, sm.G[0][t][s], sm.G[1][t][s]);
                     }
             } else {
@@ -294,27 +313,36 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
                 }
             }
 
-        // ---- B'^T [n][s] = exp(cs_Q - cs_s) Delta_s B_s[n], hi / lo
-        for (int i = tid; i < kN * kQ; i += kST) {
-            const int n = i / kQ, s = i % kQ;
-            const float v = __bfloat162float(sm.B[buf][s][n]) * sm.wq[s];
-            split_bf16(v, sm.Bt[0][n][s], sm.Bt[1][n][s]);
-        }
-        __syncthreads();
-
-        // ---- S_out^T = exp(cs_Q) S_in^T + X^T B'  (rows p, columns n)
+        // ---- S_out^T = exp(cs_Q) S_in^T + (x w)^T B  (rows p, columns n): A
+        // from the weighted x (hi / lo), B straight from the chunk's B rows
         const float decay = __expf(cs_end);
 #pragma unroll
         for (int j = 0; j < 16; ++j)
 #pragma unroll
             for (int e = 0; e < 4; ++e) sacc[j][e] *= decay;
 #pragma unroll
-        for (int k0 = 0; k0 < kQ; k0 += 16)
+        for (int k0 = 0; k0 < kQ; k0 += 16) {
+            uint32_t ah[4], al[4];
+            {
+                const __nv_bfloat16 *ar = &sm.Xw[0][pw + gid][k0 + 2 * tig];
+                const __nv_bfloat16 *lr = &sm.Xw[1][pw + gid][k0 + 2 * tig];
+                ah[0] = ld32(ar); ah[1] = ld32(ar + 8 * kLdQ); ah[2] = ld32(ar + 8); ah[3] = ld32(ar + 8 * kLdQ + 8);
+                al[0] = ld32(lr); al[1] = ld32(lr + 8 * kLdQ); al[2] = ld32(lr + 8); al[3] = ld32(lr + 8 * kLdQ + 8);
+            }
 #pragma unroll
-            for (int j = 0; j < 16; ++j)
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-                    mma_tile(sacc[j], &sm.Xt[0][0], kLdQ, pw, &sm.Bt[part][0][0], kLdQ, 8 * j, k0, gid, tig);
+            for (int j = 0; j < 16; j += 2) {
+                // lanes 0-15: rows k0..k0+15 of columns 8j..; lanes 16-31: columns 8(j+1)..
+                const __nv_bfloat16 *rowp = &sm.B[buf][k0 + (lane & 15)][8 * j + 8 * (lane >> 4)];
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_trans(rowp, b0, b1, b2, b3);
+                mma_bf16(sacc[j], ah[0], ah[1], ah[2], ah[3], b0, b1);
+                mma_bf16(sacc[j + 1], ah[0], ah[1], ah[2], ah[3], b2, b3);
+                mma_bf16(sacc[j], al[0], al[1], al[2], al[3], b0, b1);
+                mma_bf16(sacc[j + 1], al[0], al[1], al[2], al[3], b2, b3);
+            }
+        }
+        // warp 0 prepares the next chunk's parameters (its dt has arrived)
+        if (ck + 1 < nch) chunk_params(ck + 1, buf ^ 1);
     }
 
     if (a.s_last != nullptr) {

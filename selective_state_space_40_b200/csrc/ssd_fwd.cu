@@ -60,6 +60,26 @@ struct SsdSmem {
     float ecs[2][kQ];                 // exp(cs_t)
 };
 
+// A operand fragment of the 16 x 16 tile at (m0, k0) of a row-major [m][k]
+// bf16 array, in one ldmatrix (lane l addresses row m0 + l%8 + 8((l/8)%2),
+// column k0 + 8(l/16)).
+__device__ __forceinline__ void ldsm_a(const __nv_bfloat16 *base, int ld, int m0, int k0, int lane, uint32_t (&a)[4]) {
+    const __nv_bfloat16 *p = base + (m0 + (lane & 7) + 8 * ((lane >> 3) & 1)) * ld + k0 + 8 * (lane >> 4);
+    const unsigned ad = static_cast<unsigned>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                 : "r"(ad));
+}
+// B operand fragments (b0, b1) of the two 8-wide n-tiles at n0 and n0 + 8,
+// k-step k0, from a [n][k] bf16 array (k contiguous), in one ldmatrix.
+__device__ __forceinline__ void ldsm_b2(const __nv_bfloat16 *base, int ld, int n0, int k0, int lane, uint32_t (&b)[4]) {
+    const __nv_bfloat16 *p = base + (n0 + (lane & 7) + 8 * (lane >> 4)) * ld + k0 + 8 * ((lane >> 3) & 1);
+    const unsigned ad = static_cast<unsigned>(__cvta_generic_to_shared(p));
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                 : "r"(ad));
+}
+
 // B operand fragments of two adjacent 8-column tiles from a row-major [k][n]
 // bf16 tile (k rows 16 bytes apart per 8 columns): ldmatrix with transpose
 // hands each thread the (k = 2tig, 2tig+1) pairs of its column.
@@ -94,17 +114,6 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], uint32_t a0, uint32_t a1
         "{%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
         : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t ld32(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint32_t *>(p); }
-
-// acc[16 x 8 tile] += A[m0.., k0..k0+16) * B[k0.., n0..n0+8), with A stored
-// [m][k] (row stride lda) and B stored [n][k] (row stride ldb), bf16.
-__device__ __forceinline__ void mma_tile(float (&acc)[4], const __nv_bfloat16 *A, int lda, int m0,
-                                         const __nv_bfloat16 *Bm, int ldb, int n0, int k0, int gid, int tig) {
-    const __nv_bfloat16 *ar = A + (m0 + gid) * lda + k0 + 2 * tig;
-    const __nv_bfloat16 *br = Bm + (n0 + gid) * ldb + k0 + 2 * tig;
-    mma_bf16(acc, ld32(ar), ld32(ar + 8 * lda), ld32(ar + 8), ld32(ar + 8 * lda + 8), ld32(br), ld32(br + 8));
 }
 
 __device__ __forceinline__ void split_bf16(float v, __nv_bfloat16 &hi, __nv_bfloat16 &lo) {
@@ -241,11 +250,13 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
             split_pair(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1], ah[2], al[2]);
             split_pair(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3], ah[3], al[3]);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                const __nv_bfloat16 *br = &sm.C[buf][8 * nt + gid][16 * kk + 2 * tig];
-                const uint32_t b0 = ld32(br), b1 = ld32(br + 8);
-                mma_bf16(yacc[nt], ah[0], ah[1], ah[2], ah[3], b0, b1);
-                mma_bf16(yacc[nt], al[0], al[1], al[2], al[3], b0, b1);
+            for (int np = 0; np < 2; ++np) {
+                uint32_t bb[4];
+                ldsm_b2(&sm.C[buf][0][0], kLdN, 16 * np, 16 * kk, lane, bb);
+                mma_bf16(yacc[2 * np], ah[0], ah[1], ah[2], ah[3], bb[0], bb[1]);
+                mma_bf16(yacc[2 * np + 1], ah[0], ah[1], ah[2], ah[3], bb[2], bb[3]);
+                mma_bf16(yacc[2 * np], al[0], al[1], al[2], al[3], bb[0], bb[1]);
+                mma_bf16(yacc[2 * np + 1], al[0], al[1], al[2], al[3], bb[2], bb[3]);
             }
         }
 #pragma unroll
@@ -265,10 +276,13 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) gacc[nt][e] = 0.0f;
 #pragma unroll
-                for (int k0 = 0; k0 < kN; k0 += 16)
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt)
-                        mma_tile(gacc[nt], &sm.C[buf][0][0], kLdN, gm, &sm.B[buf][0][0], kLdN, gn + 8 * nt, k0, gid, tig);
+                for (int k0 = 0; k0 < kN; k0 += 16) {
+                    uint32_t af[4], bb[4];
+                    ldsm_a(&sm.C[buf][0][0], kLdN, gm, k0, lane, af);
+                    ldsm_b2(&sm.B[buf][0][0], kLdN, gn, k0, lane, bb);
+                    mma_bf16(gacc[0], af[0], af[1], af[2], af[3], bb[0], bb[1]);
+                    mma_bf16(gacc[1], af[0], af[1], af[2], af[3], bb[2], bb[3]);
+                }
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -291,14 +305,20 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 
         // ---- Y^T += X^T G'^T over the causal part, then y = Y + D x
 #pragma unroll
-        for (int k0 = 0; k0 < kQ; k0 += 16)
+        for (int k0 = 0; k0 < kQ; k0 += 16) {
+            uint32_t af[4];
+            ldsm_a(&sm.Xt[0][0], kLdQ, pw, k0, lane, af);
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-                if (k0 > 8 * nt + 7) continue;  // s > t for the whole tile
+            for (int part = 0; part < 2; ++part)
 #pragma unroll
-                for (int part = 0; part < 2; ++part)
-                    mma_tile(yacc[nt], &sm.Xt[0][0], kLdQ, pw, &sm.G[part][0][0], kLdQ, 8 * nt, k0, gid, tig);
-            }
+                for (int np = 0; np < 2; ++np) {
+                    if (k0 > 16 * np + 15) continue;  // s > t for both tiles
+                    uint32_t bb[4];
+                    ldsm_b2(&sm.G[part][0][0], kLdQ, 16 * np, k0, lane, bb);
+                    mma_bf16(yacc[2 * np], af[0], af[1], af[2], af[3], bb[0], bb[1]);
+                    mma_bf16(yacc[2 * np + 1], af[0], af[1], af[2], af[3], bb[2], bb[3]);
+                }
+        }
 #pragma unroll
         for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
@@ -323,12 +343,8 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 #pragma unroll
         for (int k0 = 0; k0 < kQ; k0 += 16) {
             uint32_t ah[4], al[4];
-            {
-                const __nv_bfloat16 *ar = &sm.Xw[0][pw + gid][k0 + 2 * tig];
-                const __nv_bfloat16 *lr = &sm.Xw[1][pw + gid][k0 + 2 * tig];
-                ah[0] = ld32(ar); ah[1] = ld32(ar + 8 * kLdQ); ah[2] = ld32(ar + 8); ah[3] = ld32(ar + 8 * kLdQ + 8);
-                al[0] = ld32(lr); al[1] = ld32(lr + 8 * kLdQ); al[2] = ld32(lr + 8); al[3] = ld32(lr + 8 * kLdQ + 8);
-            }
+            ldsm_a(&sm.Xw[0][0][0], kLdQ, pw, k0, lane, ah);
+            ldsm_a(&sm.Xw[1][0][0], kLdQ, pw, k0, lane, al);
 #pragma unroll
             for (int j = 0; j < 16; j += 2) {
                 // lanes 0-15: rows k0..k0+15 of columns 8j..; lanes 16-31: columns 8(j+1)..

@@ -303,6 +303,34 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
                    ms_stream_t stream);
 
 /*
+ * Mamba-2 SSD layer, one token (decode): the recurrent view of the same model
+ * (blog, section 3: generation updates the state once per token). For batch
+ * row b, head h, group g = h / (nheads / ngroups):
+ *     Delta = softplus(dt[b,h] + dt_bias[h])   (plain sum when the flag is 0)
+ *     S[p][n] = exp(Delta A[h]) S[p][n] + Delta x[b,h,p] B[b,g,n]
+ *     y[b,h,p] = sum_n C[b,g,n] S[p][n] + D[h] x[b,h,p]
+ * state [batch, nheads, headdim, dstate] fp32 is read and overwritten; each
+ * head's [headdim, dstate] block is dense, 16-byte aligned. x, y [batch,
+ * nheads, headdim]; dt [batch, nheads]; B, C [batch, ngroups, dstate]
+ * (innermost dimension dense). This version runs dstate 128 (MS_ERR_SHAPE
+ * otherwise), any headdim; x, dt, B, C fp32 or bf16, y fp32 or bf16.
+ */
+typedef struct {
+    int64_t batch, nheads, headdim, dstate, ngroups;
+    int64_t x_sb, x_sh;
+    int64_t dt_sb;
+    int64_t B_sb, B_sg;
+    int64_t C_sb, C_sg;
+    int64_t y_sb, y_sh;
+    int64_t state_sb, state_sh;
+    int32_t in_dtype, out_dtype;
+} ms_ssd_update_dims;
+
+int mamba2_ssd_state_update(float *state, const void *x, const void *dt, const float *A, const void *B,
+                            const void *C, const float *D, const float *dt_bias, int softplus_flag, void *y,
+                            const ms_ssd_update_dims *dims, int *dev_status, ms_stream_t stream);
+
+/*
  * Sizes and strides of one decode step.
  *   x, delta, z, y : [batch, dim]     element (b,d) at b*x_sb + d
  *   B, C           : [batch, dstate]  element (b,n) at b*x_sb + n

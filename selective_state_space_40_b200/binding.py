@@ -53,6 +53,12 @@ class SsdDims(ctypes.Structure):
         ("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
 
 
+class SsdUpdateDims(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int64) for n in (
+        "batch", "nheads", "headdim", "dstate", "ngroups", "x_sb", "x_sh", "dt_sb", "B_sb", "B_sg", "C_sb", "C_sg",
+        "y_sb", "y_sh", "state_sb", "state_sh")] + [("in_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
 class MambaScanError(RuntimeError):
     def __init__(self, code: int, what: str):
         super().__init__(f"{what}: status {code} ({mamba_status_string(code)})")
@@ -100,6 +106,9 @@ def library() -> ctypes.CDLL:
         lib.mamba_scan_bwd_noalloc.restype = ctypes.c_int
         lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
+        lib.mamba2_ssd_state_update.argtypes = [_vp] * 8 + [ctypes.c_int, _vp, ctypes.POINTER(SsdUpdateDims),
+                                                            _vp, _vp]
+        lib.mamba2_ssd_state_update.restype = ctypes.c_int
         lib.mamba_state_update.argtypes = [_vp] * 9 + [ctypes.c_int, _vp, ctypes.POINTER(UpdateDims),
                                                        _vp, _vp]
         lib.mamba_state_update.restype = ctypes.c_int
@@ -178,6 +187,12 @@ def mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, softplus_flag, initial_state, y, 
                    dev_status, stream) -> int:
     return library().mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, int(softplus_flag), initial_state, y, final_state,
                                     ctypes.byref(dims), dev_status, stream)
+
+
+def mamba2_ssd_state_update(state, x, dt, A, B, C, D, dt_bias, softplus_flag, y, dims: SsdUpdateDims,
+                            dev_status, stream) -> int:
+    return library().mamba2_ssd_state_update(state, x, dt, A, B, C, D, dt_bias, int(softplus_flag), y,
+                                             ctypes.byref(dims), dev_status, stream)
 
 
 def mamba_conv_scan_fwd(x, conv_w, conv_b, conv_x0, u_out, cdims: ConvDims, delta, A, B, C, D, z,
@@ -417,6 +432,32 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba2_ssd_fwd")
     return y, fs
+
+
+def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, out_dtype=None,
+                     y=None, stream=None, dev_status=None):
+    """One Mamba-2 decode step on torch CUDA tensors: state [b, H, P, 128]
+    fp32 (updated in place), x [b, H, P], dt [b, H], B/C [b, G, 128].
+    Returns y [b, H, P]."""
+    torch = _torch()
+    if out_dtype is None:
+        out_dtype = torch.float32
+    batch, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    if state.dtype != torch.float32 or state.stride(-1) != 1 or state.stride(-2) != N:
+        raise ValueError("state must be fp32 with dense [headdim, dstate] blocks")
+    for t, n in ((x, "x"), (dt, "dt"), (B, "B"), (C, "C")):
+        _inner_contiguous(t, n)
+    if y is None:
+        y = torch.empty((batch, H, P), dtype=out_dtype, device=x.device)
+    dims = SsdUpdateDims(batch, H, P, N, G, x.stride(0), x.stride(1), dt.stride(0), B.stride(0), B.stride(1),
+                         C.stride(0), C.stride(1), y.stride(0), y.stride(1), state.stride(0), state.stride(1),
+                         _dtype_code(x), _dtype_code(y))
+    rc = mamba2_ssd_state_update(_ptr(state), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias),
+                                 softplus, _ptr(y), dims, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba2_ssd_state_update")
+    return y
 
 
 def update_dims_for(state, x, delta, B, C, z, y) -> UpdateDims:

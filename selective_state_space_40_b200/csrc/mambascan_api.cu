@@ -452,6 +452,47 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
     return MS_OK;
 }
 
+int mamba2_ssd_state_update(float *state, const void *x, const void *dt, const float *A, const void *B,
+                            const void *C, const float *D, const float *dt_bias, int softplus_flag, void *y,
+                            const ms_ssd_update_dims *dm, int *dev_status, ms_stream_t stream) {
+    (void)dev_status;
+    if (!dm) return MS_ERR_NULL;
+    if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) || (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
+        return MS_ERR_DTYPE;
+    if (dm->batch < 0 || dm->nheads < 1 || dm->ngroups < 1 || dm->nheads % dm->ngroups != 0 || dm->headdim < 1 ||
+        dm->headdim > INT32_MAX || dm->dstate != 128)
+        return MS_ERR_SHAPE;
+    if (dm->x_sb < 0 || dm->x_sh < 0 || dm->dt_sb < 0 || dm->B_sb < 0 || dm->B_sg < 0 || dm->C_sb < 0 ||
+        dm->C_sg < 0 || dm->y_sb < 0 || dm->y_sh < 0 || dm->state_sb < 0 || dm->state_sh < 0)
+        return MS_ERR_STRIDE;
+    if (dm->batch == 0) return MS_OK;
+    if (!state || !x || !dt || !A || !B || !C || !y) return MS_ERR_NULL;
+    const int ei = elem_bytes(dm->in_dtype), eo = elem_bytes(dm->out_dtype);
+    if (!aligned(state, 16) || dm->state_sb % 4 || dm->state_sh % 4 || !aligned(x, ei) || !aligned(dt, ei) ||
+        !aligned(B, ei) || !aligned(C, ei) || !aligned(y, eo) || !aligned(A, 4) || (D && !aligned(D, 4)) ||
+        (dt_bias && !aligned(dt_bias, 4)))
+        return MS_ERR_ALIGN;
+    const int64_t H = dm->nheads, G = dm->ngroups, P = dm->headdim;
+    if (max_offset3(dm->batch, dm->state_sb, H, dm->state_sh, P * 128) < 0 ||
+        max_offset3(dm->batch, dm->x_sb, H, dm->x_sh, P) < 0 || max_offset3(dm->batch, dm->y_sb, H, dm->y_sh, P) < 0 ||
+        max_offset3(dm->batch, dm->dt_sb, 1, 0, H) < 0 || max_offset3(dm->batch, dm->B_sb, G, dm->B_sg, 128) < 0 ||
+        max_offset3(dm->batch, dm->C_sb, G, dm->C_sg, 128) < 0)
+        return MS_ERR_SHAPE;
+    ms::SsdUpdArgs a{};
+    a.state = state; a.x = x; a.dt = dt; a.B = B; a.C = C; a.A = A; a.D = D; a.dt_bias = dt_bias; a.y = y;
+    a.batch = dm->batch; a.H = H; a.G = G; a.P = (int)P;
+    a.x_sb = dm->x_sb; a.x_sh = dm->x_sh; a.dt_sb = dm->dt_sb; a.B_sb = dm->B_sb; a.B_sg = dm->B_sg;
+    a.C_sb = dm->C_sb; a.C_sg = dm->C_sg; a.y_sb = dm->y_sb; a.y_sh = dm->y_sh;
+    a.st_sb = dm->state_sb; a.st_sh = dm->state_sh;
+    a.softplus = softplus_flag ? 1 : 0;
+    cudaError_t e = ms::launch_ssd_update(a, dm->in_dtype == MS_BF16, dm->out_dtype == MS_BF16, (cudaStream_t)stream);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
 int mamba_state_update(float *state, const void *x, const void *delta, const float *A, const void *B,
                        const void *C, const float *D, const void *z, const float *delta_bias,
                        int softplus_flag, void *y, const ms_update_dims *dm, int *dev_status,

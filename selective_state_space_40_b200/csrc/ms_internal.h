@@ -66,6 +66,20 @@ struct SsdArgs {
     int softplus;
 };
 bool ssd_shape_supported(int64_t headdim, int64_t dstate);
+
+// Arguments of the Mamba-2 SSD one-token state update (state [b, H, P, 128]
+// fp32, each head's [P, 128] block dense).
+struct SsdUpdArgs {
+    float *state;
+    const void *x, *dt, *B, *C;
+    const float *A, *D, *dt_bias;
+    void *y;
+    int64_t batch, H, G;
+    int P;
+    int64_t x_sb, x_sh, dt_sb, B_sb, B_sg, C_sb, C_sg, y_sb, y_sh, st_sb, st_sh;
+    int softplus;
+};
+cudaError_t launch_ssd_update(const SsdUpdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
 cudaError_t launch_ssd_fwd(const SsdArgs &a, bool out_bf16, cudaStream_t stream);
 
 // Launch shape chosen on the host for one scan call.

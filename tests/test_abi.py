@@ -226,6 +226,26 @@ def test_ssd_rejects_bad_arguments(lib):
     assert call(_sdims(batch=0)) == mb.MS_OK
 
 
+def test_ssd_update_rejects_bad_arguments(lib):
+    def dims(**kw):
+        d = dict(batch=2, nheads=4, headdim=64, dstate=128, ngroups=1, x_sb=256, x_sh=64, dt_sb=4, B_sb=128,
+                 B_sg=128, C_sb=128, C_sg=128, y_sb=256, y_sh=64, state_sb=4 * 64 * 128, state_sh=64 * 128,
+                 in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)
+        d.update(kw)
+        return mb.SsdUpdateDims(**d)
+
+    def call(dm, state=FAKE):
+        return mb.mamba2_ssd_state_update(state, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, FAKE, dm, None, None)
+    assert call(dims(dstate=64)) == mb.MS_ERR_SHAPE
+    assert call(dims(nheads=3, ngroups=2)) == mb.MS_ERR_SHAPE
+    assert call(dims(in_dtype=3)) == mb.MS_ERR_DTYPE
+    assert call(dims(x_sh=-1)) == mb.MS_ERR_STRIDE
+    assert call(dims(), state=None) == mb.MS_ERR_NULL
+    assert call(dims(), state=FAKE + 4) == mb.MS_ERR_ALIGN
+    assert call(dims(state_sh=64 * 128 + 2)) == mb.MS_ERR_ALIGN
+    assert call(dims(batch=0)) == mb.MS_OK
+
+
 def _udims(**kw):
     d = dict(batch=4, dim=8, dstate=16, x_sb=8, delta_sb=8, z_sb=8, y_sb=8, B_sb=16, C_sb=16,
              state_sb=128, state_sd=16, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)

@@ -134,3 +134,56 @@ def test_full_2p7b_layer_sampled_heads():
         ib, ih = torch.as_tensor([int(b)]), torch.as_tensor(hs)
         check_bf16(f64(y[ib][:, :, ih]), yr, f"2.7B b={b} heads {hs} y")
         check_bf16(f64(fs[ib][:, ih]), fr, f"2.7B b={b} heads {hs} final_state")
+
+
+# ------------------------------------------------------------ decode step ----
+
+def _decode_inputs(b, H, P, G, seed, dtype=torch.bfloat16):
+    gen = torch.Generator().manual_seed(seed)
+    x = torch.randn(b, H, P, generator=gen).to(dtype)
+    dt = torch.randn(b, H, generator=gen).to(dtype)
+    B = torch.randn(b, G, 128, generator=gen).to(dtype)
+    C = torch.randn(b, G, 128, generator=gen).to(dtype)
+    return x, dt, B, C
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("P,G", [(64, 1), (48, 2), (8, 4)])
+def test_decode_steps_against_oracle(dtype, P, G):
+    """Several one-token steps from a random state, each against the oracle's
+    recurrence with one token (y every step, the state at the end)."""
+    b, H = 3, 4
+    w = syn.SsdWorkload("d", b, 1, H, P, 128, G)
+    par = syn.ssd_inputs(w)
+    state = 0.3 * torch.randn(b, H, P, 128, generator=torch.Generator().manual_seed(2))
+    sg = state.to(DEV)
+    sr = f64(state)
+    for k in range(6):
+        x, dt, B, C = _decode_inputs(b, H, P, G, 100 + k, dtype)
+        y = mb.ssd_state_update(sg, x.to(DEV), dt.to(DEV), par["A"].to(DEV), B.to(DEV), C.to(DEV),
+                                par["D"].to(DEV), par["dt_bias"].to(DEV), True)
+        torch.cuda.synchronize()
+        yr, sr = oracle.ssd(f64(x)[:, None], f64(dt)[:, None], f64(par["A"]), f64(B)[:, None], f64(C)[:, None],
+                            f64(par["D"]), f64(par["dt_bias"]), True, sr)
+        check_bf16(f64(y), yr[:, 0], f"ssd decode step {k} y")
+    check_bf16(f64(sg), sr, "ssd decode final state")
+
+
+def test_decode_steps_equal_chunked_forward():
+    """L one-token steps from a state equal the chunked forward over the same
+    L tokens (recurrent view == matrix view) on the GPU."""
+    b, L, H, G = 2, 40, 4, 1
+    w, inp = _case(b, L, H, G, 120)
+    s0 = 0.2 * torch.randn(b, H, 64, 128, generator=torch.Generator().manual_seed(3))
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    yf, sf = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                        initial_state=s0.to(DEV))
+    st = s0.to(DEV).clone()
+    ys = []
+    for t in range(L):
+        ys.append(mb.ssd_state_update(st, g["x"][:, t].contiguous(), g["dt"][:, t].contiguous(), g["A"],
+                                      g["B"][:, t].contiguous(), g["C"][:, t].contiguous(), g["D"], g["dt_bias"], True))
+    torch.cuda.synchronize()
+    yd = torch.stack(ys, dim=1)
+    check_bf16(f64(yd), f64(yf), "decode steps vs chunked y")
+    check_bf16(f64(st), f64(sf), "decode steps vs chunked final state")

@@ -512,6 +512,36 @@ def main(argv=None):
     sflops = ssd_flops(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate)
     del ssd_in
 
+    # ---- Mamba-2 SSD decode step (2.7B-class layer, 64 sequences): the fp32
+    # state [64, 80, 64, 128] (168 MB) read and written once per step; two
+    # states rotate (336 MB > L2)
+    ub, uH, uP, uN = 64, sw.nheads, sw.headdim, sw.dstate
+    gsd = torch.Generator().manual_seed(11)
+    ust = [(0.1 * torch.randn(ub, uH, uP, uN, generator=gsd)).to(dev) for _ in range(2)]
+    ux = torch.randn(ub, uH, uP, generator=gsd).to(torch.bfloat16).to(dev)
+    udt = torch.randn(ub, uH, generator=gsd).to(torch.bfloat16).to(dev)
+    uB = torch.randn(ub, 1, uN, generator=gsd).to(torch.bfloat16).to(dev)
+    uC = torch.randn(ub, 1, uN, generator=gsd).to(torch.bfloat16).to(dev)
+    upar = {k: v.to(dev) for k, v in syn.ssd_inputs(syn.SsdWorkload("p", 1, 1, uH, uP, uN, 1)).items()}
+    uy = torch.empty(ub, uH, uP, dtype=torch.float32, device=dev)
+
+    def ssd_dec(i):
+        mb.ssd_state_update(ust[i & 1], ux, udt, upar["A"], uB, uC, upar["D"], upar["dt_bias"], True, y=uy,
+                            stream=stream)
+
+    for i in range(4):
+        ssd_dec(i)
+    u0, u1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    u0.record(stream)
+    for i in range(40):
+        ssd_dec(i)
+    u1.record(stream)
+    torch.cuda.synchronize()
+    ssd_dec_ms = max_over_ranks(u0.elapsed_time(u1) / 40, world, dev)
+    udbytes = ub * uH * uP * uN * 8 + ub * uH * uP * (2 + 4) + ub * uH * 2 + ub * 2 * uN * 2 + 3 * uH * 4
+    del ust
+
     # ---- CPU baseline: the oracle on this host's cores, whole passes over the
     # workload repeated until about ten seconds of wall time have gone by
     cpu = None
@@ -567,6 +597,10 @@ def main(argv=None):
                     "bound": "hbm (bytes / 6443 GB/s exceed flops / bf16 peak)",
                     "timing": "mean of per-launch event pairs, two rotating input sets",
                     "traffic": recorded_traffic("ssd_2p7b")},
+            "ssd_decode": {"workload": "mamba2-2.7b-class decode b64 H80 P64 N128 bf16, fp32 state",
+                           "ms": ssd_dec_ms, "bytes": udbytes, "value": udbytes / (ssd_dec_ms * 1e-3) / 1e9,
+                           "unit": "GB/s", "frac": udbytes / (ssd_dec_ms * 1e-3) / 1e9 / peak,
+                           "timing": "one event pair around 40 back-to-back steps over two rotating states"},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

@@ -360,6 +360,18 @@ int mamba_state_update(float *state, const void *x, const void *delta, const flo
                        const float *delta_bias, int softplus_flag, void *y,
                        const ms_update_dims *dims, int *dev_status, ms_stream_t stream);
 
+/*
+ * Test hook for device failure detection (the pages have no counterpart):
+ * launches one CTA that waits, with the library's bounded barrier wait, on a
+ * barrier that nothing completes. After `rounds` tries (1 .. 1048576) the
+ * wait gives up, MS_ERR_TIMEOUT is ORed into *dev_status (required device
+ * int) and the kernel ends; the context stays usable. This is the path every
+ * bounded wait of the library takes when what it waits for never comes.
+ * Returns MS_ERR_NULL / MS_ERR_SHAPE for bad arguments, else MS_OK or
+ * MS_ERR_CUDA (the timeout itself is reported through *dev_status).
+ */
+int mamba_debug_bounded_wait(uint32_t rounds, int *dev_status, ms_stream_t stream);
+
 /* Static English text for a status code (never NULL). */
 const char *mamba_status_string(int code);
 

@@ -114,6 +114,8 @@ def library() -> ctypes.CDLL:
         lib.mamba_state_update.restype = ctypes.c_int
         lib.mamba_status_string.argtypes = [ctypes.c_int]
         lib.mamba_status_string.restype = ctypes.c_char_p
+        lib.mamba_debug_bounded_wait.argtypes = [ctypes.c_uint32, _vp, _vp]
+        lib.mamba_debug_bounded_wait.restype = ctypes.c_int
         lib.mamba_device_check.argtypes = []
         lib.mamba_device_check.restype = ctypes.c_int
         _lib = lib
@@ -128,6 +130,10 @@ def mamba_status_string(code: int) -> str:
 
 def mamba_device_check() -> int:
     return library().mamba_device_check()
+
+
+def mamba_debug_bounded_wait(rounds: int, dev_status, stream) -> int:
+    return library().mamba_debug_bounded_wait(int(rounds), dev_status, stream)
 
 
 def mamba_scan_workspace_size(dims: ScanDims) -> int:

@@ -62,6 +62,17 @@ const char *mamba_status_string(int code) {
     }
 }
 
+int mamba_debug_bounded_wait(uint32_t rounds, int *dev_status, ms_stream_t stream) {
+    if (!dev_status) return MS_ERR_NULL;
+    if (rounds < 1 || rounds > (1u << 20)) return MS_ERR_SHAPE;
+    if (!aligned(dev_status, 4)) return MS_ERR_ALIGN;
+    if (ms::launch_bounded_wait_probe(dev_status, rounds, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
 int mamba_device_check(void) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -114,6 +114,9 @@ cudaError_t launch_state_update(const UpdateArgs &a, bool in_bf16, bool out_bf16
 // multiple of 128, 16-byte aligned rows).
 bool state_update_stream_applies(const UpdateArgs &a, int in_bytes, int out_bytes);
 cudaError_t launch_state_update_stream(const UpdateArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
+// One CTA waits `rounds` bounded tries on a barrier nothing completes, then
+// ORs MS_ERR_TIMEOUT into *status (tests the device timeout path).
+cudaError_t launch_bounded_wait_probe(int *status, uint32_t rounds, cudaStream_t stream);
 
 cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
 

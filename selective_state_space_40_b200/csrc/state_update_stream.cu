@@ -51,9 +51,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
                  : "memory");
 }
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait_n(uint64_t *bar, uint32_t parity, uint32_t limit) {
     const uint32_t a = saddr(bar);
-    for (uint32_t i = 0; i < kSpinLimit; ++i) {
+    for (uint32_t i = 0; i < limit; ++i) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -66,6 +66,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
     }
     return false;
 }
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) { return mbar_wait_n(bar, parity, kSpinLimit); }
 __device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
     asm volatile(
         "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -261,6 +262,27 @@ cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 }  // namespace
+
+namespace {
+
+// Test hook for the timeout path: one thread waits, with the bounded wait the
+// stream kernel uses, on a barrier that nothing completes (no arrival is ever
+// made); when the wait gives up it records MS_ERR_TIMEOUT and the kernel ends.
+__global__ void bounded_wait_probe_kernel(int *status, uint32_t rounds) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        if (!mbar_wait_n(&bar, 0, rounds)) atomicOr(status, MS_ERR_TIMEOUT);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_bounded_wait_probe(int *status, uint32_t rounds, cudaStream_t stream) {
+    bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(status, rounds);
+    return cudaGetLastError();
+}
 
 bool state_update_stream_applies(const UpdateArgs &a, int in_bytes, int out_bytes) {
     if (a.N != 16 || a.st_sd != 16 || a.dim % kTC != 0) return false;

@@ -246,6 +246,13 @@ def test_ssd_update_rejects_bad_arguments(lib):
     assert call(dims(batch=0)) == mb.MS_OK
 
 
+def test_debug_bounded_wait_argument_checks(lib):
+    assert mb.mamba_debug_bounded_wait(16, None, None) == mb.MS_ERR_NULL
+    assert mb.mamba_debug_bounded_wait(0, FAKE, None) == mb.MS_ERR_SHAPE
+    assert mb.mamba_debug_bounded_wait((1 << 20) + 1, FAKE, None) == mb.MS_ERR_SHAPE
+    assert mb.mamba_debug_bounded_wait(16, FAKE + 2, None) == mb.MS_ERR_ALIGN
+
+
 def _udims(**kw):
     d = dict(batch=4, dim=8, dstate=16, x_sb=8, delta_sb=8, z_sb=8, y_sb=8, B_sb=16, C_sb=16,
              state_sb=128, state_sd=16, in_dtype=mb.MS_BF16, out_dtype=mb.MS_F32)

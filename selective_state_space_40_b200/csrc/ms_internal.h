@@ -2,6 +2,7 @@
 // launchers (not part of the public ABI).
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 

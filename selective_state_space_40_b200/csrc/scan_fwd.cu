@@ -562,16 +562,16 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // Opt in to more than 48 KB of dynamic shared memory once per device and
-    // instantiation (idempotent, so a race between host threads is harmless).
-    static bool opted[64] = {};
+    // instantiation (setting it twice from two host threads is harmless).
+    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev]) {
+    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
         if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev] = true;
+        if (dev < 64) opted[dev].store(true, std::memory_order_release);
     }
     scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
     return cudaGetLastError();

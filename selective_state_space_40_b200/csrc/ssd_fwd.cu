@@ -376,15 +376,15 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 
 template <typename TOut>
 cudaError_t launch_ssd_t(const SsdArgs &a, cudaStream_t stream) {
-    static bool opted[64] = {};
+    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev]) {
+    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(ssd_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)sizeof(SsdSmem));
         if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev] = true;
+        if (dev < 64) opted[dev].store(true, std::memory_order_release);
     }
     const int64_t blocks = a.batch * a.H;
     if (blocks <= 0) return cudaSuccess;

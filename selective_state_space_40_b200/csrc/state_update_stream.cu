@@ -237,15 +237,15 @@ state_update_stream_kernel(const UpdateArgs a) {
 template <typename TIn, typename TOut>
 cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
     using Sm = StreamSmem<TIn, TOut>;
-    static bool opted[64] = {};
+    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev]) {
+    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
         e = cudaFuncSetAttribute(state_update_stream_kernel<TIn, TOut>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
         if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev] = true;
+        if (dev < 64) opted[dev].store(true, std::memory_order_release);
     }
     int sms = 148, per_sm = 1;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);

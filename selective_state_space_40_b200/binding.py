@@ -247,6 +247,14 @@ def _inner_contiguous(t, name):
         raise ValueError(f"{name} must have unit stride along its last dimension")
 
 
+def _check_f32(**tensors):
+    """Parameters and states cross the C ABI as dense fp32 arrays."""
+    torch = _torch()
+    for n, t in tensors.items():
+        if t is not None and (t.dtype != torch.float32 or not t.is_contiguous()):
+            raise ValueError(f"{n} must be a contiguous fp32 tensor")
+
+
 def scan_dims_for(u, delta, B, C, z, y) -> ScanDims:
     """ScanDims read off tensors u/delta/z/y [b, d, L] and B/C [b, N, L]."""
     for t, n in ((u, "u"), (delta, "delta"), (B, "B"), (C, "C"), (z, "z"), (y, "y")):
@@ -320,6 +328,8 @@ def conv_scan_fwd(x, conv_w, delta, A, B, C, D=None, z=None, delta_bias=None, so
             raise ValueError(f"{n} must be a contiguous fp32 tensor")
     if conv_x0 is not None and (conv_x0.dtype != x.dtype or not conv_x0.is_contiguous()):
         raise ValueError("conv_x0 must be contiguous with the dtype of x")
+    if u_out is not None and u_out.dtype != x.dtype:
+        raise ValueError("u_out must have the dtype of x")
     _inner_contiguous(u_out, "u_out")
     dims = scan_dims_for(x, delta, B, C, z, y)
     uo = u_out if u_out is not None else x
@@ -343,6 +353,7 @@ def scan_fwd_train(u, delta, A, B, C, D=None, z=None, delta_bias=None, softplus:
         out_dtype = torch.float32
     batch, dim, L = u.shape
     N = A.shape[1]
+    _check_f32(A=A, D=D, delta_bias=delta_bias, initial_state=initial_state)
     y = torch.empty((batch, dim, L), dtype=out_dtype, device=u.device)
     last = torch.empty((batch, dim, N), dtype=torch.float32, device=u.device)
     ckpt = torch.empty((batch, dim, (L + 63) // 64, N), dtype=torch.float32, device=u.device)
@@ -364,6 +375,7 @@ def scan_bwd(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, dlast=No
     batch, dim, L = u.shape
     N = A.shape[1]
     dev = u.device
+    _check_f32(A=A, D=D, delta_bias=delta_bias, initial_state=initial_state, ckpt=ckpt, dlast=dlast)
     f32 = dict(dtype=torch.float32, device=dev)
     g = {"du": torch.empty((batch, dim, L), **f32), "ddelta": torch.empty((batch, dim, L), **f32),
          "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
@@ -396,6 +408,7 @@ def scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, 
     torch = _torch()
     batch, dim, L = u.shape
     N = A.shape[1]
+    _check_f32(A=A, D=D, delta_bias=delta_bias, initial_state=initial_state, dlast=dlast)
     f32 = dict(dtype=torch.float32, device=u.device)
     g = {"du": torch.empty((batch, dim, L), **f32), "ddelta": torch.empty((batch, dim, L), **f32),
          "dA": torch.empty((dim, N), **f32), "dB": torch.empty((batch, N, L), **f32),
@@ -425,6 +438,7 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial
         out_dtype = torch.float32
     batch, L, H, P = x.shape
     G, N = B.shape[2], B.shape[3]
+    _check_f32(A=A, D=D, dt_bias=dt_bias, initial_state=initial_state)
     for t, n in ((x, "x"), (dt, "dt"), (B, "B"), (C, "C")):
         _inner_contiguous(t, n)
     if y is None:
@@ -450,6 +464,7 @@ def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, softplus: bool
         out_dtype = torch.float32
     batch, H, P = x.shape
     G, N = B.shape[1], B.shape[2]
+    _check_f32(A=A, D=D, dt_bias=dt_bias)
     if state.dtype != torch.float32 or state.stride(-1) != 1 or state.stride(-2) != N:
         raise ValueError("state must be fp32 with dense [headdim, dstate] blocks")
     for t, n in ((x, "x"), (dt, "dt"), (B, "B"), (C, "C")):
@@ -485,6 +500,7 @@ def state_update(state, x, delta, A, B, C, D=None, z=None, delta_bias=None, soft
         out_dtype = torch.float32
     if state.dtype != torch.float32:
         raise ValueError("state must be fp32")
+    _check_f32(A=A, D=D, delta_bias=delta_bias)
     batch, dim, N = state.shape
     if y is None:
         y = torch.empty((batch, dim), dtype=out_dtype, device=state.device)

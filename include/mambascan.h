@@ -89,10 +89,16 @@ typedef struct {
 } ms_scan_dims;
 
 /*
- * Workspace bytes mamba_scan_fwd needs for these dims. The scan keeps its
- * state in registers and its tiles in shared memory, so this is 0; the
- * argument pair stays in the ABI so callers need not change if a future
- * kernel needs scratch.
+ * Workspace bytes mamba_scan_fwd needs for these dims. Usually 0: the scan
+ * keeps its state in registers and its tiles in shared memory. When there are
+ * too few channels to fill the GPU (batch x dim below ~9,500 on 148 SMs) and
+ * the sequence is long (seqlen >= 8192), mamba_scan_fwd splits every batch
+ * row's sequence into segments scanned in parallel: a first pass scans the
+ * segments from zero for their end states and Delta sums, the carries are
+ * chained (the recurrence is linear in the state), and a second pass scans
+ * every segment from its true initial state. The workspace (16-byte
+ * aligned) holds the segments' states; mamba_scan_fwd_plan with an explicit
+ * plan never splits.
  */
 size_t mamba_scan_workspace_size(const ms_scan_dims *dims);
 
@@ -111,8 +117,7 @@ size_t mamba_scan_workspace_size(const ms_scan_dims *dims);
  *   last_state       optional fp32 [batch, dim, dstate] output: the state after
  *                    token seqlen-1 (equal to initial_state, or 0, if seqlen = 0).
  *   workspace        device scratch of mamba_scan_workspace_size() bytes, or
- *                    NULL with workspace_bytes = 0 when that size is 0 (it
- *                    is 0 for every size in this version).
+ *                    NULL with workspace_bytes = 0 when that size is 0.
  * Returns MS_OK or an MS_ERR_* code.
  */
 int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void *B,

@@ -125,9 +125,51 @@ static int check_scan(const void *u, const void *delta, const float *A, const vo
     return MS_OK;
 }
 
+// Sequence split for layers with too few channels to fill the GPU: S
+// segments of Ls tokens per batch row (the last one may be shorter). S = 1:
+// no split. Each batch row is split on its own, so the parallel work of one
+// pass is (S - 1) or S segments x dim channels.
+struct SplitPlan {
+    int64_t S, Ls;
+};
+
+static SplitPlan split_plan(const ms_scan_dims *d, int num_sms) {
+    SplitPlan sp{1, d->seqlen};
+    const int64_t ch = d->batch * d->dim, L = d->seqlen;
+    if (ch <= 0 || d->dim <= 0 || L < 8192 || ch * 4 / 32 >= (int64_t)num_sms * 8) return sp;
+    const int64_t target_warps = (int64_t)num_sms * 12;  // at 4 lanes per channel
+    int64_t S0 = (target_warps * 8 + d->dim - 1) / d->dim;
+    const int64_t cap = L / 1024 < 256 ? L / 1024 : 256;
+    S0 = S0 > cap ? cap : S0;
+    if (S0 < 2) return sp;
+    // prefer a count that cuts L into equal segments of whole 64-token multiples
+    for (int64_t s = S0; s <= 2 * S0 && s <= cap; ++s) {
+        if (L % s == 0 && (L / s) % 64 == 0) {
+            sp.S = s;
+            sp.Ls = L / s;
+            return sp;
+        }
+    }
+    sp.Ls = ((L + S0 - 1) / S0 + 63) / 64 * 64;
+    sp.S = (L + sp.Ls - 1) / sp.Ls;
+    if (sp.S < 2) return SplitPlan{1, L};
+    return sp;
+}
+
+// Workspace of a split, in floats per batch row (reused row after row): end
+// states E [S-1, dim, N], Delta sums [S-1, dim], initial states Sin [S, dim,
+// N], last states of the segments [S, dim, N]; each region 16-byte aligned.
+static int64_t round4(int64_t v) { return (v + 3) / 4 * 4; }
+static int64_t split_ws_floats(const ms_scan_dims *d, const SplitPlan &sp) {
+    if (sp.S < 2) return 0;
+    const int64_t cn = d->dim * d->dstate;
+    return round4((sp.S - 1) * cn) + round4((sp.S - 1) * d->dim) + round4(sp.S * cn) + round4(sp.S * cn);
+}
+
 size_t mamba_scan_workspace_size(const ms_scan_dims *dims) {
-    (void)dims;
-    return 0;  // the scan keeps everything in registers and shared memory
+    if (!dims || dims->dstate < 1 || dims->dstate > MS_MAX_DSTATE) return 0;
+    const SplitPlan sp = split_plan(dims, num_sms_current());
+    return (size_t)split_ws_floats(dims, sp) * sizeof(float);
 }
 
 static bool plan_valid(const ms_scan_plan *p) {
@@ -239,6 +281,75 @@ static int scan_common(const void *u, const void *delta, const float *A, const v
     return MS_OK;
 }
 
+// The scan of one batch row split into segments (see split_plan): pass 1
+// scans segments 0..S-2 from zero for their end states and Delta sums, the
+// carries are chained, pass 2 scans every segment from its true initial
+// state. Exact up to rounding: the recurrence is linear in the state.
+static int scan_split(const void *u, const void *delta, const float *A, const void *B, const void *C,
+                      const float *D, const void *z, const float *delta_bias, int softplus_flag,
+                      const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
+                      const SplitPlan &sp, float *ws, int *dev_status, ms_stream_t stream) {
+    const int ei = elem_bytes(dims->in_dtype), eo = elem_bytes(dims->out_dtype);
+    const int64_t dim = dims->dim, N = dims->dstate, L = dims->seqlen, S = sp.S, Ls = sp.Ls, cn = dim * N;
+    float *E = ws;
+    float *dsum = E + round4((S - 1) * cn);
+    float *Sin = dsum + round4((S - 1) * dim);
+    float *Slast = Sin + round4(S * cn);
+    const int64_t S_full = (S * Ls == L) ? S : S - 1;  // segments of exactly Ls tokens
+    const cudaStream_t st = (cudaStream_t)stream;
+    auto at = [](const void *p, int64_t elems, int es) -> const void * {
+        return p ? static_cast<const char *>(p) + elems * es : nullptr;
+    };
+    for (int64_t b = 0; b < dims->batch; ++b) {
+        const void *ub = at(u, b * dims->u_sb, ei), *db = at(delta, b * dims->delta_sb, ei);
+        const void *zb = at(z, b * dims->z_sb, ei), *Bb = at(B, b * dims->B_sb, ei), *Cb = at(C, b * dims->C_sb, ei);
+        void *yb = static_cast<char *>(y) + b * dims->y_sb * eo;
+        // a run of `nseg` segments starting at segment k0 as a batch of scans
+        auto segments = [&](int64_t k0, int64_t nseg, int64_t len, const float *h0, void *yv, float *last,
+                            float *ds) -> int {
+            ms_scan_dims v = *dims;
+            v.batch = nseg;
+            v.seqlen = len;
+            v.u_sb = v.delta_sb = v.z_sb = v.y_sb = v.B_sb = v.C_sb = Ls;
+            const int64_t off = k0 * Ls;
+            ms::ScanArgs a{};
+            a.u = at(ub, off, ei); a.delta = at(db, off, ei); a.z = at(zb, off, ei);
+            a.B = at(Bb, off, ei); a.C = at(Cb, off, ei);
+            a.A = A; a.D = D; a.bias = delta_bias; a.h0 = h0;
+            a.y = yv ? static_cast<char *>(yv) + off * eo : nullptr;
+            a.last = last; a.status = dev_status; a.dsum = ds;
+            a.batch = nseg; a.dim = dim; a.L = len; a.N = (int)N;
+            a.u_sb = Ls; a.u_sd = dims->u_sd; a.dl_sb = Ls; a.dl_sd = dims->delta_sd;
+            a.z_sb = Ls; a.z_sd = dims->z_sd; a.y_sb = Ls; a.y_sd = dims->y_sd;
+            a.B_sb = Ls; a.B_sn = dims->B_sn; a.C_sb = Ls; a.C_sn = dims->C_sn;
+            a.softplus = softplus_flag ? 1 : 0;
+            a.vec_in = vec_ok(a.u, Ls, a.u_sd, ei) && vec_ok(a.delta, Ls, a.dl_sd, ei) && vec_ok(a.z, Ls, a.z_sd, ei);
+            a.vec_out = a.y == nullptr || vec_ok(a.y, Ls, a.y_sd, eo);
+            const ms::ScanPlan pl = ms::plan_scan(a, dims->in_dtype == MS_BF16, num_sms_current());
+            return ms::launch_scan_fwd(a, pl, dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, st) ==
+                           cudaSuccess
+                       ? MS_OK
+                       : MS_ERR_CUDA;
+        };
+        const float *h0b = initial_state ? initial_state + b * cn : nullptr;
+        // pass 1: end states and Delta sums of segments 0..S-2, from zero
+        if (segments(0, S - 1, Ls, nullptr, nullptr, E, dsum) != MS_OK) return MS_ERR_CUDA;
+        if (ms::launch_carry_combine(E, dsum, A, h0b, Sin, dim, (int)N, S, st) != cudaSuccess) return MS_ERR_CUDA;
+        // pass 2: every segment from its initial state
+        float *lastb = last_state ? last_state + b * cn : nullptr;
+        if (segments(0, S_full, Ls, Sin, yb, Slast, nullptr) != MS_OK) return MS_ERR_CUDA;
+        if (S_full < S) {
+            if (segments(S - 1, 1, L - (S - 1) * Ls, Sin + (S - 1) * cn, yb, lastb, nullptr) != MS_OK)
+                return MS_ERR_CUDA;
+        } else if (lastb) {
+            if (cudaMemcpyAsync(lastb, Slast + (S - 1) * cn, cn * sizeof(float), cudaMemcpyDeviceToDevice, st) !=
+                cudaSuccess)
+                return MS_ERR_CUDA;
+        }
+    }
+    return MS_OK;
+}
+
 int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B, const void *C,
                         const float *D, const void *z, const float *delta_bias, int softplus_flag,
                         const float *initial_state, void *y, float *last_state, const ms_scan_dims *dims,
@@ -251,6 +362,16 @@ int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const 
         return MS_ERR_WORKSPACE;
     if (dims->batch == 0 || dims->dim == 0) return MS_OK;
     if (dims->seqlen == 0 && !last_state) return MS_OK;
+    if (!plan) {
+        const SplitPlan sp = split_plan(dims, num_sms_current());
+        if (sp.S > 1) {
+            if (!aligned(workspace, 16)) return MS_ERR_ALIGN;
+            rc = scan_split(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state, dims, sp,
+                            static_cast<float *>(workspace), dev_status, stream);
+            if (rc != MS_OK) cudaGetLastError();
+            return rc;
+        }
+    }
     return scan_common(u, delta, A, B, C, D, z, delta_bias, softplus_flag, initial_state, y, last_state,
                        dims, dev_status, stream, plan, nullptr);
 }

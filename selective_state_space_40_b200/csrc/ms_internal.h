@@ -33,7 +33,16 @@ struct ScanArgs {
     // Training: the state before every kCkptTokens-token block, [batch, dim,
     // ceil(L / kCkptTokens), N] fp32 (null: not written). y may be null then.
     float *ckpt;
+    // Sequence split: sum of Delta over the sequence per channel, [batch, dim]
+    // (null: not written). Like ckpt, it selects the saved-state kernels.
+    float *dsum;
 };
+
+// Carry combine of a sequence split into S segments for one batch row:
+// Sin[0] = h0 (or 0), Sin[k+1] = exp(A dsum[k]) Sin[k] + E[k], with E[k] the
+// end state of segment k scanned from zero and dsum[k] its sum of Delta.
+cudaError_t launch_carry_combine(const float *E, const float *dsum, const float *A, const float *h0, float *Sin,
+                                 int64_t dim, int N, int64_t S, cudaStream_t stream);
 
 // Tokens between two saved states of the forward (the backward recomputes
 // each block from its saved state).

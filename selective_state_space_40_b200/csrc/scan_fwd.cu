@@ -370,10 +370,11 @@ scan_fwd_kernel(const ScanArgs a) {
     if (ntiles > 0) prefetch(0);
 
     const int64_t nck = (L + kCkptTokens - 1) / kCkptTokens;
+    float dsum_acc = 0.0f;  // this lane's tokens' Delta (saved-state kernels)
     for (int64_t k = 0; k < ntiles; ++k) {
         const int64_t t0 = k * TT;
         const int buf = (int)(k & 1);
-        if (CKPT && active && t0 % kCkptTokens == 0) {
+        if (CKPT && a.ckpt != nullptr && active && t0 % kCkptTokens == 0) {
             // Training: the state before this block, for the backward's recompute.
             float *cs = a.ckpt + ((b * a.dim + d) * nck + t0 / kCkptTokens) * N;
 #pragma unroll
@@ -429,6 +430,7 @@ scan_fwd_kernel(const ScanArgs a) {
                 const float v = nd[i].get(j) + bias;
                 const float step = sp ? softplus_f(v) : v;
                 dl[i][j] = (ts + j < L) ? step : 0.0f;  // past the end: the state is left alone
+                if constexpr (CKPT) dsum_acc += dl[i][j];
                 dlu[i][j] = dl[i][j] * uj;
                 gate[i][j] = has_z ? silu_f(nz[i].get(j)) : 1.0f;
                 dug[i][j] = Dd * uj * gate[i][j];
@@ -540,6 +542,14 @@ scan_fwd_kernel(const ScanArgs a) {
         }
     }
 
+    if constexpr (CKPT) {
+        if (a.dsum != nullptr) {
+            // the channel's G lanes hold disjoint token chunks: sum them
+#pragma unroll
+            for (int off = 1; off < G; off <<= 1) dsum_acc += __shfl_xor_sync(0xffffffffu, dsum_acc, off);
+            if (active && g == 0) a.dsum[b * a.dim + d] = dsum_acc;
+        }
+    }
     if (active && a.last != nullptr) {
         float *ls = a.last + (b * a.dim + d) * N;
 #pragma unroll
@@ -639,7 +649,7 @@ cudaError_t launch_types_ckpt(const ScanArgs &a, const ScanPlan &pl, cudaStream_
 
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16,
                             cudaStream_t stream) {
-    if (a.ckpt != nullptr) {
+    if (a.ckpt != nullptr || a.dsum != nullptr) {
         if (plan.chunks_per_lane != 1 || (plan.poly8 != 0 && plan.poly8 != 8)) return cudaErrorInvalidValue;
         if (in_bf16) {
             return out_bf16 ? launch_types_ckpt<__nv_bfloat16, __nv_bfloat16>(a, plan, stream)
@@ -662,6 +672,35 @@ cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf1
     }
     return out_bf16 ? launch_types<float, __nv_bfloat16>(a, plan, stream)
                     : launch_types<float, float>(a, plan, stream);
+}
+
+namespace {
+
+__global__ void carry_combine_kernel(const float *E, const float *dsum, const float *A, const float *h0, float *Sin,
+                                     int64_t dim, int N, int64_t S) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;  // (d, n)
+    const int64_t cn = dim * N;
+    if (i >= cn) return;
+    const int64_t d = i / N;
+    const float a = A[i];
+    float st = h0 ? h0[i] : 0.0f;
+    Sin[i] = st;
+    for (int64_t k = 0; k + 1 < S; ++k) {
+        st = fmaf(expf(a * dsum[k * dim + d]), st, E[k * cn + i]);
+        Sin[(k + 1) * cn + i] = st;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_carry_combine(const float *E, const float *dsum, const float *A, const float *h0, float *Sin,
+                                 int64_t dim, int N, int64_t S, cudaStream_t stream) {
+    const int64_t cn = dim * N;
+    if (cn <= 0) return cudaSuccess;
+    const int64_t blocks = (cn + 255) / 256;
+    if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    carry_combine_kernel<<<(unsigned)blocks, 256, 0, stream>>>(E, dsum, A, h0, Sin, dim, N, S);
+    return cudaGetLastError();
 }
 
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms) {

@@ -218,3 +218,36 @@ def test_full_2p8b_sampled():
 @pytest.mark.slow
 def test_full_long_context_sampled():
     sampled_parity(syn.LONG, 10)
+
+
+# ------------------------------------------------------ sequence split ------
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("b,d,L", [(1, 64, 20000), (2, 40, 9000), (1, 128, 16384)])
+def test_sequence_split_against_oracle(dtype, b, d, L):
+    """Few channels and a long sequence: mamba_scan_fwd splits each row into
+    segments (ragged last segment for 20000 and 9000 tokens, equal segments
+    for 16384), chains the carries and rescans; every output is checked."""
+    w = syn.scaled(syn.LONG, batch=b, dim=d, seqlen=L, in_dtype=dtype, seed=L + d)
+    inp = syn.scan_inputs(w)
+    dims = mb.scan_dims_for(inp["u"], inp["delta"], inp["B"], inp["C"], inp["z"],
+                            torch.empty(b, d, L))
+    assert mb.mamba_scan_workspace_size(dims) > 0  # the split path runs
+    h0 = 0.5 * torch.randn(b, d, 16, generator=torch.Generator().manual_seed(4))
+    compare_full(inp, f"split b{b} d{d} L{L} {dtype}", initial_state=h0)
+
+
+@pytest.mark.parametrize("flags", [dict(use_z=False), dict(use_D=False), dict(use_bias=False)])
+def test_sequence_split_options(flags):
+    w = syn.scaled(syn.LONG, batch=1, dim=48, seqlen=12000, in_dtype=torch.float32, seed=77)
+    compare_full(syn.scan_inputs(w), f"split {flags}", **flags)
+
+
+def test_sequence_split_matches_unsplit_plan():
+    """The split result equals an explicit (never split) plan up to rounding."""
+    w = syn.scaled(syn.LONG, batch=1, dim=96, seqlen=16384, in_dtype=torch.bfloat16, seed=78)
+    inp = syn.scan_inputs(w)
+    y1, l1 = run_gpu(inp)
+    y0, l0 = run_gpu(inp, plan=(8, 1, 0))
+    check_fp32(f64(y1), f64(y0), "split vs unsplit y")
+    check_fp32(f64(l1), f64(l0), "split vs unsplit last_state")

@@ -600,7 +600,8 @@ def main(argv=None):
             "ssd_decode": {"workload": "mamba2-2.7b-class decode b64 H80 P64 N128 bf16, fp32 state",
                            "ms": ssd_dec_ms, "bytes": udbytes, "value": udbytes / (ssd_dec_ms * 1e-3) / 1e9,
                            "unit": "GB/s", "frac": udbytes / (ssd_dec_ms * 1e-3) / 1e9 / peak,
-                           "timing": "one event pair around 40 back-to-back steps over two rotating states"},
+                           "timing": "one event pair around 40 back-to-back steps over two rotating states",
+                           "traffic": recorded_traffic("ssd_decode")},
             "gpu_launches": args.steps,
             "clocks": clk.summary(),
             "cpu_baseline": cpu,

@@ -307,10 +307,6 @@ static int scan_split(const void *u, const void *delta, const float *A, const vo
         // a run of `nseg` segments starting at segment k0 as a batch of scans
         auto segments = [&](int64_t k0, int64_t nseg, int64_t len, const float *h0, void *yv, float *last,
                             float *ds) -> int {
-            ms_scan_dims v = *dims;
-            v.batch = nseg;
-            v.seqlen = len;
-            v.u_sb = v.delta_sb = v.z_sb = v.y_sb = v.B_sb = v.C_sb = Ls;
             const int64_t off = k0 * Ls;
             ms::ScanArgs a{};
             a.u = at(ub, off, ei); a.delta = at(db, off, ei); a.z = at(zb, off, ei);

@@ -19,7 +19,9 @@
 // registers and runs the adjoint back over those 8 tokens. Work split as in
 // the forward: 4 lanes per channel, 4 states each; a CTA holds 32 channels of
 // one batch row. B_t and C_t of the block are staged once per CTA as fp32
-// token rows. Sums over channels (dB, dC) are reduced within the warp by
+// token rows; u and dout of each sub-chunk reach shared memory by
+// asynchronous copies issued one sub-chunk ahead. Sums over channels (dB, dC)
+// are reduced within the warp by
 // reduce-scatter shuffles, across the CTA's warps in shared memory, then
 // added to global memory with fp32 atomics (run-to-run order of those adds
 // varies, so dB/dC/dA/dD/dbias can differ in the last bits between runs).
@@ -48,6 +50,11 @@ struct BwdSmem {
     float sub[kBNW][kNSub][4][32];       // state at each sub-chunk start [warp][s][state][lane]
     float red[2][kBNW][kSub][32];        // warp sums of dB/dC per token, two sub-chunks in turn
     float tok[4][kBNW][kCW][kBlk + 4];   // per channel and token: Delta, softplus', gate, gate'
+    // u and dout of one sub-chunk per channel in their storage format (up
+    // to 8 fp32), two steps in turn: filled by asynchronous copies one step
+    // ahead of their use
+    alignas(16) unsigned char raw_u[2][kBNW][kCW][32];
+    alignas(16) unsigned char raw_o[2][kBNW][kCW][32];
 };
 enum { kTokDelta = 0, kTokSig = 1, kTokGate = 2, kTokGateGrad = 3 };
 
@@ -75,6 +82,51 @@ __device__ __forceinline__ void load8(const T *row, int64_t t, int64_t L, bool v
     } else {
 #pragma unroll
         for (int j = 0; j < 8; ++j) v[j] = (t + j < L) ? ld_elem(row + t + j) : 0.0f;
+    }
+}
+
+// 16-byte asynchronous copy global -> shared (cached in L2 only).
+__device__ __forceinline__ void cp_async16(void *sdst, const void *gsrc) {
+    const unsigned d = static_cast<unsigned>(__cvta_generic_to_shared(sdst));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// Piece `piece` (16 bytes) of tokens [t, t+8) of `row` into dst, which holds
+// the 8 elements in their storage format (zero past L): an asynchronous copy
+// when the row allows 16-byte access, else element loads.
+template <typename T>
+__device__ __forceinline__ void stage8(unsigned char *dst, const T *row, int64_t t, int64_t L, bool vec, int piece) {
+    constexpr int kPer = 16 / (int)sizeof(T);  // elements per piece
+    if (vec && t + 8 <= L) {
+        cp_async16(dst + 16 * piece, row + t + kPer * piece);
+    } else {
+#pragma unroll
+        for (int j = 0; j < kPer; ++j) {
+            const int e = kPer * piece + j;
+            const int64_t tt = t + e;
+            if constexpr (sizeof(T) == 4) {
+                reinterpret_cast<float *>(dst)[e] = tt < L ? __ldg(reinterpret_cast<const float *>(row) + tt) : 0.0f;
+            } else {
+                reinterpret_cast<unsigned short *>(dst)[e] =
+                    tt < L ? __ldg(reinterpret_cast<const unsigned short *>(row) + tt) : (unsigned short)0;
+            }
+        }
+    }
+}
+// The 8 staged elements as fp32.
+template <typename T>
+__device__ __forceinline__ void unstage8(const unsigned char *src, float (&v)[8]) {
+    if constexpr (sizeof(T) == 4) {
+        const float4 a = reinterpret_cast<const float4 *>(src)[0];
+        const float4 b = reinterpret_cast<const float4 *>(src)[1];
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+        v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+        const uint4 w = *reinterpret_cast<const uint4 *>(src);
+        v[0] = bf16_lo(w.x); v[1] = bf16_hi(w.x); v[2] = bf16_lo(w.y); v[3] = bf16_hi(w.y);
+        v[4] = bf16_lo(w.z); v[5] = bf16_hi(w.z); v[6] = bf16_lo(w.w); v[7] = bf16_hi(w.w);
     }
 }
 
@@ -192,7 +244,33 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     const float *tk_gate = sm.tok[kTokGate][warp][c];
     const float *tk_gp = sm.tok[kTokGateGrad][warp][c];
 
+    // u and dout arrive one step ahead. The steps of block kb are numbered
+    // li = 0..15: pass A's sub-chunks 0..7 (u), then pass B's sub-chunks
+    // 7..0 (u and dout); step li uses buffer li & 1. The u piece(s) are
+    // copied by lanes g < kUPieces, the dout piece(s) by lanes 2, 3.
+    constexpr int kUPieces = 8 * (int)sizeof(TIn) / 16;
+    constexpr int kOPieces = 8 * (int)sizeof(TOut) / 16;
+    auto issue_step = [&](int64_t kb2, int li2) {
+        if (kb2 >= 0) {
+            const int s2 = li2 < kNSub ? li2 : 2 * kNSub - 1 - li2;
+            const int64_t t = kb2 * kBlk + s2 * kSub;
+            const int bf = li2 & 1;
+            if (g < kUPieces) stage8<TIn>(sm.raw_u[bf][warp][c], u_row, t, L, vin, g);
+            if (li2 >= kNSub && g >= 2 && g < 2 + kOPieces) stage8<TOut>(sm.raw_o[bf][warp][c], o_row, t, L, vout, g - 2);
+        }
+        cp_async_commit();  // one group per step, empty past the last
+    };
+    // start of step li of block kb: issue the next step's copies, wait for this one's
+    auto begin_step = [&](int64_t kb2, int li2) {
+        __syncwarp();  // every lane is done with the buffers the next copies fill
+        const bool wrap = li2 == 2 * kNSub - 1;
+        issue_step(wrap ? kb2 - 1 : kb2, wrap ? 0 : li2 + 1);
+        cp_async_wait1();
+        __syncwarp();
+    };
+
     const int64_t nblk = (L + kBlk - 1) / kBlk;
+    if (nblk > 0) issue_step(nblk - 1, 0);
     for (int64_t kb = nblk - 1; kb >= 0; --kb) {
         const int64_t tb = kb * kBlk;
         __syncthreads();  // the previous block is done with bc and tok
@@ -255,8 +333,9 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 sm.sub[warp][s][2 * p][lane] = lo;
                 sm.sub[warp][s][2 * p + 1][lane] = hi;
             }
+            begin_step(kb, s);
             float uv[8];
-            load8(u_row, tb + s * kSub, L, vin, uv);
+            unstage8<TIn>(sm.raw_u[s & 1][warp][c], uv);
             const F4 dl0 = lds4(tk_dl + s * kSub), dl1 = lds4(tk_dl + s * kSub + 4);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) {
@@ -273,11 +352,13 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
         for (int s = kNSub - 1; s >= 0; --s) {
             const int64_t ts = tb + s * kSub;
             const int rb = s & 1;
+            const int li = 2 * kNSub - 1 - s;
+            begin_step(kb, li);
             float uv[8], ov[8];
-            load8(u_row, ts, L, vin, uv);
+            unstage8<TIn>(sm.raw_u[li & 1][warp][c], uv);
             // an idle lane (channel past dim) gets dout = 0: with its zero
             // starting adjoint every contribution to the channel sums is 0
-            if (active) load8(o_row, ts, L, vout, ov);
+            unstage8<TOut>(sm.raw_o[li & 1][warp][c], ov);
 #pragma unroll
             for (int j = 0; j < kSub; ++j) ov[j] = active ? ov[j] : 0.0f;
             float dl[8], gate[8];

@@ -24,7 +24,10 @@
 // bf16 inputs (the scaled G', B' and the state) are split into a high and a
 // low bf16 part, v = hi + lo, and both parts are multiplied, which keeps
 // about 16 significant bits. The next chunk's inputs are copied in
-// asynchronously while the current one computes.
+// asynchronously while the current one computes. A chunk has two phases
+// between barriers: (1) the readout of the entering state, the masked C B^T
+// and the weighted, split x^T; (2) the intra-chunk product, the output and
+// the state update.
 
 #include <cstdint>
 
@@ -44,13 +47,13 @@ constexpr int kST = kSW * 32;     // threads
 // words of one fragment load fall in 32 distinct banks.
 constexpr int kLdN = kN + 8;      // rows of K = N
 constexpr int kLdQ = kQ + 8;      // rows of K = Q
+constexpr int kLdP = kP + 8;      // x rows (p contiguous): 8 rows of a transposing fragment load hit distinct banks
 static_assert(kQ == 32, "warp 0 handles one token of the chunk per lane");
 
 struct SsdSmem {
     __nv_bfloat16 C[2][kQ][kLdN];     // C_t [t][n], this chunk and the next (copies in flight)
     __nv_bfloat16 B[2][kQ][kLdN];     // B_s [s][n]
-    __nv_bfloat16 X[2][kQ][kP];       // x [s][p] as loaded
-    __nv_bfloat16 Xt[kP][kLdQ];       // x^T [p][s]
+    __nv_bfloat16 X[2][kQ][kLdP];     // x [s][p] as loaded
     __nv_bfloat16 G[2][kQ][kLdQ];     // G' hi / lo [t][s]
     __nv_bfloat16 Xw[2][kP][kLdQ];    // (x_s w_s)^T hi / lo [p][s], w_s = exp(cs_Q - cs_s) Delta_s
     // per-token chunk parameters, for this chunk and the next
@@ -218,22 +221,27 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
         const int64_t t0 = ck * kQ;
         const int buf = (int)(ck & 1);
         asm volatile("cp.async.wait_group 0;" ::: "memory");
-        __syncthreads();  // chunk ck in buf for everyone; the previous chunk's tiles are free
-        // ---- x^T and (x w)^T (hi / lo) for the products
-        const float *pcs = sm.cs[buf], *pdl = sm.dl[buf], *pwq = sm.wq[buf], *pecs = sm.ecs[buf];
-        for (int i = tid; i < kQ * kP; i += kST) {
-            const int t = i / kP, p = i % kP;
-            const __nv_bfloat16 xv = sm.X[buf][t][p];
-            sm.Xt[p][t] = xv;
-            split_bf16(__bfloat162float(xv) * pwq[t], sm.Xw[0][p][t], sm.Xw[1][p][t]);
-        }
-        // next chunk's copies run under this chunk's products
+        __syncthreads();  // chunk ck in buf for everyone; chunk ck-1 is done with every tile
+        // next chunk's copies (into the buffers chunk ck-1 used) run under this chunk's products
         if (ck + 1 < nch) {
             issue_chunk(ck + 1, buf ^ 1);
             load_dt(ck + 1);
         }
-        __syncthreads();
+        const float *pcs = sm.cs[buf], *pdl = sm.dl[buf], *pwq = sm.wq[buf], *pecs = sm.ecs[buf];
         const float cs_end = pcs[kQ - 1];
+        // ---- (x w)^T, hi / lo: warp task = 8 rows p x 8 tokens s; lane
+        // (r, k) = (lane / 4, lane % 4) converts tokens 2k, 2k+1 of row r
+        // (one bf16 pair per part: 32 distinct banks per store)
+        for (int task = warp; task < (kP / 8) * (kQ / 8); task += kSW) {
+            const int p = 8 * (task % (kP / 8)) + (lane >> 2);
+            const int s = 8 * (task / (kP / 8)) + 2 * (lane & 3);
+            const float x0 = __bfloat162float(sm.X[buf][s][p]) * pwq[s];
+            const float x1 = __bfloat162float(sm.X[buf][s + 1][p]) * pwq[s + 1];
+            uint32_t hi, lo;
+            split_pair(x0, x1, hi, lo);
+            *reinterpret_cast<uint32_t *>(&sm.Xw[0][p][s]) = hi;
+            *reinterpret_cast<uint32_t *>(&sm.Xw[1][p][s]) = lo;
+        }
 
         // ---- Y^T = S_in^T C^T, columns scaled by exp(cs_t): the state
         // accumulators are the A operand (hi and lo parts), C rows the B operand
@@ -306,8 +314,11 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
         // ---- Y^T += X^T G'^T over the causal part, then y = Y + D x
 #pragma unroll
         for (int k0 = 0; k0 < kQ; k0 += 16) {
+            // A = x^T rows p, columns s: transposing loads of the x tile
+            // (matrix i = lane / 8: rows p + 8 (i & 1), tokens k0 + 8 (i / 2))
             uint32_t af[4];
-            ldsm_a(&sm.Xt[0][0], kLdQ, pw, k0, lane, af);
+            ldsm_x4_trans(&sm.X[buf][k0 + 8 * (lane >> 4) + (lane & 7)][pw + 8 * ((lane >> 3) & 1)], af[0], af[1],
+                          af[2], af[3]);
 #pragma unroll
             for (int part = 0; part < 2; ++part)
 #pragma unroll
@@ -326,7 +337,7 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
                 const int p = pw + gid + (e >= 2 ? 8 : 0);
                 const int t = 8 * nt + 2 * tig + (e & 1);
                 if (t0 + t < L) {
-                    const float v = yacc[nt][e] + Dh * __bfloat162float(sm.Xt[p][t]);
+                    const float v = yacc[nt][e] + Dh * __bfloat162float(sm.X[buf][t][p]);
                     TOut *dst = yb + (t0 + t) * a.y_sl + p;
                     if constexpr (sizeof(TOut) == 4) *dst = v;
                     else *dst = __float2bfloat16_rn(v);

@@ -48,7 +48,10 @@ constexpr int kST = kSW * 32;     // threads
 constexpr int kLdN = kN + 8;      // rows of K = N
 constexpr int kLdQ = kQ + 8;      // rows of K = Q
 constexpr int kLdP = kP + 8;      // x rows (p contiguous): 8 rows of a transposing fragment load hit distinct banks
-static_assert(kQ == 32, "warp 0 handles one token of the chunk per lane");
+static_assert(kQ == 32, "one warp handles one token of the chunk per lane");
+// the warp that prepares the chunk parameters (its tile of C B^T lies above
+// the diagonal, so its share of that product is a zero fill)
+constexpr int kParamWarp = 2;
 
 struct SsdSmem {
     __nv_bfloat16 C[2][kQ][kLdN];     // C_t [t][n], this chunk and the next (copies in flight)
@@ -168,7 +171,7 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
     const int64_t nch = (L + kQ - 1) / kQ;
     // Chunk inputs arrive by asynchronous copies one chunk ahead (rows past L
     // are zero-filled); dt goes through a register, one token per thread of
-    // warp 0.
+    // the parameter warp.
     auto issue_chunk = [&](int64_t ck, int buf) {
         const int64_t t0 = ck * kQ;
         for (int i = tid; i < kQ * (kN / 8); i += kST) {
@@ -189,12 +192,12 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
     float dt_next = 0.0f;
     auto load_dt = [&](int64_t ck) {
         const int64_t t = ck * kQ + lane;
-        dt_next = (warp == 0 && t < L) ? ld1(dtb + t * a.dt_sl) : 0.0f;
+        dt_next = (warp == kParamWarp && t < L) ? ld1(dtb + t * a.dt_sl) : 0.0f;
     };
-    // warp 0: Delta, the decay prefix and the per-token weights of chunk ck
+    // parameter warp: Delta, the decay prefix and the per-token weights of chunk ck
     // (its dt already in dt_next) into parameter buffer pb
     auto chunk_params = [&](int64_t ck, int pb) {
-        if (warp != 0) return;
+        if (warp != kParamWarp) return;
         float d = 0.0f;
         if (ck * kQ + lane < L) {
             const float v = dt_next + bias;
@@ -309,6 +312,9 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
                 }
             }
         }
+        // the next chunk's parameters (its dt has arrived during this phase);
+        // this chunk's were read above, the next chunk reads them after a barrier
+        if (ck + 1 < nch) chunk_params(ck + 1, buf ^ 1);
         __syncthreads();
 
         // ---- Y^T += X^T G'^T over the causal part, then y = Y + D x
@@ -368,8 +374,6 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
                 mma_bf16(sacc[j + 1], al[0], al[1], al[2], al[3], b2, b3);
             }
         }
-        // warp 0 prepares the next chunk's parameters (its dt has arrived)
-        if (ck + 1 < nch) chunk_params(ck + 1, buf ^ 1);
     }
 
     if (a.s_last != nullptr) {

@@ -297,18 +297,24 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 #pragma unroll
                 for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int t = gm + gid + (e >= 2 ? 8 : 0);
-                        const int s = gn + 8 * nt + 2 * tig + (e & 1);
-                        const float v = s <= t ? gacc[nt][e] * __expf(pcs[t] - pcs[s]) * pdl[s] : 0.0f;
-                        split_bf16(v, sm.G[0][t][s], sm.G[1][t][s]);
+                    for (int r = 0; r < 2; ++r) {
+                        // elements (t, s) and (t, s + 1): one bf16 pair per part
+                        const int t = gm + gid + 8 * r;
+                        const int s = gn + 8 * nt + 2 * tig;
+                        const float v0 = s <= t ? gacc[nt][2 * r] * __expf(pcs[t] - pcs[s]) * pdl[s] : 0.0f;
+                        const float v1 =
+                            s + 1 <= t ? gacc[nt][2 * r + 1] * __expf(pcs[t] - pcs[s + 1]) * pdl[s + 1] : 0.0f;
+                        uint32_t hi, lo;
+                        split_pair(v0, v1, hi, lo);
+                        *reinterpret_cast<uint32_t *>(&sm.G[0][t][s]) = hi;
+                        *reinterpret_cast<uint32_t *>(&sm.G[1][t][s]) = lo;
                     }
             } else {
                 // strictly above the diagonal: zeros
-                for (int i = lane; i < 16 * 16; i += 32) {
-                    const int t = gm + i / 16, s = gn + i % 16;
-                    sm.G[0][t][s] = __float2bfloat16_rn(0.0f);
-                    sm.G[1][t][s] = __float2bfloat16_rn(0.0f);
+                for (int i = lane; i < 16 * 8; i += 32) {
+                    const int t = gm + i / 8, s = gn + 2 * (i % 8);
+                    *reinterpret_cast<uint32_t *>(&sm.G[0][t][s]) = 0u;
+                    *reinterpret_cast<uint32_t *>(&sm.G[1][t][s]) = 0u;
                 }
             }
         }

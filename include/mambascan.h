@@ -308,6 +308,24 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
                    ms_stream_t stream);
 
 /*
+ * Mamba-2 SSD layer: the intra-chunk products of the chunked matrix view
+ * ('Mamba-1/2/3 Markdown図解' blog, section 3: inside a chunk the output is
+ * built from the products C_t . B_s of the chunk's tokens), for chunks of 32
+ * tokens, computed on the tcgen05 tensor cores once per group:
+ *     cb[b][g][k][i][j] = sum_n C[b, 32k+i, g, n] B[b, 32k+j, g, n]
+ * for i, j < 32 (tokens at or past seqlen count as zero). cb is [batch,
+ * ngroups, ceil(seqlen / 32), 32, 32] fp32, dense, caller-owned device memory
+ * of mamba2_ssd_chunk_cb_size() bytes, 16-byte aligned. B, C and their
+ * fields of dims are as for mamba2_ssd_fwd (bf16, dstate 128, rows 16-byte
+ * aligned: MS_ERR_DTYPE / MS_ERR_SHAPE / MS_ERR_ALIGN otherwise); the other
+ * fields of dims are not read. dev_status receives MS_ERR_TIMEOUT if a
+ * product did not complete within the kernel's bounded wait.
+ */
+size_t mamba2_ssd_chunk_cb_size(const ms_ssd_dims *dims);
+int mamba2_ssd_chunk_cb(const void *B, const void *C, float *cb, const ms_ssd_dims *dims, int *dev_status,
+                        ms_stream_t stream);
+
+/*
  * Mamba-2 SSD layer, one token (decode): the recurrent view of the same model
  * (blog, section 3: generation updates the state once per token). For batch
  * row b, head h, group g = h / (nheads / ngroups):

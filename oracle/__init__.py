@@ -15,6 +15,7 @@ from .oracle import (  # noqa: F401
     scan_bwd,
     scan_mt,
     ssd,
+    ssd_chunk_cb,
     state_update,
     softplus,
     silu,

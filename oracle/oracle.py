@@ -194,6 +194,27 @@ def ssd(x, dt, A, B, C, D=None, dt_bias=None, softplus_flag=True, s0=None, lib=N
     return y, last
 
 
+def ssd_chunk_cb(B, C, chunk: int = 32):
+    """The intra-chunk products of the SSD matrix view ('Mamba-1/2/3
+    Markdown図解' blog, section 3: inside a chunk the output is built from
+    C_t . B_s of the chunk's tokens), fp64, by definition: for chunk k and
+    i, j < chunk, cb[b, g, k, i, j] = sum_n C[b, k*chunk+i, g, n] *
+    B[b, k*chunk+j, g, n], tokens at or past L counting as zero (one matrix
+    product per chunk). B, C [b, L, G, N]; returns [b, G, ceil(L / chunk),
+    chunk, chunk]."""
+    B, C = _f64(B), _f64(C)
+    batch, L, G, N = B.shape
+    assert C.shape == B.shape
+    nch = (L + chunk - 1) // chunk
+    out = np.zeros((batch, G, nch, chunk, chunk))
+    for k in range(nch):
+        t0, t1 = k * chunk, min(L, (k + 1) * chunk)
+        for b in range(batch):
+            for g in range(G):
+                out[b, g, k, : t1 - t0, : t1 - t0] = C[b, t0:t1, g, :] @ B[b, t0:t1, g, :].T
+    return out
+
+
 def causal_conv(x, w, bias=None, x0=None, silu_flag=True, lib=None):
     """Causal depthwise convolution + silu of the block's input path, fp64.
     x [batch, dim, L]; w [dim, W]; bias [dim]; x0 [batch, dim, W-1] (the W-1

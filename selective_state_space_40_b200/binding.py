@@ -106,6 +106,10 @@ def library() -> ctypes.CDLL:
         lib.mamba_scan_bwd_noalloc.restype = ctypes.c_int
         lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
+        lib.mamba2_ssd_chunk_cb_size.argtypes = [ctypes.POINTER(SsdDims)]
+        lib.mamba2_ssd_chunk_cb_size.restype = ctypes.c_size_t
+        lib.mamba2_ssd_chunk_cb.argtypes = [_vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
+        lib.mamba2_ssd_chunk_cb.restype = ctypes.c_int
         lib.mamba2_ssd_state_update.argtypes = [_vp] * 8 + [ctypes.c_int, _vp, ctypes.POINTER(SsdUpdateDims),
                                                             _vp, _vp]
         lib.mamba2_ssd_state_update.restype = ctypes.c_int
@@ -187,6 +191,14 @@ def mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus_flag, i
     return library().mamba_scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, int(softplus_flag),
                                             initial_state, dout, dlast, du, ddelta, dA, dB, dC, dD, dz,
                                             ddelta_bias, dinitial_state, ctypes.byref(dims), dev_status, stream)
+
+
+def mamba2_ssd_chunk_cb_size(dims: SsdDims) -> int:
+    return library().mamba2_ssd_chunk_cb_size(ctypes.byref(dims))
+
+
+def mamba2_ssd_chunk_cb(B, C, cb, dims: SsdDims, dev_status=None, stream=None) -> int:
+    return library().mamba2_ssd_chunk_cb(B, C, cb, ctypes.byref(dims), dev_status, stream)
 
 
 def mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, softplus_flag, initial_state, y, final_state, dims: SsdDims,
@@ -452,6 +464,24 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba2_ssd_fwd")
     return y, fs
+
+
+def ssd_chunk_cb(B, C, cb=None, stream=None, dev_status=None):
+    """Per-chunk products C_t . B_s (chunks of 32 tokens) of B/C [b, L, G,
+    128] bf16 CUDA tensors, through mamba2_ssd_chunk_cb (tcgen05 tensor
+    cores). Returns cb [b, G, ceil(L / 32), 32, 32] fp32."""
+    torch = _torch()
+    batch, L, G, N = B.shape
+    for t, n in ((B, "B"), (C, "C")):
+        _inner_contiguous(t, n)
+    if cb is None:
+        cb = torch.empty((batch, G, (L + 31) // 32, 32, 32), dtype=torch.float32, device=B.device)
+    dims = SsdDims(batch, L, 1, 64, N, G, 0, 0, 0, 0, 0, B.stride(0), B.stride(1), B.stride(2), C.stride(0),
+                   C.stride(1), C.stride(2), 0, 0, 0, _dtype_code(B), MS_F32)
+    rc = mamba2_ssd_chunk_cb(_ptr(B), _ptr(C), _ptr(cb), dims, _ptr(dev_status), _stream_handle(stream))
+    if rc != MS_OK:
+        raise MambaScanError(rc, "mamba2_ssd_chunk_cb")
+    return cb
 
 
 def ssd_state_update(state, x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, out_dtype=None,

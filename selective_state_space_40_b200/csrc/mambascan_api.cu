@@ -580,6 +580,42 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
     return MS_OK;
 }
 
+size_t mamba2_ssd_chunk_cb_size(const ms_ssd_dims *dm) {
+    if (!dm || dm->batch < 0 || dm->seqlen < 0 || dm->ngroups < 1) return 0;
+    return (size_t)dm->batch * (size_t)dm->ngroups * (size_t)((dm->seqlen + 31) / 32) * 32 * 32 * sizeof(float);
+}
+
+int mamba2_ssd_chunk_cb(const void *B, const void *C, float *cb, const ms_ssd_dims *dm, int *dev_status,
+                        ms_stream_t stream) {
+    if (!dm) return MS_ERR_NULL;
+    if (dm->in_dtype != MS_BF16) return MS_ERR_DTYPE;
+    if (dm->batch < 0 || dm->seqlen < 0 || dm->ngroups < 1 || !ms::ssd_cb_shape_supported(dm->dstate))
+        return MS_ERR_SHAPE;
+    if (dm->B_sb < 0 || dm->B_sl < 0 || dm->B_sg < 0 || dm->C_sb < 0 || dm->C_sl < 0 || dm->C_sg < 0)
+        return MS_ERR_STRIDE;
+    if (dm->batch == 0 || dm->seqlen == 0) return MS_OK;
+    if (!B || !C || !cb) return MS_ERR_NULL;
+    auto rows16 = [](const void *p, int64_t s1, int64_t s2, int64_t s3) {
+        return aligned(p, 16) && (s1 * 2) % 16 == 0 && (s2 * 2) % 16 == 0 && (s3 * 2) % 16 == 0;
+    };
+    if (!rows16(B, dm->B_sb, dm->B_sl, dm->B_sg) || !rows16(C, dm->C_sb, dm->C_sl, dm->C_sg) || !aligned(cb, 16))
+        return MS_ERR_ALIGN;
+    const int64_t L = dm->seqlen, G = dm->ngroups;
+    if (max_offset3(dm->batch, dm->B_sb, L, dm->B_sl, 1) < 0 || max_offset3(G, dm->B_sg, 1, 0, 128) < 0 ||
+        max_offset3(dm->batch, dm->C_sb, L, dm->C_sl, 1) < 0 || max_offset3(G, dm->C_sg, 1, 0, 128) < 0)
+        return MS_ERR_SHAPE;
+    ms::SsdCbArgs a{};
+    a.B = B; a.C = C; a.cb = cb; a.status = dev_status;
+    a.batch = dm->batch; a.L = L; a.G = G;
+    a.B_sb = dm->B_sb; a.B_sl = dm->B_sl; a.B_sg = dm->B_sg;
+    a.C_sb = dm->C_sb; a.C_sl = dm->C_sl; a.C_sg = dm->C_sg;
+    if (ms::launch_ssd_chunk_cb(a, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+}
+
 int mamba2_ssd_state_update(float *state, const void *x, const void *dt, const float *A, const void *B,
                             const void *C, const float *D, const float *dt_bias, int softplus_flag, void *y,
                             const ms_ssd_update_dims *dm, int *dev_status, ms_stream_t stream) {

@@ -77,6 +77,18 @@ struct SsdArgs {
 };
 bool ssd_shape_supported(int64_t headdim, int64_t dstate);
 
+// Arguments of the per-chunk C B^T of the SSD layer (bf16 B, C with dstate
+// 128; cb [batch, G, ceil(L / 32), 32, 32] fp32, dense).
+struct SsdCbArgs {
+    const void *B, *C;
+    float *cb;
+    int *status;
+    int64_t batch, L, G;
+    int64_t B_sb, B_sl, B_sg, C_sb, C_sl, C_sg;
+};
+bool ssd_cb_shape_supported(int64_t dstate);
+cudaError_t launch_ssd_chunk_cb(const SsdCbArgs &a, cudaStream_t stream);
+
 // Arguments of the Mamba-2 SSD one-token state update (state [b, H, P, 128]
 // fp32, each head's [P, 128] block dense).
 struct SsdUpdArgs {

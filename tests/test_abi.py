@@ -24,7 +24,7 @@ def declared_functions():
     for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
         text = open(h).read()
         text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(mamba_\w+)\s*\(", text, flags=re.M):
+        for m in re.finditer(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(mamba2?_\w+)\s*\(", text, flags=re.M):
             names.add(m.group(1))
     return sorted(names)
 
@@ -33,7 +33,8 @@ def test_header_declares_entry_points():
     names = declared_functions()
     for n in ("mamba_scan_fwd", "mamba_state_update", "mamba_scan_workspace_size",
               "mamba_status_string", "mamba_device_check", "mamba_scan_fwd_plan",
-              "mamba_scan_choose_plan", "mamba_conv_scan_fwd"):
+              "mamba_scan_choose_plan", "mamba_conv_scan_fwd", "mamba2_ssd_fwd", "mamba2_ssd_state_update",
+              "mamba2_ssd_chunk_cb", "mamba2_ssd_chunk_cb_size"):
         assert n in names
 
 
@@ -224,6 +225,24 @@ def test_ssd_rejects_bad_arguments(lib):
     assert call(_sdims(B_sl=132)) == mb.MS_ERR_ALIGN         # row stride not a multiple of 8 elements
     assert call(_sdims(), y=FAKE + 4) == mb.MS_ERR_ALIGN      # fp32 pairs need 8-byte alignment
     assert call(_sdims(batch=0)) == mb.MS_OK
+
+
+def test_ssd_chunk_cb_rejects_bad_arguments(lib):
+    def call(dims, B=FAKE, C=FAKE, cb=FAKE):
+        return mb.mamba2_ssd_chunk_cb(B, C, cb, dims, None, None)
+    assert call(_sdims(dstate=64)) == mb.MS_ERR_SHAPE
+    assert call(_sdims(ngroups=0)) == mb.MS_ERR_SHAPE
+    assert call(_sdims(in_dtype=mb.MS_F32)) == mb.MS_ERR_DTYPE
+    assert call(_sdims(C_sl=-1)) == mb.MS_ERR_STRIDE
+    assert call(_sdims(), cb=None) == mb.MS_ERR_NULL
+    assert call(_sdims(), B=FAKE + 2) == mb.MS_ERR_ALIGN
+    assert call(_sdims(C_sl=132)) == mb.MS_ERR_ALIGN
+    assert call(_sdims(), cb=FAKE + 8) == mb.MS_ERR_ALIGN
+    assert call(_sdims(batch=0)) == mb.MS_OK
+    assert call(_sdims(seqlen=0)) == mb.MS_OK
+    # batch 2, 1 group, 64 tokens = 2 chunks of 32 x 32 fp32
+    assert mb.mamba2_ssd_chunk_cb_size(_sdims()) == 2 * 1 * 2 * 32 * 32 * 4
+    assert mb.mamba2_ssd_chunk_cb_size(_sdims(seqlen=65, ngroups=2)) == 2 * 2 * 3 * 32 * 32 * 4
 
 
 def test_ssd_update_rejects_bad_arguments(lib):

@@ -187,3 +187,39 @@ def test_decode_steps_equal_chunked_forward():
     yd = torch.stack(ys, dim=1)
     check_bf16(f64(yd), f64(yf), "decode steps vs chunked y")
     check_bf16(f64(st), f64(sf), "decode steps vs chunked final state")
+
+
+@pytest.mark.parametrize("batch,L,G,strided", [(1, 1, 1, False), (1, 128, 1, False), (2, 300, 2, False),
+                                               (1, 2048, 1, False), (2, 200, 2, True)])
+def test_chunk_cb_tcgen05_against_oracle(batch, L, G, strided):
+    # mamba2_ssd_chunk_cb (tcgen05 tensor cores, fp32 accumulation of exact
+    # bf16 products) against the oracle's per-chunk C B^T of the same values:
+    # only the summation order differs.
+    gen = torch.Generator().manual_seed(100 + L)
+    if strided:
+        # B and C as slices of one projection tensor [b, L, 2 G 128 + 64]
+        proj = torch.randn(batch, L, 2 * G * 128 + 64, generator=gen).to(torch.bfloat16)
+        B = proj[:, :, 64:64 + G * 128].unflatten(-1, (G, 128))
+        C = proj[:, :, 64 + G * 128:].unflatten(-1, (G, 128))
+    else:
+        B = torch.randn(batch, L, G, 128, generator=gen).to(torch.bfloat16)
+        C = torch.randn(batch, L, G, 128, generator=gen).to(torch.bfloat16)
+    cb = mb.ssd_chunk_cb(B.to(DEV), C.to(DEV)).cpu().double().numpy()
+    ref = oracle.ssd_chunk_cb(f64(B), f64(C))
+    assert cb.shape == ref.shape
+    # fp32 summation of 128 exact products in any order: error <= 127 u sum |C_n B_n|
+    bound = 127 * 2.0 ** -24 * oracle.ssd_chunk_cb(np.abs(f64(B)), np.abs(f64(C)))
+    assert np.all(np.abs(cb - ref) <= bound + 1e-30), float(np.max(np.abs(cb - ref) - bound))
+
+
+def test_chunk_cb_tcgen05_zero_rows_and_repeat():
+    # zero B rows give zero columns; two calls give identical results
+    gen = torch.Generator().manual_seed(3)
+    B = torch.randn(1, 96, 1, 128, generator=gen).to(torch.bfloat16)
+    C = torch.randn(1, 96, 1, 128, generator=gen).to(torch.bfloat16)
+    B[:, 40:48] = 0
+    cb1 = mb.ssd_chunk_cb(B.to(DEV), C.to(DEV))
+    cb2 = mb.ssd_chunk_cb(B.to(DEV), C.to(DEV))
+    torch.cuda.synchronize()
+    assert torch.equal(cb1, cb2)
+    assert float(cb1[0, 0, 1, :, 8:16].abs().max()) == 0.0

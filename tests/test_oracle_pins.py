@@ -448,6 +448,33 @@ def pin_ssd_split_resume(lib):
     return max(_rel(np.concatenate([y1, y2], axis=1), y), _rel(l2, last))
 
 
+
+def pin_ssd_chunk_cb_is_intra_chunk_product(lib):
+    # No decay (A = 0), Delta = 1 (no softplus, dt = 1, no bias), no D skip and
+    # a zero state entering each chunk: the recurrence's output inside a chunk
+    # is then exactly sum_{s <= t} (C_t . B_s) x_s, i.e. the lower triangle of
+    # the chunk's cb block times x. Chunk 0 of a 40-token run, and chunk 1 as
+    # a run of its own tokens from a zero state.
+    rng = np.random.default_rng(26)
+    b, L, H, P, N, G = 2, 40, 2, 3, 5, 2
+    x = rng.standard_normal((b, L, H, P))
+    B = rng.standard_normal((b, L, G, N))
+    C = rng.standard_normal((b, L, G, N))
+    cb = oracle.ssd_chunk_cb(B, C)
+    worst = 0.0
+    for k, (t0, t1) in enumerate(((0, 32), (32, 40))):
+        n = t1 - t0
+        y, _ = oracle.ssd(x[:, t0:t1], np.ones((b, n, H)), np.zeros(H), B[:, t0:t1], C[:, t0:t1], None, None,
+                          False, None, lib=lib)
+        for bi in range(b):
+            for h in range(H):
+                g = h // (H // G)
+                ref = np.tril(cb[bi, g, k, :n, :n]) @ x[bi, t0:t1, h]
+                worst = max(worst, _rel(y[bi, :, h], ref))
+    # rows and columns past the sequence are zero
+    worst = max(worst, float(np.abs(cb[:, :, 1, 8:, :]).max()), float(np.abs(cb[:, :, 1, :, 8:]).max()))
+    return worst
+
 PINS = {
     "softplus_silu": pin_softplus_silu,
     "lti_convolution": pin_lti_convolution,
@@ -465,6 +492,7 @@ PINS = {
     "ssd_matrix_view": pin_ssd_matrix_view,
     "ssd_is_mamba1_with_scalar_heads": pin_ssd_is_mamba1_with_scalar_heads,
     "ssd_split_resume": pin_ssd_split_resume,
+    "ssd_chunk_cb_is_intra_chunk_product": pin_ssd_chunk_cb_is_intra_chunk_product,
 }
 
 # Pins that compare against a numerical approximation carry their own bound.

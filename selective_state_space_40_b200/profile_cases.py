@@ -7,8 +7,9 @@ CASE is one of: scan130m (selective scan forward, 130M-class layer),
 conv130m (the same with the causal conv front-end, width 4), decode (one
 state update at b256 d5120 N16), bwd130m_b4 (training forward with saved
 states, then the backward, 130M-class layer with 4 batch rows), ssd2p7b_b2
-(Mamba-2 SSD layer, 2.7B-class with 2 batch rows). Each kernel of the case
-runs REPEATS times (default 3).
+(Mamba-2 SSD layer, 2.7B-class with 2 batch rows), ssdcb2p7b (the per-chunk
+C B^T of that layer on the tcgen05 tensor cores, 4 batch rows). Each kernel
+of the case runs REPEATS times (default 3).
 """
 from __future__ import annotations
 
@@ -64,12 +65,21 @@ def _ssd(reps):
         mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True, return_final_state=False)
 
 
+def _ssd_cb(reps):
+    w = syn.SSD_2P7B
+    g = {k: v.cuda() for k, v in syn.ssd_inputs(w).items()}
+    cb = torch.empty(w.batch, w.ngroups, (w.seqlen + 31) // 32, 32, 32, device="cuda")
+    for _ in range(reps):
+        mb.ssd_chunk_cb(g["B"], g["C"], cb=cb)
+
+
 CASES = {
     "scan130m": lambda r: _scan(r),
     "conv130m": lambda r: _scan(r, conv=True),
     "decode": _decode,
     "bwd130m_b4": _bwd,
     "ssd2p7b_b2": _ssd,
+    "ssdcb2p7b": _ssd_cb,
 }
 
 

@@ -55,3 +55,37 @@ def test_some_pin_catches_mutant(mutant, mutant_dir):
         if not (err <= pin_tol(name)):
             caught.append(name)
     assert caught, f"no pin caught mutant {mutant} ({MUTANTS[mutant]})"
+
+
+# The per-chunk C B^T of the SSD matrix view is a numpy definition in
+# oracle.oracle; its mutants replace that function for one pin run.
+def _cb_transposed(B, C, chunk=32):
+    return np.swapaxes(_CB_REAL(B, C, chunk), -1, -2)
+
+
+def _cb_chunk_shifted(B, C, chunk=32):
+    # chunk k built from the tokens one position later
+    return _CB_REAL(np.roll(B, -1, axis=1), np.roll(C, -1, axis=1), chunk)
+
+
+def _cb_tail_not_zero(B, C, chunk=32):
+    # tokens past L taken from the start of the sequence instead of zero
+    batch, L = B.shape[:2]
+    pad = (-L) % chunk
+    Bp = np.concatenate([B, B[:, :pad]], axis=1)
+    Cp = np.concatenate([C, C[:, :pad]], axis=1)
+    return _CB_REAL(Bp, Cp, chunk)
+
+
+_CB_REAL = ow.ssd_chunk_cb
+CB_MUTANTS = {"transposed": _cb_transposed, "chunk shifted by a token": _cb_chunk_shifted,
+              "tail past L not zero": _cb_tail_not_zero}
+
+
+@pytest.mark.parametrize("name", sorted(CB_MUTANTS))
+def test_chunk_cb_pin_catches_mutant(name, oracle_lib, monkeypatch):
+    monkeypatch.setattr(ow, "ssd_chunk_cb", CB_MUTANTS[name])
+    import oracle
+    monkeypatch.setattr(oracle, "ssd_chunk_cb", CB_MUTANTS[name])
+    pin = "ssd_chunk_cb_is_intra_chunk_product"
+    assert PINS[pin](oracle_lib) > pin_tol(pin), f"pin {pin} misses the mutant '{name}'"

@@ -99,9 +99,29 @@ def measured_bf16_tflops():
         return 1590.0
 
 
-def csrc_digest():
+# Sources that decide what a recorded kernel does: its own file, the shared
+# device and argument headers, the public header and the ABI layer (which
+# chooses the launch).
+_SHARED_SOURCES = ("selective_state_space_40_b200/csrc/ms_device.cuh", "selective_state_space_40_b200/csrc/ms_internal.h",
+                   "selective_state_space_40_b200/csrc/mambascan_api.cu", "include/mambascan.h")
+KERNEL_SOURCES = {
+    "scan_fwd_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
+    "conv_scan_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
+    "decode_step": ("selective_state_space_40_b200/csrc/state_update_stream.cu",),
+    "scan_bwd_130m": ("selective_state_space_40_b200/csrc/scan_bwd.cu",),
+    "ssd_2p7b": ("selective_state_space_40_b200/csrc/ssd_fwd.cu",),
+    "ssd_decode": ("selective_state_space_40_b200/csrc/ssd_update.cu",),
+}
+
+
+def csrc_digest(kernel=None):
+    """Hash of the sources of one recorded kernel (all of csrc/ when kernel is None)."""
+    if kernel is None:
+        paths = sorted(glob.glob(os.path.join(ROOT, "selective_state_space_40_b200", "csrc", "*")))
+    else:
+        paths = [os.path.join(ROOT, p) for p in sorted(KERNEL_SOURCES[kernel] + _SHARED_SOURCES)]
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "selective_state_space_40_b200", "csrc", "*"))):
+    for p in paths:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
@@ -109,14 +129,14 @@ def csrc_digest():
 
 def recorded_traffic(kernel):
     """DRAM bytes per launch from the committed ncu capture, if it was taken
-    on the current kernel sources (else None)."""
+    on the kernel's current sources (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f).get(kernel)
     except Exception:
         return None
-    if not rec or rec.get("csrc_sha") != csrc_digest():
+    if not rec or kernel not in KERNEL_SOURCES or rec.get("csrc_sha") != csrc_digest(kernel):
         return None
     return rec.get("dram_bytes_per_launch")
 

@@ -101,3 +101,18 @@ def test_reference_arm_other_ranks_exit_quietly():
 def test_warmup_floor():
     with pytest.raises(SystemExit):
         bench.main(["--warmup", "1"])
+
+
+def test_traffic_records_are_keyed_on_existing_kernel_sources():
+    # every DRAM-traffic record names a kernel whose source list exists, so a
+    # change to one kernel invalidates only that kernel's record
+    import json
+    for k, paths in bench.KERNEL_SOURCES.items():
+        for p in paths + bench._SHARED_SOURCES:
+            assert os.path.exists(os.path.join(bench.ROOT, p)), p
+        assert len(bench.csrc_digest(k)) == 16
+    with open(os.path.join(bench.ROOT, "profiles", "traffic.json")) as f:
+        recs = json.load(f)
+    assert set(recs) <= set(bench.KERNEL_SOURCES)
+    for rec in recs.values():
+        assert rec["dram_bytes_per_launch"] == rec["dram_bytes_read"] + rec["dram_bytes_write"]

@@ -312,3 +312,27 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(mb, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         mb.library()
+
+
+def _long_dims(batch=1, dim=2048, L=131072, N=16):
+    return _dims(batch=batch, dim=dim, dstate=N, seqlen=L, u_sb=dim * L, u_sd=L, delta_sb=dim * L, delta_sd=L,
+                 z_sb=dim * L, z_sd=L, y_sb=dim * L, y_sd=L, B_sb=N * L, B_sn=L, C_sb=N * L, C_sn=L)
+
+
+def test_sequence_split_workspace(lib):
+    # few channels and a long sequence: the sequence is split and the call
+    # needs a workspace for the segments' end states, Delta sums, initial and
+    # last states (16-byte aligned regions); no split otherwise
+    ws = mb.mamba_scan_workspace_size(_long_dims())
+    assert ws > 0 and ws % 16 == 0
+    dim, N = 2048, 16
+    S = None
+    for s in range(2, 257):   # the workspace is a whole-region formula in S
+        if ((s - 1) * dim * N + (s - 1) * dim + 2 * s * dim * N) * 4 == ws:
+            S = s
+    assert S is not None and 131072 % S == 0 and (131072 // S) % 64 == 0
+    assert mb.mamba_scan_workspace_size(_long_dims(L=4096)) == 0            # short: no split
+    assert mb.mamba_scan_workspace_size(_long_dims(batch=8, dim=1536)) == 0  # many channels: no split
+    # a split call without its workspace is refused before any launch
+    assert _scan(_long_dims(), ws=None, ws_bytes=0) == mb.MS_ERR_WORKSPACE
+    assert _scan(_long_dims(), ws=FAKE, ws_bytes=ws - 16) == mb.MS_ERR_WORKSPACE

@@ -4,11 +4,14 @@
 
 One step = one selective-scan forward (mamba_scan_fwd through the C ABI) over
 the 130M-class layer: batch 8, d_inner 1536, d_state 16, L 2048, bf16 inputs,
-fp32 y and last_state. Inputs are synthetic, seeded, resident in HBM; two
-copies of them are rotated so that every step reads inputs not touched by the
-previous step (254 MB per set, above the 126 MB L2). Rank 0 prints one JSON
-line. Under torchrun every rank runs its own layer (weak scaling, no
-collective on the data path); the device time is the max over ranks.
+fp32 y and last_state. Inputs are synthetic, seeded, resident in HBM; three
+copies of them (and two of y) are rotated so that every step reads inputs not
+touched by the two previous steps (254 MB per set, above the 126 MB L2). Rank
+0 prints one JSON line. Under torchrun every rank runs its own layer (weak
+scaling, no collective on the data path); the device time is the max over
+ranks. The same line carries legs for the other forward workloads (2.8B-class
+layer, long context), the decode step and the widened entry points, each with
+its bytes, time, roofline fraction and clocks.
 
 `--impl reference` times the fp64 CPU oracle on the host cores instead, on a
 bounded sample of the same workload per step.
@@ -240,6 +243,60 @@ def barrier(world):
         dist.barrier()
 
 
+# -------------------------------------------------------------- timing ----
+
+def time_launches(torch, stream, fn, steps, warmup, device_index):
+    """Mean per-launch time (ms) of fn(i) with CUDA events on the launching
+    stream, after `warmup` untimed launches; the NVML clock record of the
+    timed launches beside it."""
+    for i in range(warmup):
+        fn(i)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    torch.cuda.synchronize()
+    with ClockSampler(device_index, period=0.001) as clk:
+        for i in range(steps):
+            ev[i][0].record(stream)
+            fn(warmup + i)
+            ev[i][1].record(stream)
+        torch.cuda.synchronize()
+    return statistics.fmean(a.elapsed_time(b) for a, b in ev), clk.summary()
+
+
+def forward_leg(torch, mb, syn, w, stream, dev, local, world, peak, steps, nsets, traffic_key):
+    """One forward workload timed launch by launch over `nsets` rotating input
+    sets (each above the 126 MB L2), automatic plan, fp32 y and last_state."""
+    es = 2 if w.in_dtype == torch.bfloat16 else 4
+    host = syn.scan_inputs(w)
+    sets = [{k: v.to(dev) for k, v in host.items()} for _ in range(nsets)]
+    del host
+    y = torch.empty(w.batch, w.dim, w.seqlen, dtype=torch.float32, device=dev)
+    last = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
+    dims = mb.scan_dims_for(sets[0]["u"], sets[0]["delta"], sets[0]["B"], sets[0]["C"], sets[0]["z"], y)
+    wsb = mb.mamba_scan_workspace_size(dims)
+    ws = torch.empty(max(wsb, 16), dtype=torch.uint8, device=dev) if wsb else None
+
+    def run(i):
+        g = sets[i % nsets]
+        mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                    y=y, last_state=last, stream=stream, workspace=ws)
+
+    ms, clk = time_launches(torch, stream, run, steps, 3, local)
+    ms = max_over_ranks(ms, world, dev)
+    nb = scan_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4)
+    gbs = nb / (ms * 1e-3) / 1e9
+    rc, pl = mb.mamba_scan_choose_plan(dims)
+    plan = [pl.lanes_per_channel, pl.chunks_per_lane, pl.poly8] if rc == mb.MS_OK else None
+    out = {"workload": w.name, "ms": ms, "bytes": nb, "value": gbs, "unit": "GB/s",
+           "gct_per_s": w.channel_tokens / (ms * 1e-3) / 1e9, "frac": gbs / peak,
+           "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "traffic": recorded_traffic(traffic_key),
+           "plan": plan, "split_workspace_bytes": wsb,
+           "l2": f"{nsets} rotating input sets of {nb / 1e6:.0f} MB (> 126 MB L2)",
+           "timing": f"mean of {steps} per-launch event pairs", "clocks": clk}
+    del sets, y, last, ws
+    torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------- CPU baseline ----
 
 def oracle_sample_time(inp, n_batch_rows, nthreads):
@@ -339,15 +396,17 @@ def main(argv=None):
 
     es = 2 if w.in_dtype == torch.bfloat16 else 4
     host = syn.scan_inputs(w)
-    sets = [{k: v.to(dev) for k, v in host.items()} for _ in range(2)]
+    NSETS = 3
+    sets = [{k: v.to(dev) for k, v in host.items()} for _ in range(NSETS)]
     y = torch.empty(w.batch, w.dim, w.seqlen, dtype=torch.float32, device=dev)
+    y_alt = torch.empty_like(y)
     last = torch.empty(w.batch, w.dim, w.dstate, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def step(i):
-        g = sets[i & 1]
+        g = sets[i % NSETS]
         mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                    True, y=y, last_state=last, stream=stream)
+                    True, y=y if i & 1 == 0 else y_alt, last_state=last, stream=stream)
 
     for i in range(args.warmup):
         step(i)
@@ -359,7 +418,7 @@ def main(argv=None):
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clk:
+    with ClockSampler(local, period=0.001) as clk:
         t0.record(stream)
         for i in range(args.steps):
             ev[i][0].record(stream)
@@ -401,7 +460,7 @@ def main(argv=None):
     def e2e_run(n):
         for i in range(n):
             k = i & 1
-            d_in = sets[k]
+            d_in = sets[k]  # two of the device sets serve as the e2e buffers
             if i >= 2:
                 s_in.wait_event(comp_done[k])       # the scan of step i-2 has read these inputs
             with torch.cuda.stream(s_in):
@@ -459,6 +518,13 @@ def main(argv=None):
     dbytes = decode_bytes(dw.batch, dw.dim, dw.dstate, 2, 4)
     dec_gbs = dbytes / (dec_ms * 1e-3) / 1e9
     del states
+
+    # ---- the other forward workloads: the 2.8B-class layer (two rotating
+    # 842 MB input sets) and the long-context fp32 layer (4.3 GB per launch,
+    # sequence split in segments; one input set is far above L2)
+    del sets[2:]
+    fwd_2p8b = forward_leg(torch, mb, syn, syn.M2P8, stream, dev, local, world, peak, 30, 2, "scan_fwd_2p8b")
+    fwd_long = forward_leg(torch, mb, syn, syn.LONG, stream, dev, local, world, peak, 8, 1, "scan_fwd_long")
 
     # ---- scan with the causal conv front-end (width 4) on the same layer: u is
     # formed from the conv input x in the load stage, so the bytes are the
@@ -590,16 +656,19 @@ def main(argv=None):
             "config": {"workload": w.name, "batch": w.batch, "dim": w.dim, "dstate": w.dstate,
                        "seqlen": w.seqlen, "in_dtype": "bf16", "out_dtype": "f32",
                        "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": "two rotating input sets of 254 MB each (> 126 MB L2), no flush"},
+                       "l2": "three rotating input sets of 254 MB each and two y buffers (> 126 MB L2), no flush"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
                          "kernel": "scan_fwd_kernel", "bytes_per_launch": nbytes,
                          "kernel_ms": kernel_ms, "nominal_peak": NOMINAL_HBM_GBS,
-                         "frac_of_nominal": achieved / NOMINAL_HBM_GBS},
+                         "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
+                         "traffic_over_bytes": None if traffic is None else traffic / nbytes},
             "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": e2e_steps,
                     "pipelining": "upload, scan and download of consecutive steps overlap on three streams"},
+            "scan_2p8b": fwd_2p8b,
+            "scan_long": fwd_long,
             "decode_step": {"workload": dw.name, "value": dec_gbs, "unit": "GB/s",
                             "ms": dec_ms, "bytes": dbytes, "frac": dec_gbs / peak,
                             "frac_of_nominal": dec_gbs / NOMINAL_HBM_GBS,

@@ -21,9 +21,12 @@
  * steps open and this library fixes that reading.
  *
  * Conventions common to every entry point:
- *  - All array pointers are device pointers owned by the caller. The library
- *    keeps no global mutable state; calls are re-entrant and asynchronous on
- *    the given stream (NULL = the legacy default stream).
+ *  - All array pointers are device pointers owned by the caller. Calls are
+ *    re-entrant and asynchronous on the given stream (NULL = the legacy
+ *    default stream). The library's only process-wide state is (a) per-device
+ *    caches of kernel attributes and symbol addresses, keyed on the CUDA
+ *    context and set up under a lock, and (b) the fixed device scratch of
+ *    mamba_scan_bwd_noalloc (below), which calls of that entry point share.
  *  - Strides are in ELEMENTS, and the innermost stride is always 1.
  *  - Arguments are checked on the host before anything touches the GPU; a
  *    failed check returns its MS_ERR_* code and launches nothing.
@@ -62,7 +65,8 @@ enum {
     MS_ERR_CUDA = 7,      /* a CUDA runtime call failed (no device, launch error)*/
     MS_ERR_TIMEOUT = 8,   /* device: a bounded wait gave up                      */
     MS_ERR_DEVICE = 9,    /* device is not compute capability 10.0 (B200)        */
-    MS_ERR_SCRATCH = 10   /* needs more scratch than the library's fixed buffer  */
+    MS_ERR_SCRATCH = 10,  /* needs more scratch than the library's fixed buffer  */
+    MS_ERR_BOUNDS = 11    /* device, debug build: an index failed a bounds check */
 };
 
 /* Maximum d_state the kernels support (Mamba-1 layers use 16). */
@@ -137,15 +141,32 @@ int mamba_scan_fwd(const void *u, const void *delta, const float *A, const void 
  *                      8 * lanes_per_channel * chunks_per_lane tokens.
  *   poly8              0, 2, 4 or 8: eighths of the exponentials computed by
  *                      a polynomial on the FMA pipe instead of the MUFU unit.
+ *   engine             MS_ENGINE_REGISTER: the kernel that prefetches each
+ *                      lane's token chunks into registers and stages B/C in
+ *                      shared memory (any sizes and strides, every option).
+ *                      MS_ENGINE_TMEM: token tiles streamed by the TMA engine
+ *                      into a shared-memory ring and B/C broadcast to the
+ *                      lanes through tensor memory by one tcgen05 product per
+ *                      32-token tile (lanes_per_channel 4, chunks_per_lane 1;
+ *                      needs dstate 16, seqlen a multiple of 8, 16-byte
+ *                      aligned rows and pointers; not for the conv front-end
+ *                      or the training forward). Finite B and C are assumed:
+ *                      a non-finite value also spoils the other states of its
+ *                      token in this engine.
+ * mamba_scan_fwd uses MS_ENGINE_TMEM wherever it applies.
  */
+enum { MS_ENGINE_REGISTER = 0, MS_ENGINE_TMEM = 1 };
+
 typedef struct {
     int32_t lanes_per_channel;
     int32_t chunks_per_lane;
     int32_t poly8;
+    int32_t engine;
 } ms_scan_plan;
 
 /* mamba_scan_fwd with an explicit plan (NULL = choose automatically).
-   Returns MS_ERR_SHAPE for a plan value outside the lists above. */
+   Returns MS_ERR_SHAPE for a plan value outside the lists above, or for
+   MS_ENGINE_TMEM where that engine does not apply. */
 int mamba_scan_fwd_plan(const void *u, const void *delta, const float *A, const void *B,
                         const void *C, const float *D, const void *z, const float *delta_bias,
                         int softplus_flag, const float *initial_state, void *y, float *last_state,
@@ -246,21 +267,31 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
                    void *workspace, size_t workspace_bytes, int *dev_status, ms_stream_t stream);
 
 /*
- * mamba_scan_bwd without saved states and without any allocation or caller
- * workspace. The pages have no counterpart: this is a packaging of
- * mamba_scan_bwd for callers that may not allocate (e.g. inside a captured
- * CUDA graph). The recomputed saved states go to a fixed scratch buffer of
- * MS_BWD_NOALLOC_MAX_BYTES compiled into the library (one per device, set up
- * by the first call on that device); nothing is allocated, ever.
+ * mamba_scan_bwd without saved states, without a caller workspace and without
+ * any allocation. The pages have no counterpart: this is mamba_scan_bwd
+ * packaged for callers that must not allocate device memory, such as a
+ * serving or training runtime whose memory pool claimed the device's free
+ * memory at start-up (a cudaMalloc there fails or defeats the pool's
+ * accounting), or a latency-critical path where cudaMalloc/cudaFree may
+ * synchronize the device and stall other streams. The recomputed saved
+ * states go to a fixed scratch array of MS_BWD_NOALLOC_MAX_BYTES compiled
+ * into the library as a file-scope __device__ array: every GPU that loads the
+ * library holds it until the process exits.
+ *  - Set-up: the first call on a device (and the first call after that
+ *    device's context was replaced, e.g. by a device reset) looks up the
+ *    array's device address with that device current, which may load the
+ *    library's module. Make the first call on each device before any stream
+ *    capture on it.
  *  - Calls needing more than MS_BWD_NOALLOC_MAX_BYTES of saved states
- *    (mamba_scan_bwd_workspace_size()) return MS_ERR_SCRATCH and do nothing.
- *  - The buffer is shared by all calls on a device: two calls that run at the
- *    same time on one device (different streams or host threads without
- *    ordering) overwrite each other's scratch. Order them (one stream, or
- *    events); calls on one stream are safe.
- *  - The first call on a device looks the buffer up and may load the module:
- *    make it before any stream capture on that device; later calls only
- *    launch kernels and memsets and can be captured.
+ *    (mamba_scan_bwd_workspace_size()) return MS_ERR_SCRATCH before any
+ *    GPU work.
+ *  - The array is shared by all calls on a device and keeps the last call's
+ *    contents (every call rewrites what it reads; the accumulated gradients
+ *    are zeroed on the stream as in mamba_scan_bwd). Two calls that overlap
+ *    on one device (different streams, or host threads without ordering)
+ *    race on it; calls on one stream, or ordered by events, are safe.
+ *  - Nothing is allocated: no cudaMalloc, cudaFree or allocating library
+ *    routine, on any call.
  * Arguments and results are those of mamba_scan_bwd with ckpt = NULL.
  */
 #define MS_BWD_NOALLOC_MAX_BYTES ((size_t)96 << 20)
@@ -394,6 +425,23 @@ int mamba_state_update(float *state, const void *x, const void *delta, const flo
  * MS_ERR_CUDA (the timeout itself is reported through *dev_status).
  */
 int mamba_debug_bounded_wait(uint32_t rounds, int *dev_status, ms_stream_t stream);
+
+/*
+ * Debug build check (the pages have no counterpart). libmambascan_debug.so is
+ * this library compiled with MS_DEBUG: its kernels test their shared-memory,
+ * tensor-memory and global indexes against the buffers they address, and a
+ * failing test ORs MS_ERR_BOUNDS into *dev_status and skips the access
+ * instead of performing it (the stand-in for a memory checker on a pool where
+ * none can run). This hook launches one thread that writes element `index` of
+ * a 16-int device array through such a check: index in [0, 16) writes, any
+ * other index is recorded and skipped. In the product library (not built with
+ * MS_DEBUG) it launches nothing and returns MS_ERR_SHAPE.
+ * Returns MS_ERR_NULL without dev_status, else MS_OK or MS_ERR_CUDA.
+ */
+int mamba_debug_bounds_probe(int32_t index, int *dev_status, ms_stream_t stream);
+
+/* 1 when this library is the MS_DEBUG build, else 0. */
+int mamba_debug_build(void);
 
 /* Static English text for a status code (never NULL). */
 const char *mamba_status_string(int code);

@@ -8,6 +8,7 @@ library. A missing library raises: there is no CPU fallback.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 from typing import Optional, Tuple
@@ -18,9 +19,10 @@ LIB_PATH = os.path.join(_PKG, "libmambascan.so")
 MS_F32, MS_BF16 = 0, 1
 MS_OK, MS_ERR_NULL, MS_ERR_DTYPE, MS_ERR_SHAPE, MS_ERR_STRIDE = 0, 1, 2, 3, 4
 MS_ERR_ALIGN, MS_ERR_WORKSPACE, MS_ERR_CUDA, MS_ERR_TIMEOUT, MS_ERR_DEVICE = 5, 6, 7, 8, 9
-MS_ERR_SCRATCH = 10
+MS_ERR_SCRATCH, MS_ERR_BOUNDS = 10, 11
 MS_BWD_NOALLOC_MAX_BYTES = 96 << 20
 MS_MAX_DSTATE = 16
+MS_ENGINE_REGISTER, MS_ENGINE_TMEM = 0, 1
 
 
 class ScanDims(ctypes.Structure):
@@ -38,7 +40,7 @@ class UpdateDims(ctypes.Structure):
 
 class ScanPlan(ctypes.Structure):
     _fields_ = [("lanes_per_channel", ctypes.c_int32), ("chunks_per_lane", ctypes.c_int32),
-                ("poly8", ctypes.c_int32)]
+                ("poly8", ctypes.c_int32), ("engine", ctypes.c_int32)]
 
 
 class ConvDims(ctypes.Structure):
@@ -66,6 +68,7 @@ class MambaScanError(RuntimeError):
 
 
 _lib = None
+_loaded = {}
 _vp = ctypes.c_void_p
 
 
@@ -73,10 +76,29 @@ def library() -> ctypes.CDLL:
     """Load libmambascan.so (raises if it has not been built)."""
     global _lib
     if _lib is None:
-        if not os.path.exists(LIB_PATH):
+        _lib = _load(LIB_PATH)
+    return _lib
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route every call of this module to another build of the library (the
+    MS_DEBUG build, in the tests) inside the `with` block."""
+    global _lib
+    saved = library()
+    _lib = _load(path)
+    try:
+        yield _lib
+    finally:
+        _lib = saved
+
+
+def _load(path: str) -> ctypes.CDLL:
+    if path not in _loaded:
+        if not os.path.exists(path):
             raise RuntimeError(
-                f"{LIB_PATH} is missing: build it with `python -m selective_state_space_40_b200.build`")
-        lib = ctypes.CDLL(LIB_PATH)
+                f"{path} is missing: build it with `python -m selective_state_space_40_b200.build`")
+        lib = ctypes.CDLL(path)
         lib.mamba_scan_workspace_size.argtypes = [ctypes.POINTER(ScanDims)]
         lib.mamba_scan_workspace_size.restype = ctypes.c_size_t
         scan_args = [_vp] * 8 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(ScanDims), _vp,
@@ -122,8 +144,12 @@ def library() -> ctypes.CDLL:
         lib.mamba_debug_bounded_wait.restype = ctypes.c_int
         lib.mamba_device_check.argtypes = []
         lib.mamba_device_check.restype = ctypes.c_int
-        _lib = lib
-    return _lib
+        lib.mamba_debug_bounds_probe.argtypes = [ctypes.c_int32, _vp, _vp]
+        lib.mamba_debug_bounds_probe.restype = ctypes.c_int
+        lib.mamba_debug_build.argtypes = []
+        lib.mamba_debug_build.restype = ctypes.c_int
+        _loaded[path] = lib
+    return _loaded[path]
 
 
 # ------------------------------------------------------------ raw C entry ----
@@ -134,6 +160,14 @@ def mamba_status_string(code: int) -> str:
 
 def mamba_device_check() -> int:
     return library().mamba_device_check()
+
+
+def mamba_debug_build() -> int:
+    return library().mamba_debug_build()
+
+
+def mamba_debug_bounds_probe(index: int, dev_status, stream) -> int:
+    return library().mamba_debug_bounds_probe(int(index), dev_status, stream)
 
 
 def mamba_debug_bounded_wait(rounds: int, dev_status, stream) -> int:

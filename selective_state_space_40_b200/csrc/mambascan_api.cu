@@ -43,6 +43,53 @@ bool vec_ok(const void *p, int64_t sb, int64_t sd, int es) {
 
 }  // namespace
 
+namespace ms {
+
+namespace {
+using PfnCtxGetCurrent = int (*)(void **);
+using PfnCtxGetId = int (*)(void *, unsigned long long *);
+PfnCtxGetCurrent g_ctx_get_current = nullptr;
+PfnCtxGetId g_ctx_get_id = nullptr;
+std::once_flag g_ctx_fns_once;
+}  // namespace
+
+uint64_t current_context_id() {
+    std::call_once(g_ctx_fns_once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get_current = reinterpret_cast<PfnCtxGetCurrent>(f);
+        f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &f, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_ctx_get_id = reinterpret_cast<PfnCtxGetId>(f);
+        cudaGetLastError();
+    });
+    if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+    void *ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != 0 || ctx == nullptr) return 0;
+    unsigned long long id = 0;
+    if (g_ctx_get_id(ctx, &id) != 0) return 0;
+    return (uint64_t)id + 1;
+}
+
+cudaError_t SmemOptIn::ensure(const void *func, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t ctx = current_context_id();
+    if (ctx != 0 && dev >= 0 && dev < 64 && ctx_[dev].load(std::memory_order_acquire) == ctx) return cudaSuccess;
+    e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    // the attribute call has made the device's primary context current
+    const uint64_t now = current_context_id();
+    if (now != 0 && dev >= 0 && dev < 64) ctx_[dev].store(now, std::memory_order_release);
+    return cudaSuccess;
+}
+
+}  // namespace ms
+
 extern "C" {
 
 const char *mamba_status_string(int code) {
@@ -58,6 +105,7 @@ const char *mamba_status_string(int code) {
         case MS_ERR_TIMEOUT: return "device wait timed out";
         case MS_ERR_DEVICE: return "device is not compute capability 10.0";
         case MS_ERR_SCRATCH: return "needs more scratch than the library's fixed buffer holds";
+        case MS_ERR_BOUNDS: return "a device bounds check failed (debug build)";
         default: return "unknown status code";
     }
 }
@@ -71,6 +119,30 @@ int mamba_debug_bounded_wait(uint32_t rounds, int *dev_status, ms_stream_t strea
         return MS_ERR_CUDA;
     }
     return MS_OK;
+}
+
+int mamba_debug_build(void) {
+#ifdef MS_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+int mamba_debug_bounds_probe(int32_t index, int *dev_status, ms_stream_t stream) {
+    if (!dev_status) return MS_ERR_NULL;
+    if (!aligned(dev_status, 4)) return MS_ERR_ALIGN;
+#ifdef MS_DEBUG
+    if (ms::launch_bounds_probe(index, dev_status, (cudaStream_t)stream) != cudaSuccess) {
+        cudaGetLastError();
+        return MS_ERR_CUDA;
+    }
+    return MS_OK;
+#else
+    (void)index;
+    (void)stream;
+    return MS_ERR_SHAPE;
+#endif
 }
 
 int mamba_device_check(void) {
@@ -173,18 +245,48 @@ size_t mamba_scan_workspace_size(const ms_scan_dims *dims) {
 }
 
 static bool plan_valid(const ms_scan_plan *p) {
-    const int g = p->lanes_per_channel, c = p->chunks_per_lane, q = p->poly8;
-    return (g == 1 || g == 2 || g == 4 || g == 8) && (c == 1 || (c == 2 && g != 8)) &&
+    const int g = p->lanes_per_channel, c = p->chunks_per_lane, q = p->poly8, e = p->engine;
+    if (e == MS_ENGINE_TMEM) return g == 4 && c == 1 && (q == 0 || q == 2 || q == 4 || q == 8);
+    return e == MS_ENGINE_REGISTER && (g == 1 || g == 2 || g == 4 || g == 8) && (c == 1 || (c == 2 && g != 8)) &&
            (q == 0 || q == 2 || q == 4 || q == 8);
 }
 
-static ms::ScanPlan auto_plan(const ms_scan_dims *dims) {
+// Exponentials on the FMA-pipe polynomial in the tensor-memory kernel, in
+// eighths: bf16 inputs balance the MUFU and FMA pipes; fp32 inputs take every
+// exponential from the polynomial (unbiased near 1, see ms_device.cuh).
+constexpr int kTmemPoly8Bf16 = 0;
+
+// The plan a call without an explicit plan runs: the tensor-memory kernel
+// where it applies (sizes, strides, alignment and outputs), else the
+// register-prefetch kernel with its own heuristic.
+static ms::ScanPlan auto_plan_args(const ms::ScanArgs &a, bool in_bf16, bool out_bf16, bool check_pointers) {
+    ms::ScanPlan pl = ms::plan_scan(a, in_bf16, num_sms_current());
+    const int eo = out_bf16 ? 2 : 4;
+    if (check_pointers ? ms::scan_tmem_applies(a, in_bf16, eo) : ms::scan_tmem_shape_ok(a, in_bf16, eo)) {
+        pl.engine = MS_ENGINE_TMEM;
+        pl.lanes_per_channel = 4;
+        pl.chunks_per_lane = 1;
+        pl.poly8 = in_bf16 ? kTmemPoly8Bf16 : 8;
+    }
+    return pl;
+}
+
+static ms::ScanArgs dims_args(const ms_scan_dims *dims) {
     ms::ScanArgs a{};
     a.batch = dims->batch;
     a.dim = dims->dim;
     a.L = dims->seqlen;
     a.N = (int)dims->dstate;
-    return ms::plan_scan(a, dims->in_dtype == MS_BF16, num_sms_current());
+    a.u_sb = dims->u_sb; a.u_sd = dims->u_sd;
+    a.dl_sb = dims->delta_sb; a.dl_sd = dims->delta_sd;
+    a.z_sb = dims->z_sb; a.z_sd = dims->z_sd;
+    a.y_sb = dims->y_sb; a.y_sd = dims->y_sd;
+    a.B_sb = dims->B_sb; a.B_sn = dims->B_sn; a.C_sb = dims->C_sb; a.C_sn = dims->C_sn;
+    return a;
+}
+
+static ms::ScanPlan auto_plan(const ms_scan_dims *dims) {
+    return auto_plan_args(dims_args(dims), dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, false);
 }
 
 int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan) {
@@ -196,6 +298,7 @@ int mamba_scan_choose_plan(const ms_scan_dims *dims, ms_scan_plan *plan) {
     plan->lanes_per_channel = p.lanes_per_channel;
     plan->chunks_per_lane = p.chunks_per_lane;
     plan->poly8 = p.poly8;
+    plan->engine = p.engine;
     return MS_OK;
 }
 
@@ -267,11 +370,13 @@ static int scan_common(const void *u, const void *delta, const float *A, const v
     }
 
     const bool in_bf16 = dims->in_dtype == MS_BF16, out_bf16 = dims->out_dtype == MS_BF16;
-    ms::ScanPlan pl = auto_plan(dims);
+    ms::ScanPlan pl = auto_plan_args(a, in_bf16, out_bf16, true);
     if (plan) {
         pl.lanes_per_channel = plan->lanes_per_channel;
         pl.chunks_per_lane = plan->chunks_per_lane;
         pl.poly8 = plan->poly8;
+        pl.engine = plan->engine;
+        if (pl.engine == MS_ENGINE_TMEM && !ms::scan_tmem_applies(a, in_bf16, eo)) return MS_ERR_SHAPE;
     }
     cudaError_t e = ms::launch_scan_fwd(a, pl, in_bf16, out_bf16, (cudaStream_t)stream);
     if (e != cudaSuccess) {
@@ -321,7 +426,7 @@ static int scan_split(const void *u, const void *delta, const float *A, const vo
             a.softplus = softplus_flag ? 1 : 0;
             a.vec_in = vec_ok(a.u, Ls, a.u_sd, ei) && vec_ok(a.delta, Ls, a.dl_sd, ei) && vec_ok(a.z, Ls, a.z_sd, ei);
             a.vec_out = a.y == nullptr || vec_ok(a.y, Ls, a.y_sd, eo);
-            const ms::ScanPlan pl = ms::plan_scan(a, dims->in_dtype == MS_BF16, num_sms_current());
+            const ms::ScanPlan pl = auto_plan_args(a, dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, true);
             return ms::launch_scan_fwd(a, pl, dims->in_dtype == MS_BF16, dims->out_dtype == MS_BF16, st) ==
                            cudaSuccess
                        ? MS_OK
@@ -378,7 +483,8 @@ int mamba_conv_scan_fwd(const void *x, const float *conv_w, const float *conv_b,
                         const float *delta_bias, int softplus_flag, const float *initial_state,
                         void *y, float *last_state, const ms_scan_dims *dims,
                         const ms_scan_plan *plan, int *dev_status, ms_stream_t stream) {
-    if (plan && (!plan_valid(plan) || plan->chunks_per_lane != 1 || (plan->poly8 != 0 && plan->poly8 != 8)))
+    if (plan && (!plan_valid(plan) || plan->engine != MS_ENGINE_REGISTER || plan->chunks_per_lane != 1 ||
+                 (plan->poly8 != 0 && plan->poly8 != 8)))
         return MS_ERR_SHAPE;
     int rc = check_scan(x, delta, A, B, C, D, z, delta_bias, initial_state, y, last_state, dims);
     if (rc != MS_OK) return rc;
@@ -480,24 +586,29 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
     return MS_OK;
 }
 
-// Device address of g_bwd_scratch on the current device, looked up once per
-// device (the lookup may load the module, so it must not happen in capture).
+// Device address of g_bwd_scratch on the current device: looked up with the
+// device current on the first call, and again whenever the device's context
+// has changed since (after a device reset the module is loaded anew and the
+// array may sit elsewhere), or when the context's id cannot be read.
 static int bwd_scratch(void **p) {
     static std::mutex mtx;
     static void *addr[64] = {};
+    static uint64_t ctx_of[64] = {};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return MS_ERR_CUDA;
     }
     std::lock_guard<std::mutex> lock(mtx);
-    if (addr[dev] == nullptr) {
+    const uint64_t ctx = ms::current_context_id();
+    if (addr[dev] == nullptr || ctx == 0 || ctx != ctx_of[dev]) {
         void *a = nullptr;
         if (cudaGetSymbolAddress(&a, g_bwd_scratch) != cudaSuccess || a == nullptr) {
             cudaGetLastError();
             return MS_ERR_CUDA;
         }
         addr[dev] = a;
+        ctx_of[dev] = ms::current_context_id();  // the lookup made the primary context current
     }
     *p = addr[dev];
     return MS_OK;

@@ -9,6 +9,23 @@
 
 namespace ms {
 
+// ------------------------------------------------------ debug bounds checks --
+// In the debug build (-DMS_DEBUG, libmambascan_debug.so) MS_CHECK(status, ok)
+// evaluates `ok`; when it is false it ORs MS_ERR_BOUNDS (11) into the
+// caller's device status word (when given) and yields false, and the guarded
+// access is skipped: an index out of range is recorded, never performed. In
+// the product build the check compiles to `true` (no cost).
+constexpr int kErrBounds = 11;
+__device__ __forceinline__ bool debug_check(int *status, bool ok) {
+    if (!ok && status != nullptr) atomicOr(status, kErrBounds);
+    return ok;
+}
+#ifdef MS_DEBUG
+#define MS_CHECK(status, cond) ::ms::debug_check((status), (cond))
+#else
+#define MS_CHECK(status, cond) true
+#endif
+
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 

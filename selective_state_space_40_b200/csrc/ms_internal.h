@@ -109,6 +109,7 @@ struct ScanPlan {
     int lanes_per_channel;  // G: lanes sharing one channel (1, 2, 4, 8), 16/G states each
     int chunks_per_lane;    // CH: 8-token chunks per lane per tile (1, 2; 1 when G = 8)
     int poly8;              // eighths of the exponentials evaluated on the FMA pipe
+    int engine;             // 0: register-prefetch kernel; 1: TMA + tensor-memory kernel (G = 4)
 };
 
 struct UpdateArgs {
@@ -139,10 +140,40 @@ cudaError_t launch_state_update_stream(const UpdateArgs &a, bool in_bf16, bool o
 // One CTA waits `rounds` bounded tries on a barrier nothing completes, then
 // ORs MS_ERR_TIMEOUT into *status (tests the device timeout path).
 cudaError_t launch_bounded_wait_probe(int *status, uint32_t rounds, cudaStream_t stream);
+#ifdef MS_DEBUG
+// One thread writes element `index` of a 16-int device array through
+// MS_CHECK (debug build only).
+cudaError_t launch_bounds_probe(int index, int *status, cudaStream_t stream);
+#endif
 
 cudaError_t launch_scan_bwd(const BwdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
 
-// Plan for a call (host heuristic from sizes and dtypes).
+// Plan for a call (host heuristic from sizes, strides and dtypes).
 ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms);
+
+// The TMA + tensor-memory scan kernel (scan_fwd_tmem.cu): sizes and strides
+// it takes (d_state 16, L a multiple of 8, 16-byte rows), and the full check
+// including pointer alignment and the outputs requested.
+bool scan_tmem_shape_ok(const ScanArgs &a, bool in_bf16, int out_bytes);
+bool scan_tmem_applies(const ScanArgs &a, bool in_bf16, int out_bytes);
+cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16, int num_sms,
+                                 cudaStream_t stream);
+
+// Unique id of the calling thread's current CUDA context, never 0; 0 when it
+// cannot be read. A device reset replaces the primary context, so caches of
+// per-context facts (kernel attributes, device addresses of symbols) are
+// keyed on this id and redone when it changes.
+uint64_t current_context_id();
+
+// Raises a kernel's dynamic shared memory limit to `bytes` once per device
+// and context (cudaFuncSetAttribute is repeated when the context changed or
+// its id cannot be read).
+class SmemOptIn {
+  public:
+    cudaError_t ensure(const void *func, int bytes);
+
+  private:
+    std::atomic<uint64_t> ctx_[64] = {};  // per device: context the attribute was set in
+};
 
 }  // namespace ms

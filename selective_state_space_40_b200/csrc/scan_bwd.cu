@@ -513,16 +513,9 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
 template <typename TIn, typename TOut>
 cudaError_t launch_bwd(const BwdArgs &a, unsigned grid, cudaStream_t stream) {
     // more than 48 KB of shared memory: opt in once per device
-    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(scan_bwd_kernel<TIn, TOut>), (int)sizeof(BwdSmem));
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(scan_bwd_kernel<TIn, TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(BwdSmem));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev].store(true, std::memory_order_release);
-    }
     scan_bwd_kernel<TIn, TOut><<<grid, kBThreads, sizeof(BwdSmem), stream>>>(a);
     return cudaGetLastError();
 }

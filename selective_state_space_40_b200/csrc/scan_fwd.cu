@@ -447,7 +447,7 @@ scan_fwd_kernel(const ScanArgs a) {
 #pragma unroll
         for (int r = 0; r < kBCPer; ++r) {
             const int rr = threadIdx.x + r * kThreads;
-            if (rr < 2 * TT) {
+            if (rr < 2 * TT && MS_CHECK(a.status, buf < 2 && rr % TT < TT)) {
                 float4 *row = reinterpret_cast<float4 *>(&sBC[buf][rr % TT][rr >= TT ? 16 : 0]);
 #pragma unroll
                 for (int q = 0; q < 4; ++q)
@@ -530,6 +530,7 @@ scan_fwd_kernel(const ScanArgs a) {
 #pragma unroll
             for (int i = 0; i < CH; ++i) {
                 const int off = 8 * (g * CH + i);
+                if (!MS_CHECK(a.status, off + 8 <= Gm::kRow && c < ROWS && warp < kNW)) continue;
                 const float4 y0 = *reinterpret_cast<const float4 *>(&sY[warp][c][off]);
                 const float4 y1 = *reinterpret_cast<const float4 *>(&sY[warp][c][off + 4]);
                 const float ys[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
@@ -573,16 +574,9 @@ cudaError_t launch_one(const ScanArgs &a, cudaStream_t stream) {
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
     // Opt in to more than 48 KB of dynamic shared memory once per device and
     // instantiation (setting it twice from two host threads is harmless).
-    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT>), Sm::kTotal);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev].store(true, std::memory_order_release);
-    }
     scan_fwd_kernel<TIn, TOut, G, CH, POLY8, CONV, CKPT><<<(unsigned)blocks, kThreads, Sm::kTotal, stream>>>(a);
     return cudaGetLastError();
 }
@@ -649,6 +643,12 @@ cudaError_t launch_types_ckpt(const ScanArgs &a, const ScanPlan &pl, cudaStream_
 
 cudaError_t launch_scan_fwd(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16,
                             cudaStream_t stream) {
+    if (plan.engine == 1) {
+        if (!scan_tmem_applies(a, in_bf16, out_bf16 ? 2 : 4)) return cudaErrorInvalidValue;
+        int dev = 0, sms = 148;
+        if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        return launch_scan_fwd_tmem(a, plan, in_bf16, out_bf16, sms > 0 ? sms : 148, stream);
+    }
     if (a.ckpt != nullptr || a.dsum != nullptr) {
         if (plan.chunks_per_lane != 1 || (plan.poly8 != 0 && plan.poly8 != 8)) return cudaErrorInvalidValue;
         if (in_bf16) {
@@ -710,6 +710,7 @@ ScanPlan plan_scan(const ScanArgs &a, bool in_bf16, int num_sms) {
     pl.lanes_per_channel = (channels * 4 / 32 >= want_warps) ? 4 : 8;
     pl.chunks_per_lane = 1;
     pl.poly8 = in_bf16 ? 0 : 8;
+    pl.engine = 0;
     return pl;
 }
 

@@ -196,16 +196,9 @@ __global__ void __launch_bounds__(kCbThreads) ssd_chunk_cb_kernel(const SsdCbArg
 bool ssd_cb_shape_supported(int64_t dstate) { return dstate == kK; }
 
 cudaError_t launch_ssd_chunk_cb(const SsdCbArgs &a, cudaStream_t stream) {
-    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_chunk_cb_kernel), (int)sizeof(CbSmem));
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(ssd_chunk_cb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(CbSmem));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev].store(true, std::memory_order_release);
-    }
     const int64_t tiles = (a.L + kTileTok - 1) / kTileTok;
     const int64_t blocks = a.batch * a.G * tiles;
     if (blocks <= 0) return cudaSuccess;

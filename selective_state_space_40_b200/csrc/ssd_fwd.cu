@@ -397,16 +397,9 @@ __global__ void __launch_bounds__(kST, 3) ssd_fwd_kernel(const SsdArgs a) {
 
 template <typename TOut>
 cudaError_t launch_ssd_t(const SsdArgs &a, cudaStream_t stream) {
-    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_fwd_kernel<TOut>), (int)sizeof(SsdSmem));
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(ssd_fwd_kernel<TOut>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)sizeof(SsdSmem));
-        if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev].store(true, std::memory_order_release);
-    }
     const int64_t blocks = a.batch * a.H;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;

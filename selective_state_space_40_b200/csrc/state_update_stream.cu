@@ -139,6 +139,13 @@ state_update_stream_kernel(const UpdateArgs a) {
         for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
     }
+    // Back-to-back steps: this grid may have been launched while the previous
+    // kernel on the stream still runs (programmatic dependent launch). Let the
+    // next step's grid get scheduled now, and wait here until everything the
+    // previous kernel wrote (the state) is complete and visible. Without that
+    // launch attribute both instructions do nothing.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
     // Prologue: the first kStages - 1 tiles of this CTA.
     if (threadIdx.x == 0) {
@@ -181,6 +188,7 @@ state_update_stream_kernel(const UpdateArgs a) {
         for (int half = 0; half < kTC * 4 / kThreads; ++half) {
             const int cl = (threadIdx.x >> 2) + half * (kThreads / 4);  // channel within the tile
             const int64_t d = d0 + cl;
+            if (!MS_CHECK(a.status, cl < kTC && d < a.dim)) continue;
             float4 hv = *reinterpret_cast<const float4 *>(sstate + cl * 16 + n0);
             float h[4] = {hv.x, hv.y, hv.z, hv.w};
             const float4 Av = __ldg(reinterpret_cast<const float4 *>(a.A + d * 16 + n0));
@@ -237,17 +245,12 @@ state_update_stream_kernel(const UpdateArgs a) {
 template <typename TIn, typename TOut>
 cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
     using Sm = StreamSmem<TIn, TOut>;
-    static std::atomic<bool> opted[64];  // per device: attribute set (zero-initialised)
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(state_update_stream_kernel<TIn, TOut>), Sm::kTotal);
     if (e != cudaSuccess) return e;
-    if (dev >= 64 || !opted[dev].load(std::memory_order_acquire)) {
-        e = cudaFuncSetAttribute(state_update_stream_kernel<TIn, TOut>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, Sm::kTotal);
-        if (e != cudaSuccess) return e;
-        if (dev < 64) opted[dev].store(true, std::memory_order_release);
-    }
-    int sms = 148, per_sm = 1;
+    int dev = 0, sms = 148, per_sm = 1;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, state_update_stream_kernel<TIn, TOut>, kThreads,
                                                   Sm::kTotal);
@@ -255,8 +258,20 @@ cudaError_t launch_t(const UpdateArgs &a, cudaStream_t stream) {
     const int64_t ntiles = a.batch * (a.dim / kTC);
     const int64_t grid = ntiles < (int64_t)sms * per_sm ? ntiles : (int64_t)sms * per_sm;
     if (grid <= 0) return cudaSuccess;
-    state_update_stream_kernel<TIn, TOut><<<(unsigned)grid, kThreads, Sm::kTotal, stream>>>(a);
-    return cudaGetLastError();
+    // programmatic dependent launch: the grid is scheduled while the previous
+    // kernel on the stream drains; the kernel waits (griddepcontrol.wait)
+    // before it reads any memory
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = Sm::kTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, state_update_stream_kernel<TIn, TOut>, a);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -278,6 +293,20 @@ __global__ void bounded_wait_probe_kernel(int *status, uint32_t rounds) {
 }
 
 }  // namespace
+
+#ifdef MS_DEBUG
+namespace {
+__device__ int g_bounds_probe[16];
+__global__ void bounds_probe_kernel(int index, int *status) {
+    if (MS_CHECK(status, index >= 0 && index < 16)) g_bounds_probe[index] = index + 1;
+}
+}  // namespace
+
+cudaError_t launch_bounds_probe(int index, int *status, cudaStream_t stream) {
+    bounds_probe_kernel<<<1, 1, 0, stream>>>(index, status);
+    return cudaGetLastError();
+}
+#endif
 
 cudaError_t launch_bounded_wait_probe(int *status, uint32_t rounds, cudaStream_t stream) {
     bounded_wait_probe_kernel<<<1, 32, 0, stream>>>(status, rounds);

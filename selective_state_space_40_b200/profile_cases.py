@@ -4,6 +4,9 @@ profiling it (for example under ncu with a kernel filter and a launch skip):
     python -m selective_state_space_40_b200.profile_cases CASE [REPEATS]
 
 CASE is one of: scan130m (selective scan forward, 130M-class layer),
+scan130m_reg (the same with the register-prefetch engine), scan2p8b (the
+2.8B-class layer), scanlong (the long-context fp32 layer, sequence split),
+scanlong_b1_L16k (its first 16384 tokens: a small case of the same kernels),
 conv130m (the same with the causal conv front-end, width 4), decode (one
 state update at b256 d5120 N16), bwd130m_b4 (training forward with saved
 states, then the backward, 130M-class layer with 4 batch rows), ssd2p7b_b2
@@ -21,8 +24,7 @@ from . import binding as mb
 from . import synthetic as syn
 
 
-def _scan(reps, conv=False):
-    w = syn.M130
+def _scan(reps, conv=False, w=syn.M130, plan=None):
     g = {k: v.cuda() for k, v in syn.scan_inputs(w).items()}
     y = torch.empty(w.batch, w.dim, w.seqlen, device="cuda")
     last = torch.empty(w.batch, w.dim, w.dstate, device="cuda")
@@ -33,7 +35,7 @@ def _scan(reps, conv=False):
                              g["delta_bias"], True, conv_b=cp["conv_b"], y=y, last_state=last)
         else:
             mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
-                        y=y, last_state=last)
+                        y=y, last_state=last, plan=plan)
 
 
 def _decode(reps):
@@ -75,6 +77,10 @@ def _ssd_cb(reps):
 
 CASES = {
     "scan130m": lambda r: _scan(r),
+    "scan130m_reg": lambda r: _scan(r, plan=(4, 1, 0, mb.MS_ENGINE_REGISTER)),
+    "scan2p8b": lambda r: _scan(r, w=syn.M2P8),
+    "scanlong": lambda r: _scan(r, w=syn.LONG),
+    "scanlong_b1_L16k": lambda r: _scan(r, w=syn.scaled(syn.LONG, seqlen=16384)),
     "conv130m": lambda r: _scan(r, conv=True),
     "decode": _decode,
     "bwd130m_b4": _bwd,

@@ -8,8 +8,10 @@ Recipe (one ``torch.Generator`` on the CPU, seeded per workload; the draw order
 is fixed): u, delta_raw, z, B, C ~ N(0, 1) drawn in fp32 and rounded to the
 storage dtype; then U ~ Uniform[lo, hi] giving delta_bias = log(expm1(U)) (so
 softplus(delta_bias) = U); then D ~ N(1, 0.1) (0.1 is the standard deviation).
-A[d, n] = -(n + 1) for every channel (no draw). The tiny workload keeps
-bias = 0 and D = 1. The decode workload draws state0 ~ N(0, 0.1) and the
+A[d, n] = -(n + 1) for every channel (no draw) in the workloads; parity cases
+also use ``a_matrix_varied`` (A drawn per channel and state, with one
+slow-decay channel) and ``tail_inputs`` (raw steps, gates and biases far out
+in the tails of softplus and silu). The tiny workload keeps bias = 0 and D = 1. The decode workload draws state0 ~ N(0, 0.1) and the
 per-channel parameters from ``seed``, and the inputs of step k from seed 1 + k.
 
 The workloads stand in for Mamba layers of 130M- and 2.8B-class models
@@ -93,6 +95,33 @@ def a_matrix(dim: int, dstate: int) -> torch.Tensor:
     return -torch.arange(1, dstate + 1, dtype=torch.float32).repeat(dim, 1).contiguous()
 
 
+def a_matrix_varied(dim: int, dstate: int, seed: int = 0, slow_channel: bool = True) -> torch.Tensor:
+    """A[d, n] = -exp(N(0, 1)) drawn independently per channel and state (so a
+    wrong channel or state index into A changes the result), from its own
+    generator (seed + 2000); channel dim // 2 gets A[d, n] = -1e-4 (n + 1), a
+    state that decays very slowly."""
+    g = torch.Generator().manual_seed(seed + 2000)
+    A = -torch.exp(torch.randn(dim, dstate, generator=g, dtype=torch.float32))
+    if slow_channel and dim > 0:
+        A[dim // 2] = -1e-4 * torch.arange(1, dstate + 1, dtype=torch.float32)
+    return A.contiguous()
+
+
+def tail_inputs(inp: Dict[str, torch.Tensor], seed: int = 0, lim: float = 40.0,
+                bias_lim: float = 15.0) -> Dict[str, torch.Tensor]:
+    """A copy of scan inputs whose raw step and gate are Uniform[-lim, lim]
+    and whose delta_bias is Uniform[-bias_lim, bias_lim] (own generator, seed
+    + 3000), stored in the inputs' dtype: softplus and silu are then evaluated
+    far into both tails, and exp(Delta A) both underflows and sits near 1."""
+    g = torch.Generator().manual_seed(seed + 3000)
+    out = dict(inp)
+    dt = inp["delta"].dtype
+    out["delta"] = ((torch.rand(inp["delta"].shape, generator=g) * 2 - 1) * lim).to(dt)
+    out["z"] = ((torch.rand(inp["z"].shape, generator=g) * 2 - 1) * lim).to(dt)
+    out["delta_bias"] = ((torch.rand(inp["delta_bias"].shape, generator=g) * 2 - 1) * bias_lim).to(torch.float32)
+    return out
+
+
 def scan_inputs(w: ScanWorkload, seed: Optional[int] = None) -> Dict[str, torch.Tensor]:
     """CPU tensors: u, delta, z [b, d, L] and B, C [b, N, L] in ``w.in_dtype``;
     A [d, N], D [d], delta_bias [d] in fp32."""
@@ -159,13 +188,15 @@ def ssd_inputs(w: SsdWorkload, seed: Optional[int] = None) -> Dict[str, torch.Te
     return dict(x=x, dt=dt, B=B, C=C, A=A, dt_bias=dt_bias, D=D)
 
 
-def decode_params(w: DecodeWorkload) -> Dict[str, torch.Tensor]:
-    """state0 [b, d, N] fp32 ~ N(0, 0.1); A, D, delta_bias as the 130M-class layer."""
+def decode_params(w: DecodeWorkload, varied_A: bool = False) -> Dict[str, torch.Tensor]:
+    """state0 [b, d, N] fp32 ~ N(0, 0.1); A, D, delta_bias as the 130M-class
+    layer (``varied_A``: A from ``a_matrix_varied`` instead)."""
     g = torch.Generator().manual_seed(w.seed)
     state0 = _normal(g, (w.batch, w.dim, w.dstate), torch.float32, std=0.1)
     bias = _inv_softplus_uniform(g, w.dim, w.bias_lo, w.bias_hi)
     D = _normal(g, (w.dim,), torch.float32, std=0.1, mean=1.0)
-    return dict(state0=state0, A=a_matrix(w.dim, w.dstate), D=D, delta_bias=bias)
+    A = a_matrix_varied(w.dim, w.dstate, w.seed) if varied_A else a_matrix(w.dim, w.dstate)
+    return dict(state0=state0, A=A, D=D, delta_bias=bias)
 
 
 def decode_step_inputs(w: DecodeWorkload, k: int) -> Dict[str, torch.Tensor]:

@@ -105,6 +105,13 @@ def test_scan_rejects_bad_plan_and_workspace(lib):
     assert _scan(_dims(), plan=mb.ScanPlan(4, 3, 0)) == mb.MS_ERR_SHAPE
     assert _scan(_dims(), plan=mb.ScanPlan(8, 2, 0)) == mb.MS_ERR_SHAPE
     assert _scan(_dims(), plan=mb.ScanPlan(4, 1, 5)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(4, 1, 0, 2)) == mb.MS_ERR_SHAPE      # no such engine
+    assert _scan(_dims(), plan=mb.ScanPlan(8, 1, 0, mb.MS_ENGINE_TMEM)) == mb.MS_ERR_SHAPE
+    assert _scan(_dims(), plan=mb.ScanPlan(4, 2, 0, mb.MS_ENGINE_TMEM)) == mb.MS_ERR_SHAPE
+    # the tensor-memory engine needs seqlen % 8 == 0 (and a device): refused before any launch
+    assert _scan(_dims(seqlen=30, u_sb=240, u_sd=30, delta_sb=240, delta_sd=30, z_sb=240, z_sd=30, y_sb=240,
+                       y_sd=30, B_sb=480, B_sn=30, C_sb=480, C_sn=30),
+                 plan=mb.ScanPlan(4, 1, 0, mb.MS_ENGINE_TMEM)) == mb.MS_ERR_SHAPE
     assert _scan(_dims(), ws=None, ws_bytes=64) == mb.MS_ERR_WORKSPACE
 
 
@@ -119,6 +126,15 @@ def test_choose_plan(lib):
     rc, plan = mb.mamba_scan_choose_plan(_dims(batch=8, dim=1536, seqlen=2048, in_dtype=mb.MS_BF16))
     assert rc == mb.MS_OK and plan.lanes_per_channel in (1, 2, 4, 8) and plan.poly8 in (0, 2, 4, 8)
     assert plan.chunks_per_lane in (1, 2)
+    # 130M-class shape: the tensor-memory engine (by sizes and strides)
+    d130 = _dims(batch=8, dim=1536, seqlen=2048, in_dtype=mb.MS_BF16, u_sb=1536 * 2048, u_sd=2048,
+                 delta_sb=1536 * 2048, delta_sd=2048, z_sb=1536 * 2048, z_sd=2048, y_sb=1536 * 2048, y_sd=2048,
+                 B_sb=16 * 2048, B_sn=2048, C_sb=16 * 2048, C_sn=2048)
+    rc, plan = mb.mamba_scan_choose_plan(d130)
+    assert rc == mb.MS_OK and plan.engine == mb.MS_ENGINE_TMEM and plan.lanes_per_channel == 4
+    # seqlen not a multiple of 8: the register engine
+    rc, plan = mb.mamba_scan_choose_plan(_dims(seqlen=30, u_sd=30, delta_sd=30, z_sd=30, y_sd=30, B_sn=30, C_sn=30))
+    assert rc == mb.MS_OK and plan.engine == mb.MS_ENGINE_REGISTER
     rc, _ = mb.mamba_scan_choose_plan(_dims(dstate=40))
     assert rc == mb.MS_ERR_SHAPE
 
@@ -146,6 +162,7 @@ def test_conv_scan_rejects_bad_arguments(lib):
     assert _conv(_dims(), plan=mb.ScanPlan(4, 2, 0)) == mb.MS_ERR_SHAPE
     assert _conv(_dims(), plan=mb.ScanPlan(4, 1, 2)) == mb.MS_ERR_SHAPE
     assert _conv(_dims(), plan=mb.ScanPlan(3, 1, 0)) == mb.MS_ERR_SHAPE
+    assert _conv(_dims(), plan=mb.ScanPlan(4, 1, 0, mb.MS_ENGINE_TMEM)) == mb.MS_ERR_SHAPE
     cd = mb.ConvDims(4, 0, 0, 1)
     assert mb.library().mamba_conv_scan_fwd(FAKE, FAKE, None, None, None, None, FAKE, FAKE, FAKE, FAKE,
                                             None, None, None, 1, None, FAKE, None, ctypes.byref(_dims()),

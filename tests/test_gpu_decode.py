@@ -1,4 +1,14 @@
-"""GPU parity of mamba_state_update (decode) against the fp64 oracle."""
+"""GPU parity of mamba_state_update (decode) against the fp64 oracle.
+
+Most cases use A drawn per channel and state (one slow channel) so that a
+wrong channel or state index into A fails; one case puts the raw step, gate
+and bias far in the tails. The full-size decode (b256 d5120, 1000 steps) is
+compared on every y of every step and on the whole final state, with the
+oracle split over batch rows on the host's cores.
+"""
+import os
+from concurrent.futures import ThreadPoolExecutor
+
 import numpy as np
 import pytest
 import torch
@@ -6,7 +16,7 @@ import torch
 import oracle
 from selective_state_space_40_b200 import binding as mb
 from selective_state_space_40_b200 import synthetic as syn
-from parity_util import check, check_bf16, check_fp32, check_out_bf16, f64
+from parity_util import StreamCheck, check, check_bf16, check_fp32, check_out_bf16, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -30,7 +40,7 @@ def _step_gpu(state, inp, params, use_z=True, use_D=True, use_bias=True, softplu
 @pytest.mark.parametrize("N", [1, 3, 4, 5, 16])
 def test_small_steps_full(dtype, N):
     w = syn.DecodeWorkload("small", batch=3, dim=37, dstate=N, steps=20, in_dtype=dtype)
-    p = syn.decode_params(w)
+    p = syn.decode_params(w, varied_A=True)
     params = {k: v.to(DEV) for k, v in p.items()}
     state = params["state0"].clone()
     h = f64(p["state0"])
@@ -47,7 +57,7 @@ def test_small_steps_full(dtype, N):
 @pytest.mark.parametrize("flags", [dict(use_z=False), dict(use_D=False), dict(use_bias=False)])
 def test_optional_inputs(flags):
     w = syn.DecodeWorkload("small", batch=4, dim=64, dstate=16, steps=5, in_dtype=torch.float32)
-    p = syn.decode_params(w)
+    p = syn.decode_params(w, varied_A=True)
     params = {k: v.to(DEV) for k, v in p.items()}
     state = params["state0"].clone()
     h = f64(p["state0"])
@@ -106,33 +116,60 @@ def test_scan_equals_decode_on_gpu():
 
 
 @pytest.mark.slow
-def test_full_decode_1000_steps_sampled():
-    """b256 d5120 N16, 1000 steps on the GPU at full size; a seeded sample of
-    channels is followed by the oracle through every step (every y) and the
-    final state."""
+def test_full_decode_1000_steps_every_output():
+    """b256 d5120 N16, 1000 steps on the GPU at full size; the oracle follows
+    every channel through every step: every y of every step and the whole
+    final state are compared."""
     w = syn.DECODE
     p = syn.decode_params(w)
     params = {k: v.to(DEV) for k, v in p.items()}
     state = params["state0"].clone()
-    rng = np.random.default_rng(99)
-    nb = 24
-    bs = np.sort(rng.choice(w.batch, nb, replace=False))
-    ds = np.sort(rng.choice(w.dim, 48, replace=False))
-    h = f64(p["state0"][bs][:, ds])
-    A, D, bias = f64(p["A"][ds]), f64(p["D"][ds]), f64(p["delta_bias"][ds])
-    y_all, yr_all = [], []
-    for k in range(w.steps):
-        inp = syn.decode_step_inputs(w, k)
-        y = _step_gpu(state, inp, params)
-        sel = lambda t: f64(t[bs][:, ds])  # noqa: E731
-        yr, h = oracle.state_update(h, sel(inp["x"]), sel(inp["delta"]), A, f64(inp["B"][bs]),
-                                    f64(inp["C"][bs]), D, sel(inp["z"]), bias, True)
-        y_all.append(f64(y[torch.as_tensor(bs)][:, torch.as_tensor(ds)]))
-        yr_all.append(yr)
+    h = f64(p["state0"])
+    A, D, bias = f64(p["A"]), f64(p["D"]), f64(p["delta_bias"])
+    nthreads = max(1, min(32, os.cpu_count() or 1))
+    rows = [ix for ix in np.array_split(np.arange(w.batch), nthreads) if len(ix)]
+    slices = [slice(int(ix[0]), int(ix[-1]) + 1) for ix in rows]
+    hs = [h[sl].copy() for sl in slices]  # each thread's rows of the oracle state
+    cy = StreamCheck(w.in_dtype, "decode every y of every step")
+
+    def oracle_rows(i, inp):
+        sl = slices[i]
+        yr, hs[i] = oracle.state_update(hs[i], f64(inp["x"][sl]), f64(inp["delta"][sl]), A, f64(inp["B"][sl]),
+                                        f64(inp["C"][sl]), D, f64(inp["z"][sl]), bias, True)
+        return yr
+
+    with ThreadPoolExecutor(len(slices)) as pool:  # ctypes calls release the GIL
+        for k in range(w.steps):
+            inp = syn.decode_step_inputs(w, k)
+            y = _step_gpu(state, inp, params)
+            yr = np.concatenate(list(pool.map(lambda i: oracle_rows(i, inp), range(len(slices)))))
+            cy.add(f64(y), yr)
     torch.cuda.synchronize()
-    assert torch.isfinite(state).all()
-    check_bf16(np.stack(y_all), np.stack(yr_all), "decode every y (sampled channels)")
-    check_bf16(f64(state[torch.as_tensor(bs)][:, torch.as_tensor(ds)]), h, "decode final state (sampled)")
+    cy.finish()
+    check_bf16(f64(state), np.concatenate(hs), "decode final state (every element)")
+
+
+def test_tails_both_kernels():
+    """Raw steps and gates in [-40, 40], biases in [-15, 15], A per channel:
+    the bulk-copy stream kernel (dim 256) and the general kernel (dim 37)."""
+    for dim in (256, 37):
+        w = syn.DecodeWorkload("tails", batch=3, dim=dim, dstate=16, steps=6, in_dtype=torch.float32)
+        p = syn.decode_params(w, varied_A=True)
+        gen = torch.Generator().manual_seed(dim)
+        p["delta_bias"] = (torch.rand(dim, generator=gen) * 2 - 1) * 15.0
+        params = {k: v.to(DEV) for k, v in p.items()}
+        state = params["state0"].clone()
+        h = f64(p["state0"])
+        for k in range(w.steps):
+            inp = syn.decode_step_inputs(w, k)
+            inp["delta"] = (torch.rand(inp["delta"].shape, generator=gen) * 2 - 1) * 40.0
+            inp["z"] = (torch.rand(inp["z"].shape, generator=gen) * 2 - 1) * 40.0
+            y = _step_gpu(state, inp, params)
+            yr, h = oracle.state_update(h, f64(inp["x"]), f64(inp["delta"]), f64(p["A"]), f64(inp["B"]),
+                                        f64(inp["C"]), f64(p["D"]), f64(inp["z"]), f64(p["delta_bias"]), True)
+            torch.cuda.synchronize()
+            check_fp32(f64(y), yr, f"tails dim {dim} step {k} y")
+        check_fp32(f64(state), h, f"tails dim {dim} final state")
 
 
 @pytest.mark.parametrize("dtype,out_dtype,use_z", [
@@ -142,7 +179,7 @@ def test_stream_path_small(dtype, out_dtype, use_z):
     """dim a multiple of 128 with dense 16-state rows: the bulk-copy stream
     kernel runs (several tiles per CTA, every step checked)."""
     w = syn.DecodeWorkload("stream", batch=5, dim=384, dstate=16, steps=12, in_dtype=dtype)
-    p = syn.decode_params(w)
+    p = syn.decode_params(w, varied_A=True)
     params = {k: v.to(DEV) for k, v in p.items()}
     state = params["state0"].clone()
     h = f64(p["state0"])

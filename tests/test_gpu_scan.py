@@ -1,10 +1,15 @@
 """GPU parity of mamba_scan_fwd against the fp64 oracle (called through the C ABI).
 
-Small cases are compared element by element in full; the full-size workloads
-(130M-class, 2.8B-class, long context) are run whole on the GPU in the launch
-configuration the benchmark uses, and a seeded sample of whole channels (every
-token and the final state) is recomputed by the oracle one channel at a time.
+Small cases are compared element by element in full, most of them with A drawn
+per channel and state (so a wrong channel or state index into A fails) and
+some with raw steps, gates and biases far in the tails of softplus and silu.
+The full-size workloads (130M-class, 2.8B-class, long context) are run whole
+on the GPU in the launch configuration the benchmark uses, and every output
+(all of y and last_state) is compared with the oracle, which runs over blocks
+of channels on the host's cores.
 """
+import os
+
 import numpy as np
 import pytest
 import torch
@@ -12,7 +17,7 @@ import torch
 import oracle
 from selective_state_space_40_b200 import binding as mb
 from selective_state_space_40_b200 import synthetic as syn
-from parity_util import check, check_fp32, check_out_bf16, f64
+from parity_util import StreamCheck, check, check_fp32, check_out_bf16, f64
 
 pytestmark = pytest.mark.gpu
 
@@ -29,6 +34,16 @@ def _lib():
 
 def _to_dev(inp):
     return {k: v.to(DEV) for k, v in inp.items()}
+
+
+def varied(inp, seed=0):
+    """The same inputs with A drawn per channel and state (one slow channel)."""
+    out = dict(inp)
+    out["A"] = syn.a_matrix_varied(inp["A"].shape[0], inp["A"].shape[1], seed)
+    return out
+
+
+ORACLE_THREADS = max(1, min(32, os.cpu_count() or 1))
 
 
 def run_gpu(inp, softplus=True, use_z=True, use_D=True, use_bias=True, initial_state=None,
@@ -50,7 +65,7 @@ def run_oracle(inp, softplus=True, use_z=True, use_D=True, use_bias=True, h0=Non
                        h0=None if h0 is None else f64(h0))
 
 
-def compare_full(inp, what, **kw):
+def compare_full(inp, what, scaled=False, **kw):
     okw = {k: kw[k] for k in ("softplus", "use_z", "use_D", "use_bias") if k in kw}
     h0 = kw.get("initial_state")
     y, last = run_gpu(inp, **kw)
@@ -59,8 +74,8 @@ def compare_full(inp, what, **kw):
     if kw.get("out_dtype", torch.float32) == torch.bfloat16:
         check_out_bf16(f64(y), yr, f"{what} y(bf16 out)")
     else:
-        check(f64(y), yr, dt, f"{what} y")
-    check(f64(last), lr, dt, f"{what} last_state")
+        check(f64(y), yr, dt, f"{what} y", scaled=scaled)
+    check(f64(last), lr, dt, f"{what} last_state", scaled=scaled)
     return y, last
 
 
@@ -75,13 +90,13 @@ def test_tiny_workload_full():
 @pytest.mark.parametrize("L", [1, 7, 63, 64, 65, 1000])
 def test_lengths_ragged(dtype, L):
     w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=L, in_dtype=dtype, seed=L)
-    compare_full(syn.scan_inputs(w), f"L={L} {dtype}")
+    compare_full(varied(syn.scan_inputs(w), L), f"L={L} {dtype}")
 
 
 @pytest.mark.parametrize("N", [1, 2, 3, 4, 9, 16])
 def test_dstate(N):
     w = syn.scaled(syn.M130, batch=2, dim=24, dstate=N, seqlen=300, in_dtype=torch.float32, seed=100 + N)
-    compare_full(syn.scan_inputs(w), f"N={N}")
+    compare_full(varied(syn.scan_inputs(w), N), f"N={N}")
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -89,7 +104,27 @@ def test_dstate(N):
 @pytest.mark.parametrize("poly", [0, 2, 4, 8])
 def test_every_plan(dtype, lanes, chunks, poly):
     w = syn.scaled(syn.M130, batch=3, dim=136, seqlen=517, in_dtype=dtype, seed=7)
-    compare_full(syn.scan_inputs(w), f"plan {lanes}/{chunks}/{poly} {dtype}", plan=(lanes, chunks, poly))
+    compare_full(varied(syn.scan_inputs(w), 7), f"plan {lanes}/{chunks}/{poly} {dtype}",
+                 plan=(lanes, chunks, poly))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("lanes,chunks", [(1, 1), (2, 2), (4, 1), (8, 1)])
+@pytest.mark.parametrize("poly", [0, 8])
+def test_tails(dtype, lanes, chunks, poly):
+    """Raw steps and gates in [-40, 40], biases in [-15, 15], A per channel:
+    softplus on both of its branches and far into both tails, silu at large
+    |z|, exp(Delta A) from 1 down to underflow (the polynomial's clamp)."""
+    w = syn.scaled(syn.M130, batch=2, dim=72, seqlen=300, in_dtype=dtype, seed=17)
+    inp = syn.tail_inputs(varied(syn.scan_inputs(w), 17), seed=17)
+    compare_full(inp, f"tails {lanes}/{chunks}/{poly} {dtype}", scaled=True, plan=(lanes, chunks, poly))
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_tails_automatic_plan(dtype):
+    w = syn.scaled(syn.M130, batch=2, dim=200, seqlen=1000, in_dtype=dtype, seed=18)
+    inp = syn.tail_inputs(varied(syn.scan_inputs(w), 18), seed=18)
+    compare_full(inp, f"tails auto {dtype}", scaled=True)
 
 
 @pytest.mark.parametrize("flags", [
@@ -97,7 +132,7 @@ def test_every_plan(dtype, lanes, chunks, poly):
     dict(use_z=False, use_D=False, use_bias=False)])
 def test_optional_inputs(flags):
     w = syn.scaled(syn.M130, batch=2, dim=64, seqlen=200, in_dtype=torch.float32, seed=3)
-    inp = syn.scan_inputs(w)
+    inp = varied(syn.scan_inputs(w), 3)
     if not flags.get("softplus", True):
         inp["delta"] = inp["delta"].abs() * 0.05  # keep the step positive without softplus
     compare_full(inp, f"flags {flags}", **flags)
@@ -111,7 +146,7 @@ def test_bf16_output(dtype):
 
 def test_initial_state_and_split():
     w = syn.scaled(syn.M130, batch=2, dim=48, seqlen=700, in_dtype=torch.float32, seed=9)
-    inp = syn.scan_inputs(w)
+    inp = varied(syn.scan_inputs(w), 9)
     h0 = torch.randn(2, 48, 16, generator=torch.Generator().manual_seed(1)) * 0.3
     compare_full(inp, "initial_state", initial_state=h0)
     # scan [0, m) then [m, L) from the returned state == scan [0, L)
@@ -178,46 +213,39 @@ def test_repeat_is_bitwise_deterministic():
 
 # ------------------------------------------------- full-size workloads ----
 
-def sampled_parity(w, n_samples, seed=1234):
+def full_parity(w, block):
+    """The whole workload on the GPU (automatic plan, as benchmarked); every
+    element of y and last_state against the oracle, run over blocks of
+    `block` channels (all batch rows) on the host's cores."""
     inp = syn.scan_inputs(w)
-    y, last = run_gpu(inp)  # the launch configuration the benchmark uses
-    assert torch.isfinite(y).all() and torch.isfinite(last).all()
-    rng = np.random.default_rng(seed)
-    picks = [(int(rng.integers(w.batch)), int(rng.integers(w.dim))) for _ in range(n_samples)]
-    picks += [(0, 0), (w.batch - 1, w.dim - 1)]
-    ys, yrs, ls, lrs = [], [], [], []
-    for b, d in picks:
-        yr, lr = oracle.scan(f64(inp["u"][b:b + 1, d:d + 1]), f64(inp["delta"][b:b + 1, d:d + 1]),
-                             f64(inp["A"][d:d + 1]), f64(inp["B"][b:b + 1]), f64(inp["C"][b:b + 1]),
-                             f64(inp["D"][d:d + 1]), f64(inp["z"][b:b + 1, d:d + 1]),
-                             f64(inp["delta_bias"][d:d + 1]), True)
-        ys.append(f64(y[b, d]))
-        yrs.append(yr[0, 0])
-        ls.append(f64(last[b, d]))
-        lrs.append(lr[0, 0])
-    dt = w.in_dtype
-    if dt == torch.bfloat16:
-        check(np.concatenate(ys), np.concatenate(yrs), dt, f"{w.name} sampled y")
-        check(np.concatenate(ls), np.concatenate(lrs), dt, f"{w.name} sampled last_state")
-    else:
-        for i, (b, d) in enumerate(picks):
-            check_fp32(ys[i], yrs[i], f"{w.name} y[{b},{d}]")
-            check_fp32(ls[i], lrs[i], f"{w.name} last[{b},{d}]")
+    y, last = run_gpu(inp)
+    y, last = y.cpu(), last.cpu()
+    cy = StreamCheck(w.in_dtype, f"{w.name} y (every element)")
+    cl = StreamCheck(w.in_dtype, f"{w.name} last_state (every element)")
+    for d0 in range(0, w.dim, block):
+        d1 = min(w.dim, d0 + block)
+        yr, lr = oracle.scan(f64(inp["u"][:, d0:d1]), f64(inp["delta"][:, d0:d1]), f64(inp["A"][d0:d1]),
+                             f64(inp["B"]), f64(inp["C"]), f64(inp["D"][d0:d1]), f64(inp["z"][:, d0:d1]),
+                             f64(inp["delta_bias"][d0:d1]), True, nthreads=ORACLE_THREADS)
+        cy.add(f64(y[:, d0:d1]), yr)
+        cl.add(f64(last[:, d0:d1]), lr)
+    cy.finish()
+    cl.finish()
 
 
 @pytest.mark.slow
-def test_full_130m_sampled():
-    sampled_parity(syn.M130, 48)
+def test_full_130m_every_output():
+    full_parity(syn.M130, 768)
 
 
 @pytest.mark.slow
-def test_full_2p8b_sampled():
-    sampled_parity(syn.M2P8, 32)
+def test_full_2p8b_every_output():
+    full_parity(syn.M2P8, 512)
 
 
 @pytest.mark.slow
-def test_full_long_context_sampled():
-    sampled_parity(syn.LONG, 10)
+def test_full_long_context_every_output():
+    full_parity(syn.LONG, 128)
 
 
 # ------------------------------------------------------ sequence split ------
@@ -229,7 +257,7 @@ def test_sequence_split_against_oracle(dtype, b, d, L):
     segments (ragged last segment for 20000 and 9000 tokens, equal segments
     for 16384), chains the carries and rescans; every output is checked."""
     w = syn.scaled(syn.LONG, batch=b, dim=d, seqlen=L, in_dtype=dtype, seed=L + d)
-    inp = syn.scan_inputs(w)
+    inp = varied(syn.scan_inputs(w), L + d)
     dims = mb.scan_dims_for(inp["u"], inp["delta"], inp["B"], inp["C"], inp["z"],
                             torch.empty(b, d, L))
     assert mb.mamba_scan_workspace_size(dims) > 0  # the split path runs
@@ -240,7 +268,14 @@ def test_sequence_split_against_oracle(dtype, b, d, L):
 @pytest.mark.parametrize("flags", [dict(use_z=False), dict(use_D=False), dict(use_bias=False)])
 def test_sequence_split_options(flags):
     w = syn.scaled(syn.LONG, batch=1, dim=48, seqlen=12000, in_dtype=torch.float32, seed=77)
-    compare_full(syn.scan_inputs(w), f"split {flags}", **flags)
+    compare_full(varied(syn.scan_inputs(w), 77), f"split {flags}", **flags)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_sequence_split_tails(dtype):
+    w = syn.scaled(syn.LONG, batch=1, dim=64, seqlen=10000, in_dtype=dtype, seed=79)
+    inp = syn.tail_inputs(varied(syn.scan_inputs(w), 79), seed=79)
+    compare_full(inp, f"split tails {dtype}", scaled=True)
 
 
 def test_sequence_split_matches_unsplit_plan():

@@ -30,8 +30,10 @@ def _lib():
     mb.library()
 
 
-def _grads_inputs(w, seed, out_dtype=torch.float32, with_dlast=True, with_h0=False):
+def _grads_inputs(w, seed, out_dtype=torch.float32, with_dlast=True, with_h0=False, varied_A=True):
     inp = syn.scan_inputs(w)
+    if varied_A:  # A per channel and state (one slow channel): dA and A's indexing are exercised
+        inp["A"] = syn.a_matrix_varied(w.dim, w.dstate, seed)
     g = torch.Generator().manual_seed(seed)
     dout = torch.randn(w.batch, w.dim, w.seqlen, generator=g).to(out_dtype)
     dlast = torch.randn(w.batch, w.dim, w.dstate, generator=g) if with_dlast else None
@@ -60,15 +62,15 @@ def run_oracle(inp, dout, dlast, h0, use_z=True, use_D=True, use_bias=True, soft
                            h0=None if h0 is None else f64(h0), dlast=None if dlast is None else f64(dlast))
 
 
-def compare(gg, rr, dtype, what):
+def compare(gg, rr, dtype, what, scaled=False):
     torch.cuda.synchronize()
     for k in GRADS:
         if rr[k] is None:
             assert gg[k] is None, f"{what}: {k} returned for a missing input"
             continue
-        check(f64(gg[k]), rr[k], dtype, f"{what} {k}")
+        check(f64(gg[k]), rr[k], dtype, f"{what} {k}", scaled=scaled)
     if gg["dinitial_state"] is not None:
-        check(f64(gg["dinitial_state"]), rr["dh0"], dtype, f"{what} dinitial_state")
+        check(f64(gg["dinitial_state"]), rr["dh0"], dtype, f"{what} dinitial_state", scaled=scaled)
 
 
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
@@ -96,6 +98,16 @@ def test_optional_inputs(flags):
         inp["delta_bias"] = torch.zeros_like(inp["delta_bias"])
     compare(run_gpu(inp, dout, dlast, h0, **flags), run_oracle(inp, dout, dlast, h0, **flags),
             torch.float32, f"{flags}")
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_tails(dtype):
+    """Raw steps and gates in [-20, 20], biases in [-10, 10]: softplus' and
+    silu' far into their tails, A_bar from 1 down to underflow."""
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=150, in_dtype=dtype, seed=450)
+    inp, dout, dlast, h0 = _grads_inputs(w, 23, with_h0=True)
+    inp = syn.tail_inputs(inp, seed=450, lim=20.0, bias_lim=10.0)
+    compare(run_gpu(inp, dout, dlast, h0), run_oracle(inp, dout, dlast, h0), dtype, f"tails {dtype}", scaled=True)
 
 
 def test_bf16_dout():

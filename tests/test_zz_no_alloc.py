@@ -1,14 +1,15 @@
 """mamba_scan_bwd_noalloc (collected last): the allocation-free backward,
 whose recomputed saved states live in the library's fixed device scratch,
 gives the results of mamba_scan_bwd with a caller workspace, on two calls in
-a row (the second call reuses the same scratch). Passes alone and after the
-other tests."""
+a row (the second call reuses the same scratch), and each call's gradients
+match the fp64 oracle's. Passes alone and after the other tests."""
 import pytest
 import torch
 
+import oracle
 from selective_state_space_40_b200 import binding as mb
 from selective_state_space_40_b200 import synthetic as syn
-from parity_util import check_fp32, f64
+from parity_util import check, check_fp32, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -24,7 +25,9 @@ def _lib():
 @pytest.mark.parametrize("dtype,L", [(torch.float32, 300), (torch.bfloat16, 1000)])
 def test_noalloc_matches_workspace_backward_twice(dtype, L):
     w = syn.scaled(syn.M130, batch=3, dim=96, seqlen=L, in_dtype=dtype, seed=900 + L)
-    inp = {k: v.to(DEV) for k, v in syn.scan_inputs(w).items()}
+    host = syn.scan_inputs(w)
+    host["A"] = syn.a_matrix_varied(w.dim, w.dstate, 900 + L)
+    inp = {k: v.to(DEV) for k, v in host.items()}
     gen = torch.Generator().manual_seed(5)
     dout = torch.randn(w.batch, w.dim, w.seqlen, generator=gen).to(DEV)
     dlast = torch.randn(w.batch, w.dim, w.dstate, generator=gen).to(DEV)
@@ -38,6 +41,13 @@ def test_noalloc_matches_workspace_backward_twice(dtype, L):
             assert torch.equal(r[k], ref[k]), k
         for k in ("dA", "dB", "dC", "dD", "ddelta_bias"):    # fp32 atomic sums: order may differ
             check_fp32(f64(r[k]), f64(ref[k]), f"noalloc {k}")
+    # and directly against the oracle's gradients of the same inputs
+    rr = oracle.scan_bwd(*(f64(host[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")), True,
+                         f64(dout), h0=f64(h0), dlast=f64(dlast))
+    for r in runs:
+        for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"):
+            check(f64(r[k]), rr[k], dtype, f"noalloc vs oracle {k}")
+        check(f64(r["dinitial_state"]), rr["dh0"], dtype, "noalloc vs oracle dinitial_state")
 
 
 def test_noalloc_oversize_is_rejected_without_launch():

@@ -623,13 +623,16 @@ constexpr int kSmemLimit = 227 * 1024;
 constexpr int kOneCtaSmem = 116 * 1024;
 
 // Compute warps per CTA: the fewest that put every (batch row, channel
-// block) CTA in one wave on the SMs, at most kMaxWLarge.
-int choose_w(int64_t batch, int64_t dim, int num_sms) {
+// block) CTA in one wave on the SMs, at most kMaxWLarge and at most what two
+// stages of the input dtype leave room for in shared memory.
+int choose_w(int64_t batch, int64_t dim, int num_sms, int in_bytes) {
     const int64_t units = (dim + kCW - 1) / kCW;
+    int wmax = kMaxWLarge;
+    while (wmax > 1 && TmLayout{wmax, 2, in_bytes}.total() > kSmemLimit) --wmax;
     int64_t w = (batch * units + num_sms - 1) / num_sms;
     if (w < 1) w = 1;
-    while (w < kMaxWLarge && batch * ((units + w - 1) / w) > num_sms) ++w;
-    if (w > kMaxWLarge) w = kMaxWLarge;
+    while (w < wmax && batch * ((units + w - 1) / w) > num_sms) ++w;
+    if (w > wmax) w = wmax;
     if (w > units) w = units;
     return (int)w;
 }
@@ -702,8 +705,8 @@ bool scan_tmem_applies(const ScanArgs &a, bool in_bf16, int out_bytes) {
 
 cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool in_bf16, bool out_bf16, int num_sms,
                                  cudaStream_t stream) {
-    const int W = choose_w(a.batch, a.dim, num_sms);
     const int es = in_bf16 ? 2 : 4;
+    const int W = choose_w(a.batch, a.dim, num_sms, es);
     int S = 3;
     while (S > 2 && TmLayout{W, S, es}.total() > kSmemLimit) --S;
     if (TmLayout{W, S, es}.total() > kSmemLimit) return cudaErrorInvalidConfiguration;

@@ -140,6 +140,25 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256
 // with 16 K elements: core matrix (r / 8, kc) at ((r / 8) * 2 + kc) * 128.
 __device__ __forceinline__ int op_off(int r, int kc) { return (((r >> 3) * 2 + kc) * 8 + (r & 7)) * 16; }
 
+// 16 consecutive tensor-memory columns of this warp's 32 lanes.
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait16(uint32_t (&v)[16]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),
+                   "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),
+                   "+r"(v[15])
+                 :
+                 : "memory");
+}
+
 // 32 consecutive tensor-memory columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
@@ -163,6 +182,34 @@ __device__ __forceinline__ void tmem_wait(uint32_t (&v)[32]) {
                    "+r"(v[29]), "+r"(v[30]), "+r"(v[31])
                  :
                  : "memory");
+}
+
+template <int NCOL>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, uint32_t (&v)[NCOL]) {
+    if constexpr (NCOL == 32) tmem_ld32(taddr, v);
+    else tmem_ld16(taddr, v);
+}
+template <int NCOL>
+__device__ __forceinline__ void tmem_wait(uint32_t (&v)[NCOL]) {
+    if constexpr (NCOL == 32) tmem_wait(v);
+    else tmem_wait16(v);
+}
+
+// N (2 or 4) consecutive floats of shared memory (8- or 16-byte aligned).
+template <int N>
+__device__ __forceinline__ void lds_vec(const float *p, float (&v)[N]) {
+    if constexpr (N == 4) {
+        const float4 q = *reinterpret_cast<const float4 *>(p);
+        v[0] = q.x; v[1] = q.y; v[2] = q.z; v[3] = q.w;
+    } else {
+        const float2 q = *reinterpret_cast<const float2 *>(p);
+        v[0] = q.x; v[1] = q.y;
+    }
+}
+template <int N>
+__device__ __forceinline__ void sts_vec(float *p, const float (&v)[N]) {
+    if constexpr (N == 4) *reinterpret_cast<float4 *>(p) = make_float4(v[0], v[1], v[2], v[3]);
+    else *reinterpret_cast<float2 *>(p) = make_float2(v[0], v[1]);
 }
 
 __device__ __forceinline__ void report_abort(const ScanArgs &a, volatile int *abort_flag) {
@@ -191,6 +238,9 @@ template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT>
 __global__ void __launch_bounds__(32 * (MAXW + 1), 1)
 scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, const int W, const int S) {
     extern __shared__ __align__(1024) unsigned char smem[];
+    // tokens per tensor-memory load: 4 (32 columns) where registers allow two
+    // such sets without spilling, 2 (16 columns) in the larger instantiations
+    constexpr int TOK = MAXW <= 11 ? 4 : 2;
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cwc = lay.cwc();
@@ -471,28 +521,32 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             ok = __all_sync(0xffffffffu, bar_wait(bar(mma0 + vb), (uint32_t)((k >> 1) & 1)));
             if (!ok) break;
             asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-            // ---- states: 8 groups of 4 tokens
-#pragma unroll 1
-            for (int j = 0; j < 8; ++j) {
-                uint32_t bc[32];
-                MS_CHECK(a.status, vb * kBufCols + 32 * j + 32 <= kTmemCols && 4 * c + g < 32);
-                tmem_ld32(tmem + trow + (uint32_t)(vb * kBufCols + 32 * j), bc);
-                const float4 dl4 = *reinterpret_cast<const float4 *>(xd + c * kRow + 4 * j);
-                const float4 du4 = *reinterpret_cast<const float4 *>(xu + c * kRow + 4 * j);
-                tmem_wait(bc);
-                const float dls[4] = {dl4.x, dl4.y, dl4.z, dl4.w};
-                const float dus[4] = {du4.x, du4.y, du4.z, du4.w};
-                float part[4];
+            // ---- states: groups of TOK tokens; the tensor-memory load and the
+            // Delta / Delta*u loads of the next group are in flight while a
+            // group computes (two register sets, used alternately)
+            const uint32_t tcol = tmem + trow + (uint32_t)(vb * kBufCols);
+            uint32_t bcA[8 * TOK], bcB[8 * TOK];
+            float dlA[TOK], duA[TOK], dlB[TOK], duB[TOK];
+            auto fetch = [&](int j, uint32_t(&bc)[8 * TOK], float(&dl)[TOK], float(&du)[TOK]) {
+                MS_CHECK(a.status, vb * kBufCols + 8 * TOK * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                tmem_ld<8 * TOK>(tcol + (uint32_t)(8 * TOK * j), bc);
+                lds_vec<TOK>(xd + c * kRow + TOK * j, dl);
+                lds_vec<TOK>(xu + c * kRow + TOK * j, du);
+            };
+            auto group = [&](int j, const uint32_t(&bc)[8 * TOK], const float(&dls)[TOK], const float(&dus)[TOK]) {
+                float part[TOK];
 #pragma unroll
-                for (int t = 0; t < 4; ++t) {
+                for (int t = 0; t < TOK; ++t) {
                     const f2 dl2 = f2_splat(dls[t]);
                     const f2 du2 = f2_splat(dus[t]);
                     f2 acc = 0ull;
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        const f2 Bp = f2_make(__uint_as_float(bc[8 * t + 2 * p]), __uint_as_float(bc[8 * t + 2 * p + 1]));
+                        const f2 Bp =
+                            f2_make(__uint_as_float(bc[8 * t + 2 * p]), __uint_as_float(bc[8 * t + 2 * p + 1]));
                         const f2 x = f2_mul(A2[p], dl2);
-                        const bool poly = (2 * t + p) < POLY8;
+                        // a fixed share of the (token, pair) slots of every 4 tokens on the polynomial
+                        const bool poly = (2 * ((TOK * j + t) & 3) + p) < POLY8;
                         f2 ab;
                         if (poly) {
                             ab = exp2_poly2(x);
@@ -512,9 +566,19 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                     f2_split(acc, lo, hi);
                     part[t] = lo + hi;
                 }
-                if constexpr (YOUT)
-                    *reinterpret_cast<float4 *>(pr + (c * 4 + g) * kRow + 4 * j) =
-                        make_float4(part[0], part[1], part[2], part[3]);
+                if constexpr (YOUT) sts_vec<TOK>(pr + (c * 4 + g) * kRow + TOK * j, part);
+            };
+            constexpr int NG = kT / TOK;
+            fetch(0, bcA, dlA, duA);
+            tmem_wait<8 * TOK>(bcA);
+#pragma unroll 1
+            for (int j = 0; j < NG; j += 2) {
+                fetch(j + 1, bcB, dlB, duB);
+                group(j, bcA, dlA, duA);
+                tmem_wait<8 * TOK>(bcB);
+                if (j + 2 < NG) fetch(j + 2, bcA, dlA, duA);
+                group(j + 1, bcB, dlB, duB);
+                if (j + 2 < NG) tmem_wait<8 * TOK>(bcA);
             }
             // tensor-memory buffer vb is read: release it to the producer
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
@@ -617,7 +681,11 @@ bool encode3(CUtensorMap *m, const void *base, bool bf16, int64_t L, int64_t mid
 
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-constexpr int kMaxWSmall = 12;
+// Instantiations by compute warps per CTA: the block's warps spread over the
+// SM's four schedulers, each with a quarter of the register file, so 12
+// warps leave 168 registers a thread, 16 warps 128 and 19 warps 96.
+constexpr int kMaxWSmall = 11;
+constexpr int kMaxWMid = 15;
 constexpr int kMaxWLarge = 18;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kOneCtaSmem = 116 * 1024;
@@ -657,6 +725,7 @@ cudaError_t launch_tm(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaS
 template <typename TIn, typename TOut, int POLY8, bool YOUT = true>
 cudaError_t launch_w(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaStream_t stream) {
     if (W <= kMaxWSmall) return launch_tm<TIn, TOut, POLY8, kMaxWSmall, YOUT>(a, maps, W, S, stream);
+    if (W <= kMaxWMid) return launch_tm<TIn, TOut, POLY8, kMaxWMid, YOUT>(a, maps, W, S, stream);
     return launch_tm<TIn, TOut, POLY8, kMaxWLarge, YOUT>(a, maps, W, S, stream);
 }
 

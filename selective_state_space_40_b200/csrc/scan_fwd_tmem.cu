@@ -62,9 +62,15 @@ namespace {
 constexpr int kT = 32;                 // tokens per tile
 constexpr int kCW = 8;                 // channels per compute warp (4 lanes each)
 constexpr int kRow = 36;               // floats per padded exchange row (bank spread)
+constexpr int kRowS = 4 * 32 + 4;      // floats per padded row of splatted pairs
 constexpr int kTmemCols = 512;         // two buffers of 256 columns
 constexpr int kBufCols = 256;          // 32 tokens x 8 values
-constexpr uint32_t kSpin = 1u << 20;   // try_wait rounds before a wait gives up
+// Bounded waits: a try may suspend the thread for up to kSuspendNs while the
+// phase is incomplete (it resumes as soon as the phase completes), so a
+// waiting warp issues a few instructions per microsecond instead of spinning;
+// kSpin tries bound a wait to well under a second.
+constexpr uint32_t kSuspendNs = 20000;
+constexpr uint32_t kSpin = 1u << 15;
 
 // Shared memory layout for W compute warps and S stages (host and device).
 struct TmLayout {
@@ -79,7 +85,13 @@ struct TmLayout {
     __host__ __device__ int bc_tile() const { return 16 * kT * in_bytes; }
     __host__ __device__ int stage_bytes() const { return 3 * chan_tile() + 2 * bc_tile(); }
     __host__ __device__ int stage(int s) const { return 1024 + 4096 + 2 * 8192 + s * stage_bytes(); }
-    __host__ __device__ int xch_bytes() const { return (2 * kCW * kRow + kCW * 4 * kRow) * 4; }
+    // per-warp exchange: Delta and Delta*u (as splatted pairs (Delta, Delta,
+    // Delta*u, Delta*u) per token in the 12-warp instantiation, else two
+    // plain rows), then the partial readouts [8 channels x 4 lanes][kRow]
+    __host__ __device__ bool splat() const { return W <= 11; }
+    __host__ __device__ int xch_bytes() const {
+        return ((splat() ? kCW * kRowS : 2 * kCW * kRow) + kCW * 4 * kRow) * 4;
+    }
     __host__ __device__ int xch(int w) const { return stage(S) + w * xch_bytes(); }
     __host__ __device__ int total() const { return xch(W); }
 };
@@ -104,10 +116,10 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
-            : "r"(bar), "r"(parity)
+            : "r"(bar), "r"(parity), "r"(kSuspendNs)
             : "memory");
         if (done) return true;
     }
@@ -241,6 +253,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
     // tokens per tensor-memory load: 4 (32 columns) where registers allow two
     // such sets without spilling, 2 (16 columns) in the larger instantiations
     constexpr int TOK = MAXW <= 11 ? 4 : 2;
+    constexpr bool SPLAT = MAXW <= 11;  // matches TmLayout::splat()
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cwc = lay.cwc();
@@ -330,18 +343,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
         bool ok = true;
         for (int k = 0; k < ntiles && ok; ++k) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
-            // (1) loads of tile k + S - 1 into the stage tile k - 1 used
-            const int kk = k + S - 1;
-            if (kk < ntiles) {
-                if (lane == 0) {
-                    if (kk >= S) ok = bar_wait(bar(empty0 + kk % S), (uint32_t)(((kk - S) / S) & 1));
-                    if (ok) issue(kk);
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-                if (!ok) break;
-                issued = kk + 1;
-            }
-            // (2) tile k's B/C -> V[k % 2], once MMA k - 2 has finished reading it
+            // (1) tile k's B/C -> V[k % 2], once MMA k - 2 has finished reading it
             const int s = k % S, vb = k & 1;
             ok = bar_wait(bar(full0 + s), (uint32_t)((k / S) & 1));
             if (ok && k >= 2) ok = bar_wait(bar(mma0 + vb), (uint32_t)(((k - 2) >> 1) & 1));
@@ -357,18 +359,18 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 for (int r = lane; r < 256; r += 32) {
                     const int t = r >> 3, v = r & 7;
                     if (!MS_CHECK(a.status, op_off(r, 1) + 16 <= 8192 && t < kT)) continue;
-                    float val[4];
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) val[k4] = bc_value<TIn>(Bs, Cs, t, k4, v);
                     if constexpr (sizeof(TIn) == 2) {
-                        // bf16 inputs: exact in one part (columns 0..3; 4..11 stay zero)
-                        *reinterpret_cast<uint2 *>(V + op_off(r, 0)) =
-                            make_uint2(pack_bf16(val[0], val[1]), pack_bf16(val[2], val[3]));
+                        // bf16 inputs: exact in one part (columns 0..3; 4..11 stay
+                        // zero), moved as raw 16-bit values
+                        const uint16_t *src = reinterpret_cast<const uint16_t *>(v < 4 ? Bs : Cs) + (v & 3) * kT + t;
+                        const uint32_t e0 = src[0], e1 = src[4 * kT], e2 = src[8 * kT], e3 = src[12 * kT];
+                        *reinterpret_cast<uint2 *>(V + op_off(r, 0)) = make_uint2(e0 | (e1 << 16), e2 | (e3 << 16));
                     } else {
                         // fp32 inputs: v = hi + mid + lo, each part bf16 (exact: 3 x 8 bits)
-                        float hi[4], mid[4], lo[4];
+                        float val[4], hi[4], mid[4], lo[4];
 #pragma unroll
                         for (int k4 = 0; k4 < 4; ++k4) {
+                            val[k4] = bc_value<TIn>(Bs, Cs, t, k4, v);
                             hi[k4] = __bfloat162float(__float2bfloat16_rn(val[k4]));
                             const float r1 = val[k4] - hi[k4];
                             mid[k4] = __bfloat162float(__float2bfloat16_rn(r1));
@@ -386,7 +388,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             __syncwarp();
             if (lane == 0) {
                 bar_arrive(bar(empty0 + s));  // this warp is done with the stage's B/C
-                // (3) D[vb] = S x V[vb]^T once the compute warps have read tile k - 2's columns
+                // (2) D[vb] = S x V[vb]^T once the compute warps have read tile k - 2's columns
                 if (k >= 2) ok = bar_wait(bar(tfree0 + vb), (uint32_t)(((k - 2) >> 1) & 1));
                 if (ok) {
                     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
@@ -406,7 +408,20 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 }
             }
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
-            if (ok) mmas = k + 1;
+            if (!ok) break;
+            mmas = k + 1;
+            // (3) loads of tile k + S - 1 into the stage tile k - 1 used, once
+            // every compute warp has read that tile's u, delta, z
+            const int kk = k + S - 1;
+            if (kk < ntiles) {
+                if (lane == 0) {
+                    if (kk >= S) ok = bar_wait(bar(empty0 + kk % S), (uint32_t)(((kk - S) / S) & 1));
+                    if (ok) issue(kk);
+                }
+                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+                if (!ok) break;
+                issued = kk + 1;
+            }
         }
         if (!ok && lane == 0) report_abort(a, abort_flag);
         // drain: loads issued but not consumed here, and the last MMAs
@@ -437,9 +452,9 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
         const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
         const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
         const bool sp = a.softplus != 0;
-        float *xd = reinterpret_cast<float *>(smem + lay.xch(warp));   // [8][kRow] Delta
+        float *xd = reinterpret_cast<float *>(smem + lay.xch(warp));   // [8][kRow] Delta (or the pairs)
         float *xu = xd + kCW * kRow;                                     // [8][kRow] Delta*u
-        float *pr = xu + kCW * kRow;                                     // [8*4][kRow] partial readouts
+        float *pr = xd + (SPLAT ? kCW * kRowS : 2 * kCW * kRow);         // [8*4][kRow] partial readouts
         TOut *y_row = static_cast<TOut *>(a.y) + b * a.y_sb + dd * a.y_sd;
         const uint32_t trow = (uint32_t)(32 * (warp & 3)) << 16;        // this warp's accumulator lanes
 
@@ -509,12 +524,18 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                         dsum_acc += dl[j];
                     }
                 }
-                float4 *pd = reinterpret_cast<float4 *>(xd + c * kRow + 8 * g);
-                float4 *pu = reinterpret_cast<float4 *>(xu + c * kRow + 8 * g);
-                pd[0] = make_float4(dl[0], dl[1], dl[2], dl[3]);
-                pd[1] = make_float4(dl[4], dl[5], dl[6], dl[7]);
-                pu[0] = make_float4(dlu[0], dlu[1], dlu[2], dlu[3]);
-                pu[1] = make_float4(dlu[4], dlu[5], dlu[6], dlu[7]);
+                if constexpr (SPLAT) {
+                    float4 *px = reinterpret_cast<float4 *>(xd + c * kRowS + 4 * (8 * g));
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) px[j] = make_float4(dl[j], dl[j], dlu[j], dlu[j]);
+                } else {
+                    float4 *pd = reinterpret_cast<float4 *>(xd + c * kRow + 8 * g);
+                    float4 *pu = reinterpret_cast<float4 *>(xu + c * kRow + 8 * g);
+                    pd[0] = make_float4(dl[0], dl[1], dl[2], dl[3]);
+                    pd[1] = make_float4(dl[4], dl[5], dl[6], dl[7]);
+                    pu[0] = make_float4(dlu[0], dlu[1], dlu[2], dlu[3]);
+                    pu[1] = make_float4(dlu[4], dlu[5], dlu[6], dlu[7]);
+                }
             }
             __syncwarp();
             // ---- the tile's B/C in tensor memory
@@ -526,19 +547,31 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             // group computes (two register sets, used alternately)
             const uint32_t tcol = tmem + trow + (uint32_t)(vb * kBufCols);
             uint32_t bcA[8 * TOK], bcB[8 * TOK];
-            float dlA[TOK], duA[TOK], dlB[TOK], duB[TOK];
-            auto fetch = [&](int j, uint32_t(&bc)[8 * TOK], float(&dl)[TOK], float(&du)[TOK]) {
+            f2 dlA[TOK], duA[TOK], dlB[TOK], duB[TOK];
+            auto fetch = [&](int j, uint32_t(&bc)[8 * TOK], f2(&dl)[TOK], f2(&du)[TOK]) {
                 MS_CHECK(a.status, vb * kBufCols + 8 * TOK * (j + 1) <= kTmemCols && 4 * c + g < 32);
                 tmem_ld<8 * TOK>(tcol + (uint32_t)(8 * TOK * j), bc);
-                lds_vec<TOK>(xd + c * kRow + TOK * j, dl);
-                lds_vec<TOK>(xu + c * kRow + TOK * j, du);
+                if constexpr (SPLAT) {
+                    // (Delta, Delta, Delta*u, Delta*u) per token: both pairs in one load
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) lds_f2x2(xd + c * kRowS + 4 * (TOK * j + t), dl[t], du[t]);
+                } else {
+                    float dls[TOK], dus[TOK];
+                    lds_vec<TOK>(xd + c * kRow + TOK * j, dls);
+                    lds_vec<TOK>(xu + c * kRow + TOK * j, dus);
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) {
+                        dl[t] = f2_splat(dls[t]);
+                        du[t] = f2_splat(dus[t]);
+                    }
+                }
             };
-            auto group = [&](int j, const uint32_t(&bc)[8 * TOK], const float(&dls)[TOK], const float(&dus)[TOK]) {
+            auto group = [&](int j, const uint32_t(&bc)[8 * TOK], const f2(&dl2s)[TOK], const f2(&du2s)[TOK]) {
                 float part[TOK];
 #pragma unroll
                 for (int t = 0; t < TOK; ++t) {
-                    const f2 dl2 = f2_splat(dls[t]);
-                    const f2 du2 = f2_splat(dus[t]);
+                    const f2 dl2 = dl2s[t];
+                    const f2 du2 = du2s[t];
                     f2 acc = 0ull;
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {

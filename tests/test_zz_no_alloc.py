@@ -46,7 +46,8 @@ def test_noalloc_matches_workspace_backward_twice(dtype, L):
                          f64(dout), h0=f64(h0), dlast=f64(dlast))
     for r in runs:
         for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"):
-            check(f64(r[k]), rr[k], dtype, f"noalloc vs oracle {k}")
+            # sums over batch rows, channels or tokens: the bf16 rule's absolute bound scales with their rms
+            check(f64(r[k]), rr[k], dtype, f"noalloc vs oracle {k}", scaled=k in ("dA", "dB", "dC", "dD", "ddelta_bias"))
         check(f64(r["dinitial_state"]), rr["dh0"], dtype, "noalloc vs oracle dinitial_state")
 
 

@@ -65,12 +65,33 @@ constexpr int kRow = 36;               // floats per padded exchange row (bank s
 constexpr int kRowS = 4 * 32 + 4;      // floats per padded row of splatted pairs
 constexpr int kTmemCols = 512;         // two buffers of 256 columns
 constexpr int kBufCols = 256;          // 32 tokens x 8 values
-// Bounded waits: a try may suspend the thread for up to kSuspendNs while the
-// phase is incomplete (it resumes as soon as the phase completes), so a
-// waiting warp issues a few instructions per microsecond instead of spinning;
-// kSpin tries bound a wait to well under a second.
+// Compile-time variants (measured; the defaults are the faster ones):
+//   MS_TMEM_SPLAT    1: Delta / Delta*u stored as splatted pairs (one 16-byte
+//                    load per token gives both f32x2 operands) in the 12-warp
+//                    variant; 0: plain rows, pairs formed in registers.
+//   MS_TMEM_SUSPEND  1: bounded waits pass a suspend-time hint to try_wait.
+//   MS_TMEM_MMA_FIRST 1: the producer issues a tile's product before the next
+//                    tile's loads; 0: loads first.
+#ifndef MS_TMEM_SPLAT
+#define MS_TMEM_SPLAT 0
+#endif
+#ifndef MS_TMEM_SUSPEND
+#define MS_TMEM_SUSPEND 0
+#endif
+#ifndef MS_TMEM_MMA_FIRST
+#define MS_TMEM_MMA_FIRST 0
+#endif
+//   MS_TMEM_SCALAR   1: the state loop in scalar fp32 (no register pairs to
+//                    form from the tensor-memory loads, no Delta splats);
+//                    0: packed f32x2 pairs.
+#ifndef MS_TMEM_SCALAR
+#define MS_TMEM_SCALAR 0
+#endif
+
+// Bounded waits: kSpin tries of mbarrier.try_wait (each may suspend the
+// thread for a system-dependent time, or up to kSuspendNs with the hint).
 constexpr uint32_t kSuspendNs = 20000;
-constexpr uint32_t kSpin = 1u << 15;
+constexpr uint32_t kSpin = MS_TMEM_SUSPEND ? (1u << 15) : (1u << 20);
 
 // Shared memory layout for W compute warps and S stages (host and device).
 struct TmLayout {
@@ -88,7 +109,7 @@ struct TmLayout {
     // per-warp exchange: Delta and Delta*u (as splatted pairs (Delta, Delta,
     // Delta*u, Delta*u) per token in the 12-warp instantiation, else two
     // plain rows), then the partial readouts [8 channels x 4 lanes][kRow]
-    __host__ __device__ bool splat() const { return W <= 11; }
+    __host__ __device__ bool splat() const { return MS_TMEM_SPLAT && !MS_TMEM_SCALAR && W <= 11; }
     __host__ __device__ int xch_bytes() const {
         return ((splat() ? kCW * kRowS : 2 * kCW * kRow) + kCW * 4 * kRow) * 4;
     }
@@ -116,7 +137,11 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
+#if MS_TMEM_SUSPEND
             "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+#else
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+#endif
             "selp.u32 %0, 1, 0, p;\n\t}"
             : "=r"(done)
             : "r"(bar), "r"(parity), "r"(kSuspendNs)
@@ -253,7 +278,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
     // tokens per tensor-memory load: 4 (32 columns) where registers allow two
     // such sets without spilling, 2 (16 columns) in the larger instantiations
     constexpr int TOK = MAXW <= 11 ? 4 : 2;
-    constexpr bool SPLAT = MAXW <= 11;  // matches TmLayout::splat()
+    constexpr bool SPLAT = MS_TMEM_SPLAT && !MS_TMEM_SCALAR && MAXW <= 11;  // matches TmLayout::splat()
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int cwc = lay.cwc();
@@ -341,8 +366,27 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
         int mmas = 0;      // MMAs issued
         int consumed = 0;  // tiles whose full barrier this warp has passed
         bool ok = true;
+        // loads of tile k + S - 1 into the stage tile k - 1 used, once every
+        // compute warp has read that tile's u, delta, z
+        auto prefetch = [&](int k) -> bool {
+            bool good = true;
+            const int kk = k + S - 1;
+            if (kk < ntiles) {
+                if (lane == 0) {
+                    if (kk >= S) good = bar_wait(bar(empty0 + kk % S), (uint32_t)(((kk - S) / S) & 1));
+                    if (good) issue(kk);
+                }
+                good = __shfl_sync(0xffffffffu, good ? 1 : 0, 0) != 0;
+                if (good) issued = kk + 1;
+            }
+            return good;
+        };
         for (int k = 0; k < ntiles && ok; ++k) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            if (!MS_TMEM_MMA_FIRST) {
+                ok = prefetch(k);
+                if (!ok) break;
+            }
             // (1) tile k's B/C -> V[k % 2], once MMA k - 2 has finished reading it
             const int s = k % S, vb = k & 1;
             ok = bar_wait(bar(full0 + s), (uint32_t)((k / S) & 1));
@@ -410,17 +454,9 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
             if (!ok) break;
             mmas = k + 1;
-            // (3) loads of tile k + S - 1 into the stage tile k - 1 used, once
-            // every compute warp has read that tile's u, delta, z
-            const int kk = k + S - 1;
-            if (kk < ntiles) {
-                if (lane == 0) {
-                    if (kk >= S) ok = bar_wait(bar(empty0 + kk % S), (uint32_t)(((kk - S) / S) & 1));
-                    if (ok) issue(kk);
-                }
-                ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+            if (MS_TMEM_MMA_FIRST) {
+                ok = prefetch(k);
                 if (!ok) break;
-                issued = kk + 1;
             }
         }
         if (!ok && lane == 0) report_abort(a, abort_flag);
@@ -568,6 +604,34 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             };
             auto group = [&](int j, const uint32_t(&bc)[8 * TOK], const f2(&dl2s)[TOK], const f2(&du2s)[TOK]) {
                 float part[TOK];
+                if constexpr (MS_TMEM_SCALAR) {
+                    // the pairs hold (Delta, Delta) and (Delta*u, Delta*u): use one half
+                    float hs[4], As[4];
+                    f2_split(h[0], hs[0], hs[1]);
+                    f2_split(h[1], hs[2], hs[3]);
+                    f2_split(A2[0], As[0], As[1]);
+                    f2_split(A2[1], As[2], As[3]);
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) {
+                        float dl, du, unused;
+                        f2_split(dl2s[t], dl, unused);
+                        f2_split(du2s[t], du, unused);
+                        float acc = 0.0f;
+#pragma unroll
+                        for (int n = 0; n < 4; ++n) {
+                            const float x = As[n] * dl;
+                            const bool poly = (2 * ((TOK * j + t) & 3) + (n >> 1)) < POLY8;
+                            const float ab = poly ? exp2_poly(x) : exp2_mufu(x);
+                            hs[n] = fmaf(ab, hs[n], du * __uint_as_float(bc[8 * t + n]));
+                            if constexpr (YOUT) acc = fmaf(__uint_as_float(bc[8 * t + 4 + n]), hs[n], acc);
+                        }
+                        part[t] = acc;
+                    }
+                    h[0] = f2_make(hs[0], hs[1]);
+                    h[1] = f2_make(hs[2], hs[3]);
+                    if constexpr (YOUT) sts_vec<TOK>(pr + (c * 4 + g) * kRow + TOK * j, part);
+                    return;
+                }
 #pragma unroll
                 for (int t = 0; t < TOK; ++t) {
                     const f2 dl2 = dl2s[t];

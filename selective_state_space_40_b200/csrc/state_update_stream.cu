@@ -6,10 +6,13 @@
 // the same model), organised for HBM streaming: a persistent CTA walks tiles
 // of kTC consecutive channels of one batch row. The tile's state rows (kTC x 64
 // bytes) and its x, delta, z values arrive by bulk copies (TMA engine) into a
-// ring of kStages shared-memory stages tracked by mbarriers; the threads update
-// the state in place in shared memory; bulk copies write the state and y back.
-// Loads run up to kStages - 1 tiles ahead, so the copy engine, not the
-// threads, keeps the HBM requests in flight. No cluster multicast is used.
+// ring of kStages shared-memory stages tracked by mbarriers; the compute
+// threads update the state in place in shared memory; a producer warp writes
+// the state and y back by bulk copies once every compute warp is done with a
+// stage, and refills the stage once those stores have read it. Loads run up
+// to kStages tiles ahead, so the copy engine, not the threads, keeps the HBM
+// requests in flight, and no compute thread waits on the store path. No
+// cluster multicast is used.
 //
 // Used when the state rows are dense (16 fp32 per channel, 16-byte aligned),
 // d_state is 16, dim is a multiple of kTC and every row start is 16-byte
@@ -35,10 +38,11 @@ namespace {
 #ifndef MS_STREAM_STAGES
 #define MS_STREAM_STAGES 4
 #endif
-constexpr int kTC = MS_STREAM_TC;            // channels per tile
-constexpr int kThreads = MS_STREAM_THREADS;  // 4 lanes per channel
+constexpr int kTC = MS_STREAM_TC;                    // channels per tile
+constexpr int kComputeThreads = MS_STREAM_THREADS;   // 4 lanes per channel
+constexpr int kThreads = kComputeThreads + 32;       // + one producer warp
 constexpr int kStages = MS_STREAM_STAGES;
-static_assert(kTC * 4 % kThreads == 0, "whole channels per pass");
+static_assert(kTC * 4 % kComputeThreads == 0, "whole channels per pass");
 constexpr uint32_t kSpinLimit = 1u << 20;  // try_wait rounds before giving up
 
 __device__ __forceinline__ uint32_t saddr(const void *p) {
@@ -46,6 +50,9 @@ __device__ __forceinline__ uint32_t saddr(const void *p) {
 }
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(saddr(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(saddr(bar)) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(saddr(bar)), "r"(bytes)
@@ -99,7 +106,7 @@ struct StreamSmem {
     static constexpr int kInBytes = kTC * (int)sizeof(TIn);
     static constexpr int kYBytes = kTC * (int)sizeof(TOut);
     static constexpr int kStageBytes = kStateBytes + 3 * kInBytes + ((kYBytes + 15) & ~15);
-    static constexpr int kOffStages = 128;  // mbarriers first
+    static constexpr int kOffStages = 128;  // mbarriers first (full[kStages], done[kStages])
     static constexpr int kTotal = kOffStages + kStages * kStageBytes;
 };
 
@@ -108,12 +115,17 @@ __global__ void __launch_bounds__(kThreads)
 state_update_stream_kernel(const UpdateArgs a) {
     using Sm = StreamSmem<TIn, TOut>;
     extern __shared__ __align__(128) unsigned char smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // stage s loaded
+    uint64_t *done = full + kStages;                       // stage s computed (one arrival per compute warp)
     auto stage = [&](int s) { return smem + Sm::kOffStages + s * Sm::kStageBytes; };
 
     const int64_t tiles_per_row = a.dim / kTC;
     const int64_t ntiles = a.batch * tiles_per_row;
+    // this CTA's tiles: blockIdx.x, blockIdx.x + gridDim.x, ...
+    const int64_t my_tiles = blockIdx.x < ntiles ? (ntiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    auto tile_of = [&](int64_t i) { return (int64_t)blockIdx.x + i * (int64_t)gridDim.x; };
     const bool has_z = a.z != nullptr;
+    const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
     const int q = lane & 3;        // states 4q..4q+3
     const int n0 = 4 * q;
@@ -136,7 +148,10 @@ state_update_stream_kernel(const UpdateArgs a) {
     };
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&done[s], kComputeThreads / 32);
+        }
         fence_mbar_init();
     }
     // Back-to-back steps: this grid may have been launched while the previous
@@ -147,33 +162,52 @@ state_update_stream_kernel(const UpdateArgs a) {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
     __syncthreads();
-    // Prologue: the first kStages - 1 tiles of this CTA.
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages - 1; ++s) {
-            const int64_t tile = blockIdx.x + (int64_t)s * gridDim.x;
-            if (tile < ntiles) issue(s, tile);
+
+    if (warp == kComputeThreads / 32) {
+        // ---- producer warp (lane 0): loads run kStages tiles ahead; a tile's
+        // state and y go back by bulk stores once every compute warp is done
+        // with it, and its stage is refilled once those stores have read it.
+        if (lane == 0) {
+            int64_t issued = 0, stored = 0;
+            for (; issued < kStages && issued < my_tiles; ++issued) issue((int)issued, tile_of(issued));
+            bool ok = true;
+            for (int64_t i = 0; i < my_tiles; ++i) {
+                const int s = (int)(i % kStages);
+                ok = mbar_wait(&done[s], (uint32_t)((i / kStages) & 1));
+                if (!ok) break;
+                const int64_t tile = tile_of(i);
+                const int64_t b = tile / tiles_per_row;
+                const int64_t d0 = (tile % tiles_per_row) * kTC;
+                unsigned char *st = stage(s);
+                bulk_store(a.state + b * a.st_sb + d0 * 16, st, Sm::kStateBytes);
+                bulk_store(static_cast<TOut *>(a.y) + b * a.y_sb + d0, st + Sm::kStateBytes + 3 * Sm::kInBytes,
+                           Sm::kYBytes);
+                bulk_commit();
+                stored = i + 1;
+                if (issued < my_tiles) {
+                    bulk_wait_read<0>();  // this stage's stores have read it
+                    issue(s, tile_of(issued));
+                    ++issued;
+                }
+            }
+            if (!ok) {
+                if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+                // Drain (bounded) the loads this CTA may still have in flight.
+                for (int64_t k = stored; k < issued; ++k)
+                    mbar_wait(&full[k % kStages], (uint32_t)((k / kStages) & 1));
+            }
+            bulk_wait_all();
         }
+        return;
     }
 
-    bool failed = false;
-    int64_t i = 0;
-    for (int64_t tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++i) {
+    // ---- compute warps: 4 lanes per channel, 4 states each
+    for (int64_t i = 0; i < my_tiles; ++i) {
         const int s = (int)(i % kStages);
-        const bool ok = mbar_wait(&full[s], (uint32_t)((i / kStages) & 1));
-        if (__syncthreads_or(!ok)) {  // one decision for the whole CTA
-            failed = true;
-            break;
-        }
+        const int64_t tile = tile_of(i);
         const int64_t b = tile / tiles_per_row;
         const int64_t d0 = (tile % tiles_per_row) * kTC;
-        unsigned char *st = stage(s);
-        float *sstate = reinterpret_cast<float *>(st);
-        const TIn *sx = reinterpret_cast<const TIn *>(st + Sm::kStateBytes);
-        const TIn *sdl = sx + kTC;
-        const TIn *sz = sdl + kTC;
-        TOut *sy = reinterpret_cast<TOut *>(st + Sm::kStateBytes + 3 * Sm::kInBytes);
-
-        // B and C of this batch row (4 states of this quad lane).
+        // the tile's parameters (global, L2-resident) load while the stage may still be in flight
         float Bv[4], Cv[4];
         {
             const TIn *Bb = static_cast<const TIn *>(a.B) + b * a.B_sb + n0;
@@ -184,17 +218,37 @@ state_update_stream_kernel(const UpdateArgs a) {
                 Cv[k] = Elem<TIn>::load(Cb + k);
             }
         }
+        constexpr int kHalves = kTC * 4 / kComputeThreads;
+        float4 Av[kHalves];
+        float biasv[kHalves], Dv[kHalves];
 #pragma unroll
-        for (int half = 0; half < kTC * 4 / kThreads; ++half) {
-            const int cl = (threadIdx.x >> 2) + half * (kThreads / 4);  // channel within the tile
+        for (int half = 0; half < kHalves; ++half) {
+            const int64_t d = d0 + (threadIdx.x >> 2) + half * (kComputeThreads / 4);
+            Av[half] = __ldg(reinterpret_cast<const float4 *>(a.A + d * 16 + n0));
+            biasv[half] = a.bias ? __ldg(a.bias + d) : 0.0f;
+            Dv[half] = a.D ? __ldg(a.D + d) : 0.0f;
+        }
+        const bool ok = __all_sync(0xffffffffu, mbar_wait(&full[s], (uint32_t)((i / kStages) & 1)));
+        if (!ok) {
+            if (lane == 0 && a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+            break;
+        }
+        unsigned char *st = stage(s);
+        float *sstate = reinterpret_cast<float *>(st);
+        const TIn *sx = reinterpret_cast<const TIn *>(st + Sm::kStateBytes);
+        const TIn *sdl = sx + kTC;
+        const TIn *sz = sdl + kTC;
+        TOut *sy = reinterpret_cast<TOut *>(st + Sm::kStateBytes + 3 * Sm::kInBytes);
+#pragma unroll
+        for (int half = 0; half < kHalves; ++half) {
+            const int cl = (threadIdx.x >> 2) + half * (kComputeThreads / 4);  // channel within the tile
             const int64_t d = d0 + cl;
             if (!MS_CHECK(a.status, cl < kTC && d < a.dim)) continue;
             float4 hv = *reinterpret_cast<const float4 *>(sstate + cl * 16 + n0);
             float h[4] = {hv.x, hv.y, hv.z, hv.w};
-            const float4 Av = __ldg(reinterpret_cast<const float4 *>(a.A + d * 16 + n0));
-            const float A[4] = {Av.x, Av.y, Av.z, Av.w};
+            const float A[4] = {Av[half].x, Av[half].y, Av[half].z, Av[half].w};
             const float x = to_f32(sx[cl]);
-            const float v = to_f32(sdl[cl]) + (a.bias ? __ldg(a.bias + d) : 0.0f);
+            const float v = to_f32(sdl[cl]) + biasv[half];
             const float dt = a.softplus ? softplus_f(v) : v;
             const float dx = dt * x;
             const float dtl = dt * kLog2e;
@@ -208,37 +262,14 @@ state_update_stream_kernel(const UpdateArgs a) {
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             *reinterpret_cast<float4 *>(sstate + cl * 16 + n0) = make_float4(h[0], h[1], h[2], h[3]);
             if (q == 0) {
-                float yv = acc + (a.D ? __ldg(a.D + d) : 0.0f) * x;
+                float yv = acc + Dv[half] * x;
                 if (has_z) yv *= silu_f(to_f32(sz[cl]));
                 Elem<TOut>::store(sy + cl, yv);
             }
         }
         fence_proxy_async();  // this thread's shared writes -> visible to the copy engine
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            bulk_store(a.state + b * a.st_sb + d0 * 16, sstate, Sm::kStateBytes);
-            bulk_store(static_cast<TOut *>(a.y) + b * a.y_sb + d0, sy, Sm::kYBytes);
-            bulk_commit();
-            // Refill the stage freed by the previous tile once its stores
-            // have finished reading it.
-            const int64_t next = tile + (int64_t)(kStages - 1) * gridDim.x;
-            if (next < ntiles) {
-                bulk_wait_read<1>();
-                issue((int)((i + kStages - 1) % kStages), next);
-            }
-        }
-    }
-
-    if (threadIdx.x == 0) {
-        if (failed) {
-            if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
-            // Drain (bounded) the loads this CTA may still have in flight.
-            for (int k = 1; k < kStages; ++k) {
-                const int64_t tile = blockIdx.x + (i + k - 1) * (int64_t)gridDim.x;
-                if (tile < ntiles) mbar_wait(&full[(i + k - 1) % kStages], (uint32_t)(((i + k - 1) / kStages) & 1));
-            }
-        }
-        bulk_wait_all();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&done[s]);
     }
 }
 

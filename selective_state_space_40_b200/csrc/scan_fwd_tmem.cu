@@ -87,6 +87,23 @@ constexpr int kBufCols = 256;          // 32 tokens x 8 values
 #ifndef MS_TMEM_SCALAR
 #define MS_TMEM_SCALAR 0
 #endif
+//   MS_TMEM_DB       1: the next group's tensor-memory load in flight while a
+//                    group computes (4-token loads in the 12-warp variant,
+//                    2-token loads in the larger ones); 0: one 4-token load
+//                    per group, waited for at once.
+#ifndef MS_TMEM_DB
+#define MS_TMEM_DB 0
+#endif
+//   MS_TMEM_FUSED    1: in the 12-warp variant, the next tile's per-token
+//                    quantities (Delta, Delta*u, silu(z), D*u*silu(z)) are
+//                    computed inside the current tile's state loop, one
+//                    token of the lane's chunk per group of 4 tokens, so
+//                    their chains interleave with the recurrence and the
+//                    MUFU work is spread over the tile; 0: a separate
+//                    prologue per tile.
+#ifndef MS_TMEM_FUSED
+#define MS_TMEM_FUSED 1
+#endif
 
 // Bounded waits: kSpin tries of mbarrier.try_wait (each may suspend the
 // thread for a system-dependent time, or up to kSuspendNs with the hint).
@@ -176,6 +193,22 @@ constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(256
 // Byte offset of row r (16-byte piece kc of K) in a K-major no-swizzle tile
 // with 16 K elements: core matrix (r / 8, kc) at ((r / 8) * 2 + kc) * 128.
 __device__ __forceinline__ int op_off(int r, int kc) { return (((r >> 3) * 2 + kc) * 8 + (r & 7)) * 16; }
+
+// 32 consecutive tensor-memory columns, loaded and waited for in one asm
+// statement: where registers are short (the larger instantiations spill a
+// few values) nothing can be spilled while the load is still in flight.
+__device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
+          "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+          "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
+        : "r"(taddr)
+        : "memory");
+}
 
 // 16 consecutive tensor-memory columns of this warp's 32 lanes.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
@@ -277,7 +310,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
     extern __shared__ __align__(1024) unsigned char smem[];
     // tokens per tensor-memory load: 4 (32 columns) where registers allow two
     // such sets without spilling, 2 (16 columns) in the larger instantiations
-    constexpr int TOK = MAXW <= 11 ? 4 : 2;
+    constexpr int TOK = (MAXW <= 11 || !MS_TMEM_DB) ? 4 : 2;
     constexpr bool SPLAT = MS_TMEM_SPLAT && !MS_TMEM_SCALAR && MAXW <= 11;  // matches TmLayout::splat()
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -496,7 +529,175 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
 
         bool ok = true;
         float dsum_acc = 0.0f;  // this lane's tokens' Delta (first pass of a split)
-        for (int k = 0; k < ntiles; ++k) {
+        constexpr bool FUSED = MS_TMEM_FUSED && YOUT && MAXW <= 11 && !SPLAT && !MS_TMEM_SCALAR && TOK == 4;
+        if constexpr (FUSED) {
+            constexpr int kWords = 8 * (int)sizeof(TIn) / 4;  // one 8-token chunk in 32-bit words
+            // raw inputs of chunk g of channel c from a stage, as stored
+            auto load_raw = [&](int k, uint32_t(&uw)[kWords], uint32_t(&dw)[kWords], uint32_t(&zw)[kWords]) {
+                const unsigned char *st = smem + lay.stage(k % S);
+                int off = (cc * kT + 8 * g) * (int)sizeof(TIn);
+                if (!MS_CHECK(a.status, off + 8 * (int)sizeof(TIn) <= (int)chan_bytes && cc < cwc)) off = 0;
+#pragma unroll
+                for (int q = 0; q < kWords / 4; ++q) {
+                    const uint4 U = *reinterpret_cast<const uint4 *>(st + off + 16 * q);
+                    const uint4 Dl = *reinterpret_cast<const uint4 *>(st + chan_bytes + off + 16 * q);
+                    uw[4 * q] = U.x; uw[4 * q + 1] = U.y; uw[4 * q + 2] = U.z; uw[4 * q + 3] = U.w;
+                    dw[4 * q] = Dl.x; dw[4 * q + 1] = Dl.y; dw[4 * q + 2] = Dl.z; dw[4 * q + 3] = Dl.w;
+                    if (has_z) {
+                        const uint4 Z = *reinterpret_cast<const uint4 *>(st + 2 * chan_bytes + off + 16 * q);
+                        zw[4 * q] = Z.x; zw[4 * q + 1] = Z.y; zw[4 * q + 2] = Z.z; zw[4 * q + 3] = Z.w;
+                    } else {
+                        zw[4 * q] = zw[4 * q + 1] = zw[4 * q + 2] = zw[4 * q + 3] = 0u;
+                    }
+                }
+            };
+            auto elem = [&](const uint32_t(&w)[kWords], int j) -> float {
+                if constexpr (sizeof(TIn) == 4) return __uint_as_float(w[j]);
+                else return (j & 1) ? bf16_hi(w[j >> 1]) : bf16_lo(w[j >> 1]);
+            };
+            // token j of the chunk: Delta, Delta*u, silu(z), D*u*silu(z)
+            auto prol = [&](const uint32_t(&uw)[kWords], const uint32_t(&dw)[kWords], const uint32_t(&zw)[kWords],
+                            int j, bool live, float &dl, float &dlu, float &gate, float &dug) {
+                const float u = elem(uw, j);
+                const float v = elem(dw, j) + bias;
+                dl = live ? (sp ? softplus_f(v) : v) : 0.0f;  // past the end: the state is left alone
+                dlu = dl * u;
+                gate = has_z ? silu_f(elem(zw, j)) : 1.0f;
+                dug = Dd * u * gate;
+            };
+            auto write_x = [&](const float(&dl)[8], const float(&dlu)[8]) {
+                float4 *pd = reinterpret_cast<float4 *>(xd + c * kRow + 8 * g);
+                float4 *pu = reinterpret_cast<float4 *>(xu + c * kRow + 8 * g);
+                pd[0] = make_float4(dl[0], dl[1], dl[2], dl[3]);
+                pd[1] = make_float4(dl[4], dl[5], dl[6], dl[7]);
+                pu[0] = make_float4(dlu[0], dlu[1], dlu[2], dlu[3]);
+                pu[1] = make_float4(dlu[4], dlu[5], dlu[6], dlu[7]);
+            };
+            float gate[8], dug[8];  // the current tile's chunk
+            uint32_t uw[kWords], dw[kWords], zw[kWords];
+            if (ntiles > 0) {
+                ok = __all_sync(0xffffffffu, bar_wait(bar(full0), 0u));
+                if (ok) {
+                    load_raw(0, uw, dw, zw);
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(bar(empty0));  // this warp is done with stage 0
+                    float dl[8], dlu[8];
+                    const bool live = 8 * g < L;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) prol(uw, dw, zw, j, live, dl[j], dlu[j], gate[j], dug[j]);
+                    write_x(dl, dlu);
+                    __syncwarp();
+                }
+            }
+            for (int k = 0; k < ntiles && ok; ++k) {
+                if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+                const int vb = k & 1;
+                const int64_t t0 = (int64_t)k * kT;
+                const bool has_next = k + 1 < ntiles;
+                const bool live_next = t0 + kT + 8 * g < L;
+                // the next tile's raw inputs, into registers; its stage is then free
+                if (has_next) {
+                    ok = __all_sync(0xffffffffu, bar_wait(bar(full0 + (k + 1) % S), (uint32_t)(((k + 1) / S) & 1)));
+                    if (!ok) break;
+                    load_raw(k + 1, uw, dw, zw);
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(bar(empty0 + (k + 1) % S));
+                }
+                ok = __all_sync(0xffffffffu, bar_wait(bar(mma0 + vb), (uint32_t)((k >> 1) & 1)));
+                if (!ok) break;
+                asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+                const uint32_t tcol = tmem + trow + (uint32_t)(vb * kBufCols);
+                float dln[8], dlun[8], gaten[8], dugn[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    uint32_t bc[32];
+                    MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                    tmem_ld32(tcol + (uint32_t)(32 * j), bc);
+                    const float4 dl4 = *reinterpret_cast<const float4 *>(xd + c * kRow + 4 * j);
+                    const float4 du4 = *reinterpret_cast<const float4 *>(xu + c * kRow + 4 * j);
+                    // the next tile's token j (independent of this group's chains)
+                    if (has_next) prol(uw, dw, zw, j, live_next, dln[j], dlun[j], gaten[j], dugn[j]);
+                    tmem_wait(bc);
+                    const float dls[4] = {dl4.x, dl4.y, dl4.z, dl4.w};
+                    const float dus[4] = {du4.x, du4.y, du4.z, du4.w};
+                    float part[4];
+#pragma unroll
+                    for (int t = 0; t < 4; ++t) {
+                        const f2 dl2 = f2_splat(dls[t]);
+                        const f2 du2 = f2_splat(dus[t]);
+                        f2 acc = 0ull;
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            const f2 Bp = f2_make(__uint_as_float(bc[8 * t + 2 * p]), __uint_as_float(bc[8 * t + 2 * p + 1]));
+                            const f2 Cp = f2_make(__uint_as_float(bc[8 * t + 4 + 2 * p]), __uint_as_float(bc[8 * t + 5 + 2 * p]));
+                            const f2 x = f2_mul(A2[p], dl2);
+                            const bool poly = (2 * t + p) < POLY8;
+                            f2 ab;
+                            if (poly) {
+                                ab = exp2_poly2(x);
+                            } else {
+                                float xa, xb;
+                                f2_split(x, xa, xb);
+                                ab = f2_make(exp2_mufu(xa), exp2_mufu(xb));
+                            }
+                            h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp));
+                            acc = p == 0 ? f2_mul(Cp, h[p]) : f2_fma(Cp, h[p], acc);
+                        }
+                        float lo, hi;
+                        f2_split(acc, lo, hi);
+                        part[t] = lo + hi;
+                    }
+                    *reinterpret_cast<float4 *>(pr + (c * 4 + g) * kRow + 4 * j) =
+                        make_float4(part[0], part[1], part[2], part[3]);
+                }
+                // tensor-memory buffer vb is read: release it to the producer
+                asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+                __syncwarp();
+                if (lane == 0) bar_arrive(bar(tfree0 + vb));
+                // ---- epilogue of this tile: chunk g of channel c
+                float ys[8];
+                {
+                    const float4 *p0 = reinterpret_cast<const float4 *>(pr + (c * 4) * kRow + 8 * g);
+                    float4 a0 = p0[0], a1 = p0[1];
+#pragma unroll
+                    for (int q = 1; q < 4; ++q) {
+                        const float4 *pq = reinterpret_cast<const float4 *>(pr + (c * 4 + q) * kRow + 8 * g);
+                        const float4 b0 = pq[0], b1 = pq[1];
+                        a0.x += b0.x; a0.y += b0.y; a0.z += b0.z; a0.w += b0.w;
+                        a1.x += b1.x; a1.y += b1.y; a1.z += b1.z; a1.w += b1.w;
+                    }
+                    ys[0] = a0.x; ys[1] = a0.y; ys[2] = a0.z; ys[3] = a0.w;
+                    ys[4] = a1.x; ys[5] = a1.y; ys[6] = a1.z; ys[7] = a1.w;
+                }
+                const bool live = t0 + 8 * g < L;
+                if (active && live && MS_CHECK(a.status, t0 + 8 * g + 8 <= L && d < a.dim)) {
+                    float yo[8];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) yo[j] = fmaf(ys[j], gate[j], dug[j]);
+                    TOut *yp = y_row + t0 + 8 * g;
+                    if constexpr (sizeof(TOut) == 4) {
+                        float4 *pp = reinterpret_cast<float4 *>(yp);
+                        __stcs(pp, make_float4(yo[0], yo[1], yo[2], yo[3]));
+                        __stcs(pp + 1, make_float4(yo[4], yo[5], yo[6], yo[7]));
+                    } else {
+                        __stcs(reinterpret_cast<uint4 *>(yp), make_uint4(pack_bf16(yo[0], yo[1]), pack_bf16(yo[2], yo[3]),
+                                                                         pack_bf16(yo[4], yo[5]), pack_bf16(yo[6], yo[7])));
+                    }
+                }
+                // every lane is past this tile's Delta rows and partials
+                __syncwarp();
+                if (has_next) {
+                    write_x(dln, dlun);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        gate[j] = gaten[j];
+                        dug[j] = dugn[j];
+                    }
+                    __syncwarp();
+                }
+            }
+        }
+        for (int k = 0; k < ntiles && !FUSED; ++k) {
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const int s = k % S, vb = k & 1;
             const int64_t t0 = (int64_t)k * kT;
@@ -666,6 +867,23 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 if constexpr (YOUT) sts_vec<TOK>(pr + (c * 4 + g) * kRow + TOK * j, part);
             };
             constexpr int NG = kT / TOK;
+            if constexpr (!MS_TMEM_DB) {
+#pragma unroll 1
+                for (int j = 0; j < NG; ++j) {
+                    static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
+                    MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                    float dls[TOK], dus[TOK];
+                    lds_vec<TOK>(xd + c * kRow + TOK * j, dls);
+                    lds_vec<TOK>(xu + c * kRow + TOK * j, dus);
+                    tmem_ld32_sync(tcol + (uint32_t)(32 * j), bcA);
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) {
+                        dlA[t] = f2_splat(dls[t]);
+                        duA[t] = f2_splat(dus[t]);
+                    }
+                    group(j, bcA, dlA, duA);
+                }
+            } else {
             fetch(0, bcA, dlA, duA);
             tmem_wait<8 * TOK>(bcA);
 #pragma unroll 1
@@ -676,6 +894,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 if (j + 2 < NG) fetch(j + 2, bcA, dlA, duA);
                 group(j + 1, bcB, dlB, duB);
                 if (j + 2 < NG) tmem_wait<8 * TOK>(bcA);
+            }
             }
             // tensor-memory buffer vb is read: release it to the producer
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");

@@ -112,7 +112,12 @@ NOMINAL_HBM_GBS = 8000.0
 _SHARED_SOURCES = ("selective_state_space_40_b200/csrc/ms_device.cuh", "selective_state_space_40_b200/csrc/ms_internal.h",
                    "selective_state_space_40_b200/csrc/mambascan_api.cu", "include/mambascan.h")
 KERNEL_SOURCES = {
-    "scan_fwd_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
+    "scan_fwd_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",
+                      "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
+    "scan_fwd_2p8b": ("selective_state_space_40_b200/csrc/scan_fwd.cu",
+                      "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
+    "scan_fwd_long": ("selective_state_space_40_b200/csrc/scan_fwd.cu",
+                      "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
     "conv_scan_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
     "decode_step": ("selective_state_space_40_b200/csrc/state_update_stream.cu",),
     "scan_bwd_130m": ("selective_state_space_40_b200/csrc/scan_bwd.cu",),

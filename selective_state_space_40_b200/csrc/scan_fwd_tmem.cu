@@ -102,8 +102,31 @@ constexpr int kBufCols = 256;          // 32 tokens x 8 values
 //                    MUFU work is spread over the tile; 0: a separate
 //                    prologue per tile.
 #ifndef MS_TMEM_FUSED
-#define MS_TMEM_FUSED 1
+#define MS_TMEM_FUSED 0
 #endif
+//   MS_TMEM_UNROLL   groups of 4 tokens unrolled together in the state loop
+//                    of the kernels that write y (8 = the whole tile in one
+//                    basic block); the y-less pass keeps the loop rolled.
+#ifndef MS_TMEM_UNROLL
+#define MS_TMEM_UNROLL 8
+#endif
+//   MS_TMEM_LD64     1: in the 12-warp variant one 64-column load (two groups
+//                    of 4 tokens) per wait; 0: one 32-column load per group.
+#ifndef MS_TMEM_LD64
+#define MS_TMEM_LD64 1
+#endif
+//   MS_TMEM_LDCLOB   1: the combined load-and-wait is a compiler memory
+//                    barrier; 0: it only defines its registers (shared
+//                    loads of later groups may move above it).
+#ifndef MS_TMEM_LDCLOB
+#define MS_TMEM_LDCLOB 1
+#endif
+#if MS_TMEM_LDCLOB
+#define MS_TMEM_LD_CLOBBER : "memory"
+#else
+#define MS_TMEM_LD_CLOBBER
+#endif
+constexpr int kUnrollGroups = MS_TMEM_UNROLL;
 
 // Bounded waits: kSpin tries of mbarrier.try_wait (each may suspend the
 // thread for a system-dependent time, or up to kSuspendNs with the hint).
@@ -206,8 +229,17 @@ __device__ __forceinline__ void tmem_ld32_sync(uint32_t taddr, uint32_t (&v)[32]
           "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),
           "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
           "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
-        : "r"(taddr)
-        : "memory");
+        : "r"(taddr) MS_TMEM_LD_CLOBBER);
+}
+
+// 64 consecutive tensor-memory columns of this warp's 32 lanes, waited for in
+// the same statement.
+__device__ __forceinline__ void tmem_ld64_sync(uint32_t taddr, uint32_t (&v)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31]), "=r"(v[32]), "=r"(v[33]), "=r"(v[34]), "=r"(v[35]), "=r"(v[36]), "=r"(v[37]), "=r"(v[38]), "=r"(v[39]), "=r"(v[40]), "=r"(v[41]), "=r"(v[42]), "=r"(v[43]), "=r"(v[44]), "=r"(v[45]), "=r"(v[46]), "=r"(v[47]), "=r"(v[48]), "=r"(v[49]), "=r"(v[50]), "=r"(v[51]), "=r"(v[52]), "=r"(v[53]), "=r"(v[54]), "=r"(v[55]), "=r"(v[56]), "=r"(v[57]), "=r"(v[58]), "=r"(v[59]), "=r"(v[60]), "=r"(v[61]), "=r"(v[62]), "=r"(v[63])
+        : "r"(taddr) MS_TMEM_LD_CLOBBER);
 }
 
 // 16 consecutive tensor-memory columns of this warp's 32 lanes.
@@ -371,7 +403,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
     {
         uint32_t dyn;
         asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
-        MS_CHECK(a.status, (uint32_t)lay.total() <= dyn && W >= 1 && W <= MAXW && S >= 2 && (int)blockDim.x == 32 * (W + 1));
+        (void)MS_CHECK(a.status, (uint32_t)lay.total() <= dyn && W >= 1 && W <= MAXW && S >= 2 && (int)blockDim.x == 32 * (W + 1));
     }
 #endif
 
@@ -611,7 +643,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     uint32_t bc[32];
-                    MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                    (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
                     tmem_ld32(tcol + (uint32_t)(32 * j), bc);
                     const float4 dl4 = *reinterpret_cast<const float4 *>(xd + c * kRow + 4 * j);
                     const float4 du4 = *reinterpret_cast<const float4 *>(xu + c * kRow + 4 * j);
@@ -786,7 +818,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             uint32_t bcA[8 * TOK], bcB[8 * TOK];
             f2 dlA[TOK], duA[TOK], dlB[TOK], duB[TOK];
             auto fetch = [&](int j, uint32_t(&bc)[8 * TOK], f2(&dl)[TOK], f2(&du)[TOK]) {
-                MS_CHECK(a.status, vb * kBufCols + 8 * TOK * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                (void)MS_CHECK(a.status, vb * kBufCols + 8 * TOK * (j + 1) <= kTmemCols && 4 * c + g < 32);
                 tmem_ld<8 * TOK>(tcol + (uint32_t)(8 * TOK * j), bc);
                 if constexpr (SPLAT) {
                     // (Delta, Delta, Delta*u, Delta*u) per token: both pairs in one load
@@ -867,11 +899,35 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 if constexpr (YOUT) sts_vec<TOK>(pr + (c * 4 + g) * kRow + TOK * j, part);
             };
             constexpr int NG = kT / TOK;
-            if constexpr (!MS_TMEM_DB) {
-#pragma unroll 1
+            if constexpr (!MS_TMEM_DB && MS_TMEM_LD64 && MAXW <= 11) {
+                uint32_t bc2[16 * TOK];
+#pragma unroll
+                for (int j = 0; j < NG; j += 2) {
+                    static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
+                    (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 2) <= kTmemCols && 4 * c + g < 32);
+                    float dls0[TOK], dus0[TOK], dls1[TOK], dus1[TOK];
+                    lds_vec<TOK>(xd + c * kRow + TOK * j, dls0);
+                    lds_vec<TOK>(xu + c * kRow + TOK * j, dus0);
+                    lds_vec<TOK>(xd + c * kRow + TOK * (j + 1), dls1);
+                    lds_vec<TOK>(xu + c * kRow + TOK * (j + 1), dus1);
+                    tmem_ld64_sync(tcol + (uint32_t)(32 * j), bc2);
+#pragma unroll
+                    for (int t = 0; t < TOK; ++t) {
+                        dlA[t] = f2_splat(dls0[t]);
+                        duA[t] = f2_splat(dus0[t]);
+                        dlB[t] = f2_splat(dls1[t]);
+                        duB[t] = f2_splat(dus1[t]);
+                    }
+                    group(j, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2), dlA, duA);
+                    group(j + 1, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2 + 8 * TOK), dlB, duB);
+                }
+            } else if constexpr (!MS_TMEM_DB) {
+                // the y-less pass keeps the loop rolled (unrolled it spills)
+                constexpr int kUnr = YOUT ? kUnrollGroups : 1;
+#pragma unroll kUnr
                 for (int j = 0; j < NG; ++j) {
                     static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
-                    MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                    (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
                     float dls[TOK], dus[TOK];
                     lds_vec<TOK>(xd + c * kRow + TOK * j, dls);
                     lds_vec<TOK>(xu + c * kRow + TOK * j, dus);

@@ -76,7 +76,7 @@ def ssd_bytes(batch, seqlen, nheads, headdim, dstate, ngroups, in_bytes, out_byt
             + batch * nheads * headdim * dstate * 4)
 
 
-def ssd_flops(batch, seqlen, nheads, headdim, dstate, chunk=32):
+def ssd_flops(batch, seqlen, nheads, headdim, dstate, chunk=128):
     """Multiply-adds x 2 of the chunked matrix view per (batch, head, chunk):
     C S_in (Q N P), C B^T (Q Q N), G' X (Q Q P), B'^T X (N Q P)."""
     nch = (seqlen + chunk - 1) // chunk
@@ -121,7 +121,7 @@ KERNEL_SOURCES = {
     "conv_scan_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
     "decode_step": ("selective_state_space_40_b200/csrc/state_update_stream.cu",),
     "scan_bwd_130m": ("selective_state_space_40_b200/csrc/scan_bwd.cu",),
-    "ssd_2p7b": ("selective_state_space_40_b200/csrc/ssd_fwd.cu",),
+    "ssd_2p7b": ("selective_state_space_40_b200/csrc/ssd_fwd_tc.cu",),
     "ssd_decode": ("selective_state_space_40_b200/csrc/ssd_update.cu",),
 }
 
@@ -586,11 +586,15 @@ def main(argv=None):
     ssd_in = [{k: v.to(dev) for k, v in syn.ssd_inputs(sw).items()} for _ in range(2)]
     ssd_y = torch.empty(sw.batch, sw.seqlen, sw.nheads, sw.headdim, dtype=torch.float32, device=dev)
     ssd_steps = 20
+    sdims = mb.SsdDims(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate, sw.ngroups, *ssd_in[0]["x"].stride()[:3],
+                       *ssd_in[0]["dt"].stride()[:2], *ssd_in[0]["B"].stride()[:3], *ssd_in[0]["C"].stride()[:3],
+                       *ssd_y.stride()[:3], mb.MS_BF16, mb.MS_F32)
+    ssd_ws = torch.empty(mb.mamba2_ssd_workspace_size(sdims, False), dtype=torch.uint8, device=dev)
 
     def ssd_step(i):
         g = ssd_in[i & 1]
         mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True, y=ssd_y,
-                   return_final_state=False, stream=stream)
+                   return_final_state=False, stream=stream, workspace=ssd_ws)
 
     for i in range(3):
         ssd_step(i)
@@ -604,8 +608,8 @@ def main(argv=None):
     ssd_ms = max_over_ranks(statistics.fmean(a.elapsed_time(b) for a, b in sev), world, dev)
     sbytes = ssd_bytes(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate, sw.ngroups, 2, 4) \
         - sw.batch * sw.nheads * sw.headdim * sw.dstate * 4  # no final state requested
-    sflops = ssd_flops(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate)
-    del ssd_in
+    sflops = ssd_flops(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate, chunk=128)
+    del ssd_in, ssd_ws
 
     # ---- Mamba-2 SSD decode step (2.7B-class layer, 64 sequences): the fp32
     # state [64, 80, 64, 128] (168 MB) read and written once per step; two

@@ -321,7 +321,17 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
  * bf16 x, dt, B, C (MS_ERR_SHAPE / MS_ERR_DTYPE otherwise); x, B, C rows must
  * be 16-byte aligned and y rows aligned to two elements (MS_ERR_ALIGN).
  * y is fp32 or bf16 (out_dtype). D, dt_bias, initial_state, final_state may
- * be NULL.
+ * be NULL; initial_state may be the same array as final_state.
+ * The chunks (128 tokens) run in parallel on the tcgen05 tensor cores; the
+ * state entering a chunk is handed over from the previous chunk's work item
+ * through final_state (or, when it is NULL, the workspace).
+ *   workspace        caller-owned device memory of mamba2_ssd_workspace_size()
+ *                    bytes (for these dims and final_state given or not),
+ *                    16-byte aligned; its contents need not be kept between
+ *                    calls, but two calls in flight at once need two
+ *                    workspaces. Too small: MS_ERR_WORKSPACE.
+ *   dev_status       receives MS_ERR_TIMEOUT if a bounded wait inside the
+ *                    kernel ran out (y and final_state are then undefined).
  */
 typedef struct {
     int64_t batch, seqlen, nheads, headdim, dstate, ngroups;
@@ -333,10 +343,11 @@ typedef struct {
     int32_t in_dtype, out_dtype;
 } ms_ssd_dims;
 
+size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dims, int with_final_state);
 int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
                    const float *D, const float *dt_bias, int softplus_flag, const float *initial_state,
-                   void *y, float *final_state, const ms_ssd_dims *dims, int *dev_status,
-                   ms_stream_t stream);
+                   void *y, float *final_state, const ms_ssd_dims *dims, void *workspace,
+                   size_t workspace_bytes, int *dev_status, ms_stream_t stream);
 
 /*
  * Mamba-2 SSD layer: the intra-chunk products of the chunked matrix view

@@ -126,8 +126,11 @@ def _load(path: str) -> ctypes.CDLL:
         lib.mamba_scan_bwd_noalloc.argtypes = ([_vp] * 8 + [ctypes.c_int] + [_vp] * 12 +
                                                [ctypes.POINTER(ScanDims), _vp, _vp])
         lib.mamba_scan_bwd_noalloc.restype = ctypes.c_int
-        lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
+        lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp,
+                                                   ctypes.c_size_t, _vp, _vp]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
+        lib.mamba2_ssd_workspace_size.argtypes = [ctypes.POINTER(SsdDims), ctypes.c_int]
+        lib.mamba2_ssd_workspace_size.restype = ctypes.c_size_t
         lib.mamba2_ssd_chunk_cb_size.argtypes = [ctypes.POINTER(SsdDims)]
         lib.mamba2_ssd_chunk_cb_size.restype = ctypes.c_size_t
         lib.mamba2_ssd_chunk_cb.argtypes = [_vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp, _vp]
@@ -235,10 +238,14 @@ def mamba2_ssd_chunk_cb(B, C, cb, dims: SsdDims, dev_status=None, stream=None) -
     return library().mamba2_ssd_chunk_cb(B, C, cb, ctypes.byref(dims), dev_status, stream)
 
 
+def mamba2_ssd_workspace_size(dims: SsdDims, with_final_state: bool) -> int:
+    return int(library().mamba2_ssd_workspace_size(ctypes.byref(dims), int(bool(with_final_state))))
+
+
 def mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, softplus_flag, initial_state, y, final_state, dims: SsdDims,
-                   dev_status, stream) -> int:
+                   workspace, workspace_bytes, dev_status, stream) -> int:
     return library().mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, int(softplus_flag), initial_state, y, final_state,
-                                    ctypes.byref(dims), dev_status, stream)
+                                    ctypes.byref(dims), workspace, workspace_bytes, dev_status, stream)
 
 
 def mamba2_ssd_state_update(state, x, dt, A, B, C, D, dt_bias, softplus_flag, y, dims: SsdUpdateDims,
@@ -475,10 +482,14 @@ def scan_bwd_noalloc(u, delta, A, B, C, D, z, delta_bias, softplus: bool, dout, 
 
 
 def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial_state=None,
-            out_dtype=None, return_final_state: bool = True, y=None, stream=None, dev_status=None):
+            out_dtype=None, return_final_state: bool = True, y=None, stream=None, dev_status=None,
+            final_state=None, workspace=None):
     """Mamba-2 SSD layer forward on torch CUDA tensors: x [b, L, H, P], dt
     [b, L, H], B/C [b, L, G, N] (bf16), A/D/dt_bias [H] fp32. Returns (y,
-    final_state [b, H, P, N] or None)."""
+    final_state [b, H, P, N] or None). ``final_state`` (fp32, dense) may be
+    given to be written in place (it may be ``initial_state`` itself);
+    ``workspace`` (uint8 CUDA tensor of at least ``mamba2_ssd_workspace_size``
+    bytes) is allocated per call when omitted."""
     torch = _torch()
     if out_dtype is None:
         out_dtype = torch.float32
@@ -489,12 +500,20 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial
         _inner_contiguous(t, n)
     if y is None:
         y = torch.empty((batch, L, H, P), dtype=out_dtype, device=x.device)
-    fs = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device) if return_final_state else None
+    fs = final_state
+    if fs is None and return_final_state:
+        fs = torch.empty((batch, H, P, N), dtype=torch.float32, device=x.device)
+    if fs is not None:
+        _check_f32(final_state=fs)
     dims = SsdDims(batch, L, H, P, N, G, x.stride(0), x.stride(1), x.stride(2), dt.stride(0), dt.stride(1),
                    B.stride(0), B.stride(1), B.stride(2), C.stride(0), C.stride(1), C.stride(2),
                    y.stride(0), y.stride(1), y.stride(2), _dtype_code(x), _dtype_code(y))
+    ws_bytes = mamba2_ssd_workspace_size(dims, fs is not None)
+    if workspace is None:
+        workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     rc = mamba2_ssd_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias), softplus,
-                        _ptr(initial_state), _ptr(y), _ptr(fs), dims, _ptr(dev_status), _stream_handle(stream))
+                        _ptr(initial_state), _ptr(y), _ptr(fs), dims, _ptr(workspace),
+                        workspace.numel() * workspace.element_size(), _ptr(dev_status), _stream_handle(stream))
     if rc != MS_OK:
         raise MambaScanError(rc, "mamba2_ssd_fwd")
     return y, fs

@@ -636,10 +636,15 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
                           need > 0 ? MS_BWD_NOALLOC_MAX_BYTES : 0, dev_status, stream);
 }
 
+size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dm, int with_final_state) {
+    if (!dm || dm->batch < 0 || dm->nheads < 1) return 0;
+    return ms::ssd_tc_workspace_size(dm->batch, dm->nheads, with_final_state == 0);
+}
+
 int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
                    const float *dt_bias, int softplus_flag, const float *initial_state, void *y, float *final_state,
-                   const ms_ssd_dims *dm, int *dev_status, ms_stream_t stream) {
-    (void)dev_status;
+                   const ms_ssd_dims *dm, void *workspace, size_t workspace_bytes, int *dev_status,
+                   ms_stream_t stream) {
     if (!dm) return MS_ERR_NULL;
     if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) || (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
         return MS_ERR_DTYPE;
@@ -674,7 +679,24 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
             max_offset3(dm->batch, dm->C_sb, L, dm->C_sl, 1) < 0 || max_offset3(G, dm->C_sg, 1, 0, 128) < 0)
             return MS_ERR_SHAPE;
     }
-    if (dm->seqlen == 0 && !final_state) return MS_OK;
+    if (dm->seqlen == 0) {
+        // no tokens: the final state is the initial one
+        if (!final_state) return MS_OK;
+        const size_t bytes = (size_t)dm->batch * dm->nheads * dm->headdim * dm->dstate * sizeof(float);
+        cudaError_t e = initial_state ? (initial_state == final_state
+                                             ? cudaSuccess
+                                             : cudaMemcpyAsync(final_state, initial_state, bytes,
+                                                               cudaMemcpyDeviceToDevice, (cudaStream_t)stream))
+                                      : cudaMemsetAsync(final_state, 0, bytes, (cudaStream_t)stream);
+        if (e != cudaSuccess) {
+            cudaGetLastError();
+            return MS_ERR_CUDA;
+        }
+        return MS_OK;
+    }
+    const size_t need = ms::ssd_tc_workspace_size(dm->batch, dm->nheads, final_state == nullptr);
+    if (!workspace || workspace_bytes < need) return MS_ERR_WORKSPACE;
+    if (!aligned(workspace, 16)) return MS_ERR_ALIGN;
     ms::SsdArgs a{};
     a.x = x; a.dt = dt; a.B = B; a.C = C; a.A = A; a.D = D; a.dt_bias = dt_bias; a.s0 = initial_state;
     a.y = y; a.s_last = final_state;
@@ -683,7 +705,8 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
     a.B_sb = dm->B_sb; a.B_sl = dm->B_sl; a.B_sg = dm->B_sg; a.C_sb = dm->C_sb; a.C_sl = dm->C_sl;
     a.C_sg = dm->C_sg; a.y_sb = dm->y_sb; a.y_sl = dm->y_sl; a.y_sh = dm->y_sh;
     a.softplus = softplus_flag ? 1 : 0;
-    cudaError_t e = ms::launch_ssd_fwd(a, dm->out_dtype == MS_BF16, (cudaStream_t)stream);
+    a.status = dev_status;
+    cudaError_t e = ms::launch_ssd_fwd_tc(a, dm->out_dtype == MS_BF16, workspace, num_sms_current(), (cudaStream_t)stream);
     if (e != cudaSuccess) {
         cudaGetLastError();
         return MS_ERR_CUDA;

@@ -176,6 +176,33 @@ __device__ __forceinline__ f2 exp2_poly2(f2 x2) {
     return f2_make(pa, pb);
 }
 
+// exp2(y) - 1 for a pair with |y| <= 1/(2 ln 2) (|y ln 2| <= 1/2), by the
+// Taylor series of expm1 in y ln 2 to degree 8: coefficient k is
+// (ln 2)^k / k!; the first omitted term is below 5.4e-9, relative to the
+// result under 1.4e-8. Used as A_bar - 1, so that h + (A_bar - 1) h keeps the
+// low bits of a decay factor close to 1 that 1 + (A_bar - 1) would round off.
+struct Expm1Series {
+    static constexpr float c1 = 0.693147180559945f;
+    static constexpr float c2 = 0.240226506959101f;
+    static constexpr float c3 = 0.0555041086648216f;
+    static constexpr float c4 = 0.00961812910762848f;
+    static constexpr float c5 = 0.00133335581464284f;
+    static constexpr float c6 = 0.000154035303933816f;
+    static constexpr float c7 = 1.52527338040598e-05f;
+    static constexpr float c8 = 1.32154867901443e-06f;
+    static constexpr float kMaxArg = 0.721347520444482f;  // 1 / (2 ln 2)
+};
+__device__ __forceinline__ f2 exp2m1_series2(f2 y) {
+    f2 q = f2_fma(y, f2_splat(Expm1Series::c8), f2_splat(Expm1Series::c7));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c6));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c5));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c4));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c3));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c2));
+    q = f2_fma(q, y, f2_splat(Expm1Series::c1));
+    return f2_mul(q, y);
+}
+
 __device__ __forceinline__ f2 exp2_mufu2(f2 x2) {
     float xa, xb;
     f2_split(x2, xa, xb);

@@ -74,8 +74,24 @@ struct SsdArgs {
     int64_t batch, L, H, G;
     int64_t x_sb, x_sl, x_sh, dt_sb, dt_sl, B_sb, B_sl, B_sg, C_sb, C_sl, C_sg, y_sb, y_sl, y_sh;
     int softplus;
+    int *status;
 };
 bool ssd_shape_supported(int64_t headdim, int64_t dstate);
+
+// Chunk-parallel SSD forward on the tcgen05 tensor cores: per-launch state
+// of the chunk hand-off (flags [batch * H] then the ticket counter, zeroed
+// before the launch; the running state [batch, H, P, N], final_state when
+// given), the heads per work item, and whether y rows take 16-byte stores.
+struct SsdTcArgs {
+    int *flags;
+    int *counter;
+    float *state;
+    int hb;
+    int y_vec16;
+};
+int ssd_tc_head_block(int64_t batch, int64_t seqlen, int64_t nheads, int64_t ngroups, int num_sms);
+size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads, bool need_state);
+cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, int num_sms, cudaStream_t stream);
 
 // Arguments of the per-chunk C B^T of the SSD layer (bf16 B, C with dstate
 // 128; cb [batch, G, ceil(L / 32), 32, 32] fp32, dense).
@@ -102,7 +118,6 @@ struct SsdUpdArgs {
     int softplus;
 };
 cudaError_t launch_ssd_update(const SsdUpdArgs &a, bool in_bf16, bool out_bf16, cudaStream_t stream);
-cudaError_t launch_ssd_fwd(const SsdArgs &a, bool out_bf16, cudaStream_t stream);
 
 // Launch shape chosen on the host for one scan call.
 struct ScanPlan {

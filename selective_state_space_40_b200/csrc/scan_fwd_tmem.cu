@@ -110,14 +110,24 @@ constexpr int kBufCols = 256;          // 32 tokens x 8 values
 #ifndef MS_TMEM_UNROLL
 #define MS_TMEM_UNROLL 8
 #endif
-//   MS_TMEM_LD64     1: in the 12-warp variant one 64-column load (two groups
-//                    of 4 tokens) per wait; 0: one 32-column load per group.
+//   MS_TMEM_LD64     1: in the 12-warp variant that writes y, one 64-column
+//                    load (two groups of 4 tokens) per wait; 0: one 32-column
+//                    load per group.
 #ifndef MS_TMEM_LD64
 #define MS_TMEM_LD64 1
 #endif
 //   MS_TMEM_LDCLOB   1: the combined load-and-wait is a compiler memory
 //                    barrier; 0: it only defines its registers (shared
 //                    loads of later groups may move above it).
+//   MS_TMEM_SERIES   1: with every exponential on the FMA pipe (poly8 = 8),
+//                    a token (or a whole tile) whose exponents |Delta A| are
+//                    all <= 1/2 on every lane of the warp takes its decays
+//                    from the expm1 series; 0: the polynomial throughout. On
+//                    the long-context layer few tiles qualify and the
+//                    per-token vote costs more than the series saves.
+#ifndef MS_TMEM_SERIES
+#define MS_TMEM_SERIES 0
+#endif
 #ifndef MS_TMEM_LDCLOB
 #define MS_TMEM_LDCLOB 1
 #endif
@@ -541,15 +551,19 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
         const int64_t dd = active ? d : 0;
         const int n0 = 4 * g;
         f2 A2[2], h[2];
+        float amax2;  // max |A| log2(e) over the channel's 16 states (after the shuffles below)
         {
             const float4 Av = *reinterpret_cast<const float4 *>(a.A + dd * 16 + n0);
             A2[0] = f2_make(Av.x * kLog2e, Av.y * kLog2e);
             A2[1] = f2_make(Av.z * kLog2e, Av.w * kLog2e);
+            amax2 = kLog2e * fmaxf(fmaxf(fabsf(Av.x), fabsf(Av.y)), fmaxf(fabsf(Av.z), fabsf(Av.w)));
             float4 hv = make_float4(0.f, 0.f, 0.f, 0.f);
             if (a.h0 != nullptr && active) hv = *reinterpret_cast<const float4 *>(a.h0 + (b * a.dim + d) * 16 + n0);
             h[0] = f2_make(hv.x, hv.y);
             h[1] = f2_make(hv.z, hv.w);
         }
+        amax2 = fmaxf(amax2, __shfl_xor_sync(0xffffffffu, amax2, 1));
+        amax2 = fmaxf(amax2, __shfl_xor_sync(0xffffffffu, amax2, 2));
         const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
         const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
         const bool sp = a.softplus != 0;
@@ -779,12 +793,16 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             if (lane == 0) bar_arrive(bar(empty0 + s));  // this warp is done with the stage
             const bool live = t0 + 8 * g < L;  // L % 8 == 0: whole chunks are in or out
             float gate[8], dug[8];
+            // every exponent |Delta A| log2(e) of the warp's tile within the
+            // series' range: the tile's decays come from the expm1 series
+            bool series_tile = false;
             {
-                float dl[8], dlu[8];
+                float dl[8], dlu[8], dmax = 0.0f;
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float v = dv[j] + bias;
                     dl[j] = live ? (sp ? softplus_f(v) : v) : 0.0f;  // past the end: the state is left alone
+                    dmax = fmaxf(dmax, fabsf(dl[j]));
                     dlu[j] = dl[j] * uv[j];
                     if constexpr (YOUT) {
                         gate[j] = has_z ? silu_f(zv[j]) : 1.0f;
@@ -793,6 +811,7 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                         dsum_acc += dl[j];
                     }
                 }
+                if constexpr (POLY8 == 8 && MS_TMEM_SERIES) series_tile = __all_sync(0xffffffffu, dmax * amax2 <= Expm1Series::kMaxArg);
                 if constexpr (SPLAT) {
                     float4 *px = reinterpret_cast<float4 *>(xd + c * kRowS + 4 * (8 * g));
 #pragma unroll
@@ -835,7 +854,10 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                     }
                 }
             };
-            auto group = [&](int j, const uint32_t(&bc)[8 * TOK], const f2(&dl2s)[TOK], const f2(&du2s)[TOK]) {
+            // series: a tile whose decays all come from the expm1 series
+            // (h += (A_bar - 1) h + Delta u B); the callers pass a constant
+            auto group = [&](bool series, int j, const uint32_t(&bc)[8 * TOK], const f2(&dl2s)[TOK],
+                             const f2(&du2s)[TOK]) {
                 float part[TOK];
                 if constexpr (MS_TMEM_SCALAR) {
                     // the pairs hold (Delta, Delta) and (Delta*u, Delta*u): use one half
@@ -869,23 +891,34 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 for (int t = 0; t < TOK; ++t) {
                     const f2 dl2 = dl2s[t];
                     const f2 du2 = du2s[t];
+                    // this token's exponents within the series' range on every lane of the warp
+                    bool ser_t = false;
+                    if constexpr (POLY8 == 8 && MS_TMEM_SERIES) {
+                        float d0, d1;
+                        f2_split(dl2, d0, d1);
+                        ser_t = series || __all_sync(0xffffffffu, fabsf(d0) * amax2 <= Expm1Series::kMaxArg);
+                    }
                     f2 acc = 0ull;
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         const f2 Bp =
                             f2_make(__uint_as_float(bc[8 * t + 2 * p]), __uint_as_float(bc[8 * t + 2 * p + 1]));
                         const f2 x = f2_mul(A2[p], dl2);
-                        // a fixed share of the (token, pair) slots of every 4 tokens on the polynomial
-                        const bool poly = (2 * ((TOK * j + t) & 3) + p) < POLY8;
-                        f2 ab;
-                        if (poly) {
-                            ab = exp2_poly2(x);
+                        if (POLY8 == 8 && ser_t) {
+                            h[p] = f2_fma(exp2m1_series2(x), h[p], f2_fma(du2, Bp, h[p]));
                         } else {
-                            float xa, xb;
-                            f2_split(x, xa, xb);
-                            ab = f2_make(exp2_mufu(xa), exp2_mufu(xb));
+                            // a fixed share of the (token, pair) slots of every 4 tokens on the polynomial
+                            const bool poly = (2 * ((TOK * j + t) & 3) + p) < POLY8;
+                            f2 ab;
+                            if (poly) {
+                                ab = exp2_poly2(x);
+                            } else {
+                                float xa, xb;
+                                f2_split(x, xa, xb);
+                                ab = f2_make(exp2_mufu(xa), exp2_mufu(xb));
+                            }
+                            h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp));
                         }
-                        h[p] = f2_fma(ab, h[p], f2_mul(du2, Bp));
                         if constexpr (YOUT) {
                             const f2 Cp = f2_make(__uint_as_float(bc[8 * t + 4 + 2 * p]),
                                                   __uint_as_float(bc[8 * t + 5 + 2 * p]));
@@ -898,60 +931,64 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
                 }
                 if constexpr (YOUT) sts_vec<TOK>(pr + (c * 4 + g) * kRow + TOK * j, part);
             };
-            constexpr int NG = kT / TOK;
-            if constexpr (!MS_TMEM_DB && MS_TMEM_LD64 && MAXW <= 11) {
-                uint32_t bc2[16 * TOK];
+            // the y-less pass keeps the loop rolled (unrolled it spills)
+            constexpr int kUnr = YOUT ? kUnrollGroups : 1;
+            auto run_tile = [&](bool sc) {
+                constexpr int NG = kT / TOK;
+                if constexpr (!MS_TMEM_DB && MS_TMEM_LD64 && MAXW <= 11 && YOUT) {
+                    uint32_t bc2[16 * TOK];
 #pragma unroll
-                for (int j = 0; j < NG; j += 2) {
-                    static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
-                    (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 2) <= kTmemCols && 4 * c + g < 32);
-                    float dls0[TOK], dus0[TOK], dls1[TOK], dus1[TOK];
-                    lds_vec<TOK>(xd + c * kRow + TOK * j, dls0);
-                    lds_vec<TOK>(xu + c * kRow + TOK * j, dus0);
-                    lds_vec<TOK>(xd + c * kRow + TOK * (j + 1), dls1);
-                    lds_vec<TOK>(xu + c * kRow + TOK * (j + 1), dus1);
-                    tmem_ld64_sync(tcol + (uint32_t)(32 * j), bc2);
+                    for (int j = 0; j < NG; j += 2) {
+                        static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
+                        (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 2) <= kTmemCols && 4 * c + g < 32);
+                        float dls0[TOK], dus0[TOK], dls1[TOK], dus1[TOK];
+                        lds_vec<TOK>(xd + c * kRow + TOK * j, dls0);
+                        lds_vec<TOK>(xu + c * kRow + TOK * j, dus0);
+                        lds_vec<TOK>(xd + c * kRow + TOK * (j + 1), dls1);
+                        lds_vec<TOK>(xu + c * kRow + TOK * (j + 1), dus1);
+                        tmem_ld64_sync(tcol + (uint32_t)(32 * j), bc2);
 #pragma unroll
-                    for (int t = 0; t < TOK; ++t) {
-                        dlA[t] = f2_splat(dls0[t]);
-                        duA[t] = f2_splat(dus0[t]);
-                        dlB[t] = f2_splat(dls1[t]);
-                        duB[t] = f2_splat(dus1[t]);
+                        for (int t = 0; t < TOK; ++t) {
+                            dlA[t] = f2_splat(dls0[t]);
+                            duA[t] = f2_splat(dus0[t]);
+                            dlB[t] = f2_splat(dls1[t]);
+                            duB[t] = f2_splat(dus1[t]);
+                        }
+                        group(sc, j, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2), dlA, duA);
+                        group(sc, j + 1, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2 + 8 * TOK), dlB, duB);
                     }
-                    group(j, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2), dlA, duA);
-                    group(j + 1, *reinterpret_cast<const uint32_t(*)[8 * TOK]>(bc2 + 8 * TOK), dlB, duB);
-                }
-            } else if constexpr (!MS_TMEM_DB) {
-                // the y-less pass keeps the loop rolled (unrolled it spills)
-                constexpr int kUnr = YOUT ? kUnrollGroups : 1;
+                } else if constexpr (!MS_TMEM_DB) {
 #pragma unroll kUnr
-                for (int j = 0; j < NG; ++j) {
-                    static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
-                    (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
-                    float dls[TOK], dus[TOK];
-                    lds_vec<TOK>(xd + c * kRow + TOK * j, dls);
-                    lds_vec<TOK>(xu + c * kRow + TOK * j, dus);
-                    tmem_ld32_sync(tcol + (uint32_t)(32 * j), bcA);
+                    for (int j = 0; j < NG; ++j) {
+                        static_assert(TOK == 4 && !SPLAT, "single loads: 4 tokens, plain Delta rows");
+                        (void)MS_CHECK(a.status, vb * kBufCols + 32 * (j + 1) <= kTmemCols && 4 * c + g < 32);
+                        float dls[TOK], dus[TOK];
+                        lds_vec<TOK>(xd + c * kRow + TOK * j, dls);
+                        lds_vec<TOK>(xu + c * kRow + TOK * j, dus);
+                        tmem_ld32_sync(tcol + (uint32_t)(32 * j), bcA);
 #pragma unroll
-                    for (int t = 0; t < TOK; ++t) {
-                        dlA[t] = f2_splat(dls[t]);
-                        duA[t] = f2_splat(dus[t]);
+                        for (int t = 0; t < TOK; ++t) {
+                            dlA[t] = f2_splat(dls[t]);
+                            duA[t] = f2_splat(dus[t]);
+                        }
+                        group(sc, j, bcA, dlA, duA);
                     }
-                    group(j, bcA, dlA, duA);
-                }
-            } else {
-            fetch(0, bcA, dlA, duA);
-            tmem_wait<8 * TOK>(bcA);
+                } else {
+                fetch(0, bcA, dlA, duA);
+                tmem_wait<8 * TOK>(bcA);
 #pragma unroll 1
-            for (int j = 0; j < NG; j += 2) {
-                fetch(j + 1, bcB, dlB, duB);
-                group(j, bcA, dlA, duA);
-                tmem_wait<8 * TOK>(bcB);
-                if (j + 2 < NG) fetch(j + 2, bcA, dlA, duA);
-                group(j + 1, bcB, dlB, duB);
-                if (j + 2 < NG) tmem_wait<8 * TOK>(bcA);
-            }
-            }
+                for (int j = 0; j < NG; j += 2) {
+                    fetch(j + 1, bcB, dlB, duB);
+                    group(sc, j, bcA, dlA, duA);
+                    tmem_wait<8 * TOK>(bcB);
+                    if (j + 2 < NG) fetch(j + 2, bcA, dlA, duA);
+                    group(sc, j + 1, bcB, dlB, duB);
+                    if (j + 2 < NG) tmem_wait<8 * TOK>(bcA);
+                }
+                }
+            };
+            if (POLY8 == 8 && series_tile) run_tile(true);
+            else run_tile(false);
             // tensor-memory buffer vb is read: release it to the producer
             asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
             __syncwarp();

@@ -1,0 +1,677 @@
+// ssd_fwd_tc.cu -- Mamba-2 state space duality (SSD) layer, forward, chunk-
+// parallel on the sm_100a tensor cores (tcgen05, accumulators in tensor
+// memory).
+//
+// 'Mamba-1/2/3 Markdown図解' blog, section 3: the SSD model has a recurrent
+// view and a matrix view computed chunk by chunk -- matrix products inside a
+// chunk, the state handed from one chunk to the next; the transition is a
+// scalar times the identity within a head. Per batch row b and head h (state
+// S [N x P] here, group g of B and C):
+//   S_t = exp(Delta_t A_h) S_{t-1} + B_t (Delta_t x_t)^T,   y_t = S_t^T C_t + D_h x_t
+// With cs_t = A_h sum_{r<=t} Delta_r inside a chunk of Q tokens (t = 0..Q-1)
+// and S_in the state entering it:
+//   y_t   = exp(cs_t) sum_n C_t[n] S_in[n][.] + sum_{s<=t} (C_t . B_s) exp(cs_t - cs_s) Delta_s x_s + D x_t
+//   S_out = exp(cs_{Q-1}) S_in + sum_s B_s (w_s x_s)^T,   w_s = exp(cs_{Q-1} - cs_s) Delta_s
+// Four products per chunk and head, each M = 128 on the tensor cores
+// (bf16 x bf16 -> fp32):
+//   CB    [Q x Q] = C B^T                       (once per chunk and group)
+//   S_c   [N x P] = B^T X'        X'[s] = w_s x_s
+//   Y_i   [Q x P] = G' X          G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s (s <= t)
+//   Y_s   [Q x P] = C S_in
+// and y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t, S_out = exp(cs_{Q-1}) S_in + S_c.
+// Operands that are not bf16 inputs (X', G', S_in) are split into a high and
+// a low bf16 part, v = hi + lo, and both are multiplied (about 16 significant
+// bits).
+//
+// Work item = (chunk k, batch row b, block of up to 8 heads of one group).
+// Items are claimed in ticket order from a global counter, chunk-major, so the
+// item holding chunk k - 1 of the same heads started before this one. Only
+// Y_s and S_out depend on the entering state: each head's item computes
+// CB, S_c and Y_i first, then waits for chunk k - 1's item to publish S_in
+// (a per-(b, h) counter in global memory), writes S_out over it and
+// publishes it for chunk k + 1. The running state lives in final_state (or
+// the workspace) and crosses chunks through L2, so HBM sees each input once.
+//
+// CTA: 8 compute warps (warp w: tensor-memory lanes 32 (w % 4).., column half
+// w / 4) and one MMA warp whose lane 0 issues every tcgen05.mma and commit.
+// Shared-memory operands use the canonical layouts without swizzle (8-row x
+// 16-byte core matrices): K-major for C (and B in C B^T) and G', MN-major for
+// B (in B^T X'), x, X' and S_in -- the same bytes of the B tile serve both of
+// its roles. Every wait is bounded: on a timeout the CTA records
+// MS_ERR_TIMEOUT, stops, waits (bounded) for its issued products and frees its
+// tensor memory.
+
+#include <cstdint>
+
+#include "mambascan.h"
+#include "ms_device.cuh"
+#include "ms_internal.h"
+
+// MN-major no-swizzle descriptor fields: 1 = leading byte offset along K,
+// stride byte offset along M/N (the K-major assignment); 0 = the reverse.
+#ifndef MS_SSD_MN_LBO_K
+#define MS_SSD_MN_LBO_K 1
+#endif
+
+namespace ms {
+
+namespace {
+
+constexpr int kQ = 128;        // tokens per chunk
+constexpr int kP = 64;         // head dim
+constexpr int kN = 128;        // state size
+constexpr int kHB = 8;         // most heads per work item
+constexpr int kComputeThreads = 256;
+constexpr int kThreads = kComputeThreads + 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColCB = 0, kColSC = 128, kColYI = 192, kColYS = 256;
+constexpr uint32_t kSpinTries = 1u << 20;       // mbarrier try_wait rounds
+constexpr uint32_t kFlagTries = 1u << 22;       // polls of a predecessor's counter (with a short sleep)
+
+// shared-memory map (bytes)
+constexpr int kOffC = 0;                          // C tile   [t][n] K-major, 32 KB
+constexpr int kOffB = kOffC + kQ * kN * 2;        // B tile   [s][n], 32 KB
+constexpr int kOffX = kOffB + kQ * kN * 2;        // x of two heads [s][p] MN-major, 2 x 16 KB
+constexpr int kOffXP = kOffX + 2 * kQ * kP * 2;   // X' hi / lo, later S_in hi / lo: 2 x 16 KB
+constexpr int kOffG = kOffXP + 2 * kQ * kP * 2;   // G' hi / lo [t][s] K-major: 2 x 32 KB
+constexpr int kOffPar = kOffG + 2 * kQ * kQ * 2;  // dl, cs2, w: [kHB][kQ] floats each
+constexpr int kOffBar = kOffPar + 3 * kHB * kQ * 4;
+constexpr int kNumBars = 9;
+constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tensor-memory base, ticket, abort
+constexpr int kSmemBytes = kOffMisc + 16;
+constexpr int kTileHalf = kQ * kP * 2;            // 16 KB: one [128 x 64] bf16 operand
+enum { kBarCB = 0, kBarXP, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarLD, kBarEnd };
+
+// K-major no-swizzle [rows x 128] bf16 tile: core matrix (row / 8, k / 8) at
+// (row / 8) * 2048 + (k / 8) * 128, row % 8 at 16-byte steps inside it.
+__device__ __forceinline__ uint32_t kmaj_off(int row, int kc) {
+    return (uint32_t)((row >> 3) * 2048 + kc * 128 + (row & 7) * 16);
+}
+// MN-major no-swizzle [k rows x 64] bf16 operand (k = token or state, 64
+// columns p): core matrix (k / 8, p / 8) at (k / 8) * 1024 + (p / 8) * 128,
+// k % 8 at 16-byte steps inside it.
+__device__ __forceinline__ uint32_t mn64_off(int k, int pc) {
+    return (uint32_t)((k >> 3) * 1024 + pc * 128 + (k & 7) * 16);
+}
+
+__device__ __forceinline__ uint32_t saddr(const void *p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t sdesc(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((addr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46);
+}
+// K-major: leading offset between the two core matrices along K, stride
+// between 8-row groups.
+__device__ __forceinline__ uint64_t desc_k(uint32_t addr, uint32_t k_stride, uint32_t mn_stride) {
+    return sdesc(addr, k_stride, mn_stride);
+}
+__device__ __forceinline__ uint64_t desc_mn(uint32_t addr, uint32_t k_stride, uint32_t mn_stride) {
+#if MS_SSD_MN_LBO_K
+    return sdesc(addr, k_stride, mn_stride);
+#else
+    return sdesc(addr, mn_stride, k_stride);
+#endif
+}
+// Instruction descriptor, kind::f16: fp32 D (bits 4-5), bf16 A and B (bits
+// 7-9, 10-12), A / B major-ness (bit 15 / 16: 1 = M/N-major), N >> 3 at bit
+// 17, M >> 4 at bit 24.
+constexpr uint32_t idesc(int n, bool a_mn, bool b_mn) {
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((a_mn ? 1u : 0u) << 15) | ((b_mn ? 1u : 0u) << 16) |
+           ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t id, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :
+        : "r"(tmem_d), "l"(da), "l"(db), "r"(id), "r"(acc ? 1u : 0u)
+        : "memory");
+}
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+                 : "memory");
+}
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t i = 0; i < kSpinTries; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(done)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// named barrier 1 over the compute warps, and-reducing a predicate
+__device__ __forceinline__ bool compute_sync_and(bool ok) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "barrier.cta.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"(ok ? 1u : 0u), "n"(kComputeThreads)
+        : "memory");
+    return r != 0;
+}
+__device__ __forceinline__ void cp_async16(uint32_t sdst, const void *gsrc, int src_bytes) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sdst), "l"(gsrc), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 32 columns of this warp's 32 tensor-memory lanes, waited for in the same statement
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr)
+        : "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint32_t pack2(float lo_elem, float hi_elem) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
+    return *reinterpret_cast<uint32_t *>(&v);
+}
+// 8 floats -> one 16-byte piece of high parts and one of low parts
+__device__ __forceinline__ void split8(const float *v, uint4 &hi, uint4 &lo) {
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+        h[i] = *reinterpret_cast<const uint32_t *>(&hh);
+        l[i] = pack2(v[2 * i] - __low2float(hh), v[2 * i + 1] - __high2float(hh));
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+__device__ __forceinline__ void unpack8(const uint4 &q, float *v) {
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        v[2 * i] = __uint_as_float(w[i] << 16);
+        v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+__device__ __forceinline__ int ld_acquire(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+template <typename TOut>
+__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a, const SsdTcArgs w) {
+    extern __shared__ __align__(1024) unsigned char smem[];
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const uint32_t sbase = saddr(smem);
+    auto bar = [&](int i) { return sbase + (uint32_t)(kOffBar + 8 * i); };
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kOffMisc);  // [0] tmem base, [1] ticket, [2] abort
+    volatile uint32_t *abort_flag = misc + 2;
+
+    if (tid == 0) {
+        misc[1] = (uint32_t)atomicAdd(w.counter, 1);
+        misc[2] = 0u;
+        bar_init(bar(kBarCB), 1);
+        bar_init(bar(kBarXP), 8);
+        bar_init(bar(kBarSC), 1);
+        bar_init(bar(kBarG), 8);
+        bar_init(bar(kBarYI), 1);
+        bar_init(bar(kBarS), 8);
+        bar_init(bar(kBarYS), 1);
+        bar_init(bar(kBarLD), 1);
+        bar_init(bar(kBarEnd), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 8) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sbase + kOffMisc),
+                     "r"(kTmemCols)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_before();
+    __syncthreads();
+    tc_after();
+    const uint32_t tmem = misc[0];
+    const int64_t ticket = (int64_t)misc[1];
+
+    // ---- work item
+    const int64_t hpg = a.H / a.G;                       // heads per group
+    const int64_t nhb = (hpg + w.hb - 1) / w.hb;         // head blocks per group
+    const int64_t per_chunk = a.batch * a.G * nhb;
+    const int64_t k = ticket / per_chunk;
+    const int64_t r0 = ticket % per_chunk;
+    const int64_t b = r0 / (a.G * nhb);
+    const int64_t g = (r0 / nhb) % a.G;
+    const int64_t hbk = r0 % nhb;
+    const int64_t h0 = g * hpg + hbk * w.hb;
+    const int64_t left = hpg - hbk * w.hb;
+    const int nh = (int)(left < (int64_t)w.hb ? left : (int64_t)w.hb);
+    const int64_t t0 = k * kQ;
+    const int64_t L = a.L;
+
+    const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
+    const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
+    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(a.x) + b * a.x_sb;
+    float *dlp = reinterpret_cast<float *>(smem + kOffPar);   // [kHB][kQ] Delta
+    float *cs2p = dlp + kHB * kQ;                             // [kHB][kQ] cs log2(e)
+    float *wp = cs2p + kHB * kQ;                              // [kHB][kQ] w_s
+
+    if (warp == 8) {
+        // ================================ MMA warp ================================
+        bool ok = true;
+        if (lane == 0) {
+            const uint32_t sC = sbase + kOffC, sB = sbase + kOffB, sXP = sbase + kOffXP, sG = sbase + kOffG;
+            // CB = C B^T: both K-major [128 x 128], once the C and B tiles are in
+            ok = bar_wait(bar(kBarLD), 0u) && *abort_flag == 0u;
+            if (ok) {
+                tc_after();
+#pragma unroll 1
+                for (int ks = 0; ks < kN / 16; ++ks)
+                    mma(tmem + kColCB, desc_k(sC + 256u * ks, 128u, 2048u), desc_k(sB + 256u * ks, 128u, 2048u),
+                        idesc(kQ, false, false), ks > 0);
+                mma_commit(bar(kBarCB));
+            }
+            for (int j = 0; j < nh && ok; ++j) {
+                const uint32_t ph = (uint32_t)(j & 1);
+                const uint32_t sX = sbase + kOffX + (uint32_t)((j & 1) * kTileHalf);
+                // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo) N(p)-major
+                ok = bar_wait(bar(kBarXP), ph) && *abort_flag == 0u;
+                if (!ok) break;
+                tc_after();
+#pragma unroll 1
+                for (int ks = 0; ks < kQ / 16; ++ks)
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+                        mma(tmem + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
+                            desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                            idesc(kP, true, true), ks > 0 || part > 0);
+                mma_commit(bar(kBarSC));
+                // Y_i [t x p] = G' X: A = G' (hi, lo) K-major, B = x N(p)-major
+                ok = bar_wait(bar(kBarG), ph) && *abort_flag == 0u;
+                if (!ok) break;
+                tc_after();
+#pragma unroll 1
+                for (int ks = 0; ks < kQ / 16; ++ks)
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+                        mma(tmem + kColYI, desc_k(sG + (uint32_t)(part * 2 * kTileHalf) + 256u * ks, 128u, 2048u),
+                            desc_mn(sX + 2048u * ks, 1024u, 128u), idesc(kP, false, true), ks > 0 || part > 0);
+                mma_commit(bar(kBarYI));
+                // Y_s [t x p] = C S_in: A = C K-major, B = S_in (hi, lo) N(p)-major
+                ok = bar_wait(bar(kBarS), ph) && *abort_flag == 0u;
+                if (!ok) break;
+                tc_after();
+#pragma unroll 1
+                for (int ks = 0; ks < kN / 16; ++ks)
+#pragma unroll
+                    for (int part = 0; part < 2; ++part)
+                        mma(tmem + kColYS, desc_k(sC + 256u * ks, 128u, 2048u),
+                            desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                            idesc(kP, false, true), ks > 0 || part > 0);
+                mma_commit(bar(kBarYS));
+            }
+            if (!ok) {
+                *abort_flag = 1u;
+                if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+            }
+            // every product issued above has completed before the tensor memory is freed
+            mma_commit(bar(kBarEnd));
+            (void)bar_wait(bar(kBarEnd), 0u);
+        }
+        __syncwarp();
+    } else {
+        // ============================== compute warps ==============================
+        const int qd = warp & 3, hf = warp >> 2;
+        const int row = 32 * qd + lane;                    // accumulator lane: token t or state n
+        const uint32_t trow = (uint32_t)(32 * qd) << 16;
+        bool ok = true;
+
+        // chunk tiles: C, B (rows past L zero-filled), x of heads 0 and 1
+        auto load_x = [&](int j) {
+            if (j < nh) {
+                const __nv_bfloat16 *xh = xb + (h0 + j) * a.x_sh;
+                const uint32_t dst = sbase + kOffX + (uint32_t)((j & 1) * kTileHalf);
+                for (int i = tid; i < kQ * (kP / 8); i += kComputeThreads) {
+                    const int s = i >> 3, pc = i & 7;
+                    const bool in = t0 + s < L;
+                    cp_async16(dst + mn64_off(s, pc), xh + (in ? t0 + s : 0) * a.x_sl + 8 * pc, in ? 16 : 0);
+                }
+            }
+            cp_commit();
+        };
+        for (int i = tid; i < kQ * (kN / 8); i += kComputeThreads) {
+            const int t = i >> 4, kc = i & 15;
+            const bool in = t0 + t < L;
+            const int64_t tt = in ? t0 + t : 0;
+            cp_async16(sbase + kOffC + kmaj_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
+            cp_async16(sbase + kOffB + kmaj_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
+        }
+        load_x(0);  // group 0: C, B, x of head 0
+        load_x(1);  // group 1: x of head 1 (empty when absent)
+
+        // per-head chunk parameters: warp j < nh takes head h0 + j, 4 tokens per lane
+        if (warp < nh) {
+            const int64_t h = h0 + warp;
+            const float A2 = __ldg(a.A + h) * kLog2e;
+            const float bias = a.dt_bias ? __ldg(a.dt_bias + h) : 0.0f;
+            const unsigned short *dtp = static_cast<const unsigned short *>(a.dt) + b * a.dt_sb + h;
+            float dl[4], c = 0.0f;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int64_t t = t0 + 4 * lane + i;
+                float d = 0.0f;
+                if (t < L) {
+                    const float v = bf16_bits_to_f32(__ldg(dtp + t * a.dt_sl)) + bias;
+                    d = a.softplus ? softplus_f(v) : v;
+                }
+                dl[i] = d;
+                c += d;
+            }
+            // inclusive prefix of the lanes' sums
+            float incl = c;
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const float o = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += o;
+            }
+            float run = incl - c;  // sum before this lane's tokens
+            const float total = __shfl_sync(0xffffffffu, incl, 31);
+            const float cend = A2 * total;  // cs_{Q-1} log2(e): padded tokens add nothing
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                run += dl[i];
+                const int t = 4 * lane + i;
+                const float c2 = A2 * run;
+                dlp[warp * kQ + t] = dl[i];
+                cs2p[warp * kQ + t] = c2;
+                wp[warp * kQ + t] = exp2_mufu(cend - c2) * dl[i];
+            }
+        }
+        cp_wait1();          // this thread's copies of group 0 are in
+        fence_async_smem();  // ... and visible to the tensor cores
+        // everyone's copies and parameters are in: the MMA warp starts C B^T
+        ok = compute_sync_and(ok);
+        if (tid == 0) bar_arrive(bar(kBarLD));
+
+        for (int j = 0; j < nh; ++j) {
+            const uint32_t ph = (uint32_t)(j & 1);
+            const int64_t h = h0 + j;
+            const unsigned char *X = smem + kOffX + (j & 1) * kTileHalf;
+            unsigned char *XP = smem + kOffXP;
+            unsigned char *G = smem + kOffG;
+            const float *cs2 = cs2p + j * kQ;
+            if (j > 0) {
+                cp_wait1();  // x of head j is in (the newest group may still be in flight)
+                fence_async_smem();
+                ok = compute_sync_and(ok && *abort_flag == 0u);
+                if (!ok) break;
+            }
+            // ---- X' = w_s x_s (row s, columns p of this half), hi / lo
+            {
+                const int s = row;
+                const float ws = wp[j * kQ + s];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int pc = 4 * hf + q;
+                    float v[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(s, pc)), v);
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) v[e] *= ws;
+                    uint4 hi, lo;
+                    split8(v, hi, lo);
+                    *reinterpret_cast<uint4 *>(XP + mn64_off(s, pc)) = hi;
+                    *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(s, pc)) = lo;
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarXP));
+
+            // ---- G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s for s <= t (s in this half), hi / lo
+            if (j == 0) {
+                ok = __all_sync(0xffffffffu, bar_wait(bar(kBarCB), 0u));
+                tc_after();
+            }
+            {
+                const int t = row;
+                const float ct = cs2[t];
+                const float *dls = dlp + j * kQ;
+                const bool zero_half = hf == 1 && qd < 2;  // s >= 64 > t for every lane of the warp
+#pragma unroll
+                for (int c32 = 0; c32 < 2; ++c32) {
+                    float v[32];
+                    if (!zero_half && ok) {
+                        tmem_ld32(tmem + trow + kColCB + (uint32_t)(64 * hf + 32 * c32), v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) {
+                            const int s = 64 * hf + 32 * c32 + e;
+                            v[e] = s <= t ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+                    }
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        const int kc = 8 * hf + 4 * c32 + q;
+                        uint4 hi, lo;
+                        split8(v + 8 * q, hi, lo);
+                        *reinterpret_cast<uint4 *>(G + kmaj_off(t, kc)) = hi;
+                        *reinterpret_cast<uint4 *>(G + 2 * kTileHalf + kmaj_off(t, kc)) = lo;
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_before();
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarG));
+
+            // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out
+            ok = __all_sync(0xffffffffu, ok && bar_wait(bar(kBarSC), ph));
+            tc_after();
+            {
+                int *flag = w.flags + (b * a.H + h);
+                if (k > 0 && ok) {
+                    uint32_t i = 0;
+                    while (ld_acquire(flag) < (int)k && i < kFlagTries) {
+                        __nanosleep(64);
+                        ++i;
+                    }
+                    ok = i < kFlagTries;
+                }
+                ok = __all_sync(0xffffffffu, ok);
+                const int n = row;
+                const size_t blk = (size_t)(b * a.H + h) * kP * kN;
+                float *st = w.state + blk;
+                const float *sin = k > 0 ? st : (a.s0 ? a.s0 + blk : nullptr);
+                const float decay = exp2_mufu(cs2[kQ - 1]);
+                float sc[32];
+                if (ok) tmem_ld32(tmem + trow + kColSC + (uint32_t)(32 * hf), sc);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float v[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int p = 32 * hf + 8 * q + e;
+                        v[e] = (sin != nullptr && ok) ? sin[(size_t)p * kN + n] : 0.0f;
+                    }
+                    if (ok) {
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int p = 32 * hf + 8 * q + e;
+                            st[(size_t)p * kN + n] = fmaf(decay, v[e], sc[8 * q + e]);
+                        }
+                    }
+                    uint4 hi, lo;
+                    split8(v, hi, lo);
+                    const int pc = 4 * hf + q;
+                    *reinterpret_cast<uint4 *>(XP + mn64_off(n, pc)) = hi;
+                    *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(n, pc)) = lo;
+                }
+                fence_async_smem();
+                tc_before();
+                // every compute thread's S_out is stored: publish it for chunk k + 1
+                ok = compute_sync_and(ok);
+                if (tid == 0 && ok) {
+                    __threadfence();
+                    st_release(flag, (int)k + 1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarS));
+            if (!ok) break;
+
+            // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t
+            ok = __all_sync(0xffffffffu, bar_wait(bar(kBarYI), ph) && bar_wait(bar(kBarYS), ph));
+            tc_after();
+            if (ok) {
+                const int t = row;
+                float ys[32], yi[32];
+                tmem_ld32(tmem + trow + kColYS + (uint32_t)(32 * hf), ys);
+                tmem_ld32(tmem + trow + kColYI + (uint32_t)(32 * hf), yi);
+                const float et = exp2_mufu(cs2[t]);
+                const float Dh = a.D ? __ldg(a.D + h) : 0.0f;
+                if (t0 + t < L) {
+                    TOut *yp = static_cast<TOut *>(a.y) + b * a.y_sb + (t0 + t) * a.y_sl + h * a.y_sh + 32 * hf;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        float xv[8], yo[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(t, 4 * hf + q)), xv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], fmaf(Dh, xv[e], yi[8 * q + e]));
+                        if constexpr (sizeof(TOut) == 4) {
+                            if (w.y_vec16) {
+                                float4 *p4 = reinterpret_cast<float4 *>(yp + 8 * q);
+                                p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
+                                p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                            } else {
+                                float2 *p2 = reinterpret_cast<float2 *>(yp + 8 * q);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
+                            }
+                        } else {
+                            if (w.y_vec16) {
+                                *reinterpret_cast<uint4 *>(yp + 8 * q) =
+                                    make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]), pack2(yo[4], yo[5]),
+                                               pack2(yo[6], yo[7]));
+                            } else {
+                                uint32_t *p1 = reinterpret_cast<uint32_t *>(yp + 8 * q);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                            }
+                        }
+                    }
+                }
+            }
+            tc_before();
+            // every compute thread is done with x of head j: its buffer takes head j + 2
+            ok = compute_sync_and(ok && *abort_flag == 0u);
+            if (!ok) break;
+            load_x(j + 2);
+        }
+        if (!ok && tid == 0) {
+            *abort_flag = 1u;
+            if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+        }
+        asm volatile("cp.async.wait_all;" ::: "memory");
+    }
+
+    // ---- tear-down: the MMA warp has drained its products; free the tensor memory
+    tc_before();
+    __syncthreads();
+    if (warp == 8) {
+        tc_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+    }
+}
+
+template <typename TOut>
+cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, int64_t items, cudaStream_t stream) {
+    static SmemOptIn opt_in;
+    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_fwd_tc_kernel<TOut>), kSmemBytes);
+    if (e != cudaSuccess) return e;
+    ssd_fwd_tc_kernel<TOut><<<(unsigned)items, kThreads, kSmemBytes, stream>>>(a, w);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool ssd_shape_supported(int64_t headdim, int64_t dstate) { return headdim == kP && dstate == kN; }
+
+int ssd_tc_head_block(int64_t batch, int64_t seqlen, int64_t nheads, int64_t ngroups, int num_sms) {
+    // fewest idle SM slots over the waves of items, ties to the larger block
+    const int64_t hpg = nheads / ngroups, nch = (seqlen + kQ - 1) / kQ;
+    int best = 1;
+    double best_eff = -1.0;
+    for (int hb = kHB; hb >= 1; --hb) {
+        const int64_t items = nch * batch * ngroups * ((hpg + hb - 1) / hb);
+        const int64_t waves = (items + num_sms - 1) / num_sms;
+        const double eff = (double)items / (double)(waves * num_sms) - 0.02 * (kHB - hb);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = hb;
+        }
+    }
+    return best;
+}
+
+size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads, bool need_state) {
+    const size_t flags = ((size_t)batch * (size_t)nheads + 1) * sizeof(int);
+    const size_t flags_al = (flags + 255) / 256 * 256;
+    return flags_al + (need_state ? (size_t)batch * nheads * kP * kN * sizeof(float) : 0);
+}
+
+cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, int num_sms, cudaStream_t stream) {
+    const int64_t nch = (a.L + kQ - 1) / kQ;
+    if (a.batch <= 0 || nch <= 0) return cudaSuccess;
+    SsdTcArgs w{};
+    w.hb = ssd_tc_head_block(a.batch, a.L, a.H, a.G, num_sms);
+    const int64_t hpg = a.H / a.G;
+    const int64_t items = nch * a.batch * a.G * ((hpg + w.hb - 1) / w.hb);
+    if (items > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    const size_t flags = ((size_t)a.batch * (size_t)a.H + 1) * sizeof(int);
+    const size_t flags_al = (flags + 255) / 256 * 256;
+    w.flags = static_cast<int *>(workspace);
+    w.counter = w.flags + a.batch * a.H;
+    w.state = a.s_last != nullptr ? a.s_last : reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + flags_al);
+    const size_t ysz = out_bf16 ? 2 : 4;
+    w.y_vec16 = ((reinterpret_cast<uintptr_t>(a.y) % 16) == 0 && (a.y_sb * ysz) % 16 == 0 && (a.y_sl * ysz) % 16 == 0 &&
+                 (a.y_sh * ysz) % 16 == 0)
+                    ? 1
+                    : 0;
+    cudaError_t e = cudaMemsetAsync(workspace, 0, flags, stream);
+    if (e != cudaSuccess) return e;
+    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, items, stream) : launch_t<float>(a, w, items, stream);
+}
+
+}  // namespace ms

@@ -229,8 +229,9 @@ def _sdims(**kw):
 
 
 def test_ssd_rejects_bad_arguments(lib):
-    def call(dims, x=FAKE, y=FAKE, B=FAKE):
-        return mb.mamba2_ssd_fwd(x, FAKE, FAKE, B, FAKE, None, None, 1, None, y, None, dims, None, None)
+    def call(dims, x=FAKE, y=FAKE, B=FAKE, ws=None, ws_bytes=0):
+        return mb.mamba2_ssd_fwd(x, FAKE, FAKE, B, FAKE, None, None, 1, None, y, None, dims, ws, ws_bytes, None,
+                                 None)
     assert call(_sdims(headdim=32)) == mb.MS_ERR_SHAPE
     assert call(_sdims(dstate=64)) == mb.MS_ERR_SHAPE
     assert call(_sdims(nheads=5, ngroups=2)) == mb.MS_ERR_SHAPE
@@ -242,6 +243,13 @@ def test_ssd_rejects_bad_arguments(lib):
     assert call(_sdims(B_sl=132)) == mb.MS_ERR_ALIGN         # row stride not a multiple of 8 elements
     assert call(_sdims(), y=FAKE + 4) == mb.MS_ERR_ALIGN      # fp32 pairs need 8-byte alignment
     assert call(_sdims(batch=0)) == mb.MS_OK
+    # the chunk hand-off needs the workspace: flags, counter and (no final_state) the running state
+    need = mb.mamba2_ssd_workspace_size(_sdims(), False)
+    assert need >= 2 * 4 * 64 * 128 * 4 + (2 * 4 + 1) * 4
+    assert mb.mamba2_ssd_workspace_size(_sdims(), True) < need
+    assert call(_sdims()) == mb.MS_ERR_WORKSPACE
+    assert call(_sdims(), ws=FAKE, ws_bytes=need - 1) == mb.MS_ERR_WORKSPACE
+    assert call(_sdims(), ws=FAKE + 8, ws_bytes=need) == mb.MS_ERR_ALIGN
 
 
 def test_ssd_chunk_cb_rejects_bad_arguments(lib):

@@ -40,10 +40,10 @@ def test_ssd_models():
     # x bf16 in, y fp32 out per (token, head, p); dt per (token, head); B, C per (token, group)
     n = bench.ssd_bytes(4, 2048, 80, 64, 128, 1, 2, 4)
     assert n == 4 * 2048 * 80 * (64 * 6 + 2) + 4 * 2048 * 2 * 128 * 2 + 3 * 80 * 4 + 4 * 80 * 64 * 128 * 4
-    # per (b, h, 32-token chunk): C S (Q N P) + C B^T (Q Q N) + G' X (Q Q P) + B'^T X (N Q P), x2
+    # per (b, h, 128-token chunk): C S (Q N P) + C B^T (Q Q N) + G' X (Q Q P) + B'^T X (N Q P), x2
     f = bench.ssd_flops(4, 2048, 80, 64, 128)
-    per = 2 * (32 * 128 * 64 + 32 * 32 * 128 + 32 * 32 * 64 + 128 * 32 * 64)
-    assert f == 4 * 80 * 64 * per
+    per = 2 * (128 * 128 * 64 + 128 * 128 * 128 + 128 * 128 * 64 + 128 * 128 * 64)
+    assert f == 4 * 80 * 16 * per
 
 
 def _free_port():

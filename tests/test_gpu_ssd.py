@@ -39,7 +39,7 @@ def run(inp, s0=None, use_D=True, use_bias=True, softplus=True, out_dtype=torch.
     return y, fs, yr, fr
 
 
-@pytest.mark.parametrize("L", [1, 31, 32, 33, 100, 256])
+@pytest.mark.parametrize("L", [1, 31, 32, 33, 100, 127, 128, 129, 256, 300, 700])
 @pytest.mark.parametrize("G", [1, 2])
 def test_lengths_and_groups(L, G):
     _, inp = _case(2, L, 4, G, 10 + L + G)
@@ -77,6 +77,46 @@ def test_initial_state_and_split():
     torch.cuda.synchronize()
     check_bf16(f64(torch.cat([y1, y2], dim=1)), yr, "split y")
     check_bf16(f64(f2), fr, "split final_state")
+
+
+@pytest.mark.parametrize("b,L,H,G", [(2, 400, 20, 2), (1, 260, 9, 1), (3, 129, 16, 4)])
+def test_head_blocks_and_chunks(b, L, H, G):
+    """Several chunks of 128 tokens and several blocks of heads per group (up
+    to 8 heads per work item, a ragged last block), so chunk k's items take
+    their entering state from chunk k - 1's items of the same heads."""
+    _, inp = _case(b, L, H, G, 30 + L + H)
+    inp["A"] = -torch.exp(torch.randn(H, generator=torch.Generator().manual_seed(L)))  # a decay per head
+    s0 = 0.3 * torch.randn(b, H, 64, 128, generator=torch.Generator().manual_seed(H))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    y, fs = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                       initial_state=s0.to(DEV), dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    yr, fr = oracle.ssd(f64(inp["x"]), f64(inp["dt"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
+                        f64(inp["D"]), f64(inp["dt_bias"]), True, f64(s0))
+    check_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} y")
+    check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
+
+
+def test_state_in_place_and_in_workspace():
+    """initial_state and final_state as one array (updated in place), and no
+    final_state (the running state in the workspace): the same y."""
+    _, inp = _case(2, 300, 8, 1, 40)
+    s0 = 0.3 * torch.randn(2, 8, 64, 128, generator=torch.Generator().manual_seed(5))
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    st = s0.to(DEV).clone()
+    y1, f1 = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                        initial_state=st, final_state=st)
+    y2, f2 = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                        initial_state=s0.to(DEV), return_final_state=False)
+    torch.cuda.synchronize()
+    assert f1.data_ptr() == st.data_ptr() and f2 is None
+    assert torch.equal(y1, y2)
+    yr, fr = oracle.ssd(f64(inp["x"]), f64(inp["dt"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
+                        f64(inp["D"]), f64(inp["dt_bias"]), True, f64(s0))
+    check_bf16(f64(y1), yr, "in-place y")
+    check_bf16(f64(st), fr, "in-place final_state")
 
 
 def test_bf16_output():

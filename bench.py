@@ -589,7 +589,7 @@ def main(argv=None):
     sdims = mb.SsdDims(sw.batch, sw.seqlen, sw.nheads, sw.headdim, sw.dstate, sw.ngroups, *ssd_in[0]["x"].stride()[:3],
                        *ssd_in[0]["dt"].stride()[:2], *ssd_in[0]["B"].stride()[:3], *ssd_in[0]["C"].stride()[:3],
                        *ssd_y.stride()[:3], mb.MS_BF16, mb.MS_F32)
-    ssd_ws = torch.empty(mb.mamba2_ssd_workspace_size(sdims, False), dtype=torch.uint8, device=dev)
+    ssd_ws = torch.empty(mb.mamba2_ssd_workspace_size(sdims), dtype=torch.uint8, device=dev)
 
     def ssd_step(i):
         g = ssd_in[i & 1]

@@ -324,12 +324,13 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
  * be NULL; initial_state may be the same array as final_state.
  * The chunks (128 tokens) run in parallel on the tcgen05 tensor cores; the
  * state entering a chunk is handed over from the previous chunk's work item
- * through final_state (or, when it is NULL, the workspace).
+ * through the workspace.
  *   workspace        caller-owned device memory of mamba2_ssd_workspace_size()
- *                    bytes (for these dims and final_state given or not),
- *                    16-byte aligned; its contents need not be kept between
- *                    calls, but two calls in flight at once need two
- *                    workspaces. Too small: MS_ERR_WORKSPACE.
+ *                    bytes (batch x nheads running states of headdim x dstate
+ *                    fp32 and batch x nheads + 1 counters), 16-byte aligned;
+ *                    its contents need not be kept between calls, but two
+ *                    calls in flight at once need two workspaces. Too small:
+ *                    MS_ERR_WORKSPACE.
  *   dev_status       receives MS_ERR_TIMEOUT if a bounded wait inside the
  *                    kernel ran out (y and final_state are then undefined).
  */
@@ -343,7 +344,7 @@ typedef struct {
     int32_t in_dtype, out_dtype;
 } ms_ssd_dims;
 
-size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dims, int with_final_state);
+size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dims);
 int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C,
                    const float *D, const float *dt_bias, int softplus_flag, const float *initial_state,
                    void *y, float *final_state, const ms_ssd_dims *dims, void *workspace,

@@ -129,7 +129,7 @@ def _load(path: str) -> ctypes.CDLL:
         lib.mamba2_ssd_fwd.argtypes = [_vp] * 7 + [ctypes.c_int, _vp, _vp, _vp, ctypes.POINTER(SsdDims), _vp,
                                                    ctypes.c_size_t, _vp, _vp]
         lib.mamba2_ssd_fwd.restype = ctypes.c_int
-        lib.mamba2_ssd_workspace_size.argtypes = [ctypes.POINTER(SsdDims), ctypes.c_int]
+        lib.mamba2_ssd_workspace_size.argtypes = [ctypes.POINTER(SsdDims)]
         lib.mamba2_ssd_workspace_size.restype = ctypes.c_size_t
         lib.mamba2_ssd_chunk_cb_size.argtypes = [ctypes.POINTER(SsdDims)]
         lib.mamba2_ssd_chunk_cb_size.restype = ctypes.c_size_t
@@ -238,8 +238,8 @@ def mamba2_ssd_chunk_cb(B, C, cb, dims: SsdDims, dev_status=None, stream=None) -
     return library().mamba2_ssd_chunk_cb(B, C, cb, ctypes.byref(dims), dev_status, stream)
 
 
-def mamba2_ssd_workspace_size(dims: SsdDims, with_final_state: bool) -> int:
-    return int(library().mamba2_ssd_workspace_size(ctypes.byref(dims), int(bool(with_final_state))))
+def mamba2_ssd_workspace_size(dims: SsdDims) -> int:
+    return int(library().mamba2_ssd_workspace_size(ctypes.byref(dims)))
 
 
 def mamba2_ssd_fwd(x, dt, A, B, C, D, dt_bias, softplus_flag, initial_state, y, final_state, dims: SsdDims,
@@ -508,7 +508,7 @@ def ssd_fwd(x, dt, A, B, C, D=None, dt_bias=None, softplus: bool = True, initial
     dims = SsdDims(batch, L, H, P, N, G, x.stride(0), x.stride(1), x.stride(2), dt.stride(0), dt.stride(1),
                    B.stride(0), B.stride(1), B.stride(2), C.stride(0), C.stride(1), C.stride(2),
                    y.stride(0), y.stride(1), y.stride(2), _dtype_code(x), _dtype_code(y))
-    ws_bytes = mamba2_ssd_workspace_size(dims, fs is not None)
+    ws_bytes = mamba2_ssd_workspace_size(dims)
     if workspace is None:
         workspace = torch.empty(max(ws_bytes, 16), dtype=torch.uint8, device=x.device)
     rc = mamba2_ssd_fwd(_ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D), _ptr(dt_bias), softplus,

@@ -636,9 +636,9 @@ int mamba_scan_bwd_noalloc(const void *u, const void *delta, const float *A, con
                           need > 0 ? MS_BWD_NOALLOC_MAX_BYTES : 0, dev_status, stream);
 }
 
-size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dm, int with_final_state) {
+size_t mamba2_ssd_workspace_size(const ms_ssd_dims *dm) {
     if (!dm || dm->batch < 0 || dm->nheads < 1) return 0;
-    return ms::ssd_tc_workspace_size(dm->batch, dm->nheads, with_final_state == 0);
+    return ms::ssd_tc_workspace_size(dm->batch, dm->nheads);
 }
 
 int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B, const void *C, const float *D,
@@ -694,7 +694,7 @@ int mamba2_ssd_fwd(const void *x, const void *dt, const float *A, const void *B,
         }
         return MS_OK;
     }
-    const size_t need = ms::ssd_tc_workspace_size(dm->batch, dm->nheads, final_state == nullptr);
+    const size_t need = ms::ssd_tc_workspace_size(dm->batch, dm->nheads);
     if (!workspace || workspace_bytes < need) return MS_ERR_WORKSPACE;
     if (!aligned(workspace, 16)) return MS_ERR_ALIGN;
     ms::SsdArgs a{};

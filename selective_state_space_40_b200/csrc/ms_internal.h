@@ -80,17 +80,19 @@ bool ssd_shape_supported(int64_t headdim, int64_t dstate);
 
 // Chunk-parallel SSD forward on the tcgen05 tensor cores: per-launch state
 // of the chunk hand-off (flags [batch * H] then the ticket counter, zeroed
-// before the launch; the running state [batch, H, P, N], final_state when
-// given), the heads per work item, and whether y rows take 16-byte stores.
+// before the launch; the running state [batch, H, P / 4, N, 4] in the workspace),
+// the index of the last chunk, the heads per work item, and whether y rows
+// take 16-byte stores.
 struct SsdTcArgs {
     int *flags;
     int *counter;
     float *state;
+    int64_t last_chunk;
     int hb;
     int y_vec16;
 };
 int ssd_tc_head_block(int64_t batch, int64_t seqlen, int64_t nheads, int64_t ngroups, int num_sms);
-size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads, bool need_state);
+size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads);
 cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, int num_sms, cudaStream_t stream);
 
 // Arguments of the per-chunk C B^T of the SSD layer (bf16 B, C with dstate

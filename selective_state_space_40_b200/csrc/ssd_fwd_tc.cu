@@ -13,8 +13,9 @@
 //   y_t   = exp(cs_t) sum_n C_t[n] S_in[n][.] + sum_{s<=t} (C_t . B_s) exp(cs_t - cs_s) Delta_s x_s + D x_t
 //   S_out = exp(cs_{Q-1}) S_in + sum_s B_s (w_s x_s)^T,   w_s = exp(cs_{Q-1} - cs_s) Delta_s
 // Four products per chunk and head, each M = 128 on the tensor cores
-// (bf16 x bf16 -> fp32):
-//   CB    [Q x Q] = C B^T                       (once per chunk and group)
+// (bf16 x bf16 -> fp32; CB is formed again for every head, in the tensor
+// memory G' then takes):
+//   CB    [Q x Q] = C B^T
 //   S_c   [N x P] = B^T X'        X'[s] = w_s x_s
 //   Y_i   [Q x P] = G' X          G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s (s <= t)
 //   Y_s   [Q x P] = C S_in
@@ -26,21 +27,27 @@
 // Work item = (chunk k, batch row b, block of up to 8 heads of one group).
 // Items are claimed in ticket order from a global counter, chunk-major, so the
 // item holding chunk k - 1 of the same heads started before this one. Only
-// Y_s and S_out depend on the entering state: each head's item computes
-// CB, S_c and Y_i first, then waits for chunk k - 1's item to publish S_in
-// (a per-(b, h) counter in global memory), writes S_out over it and
-// publishes it for chunk k + 1. The running state lives in final_state (or
-// the workspace) and crosses chunks through L2, so HBM sees each input once.
+// Y_s and S_out depend on the entering state: each head computes CB, S_c and
+// Y_i first, then waits for chunk k - 1's item to publish S_in (a per-(b, h)
+// counter in global memory), writes S_out over it and publishes it for chunk
+// k + 1. The running state lives in the workspace and crosses chunks through
+// L2, so HBM sees each input once.
 //
-// CTA: 8 compute warps (warp w: tensor-memory lanes 32 (w % 4).., column half
-// w / 4) and one MMA warp whose lane 0 issues every tcgen05.mma and commit.
-// Shared-memory operands use the canonical layouts without swizzle (8-row x
-// 16-byte core matrices): K-major for C (and B in C B^T) and G', MN-major for
-// B (in B^T X'), x, X' and S_in -- the same bytes of the B tile serve both of
-// its roles. Every wait is bounded: on a timeout the CTA records
-// MS_ERR_TIMEOUT, stops, waits (bounded) for its issued products and frees its
-// tensor memory.
+// CTA: two groups of 4 compute warps and one MMA warp (lane 0 issues every
+// tcgen05.mma and commit). The groups take alternate heads of the item, each
+// with its own half of tensor memory (a slot: CB, overwritten in place by G'
+// as packed bf16 hi / lo, the A operand of Y_i; S_c, later Y_s; Y_i) and its
+// own x and X' (later S_in) buffers, so one group's products run while the
+// other group computes. In a group, thread t of warp w owns accumulator lane
+// 32 (w % 4) + lane: a token row (CB, G', Y) or a state row (S_c). The MMA
+// warp serves whichever slot is ready. Shared-memory operands use the
+// canonical layouts without swizzle (8-row x 16-byte core matrices): K-major
+// for C (and B in C B^T), MN-major for B (in B^T X'), x, X' and S_in -- the
+// same bytes of the B tile serve both of its roles. Every wait is bounded: on a
+// timeout the CTA records MS_ERR_TIMEOUT, stops, waits (bounded) for its
+// issued products and frees its tensor memory.
 
+#include <algorithm>
 #include <cstdint>
 
 #include "mambascan.h"
@@ -61,26 +68,37 @@ constexpr int kQ = 128;        // tokens per chunk
 constexpr int kP = 64;         // head dim
 constexpr int kN = 128;        // state size
 constexpr int kHB = 8;         // most heads per work item
-constexpr int kComputeThreads = 256;
+constexpr int kGroupWarps = 4;                       // one warp per 32 accumulator lanes
+constexpr int kGroupThreads = 32 * kGroupWarps;
+constexpr int kComputeThreads = 2 * kGroupThreads;
+constexpr int kMmaWarp = 2 * kGroupWarps;
 constexpr int kThreads = kComputeThreads + 32;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColCB = 0, kColSC = 128, kColYI = 192, kColYS = 256;
+constexpr uint32_t kSlotCols = 256;
+// columns inside a slot: CB (fp32, 128), then G' in place -- the 32 tokens s of
+// CB block c (columns 32c..32c+31) become 16 columns of packed hi pairs and 16
+// of lo pairs in the same columns; S_c, then Y_s (64); Y_i (64)
+constexpr uint32_t kColCB = 0, kColSC = 128, kColYI = 192;
+// G' of K-step ks (tokens 16ks..16ks+15), part 0 = hi / 1 = lo
+__host__ __device__ constexpr uint32_t g_col(int ks, int part) {
+    return (uint32_t)(32 * (ks >> 1) + 16 * part + 8 * (ks & 1));
+}
 constexpr uint32_t kSpinTries = 1u << 20;       // mbarrier try_wait rounds
 constexpr uint32_t kFlagTries = 1u << 22;       // polls of a predecessor's counter (with a short sleep)
+constexpr uint32_t kIdleTries = 1u << 24;       // MMA warp polls without an event
 
 // shared-memory map (bytes)
+constexpr int kTileHalf = kQ * kP * 2;            // 16 KB: one [128 x 64] bf16 operand
 constexpr int kOffC = 0;                          // C tile   [t][n] K-major, 32 KB
 constexpr int kOffB = kOffC + kQ * kN * 2;        // B tile   [s][n], 32 KB
-constexpr int kOffX = kOffB + kQ * kN * 2;        // x of two heads [s][p] MN-major, 2 x 16 KB
-constexpr int kOffXP = kOffX + 2 * kQ * kP * 2;   // X' hi / lo, later S_in hi / lo: 2 x 16 KB
-constexpr int kOffG = kOffXP + 2 * kQ * kP * 2;   // G' hi / lo [t][s] K-major: 2 x 32 KB
-constexpr int kOffPar = kOffG + 2 * kQ * kQ * 2;  // dl, cs2, w: [kHB][kQ] floats each
+constexpr int kOffSlot = kOffB + kQ * kN * 2;     // per slot: X' / S_in hi, lo 32 KB; x [s][p] MN-major 16 KB
+constexpr int kSlotBytes = 3 * kTileHalf;
+constexpr int kOffPar = kOffSlot + 2 * kSlotBytes;  // dl, cs2, w: [kHB][kQ] floats each
 constexpr int kOffBar = kOffPar + 3 * kHB * kQ * 4;
-constexpr int kNumBars = 9;
+enum { kBarXP = 0, kBarCB, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarsPerSlot };
+constexpr int kBarLD = 2 * kBarsPerSlot, kBarEnd = kBarLD + 1, kNumBars = kBarEnd + 1;
 constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tensor-memory base, ticket, abort
 constexpr int kSmemBytes = kOffMisc + 16;
-constexpr int kTileHalf = kQ * kP * 2;            // 16 KB: one [128 x 64] bf16 operand
-enum { kBarCB = 0, kBarXP, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarLD, kBarEnd };
 
 // K-major no-swizzle [rows x 128] bf16 tile: core matrix (row / 8, k / 8) at
 // (row / 8) * 2048 + (k / 8) * 128, row % 8 at 16-byte steps inside it.
@@ -154,25 +172,58 @@ __device__ __forceinline__ bool bar_wait(uint32_t bar, uint32_t parity) {
     }
     return false;
 }
-// named barrier 1 over the compute warps, and-reducing a predicate
-__device__ __forceinline__ bool compute_sync_and(bool ok) {
+// Named barrier `id` over `n` threads, and-reducing a predicate: the compute
+// warps (id 1) or one group (id 2 + group).
+template <int kThreadsIn>
+__device__ __forceinline__ bool sync_and(int id, bool ok) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "barrier.cta.red.and.pred q, 1, %2, p;\n\t"
+        "barrier.cta.red.and.pred q, %2, %3, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"(ok ? 1u : 0u), "n"(kComputeThreads)
+        : "r"(ok ? 1u : 0u), "r"(id), "n"(kThreadsIn)
         : "memory");
     return r != 0;
 }
+__device__ __forceinline__ bool bar_test(uint32_t bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+// D (tensor memory) [+]= A (tensor memory) x B (shared memory)
+__device__ __forceinline__ void mma_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t id, bool acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        :
+        : "r"(tmem_d), "r"(tmem_a), "l"(db), "r"(id), "r"(acc ? 1u : 0u)
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15, %16};"
+        :
+        : "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+          "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+__device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cp_async16(uint32_t sdst, const void *gsrc, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sdst), "l"(gsrc), "r"(src_bytes)
                  : "memory");
 }
 __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+__device__ __forceinline__ void cp_wait0() { asm volatile("cp.async.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 __device__ __forceinline__ void tc_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
@@ -234,24 +285,27 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = saddr(smem);
     auto bar = [&](int i) { return sbase + (uint32_t)(kOffBar + 8 * i); };
+    auto sbar = [&](int slot, int e) { return bar(slot * kBarsPerSlot + e); };
     uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kOffMisc);  // [0] tmem base, [1] ticket, [2] abort
     volatile uint32_t *abort_flag = misc + 2;
 
     if (tid == 0) {
         misc[1] = (uint32_t)atomicAdd(w.counter, 1);
         misc[2] = 0u;
-        bar_init(bar(kBarCB), 1);
-        bar_init(bar(kBarXP), 8);
-        bar_init(bar(kBarSC), 1);
-        bar_init(bar(kBarG), 8);
-        bar_init(bar(kBarYI), 1);
-        bar_init(bar(kBarS), 8);
-        bar_init(bar(kBarYS), 1);
+        for (int sl = 0; sl < 2; ++sl) {
+            bar_init(sbar(sl, kBarXP), kGroupWarps);
+            bar_init(sbar(sl, kBarCB), 1);
+            bar_init(sbar(sl, kBarSC), 1);
+            bar_init(sbar(sl, kBarG), kGroupWarps);
+            bar_init(sbar(sl, kBarYI), 1);
+            bar_init(sbar(sl, kBarS), kGroupWarps);
+            bar_init(sbar(sl, kBarYS), 1);
+        }
         bar_init(bar(kBarLD), 1);
         bar_init(bar(kBarEnd), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(sbase + kOffMisc),
                      "r"(kTmemCols)
                      : "memory");
@@ -285,59 +339,84 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
     float *cs2p = dlp + kHB * kQ;                             // [kHB][kQ] cs log2(e)
     float *wp = cs2p + kHB * kQ;                              // [kHB][kQ] w_s
 
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         // ================================ MMA warp ================================
-        bool ok = true;
         if (lane == 0) {
-            const uint32_t sC = sbase + kOffC, sB = sbase + kOffB, sXP = sbase + kOffXP, sG = sbase + kOffG;
-            // CB = C B^T: both K-major [128 x 128], once the C and B tiles are in
-            ok = bar_wait(bar(kBarLD), 0u) && *abort_flag == 0u;
-            if (ok) {
-                tc_after();
+            const uint32_t sC = sbase + kOffC, sB = sbase + kOffB;
+            bool ok = bar_wait(bar(kBarLD), 0u) && *abort_flag == 0u;
+            tc_after();
+            // per slot: its next head and step (0: X' ready -> CB, S_c; 1: G' ready
+            // -> Y_i; 2: S_in ready -> Y_s); slot s takes heads s, s + 2, ...
+            int jn[2] = {0, 1}, step[2] = {0, 0};
+            uint32_t idle = 0;
+            // CB = C B^T (both K-major) into a slot's first 128 columns: issued behind the
+            // slot's previous head's last product (products run in issue order, so
+            // that head's G' has been read), so the group finds it ready
+            auto issue_cb = [&](int sl) {
+                const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
 #pragma unroll 1
                 for (int ks = 0; ks < kN / 16; ++ks)
-                    mma(tmem + kColCB, desc_k(sC + 256u * ks, 128u, 2048u), desc_k(sB + 256u * ks, 128u, 2048u),
+                    mma(tb + kColCB, desc_k(sC + 256u * ks, 128u, 2048u), desc_k(sB + 256u * ks, 128u, 2048u),
                         idesc(kQ, false, false), ks > 0);
-                mma_commit(bar(kBarCB));
+                mma_commit(sbar(sl, kBarCB));
+            };
+            if (ok) {
+                issue_cb(0);
+                if (nh > 1) issue_cb(1);
             }
-            for (int j = 0; j < nh && ok; ++j) {
-                const uint32_t ph = (uint32_t)(j & 1);
-                const uint32_t sX = sbase + kOffX + (uint32_t)((j & 1) * kTileHalf);
-                // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo) N(p)-major
-                ok = bar_wait(bar(kBarXP), ph) && *abort_flag == 0u;
-                if (!ok) break;
-                tc_after();
+            while (ok && (jn[0] < nh || jn[1] < nh)) {
+                bool progressed = false;
 #pragma unroll 1
-                for (int ks = 0; ks < kQ / 16; ++ks)
-#pragma unroll
-                    for (int part = 0; part < 2; ++part)
-                        mma(tmem + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
-                            desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                            idesc(kP, true, true), ks > 0 || part > 0);
-                mma_commit(bar(kBarSC));
-                // Y_i [t x p] = G' X: A = G' (hi, lo) K-major, B = x N(p)-major
-                ok = bar_wait(bar(kBarG), ph) && *abort_flag == 0u;
-                if (!ok) break;
-                tc_after();
+                for (int sl = 0; sl < 2; ++sl) {
+                    const int j = jn[sl];
+                    if (j >= nh) continue;
+                    const uint32_t ph = (uint32_t)((j >> 1) & 1);
+                    const int ev = step[sl] == 0 ? kBarXP : (step[sl] == 1 ? kBarG : kBarS);
+                    if (!bar_test(sbar(sl, ev), ph)) continue;
+                    tc_after();
+                    const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
+                    const uint32_t sXP = sbase + (uint32_t)(kOffSlot + sl * kSlotBytes);
+                    const uint32_t sX = sXP + (uint32_t)(2 * kTileHalf);
+                    if (step[sl] == 0) {
+                        // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo)
 #pragma unroll 1
-                for (int ks = 0; ks < kQ / 16; ++ks)
+                        for (int ks = 0; ks < kQ / 16; ++ks)
 #pragma unroll
-                    for (int part = 0; part < 2; ++part)
-                        mma(tmem + kColYI, desc_k(sG + (uint32_t)(part * 2 * kTileHalf) + 256u * ks, 128u, 2048u),
-                            desc_mn(sX + 2048u * ks, 1024u, 128u), idesc(kP, false, true), ks > 0 || part > 0);
-                mma_commit(bar(kBarYI));
-                // Y_s [t x p] = C S_in: A = C K-major, B = S_in (hi, lo) N(p)-major
-                ok = bar_wait(bar(kBarS), ph) && *abort_flag == 0u;
-                if (!ok) break;
-                tc_after();
+                            for (int part = 0; part < 2; ++part)
+                                mma(tb + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
+                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                    idesc(kP, true, true), ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarSC));
+                    } else if (step[sl] == 1) {
+                        // Y_i [t x p] = G' X: A = G' (hi, lo) packed in tensor memory, B = x
 #pragma unroll 1
-                for (int ks = 0; ks < kN / 16; ++ks)
+                        for (int ks = 0; ks < kQ / 16; ++ks)
 #pragma unroll
-                    for (int part = 0; part < 2; ++part)
-                        mma(tmem + kColYS, desc_k(sC + 256u * ks, 128u, 2048u),
-                            desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                            idesc(kP, false, true), ks > 0 || part > 0);
-                mma_commit(bar(kBarYS));
+                            for (int part = 0; part < 2; ++part)
+                                mma_ts(tb + kColYI, tb + g_col(ks, part),
+                                       desc_mn(sX + 2048u * ks, 1024u, 128u), idesc(kP, false, true),
+                                       ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarYI));
+                    } else {
+                        // Y_s [t x p] = C S_in (hi, lo), into S_c's columns
+#pragma unroll 1
+                        for (int ks = 0; ks < kN / 16; ++ks)
+#pragma unroll
+                            for (int part = 0; part < 2; ++part)
+                                mma(tb + kColSC, desc_k(sC + 256u * ks, 128u, 2048u),
+                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                    idesc(kP, false, true), ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarYS));
+                        if (j + 2 < nh) issue_cb(sl);
+                    }
+                    if (++step[sl] == 3) {
+                        step[sl] = 0;
+                        jn[sl] += 2;
+                    }
+                    progressed = true;
+                }
+                if (progressed) idle = 0;
+                else if (++idle > kIdleTries || *abort_flag != 0u) ok = false;
             }
             if (!ok) {
                 *abort_flag = 1u;
@@ -349,18 +428,22 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         }
         __syncwarp();
     } else {
-        // ============================== compute warps ==============================
-        const int qd = warp & 3, hf = warp >> 2;
-        const int row = 32 * qd + lane;                    // accumulator lane: token t or state n
-        const uint32_t trow = (uint32_t)(32 * qd) << 16;
+        // ============================== compute groups ==============================
+        const int gi = warp / kGroupWarps, qd = warp % kGroupWarps;
+        const int gtid = tid % kGroupThreads;
+        const int gbar = 2 + gi;                                     // the group's named barrier
+        const int row = 32 * qd + lane;                              // accumulator lane: token t or state n
+        const uint32_t tb = tmem + (uint32_t)gi * kSlotCols + ((uint32_t)(32 * qd) << 16);
+        unsigned char *XP = smem + kOffSlot + gi * kSlotBytes;       // X' hi / lo, later S_in hi / lo
+        // x of the group's current head
+        auto x_buf = [&](int) { return XP + 2 * kTileHalf; };
         bool ok = true;
 
-        // chunk tiles: C, B (rows past L zero-filled), x of heads 0 and 1
-        auto load_x = [&](int j) {
+        auto load_x = [&](int j) {  // by the group's threads
             if (j < nh) {
                 const __nv_bfloat16 *xh = xb + (h0 + j) * a.x_sh;
-                const uint32_t dst = sbase + kOffX + (uint32_t)((j & 1) * kTileHalf);
-                for (int i = tid; i < kQ * (kP / 8); i += kComputeThreads) {
+                const uint32_t dst = saddr(x_buf(j));
+                for (int i = gtid; i < kQ * (kP / 8); i += kGroupThreads) {
                     const int s = i >> 3, pc = i & 7;
                     const bool in = t0 + s < L;
                     cp_async16(dst + mn64_off(s, pc), xh + (in ? t0 + s : 0) * a.x_sl + 8 * pc, in ? 16 : 0);
@@ -368,6 +451,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             }
             cp_commit();
         };
+        // chunk tiles: C, B (rows past L zero-filled) by both groups; x of each group's first head
         for (int i = tid; i < kQ * (kN / 8); i += kComputeThreads) {
             const int t = i >> 4, kc = i & 15;
             const bool in = t0 + t < L;
@@ -375,8 +459,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             cp_async16(sbase + kOffC + kmaj_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
             cp_async16(sbase + kOffB + kmaj_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
         }
-        load_x(0);  // group 0: C, B, x of head 0
-        load_x(1);  // group 1: x of head 1 (empty when absent)
+        load_x(gi);
 
         // per-head chunk parameters: warp j < nh takes head h0 + j, 4 tokens per lane
         if (warp < nh) {
@@ -416,32 +499,29 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 wp[warp * kQ + t] = exp2_mufu(cend - c2) * dl[i];
             }
         }
-        cp_wait1();          // this thread's copies of group 0 are in
+        cp_wait0();          // this thread's copies of the tiles and the first x are in
         fence_async_smem();  // ... and visible to the tensor cores
-        // everyone's copies and parameters are in: the MMA warp starts C B^T
-        ok = compute_sync_and(ok);
+        // everyone's copies and parameters are in: the MMA warp may start
+        ok = sync_and<kComputeThreads>(1, ok);
         if (tid == 0) bar_arrive(bar(kBarLD));
 
-        for (int j = 0; j < nh; ++j) {
-            const uint32_t ph = (uint32_t)(j & 1);
+        for (int j = gi; j < nh; j += 2) {
+            const uint32_t ph = (uint32_t)((j >> 1) & 1);
             const int64_t h = h0 + j;
-            const unsigned char *X = smem + kOffX + (j & 1) * kTileHalf;
-            unsigned char *XP = smem + kOffXP;
-            unsigned char *G = smem + kOffG;
             const float *cs2 = cs2p + j * kQ;
-            if (j > 0) {
-                cp_wait1();  // x of head j is in (the newest group may still be in flight)
+            const unsigned char *X = x_buf(j);
+            if (j > gi) {
+                cp_wait0();  // x of head j is in
                 fence_async_smem();
-                ok = compute_sync_and(ok && *abort_flag == 0u);
+                ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
                 if (!ok) break;
             }
-            // ---- X' = w_s x_s (row s, columns p of this half), hi / lo
+            // ---- X' = w_s x_s (row s, all 64 columns p), hi / lo
             {
                 const int s = row;
                 const float ws = wp[j * kQ + s];
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int pc = 4 * hf + q;
+                for (int pc = 0; pc < 8; ++pc) {
                     float v[8];
                     unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(s, pc)), v);
 #pragma unroll
@@ -454,56 +534,59 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             }
             fence_async_smem();
             __syncwarp();
-            if (lane == 0) bar_arrive(bar(kBarXP));
+            if (lane == 0) bar_arrive(sbar(gi, kBarXP));
 
-            // ---- G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s for s <= t (s in this half), hi / lo
-            if (j == 0) {
-                ok = __all_sync(0xffffffffu, bar_wait(bar(kBarCB), 0u));
-                tc_after();
-            }
+            // ---- G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s for s <= t, hi / lo packed
+            // in place of CB, one 32-column block at a time; blocks entirely above
+            // the diagonal are zeros
+            ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarCB), ph));
+            tc_after();
             {
                 const int t = row;
                 const float ct = cs2[t];
                 const float *dls = dlp + j * kQ;
-                const bool zero_half = hf == 1 && qd < 2;  // s >= 64 > t for every lane of the warp
-#pragma unroll
-                for (int c32 = 0; c32 < 2; ++c32) {
-                    float v[32];
-                    if (!zero_half && ok) {
-                        tmem_ld32(tmem + trow + kColCB + (uint32_t)(64 * hf + 32 * c32), v);
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t hi[16], lo[16];
+                    if (c <= qd && ok) {
+                        float v[32];
+                        tmem_ld32(tb + kColCB + (uint32_t)(32 * c), v);
 #pragma unroll
                         for (int e = 0; e < 32; ++e) {
-                            const int s = 64 * hf + 32 * c32 + e;
-                            v[e] = s <= t ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                            const int s = 32 * c + e;
+                            v[e] = (c < qd || s <= t) ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                        }
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) {
+                            const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                            hi[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                            lo[e] = pack2(v[2 * e] - __low2float(hh), v[2 * e + 1] - __high2float(hh));
                         }
                     } else {
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) v[e] = 0.0f;
+                        for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
                     }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        const int kc = 8 * hf + 4 * c32 + q;
-                        uint4 hi, lo;
-                        split8(v + 8 * q, hi, lo);
-                        *reinterpret_cast<uint4 *>(G + kmaj_off(t, kc)) = hi;
-                        *reinterpret_cast<uint4 *>(G + 2 * kTileHalf + kmaj_off(t, kc)) = lo;
-                    }
+                    tmem_st16(tb + kColCB + (uint32_t)(32 * c), hi);
+                    tmem_st16(tb + kColCB + (uint32_t)(32 * c + 16), lo);
                 }
             }
-            fence_async_smem();
+            tmem_st_wait();
             tc_before();
             __syncwarp();
-            if (lane == 0) bar_arrive(bar(kBarG));
+            if (lane == 0) bar_arrive(sbar(gi, kBarG));
 
-            // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out
-            ok = __all_sync(0xffffffffu, ok && bar_wait(bar(kBarSC), ph));
+            // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out. The
+            // running state is [p / 4][n][4] per head in the workspace (a warp's 16-byte
+            // loads of one p-quad are contiguous); the first chunk reads
+            // initial_state [p][n], the last one also writes final_state [p][n].
+            ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarSC), ph));
             tc_after();
             {
                 int *flag = w.flags + (b * a.H + h);
                 if (k > 0 && ok) {
                     uint32_t i = 0;
                     while (ld_acquire(flag) < (int)k && i < kFlagTries) {
-                        __nanosleep(64);
+                        __nanosleep(32);
                         ++i;
                     }
                     ok = i < kFlagTries;
@@ -511,94 +594,119 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 ok = __all_sync(0xffffffffu, ok);
                 const int n = row;
                 const size_t blk = (size_t)(b * a.H + h) * kP * kN;
-                float *st = w.state + blk;
-                const float *sin = k > 0 ? st : (a.s0 ? a.s0 + blk : nullptr);
+                float4 *run4 = reinterpret_cast<float4 *>(w.state + blk) + n;  // quad q at run4[q * kN]
                 const float decay = exp2_mufu(cs2[kQ - 1]);
-                float sc[32];
-                if (ok) tmem_ld32(tmem + trow + kColSC + (uint32_t)(32 * hf), sc);
+                // every S_in load of the row issued before any S_out store
+                float sv[64];
+                if (ok && k > 0) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float v[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int p = 32 * hf + 8 * q + e;
-                        v[e] = (sin != nullptr && ok) ? sin[(size_t)p * kN + n] : 0.0f;
+                    for (int q = 0; q < 16; ++q) {
+                        const float4 v4 = run4[q * kN];
+                        sv[4 * q] = v4.x; sv[4 * q + 1] = v4.y; sv[4 * q + 2] = v4.z; sv[4 * q + 3] = v4.w;
                     }
-                    if (ok) {
+                } else {
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int p = 32 * hf + 8 * q + e;
-                            st[(size_t)p * kN + n] = fmaf(decay, v[e], sc[8 * q + e]);
+                    for (int e = 0; e < 64; ++e) sv[e] = (ok && a.s0) ? a.s0[blk + (size_t)e * kN + n] : 0.0f;
+                }
+#pragma unroll
+                for (int half = 0; half < 2; ++half) {
+                    if (ok) {
+                        float sc[32];
+                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), sc);
+                        float so[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) so[e] = fmaf(decay, sv[32 * half + e], sc[e]);
+#pragma unroll
+                        for (int q = 0; q < 8; ++q)
+                            run4[(8 * half + q) * kN] = make_float4(so[4 * q], so[4 * q + 1], so[4 * q + 2], so[4 * q + 3]);
+                        if (w.last_chunk == k && a.s_last != nullptr) {
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) a.s_last[blk + (size_t)(32 * half + e) * kN + n] = so[e];
                         }
                     }
-                    uint4 hi, lo;
-                    split8(v, hi, lo);
-                    const int pc = 4 * hf + q;
-                    *reinterpret_cast<uint4 *>(XP + mn64_off(n, pc)) = hi;
-                    *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(n, pc)) = lo;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 hi, lo;
+                        split8(sv + 32 * half + 8 * q, hi, lo);
+                        const int pc = 4 * half + q;
+                        *reinterpret_cast<uint4 *>(XP + mn64_off(n, pc)) = hi;
+                        *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(n, pc)) = lo;
+                    }
                 }
                 fence_async_smem();
                 tc_before();
-                // every compute thread's S_out is stored: publish it for chunk k + 1
-                ok = compute_sync_and(ok);
-                if (tid == 0 && ok) {
-                    __threadfence();
-                    st_release(flag, (int)k + 1);
-                }
+                // the group's S_out is stored: publish it for chunk k + 1 (the release
+                // orders the group's stores, which the barrier put before it)
+                ok = sync_and<kGroupThreads>(gbar, ok);
+                if (gtid == 0 && ok) st_release(flag, (int)k + 1);
             }
             __syncwarp();
-            if (lane == 0) bar_arrive(bar(kBarS));
+            if (lane == 0) bar_arrive(sbar(gi, kBarS));
             if (!ok) break;
 
-            // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t
-            ok = __all_sync(0xffffffffu, bar_wait(bar(kBarYI), ph) && bar_wait(bar(kBarYS), ph));
+            // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t (row t, all 64 columns p): Y_i and
+            // D x first, while Y_s is still being formed
+            ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYI), ph));
             tc_after();
             if (ok) {
                 const int t = row;
-                float ys[32], yi[32];
-                tmem_ld32(tmem + trow + kColYS + (uint32_t)(32 * hf), ys);
-                tmem_ld32(tmem + trow + kColYI + (uint32_t)(32 * hf), yi);
                 const float et = exp2_mufu(cs2[t]);
                 const float Dh = a.D ? __ldg(a.D + h) : 0.0f;
-                if (t0 + t < L) {
-                    TOut *yp = static_cast<TOut *>(a.y) + b * a.y_sb + (t0 + t) * a.y_sl + h * a.y_sh + 32 * hf;
+                TOut *yp = static_cast<TOut *>(a.y) + b * a.y_sb + (t0 + t) * a.y_sl + h * a.y_sh;
+                float yi[64];
+                tmem_ld32(tb + kColYI, *reinterpret_cast<float(*)[32]>(yi));
+                tmem_ld32(tb + kColYI + 32u, *reinterpret_cast<float(*)[32]>(yi + 32));
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float xv[8], yo[8];
-                        unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(t, 4 * hf + q)), xv);
+                for (int pc = 0; pc < 8; ++pc) {
+                    float xv[8];
+                    unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(t, pc)), xv);
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], fmaf(Dh, xv[e], yi[8 * q + e]));
-                        if constexpr (sizeof(TOut) == 4) {
-                            if (w.y_vec16) {
-                                float4 *p4 = reinterpret_cast<float4 *>(yp + 8 * q);
-                                p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
-                                p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                    for (int e = 0; e < 8; ++e) yi[8 * pc + e] = fmaf(Dh, xv[e], yi[8 * pc + e]);
+                }
+                ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYS), ph));
+                tc_after();
+#pragma unroll
+                for (int half = 0; half < 2 && ok; ++half) {
+                    float ys[32];
+                    tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
+                    if (t0 + t < L) {
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            float yo[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], yi[32 * half + 8 * q + e]);
+                            TOut *yq = yp + 32 * half + 8 * q;
+                            if constexpr (sizeof(TOut) == 4) {
+                                if (w.y_vec16) {
+                                    float4 *p4 = reinterpret_cast<float4 *>(yq);
+                                    p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
+                                    p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                                } else {
+                                    float2 *p2 = reinterpret_cast<float2 *>(yq);
+#pragma unroll
+                                    for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
+                                }
                             } else {
-                                float2 *p2 = reinterpret_cast<float2 *>(yp + 8 * q);
+                                if (w.y_vec16) {
+                                    *reinterpret_cast<uint4 *>(yq) = make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]),
+                                                                                pack2(yo[4], yo[5]), pack2(yo[6], yo[7]));
+                                } else {
+                                    uint32_t *p1 = reinterpret_cast<uint32_t *>(yq);
 #pragma unroll
-                                for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
-                            }
-                        } else {
-                            if (w.y_vec16) {
-                                *reinterpret_cast<uint4 *>(yp + 8 * q) =
-                                    make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]), pack2(yo[4], yo[5]),
-                                               pack2(yo[6], yo[7]));
-                            } else {
-                                uint32_t *p1 = reinterpret_cast<uint32_t *>(yp + 8 * q);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                    for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                }
                             }
                         }
                     }
                 }
             }
             tc_before();
-            // every compute thread is done with x of head j: its buffer takes head j + 2
-            ok = compute_sync_and(ok && *abort_flag == 0u);
+            // the group is done with x of head j: the buffer takes head j + 2
+            ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
             if (!ok) break;
             load_x(j + 2);
         }
-        if (!ok && tid == 0) {
+        if (!ok && gtid == 0) {
             *abort_flag = 1u;
             if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
         }
@@ -608,7 +716,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
     // ---- tear-down: the MMA warp has drained its products; free the tensor memory
     tc_before();
     __syncthreads();
-    if (warp == 8) {
+    if (warp == kMmaWarp) {
         tc_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
                      : "memory");
@@ -629,26 +737,28 @@ cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, int64_t items, cudaSt
 bool ssd_shape_supported(int64_t headdim, int64_t dstate) { return headdim == kP && dstate == kN; }
 
 int ssd_tc_head_block(int64_t batch, int64_t seqlen, int64_t nheads, int64_t ngroups, int num_sms) {
-    // fewest idle SM slots over the waves of items, ties to the larger block
+    // time ~ waves x (item start + head steps of the busier group), a head step
+    // costing about 2.3 item starts (measured on the 2.7B-class layer)
     const int64_t hpg = nheads / ngroups, nch = (seqlen + kQ - 1) / kQ;
     int best = 1;
-    double best_eff = -1.0;
+    double best_cost = 1e300;
     for (int hb = kHB; hb >= 1; --hb) {
         const int64_t items = nch * batch * ngroups * ((hpg + hb - 1) / hb);
         const int64_t waves = (items + num_sms - 1) / num_sms;
-        const double eff = (double)items / (double)(waves * num_sms) - 0.02 * (kHB - hb);
-        if (eff > best_eff + 1e-9) {
-            best_eff = eff;
+        const int steps = (int)((std::min<int64_t>(hb, hpg) + 1) / 2);
+        const double cost = (double)waves * (1.0 + 2.3 * steps);
+        if (cost < best_cost - 1e-9) {
+            best_cost = cost;
             best = hb;
         }
     }
     return best;
 }
 
-size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads, bool need_state) {
+size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads) {
     const size_t flags = ((size_t)batch * (size_t)nheads + 1) * sizeof(int);
     const size_t flags_al = (flags + 255) / 256 * 256;
-    return flags_al + (need_state ? (size_t)batch * nheads * kP * kN * sizeof(float) : 0);
+    return flags_al + (size_t)batch * nheads * kP * kN * sizeof(float);
 }
 
 cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, int num_sms, cudaStream_t stream) {
@@ -663,7 +773,8 @@ cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, 
     const size_t flags_al = (flags + 255) / 256 * 256;
     w.flags = static_cast<int *>(workspace);
     w.counter = w.flags + a.batch * a.H;
-    w.state = a.s_last != nullptr ? a.s_last : reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + flags_al);
+    w.state = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + flags_al);
+    w.last_chunk = nch - 1;
     const size_t ysz = out_bf16 ? 2 : 4;
     w.y_vec16 = ((reinterpret_cast<uintptr_t>(a.y) % 16) == 0 && (a.y_sb * ysz) % 16 == 0 && (a.y_sl * ysz) % 16 == 0 &&
                  (a.y_sh * ysz) % 16 == 0)

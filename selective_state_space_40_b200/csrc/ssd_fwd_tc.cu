@@ -47,8 +47,12 @@
 // timeout the CTA records MS_ERR_TIMEOUT, stops, waits (bounded) for its
 // issued products and frees its tensor memory.
 
+#include <cuda.h>
+
 #include <algorithm>
 #include <cstdint>
+#include <cstring>
+#include <mutex>
 
 #include "mambascan.h"
 #include "ms_device.cuh"
@@ -217,6 +221,15 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
           "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+// Tensor store (no multicast) of a 4-D box from shared memory, and its groups
+__device__ __forceinline__ void tma_store4(const CUtensorMap *map, uint32_t src, int c0, int c1, int c2, int c3) {
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(map),
+                 "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cp_async16(uint32_t sdst, const void *gsrc, int src_bytes) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(sdst), "l"(gsrc), "r"(src_bytes)
@@ -280,7 +293,8 @@ __device__ __forceinline__ void st_release(int *p, int v) {
 }
 
 template <typename TOut>
-__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a, const SsdTcArgs w) {
+__global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a, const SsdTcArgs w,
+                                                                  const __grid_constant__ CUtensorMap ymap) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = saddr(smem);
@@ -513,6 +527,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             if (j > gi) {
                 cp_wait0();  // x of head j is in
                 fence_async_smem();
+                if (gtid == 0 && w.y_tma) bulk_wait_read0();  // the previous head's y has left the staging buffer
                 ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
                 if (!ok) break;
             }
@@ -665,39 +680,83 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 }
                 ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYS), ph));
                 tc_after();
+                if (w.y_tma) {
+                    // y row t into the staging buffer (S_in has been consumed by Y_s) in the
+                    // tensor map's box layout: rows of 128 bytes, 16-byte chunk i of row t
+                    // at chunk i ^ (t % 8) (128-byte swizzle); fp32: two boxes of 32
+                    // columns, bf16: one box of 64
 #pragma unroll
-                for (int half = 0; half < 2 && ok; ++half) {
-                    float ys[32];
-                    tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
-                    if (t0 + t < L) {
+                    for (int half = 0; half < 2 && ok; ++half) {
+                        float ys[32];
+                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
 #pragma unroll
-                        for (int q = 0; q < 4; ++q) {
-                            float yo[8];
+                        for (int e = 0; e < 32; ++e) yi[32 * half + e] = fmaf(et, ys[e], yi[32 * half + e]);
+                    }
+                    if constexpr (sizeof(TOut) == 4) {
 #pragma unroll
-                            for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], yi[32 * half + 8 * q + e]);
-                            TOut *yq = yp + 32 * half + 8 * q;
-                            if constexpr (sizeof(TOut) == 4) {
-                                if (w.y_vec16) {
-                                    float4 *p4 = reinterpret_cast<float4 *>(yq);
-                                    p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
-                                    p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                        for (int c = 0; c < 2; ++c)
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                *reinterpret_cast<float4 *>(XP + c * kTileHalf + t * 128 + ((i ^ (t & 7)) << 4)) =
+                                    make_float4(yi[32 * c + 4 * i], yi[32 * c + 4 * i + 1], yi[32 * c + 4 * i + 2],
+                                                yi[32 * c + 4 * i + 3]);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            *reinterpret_cast<uint4 *>(XP + t * 128 + ((i ^ (t & 7)) << 4)) =
+                                make_uint4(pack2(yi[8 * i], yi[8 * i + 1]), pack2(yi[8 * i + 2], yi[8 * i + 3]),
+                                           pack2(yi[8 * i + 4], yi[8 * i + 5]), pack2(yi[8 * i + 6], yi[8 * i + 7]));
+                    }
+                    fence_async_smem();
+                } else {
+    #pragma unroll
+                    for (int half = 0; half < 2 && ok; ++half) {
+                        float ys[32];
+                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
+                        if (t0 + t < L) {
+    #pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                float yo[8];
+    #pragma unroll
+                                for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], yi[32 * half + 8 * q + e]);
+                                TOut *yq = yp + 32 * half + 8 * q;
+                                if constexpr (sizeof(TOut) == 4) {
+                                    if (w.y_vec16) {
+                                        float4 *p4 = reinterpret_cast<float4 *>(yq);
+                                        p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
+                                        p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                                    } else {
+                                        float2 *p2 = reinterpret_cast<float2 *>(yq);
+    #pragma unroll
+                                        for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
+                                    }
                                 } else {
-                                    float2 *p2 = reinterpret_cast<float2 *>(yq);
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
-                                }
-                            } else {
-                                if (w.y_vec16) {
-                                    *reinterpret_cast<uint4 *>(yq) = make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]),
-                                                                                pack2(yo[4], yo[5]), pack2(yo[6], yo[7]));
-                                } else {
-                                    uint32_t *p1 = reinterpret_cast<uint32_t *>(yq);
-#pragma unroll
-                                    for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                    if (w.y_vec16) {
+                                        *reinterpret_cast<uint4 *>(yq) = make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]),
+                                                                                    pack2(yo[4], yo[5]), pack2(yo[6], yo[7]));
+                                    } else {
+                                        uint32_t *p1 = reinterpret_cast<uint32_t *>(yq);
+    #pragma unroll
+                                        for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                    }
                                 }
                             }
                         }
                     }
+                }
+                }
+            if (w.y_tma) {
+                // every thread of the group has staged its row (or given up): one thread
+                // stores the tile (rows past the sequence are outside the map, not written)
+                ok = sync_and<kGroupThreads>(gbar, ok);
+                if (gtid == 0 && ok) {
+                    if constexpr (sizeof(TOut) == 4) {
+                        tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
+                        tma_store4(&ymap, saddr(XP) + kTileHalf, 32, (int)h, (int)t0, (int)b);
+                    } else {
+                        tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
+                    }
+                    bulk_commit();
                 }
             }
             tc_before();
@@ -711,6 +770,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
         }
         asm volatile("cp.async.wait_all;" ::: "memory");
+        if (gtid == 0 && w.y_tma) bulk_wait0();
     }
 
     // ---- tear-down: the MMA warp has drained its products; free the tensor memory
@@ -724,12 +784,49 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
 }
 
 template <typename TOut>
-cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, int64_t items, cudaStream_t stream) {
+cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, const CUtensorMap &ymap, int64_t items,
+                     cudaStream_t stream) {
     static SmemOptIn opt_in;
     cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_fwd_tc_kernel<TOut>), kSmemBytes);
     if (e != cudaSuccess) return e;
-    ssd_fwd_tc_kernel<TOut><<<(unsigned)items, kThreads, kSmemBytes, stream>>>(a, w);
+    ssd_fwd_tc_kernel<TOut><<<(unsigned)items, kThreads, kSmemBytes, stream>>>(a, w, ymap);
     return cudaGetLastError();
+}
+
+using PfnEncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+PfnEncodeTiled encode_fn() {
+    static std::once_flag once;
+    static PfnEncodeTiled fn = nullptr;
+    std::call_once(once, [] {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PfnEncodeTiled>(f);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// y [batch][L][H][64] as a 4-D map {p, h, t, b}: box {128 bytes of p, 1 head,
+// 128 tokens, 1 row}, 128-byte swizzle; rows t >= L lie outside the map.
+bool encode_y(CUtensorMap *m, const SsdArgs &a, bool bf16) {
+    PfnEncodeTiled fn = encode_fn();
+    if (!fn) return false;
+    const uint64_t es = bf16 ? 2 : 4;
+    const uint64_t sh = (uint64_t)a.y_sh * es, sl = (uint64_t)a.y_sl * es;
+    const uint64_t sb = a.batch > 1 ? (uint64_t)a.y_sb * es : sl * (uint64_t)a.L;
+    if (sh == 0 || sl == 0 || sb == 0) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)kP, (cuuint64_t)a.H, (cuuint64_t)a.L, (cuuint64_t)a.batch};
+    const cuuint64_t strides[3] = {(cuuint64_t)sh, (cuuint64_t)sl, (cuuint64_t)sb};
+    const cuuint32_t box[4] = {(cuuint32_t)(128 / es), 1u, (cuuint32_t)kQ, 1u};
+    const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+    return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.y, dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -780,9 +877,15 @@ cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, 
                  (a.y_sh * ysz) % 16 == 0)
                     ? 1
                     : 0;
+    CUtensorMap ymap;
+    memset(&ymap, 0, sizeof(ymap));
+    w.y_tma = (w.y_vec16 && a.H <= 0x7fffffff && a.L <= 0x7fffffff && a.batch <= 0x7fffffff &&
+               encode_y(&ymap, a, out_bf16))
+                  ? 1
+                  : 0;
     cudaError_t e = cudaMemsetAsync(workspace, 0, flags, stream);
     if (e != cudaSuccess) return e;
-    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, items, stream) : launch_t<float>(a, w, items, stream);
+    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, ymap, items, stream) : launch_t<float>(a, w, ymap, items, stream);
 }
 
 }  // namespace ms

@@ -119,6 +119,25 @@ def test_state_in_place_and_in_workspace():
     check_bf16(f64(st), fr, "in-place final_state")
 
 
+@pytest.mark.parametrize("out_dtype", [torch.float32, torch.bfloat16])
+def test_output_rows_not_16_byte_aligned(out_dtype):
+    """y as a view whose head rows are 66 elements apart: the kernel stores the
+    rows directly instead of through the tensor map."""
+    _, inp = _case(2, 200, 4, 1, 75)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    ybuf = torch.full((2, 200, 4, 66), float("nan"), dtype=out_dtype, device=DEV)
+    y = ybuf[..., :64]
+    mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True, y=y, return_final_state=False)
+    torch.cuda.synchronize()
+    assert torch.isnan(ybuf[..., 64:].float()).all()  # the gaps are untouched
+    yr, _ = oracle.ssd(f64(inp["x"]), f64(inp["dt"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]), f64(inp["D"]),
+                       f64(inp["dt_bias"]), True)
+    if out_dtype == torch.bfloat16:
+        check_out_bf16(f64(y), yr, "strided bf16 y")
+    else:
+        check_bf16(f64(y), yr, "strided y")
+
+
 def test_bf16_output():
     _, inp = _case(1, 96, 4, 1, 70)
     y, _, yr, _ = run(inp, out_dtype=torch.bfloat16)

@@ -290,7 +290,7 @@ def forward_leg(torch, mb, syn, w, stream, dev, local, world, peak, steps, nsets
     nb = scan_bytes(w.batch, w.dim, w.dstate, w.seqlen, es, 4)
     gbs = nb / (ms * 1e-3) / 1e9
     rc, pl = mb.mamba_scan_choose_plan(dims)
-    plan = [pl.lanes_per_channel, pl.chunks_per_lane, pl.poly8] if rc == mb.MS_OK else None
+    plan = [pl.lanes_per_channel, pl.chunks_per_lane, pl.poly8, pl.engine] if rc == mb.MS_OK else None
     out = {"workload": w.name, "ms": ms, "bytes": nb, "value": gbs, "unit": "GB/s",
            "gct_per_s": w.channel_tokens / (ms * 1e-3) / 1e9, "frac": gbs / peak,
            "frac_of_nominal": gbs / NOMINAL_HBM_GBS, "traffic": recorded_traffic(traffic_key),
@@ -443,6 +443,10 @@ def main(argv=None):
     peak, peak_kind = measured_peaks()
     achieved = nbytes / (kernel_ms * 1e-3) / 1e9
     traffic = recorded_traffic("scan_fwd_130m")
+    main_dims = mb.scan_dims_for(sets[0]["u"], sets[0]["delta"], sets[0]["B"], sets[0]["C"], sets[0]["z"], y)
+    prc, mpl = mb.mamba_scan_choose_plan(main_dims)
+    main_kernel = ("scan_fwd_tmem_kernel" if prc == mb.MS_OK and mpl.engine == mb.MS_ENGINE_TMEM
+                   else "scan_fwd_kernel")
 
     # ---- end to end through the public API with host buffers: every step
     # copies its inputs from pinned host memory, scans, and copies y and
@@ -669,7 +673,7 @@ def main(argv=None):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "peak_source": f"{peak_kind} hbm_gbs (copy, burst)",
-                         "kernel": "scan_fwd_kernel", "bytes_per_launch": nbytes,
+                         "kernel": main_kernel, "bytes_per_launch": nbytes,
                          "kernel_ms": kernel_ms, "nominal_peak": NOMINAL_HBM_GBS,
                          "frac_of_nominal": achieved / NOMINAL_HBM_GBS,
                          "traffic_over_bytes": None if traffic is None else traffic / nbytes},

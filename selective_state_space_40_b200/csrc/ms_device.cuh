@@ -216,12 +216,44 @@ __device__ __forceinline__ f2 exp2_pair(f2 x2) {
 }
 
 // -------------------------------------------------------- softplus / silu --
-// softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1]. For e < 1/16
-// log1p(e) comes from its alternating series to e^6/6 (next term < 5e-10
-// relative); above that from log2(1 + e), where the rounding of 1 + e costs at
-// most ~2e-6 relative. Large |v| therefore stays accurate on both sides.
-__device__ __forceinline__ float softplus_f(float v) {
-    const float e = exp2_mufu(-fabsf(v) * kLog2e);
+// Both take one exponential on the MUFU pipe and the rest on the FMA pipe
+// (MS_FMA_NONLIN 0: the logarithm and reciprocal on MUFU as well).
+#ifndef MS_FMA_NONLIN
+#define MS_FMA_NONLIN 1
+#endif
+
+// log1p(e) / e on [0, 1]: the degree-9 polynomial through the Chebyshev
+// nodes of the interval (fitted here in fp64, rounded to fp32). Evaluated in
+// fp32, e * p(e) is within 1.6e-7 relative of log1p(e) on the whole interval,
+// so no separate form is needed near 0 or near 1.
+struct Log1pOverX {
+    static constexpr float c0 = 1.0f;
+    static constexpr float c1 = -0.49999892711639404f;
+    static constexpr float c2 = 0.33329710364341736f;
+    static constexpr float c3 = -0.24951615929603577f;
+    static constexpr float c4 = 0.1966327428817749f;
+    static constexpr float c5 = -0.1526966691017151f;
+    static constexpr float c6 = 0.10543623566627502f;
+    static constexpr float c7 = -0.056373611092567444f;
+    static constexpr float c8 = 0.019542526453733444f;
+    static constexpr float c9 = -0.0031760570127516985f;
+};
+
+// softplus(v) = max(v, 0) + log1p(e), e = exp(-|v|) in (0, 1] (given): accurate
+// at both tails (large |v|: e -> 0 and the polynomial's relative accuracy holds).
+__device__ __forceinline__ float softplus_e(float v, float e) {
+#if MS_FMA_NONLIN
+    float p = fmaf(Log1pOverX::c9, e, Log1pOverX::c8);
+    p = fmaf(p, e, Log1pOverX::c7);
+    p = fmaf(p, e, Log1pOverX::c6);
+    p = fmaf(p, e, Log1pOverX::c5);
+    p = fmaf(p, e, Log1pOverX::c4);
+    p = fmaf(p, e, Log1pOverX::c3);
+    p = fmaf(p, e, Log1pOverX::c2);
+    p = fmaf(p, e, Log1pOverX::c1);
+    p = fmaf(p, e, Log1pOverX::c0);
+    return fmaxf(v, 0.0f) + e * p;
+#else
     float s = fmaf(e, -1.0f / 6.0f, 0.2f);
     s = fmaf(e, s, -0.25f);
     s = fmaf(e, s, 1.0f / 3.0f);
@@ -230,11 +262,31 @@ __device__ __forceinline__ float softplus_f(float v) {
     const float series = e * s;
     const float logform = log2_mufu(1.0f + e) * kLn2;
     return fmaxf(v, 0.0f) + (e < 0.0625f ? series : logform);
+#endif
+}
+__device__ __forceinline__ float softplus_f(float v) { return softplus_e(v, exp2_mufu(-fabsf(v) * kLog2e)); }
+
+// 1 / d for d in [1, 2] by Newton's iteration for the reciprocal: the linear
+// seed 24/17 - 8/17 d (relative error at most 1/17 on the interval), then
+// three steps r <- r + r (1 - d r), each squaring the relative error
+// (fp32 result within 9e-8 relative).
+__device__ __forceinline__ float rcp_1to2(float d) {
+    float r = fmaf(-8.0f / 17.0f, d, 24.0f / 17.0f);
+#pragma unroll
+    for (int i = 0; i < 3; ++i) r = fmaf(r, fmaf(-d, r, 1.0f), r);
+    return r;
 }
 
-// silu(z) = z * sigmoid(z) = z / (1 + exp(-z)).
+// silu(z) = z sigma(z); sigma from e = exp(-|z|) in (0, 1]: 1 / (1 + e) for
+// z >= 0, e / (1 + e) below, so the reciprocal always sees d in [1, 2].
 __device__ __forceinline__ float silu_f(float z) {
+#if MS_FMA_NONLIN
+    const float e = exp2_mufu(-fabsf(z) * kLog2e);
+    const float r = rcp_1to2(1.0f + e);
+    return z * (z >= 0.0f ? r : e * r);
+#else
     return z * rcp_mufu(1.0f + exp2_mufu(-z * kLog2e));
+#endif
 }
 
 }  // namespace ms

@@ -176,15 +176,23 @@ __device__ __forceinline__ void reduce_scatter_lanes(float (&v)[8], int g) {
 // (same series / logarithm split as the forward's softplus).
 __device__ __forceinline__ void softplus_and_grad(float v, float &sp, float &sig) {
     const float e = exp2_mufu(-fabsf(v) * kLog2e);
-    float s = fmaf(e, -1.0f / 6.0f, 0.2f);
-    s = fmaf(e, s, -0.25f);
-    s = fmaf(e, s, 1.0f / 3.0f);
-    s = fmaf(e, s, -0.5f);
-    s = fmaf(e, s, 1.0f);
-    const float lp = e < 0.0625f ? e * s : log2_mufu(1.0f + e) * kLn2;
-    sp = fmaxf(v, 0.0f) + lp;
+    sp = softplus_e(v, e);
+#if MS_FMA_NONLIN
+    const float r = rcp_1to2(1.0f + e);
+#else
     const float r = rcp_mufu(1.0f + e);
+#endif
     sig = v >= 0.0f ? r : e * r;
+}
+// the logistic function sigma(z)
+__device__ __forceinline__ float logistic_f(float z) {
+#if MS_FMA_NONLIN
+    const float e = exp2_mufu(-fabsf(z) * kLog2e);
+    const float r = rcp_1to2(1.0f + e);
+    return z >= 0.0f ? r : e * r;
+#else
+    return rcp_mufu(1.0f + exp2_mufu(-z * kLog2e));
+#endif
 }
 
 struct F4 { float v[4]; };
@@ -302,7 +310,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 float gt = 1.0f, gp = 0.0f;
                 if (has_z) {
                     const float zz = zv[j];
-                    const float sz = rcp_mufu(1.0f + exp2_mufu(-zz * kLog2e));
+                    const float sz = logistic_f(zz);
                     gt = zz * sz;
                     gp = sz * (1.0f + zz * (1.0f - sz));
                 }

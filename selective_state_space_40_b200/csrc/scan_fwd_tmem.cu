@@ -344,9 +344,39 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&h2);
 }
 
+// One input element as fp32.
+template <typename T>
+__device__ __forceinline__ float ld_in(const T *p) {
+    if constexpr (sizeof(T) == 4) return __ldg(reinterpret_cast<const float *>(p));
+    else return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)));
+}
+// 8 fp32 values stored as 8 consecutive input-dtype elements (one or two
+// 16-byte stores when the row allows, else element stores).
+template <typename T>
+__device__ __forceinline__ void store8_in(T *p, bool vec, const float (&v)[8]) {
+    if constexpr (sizeof(T) == 4) {
+        if (vec) {
+            reinterpret_cast<float4 *>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+            reinterpret_cast<float4 *>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) reinterpret_cast<float *>(p)[j] = v[j];
+        }
+    } else {
+        if (vec) {
+            *reinterpret_cast<uint4 *>(p) =
+                make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]), pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) p[j] = __float2bfloat16_rn(v[j]);
+        }
+    }
+}
+
+
 // YOUT false: the first pass of a sequence split (no y; the end state and
 // the sum of Delta over the tokens per channel instead).
-template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT>
+template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false>
 __global__ void __launch_bounds__(32 * (MAXW + 1), 1)
 scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, const int W, const int S) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -567,6 +597,28 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
         const float Dd = a.D ? __ldg(a.D + dd) : 0.0f;
         const float bias = a.bias ? __ldg(a.bias + dd) : 0.0f;
         const bool sp = a.softplus != 0;
+        // Conv front-end: taps right-aligned in cw (cw[3] weights the current
+        // token) and the 3 inputs before this lane's next chunk (the channel's
+        // last lane's copy feeds lane g = 0 of the next tile)
+        float cw[4] = {0.0f, 0.0f, 0.0f, 0.0f}, cb = 0.0f;
+        float keep[3] = {0.0f, 0.0f, 0.0f};
+        TIn *uo_row = nullptr;
+        if constexpr (CONV) {
+            const int Wc = a.conv_width;
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int src = k - (4 - Wc);
+                if (src >= 0) cw[k] = __ldg(a.conv_w + dd * Wc + src);
+            }
+            cb = a.conv_b ? __ldg(a.conv_b + dd) : 0.0f;
+            if (a.conv_x0 != nullptr && active) {
+                const TIn *x0 = static_cast<const TIn *>(a.conv_x0) + (b * a.dim + d) * (Wc - 1);
+#pragma unroll
+                for (int j = 1; j <= 3; ++j)
+                    if (Wc - 1 - j >= 0) keep[3 - j] = ld_in<TIn>(x0 + (Wc - 1 - j));
+            }
+            if (a.u_out != nullptr) uo_row = static_cast<TIn *>(a.u_out) + b * a.uo_sb + dd * a.uo_sd;
+        }
         float *xd = reinterpret_cast<float *>(smem + lay.xch(warp));   // [8][kRow] Delta (or the pairs)
         float *xu = xd + kCW * kRow;                                     // [8][kRow] Delta*u
         float *pr = xd + (SPLAT ? kCW * kRowS : 2 * kCW * kRow);         // [8*4][kRow] partial readouts
@@ -792,6 +844,34 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             __syncwarp();
             if (lane == 0) bar_arrive(bar(empty0 + s));  // this warp is done with the stage
             const bool live = t0 + 8 * g < L;  // L % 8 == 0: whole chunks are in or out
+            if constexpr (CONV) {
+                // u from the conv input x (the stage held x): the halo x[t-3..t-1] is the
+                // previous lane's chunk tail, or for g = 0 the channel's last lane's tail
+                // of the previous tile
+                const bool last_lane = g == 3;
+                const int src = g == 0 ? lane + 3 : lane - 1;
+                const float h0 = __shfl_sync(0xffffffffu, last_lane ? keep[0] : uv[5], src);
+                const float h1 = __shfl_sync(0xffffffffu, last_lane ? keep[1] : uv[6], src);
+                const float h2 = __shfl_sync(0xffffffffu, last_lane ? keep[2] : uv[7], src);
+                keep[0] = uv[5];
+                keep[1] = uv[6];
+                keep[2] = uv[7];
+                float xs[11];
+                xs[0] = h0;
+                xs[1] = h1;
+                xs[2] = h2;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) xs[3 + j] = uv[j];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float v = fmaf(cw[0], xs[j], cb);
+                    v = fmaf(cw[1], xs[j + 1], v);
+                    v = fmaf(cw[2], xs[j + 2], v);
+                    v = fmaf(cw[3], xs[j + 3], v);
+                    uv[j] = a.conv_silu ? silu_f(v) : v;
+                }
+                if (uo_row != nullptr && active && live) store8_in<TIn>(uo_row + t0 + 8 * g, a.vec_uout != 0, uv);
+            }
             float gate[8], dug[8];
             // every exponent |Delta A| log2(e) of the warp's tile within the
             // series' range: the tile's decays come from the expm1 series
@@ -1114,12 +1194,12 @@ int choose_w(int64_t batch, int64_t dim, int num_sms, int in_bytes) {
     return (int)w;
 }
 
-template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT>
+template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false>
 cudaError_t launch_tm(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaStream_t stream) {
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     static SmemOptIn opt_in;
-    cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT>),
-                                  kSmemLimit);
+    cudaError_t e = opt_in.ensure(
+        reinterpret_cast<const void *>(scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV>), kSmemLimit);
     if (e != cudaSuccess) return e;
     const int64_t blocks = a.batch * ((a.dim + lay.cwc() - 1) / lay.cwc());
     if (blocks <= 0) return cudaSuccess;
@@ -1127,15 +1207,16 @@ cudaError_t launch_tm(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaS
     // At least half of an SM's shared memory: one CTA per SM, so the CTA's
     // 512 tensor-memory columns are always free when it allocates them.
     const int smem = lay.total() > kOneCtaSmem ? lay.total() : kOneCtaSmem;
-    scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT><<<(unsigned)blocks, 32 * (W + 1), smem, stream>>>(a, maps, W, S);
+    scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV>
+        <<<(unsigned)blocks, 32 * (W + 1), smem, stream>>>(a, maps, W, S);
     return cudaGetLastError();
 }
 
-template <typename TIn, typename TOut, int POLY8, bool YOUT = true>
+template <typename TIn, typename TOut, int POLY8, bool YOUT = true, bool CONV = false>
 cudaError_t launch_w(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaStream_t stream) {
-    if (W <= kMaxWSmall) return launch_tm<TIn, TOut, POLY8, kMaxWSmall, YOUT>(a, maps, W, S, stream);
-    if (W <= kMaxWMid) return launch_tm<TIn, TOut, POLY8, kMaxWMid, YOUT>(a, maps, W, S, stream);
-    return launch_tm<TIn, TOut, POLY8, kMaxWLarge, YOUT>(a, maps, W, S, stream);
+    if (W <= kMaxWSmall) return launch_tm<TIn, TOut, POLY8, kMaxWSmall, YOUT, CONV>(a, maps, W, S, stream);
+    if (W <= kMaxWMid) return launch_tm<TIn, TOut, POLY8, kMaxWMid, YOUT, CONV>(a, maps, W, S, stream);
+    return launch_tm<TIn, TOut, POLY8, kMaxWLarge, YOUT, CONV>(a, maps, W, S, stream);
 }
 
 // First pass of a sequence split (no y): the exponentials as for y.
@@ -1169,7 +1250,8 @@ bool scan_tmem_shape_ok(const ScanArgs &a, bool in_bf16, int out_bytes) {
 
 bool scan_tmem_applies(const ScanArgs &a, bool in_bf16, int out_bytes) {
     if (!scan_tmem_shape_ok(a, in_bf16, out_bytes)) return false;
-    if (a.ckpt || a.conv_w) return false;
+    if (a.ckpt) return false;
+    if (a.conv_w && (a.y == nullptr || a.dsum != nullptr)) return false;  // the conv front-end writes y, unsplit
     // either y (and no Delta sums), or the first pass of a split: no y, the
     // Delta sums and the end states
     if (a.y ? a.dsum != nullptr : (a.dsum == nullptr || a.last == nullptr)) return false;
@@ -1199,6 +1281,17 @@ cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool i
         return cudaErrorInvalidValue;
     if (!zmap) maps.z = maps.u;  // never loaded
     const int poly8 = plan.poly8;
+    if (a.conv_w != nullptr) {
+        // the conv front-end: every exponential on MUFU for bf16 inputs, on the
+        // FMA pipe for fp32 (the automatic plans)
+        if (poly8 != (in_bf16 ? 0 : 8)) return cudaErrorInvalidValue;
+        if (in_bf16) {
+            return out_bf16 ? launch_w<__nv_bfloat16, __nv_bfloat16, 0, true, true>(a, maps, W, S, stream)
+                            : launch_w<__nv_bfloat16, float, 0, true, true>(a, maps, W, S, stream);
+        }
+        return out_bf16 ? launch_w<float, __nv_bfloat16, 8, true, true>(a, maps, W, S, stream)
+                        : launch_w<float, float, 8, true, true>(a, maps, W, S, stream);
+    }
     if (a.y == nullptr)
         return in_bf16 ? launch_pass1<__nv_bfloat16>(a, maps, W, S, poly8, stream)
                        : launch_pass1<float>(a, maps, W, S, poly8, stream);

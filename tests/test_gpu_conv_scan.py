@@ -108,6 +108,69 @@ def test_every_plan(dtype, lanes, poly8):
     compare(inp, cp, f"plan ({lanes},1,{poly8}) {dtype}", plan=(lanes, 1, poly8), use_x0=True)
 
 
+def _tmem_plan(w):
+    # the plain scan's automatic plan for the same sizes: the conv front-end
+    # takes the tensor-memory engine exactly where the plain scan does
+    u = torch.empty(w.batch, w.dim, w.seqlen, dtype=w.in_dtype)
+    B = torch.empty(w.batch, w.dstate, w.seqlen, dtype=w.in_dtype)
+    y = torch.empty(w.batch, w.dim, w.seqlen)
+    rc, pl = mb.mamba_scan_choose_plan(mb.scan_dims_for(u, u, B, B, u, y))
+    return rc == mb.MS_OK and pl.engine == mb.MS_ENGINE_TMEM
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+@pytest.mark.parametrize("width", [1, 2, 3, 4])
+@pytest.mark.parametrize("L,dim", [(64, 40), (256, 100), (1024, 136)])
+def test_tensor_memory_engine(dtype, width, L, dim):
+    """Lengths the tensor-memory engine takes (multiples of 8), channel counts
+    that leave the last CTA's block ragged, history and u_out: the conv halo
+    crosses lanes and 32-token tiles."""
+    w = syn.scaled(syn.M130, batch=2, dim=dim, seqlen=L, in_dtype=dtype, seed=300 + L + width)
+    assert _tmem_plan(w)
+    inp, cp = _case(w, width)
+    compare(inp, cp, f"tensor-memory W={width} L={L} d={dim} {dtype}", use_x0=True, return_u=True)
+
+
+def test_tensor_memory_identity_filter_equals_plain_scan():
+    """As below, at a length the tensor-memory engine takes: u = x exactly,
+    y and last_state bit for bit those of the plain scan."""
+    w = syn.scaled(syn.M130, batch=2, dim=64, seqlen=304, in_dtype=torch.bfloat16, seed=49)
+    assert _tmem_plan(w)
+    inp = {k: v.to(DEV) for k, v in syn.scan_inputs(w).items()}
+    ones = torch.ones(w.dim, 1, device=DEV)
+    y1, l1, u1 = mb.conv_scan_fwd(inp["u"], ones, inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"],
+                                  inp["z"], inp["delta_bias"], True, conv_silu=False, return_u=True)
+    y0, l0 = mb.scan_fwd(inp["u"], inp["delta"], inp["A"], inp["B"], inp["C"], inp["D"], inp["z"],
+                         inp["delta_bias"], True)
+    torch.cuda.synchronize()
+    assert torch.equal(u1, inp["u"])
+    assert torch.equal(y1, y0) and torch.equal(l1, l0)
+
+
+def test_tensor_memory_split_resume():
+    """[0, m) then [m, L) with the last W-1 inputs as history, both lengths
+    multiples of 8, equals the whole sequence."""
+    W, m = 4, 192
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=520, in_dtype=torch.float32, seed=57)
+    inp, cp = _case(w, W)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    c = {k: v.to(DEV) for k, v in cp.items()}
+
+    def part(sl, x0=None, h0=None):
+        return mb.conv_scan_fwd(g["u"][:, :, sl].contiguous(), c["conv_w"], g["delta"][:, :, sl].contiguous(),
+                                g["A"], g["B"][:, :, sl].contiguous(), g["C"][:, :, sl].contiguous(), g["D"],
+                                g["z"][:, :, sl].contiguous(), g["delta_bias"], True, conv_b=c["conv_b"],
+                                conv_x0=x0, initial_state=h0)
+
+    y1, h1, _ = part(slice(0, m))
+    x0 = g["u"][:, :, m - W + 1:m].contiguous()
+    y2, h2, _ = part(slice(m, w.seqlen), x0=x0, h0=h1)
+    torch.cuda.synchronize()
+    yr, lr, _ = run_oracle(inp, cp)
+    check_fp32(f64(torch.cat([y1, y2], dim=2)), yr, "tensor-memory split y")
+    check_fp32(f64(h2), lr, "tensor-memory split last_state")
+
+
 def test_bf16_output():
     w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=130, in_dtype=torch.bfloat16, seed=43)
     inp, cp = _case(w, 4)

@@ -118,7 +118,8 @@ KERNEL_SOURCES = {
                       "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
     "scan_fwd_long": ("selective_state_space_40_b200/csrc/scan_fwd.cu",
                       "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
-    "conv_scan_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",),
+    "conv_scan_130m": ("selective_state_space_40_b200/csrc/scan_fwd.cu",
+                       "selective_state_space_40_b200/csrc/scan_fwd_tmem.cu"),
     "decode_step": ("selective_state_space_40_b200/csrc/state_update_stream.cu",),
     "scan_bwd_130m": ("selective_state_space_40_b200/csrc/scan_bwd.cu",),
     "ssd_2p7b": ("selective_state_space_40_b200/csrc/ssd_fwd_tc.cu",),

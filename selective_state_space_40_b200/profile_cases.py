@@ -10,7 +10,8 @@ scanlong_b1_L16k (its first 16384 tokens: a small case of the same kernels),
 conv130m (the same with the causal conv front-end, width 4), decode (one
 state update at b256 d5120 N16), bwd130m_b4 (training forward with saved
 states, then the backward, 130M-class layer with 4 batch rows), ssd2p7b_b2
-(Mamba-2 SSD layer, 2.7B-class with 2 batch rows), ssdcb2p7b (the per-chunk
+(Mamba-2 SSD layer, 2.7B-class with 2 batch rows), ssddec_b64 (its one-token
+state update for 64 sequences), ssdcb2p7b (the per-chunk
 C B^T of that layer on the tcgen05 tensor cores, 4 batch rows). Each kernel
 of the case runs REPEATS times (default 3).
 """
@@ -67,6 +68,20 @@ def _ssd(reps):
         mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True, return_final_state=False)
 
 
+def _ssd_decode(reps):
+    # one-token steps of the 2.7B-class layer for 64 sequences: fp32 state [64, 80, 64, 128]
+    w = syn.SsdWorkload("decode", 64, 1, 80, 64, 128, 1)
+    par = {k: v.cuda() for k, v in syn.ssd_inputs(w).items()}
+    gen = torch.Generator().manual_seed(11)
+    state = (0.1 * torch.randn(64, 80, 64, 128, generator=gen)).cuda()
+    x = torch.randn(64, 80, 64, generator=gen).to(torch.bfloat16).cuda()
+    dt = torch.randn(64, 80, generator=gen).to(torch.bfloat16).cuda()
+    B = torch.randn(64, 1, 128, generator=gen).to(torch.bfloat16).cuda()
+    C = torch.randn(64, 1, 128, generator=gen).to(torch.bfloat16).cuda()
+    for _ in range(reps):
+        mb.ssd_state_update(state, x, dt, par["A"], B, C, par["D"], par["dt_bias"], True)
+
+
 def _ssd_cb(reps):
     w = syn.SSD_2P7B
     g = {k: v.cuda() for k, v in syn.ssd_inputs(w).items()}
@@ -85,6 +100,7 @@ CASES = {
     "decode": _decode,
     "bwd130m_b4": _bwd,
     "ssd2p7b_b2": _ssd,
+    "ssddec_b64": _ssd_decode,
     "ssdcb2p7b": _ssd_cb,
 }
 

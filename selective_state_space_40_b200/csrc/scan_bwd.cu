@@ -443,20 +443,46 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 sm.red[rb][warp][j][lane] = reduce_scatter_channels(v8, c);
             }
             // per-token sums over the channel's 4 lanes; lane g owns tokens 2g, 2g+1
+            // and writes both with one 8-byte store per gradient (full sectors
+            // across the warp's 8 channels)
             reduce_scatter_lanes(ddt, g);
             reduce_scatter_lanes(dus, g);
+            {
+                // v[2g + k] from compile-time indices
+                auto pick = [&](const float (&v)[kSub], int k) {
+                    const float a0 = v[k], a1 = v[2 + k], a2 = v[4 + k], a3 = v[6 + k];
+                    return g == 0 ? a0 : (g == 1 ? a1 : (g == 2 ? a2 : a3));
+                };
+                const int j0 = s * kSub + 2 * g;
+                const int64_t t = ts + 2 * g;
+                float ddv[2], duv[2], dzv[2];
 #pragma unroll
-            for (int j = 0; j < kSub; ++j) {
-                // compile-time indices; the lane owning token j acts
-                const int k = j & 1;
-                const int64_t t = ts + j;
-                if ((j >> 1) == g && active && t < L) {
-                    const float ddv = ddt[k] * tk_sig[s * kSub + j];
-                    a.ddelta[grow + t] = ddv;
-                    a.du[grow + t] = fmaf(Dd, dq[j], dus[k]);
-                    if (has_z && a.dz != nullptr) a.dz[grow + t] = ov[j] * qv[j] * tk_gp[s * kSub + j];
-                    dDacc = fmaf(dq[j], uv[j], dDacc);
-                    dbacc += ddv;
+                for (int k = 0; k < 2; ++k) {
+                    const float dqk = pick(dq, k);
+                    ddv[k] = ddt[k] * tk_sig[j0 + k];
+                    duv[k] = fmaf(Dd, dqk, dus[k]);
+                    dzv[k] = pick(ov, k) * pick(qv, k) * tk_gp[j0 + k];
+                    if (active && t + k < L) {
+                        dDacc = fmaf(dqk, pick(uv, k), dDacc);
+                        dbacc += ddv[k];
+                    }
+                }
+                const bool want_dz = has_z && a.dz != nullptr;
+                if (active && t + 1 < L &&
+                    ((reinterpret_cast<uintptr_t>(a.ddelta + grow + t) | reinterpret_cast<uintptr_t>(a.du + grow + t) |
+                      (want_dz ? reinterpret_cast<uintptr_t>(a.dz + grow + t) : 0)) & 7u) == 0) {
+                    *reinterpret_cast<float2 *>(a.ddelta + grow + t) = make_float2(ddv[0], ddv[1]);
+                    *reinterpret_cast<float2 *>(a.du + grow + t) = make_float2(duv[0], duv[1]);
+                    if (want_dz) *reinterpret_cast<float2 *>(a.dz + grow + t) = make_float2(dzv[0], dzv[1]);
+                } else if (active) {
+#pragma unroll
+                    for (int k = 0; k < 2; ++k) {
+                        if (t + k < L) {
+                            a.ddelta[grow + t + k] = ddv[k];
+                            a.du[grow + t + k] = duv[k];
+                            if (want_dz) a.dz[grow + t + k] = dzv[k];
+                        }
+                    }
                 }
             }
             // dB / dC: sum the warps' partial sums (this sub-chunk's buffer;

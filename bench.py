@@ -102,6 +102,15 @@ def measured_bf16_tflops():
         return 1590.0
 
 
+def ssd_bound(nbytes, flops, hbm_gbs, tflops):
+    """Which roofline bounds the chunked SSD launch: its bytes at the HBM peak
+    against its flops at the bf16 tensor peak, the slower one."""
+    t_hbm = nbytes / (hbm_gbs * 1e9)
+    t_tc = flops / (tflops * 1e12)
+    which = "hbm" if t_hbm >= t_tc else "tensor"
+    return f"{which} (bytes / {hbm_gbs:.0f} GB/s: {t_hbm * 1e3:.4f} ms; flops / {tflops:.0f} TFLOP/s: {t_tc * 1e3:.4f} ms)"
+
+
 # B200 HBM3e nominal bandwidth (GB/s), printed beside the graded fraction of
 # the measured copy peak
 NOMINAL_HBM_GBS = 8000.0
@@ -703,7 +712,7 @@ def main(argv=None):
                     "frac_hbm": sbytes / (ssd_ms * 1e-3) / 1e9 / peak,
                     "tflops": sflops / (ssd_ms * 1e-3) / 1e12, "algorithmic_flops": sflops,
                     "frac_tensor": sflops / (ssd_ms * 1e-3) / 1e12 / measured_bf16_tflops(),
-                    "bound": "hbm (bytes / 6443 GB/s exceed flops / bf16 peak)",
+                    "bound": ssd_bound(sbytes, sflops, peak, measured_bf16_tflops()),
                     "timing": "mean of per-launch event pairs, two rotating input sets",
                     "traffic": recorded_traffic("ssd_2p7b")},
             "ssd_decode": {"workload": "mamba2-2.7b-class decode b64 H80 P64 N128 bf16, fp32 state",

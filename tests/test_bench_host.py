@@ -200,3 +200,9 @@ def test_shard_plan_reassembles_over_two_gloo_ranks():
         p.join(timeout=60)
         assert p.exitcode == 0
     assert res == {(4, 48): True, (3, 40): True}
+
+
+def test_ssd_bound_names_the_slower_roofline():
+    # the 2.7B-class SSD layer: 257 MB and 53.7 GFLOP; at 6650 GB/s and 1590 TFLOP/s the bytes take longer
+    assert bench.ssd_bound(257164224, 53687091200, 6650.0, 1590.0).startswith("hbm")
+    assert bench.ssd_bound(1, 10 ** 15, 6650.0, 1590.0).startswith("tensor")

@@ -81,12 +81,14 @@ bool ssd_shape_supported(int64_t headdim, int64_t dstate);
 // Chunk-parallel SSD forward on the tcgen05 tensor cores: per-launch state
 // of the chunk hand-off (flags [batch * H] then the ticket counter, zeroed
 // before the launch; the running state [batch, H, P / 4, N, 4] in the workspace),
-// the index of the last chunk, the heads per work item, and how y is stored.
+// the index of the last chunk, the number of work items, the heads per work
+// item, and how y is stored.
 struct SsdTcArgs {
     int *flags;
     int *counter;
     float *state;
     int64_t last_chunk;
+    int64_t items;
     int hb;
     int y_vec16;  // y rows take 16-byte stores
     int y_tma;    // y is written by tensor stores through the kernel's y map

@@ -26,15 +26,23 @@
 //
 // Work item = (chunk k, batch row b, block of up to 8 heads of one group).
 // Items are claimed in ticket order from a global counter, chunk-major, so the
-// item holding chunk k - 1 of the same heads started before this one. Only
+// item holding chunk k - 1 of the same heads was claimed before this one. The
+// kernel is persistent (one CTA per SM): a CTA holds at most the item it
+// computes and the one its producer warp prepares, and the smallest unfinished
+// ticket is always one that some CTA computes, so every wait ends. Only
 // Y_s and S_out depend on the entering state: each head computes CB, S_c and
 // Y_i first, then waits for chunk k - 1's item to publish S_in (a per-(b, h)
 // counter in global memory), writes S_out over it and publishes it for chunk
 // k + 1. The running state lives in the workspace and crosses chunks through
 // L2, so HBM sees each input once.
 //
-// CTA: two groups of 4 compute warps and one MMA warp (lane 0 issues every
-// tcgen05.mma and commit). The groups take alternate heads of the item, each
+// CTA: two groups of 4 compute warps, one MMA warp (lane 0 issues every
+// tcgen05.mma and commit) and one producer warp, which claims the next item,
+// forms its per-head Delta, cumulative decay and w_s into the other of two
+// parameter buffers while the current item computes, and loads the item's C
+// and B tiles once the previous item's products are done with them; each
+// group loads x of its first head of the next item behind its last head of
+// this one. The groups take alternate heads of the item, each
 // with its own half of tensor memory (a slot: CB, overwritten in place by G'
 // as packed bf16 hi / lo, the A operand of Y_i; S_c, later Y_s; Y_i) and its
 // own x and X' (later S_in) buffers, so one group's products run while the
@@ -74,9 +82,10 @@ constexpr int kN = 128;        // state size
 constexpr int kHB = 8;         // most heads per work item
 constexpr int kGroupWarps = 4;                       // one warp per 32 accumulator lanes
 constexpr int kGroupThreads = 32 * kGroupWarps;
-constexpr int kComputeThreads = 2 * kGroupThreads;
-constexpr int kMmaWarp = 2 * kGroupWarps;
-constexpr int kThreads = kComputeThreads + 32;
+constexpr int kComputeWarps = 2 * kGroupWarps;
+constexpr int kMmaWarp = kComputeWarps;              // issues every product
+constexpr int kProdWarp = kComputeWarps + 1;         // claims items, forms their parameters, loads C and B
+constexpr int kThreads = 32 * (kComputeWarps + 2);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kSlotCols = 256;
 // columns inside a slot: CB (fp32, 128), then G' in place -- the 32 tokens s of
@@ -97,11 +106,23 @@ constexpr int kOffC = 0;                          // C tile   [t][n] K-major, 32
 constexpr int kOffB = kOffC + kQ * kN * 2;        // B tile   [s][n], 32 KB
 constexpr int kOffSlot = kOffB + kQ * kN * 2;     // per slot: X' / S_in hi, lo 32 KB; x [s][p] MN-major 16 KB
 constexpr int kSlotBytes = 3 * kTileHalf;
-constexpr int kOffPar = kOffSlot + 2 * kSlotBytes;  // dl, cs2, w: [kHB][kQ] floats each
-constexpr int kOffBar = kOffPar + 3 * kHB * kQ * 4;
+constexpr int kParBytes = 3 * kHB * kQ * 4;          // dl, cs2, w: [kHB][kQ] floats each
+constexpr int kOffPar = kOffSlot + 2 * kSlotBytes;  // two parameter buffers (items alternate)
+constexpr int kOffBar = kOffPar + 2 * kParBytes;
 enum { kBarXP = 0, kBarCB, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarsPerSlot };
-constexpr int kBarLD = 2 * kBarsPerSlot, kBarEnd = kBarLD + 1, kNumBars = kBarEnd + 1;
-constexpr int kOffMisc = kOffBar + 8 * kNumBars;  // tensor-memory base, ticket, abort
+constexpr int kBarParFull = 2 * kBarsPerSlot;  // [2] an item's descriptor and parameters are in buffer i
+constexpr int kBarParFree = kBarParFull + 2;   // [2] every consumer is done with buffer i
+constexpr int kBarCBFull = kBarParFree + 2;    // the current item's C and B tiles are in
+constexpr int kBarCBFree = kBarCBFull + 1;     // the current item's products are done with them
+constexpr int kBarEnd = kBarCBFree + 1, kNumBars = kBarEnd + 1;
+
+// A work item as the producer warp hands it to the others (valid = 0: no more)
+struct ItemDesc {
+    long long k, b, g, h0;
+    int nh, valid;
+};
+constexpr int kOffDesc = kOffBar + 8 * kNumBars;                // ItemDesc per parameter buffer
+constexpr int kOffMisc = kOffDesc + 2 * (int)sizeof(ItemDesc);  // tensor-memory base, -, abort
 constexpr int kSmemBytes = kOffMisc + 16;
 
 // K-major no-swizzle [rows x 128] bf16 tile: core matrix (row / 8, k / 8) at
@@ -300,11 +321,11 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
     const uint32_t sbase = saddr(smem);
     auto bar = [&](int i) { return sbase + (uint32_t)(kOffBar + 8 * i); };
     auto sbar = [&](int slot, int e) { return bar(slot * kBarsPerSlot + e); };
-    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kOffMisc);  // [0] tmem base, [1] ticket, [2] abort
+    uint32_t *misc = reinterpret_cast<uint32_t *>(smem + kOffMisc);  // [0] tmem base, [2] abort
     volatile uint32_t *abort_flag = misc + 2;
+    ItemDesc *desc = reinterpret_cast<ItemDesc *>(smem + kOffDesc);
 
     if (tid == 0) {
-        misc[1] = (uint32_t)atomicAdd(w.counter, 1);
         misc[2] = 0u;
         for (int sl = 0; sl < 2; ++sl) {
             bar_init(sbar(sl, kBarXP), kGroupWarps);
@@ -315,7 +336,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             bar_init(sbar(sl, kBarS), kGroupWarps);
             bar_init(sbar(sl, kBarYS), 1);
         }
-        bar_init(bar(kBarLD), 1);
+        for (int pb = 0; pb < 2; ++pb) {
+            bar_init(bar(kBarParFull + pb), 1);
+            bar_init(bar(kBarParFree + pb), kComputeWarps + 1);
+        }
+        bar_init(bar(kBarCBFull), 1);
+        bar_init(bar(kBarCBFree), 1);
         bar_init(bar(kBarEnd), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -329,43 +355,136 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
     __syncthreads();
     tc_after();
     const uint32_t tmem = misc[0];
-    const int64_t ticket = (int64_t)misc[1];
 
-    // ---- work item
     const int64_t hpg = a.H / a.G;                       // heads per group
     const int64_t nhb = (hpg + w.hb - 1) / w.hb;         // head blocks per group
     const int64_t per_chunk = a.batch * a.G * nhb;
-    const int64_t k = ticket / per_chunk;
-    const int64_t r0 = ticket % per_chunk;
-    const int64_t b = r0 / (a.G * nhb);
-    const int64_t g = (r0 / nhb) % a.G;
-    const int64_t hbk = r0 % nhb;
-    const int64_t h0 = g * hpg + hbk * w.hb;
-    const int64_t left = hpg - hbk * w.hb;
-    const int nh = (int)(left < (int64_t)w.hb ? left : (int64_t)w.hb);
-    const int64_t t0 = k * kQ;
     const int64_t L = a.L;
+    auto params = [&](int pb) { return reinterpret_cast<float *>(smem + kOffPar + pb * kParBytes); };
 
-    const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
-    const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
-    const __nv_bfloat16 *xb = static_cast<const __nv_bfloat16 *>(a.x) + b * a.x_sb;
-    float *dlp = reinterpret_cast<float *>(smem + kOffPar);   // [kHB][kQ] Delta
-    float *cs2p = dlp + kHB * kQ;                             // [kHB][kQ] cs log2(e)
-    float *wp = cs2p + kHB * kQ;                              // [kHB][kQ] w_s
-
-    if (warp == kMmaWarp) {
+    if (warp == kProdWarp) {
+        // ============================== producer warp ==============================
+        // Claims items in ticket order (one ahead of the item it prepares), writes
+        // each item's descriptor and per-head parameters into the free buffer, and
+        // loads the item's C and B tiles once the previous item's products are done
+        // with them. The next item is thus ready while the current one computes.
+        bool ok = true;
+        long long T = 0;
+        if (lane == 0) T = (long long)(unsigned)atomicAdd(w.counter, 1);
+        T = __shfl_sync(0xffffffffu, T, 0);
+        for (int it = 0;; ++it) {
+            const int pb = it & 1;
+            if (it >= 2) ok = bar_wait(bar(kBarParFree + pb), (uint32_t)(((it - 2) >> 1) & 1));
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
+            const bool valid = ok && T < w.items;
+            const int64_t k = T / per_chunk, r0 = T % per_chunk;
+            const int64_t b = r0 / (a.G * nhb), g = (r0 / nhb) % a.G, hbk = r0 % nhb;
+            const int64_t h0 = g * hpg + hbk * w.hb;
+            const int64_t left = hpg - hbk * w.hb;
+            const int nh = valid ? (int)(left < (int64_t)w.hb ? left : (int64_t)w.hb) : 0;
+            const int64_t t0 = k * kQ;
+            long long Tn = 0;
+            if (valid && lane == 0) Tn = (long long)(unsigned)atomicAdd(w.counter, 1);
+            if (valid) {
+                // per head: Delta, cs log2(e) and w_s of the chunk's tokens, 4 tokens a lane
+                float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ;
+                const unsigned short *dtp = static_cast<const unsigned short *>(a.dt) + b * a.dt_sb + h0;
+                unsigned short raw[kHB][4];
+#pragma unroll
+                for (int jj = 0; jj < kHB; ++jj)
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) {
+                        const int64_t t = t0 + 4 * lane + i;
+                        raw[jj][i] = (jj < nh && t < L) ? __ldg(dtp + t * a.dt_sl + jj) : (unsigned short)0;
+                    }
+#pragma unroll
+                for (int jj = 0; jj < kHB; ++jj) {
+                    if (jj < nh) {
+                        const int64_t h = h0 + jj;
+                        const float A2 = __ldg(a.A + h) * kLog2e;
+                        const float bias = a.dt_bias ? __ldg(a.dt_bias + h) : 0.0f;
+                        float dl[4], c = 0.0f;
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            float d = 0.0f;
+                            if (t0 + 4 * lane + i < L) {
+                                const float v = bf16_bits_to_f32(raw[jj][i]) + bias;
+                                d = a.softplus ? softplus_f(v) : v;
+                            }
+                            dl[i] = d;
+                            c += d;
+                        }
+                        // inclusive prefix of the lanes' sums
+                        float incl = c;
+#pragma unroll
+                        for (int off = 1; off < 32; off <<= 1) {
+                            const float o = __shfl_up_sync(0xffffffffu, incl, off);
+                            if (lane >= off) incl += o;
+                        }
+                        float run = incl - c;  // sum before this lane's tokens
+                        const float total = __shfl_sync(0xffffffffu, incl, 31);
+                        const float cend = A2 * total;  // cs_{Q-1} log2(e): padded tokens add nothing
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            run += dl[i];
+                            const int t = 4 * lane + i;
+                            const float c2 = A2 * run;
+                            dlp[jj * kQ + t] = dl[i];
+                            cs2p[jj * kQ + t] = c2;
+                            wp[jj * kQ + t] = exp2_mufu(cend - c2) * dl[i];
+                        }
+                    }
+                }
+            }
+            if (lane == 0) {
+                ItemDesc d;
+                d.k = k;
+                d.b = b;
+                d.g = g;
+                d.h0 = h0;
+                d.nh = nh;
+                d.valid = valid ? 1 : 0;
+                desc[pb] = d;
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarParFull + pb));
+            if (!valid) break;
+            // the item's C and B tiles (rows past L zero-filled), once the previous
+            // item's products have read theirs
+            if (it >= 1) ok = bar_wait(bar(kBarCBFree), (uint32_t)((it - 1) & 1));
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
+            if (ok) {
+                const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
+                const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
+                for (int i = lane; i < kQ * (kN / 8); i += 32) {
+                    const int t = i >> 4, kc = i & 15;
+                    const bool in = t0 + t < L;
+                    const int64_t tt = in ? t0 + t : 0;
+                    cp_async16(sbase + kOffC + kmaj_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
+                    cp_async16(sbase + kOffB + kmaj_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
+                }
+                cp_commit();
+                cp_wait0();          // this lane's copies are in
+                fence_async_smem();  // ... and visible to the tensor cores
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarCBFull));
+            if (!ok) break;
+            T = __shfl_sync(0xffffffffu, Tn, 0);
+        }
+        if (!ok && lane == 0) {
+            *abort_flag = 1u;
+            if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
+        }
+    } else if (warp == kMmaWarp) {
         // ================================ MMA warp ================================
         if (lane == 0) {
             const uint32_t sC = sbase + kOffC, sB = sbase + kOffB;
-            bool ok = bar_wait(bar(kBarLD), 0u) && *abort_flag == 0u;
-            tc_after();
-            // per slot: its next head and step (0: X' ready -> CB, S_c; 1: G' ready
-            // -> Y_i; 2: S_in ready -> Y_s); slot s takes heads s, s + 2, ...
-            int jn[2] = {0, 1}, step[2] = {0, 0};
-            uint32_t idle = 0;
+            bool ok = true;
+            uint32_t used[2] = {0u, 0u};  // heads each slot has taken (barrier parities)
             // CB = C B^T (both K-major) into a slot's first 128 columns: issued behind the
-            // slot's previous head's last product (products run in issue order, so
-            // that head's G' has been read), so the group finds it ready
+            // slot's previous head's Y_i (products run in issue order, so that head's G'
+            // has been read), so the group finds it ready
             auto issue_cb = [&](int sl) {
                 const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
 #pragma unroll 1
@@ -374,63 +493,80 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                         idesc(kQ, false, false), ks > 0);
                 mma_commit(sbar(sl, kBarCB));
             };
-            if (ok) {
+            for (int it = 0; ok; ++it) {
+                const int pb = it & 1;
+                ok = bar_wait(bar(kBarParFull + pb), (uint32_t)((it >> 1) & 1)) && *abort_flag == 0u;
+                if (!ok) break;
+                const int nh = desc[pb].nh, valid = desc[pb].valid;
+                bar_arrive(bar(kBarParFree + pb));  // the descriptor is all this warp reads
+                if (!valid) break;
+                ok = bar_wait(bar(kBarCBFull), (uint32_t)(it & 1)) && *abort_flag == 0u;
+                if (!ok) break;
+                tc_after();
                 issue_cb(0);
                 if (nh > 1) issue_cb(1);
-            }
-            while (ok && (jn[0] < nh || jn[1] < nh)) {
-                bool progressed = false;
+                // per slot: its next head and step (0: X' ready -> S_c; 1: G' ready -> Y_i;
+                // 2: S_in ready -> Y_s); slot s takes heads s, s + 2, ...
+                int jn[2] = {0, 1}, step[2] = {0, 0};
+                uint32_t idle = 0;
+                while (ok && (jn[0] < nh || jn[1] < nh)) {
+                    bool progressed = false;
 #pragma unroll 1
-                for (int sl = 0; sl < 2; ++sl) {
-                    const int j = jn[sl];
-                    if (j >= nh) continue;
-                    const uint32_t ph = (uint32_t)((j >> 1) & 1);
-                    const int ev = step[sl] == 0 ? kBarXP : (step[sl] == 1 ? kBarG : kBarS);
-                    if (!bar_test(sbar(sl, ev), ph)) continue;
-                    tc_after();
-                    const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
-                    const uint32_t sXP = sbase + (uint32_t)(kOffSlot + sl * kSlotBytes);
-                    const uint32_t sX = sXP + (uint32_t)(2 * kTileHalf);
-                    if (step[sl] == 0) {
-                        // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo)
+                    for (int sl = 0; sl < 2; ++sl) {
+                        const int j = jn[sl];
+                        if (j >= nh) continue;
+                        const uint32_t ph = (used[sl] + (uint32_t)(j >> 1)) & 1u;
+                        const int ev = step[sl] == 0 ? kBarXP : (step[sl] == 1 ? kBarG : kBarS);
+                        if (!bar_test(sbar(sl, ev), ph)) continue;
+                        tc_after();
+                        const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
+                        const uint32_t sXP = sbase + (uint32_t)(kOffSlot + sl * kSlotBytes);
+                        const uint32_t sX = sXP + (uint32_t)(2 * kTileHalf);
+                        if (step[sl] == 0) {
+                            // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo)
 #pragma unroll 1
-                        for (int ks = 0; ks < kQ / 16; ++ks)
+                            for (int ks = 0; ks < kQ / 16; ++ks)
 #pragma unroll
-                            for (int part = 0; part < 2; ++part)
-                                mma(tb + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
-                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                                    idesc(kP, true, true), ks > 0 || part > 0);
-                        mma_commit(sbar(sl, kBarSC));
-                    } else if (step[sl] == 1) {
-                        // Y_i [t x p] = G' X: A = G' (hi, lo) packed in tensor memory, B = x
+                                for (int part = 0; part < 2; ++part)
+                                    mma(tb + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
+                                        desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                        idesc(kP, true, true), ks > 0 || part > 0);
+                            mma_commit(sbar(sl, kBarSC));
+                        } else if (step[sl] == 1) {
+                            // Y_i [t x p] = G' X: A = G' (hi, lo) packed in tensor memory, B = x
 #pragma unroll 1
-                        for (int ks = 0; ks < kQ / 16; ++ks)
+                            for (int ks = 0; ks < kQ / 16; ++ks)
 #pragma unroll
-                            for (int part = 0; part < 2; ++part)
-                                mma_ts(tb + kColYI, tb + g_col(ks, part),
-                                       desc_mn(sX + 2048u * ks, 1024u, 128u), idesc(kP, false, true),
-                                       ks > 0 || part > 0);
-                        mma_commit(sbar(sl, kBarYI));
-                    } else {
-                        // Y_s [t x p] = C S_in (hi, lo), into S_c's columns
+                                for (int part = 0; part < 2; ++part)
+                                    mma_ts(tb + kColYI, tb + g_col(ks, part), desc_mn(sX + 2048u * ks, 1024u, 128u),
+                                           idesc(kP, false, true), ks > 0 || part > 0);
+                            mma_commit(sbar(sl, kBarYI));
+                        } else {
+                            // Y_s [t x p] = C S_in (hi, lo), into S_c's columns
 #pragma unroll 1
-                        for (int ks = 0; ks < kN / 16; ++ks)
+                            for (int ks = 0; ks < kN / 16; ++ks)
 #pragma unroll
-                            for (int part = 0; part < 2; ++part)
-                                mma(tb + kColSC, desc_k(sC + 256u * ks, 128u, 2048u),
-                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                                    idesc(kP, false, true), ks > 0 || part > 0);
-                        mma_commit(sbar(sl, kBarYS));
-                        if (j + 2 < nh) issue_cb(sl);
+                                for (int part = 0; part < 2; ++part)
+                                    mma(tb + kColSC, desc_k(sC + 256u * ks, 128u, 2048u),
+                                        desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                        idesc(kP, false, true), ks > 0 || part > 0);
+                            mma_commit(sbar(sl, kBarYS));
+                            if (j + 2 < nh) issue_cb(sl);
+                        }
+                        if (++step[sl] == 3) {
+                            step[sl] = 0;
+                            jn[sl] += 2;
+                        }
+                        progressed = true;
                     }
-                    if (++step[sl] == 3) {
-                        step[sl] = 0;
-                        jn[sl] += 2;
-                    }
-                    progressed = true;
+                    if (progressed) idle = 0;
+                    else if (++idle > kIdleTries || *abort_flag != 0u) ok = false;
                 }
-                if (progressed) idle = 0;
-                else if (++idle > kIdleTries || *abort_flag != 0u) ok = false;
+                if (!ok) break;
+                used[0] += (uint32_t)((nh + 1) / 2);
+                used[1] += (uint32_t)(nh / 2);
+                // the C and B tiles are free once this item's products have completed
+                mma_commit(bar(kBarCBFree));
             }
             if (!ok) {
                 *abort_flag = 1u;
@@ -449,323 +585,301 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         const int row = 32 * qd + lane;                              // accumulator lane: token t or state n
         const uint32_t tb = tmem + (uint32_t)gi * kSlotCols + ((uint32_t)(32 * qd) << 16);
         unsigned char *XP = smem + kOffSlot + gi * kSlotBytes;       // X' hi / lo, later S_in hi / lo
-        // x of the group's current head
-        auto x_buf = [&](int) { return XP + 2 * kTileHalf; };
-        bool ok = true;
+        const unsigned char *X = XP + 2 * kTileHalf;                 // x of the group's current head
+        bool ok = true, fin = false;
+        bool x_ahead = false;  // x of the group's first head of the next item is requested
+        uint32_t used = 0;     // heads this group has taken (barrier parities of its slot)
 
-        auto load_x = [&](int j) {  // by the group's threads
-            if (j < nh) {
-                const __nv_bfloat16 *xh = xb + (h0 + j) * a.x_sh;
-                const uint32_t dst = saddr(x_buf(j));
-                for (int i = gtid; i < kQ * (kP / 8); i += kGroupThreads) {
-                    const int s = i >> 3, pc = i & 7;
-                    const bool in = t0 + s < L;
-                    cp_async16(dst + mn64_off(s, pc), xh + (in ? t0 + s : 0) * a.x_sl + 8 * pc, in ? 16 : 0);
-                }
+        auto load_x = [&](const ItemDesc &d, int j) {  // by the group's threads
+            const __nv_bfloat16 *xh =
+                static_cast<const __nv_bfloat16 *>(a.x) + d.b * a.x_sb + (d.h0 + j) * a.x_sh;
+            const int64_t xt0 = d.k * kQ;
+            const uint32_t dst = saddr(X);
+            for (int i = gtid; i < kQ * (kP / 8); i += kGroupThreads) {
+                const int s = i >> 3, pc = i & 7;
+                const bool in = xt0 + s < L;
+                cp_async16(dst + mn64_off(s, pc), xh + (in ? xt0 + s : 0) * a.x_sl + 8 * pc, in ? 16 : 0);
             }
             cp_commit();
         };
-        // chunk tiles: C, B (rows past L zero-filled) by both groups; x of each group's first head
-        for (int i = tid; i < kQ * (kN / 8); i += kComputeThreads) {
-            const int t = i >> 4, kc = i & 15;
-            const bool in = t0 + t < L;
-            const int64_t tt = in ? t0 + t : 0;
-            cp_async16(sbase + kOffC + kmaj_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
-            cp_async16(sbase + kOffB + kmaj_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
-        }
-        load_x(gi);
 
-        // per-head chunk parameters: warp j < nh takes head h0 + j, 4 tokens per lane
-        if (warp < nh) {
-            const int64_t h = h0 + warp;
-            const float A2 = __ldg(a.A + h) * kLog2e;
-            const float bias = a.dt_bias ? __ldg(a.dt_bias + h) : 0.0f;
-            const unsigned short *dtp = static_cast<const unsigned short *>(a.dt) + b * a.dt_sb + h;
-            float dl[4], c = 0.0f;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int64_t t = t0 + 4 * lane + i;
-                float d = 0.0f;
-                if (t < L) {
-                    const float v = bf16_bits_to_f32(__ldg(dtp + t * a.dt_sl)) + bias;
-                    d = a.softplus ? softplus_f(v) : v;
-                }
-                dl[i] = d;
-                c += d;
+        for (int it = 0;; ++it) {
+            const int pb = it & 1;
+            const bool got = ok && bar_wait(bar(kBarParFull + pb), (uint32_t)((it >> 1) & 1));
+            // the group agrees before anything it does together
+            ok = sync_and<kGroupThreads>(gbar, ok && got && *abort_flag == 0u);
+            if (!ok) break;
+            const ItemDesc &d = desc[pb];
+            if (!d.valid) {
+                fin = true;
+                break;
             }
-            // inclusive prefix of the lanes' sums
-            float incl = c;
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const float o = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += o;
-            }
-            float run = incl - c;  // sum before this lane's tokens
-            const float total = __shfl_sync(0xffffffffu, incl, 31);
-            const float cend = A2 * total;  // cs_{Q-1} log2(e): padded tokens add nothing
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                run += dl[i];
-                const int t = 4 * lane + i;
-                const float c2 = A2 * run;
-                dlp[warp * kQ + t] = dl[i];
-                cs2p[warp * kQ + t] = c2;
-                wp[warp * kQ + t] = exp2_mufu(cend - c2) * dl[i];
-            }
-        }
-        cp_wait0();          // this thread's copies of the tiles and the first x are in
-        fence_async_smem();  // ... and visible to the tensor cores
-        // everyone's copies and parameters are in: the MMA warp may start
-        ok = sync_and<kComputeThreads>(1, ok);
-        if (tid == 0) bar_arrive(bar(kBarLD));
+            const int nh = d.nh;
+            const int64_t k = d.k, b = d.b, t0 = k * kQ;
+            const float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ;
+            if (gi < nh && !x_ahead) load_x(d, gi);
+            x_ahead = false;
 
-        for (int j = gi; j < nh; j += 2) {
-            const uint32_t ph = (uint32_t)((j >> 1) & 1);
-            const int64_t h = h0 + j;
-            const float *cs2 = cs2p + j * kQ;
-            const unsigned char *X = x_buf(j);
-            if (j > gi) {
+            for (int j = gi; j < nh; j += 2, ++used) {
+                const uint32_t ph = used & 1u;
+                const int64_t h = d.h0 + j;
+                const float *cs2 = cs2p + j * kQ;
                 cp_wait0();  // x of head j is in
                 fence_async_smem();
                 if (gtid == 0 && w.y_tma) bulk_wait_read0();  // the previous head's y has left the staging buffer
                 ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
                 if (!ok) break;
-            }
-            // ---- X' = w_s x_s (row s, all 64 columns p), hi / lo
-            {
-                const int s = row;
-                const float ws = wp[j * kQ + s];
+                // ---- X' = w_s x_s (row s, all 64 columns p), hi / lo
+                {
+                    const int s = row;
+                    const float ws = wp[j * kQ + s];
 #pragma unroll
-                for (int pc = 0; pc < 8; ++pc) {
-                    float v[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(s, pc)), v);
+                    for (int pc = 0; pc < 8; ++pc) {
+                        float v[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(s, pc)), v);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) v[e] *= ws;
-                    uint4 hi, lo;
-                    split8(v, hi, lo);
-                    *reinterpret_cast<uint4 *>(XP + mn64_off(s, pc)) = hi;
-                    *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(s, pc)) = lo;
-                }
-            }
-            fence_async_smem();
-            __syncwarp();
-            if (lane == 0) bar_arrive(sbar(gi, kBarXP));
-
-            // ---- G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s for s <= t, hi / lo packed
-            // in place of CB, one 32-column block at a time; blocks entirely above
-            // the diagonal are zeros
-            ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarCB), ph));
-            tc_after();
-            {
-                const int t = row;
-                const float ct = cs2[t];
-                const float *dls = dlp + j * kQ;
-#pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t hi[16], lo[16];
-                    if (c <= qd && ok) {
-                        float v[32];
-                        tmem_ld32(tb + kColCB + (uint32_t)(32 * c), v);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            const int s = 32 * c + e;
-                            v[e] = (c < qd || s <= t) ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
-                        }
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) {
-                            const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
-                            hi[e] = *reinterpret_cast<const uint32_t *>(&hh);
-                            lo[e] = pack2(v[2 * e] - __low2float(hh), v[2 * e + 1] - __high2float(hh));
-                        }
-                    } else {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
-                    }
-                    tmem_st16(tb + kColCB + (uint32_t)(32 * c), hi);
-                    tmem_st16(tb + kColCB + (uint32_t)(32 * c + 16), lo);
-                }
-            }
-            tmem_st_wait();
-            tc_before();
-            __syncwarp();
-            if (lane == 0) bar_arrive(sbar(gi, kBarG));
-
-            // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out. The
-            // running state is [p / 4][n][4] per head in the workspace (a warp's 16-byte
-            // loads of one p-quad are contiguous); the first chunk reads
-            // initial_state [p][n], the last one also writes final_state [p][n].
-            ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarSC), ph));
-            tc_after();
-            {
-                int *flag = w.flags + (b * a.H + h);
-                if (k > 0 && ok) {
-                    uint32_t i = 0;
-                    while (ld_acquire(flag) < (int)k && i < kFlagTries) {
-                        __nanosleep(32);
-                        ++i;
-                    }
-                    ok = i < kFlagTries;
-                }
-                ok = __all_sync(0xffffffffu, ok);
-                const int n = row;
-                const size_t blk = (size_t)(b * a.H + h) * kP * kN;
-                float4 *run4 = reinterpret_cast<float4 *>(w.state + blk) + n;  // quad q at run4[q * kN]
-                const float decay = exp2_mufu(cs2[kQ - 1]);
-                // every S_in load of the row issued before any S_out store
-                float sv[64];
-                if (ok && k > 0) {
-#pragma unroll
-                    for (int q = 0; q < 16; ++q) {
-                        const float4 v4 = run4[q * kN];
-                        sv[4 * q] = v4.x; sv[4 * q + 1] = v4.y; sv[4 * q + 2] = v4.z; sv[4 * q + 3] = v4.w;
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) sv[e] = (ok && a.s0) ? a.s0[blk + (size_t)e * kN + n] : 0.0f;
-                }
-#pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    if (ok) {
-                        float sc[32];
-                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), sc);
-                        float so[32];
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) so[e] = fmaf(decay, sv[32 * half + e], sc[e]);
-#pragma unroll
-                        for (int q = 0; q < 8; ++q)
-                            run4[(8 * half + q) * kN] = make_float4(so[4 * q], so[4 * q + 1], so[4 * q + 2], so[4 * q + 3]);
-                        if (w.last_chunk == k && a.s_last != nullptr) {
-#pragma unroll
-                            for (int e = 0; e < 32; ++e) a.s_last[blk + (size_t)(32 * half + e) * kN + n] = so[e];
-                        }
-                    }
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
+                        for (int e = 0; e < 8; ++e) v[e] *= ws;
                         uint4 hi, lo;
-                        split8(sv + 32 * half + 8 * q, hi, lo);
-                        const int pc = 4 * half + q;
-                        *reinterpret_cast<uint4 *>(XP + mn64_off(n, pc)) = hi;
-                        *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(n, pc)) = lo;
+                        split8(v, hi, lo);
+                        *reinterpret_cast<uint4 *>(XP + mn64_off(s, pc)) = hi;
+                        *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(s, pc)) = lo;
                     }
                 }
                 fence_async_smem();
-                tc_before();
-                // the group's S_out is stored: publish it for chunk k + 1 (the release
-                // orders the group's stores, which the barrier put before it)
-                ok = sync_and<kGroupThreads>(gbar, ok);
-                if (gtid == 0 && ok) st_release(flag, (int)k + 1);
-            }
-            __syncwarp();
-            if (lane == 0) bar_arrive(sbar(gi, kBarS));
-            if (!ok) break;
-
-            // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t (row t, all 64 columns p): Y_i and
-            // D x first, while Y_s is still being formed
-            ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYI), ph));
-            tc_after();
-            if (ok) {
-                const int t = row;
-                const float et = exp2_mufu(cs2[t]);
-                const float Dh = a.D ? __ldg(a.D + h) : 0.0f;
-                TOut *yp = static_cast<TOut *>(a.y) + b * a.y_sb + (t0 + t) * a.y_sl + h * a.y_sh;
-                float yi[64];
-                tmem_ld32(tb + kColYI, *reinterpret_cast<float(*)[32]>(yi));
-                tmem_ld32(tb + kColYI + 32u, *reinterpret_cast<float(*)[32]>(yi + 32));
-#pragma unroll
-                for (int pc = 0; pc < 8; ++pc) {
-                    float xv[8];
-                    unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(t, pc)), xv);
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) yi[8 * pc + e] = fmaf(Dh, xv[e], yi[8 * pc + e]);
-                }
-                ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYS), ph));
+                __syncwarp();
+                if (lane == 0) bar_arrive(sbar(gi, kBarXP));
+                // ---- G'[t][s] = CB[t][s] exp(cs_t - cs_s) Delta_s for s <= t, hi / lo packed
+                // in place of CB, one 32-column block at a time; blocks entirely above
+                // the diagonal are zeros
+                ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarCB), ph));
                 tc_after();
-                if (w.y_tma) {
-                    // y row t into the staging buffer (S_in has been consumed by Y_s) in the
-                    // tensor map's box layout: rows of 128 bytes, 16-byte chunk i of row t
-                    // at chunk i ^ (t % 8) (128-byte swizzle); fp32: two boxes of 32
-                    // columns, bf16: one box of 64
+                {
+                    const int t = row;
+                    const float ct = cs2[t];
+                    const float *dls = dlp + j * kQ;
+#pragma unroll 1
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t hi[16], lo[16];
+                        if (c <= qd && ok) {
+                            float v[32];
+                            tmem_ld32(tb + kColCB + (uint32_t)(32 * c), v);
 #pragma unroll
-                    for (int half = 0; half < 2 && ok; ++half) {
-                        float ys[32];
-                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
+                            for (int e = 0; e < 32; ++e) {
+                                const int s = 32 * c + e;
+                                v[e] = (c < qd || s <= t) ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                            }
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) yi[32 * half + e] = fmaf(et, ys[e], yi[32 * half + e]);
+                            for (int e = 0; e < 16; ++e) {
+                                const __nv_bfloat162 hh = __floats2bfloat162_rn(v[2 * e], v[2 * e + 1]);
+                                hi[e] = *reinterpret_cast<const uint32_t *>(&hh);
+                                lo[e] = pack2(v[2 * e] - __low2float(hh), v[2 * e + 1] - __high2float(hh));
+                            }
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 16; ++e) hi[e] = lo[e] = 0u;
+                        }
+                        tmem_st16(tb + kColCB + (uint32_t)(32 * c), hi);
+                        tmem_st16(tb + kColCB + (uint32_t)(32 * c + 16), lo);
                     }
-                    if constexpr (sizeof(TOut) == 4) {
+                }
+                tmem_st_wait();
+                tc_before();
+                __syncwarp();
+                if (lane == 0) bar_arrive(sbar(gi, kBarG));
+
+                // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out. The
+                // running state is [p / 4][n][4] per head in the workspace (a warp's 16-byte
+                // loads of one p-quad are contiguous); the first chunk reads
+                // initial_state [p][n], the last one also writes final_state [p][n].
+                ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarSC), ph));
+                tc_after();
+                {
+                    int *flag = w.flags + (b * a.H + h);
+                    if (k > 0 && ok) {
+                        uint32_t i = 0;
+                        while (ld_acquire(flag) < (int)k && i < kFlagTries) {
+                            __nanosleep(32);
+                            ++i;
+                        }
+                        ok = i < kFlagTries;
+                    }
+                    ok = __all_sync(0xffffffffu, ok);
+                    const int n = row;
+                    const size_t blk = (size_t)(b * a.H + h) * kP * kN;
+                    float4 *run4 = reinterpret_cast<float4 *>(w.state + blk) + n;  // quad q at run4[q * kN]
+                    const float decay = exp2_mufu(cs2[kQ - 1]);
+                    // every S_in load of the row issued before any S_out store
+                    float sv[64];
+                    if (ok && k > 0) {
 #pragma unroll
-                        for (int c = 0; c < 2; ++c)
-#pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                *reinterpret_cast<float4 *>(XP + c * kTileHalf + t * 128 + ((i ^ (t & 7)) << 4)) =
-                                    make_float4(yi[32 * c + 4 * i], yi[32 * c + 4 * i + 1], yi[32 * c + 4 * i + 2],
-                                                yi[32 * c + 4 * i + 3]);
+                        for (int q = 0; q < 16; ++q) {
+                            const float4 v4 = run4[q * kN];
+                            sv[4 * q] = v4.x; sv[4 * q + 1] = v4.y; sv[4 * q + 2] = v4.z; sv[4 * q + 3] = v4.w;
+                        }
                     } else {
 #pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            *reinterpret_cast<uint4 *>(XP + t * 128 + ((i ^ (t & 7)) << 4)) =
-                                make_uint4(pack2(yi[8 * i], yi[8 * i + 1]), pack2(yi[8 * i + 2], yi[8 * i + 3]),
-                                           pack2(yi[8 * i + 4], yi[8 * i + 5]), pack2(yi[8 * i + 6], yi[8 * i + 7]));
+                        for (int e = 0; e < 64; ++e) sv[e] = (ok && a.s0) ? a.s0[blk + (size_t)e * kN + n] : 0.0f;
+                    }
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        if (ok) {
+                            float sc[32];
+                            tmem_ld32(tb + kColSC + (uint32_t)(32 * half), sc);
+                            float so[32];
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) so[e] = fmaf(decay, sv[32 * half + e], sc[e]);
+#pragma unroll
+                            for (int q = 0; q < 8; ++q)
+                                run4[(8 * half + q) * kN] = make_float4(so[4 * q], so[4 * q + 1], so[4 * q + 2], so[4 * q + 3]);
+                            if (w.last_chunk == k && a.s_last != nullptr) {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) a.s_last[blk + (size_t)(32 * half + e) * kN + n] = so[e];
+                            }
+                        }
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) {
+                            uint4 hi, lo;
+                            split8(sv + 32 * half + 8 * q, hi, lo);
+                            const int pc = 4 * half + q;
+                            *reinterpret_cast<uint4 *>(XP + mn64_off(n, pc)) = hi;
+                            *reinterpret_cast<uint4 *>(XP + kTileHalf + mn64_off(n, pc)) = lo;
+                        }
                     }
                     fence_async_smem();
-                } else {
-    #pragma unroll
-                    for (int half = 0; half < 2 && ok; ++half) {
-                        float ys[32];
-                        tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
-                        if (t0 + t < L) {
-    #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                float yo[8];
-    #pragma unroll
-                                for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], yi[32 * half + 8 * q + e]);
-                                TOut *yq = yp + 32 * half + 8 * q;
-                                if constexpr (sizeof(TOut) == 4) {
-                                    if (w.y_vec16) {
-                                        float4 *p4 = reinterpret_cast<float4 *>(yq);
-                                        p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
-                                        p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                    tc_before();
+                    // the group's S_out is stored: publish it for chunk k + 1 (the release
+                    // orders the group's stores, which the barrier put before it)
+                    ok = sync_and<kGroupThreads>(gbar, ok);
+                    if (gtid == 0 && ok) st_release(flag, (int)k + 1);
+                }
+                __syncwarp();
+                if (lane == 0) bar_arrive(sbar(gi, kBarS));
+                if (!ok) break;
+
+                // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t (row t, all 64 columns p): Y_i and
+                // D x first, while Y_s is still being formed
+                ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarYI), ph));
+                tc_after();
+                if (ok) {
+                    const int t = row;
+                    const float et = exp2_mufu(cs2[t]);
+                    const float Dh = a.D ? __ldg(a.D + h) : 0.0f;
+                    TOut *yp = static_cast<TOut *>(a.y) + b * a.y_sb + (t0 + t) * a.y_sl + h * a.y_sh;
+                    float yi[64];
+                    tmem_ld32(tb + kColYI, *reinterpret_cast<float(*)[32]>(yi));
+                    tmem_ld32(tb + kColYI + 32u, *reinterpret_cast<float(*)[32]>(yi + 32));
+#pragma unroll
+                    for (int pc = 0; pc < 8; ++pc) {
+                        float xv[8];
+                        unpack8(*reinterpret_cast<const uint4 *>(X + mn64_off(t, pc)), xv);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) yi[8 * pc + e] = fmaf(Dh, xv[e], yi[8 * pc + e]);
+                    }
+                    ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYS), ph));
+                    tc_after();
+                    if (w.y_tma) {
+                        // y row t into the staging buffer (S_in has been consumed by Y_s) in the
+                        // tensor map's box layout: rows of 128 bytes, 16-byte chunk i of row t
+                        // at chunk i ^ (t % 8) (128-byte swizzle); fp32: two boxes of 32
+                        // columns, bf16: one box of 64
+#pragma unroll
+                        for (int half = 0; half < 2 && ok; ++half) {
+                            float ys[32];
+                            tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
+#pragma unroll
+                            for (int e = 0; e < 32; ++e) yi[32 * half + e] = fmaf(et, ys[e], yi[32 * half + e]);
+                        }
+                        if constexpr (sizeof(TOut) == 4) {
+#pragma unroll
+                            for (int c = 0; c < 2; ++c)
+#pragma unroll
+                                for (int i = 0; i < 8; ++i)
+                                    *reinterpret_cast<float4 *>(XP + c * kTileHalf + t * 128 + ((i ^ (t & 7)) << 4)) =
+                                        make_float4(yi[32 * c + 4 * i], yi[32 * c + 4 * i + 1], yi[32 * c + 4 * i + 2],
+                                                    yi[32 * c + 4 * i + 3]);
+                        } else {
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                *reinterpret_cast<uint4 *>(XP + t * 128 + ((i ^ (t & 7)) << 4)) =
+                                    make_uint4(pack2(yi[8 * i], yi[8 * i + 1]), pack2(yi[8 * i + 2], yi[8 * i + 3]),
+                                               pack2(yi[8 * i + 4], yi[8 * i + 5]), pack2(yi[8 * i + 6], yi[8 * i + 7]));
+                        }
+                        fence_async_smem();
+                    } else {
+#pragma unroll
+                        for (int half = 0; half < 2 && ok; ++half) {
+                            float ys[32];
+                            tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
+                            if (t0 + t < L) {
+#pragma unroll
+                                for (int q = 0; q < 4; ++q) {
+                                    float yo[8];
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) yo[e] = fmaf(et, ys[8 * q + e], yi[32 * half + 8 * q + e]);
+                                    TOut *yq = yp + 32 * half + 8 * q;
+                                    if constexpr (sizeof(TOut) == 4) {
+                                        if (w.y_vec16) {
+                                            float4 *p4 = reinterpret_cast<float4 *>(yq);
+                                            p4[0] = make_float4(yo[0], yo[1], yo[2], yo[3]);
+                                            p4[1] = make_float4(yo[4], yo[5], yo[6], yo[7]);
+                                        } else {
+                                            float2 *p2 = reinterpret_cast<float2 *>(yq);
+#pragma unroll
+                                            for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
+                                        }
                                     } else {
-                                        float2 *p2 = reinterpret_cast<float2 *>(yq);
-    #pragma unroll
-                                        for (int e = 0; e < 4; ++e) p2[e] = make_float2(yo[2 * e], yo[2 * e + 1]);
-                                    }
-                                } else {
-                                    if (w.y_vec16) {
-                                        *reinterpret_cast<uint4 *>(yq) = make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]),
-                                                                                    pack2(yo[4], yo[5]), pack2(yo[6], yo[7]));
-                                    } else {
-                                        uint32_t *p1 = reinterpret_cast<uint32_t *>(yq);
-    #pragma unroll
-                                        for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                        if (w.y_vec16) {
+                                            *reinterpret_cast<uint4 *>(yq) = make_uint4(pack2(yo[0], yo[1]), pack2(yo[2], yo[3]),
+                                                                                        pack2(yo[4], yo[5]), pack2(yo[6], yo[7]));
+                                        } else {
+                                            uint32_t *p1 = reinterpret_cast<uint32_t *>(yq);
+#pragma unroll
+                                            for (int e = 0; e < 4; ++e) p1[e] = pack2(yo[2 * e], yo[2 * e + 1]);
+                                        }
                                     }
                                 }
                             }
                         }
                     }
-                }
-                }
-            if (w.y_tma) {
-                // every thread of the group has staged its row (or given up): one thread
-                // stores the tile (rows past the sequence are outside the map, not written)
-                ok = sync_and<kGroupThreads>(gbar, ok);
-                if (gtid == 0 && ok) {
-                    if constexpr (sizeof(TOut) == 4) {
-                        tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
-                        tma_store4(&ymap, saddr(XP) + kTileHalf, 32, (int)h, (int)t0, (int)b);
-                    } else {
-                        tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
                     }
-                    bulk_commit();
+                if (w.y_tma) {
+                    // every thread of the group has staged its row (or given up): one thread
+                    // stores the tile (rows past the sequence are outside the map, not written)
+                    ok = sync_and<kGroupThreads>(gbar, ok);
+                    if (gtid == 0 && ok) {
+                        if constexpr (sizeof(TOut) == 4) {
+                            tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
+                            tma_store4(&ymap, saddr(XP) + kTileHalf, 32, (int)h, (int)t0, (int)b);
+                        } else {
+                            tma_store4(&ymap, saddr(XP), 0, (int)h, (int)t0, (int)b);
+                        }
+                        bulk_commit();
+                    }
+                }
+                tc_before();
+                ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
+                if (!ok) break;
+                // the group is done with x of head j: the buffer takes the group's next head,
+                // in this item or (once its descriptor is in) the next item's first
+                if (j + 2 < nh) {
+                    load_x(d, j + 2);
+                } else {
+                    const bool gn = bar_wait(bar(kBarParFull + (pb ^ 1)), (uint32_t)(((it + 1) >> 1) & 1));
+                    ok = ok && gn;
+                    if (gn) {
+                        const ItemDesc &dn = desc[pb ^ 1];
+                        if (dn.valid && gi < dn.nh) {
+                            load_x(dn, gi);
+                            x_ahead = true;
+                        }
+                    }
                 }
             }
-            tc_before();
-            // the group is done with x of head j: the buffer takes head j + 2
-            ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
-            if (!ok) break;
-            load_x(j + 2);
+            // every warp of the group is done with this item's parameters and descriptor
+            __syncwarp();
+            if (lane == 0) bar_arrive(bar(kBarParFree + pb));
         }
-        if (!ok && gtid == 0) {
+        if (!fin && gtid == 0) {
             *abort_flag = 1u;
             if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
         }
@@ -784,12 +898,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
 }
 
 template <typename TOut>
-cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, const CUtensorMap &ymap, int64_t items,
+cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, const CUtensorMap &ymap, int64_t items, int num_sms,
                      cudaStream_t stream) {
     static SmemOptIn opt_in;
     cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_fwd_tc_kernel<TOut>), kSmemBytes);
     if (e != cudaSuccess) return e;
-    ssd_fwd_tc_kernel<TOut><<<(unsigned)items, kThreads, kSmemBytes, stream>>>(a, w, ymap);
+    // persistent: one CTA per SM (the shared memory allows no second), items claimed in ticket order
+    const int64_t grid = (num_sms > 0 && items > (int64_t)num_sms) ? (int64_t)num_sms : items;
+    ssd_fwd_tc_kernel<TOut><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, w, ymap);
     return cudaGetLastError();
 }
 
@@ -872,6 +988,7 @@ cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, 
     w.counter = w.flags + a.batch * a.H;
     w.state = reinterpret_cast<float *>(static_cast<unsigned char *>(workspace) + flags_al);
     w.last_chunk = nch - 1;
+    w.items = items;
     const size_t ysz = out_bf16 ? 2 : 4;
     w.y_vec16 = ((reinterpret_cast<uintptr_t>(a.y) % 16) == 0 && (a.y_sb * ysz) % 16 == 0 && (a.y_sl * ysz) % 16 == 0 &&
                  (a.y_sh * ysz) % 16 == 0)
@@ -885,7 +1002,8 @@ cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, 
                   : 0;
     cudaError_t e = cudaMemsetAsync(workspace, 0, flags, stream);
     if (e != cudaSuccess) return e;
-    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, ymap, items, stream) : launch_t<float>(a, w, ymap, items, stream);
+    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, ymap, items, num_sms, stream)
+                    : launch_t<float>(a, w, ymap, items, num_sms, stream);
 }
 
 }  // namespace ms

@@ -590,16 +590,16 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         bool x_ahead = false;  // x of the group's first head of the next item is requested
         uint32_t used = 0;     // heads this group has taken (barrier parities of its slot)
 
-        auto load_x = [&](const ItemDesc &d, int j) {  // by the group's threads
-            const __nv_bfloat16 *xh =
-                static_cast<const __nv_bfloat16 *>(a.x) + d.b * a.x_sb + (d.h0 + j) * a.x_sh;
-            const int64_t xt0 = d.k * kQ;
+        // x of head j of item d: each thread copies its own token row, the only row
+        // it reads (X' and D x); rows past L are zero-filled
+        auto load_x = [&](const ItemDesc &d, int j) {
+            const int64_t ts = d.k * kQ + row;
+            const bool in = ts < L;
+            const __nv_bfloat16 *src =
+                static_cast<const __nv_bfloat16 *>(a.x) + d.b * a.x_sb + (d.h0 + j) * a.x_sh + (in ? ts : 0) * a.x_sl;
             const uint32_t dst = saddr(X);
-            for (int i = gtid; i < kQ * (kP / 8); i += kGroupThreads) {
-                const int s = i >> 3, pc = i & 7;
-                const bool in = xt0 + s < L;
-                cp_async16(dst + mn64_off(s, pc), xh + (in ? xt0 + s : 0) * a.x_sl + 8 * pc, in ? 16 : 0);
-            }
+#pragma unroll
+            for (int pc = 0; pc < 8; ++pc) cp_async16(dst + mn64_off(row, pc), src + 8 * pc, in ? 16 : 0);
             cp_commit();
         };
 
@@ -775,7 +775,23 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
 #pragma unroll
                         for (int e = 0; e < 8; ++e) yi[8 * pc + e] = fmaf(Dh, xv[e], yi[8 * pc + e]);
                     }
-                    ok = __all_sync(0xffffffffu, bar_wait(sbar(gi, kBarYS), ph));
+                    // this thread is done with its x row and Y_i has read the tile: the row
+                    // takes the group's next head, in this item or (once its descriptor is
+                    // in) the next item's first, while Y_s completes
+                    if (j + 2 < nh) {
+                        load_x(d, j + 2);
+                    } else {
+                        const bool gn = bar_wait(bar(kBarParFull + (pb ^ 1)), (uint32_t)(((it + 1) >> 1) & 1));
+                        ok = ok && gn;
+                        if (gn) {
+                            const ItemDesc &dn = desc[pb ^ 1];
+                            if (dn.valid && gi < dn.nh) {
+                                load_x(dn, gi);
+                                x_ahead = true;
+                            }
+                        }
+                    }
+                    ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarYS), ph));
                     tc_after();
                     if (w.y_tma) {
                         // y row t into the staging buffer (S_in has been consumed by Y_s) in the
@@ -859,21 +875,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 tc_before();
                 ok = sync_and<kGroupThreads>(gbar, ok && *abort_flag == 0u);
                 if (!ok) break;
-                // the group is done with x of head j: the buffer takes the group's next head,
-                // in this item or (once its descriptor is in) the next item's first
-                if (j + 2 < nh) {
-                    load_x(d, j + 2);
-                } else {
-                    const bool gn = bar_wait(bar(kBarParFull + (pb ^ 1)), (uint32_t)(((it + 1) >> 1) & 1));
-                    ok = ok && gn;
-                    if (gn) {
-                        const ItemDesc &dn = desc[pb ^ 1];
-                        if (dn.valid && gi < dn.nh) {
-                            load_x(dn, gi);
-                            x_ahead = true;
-                        }
-                    }
-                }
             }
             // every warp of the group is done with this item's parameters and descriptor
             __syncwarp();

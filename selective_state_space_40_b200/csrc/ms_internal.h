@@ -92,6 +92,7 @@ struct SsdTcArgs {
     int hb;
     int y_vec16;  // y rows take 16-byte stores
     int y_tma;    // y is written by tensor stores through the kernel's y map
+    int cb_tma;   // the C and B tiles are read by tensor copies through the kernel's maps
 };
 int ssd_tc_head_block(int64_t batch, int64_t seqlen, int64_t nheads, int64_t ngroups, int num_sms);
 size_t ssd_tc_workspace_size(int64_t batch, int64_t nheads);

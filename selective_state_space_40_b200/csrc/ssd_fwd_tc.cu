@@ -125,11 +125,13 @@ constexpr int kOffDesc = kOffBar + 8 * kNumBars;                // ItemDesc per 
 constexpr int kOffMisc = kOffDesc + 2 * (int)sizeof(ItemDesc);  // tensor-memory base, -, abort
 constexpr int kSmemBytes = kOffMisc + 16;
 
-// K-major no-swizzle [rows x 128] bf16 tile: core matrix (row / 8, k / 8) at
-// (row / 8) * 2048 + (k / 8) * 128, row % 8 at 16-byte steps inside it.
-__device__ __forceinline__ uint32_t kmaj_off(int row, int kc) {
-    return (uint32_t)((row >> 3) * 2048 + kc * 128 + (row & 7) * 16);
-}
+// C / B tile [128 tokens x 128 states] bf16 as [n / 8][t][n % 8] (the order a
+// tensor copy writes its box {8 states, 128 tokens, 16 state chunks}): core
+// matrix (t / 8, n / 8) -- 8 token rows of 16 bytes -- at (n / 8) * 2048 + (t / 8)
+// * 128. Read K-major (K = n: C, and B in C B^T) the K-direction core stride is
+// 2048 and the token-direction one 128; read M(n)-major (B in B^T X') the
+// K(t)-direction stride is 128 and the n-direction one 2048.
+__device__ __forceinline__ uint32_t cb_off(int t, int kc) { return (uint32_t)(kc * 2048 + t * 16); }
 // MN-major no-swizzle [k rows x 64] bf16 operand (k = token or state, 64
 // columns p): core matrix (k / 8, p / 8) at (k / 8) * 1024 + (p / 8) * 128,
 // k % 8 at 16-byte steps inside it.
@@ -248,6 +250,18 @@ __device__ __forceinline__ void tma_store4(const CUtensorMap *map, uint32_t src,
                  "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
                  : "memory");
 }
+// Tensor copy (no multicast) of a 5-D box into shared memory, completing on an mbarrier
+__device__ __forceinline__ void tma_load5(const CUtensorMap *map, uint32_t dst, uint32_t bar, int c0, int c1, int c2,
+                                          int c3, int c4) {
+    asm volatile(
+        "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5, %6, "
+        "%7}], [%2];" ::"r"(dst),
+        "l"(map), "r"(bar), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(c4)
+        : "memory");
+}
+__device__ __forceinline__ void bar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
@@ -315,7 +329,9 @@ __device__ __forceinline__ void st_release(int *p, int v) {
 
 template <typename TOut>
 __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a, const SsdTcArgs w,
-                                                                  const __grid_constant__ CUtensorMap ymap) {
+                                                                  const __grid_constant__ CUtensorMap ymap,
+                                                                  const __grid_constant__ CUtensorMap cmap,
+                                                                  const __grid_constant__ CUtensorMap bmap) {
     extern __shared__ __align__(1024) unsigned char smem[];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t sbase = saddr(smem);
@@ -369,6 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         // loads the item's C and B tiles once the previous item's products are done
         // with them. The next item is thus ready while the current one computes.
         bool ok = true;
+        int tma_issued = -1;  // the last item whose tiles came by tensor copies
         long long T = 0;
         if (lane == 0) T = (long long)(unsigned)atomicAdd(w.counter, 1);
         T = __shfl_sync(0xffffffffu, T, 0);
@@ -453,22 +470,33 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             // item's products have read theirs
             if (it >= 1) ok = bar_wait(bar(kBarCBFree), (uint32_t)((it - 1) & 1));
             ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
-            if (ok) {
-                const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
-                const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
-                for (int i = lane; i < kQ * (kN / 8); i += 32) {
-                    const int t = i >> 4, kc = i & 15;
-                    const bool in = t0 + t < L;
-                    const int64_t tt = in ? t0 + t : 0;
-                    cp_async16(sbase + kOffC + kmaj_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
-                    cp_async16(sbase + kOffB + kmaj_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
+            if (ok && w.cb_tma) {
+                // two tensor copies (boxes {8, 128, 16, 1, 1}; rows past L zero-filled), their
+                // bytes counted on the barrier
+                if (lane == 0) {
+                    bar_arrive_tx(bar(kBarCBFull), 2u * kQ * kN * 2u);
+                    tma_load5(&cmap, sbase + kOffC, bar(kBarCBFull), 0, (int)t0, 0, (int)g, (int)b);
+                    tma_load5(&bmap, sbase + kOffB, bar(kBarCBFull), 0, (int)t0, 0, (int)g, (int)b);
                 }
-                cp_commit();
-                cp_wait0();          // this lane's copies are in
-                fence_async_smem();  // ... and visible to the tensor cores
+                tma_issued = it;
+            } else {
+                if (ok) {
+                    const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
+                    const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
+                    for (int i = lane; i < kQ * (kN / 8); i += 32) {
+                        const int t = i >> 4, kc = i & 15;
+                        const bool in = t0 + t < L;
+                        const int64_t tt = in ? t0 + t : 0;
+                        cp_async16(sbase + kOffC + cb_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
+                        cp_async16(sbase + kOffB + cb_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
+                    }
+                    cp_commit();
+                    cp_wait0();          // this lane's copies are in
+                    fence_async_smem();  // ... and visible to the tensor cores
+                }
+                __syncwarp();
+                if (lane == 0) bar_arrive(bar(kBarCBFull));
             }
-            __syncwarp();
-            if (lane == 0) bar_arrive(bar(kBarCBFull));
             if (!ok) break;
             T = __shfl_sync(0xffffffffu, Tn, 0);
         }
@@ -476,6 +504,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             *abort_flag = 1u;
             if (a.status) atomicOr(a.status, MS_ERR_TIMEOUT);
         }
+        // the last tensor copies have landed before the CTA can exit (bounded; at once
+        // when the MMA warp has consumed them)
+        if (tma_issued >= 0 && lane == 0) (void)bar_wait(bar(kBarCBFull), (uint32_t)(tma_issued & 1));
     } else if (warp == kMmaWarp) {
         // ================================ MMA warp ================================
         if (lane == 0) {
@@ -489,7 +520,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
 #pragma unroll 1
                 for (int ks = 0; ks < kN / 16; ++ks)
-                    mma(tb + kColCB, desc_k(sC + 256u * ks, 128u, 2048u), desc_k(sB + 256u * ks, 128u, 2048u),
+                    mma(tb + kColCB, desc_k(sC + 4096u * ks, 2048u, 128u), desc_k(sB + 4096u * ks, 2048u, 128u),
                         idesc(kQ, false, false), ks > 0);
                 mma_commit(sbar(sl, kBarCB));
             };
@@ -528,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                             for (int ks = 0; ks < kQ / 16; ++ks)
 #pragma unroll
                                 for (int part = 0; part < 2; ++part)
-                                    mma(tb + kColSC, desc_mn(sB + 4096u * ks, 2048u, 128u),
+                                    mma(tb + kColSC, desc_mn(sB + 256u * ks, 128u, 2048u),
                                         desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
                                         idesc(kP, true, true), ks > 0 || part > 0);
                             mma_commit(sbar(sl, kBarSC));
@@ -547,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                             for (int ks = 0; ks < kN / 16; ++ks)
 #pragma unroll
                                 for (int part = 0; part < 2; ++part)
-                                    mma(tb + kColSC, desc_k(sC + 256u * ks, 128u, 2048u),
+                                    mma(tb + kColSC, desc_k(sC + 4096u * ks, 2048u, 128u),
                                         desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
                                         idesc(kP, false, true), ks > 0 || part > 0);
                             mma_commit(sbar(sl, kBarYS));
@@ -899,14 +930,14 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
 }
 
 template <typename TOut>
-cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, const CUtensorMap &ymap, int64_t items, int num_sms,
-                     cudaStream_t stream) {
+cudaError_t launch_t(const SsdArgs &a, const SsdTcArgs &w, const CUtensorMap &ymap, const CUtensorMap &cmap,
+                     const CUtensorMap &bmap, int64_t items, int num_sms, cudaStream_t stream) {
     static SmemOptIn opt_in;
     cudaError_t e = opt_in.ensure(reinterpret_cast<const void *>(ssd_fwd_tc_kernel<TOut>), kSmemBytes);
     if (e != cudaSuccess) return e;
     // persistent: one CTA per SM (the shared memory allows no second), items claimed in ticket order
     const int64_t grid = (num_sms > 0 && items > (int64_t)num_sms) ? (int64_t)num_sms : items;
-    ssd_fwd_tc_kernel<TOut><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, w, ymap);
+    ssd_fwd_tc_kernel<TOut><<<(unsigned)grid, kThreads, kSmemBytes, stream>>>(a, w, ymap, cmap, bmap);
     return cudaGetLastError();
 }
 
@@ -943,6 +974,26 @@ bool encode_y(CUtensorMap *m, const SsdArgs &a, bool bf16) {
     const cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
     return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, a.y, dims, strides, box,
               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// B or C [batch][L][G][128] bf16 as a 5-D map {8 states, t, 16 state chunks, g, b}
+// (the row's 128 states split into chunk and element, chunk outside t): the box
+// {8, 128, 16, 1, 1} lands as [n / 8][t][n % 8]; rows t >= L lie outside the map
+// and read as zeros.
+bool encode_cb(CUtensorMap *m, const void *base, int64_t sb, int64_t sl, int64_t sg, const SsdArgs &a) {
+    PfnEncodeTiled fn = encode_fn();
+    if (!fn || reinterpret_cast<uintptr_t>(base) % 16 != 0) return false;
+    const uint64_t bsl = (uint64_t)sl * 2;
+    const uint64_t bsg = a.G > 1 ? (uint64_t)sg * 2 : 16;
+    const uint64_t bsb = a.batch > 1 ? (uint64_t)sb * 2 : 16;
+    if (bsl == 0 || bsl % 16 != 0 || bsg == 0 || bsg % 16 != 0 || bsb == 0 || bsb % 16 != 0) return false;
+    const cuuint64_t dims[5] = {8u, (cuuint64_t)a.L, (cuuint64_t)(kN / 8), (cuuint64_t)a.G, (cuuint64_t)a.batch};
+    const cuuint64_t strides[4] = {(cuuint64_t)bsl, 16u, (cuuint64_t)bsg, (cuuint64_t)bsb};
+    const cuuint32_t box[5] = {8u, (cuuint32_t)kQ, (cuuint32_t)(kN / 8), 1u, 1u};
+    const cuuint32_t estr[5] = {1u, 1u, 1u, 1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void *>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1001,10 +1052,17 @@ cudaError_t launch_ssd_fwd_tc(const SsdArgs &a, bool out_bf16, void *workspace, 
                encode_y(&ymap, a, out_bf16))
                   ? 1
                   : 0;
+    CUtensorMap cmap, bmap;
+    memset(&cmap, 0, sizeof(cmap));
+    memset(&bmap, 0, sizeof(bmap));
+    w.cb_tma = (a.L <= 0x7fffffff && a.batch <= 0x7fffffff && a.G <= 0x7fffffff &&
+                encode_cb(&cmap, a.C, a.C_sb, a.C_sl, a.C_sg, a) && encode_cb(&bmap, a.B, a.B_sb, a.B_sl, a.B_sg, a))
+                   ? 1
+                   : 0;
     cudaError_t e = cudaMemsetAsync(workspace, 0, flags, stream);
     if (e != cudaSuccess) return e;
-    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, ymap, items, num_sms, stream)
-                    : launch_t<float>(a, w, ymap, items, num_sms, stream);
+    return out_bf16 ? launch_t<__nv_bfloat16>(a, w, ymap, cmap, bmap, items, num_sms, stream)
+                    : launch_t<float>(a, w, ymap, cmap, bmap, items, num_sms, stream);
 }
 
 }  // namespace ms

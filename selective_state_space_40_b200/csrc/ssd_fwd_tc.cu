@@ -106,7 +106,7 @@ constexpr int kOffC = 0;                          // C tile   [t][n] K-major, 32
 constexpr int kOffB = kOffC + kQ * kN * 2;        // B tile   [s][n], 32 KB
 constexpr int kOffSlot = kOffB + kQ * kN * 2;     // per slot: X' / S_in hi, lo 32 KB; x [s][p] MN-major 16 KB
 constexpr int kSlotBytes = 3 * kTileHalf;
-constexpr int kParBytes = 3 * kHB * kQ * 4;          // dl, cs2, w: [kHB][kQ] floats each
+constexpr int kParBytes = 4 * kHB * kQ * 4;          // dl, cs2, w, fd: [kHB][kQ] floats each
 constexpr int kOffPar = kOffSlot + 2 * kSlotBytes;  // two parameter buffers (items alternate)
 constexpr int kOffBar = kOffPar + 2 * kParBytes;
 enum { kBarXP = 0, kBarCB, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarsPerSlot };
@@ -404,7 +404,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             if (valid && lane == 0) Tn = (long long)(unsigned)atomicAdd(w.counter, 1);
             if (valid) {
                 // per head: Delta, cs log2(e) and w_s of the chunk's tokens, 4 tokens a lane
-                float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ;
+                float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ, *fdp = wp + kHB * kQ;
                 const unsigned short *dtp = static_cast<const unsigned short *>(a.dt) + b * a.dt_sb + h0;
                 unsigned short raw[kHB][4];
 #pragma unroll
@@ -441,14 +441,21 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                         float run = incl - c;  // sum before this lane's tokens
                         const float total = __shfl_sync(0xffffffffu, incl, 31);
                         const float cend = A2 * total;  // cs_{Q-1} log2(e): padded tokens add nothing
+                        float c2[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             run += dl[i];
+                            c2[i] = A2 * run;
+                        }
+                        // cs of the last token of this lane's 32-token block (lanes 8c..8c+7)
+                        const float cblk = __shfl_sync(0xffffffffu, c2[3], lane | 7);
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
                             const int t = 4 * lane + i;
-                            const float c2 = A2 * run;
                             dlp[jj * kQ + t] = dl[i];
-                            cs2p[jj * kQ + t] = c2;
-                            wp[jj * kQ + t] = exp2_mufu(cend - c2) * dl[i];
+                            cs2p[jj * kQ + t] = c2[i];
+                            wp[jj * kQ + t] = exp2_mufu(cend - c2[i]) * dl[i];
+                            fdp[jj * kQ + t] = exp2_mufu(cblk - c2[i]) * dl[i];
                         }
                     }
                 }
@@ -647,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             }
             const int nh = d.nh;
             const int64_t k = d.k, b = d.b, t0 = k * kQ;
-            const float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ;
+            const float *dlp = params(pb), *cs2p = dlp + kHB * kQ, *wp = cs2p + kHB * kQ, *fdp = wp + kHB * kQ;
             if (gi < nh && !x_ahead) load_x(d, gi);
             x_ahead = false;
 
@@ -688,16 +695,25 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                     const int t = row;
                     const float ct = cs2[t];
                     const float *dls = dlp + j * kQ;
+                    const float *fds = fdp + j * kQ;
 #pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
                         uint32_t hi[16], lo[16];
                         if (c <= qd && ok) {
                             float v[32];
                             tmem_ld32(tb + kColCB + (uint32_t)(32 * c), v);
+                            if (c < qd) {
+                                // block below the diagonal: exp(cs_t - cs_s) = exp(cs_t - m) exp(m - cs_s),
+                                // m = cs of the block's last token, both factors <= 1
+                                const float et = exp2_mufu(ct - cs2[32 * c + 31]);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e) {
-                                const int s = 32 * c + e;
-                                v[e] = (c < qd || s <= t) ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                                for (int e = 0; e < 32; ++e) v[e] = (v[e] * et) * fds[32 * c + e];
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) {
+                                    const int s = 32 * c + e;
+                                    v[e] = s <= t ? v[e] * exp2_mufu(ct - cs2[s]) * dls[s] : 0.0f;
+                                }
                             }
 #pragma unroll
                             for (int e = 0; e < 16; ++e) {

@@ -40,9 +40,12 @@
 // tcgen05.mma and commit) and one producer warp, which claims the next item,
 // forms its per-head Delta, cumulative decay and w_s into the other of two
 // parameter buffers while the current item computes, and loads the item's C
-// and B tiles once the previous item's products are done with them; each
-// group loads x of its first head of the next item behind its last head of
-// this one. The groups take alternate heads of the item, each
+// tile into the other of two C buffers and its B tile once every S_c of the
+// previous item has completed (tensor copies). The MMA warp runs each slot's
+// heads as its own sequence, so a group enters the next item while the other
+// finishes this one; each thread of a group copies its x row of the group's
+// next head as soon as it has read the current one. The groups take alternate
+// heads of the item, each
 // with its own half of tensor memory (a slot: CB, overwritten in place by G'
 // as packed bf16 hi / lo, the A operand of Y_i; S_c, later Y_s; Y_i) and its
 // own x and X' (later S_in) buffers, so one group's products run while the
@@ -71,6 +74,11 @@
 #ifndef MS_SSD_MN_LBO_K
 #define MS_SSD_MN_LBO_K 1
 #endif
+// Back-off (ns) of the MMA warp's polling rounds that find no event: the warp
+// shares its scheduler with compute warps.
+#ifndef MS_SSD_POLL_NS
+#define MS_SSD_POLL_NS 20
+#endif
 
 namespace ms {
 
@@ -79,7 +87,7 @@ namespace {
 constexpr int kQ = 128;        // tokens per chunk
 constexpr int kP = 64;         // head dim
 constexpr int kN = 128;        // state size
-constexpr int kHB = 8;         // most heads per work item
+constexpr int kHB = 4;         // most heads per work item
 constexpr int kGroupWarps = 4;                       // one warp per 32 accumulator lanes
 constexpr int kGroupThreads = 32 * kGroupWarps;
 constexpr int kComputeWarps = 2 * kGroupWarps;
@@ -102,9 +110,10 @@ constexpr uint32_t kIdleTries = 1u << 24;       // MMA warp polls without an eve
 
 // shared-memory map (bytes)
 constexpr int kTileHalf = kQ * kP * 2;            // 16 KB: one [128 x 64] bf16 operand
-constexpr int kOffC = 0;                          // C tile   [t][n] K-major, 32 KB
-constexpr int kOffB = kOffC + kQ * kN * 2;        // B tile   [s][n], 32 KB
-constexpr int kOffSlot = kOffB + kQ * kN * 2;     // per slot: X' / S_in hi, lo 32 KB; x [s][p] MN-major 16 KB
+constexpr int kTileCB = kQ * kN * 2;              // one C or B tile, 32 KB
+constexpr int kOffC = 0;                          // two C tiles (items alternate)
+constexpr int kOffB = kOffC + 2 * kTileCB;        // the B tile
+constexpr int kOffSlot = kOffB + kTileCB;         // per slot: X' / S_in hi, lo 32 KB; x [s][p] MN-major 16 KB
 constexpr int kSlotBytes = 3 * kTileHalf;
 constexpr int kParBytes = 4 * kHB * kQ * 4;          // dl, cs2, w, fd: [kHB][kQ] floats each
 constexpr int kOffPar = kOffSlot + 2 * kSlotBytes;  // two parameter buffers (items alternate)
@@ -112,9 +121,11 @@ constexpr int kOffBar = kOffPar + 2 * kParBytes;
 enum { kBarXP = 0, kBarCB, kBarSC, kBarG, kBarYI, kBarS, kBarYS, kBarsPerSlot };
 constexpr int kBarParFull = 2 * kBarsPerSlot;  // [2] an item's descriptor and parameters are in buffer i
 constexpr int kBarParFree = kBarParFull + 2;   // [2] every consumer is done with buffer i
-constexpr int kBarCBFull = kBarParFree + 2;    // the current item's C and B tiles are in
-constexpr int kBarCBFree = kBarCBFull + 1;     // the current item's products are done with them
-constexpr int kBarEnd = kBarCBFree + 1, kNumBars = kBarEnd + 1;
+constexpr int kBarCFull = kBarParFree + 2;     // [2] item i's C tile is in buffer i % 2
+constexpr int kBarCFree = kBarCFull + 2;       // [2] the products of the item in C buffer i are done
+constexpr int kBarBFull = kBarCFree + 2;       // the B tile of the next item to read it is in
+constexpr int kBarBFree = kBarBFull + 1;       // every product reading an item's B tile is done
+constexpr int kBarEnd = kBarBFree + 1, kNumBars = kBarEnd + 1;
 
 // A work item as the producer warp hands it to the others (valid = 0: no more)
 struct ItemDesc {
@@ -356,8 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             bar_init(bar(kBarParFull + pb), 1);
             bar_init(bar(kBarParFree + pb), kComputeWarps + 1);
         }
-        bar_init(bar(kBarCBFull), 1);
-        bar_init(bar(kBarCBFree), 1);
+        for (int cb = 0; cb < 2; ++cb) {
+            bar_init(bar(kBarCFull + cb), 1);
+            bar_init(bar(kBarCFree + cb), 1);
+        }
+        bar_init(bar(kBarBFull), 1);
+        bar_init(bar(kBarBFree), 1);
         bar_init(bar(kBarEnd), 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
@@ -385,8 +400,33 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         // loads the item's C and B tiles once the previous item's products are done
         // with them. The next item is thus ready while the current one computes.
         bool ok = true;
-        int tma_issued = -1;  // the last item whose tiles came by tensor copies
+        int tma_last = -1;  // the last item whose tiles came by tensor copies
         long long T = 0;
+        // one C or B tile [128 tokens x 128 states] (rows past L zero-filled): a tensor copy
+        // whose bytes the barrier counts, else 16-byte copies by the warp; the barrier is
+        // arrived on either way (also when the CTA is stopping)
+        auto load_tile = [&](bool go, const CUtensorMap *map, const __nv_bfloat16 *src, int64_t sl, uint32_t dst,
+                             uint32_t br, int64_t t0, int64_t g, int64_t b) {
+            if (go && w.cb_tma) {
+                if (lane == 0) {
+                    bar_arrive_tx(br, (uint32_t)kTileCB);
+                    tma_load5(map, dst, br, 0, (int)t0, 0, (int)g, (int)b);
+                }
+                return;
+            }
+            if (go) {
+                for (int i = lane; i < kQ * (kN / 8); i += 32) {
+                    const int t = i >> 4, kc = i & 15;
+                    const bool in = t0 + t < L;
+                    cp_async16(dst + cb_off(t, kc), src + (in ? t0 + t : 0) * sl + 8 * kc, in ? 16 : 0);
+                }
+                cp_commit();
+                cp_wait0();          // this lane's copies are in
+                fence_async_smem();  // ... and visible to the tensor cores
+            }
+            __syncwarp();
+            if (lane == 0) bar_arrive(br);
+        };
         if (lane == 0) T = (long long)(unsigned)atomicAdd(w.counter, 1);
         T = __shfl_sync(0xffffffffu, T, 0);
         for (int it = 0;; ++it) {
@@ -473,37 +513,17 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             __syncwarp();
             if (lane == 0) bar_arrive(bar(kBarParFull + pb));
             if (!valid) break;
-            // the item's C and B tiles (rows past L zero-filled), once the previous
-            // item's products have read theirs
-            if (it >= 1) ok = bar_wait(bar(kBarCBFree), (uint32_t)((it - 1) & 1));
+            // C into buffer it % 2 once item it - 2's products are done with it; B once
+            // every product of item it - 1 that reads B has completed
+            if (it >= 2) ok = bar_wait(bar(kBarCFree + pb), (uint32_t)(((it - 2) >> 1) & 1));
             ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
-            if (ok && w.cb_tma) {
-                // two tensor copies (boxes {8, 128, 16, 1, 1}; rows past L zero-filled), their
-                // bytes counted on the barrier
-                if (lane == 0) {
-                    bar_arrive_tx(bar(kBarCBFull), 2u * kQ * kN * 2u);
-                    tma_load5(&cmap, sbase + kOffC, bar(kBarCBFull), 0, (int)t0, 0, (int)g, (int)b);
-                    tma_load5(&bmap, sbase + kOffB, bar(kBarCBFull), 0, (int)t0, 0, (int)g, (int)b);
-                }
-                tma_issued = it;
-            } else {
-                if (ok) {
-                    const __nv_bfloat16 *Cg = static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg;
-                    const __nv_bfloat16 *Bg = static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg;
-                    for (int i = lane; i < kQ * (kN / 8); i += 32) {
-                        const int t = i >> 4, kc = i & 15;
-                        const bool in = t0 + t < L;
-                        const int64_t tt = in ? t0 + t : 0;
-                        cp_async16(sbase + kOffC + cb_off(t, kc), Cg + tt * a.C_sl + 8 * kc, in ? 16 : 0);
-                        cp_async16(sbase + kOffB + cb_off(t, kc), Bg + tt * a.B_sl + 8 * kc, in ? 16 : 0);
-                    }
-                    cp_commit();
-                    cp_wait0();          // this lane's copies are in
-                    fence_async_smem();  // ... and visible to the tensor cores
-                }
-                __syncwarp();
-                if (lane == 0) bar_arrive(bar(kBarCBFull));
-            }
+            load_tile(ok, &cmap, static_cast<const __nv_bfloat16 *>(a.C) + b * a.C_sb + g * a.C_sg, a.C_sl,
+                      sbase + (uint32_t)(kOffC + pb * kTileCB), bar(kBarCFull + pb), t0, g, b);
+            if (ok && it >= 1) ok = bar_wait(bar(kBarBFree), (uint32_t)((it - 1) & 1));
+            ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
+            load_tile(ok, &bmap, static_cast<const __nv_bfloat16 *>(a.B) + b * a.B_sb + g * a.B_sg, a.B_sl,
+                      sbase + (uint32_t)kOffB, bar(kBarBFull), t0, g, b);
+            if (ok && w.cb_tma) tma_last = it;
             if (!ok) break;
             T = __shfl_sync(0xffffffffu, Tn, 0);
         }
@@ -513,98 +533,138 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         }
         // the last tensor copies have landed before the CTA can exit (bounded; at once
         // when the MMA warp has consumed them)
-        if (tma_issued >= 0 && lane == 0) (void)bar_wait(bar(kBarCBFull), (uint32_t)(tma_issued & 1));
+        if (tma_last >= 0 && lane == 0) {
+            (void)bar_wait(bar(kBarBFull), (uint32_t)(tma_last & 1));
+            for (int i = tma_last > 0 ? tma_last - 1 : 0; i <= tma_last; ++i)
+                (void)bar_wait(bar(kBarCFull + (i & 1)), (uint32_t)((i >> 1) & 1));
+        }
     } else if (warp == kMmaWarp) {
         // ================================ MMA warp ================================
         if (lane == 0) {
-            const uint32_t sC = sbase + kOffC, sB = sbase + kOffB;
+            const uint32_t sB = sbase + kOffB;
+            auto sC = [&](int cb) { return sbase + (uint32_t)(kOffC + cb * kTileCB); };
             bool ok = true;
+            // Each slot runs its own sequence of heads (s, s + 2, ... of every item) and
+            // may enter the next item while the other finishes this one. Per slot: item,
+            // head, step (-1: item's descriptor; 0: C B^T once the item's tiles are in;
+            // 1: X' ready -> S_c; 2: G' ready -> Y_i; 3: S_in ready -> Y_s).
+            int s_it[2] = {0, 0}, s_j[2] = {0, 1}, s_step[2] = {-1, -1};
+            bool s_done[2] = {false, false};
             uint32_t used[2] = {0u, 0u};  // heads each slot has taken (barrier parities)
+            // per item parity: the item read, its heads and validity, and the slots still to
+            // issue their last S_c (the item's last B readers) and their last Y_s (C readers)
+            int known[2] = {-1, -1}, inh[2] = {0, 0}, ivalid[2] = {0, 0}, sc_left[2] = {0, 0}, ys_left[2] = {0, 0};
+            uint32_t idle = 0;
             // CB = C B^T (both K-major) into a slot's first 128 columns: issued behind the
-            // slot's previous head's Y_i (products run in issue order, so that head's G'
-            // has been read), so the group finds it ready
-            auto issue_cb = [&](int sl) {
+            // slot's previous head's last product (products run in issue order, so that
+            // head's G' has been read), so the group finds it ready
+            auto issue_cb = [&](int sl, int cb) {
                 const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
 #pragma unroll 1
                 for (int ks = 0; ks < kN / 16; ++ks)
-                    mma(tb + kColCB, desc_k(sC + 4096u * ks, 2048u, 128u), desc_k(sB + 4096u * ks, 2048u, 128u),
+                    mma(tb + kColCB, desc_k(sC(cb) + 4096u * ks, 2048u, 128u), desc_k(sB + 4096u * ks, 2048u, 128u),
                         idesc(kQ, false, false), ks > 0);
                 mma_commit(sbar(sl, kBarCB));
             };
-            for (int it = 0; ok; ++it) {
-                const int pb = it & 1;
-                ok = bar_wait(bar(kBarParFull + pb), (uint32_t)((it >> 1) & 1)) && *abort_flag == 0u;
-                if (!ok) break;
-                const int nh = desc[pb].nh, valid = desc[pb].valid;
-                bar_arrive(bar(kBarParFree + pb));  // the descriptor is all this warp reads
-                if (!valid) break;
-                ok = bar_wait(bar(kBarCBFull), (uint32_t)(it & 1)) && *abort_flag == 0u;
-                if (!ok) break;
-                tc_after();
-                issue_cb(0);
-                if (nh > 1) issue_cb(1);
-                // per slot: its next head and step (0: X' ready -> S_c; 1: G' ready -> Y_i;
-                // 2: S_in ready -> Y_s); slot s takes heads s, s + 2, ...
-                int jn[2] = {0, 1}, step[2] = {0, 0};
-                uint32_t idle = 0;
-                while (ok && (jn[0] < nh || jn[1] < nh)) {
-                    bool progressed = false;
-#pragma unroll 1
-                    for (int sl = 0; sl < 2; ++sl) {
-                        const int j = jn[sl];
-                        if (j >= nh) continue;
-                        const uint32_t ph = (used[sl] + (uint32_t)(j >> 1)) & 1u;
-                        const int ev = step[sl] == 0 ? kBarXP : (step[sl] == 1 ? kBarG : kBarS);
-                        if (!bar_test(sbar(sl, ev), ph)) continue;
-                        tc_after();
-                        const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
-                        const uint32_t sXP = sbase + (uint32_t)(kOffSlot + sl * kSlotBytes);
-                        const uint32_t sX = sXP + (uint32_t)(2 * kTileHalf);
-                        if (step[sl] == 0) {
-                            // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo)
-#pragma unroll 1
-                            for (int ks = 0; ks < kQ / 16; ++ks)
+            while (ok && !(s_done[0] && s_done[1])) {
+                bool progressed = false;
 #pragma unroll
-                                for (int part = 0; part < 2; ++part)
-                                    mma(tb + kColSC, desc_mn(sB + 256u * ks, 128u, 2048u),
-                                        desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                                        idesc(kP, true, true), ks > 0 || part > 0);
-                            mma_commit(sbar(sl, kBarSC));
-                        } else if (step[sl] == 1) {
-                            // Y_i [t x p] = G' X: A = G' (hi, lo) packed in tensor memory, B = x
-#pragma unroll 1
-                            for (int ks = 0; ks < kQ / 16; ++ks)
-#pragma unroll
-                                for (int part = 0; part < 2; ++part)
-                                    mma_ts(tb + kColYI, tb + g_col(ks, part), desc_mn(sX + 2048u * ks, 1024u, 128u),
-                                           idesc(kP, false, true), ks > 0 || part > 0);
-                            mma_commit(sbar(sl, kBarYI));
-                        } else {
-                            // Y_s [t x p] = C S_in (hi, lo), into S_c's columns
-#pragma unroll 1
-                            for (int ks = 0; ks < kN / 16; ++ks)
-#pragma unroll
-                                for (int part = 0; part < 2; ++part)
-                                    mma(tb + kColSC, desc_k(sC + 4096u * ks, 2048u, 128u),
-                                        desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
-                                        idesc(kP, false, true), ks > 0 || part > 0);
-                            mma_commit(sbar(sl, kBarYS));
-                            if (j + 2 < nh) issue_cb(sl);
+                for (int sl = 0; sl < 2; ++sl) {
+                    if (s_done[sl]) continue;
+                    const int it = s_it[sl], pb = it & 1;
+                    if (s_step[sl] < 0) {
+                        if (known[pb] != it) {
+                            if (!bar_test(bar(kBarParFull + pb), (uint32_t)((it >> 1) & 1))) continue;
+                            inh[pb] = desc[pb].nh;
+                            ivalid[pb] = desc[pb].valid;
+                            known[pb] = it;
+                            sc_left[pb] = ys_left[pb] = inh[pb] < 2 ? inh[pb] : 2;
+                            bar_arrive(bar(kBarParFree + pb));  // the descriptor is all this warp reads
                         }
-                        if (++step[sl] == 3) {
-                            step[sl] = 0;
-                            jn[sl] += 2;
+                        if (!ivalid[pb]) {
+                            s_done[sl] = true;
+                        } else if (s_j[sl] >= inh[pb]) {
+                            s_it[sl] = it + 1;  // no head of this item for the slot
+                            s_j[sl] = sl;
+                        } else {
+                            s_step[sl] = 0;
                         }
                         progressed = true;
+                        continue;
                     }
-                    if (progressed) idle = 0;
-                    else if (++idle > kIdleTries || *abort_flag != 0u) ok = false;
+                    const int j = s_j[sl];
+                    const uint32_t ph = used[sl] & 1u;
+                    const uint32_t tb = tmem + (uint32_t)sl * kSlotCols;
+                    const uint32_t sXP = sbase + (uint32_t)(kOffSlot + sl * kSlotBytes);
+                    const uint32_t sX = sXP + (uint32_t)(2 * kTileHalf);
+                    const bool last = j + 2 >= inh[pb];
+                    if (s_step[sl] == 0) {
+                        if (!bar_test(bar(kBarCFull + pb), (uint32_t)((it >> 1) & 1)) ||
+                            !bar_test(bar(kBarBFull), (uint32_t)(it & 1)))
+                            continue;
+                        tc_after();
+                        issue_cb(sl, pb);
+                        s_step[sl] = 1;
+                        progressed = true;
+                        continue;
+                    }
+                    const int ev = s_step[sl] == 1 ? kBarXP : (s_step[sl] == 2 ? kBarG : kBarS);
+                    if (!bar_test(sbar(sl, ev), ph)) continue;
+                    tc_after();
+                    if (s_step[sl] == 1) {
+                        // S_c [n x p] = B^T X': A = the B tile read M(n)-major, B = X' (hi, lo)
+#pragma unroll 1
+                        for (int ks = 0; ks < kQ / 16; ++ks)
+#pragma unroll
+                            for (int part = 0; part < 2; ++part)
+                                mma(tb + kColSC, desc_mn(sB + 256u * ks, 128u, 2048u),
+                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                    idesc(kP, true, true), ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarSC));
+                        // B is free once the item's last S_c of both slots has completed (each
+                        // slot's C B^T products were issued before its S_c)
+                        if (last && --sc_left[pb] == 0) mma_commit(bar(kBarBFree));
+                        s_step[sl] = 2;
+                    } else if (s_step[sl] == 2) {
+                        // Y_i [t x p] = G' X: A = G' (hi, lo) packed in tensor memory, B = x
+#pragma unroll 1
+                        for (int ks = 0; ks < kQ / 16; ++ks)
+#pragma unroll
+                            for (int part = 0; part < 2; ++part)
+                                mma_ts(tb + kColYI, tb + g_col(ks, part), desc_mn(sX + 2048u * ks, 1024u, 128u),
+                                       idesc(kP, false, true), ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarYI));
+                        s_step[sl] = 3;
+                    } else {
+                        // Y_s [t x p] = C S_in (hi, lo), into S_c's columns
+#pragma unroll 1
+                        for (int ks = 0; ks < kN / 16; ++ks)
+#pragma unroll
+                            for (int part = 0; part < 2; ++part)
+                                mma(tb + kColSC, desc_k(sC(pb) + 4096u * ks, 2048u, 128u),
+                                    desc_mn(sXP + (uint32_t)(part * kTileHalf) + 2048u * ks, 1024u, 128u),
+                                    idesc(kP, false, true), ks > 0 || part > 0);
+                        mma_commit(sbar(sl, kBarYS));
+                        ++used[sl];
+                        if (last) {
+                            // C buffer pb is free once the item's last Y_s of both slots has completed
+                            if (--ys_left[pb] == 0) mma_commit(bar(kBarCFree + pb));
+                            s_it[sl] = it + 1;
+                            s_j[sl] = sl;
+                            s_step[sl] = -1;
+                        } else {
+                            s_j[sl] = j + 2;
+                            s_step[sl] = 0;
+                        }
+                    }
+                    progressed = true;
                 }
-                if (!ok) break;
-                used[0] += (uint32_t)((nh + 1) / 2);
-                used[1] += (uint32_t)(nh / 2);
-                // the C and B tiles are free once this item's products have completed
-                mma_commit(bar(kBarCBFree));
+                if (progressed) {
+                    idle = 0;
+                } else {
+                    if (++idle > kIdleTries || *abort_flag != 0u) ok = false;
+                    __nanosleep(MS_SSD_POLL_NS);  // leave the issue slots to the compute warps
+                }
             }
             if (!ok) {
                 *abort_flag = 1u;

@@ -854,13 +854,15 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                     }
                     fence_async_smem();
                     tc_before();
+                    // this warp has read its S_c rows and written its S_in rows: Y_s may
+                    // overwrite the one and read the other once every warp is here
+                    __syncwarp();
+                    if (lane == 0) bar_arrive(sbar(gi, kBarS));
                     // the group's S_out is stored: publish it for chunk k + 1 (the release
                     // orders the group's stores, which the barrier put before it)
                     ok = sync_and<kGroupThreads>(gbar, ok);
                     if (gtid == 0 && ok) st_release(flag, (int)k + 1);
                 }
-                __syncwarp();
-                if (lane == 0) bar_arrive(sbar(gi, kBarS));
                 if (!ok) break;
 
                 // ---- y_t = exp(cs_t) Y_s[t] + Y_i[t] + D x_t (row t, all 64 columns p): Y_i and

@@ -797,9 +797,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                 // ---- S_out = decay S_in + S_c; S_in (hi, lo) for Y_s; publish S_out. The
                 // running state is [p / 4][n][4] per head in the workspace (a warp's 16-byte
                 // loads of one p-quad are contiguous); the first chunk reads
-                // initial_state [p][n], the last one also writes final_state [p][n].
-                ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarSC), ph));
-                tc_after();
+                // initial_state [p][n], the last one also writes final_state [p][n]. S_in
+                // (once chunk k - 1 has published it) is loaded before the wait for S_c,
+                // so its trip through L2 overlaps the product.
                 {
                     int *flag = w.flags + (b * a.H + h);
                     if (k > 0 && ok) {
@@ -814,7 +814,6 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                     const int n = row;
                     const size_t blk = (size_t)(b * a.H + h) * kP * kN;
                     float4 *run4 = reinterpret_cast<float4 *>(w.state + blk) + n;  // quad q at run4[q * kN]
-                    const float decay = exp2_mufu(cs2[kQ - 1]);
                     // every S_in load of the row issued before any S_out store
                     float sv[64];
                     if (ok && k > 0) {
@@ -827,6 +826,9 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
 #pragma unroll
                         for (int e = 0; e < 64; ++e) sv[e] = (ok && a.s0) ? a.s0[blk + (size_t)e * kN + n] : 0.0f;
                     }
+                    ok = __all_sync(0xffffffffu, ok && bar_wait(sbar(gi, kBarSC), ph));
+                    tc_after();
+                    const float decay = exp2_mufu(cs2[kQ - 1]);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
                         if (ok) {

@@ -82,7 +82,7 @@ def test_initial_state_and_split():
 @pytest.mark.parametrize("b,L,H,G", [(2, 400, 20, 2), (1, 260, 9, 1), (3, 129, 16, 4)])
 def test_head_blocks_and_chunks(b, L, H, G):
     """Several chunks of 128 tokens and several blocks of heads per group (up
-    to 8 heads per work item, a ragged last block), so chunk k's items take
+    to 4 heads per work item, a ragged last block), so chunk k's items take
     their entering state from chunk k - 1's items of the same heads."""
     _, inp = _case(b, L, H, G, 30 + L + H)
     inp["A"] = -torch.exp(torch.randn(H, generator=torch.Generator().manual_seed(L)))  # a decay per head
@@ -95,6 +95,37 @@ def test_head_blocks_and_chunks(b, L, H, G):
     assert int(status.item()) == 0
     yr, fr = oracle.ssd(f64(inp["x"]), f64(inp["dt"]), f64(inp["A"]), f64(inp["B"]), f64(inp["C"]),
                         f64(inp["D"]), f64(inp["dt_bias"]), True, f64(s0))
+    check_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} y")
+    check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
+
+
+@pytest.mark.parametrize("b,L,H,G", [(16, 1024, 7, 1), (8, 2048, 9, 1), (12, 1280, 12, 3)])
+def test_many_items_per_cta(b, L, H, G):
+    """More work items than SMs, so each persistent CTA walks several items:
+    the next item's parameters, C tile, B tile and first x rows arrive while
+    the current one computes, and the two warp groups cross item boundaries
+    apart. Head blocks of 7 and 9 heads per group leave blocks of 3 or 1 head
+    (one group with fewer heads, or none, in those items)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    _, inp = _case(b, L, H, G, 100 + H)
+    inp["A"] = -torch.exp(torch.randn(H, generator=torch.Generator().manual_seed(H)))
+    s0 = 0.3 * torch.randn(b, H, 64, 128, generator=torch.Generator().manual_seed(L))
+    status = torch.zeros(1, dtype=torch.int32, device=DEV)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    y, fs = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                       initial_state=s0.to(DEV), dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+
+    def part(r):
+        return oracle.ssd(f64(inp["x"][r:r + 1]), f64(inp["dt"][r:r + 1]), f64(inp["A"]), f64(inp["B"][r:r + 1]),
+                          f64(inp["C"][r:r + 1]), f64(inp["D"]), f64(inp["dt_bias"]), True, f64(s0[r:r + 1]))
+
+    with ThreadPoolExecutor(max(1, min(16, os.cpu_count() or 1))) as pool:
+        parts = list(pool.map(part, range(b)))
+    yr = np.concatenate([p_[0] for p_ in parts])
+    fr = np.concatenate([p_[1] for p_ in parts])
     check_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} y")
     check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
 

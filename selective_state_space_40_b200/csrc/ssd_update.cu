@@ -7,8 +7,9 @@
 //   y = S C + D x
 // The state is read and written once (the step's traffic); one CTA of 8
 // warps per (b, h): lane l owns columns n in [4l, 4l+4) (one 16-byte access
-// per row), warps stride over the rows p, and each row's readout C . S is a
-// warp sum.
+// per row), warps stride over the rows p with every row's load in flight at
+// once, and each row's readout C . S is a warp sum. Back-to-back steps overlap
+// through programmatic dependent launch.
 
 #include <cstdint>
 
@@ -27,8 +28,17 @@ __device__ __forceinline__ float ldv(const T *p) {
     else return bf16_bits_to_f32(__ldg(reinterpret_cast<const unsigned short *>(p)));
 }
 
+constexpr int kRowsPerWarp = 8;  // rows of the state a warp has in flight (P <= 64)
+
 template <typename TIn, typename TOut>
 __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a) {
+    // Back-to-back steps: this grid may have been scheduled while the previous
+    // kernel on the stream still runs (programmatic dependent launch). Let the
+    // next grid be scheduled, and wait until everything the previous kernel wrote
+    // is complete and visible before reading any memory. Without that launch
+    // attribute both instructions do nothing.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t b = blockIdx.x / a.H, h = blockIdx.x % a.H;
     const int64_t g = h / (a.H / a.G);
@@ -49,19 +59,34 @@ __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a
     const TIn *xr = static_cast<const TIn *>(a.x) + b * a.x_sb + h * a.x_sh;
     TOut *yr = static_cast<TOut *>(a.y) + b * a.y_sb + h * a.y_sh;
     float *st = a.state + b * a.st_sb + h * a.st_sh + 4 * lane;
-#pragma unroll 4
-    for (int p = warp; p < P; p += kUW) {
-        float4 s = *reinterpret_cast<const float4 *>(st + (int64_t)p * N);
-        const float xv = ldv(xr + p);
-        s.x = fmaf(decay, s.x, xv * Bv[0]);
-        s.y = fmaf(decay, s.y, xv * Bv[1]);
-        s.z = fmaf(decay, s.z, xv * Bv[2]);
-        s.w = fmaf(decay, s.w, xv * Bv[3]);
-        *reinterpret_cast<float4 *>(st + (int64_t)p * N) = s;
-        float part = Cv[0] * s.x + Cv[1] * s.y + Cv[2] * s.z + Cv[3] * s.w;
+    // rows p = warp + kUW i; every load of the warp's rows issued before any store
+    for (int p0 = warp; p0 < P; p0 += kUW * kRowsPerWarp) {
+        float4 sv[kRowsPerWarp];
+        float xv[kRowsPerWarp];
 #pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-        if (lane == 0) Elem<TOut>::store(yr + p, part + Dh * xv);
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int p = p0 + kUW * i;
+            if (p < P) {
+                sv[i] = *reinterpret_cast<const float4 *>(st + (int64_t)p * N);
+                xv[i] = ldv(xr + p);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < kRowsPerWarp; ++i) {
+            const int p = p0 + kUW * i;
+            if (p < P) {
+                float4 s = sv[i];
+                s.x = fmaf(decay, s.x, xv[i] * Bv[0]);
+                s.y = fmaf(decay, s.y, xv[i] * Bv[1]);
+                s.z = fmaf(decay, s.z, xv[i] * Bv[2]);
+                s.w = fmaf(decay, s.w, xv[i] * Bv[3]);
+                *reinterpret_cast<float4 *>(st + (int64_t)p * N) = s;
+                float part = Cv[0] * s.x + Cv[1] * s.y + Cv[2] * s.z + Cv[3] * s.w;
+#pragma unroll
+                for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
+                if (lane == 0) Elem<TOut>::store(yr + p, part + Dh * xv[i]);
+            }
+        }
     }
 }
 
@@ -70,8 +95,20 @@ cudaError_t launch_t(const SsdUpdArgs &a, cudaStream_t stream) {
     const int64_t blocks = a.batch * a.H;
     if (blocks <= 0) return cudaSuccess;
     if (blocks > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    ssd_update_kernel<TIn, TOut><<<(unsigned)blocks, kUW * 32, 0, stream>>>(a);
-    return cudaGetLastError();
+    // programmatic dependent launch: the grid is scheduled while the previous
+    // kernel on the stream drains; the kernel waits (griddepcontrol.wait) before
+    // it reads any memory
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)blocks);
+    cfg.blockDim = dim3(kUW * 32);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ssd_update_kernel<TIn, TOut>, a);
 }
 
 }  // namespace

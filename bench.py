@@ -471,7 +471,9 @@ def main(argv=None):
     lasts = [last, torch.empty_like(last)]
     h2d = sum(v.numel() * v.element_size() for v in pinned.values())
     d2h = y_host[0].numel() * 4 + last_host[0].numel() * 4
-    e2e_steps = max(4, min(20, args.steps // 20))
+    # at least 12 pipelined steps (about 40 ms), so the first upload and the last
+    # download weigh little against the steady state
+    e2e_steps = max(12, min(40, args.steps // 10))
     s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
     ev = lambda: torch.cuda.Event()  # noqa: E731
     in_done, comp_done, out_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]

@@ -41,11 +41,18 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")))
 
 
+def headers():
+    """Every header the sources include: csrc/*.h, csrc/*.cuh and include/*.h.
+    An edit to any of them rebuilds every object (they key the object cache)."""
+    return sorted(glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) +
+                  glob.glob(os.path.join(INCLUDE, "*.h")))
+
+
 def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     mt = os.path.getmtime(LIB)
-    deps = sources() + glob.glob(os.path.join(CSRC, "*.h*")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+    deps = sources() + headers()
     return any(os.path.getmtime(p) > mt for p in deps)
 
 
@@ -61,7 +68,7 @@ def build_debug(force: bool = False) -> str:
     the product path)."""
     if not force and os.path.exists(LIB_DEBUG):
         mt = os.path.getmtime(LIB_DEBUG)
-        deps = sources() + glob.glob(os.path.join(CSRC, "*.h*")) + glob.glob(os.path.join(INCLUDE, "*.h"))
+        deps = sources() + headers()
         if all(os.path.getmtime(p) <= mt for p in deps):
             return LIB_DEBUG
     return build(force=True, defines=("MS_DEBUG",), out=LIB_DEBUG)
@@ -83,9 +90,8 @@ def build(force: bool = False, verbose: bool = False, defines=(), out: str = LIB
     flags = [*COMPILE_FLAGS, *(f"-D{d}" for d in defines), "-I", INCLUDE, "-I", CSRC]
     if verbose:
         flags.insert(0, "-Xptxas=-v")
-    headers = sorted(glob.glob(os.path.join(CSRC, "*.h*")) + glob.glob(os.path.join(INCLUDE, "*.h")))
     common = hashlib.sha256(" ".join(flags).encode())
-    for h in headers:
+    for h in headers():
         with open(h, "rb") as f:
             common.update(f.read())
     srcs = sources()

@@ -60,6 +60,12 @@ namespace ms {
 namespace {
 
 constexpr int kT = 32;                 // tokens per tile
+// Instantiations by compute warps per CTA: the block's warps spread over the
+// SM's four schedulers, each with a quarter of the register file, so 12
+// warps leave 168 registers a thread, 16 warps 128 and 19 warps 96.
+constexpr int kMaxWSmall = 11;
+constexpr int kMaxWMid = 15;
+constexpr int kMaxWLarge = 18;
 constexpr int kCW = 8;                 // channels per compute warp (4 lanes each)
 constexpr int kRow = 36;               // floats per padded exchange row (bank spread)
 constexpr int kRowS = 4 * 32 + 4;      // floats per padded row of splatted pairs
@@ -799,6 +805,17 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const int s = k % S, vb = k & 1;
             const int64_t t0 = (int64_t)k * kT;
+            // Training (the 12-warp instantiation only; wider layers' training forwards
+            // take the register engine): the state before this 64-token block, for the
+            // backward's recompute ([batch, dim, ceil(L / 64), 16] fp32; this lane's 4 states)
+            if (MAXW == kMaxWSmall && a.ckpt != nullptr && t0 % kCkptTokens == 0 && active) {
+                float h0a, h0b, h1a, h1b;
+                f2_split(h[0], h0a, h0b);
+                f2_split(h[1], h1a, h1b);
+                const int64_t nck = (L + kCkptTokens - 1) / kCkptTokens;
+                *reinterpret_cast<float4 *>(a.ckpt + ((b * a.dim + d) * nck + t0 / kCkptTokens) * 16 + n0) =
+                    make_float4(h0a, h0b, h1a, h1b);
+            }
             ok = __all_sync(0xffffffffu, bar_wait(bar(full0 + s), (uint32_t)((k / S) & 1)));
             if (!ok) break;
             // ---- prologue: chunk g of channel c (tokens 8g..8g+7 of the tile)
@@ -1170,12 +1187,6 @@ bool encode3(CUtensorMap *m, const void *base, bool bf16, int64_t L, int64_t mid
 
 bool al16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// Instantiations by compute warps per CTA: the block's warps spread over the
-// SM's four schedulers, each with a quarter of the register file, so 12
-// warps leave 168 registers a thread, 16 warps 128 and 19 warps 96.
-constexpr int kMaxWSmall = 11;
-constexpr int kMaxWMid = 15;
-constexpr int kMaxWLarge = 18;
 constexpr int kSmemLimit = 227 * 1024;
 constexpr int kOneCtaSmem = 116 * 1024;
 
@@ -1250,7 +1261,19 @@ bool scan_tmem_shape_ok(const ScanArgs &a, bool in_bf16, int out_bytes) {
 
 bool scan_tmem_applies(const ScanArgs &a, bool in_bf16, int out_bytes) {
     if (!scan_tmem_shape_ok(a, in_bf16, out_bytes)) return false;
-    if (a.ckpt) return false;
+    // the training forward's saved states: with y, unsplit, no conv front-end, rows
+    // 16-byte aligned, and a layer the 12-warp instantiation covers (the register
+    // engine takes the rest)
+    if (a.ckpt) {
+        if (MS_TMEM_FUSED || a.y == nullptr || a.dsum != nullptr || a.conv_w != nullptr || !al16(a.ckpt)) return false;
+        int dev = 0, sms = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
+            cudaGetLastError();
+            return false;
+        }
+        if (choose_w(a.batch, a.dim, sms, in_bf16 ? 2 : 4) > kMaxWSmall) return false;
+    }
     if (a.conv_w && (a.y == nullptr || a.dsum != nullptr)) return false;  // the conv front-end writes y, unsplit
     // either y (and no Delta sums), or the first pass of a split: no y, the
     // Delta sums and the end states
@@ -1267,6 +1290,7 @@ cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool i
                                  cudaStream_t stream) {
     const int es = in_bf16 ? 2 : 4;
     const int W = choose_w(a.batch, a.dim, num_sms, es);
+    if (a.ckpt != nullptr && W > kMaxWSmall) return cudaErrorInvalidConfiguration;  // only that instantiation saves states
     int S = 3;
     while (S > 2 && TmLayout{W, S, es}.total() > kSmemLimit) --S;
     if (TmLayout{W, S, es}.total() > kSmemLimit) return cudaErrorInvalidConfiguration;

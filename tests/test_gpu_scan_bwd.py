@@ -139,18 +139,23 @@ def test_recomputed_states_match_saved():
     assert torch.equal(y1, y0) and torch.equal(l1, l0)
 
 
-def test_saved_states_are_block_states():
+@pytest.mark.parametrize("L,dtype", [(200, torch.float32), (256, torch.bfloat16), (203, torch.bfloat16)])
+def test_saved_states_are_block_states(L, dtype):
     """ckpt[:, :, k] is the state before token 64 k (the oracle's last_state
-    of the prefix)."""
-    w = syn.scaled(syn.M130, batch=2, dim=24, seqlen=200, in_dtype=torch.float32, seed=600)
+    of the prefix): lengths that are multiples of 8 run the tensor-memory
+    engine, 203 the register engine."""
+    w = syn.scaled(syn.M130, batch=2, dim=24, seqlen=L, in_dtype=dtype, seed=600 + L)
     inp = syn.scan_inputs(w)
     g = {k: v.to(DEV) for k, v in inp.items()}
-    _, _, ck = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+    y, _, ck = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
                                  True)
+    y0, _ = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True)
     torch.cuda.synchronize()
-    assert ck.shape == (2, 24, 4, 16)
+    nck = (L + 63) // 64
+    assert ck.shape == (2, 24, nck, 16)
+    assert torch.equal(y, y0)  # the same engine as the plain forward
     assert float(ck[:, :, 0].abs().max()) == 0.0
-    for k in (1, 2, 3):
+    for k in range(1, nck):
         t = 64 * k
         pre = {n: (v[:, :, :t] if n in ("u", "delta", "z", "B", "C") else v) for n, v in inp.items()}
         _, lr = oracle.scan(f64(pre["u"]), f64(pre["delta"]), f64(pre["A"]), f64(pre["B"]), f64(pre["C"]),

@@ -139,27 +139,37 @@ def test_recomputed_states_match_saved():
     assert torch.equal(y1, y0) and torch.equal(l1, l0)
 
 
-@pytest.mark.parametrize("L,dtype", [(200, torch.float32), (256, torch.bfloat16), (203, torch.bfloat16)])
-def test_saved_states_are_block_states(L, dtype):
+@pytest.mark.parametrize("L,dtype,with_h0", [(200, torch.float32, False), (256, torch.bfloat16, False),
+                                             (203, torch.bfloat16, False), (192, torch.bfloat16, True),
+                                             (195, torch.float32, True)])
+def test_saved_states_are_block_states(L, dtype, with_h0):
     """ckpt[:, :, k] is the state before token 64 k (the oracle's last_state
-    of the prefix): lengths that are multiples of 8 run the tensor-memory
-    engine, 203 the register engine."""
+    of the prefix; ckpt[:, :, 0] is the initial state): lengths that are
+    multiples of 8 run the tensor-memory engine, 203 and 195 the register
+    engine."""
     w = syn.scaled(syn.M130, batch=2, dim=24, seqlen=L, in_dtype=dtype, seed=600 + L)
     inp = syn.scan_inputs(w)
     g = {k: v.to(DEV) for k, v in inp.items()}
+    h0 = 0.3 * torch.randn(2, 24, 16, generator=torch.Generator().manual_seed(L)) if with_h0 else None
+    h0d = None if h0 is None else h0.to(DEV)
     y, _, ck = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
-                                 True)
-    y0, _ = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True)
+                                 True, initial_state=h0d)
+    y0, _ = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                        initial_state=h0d)
     torch.cuda.synchronize()
     nck = (L + 63) // 64
     assert ck.shape == (2, 24, nck, 16)
     assert torch.equal(y, y0)  # the same engine as the plain forward
-    assert float(ck[:, :, 0].abs().max()) == 0.0
+    if h0 is None:
+        assert float(ck[:, :, 0].abs().max()) == 0.0
+    else:
+        assert torch.equal(ck[:, :, 0].cpu(), h0)
     for k in range(1, nck):
         t = 64 * k
         pre = {n: (v[:, :, :t] if n in ("u", "delta", "z", "B", "C") else v) for n, v in inp.items()}
         _, lr = oracle.scan(f64(pre["u"]), f64(pre["delta"]), f64(pre["A"]), f64(pre["B"]), f64(pre["C"]),
-                            f64(pre["D"]), f64(pre["z"]), f64(pre["delta_bias"]), True)
+                            f64(pre["D"]), f64(pre["z"]), f64(pre["delta_bias"]), True,
+                            h0=None if h0 is None else f64(h0))
         check(f64(ck[:, :, k]), lr, torch.float32, f"saved state {k}")
 
 

@@ -99,13 +99,15 @@ def test_head_blocks_and_chunks(b, L, H, G):
     check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
 
 
-@pytest.mark.parametrize("b,L,H,G", [(16, 1024, 7, 1), (8, 2048, 9, 1), (12, 1280, 12, 3)])
-def test_many_items_per_cta(b, L, H, G):
+@pytest.mark.parametrize("b,L,H,G,out_dtype", [(16, 1024, 7, 1, torch.float32), (8, 2048, 9, 1, torch.float32),
+                                                (12, 1280, 12, 3, torch.float32), (16, 1000, 7, 1, torch.bfloat16)])
+def test_many_items_per_cta(b, L, H, G, out_dtype):
     """More work items than SMs, so each persistent CTA walks several items:
     the next item's parameters, C tile, B tile and first x rows arrive while
     the current one computes, and the two warp groups cross item boundaries
     apart. Head blocks of 7 and 9 heads per group leave blocks of 3 or 1 head
-    (one group with fewer heads, or none, in those items)."""
+    (one group with fewer heads, or none, in those items); a ragged last chunk
+    and bf16 y in one case."""
     import os
     from concurrent.futures import ThreadPoolExecutor
     _, inp = _case(b, L, H, G, 100 + H)
@@ -114,7 +116,7 @@ def test_many_items_per_cta(b, L, H, G):
     status = torch.zeros(1, dtype=torch.int32, device=DEV)
     g = {k: v.to(DEV) for k, v in inp.items()}
     y, fs = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
-                       initial_state=s0.to(DEV), dev_status=status)
+                       initial_state=s0.to(DEV), dev_status=status, out_dtype=out_dtype)
     torch.cuda.synchronize()
     assert int(status.item()) == 0
 
@@ -126,7 +128,10 @@ def test_many_items_per_cta(b, L, H, G):
         parts = list(pool.map(part, range(b)))
     yr = np.concatenate([p_[0] for p_ in parts])
     fr = np.concatenate([p_[1] for p_ in parts])
-    check_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} y")
+    if out_dtype == torch.bfloat16:
+        check_out_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} bf16 y")
+    else:
+        check_bf16(f64(y), yr, f"b={b} L={L} H={H} G={G} y")
     check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
 
 

@@ -239,17 +239,35 @@ state_update_stream_kernel(const UpdateArgs a) {
         const TIn *sdl = sx + kTC;
         const TIn *sz = sdl + kTC;
         TOut *sy = reinterpret_cast<TOut *>(st + Sm::kStateBytes + 3 * Sm::kInBytes);
+        // Per-channel scalars are evaluated once per warp instruction stream: lane
+        // (slot, q) takes Delta = softplus(delta + bias) of its slot's channel in
+        // half q % kHalves and the quad reads each half's value by shuffle; after
+        // the state update, lane q < kHalves finishes half q's y (D x, silu(z)).
+        static_assert(kHalves <= 4, "one lane of the quad per half");
+        float dt_mine;
+        {
+            const int hm = q % kHalves;
+            float bias_m = biasv[0];
+#pragma unroll
+            for (int hh = 1; hh < kHalves; ++hh)
+                if (hm == hh) bias_m = biasv[hh];
+            const int clm = (threadIdx.x >> 2) + hm * (kComputeThreads / 4);
+            const float v = (MS_CHECK(a.status, clm < kTC) ? to_f32(sdl[clm]) : 0.0f) + bias_m;
+            dt_mine = a.softplus ? softplus_f(v) : v;
+        }
+        float accs[kHalves], xs[kHalves];
 #pragma unroll
         for (int half = 0; half < kHalves; ++half) {
             const int cl = (threadIdx.x >> 2) + half * (kComputeThreads / 4);  // channel within the tile
             const int64_t d = d0 + cl;
+            const float dt = __shfl_sync(0xffffffffu, dt_mine, (lane & ~3) | half);
+            accs[half] = 0.0f;
+            xs[half] = 0.0f;
             if (!MS_CHECK(a.status, cl < kTC && d < a.dim)) continue;
             float4 hv = *reinterpret_cast<const float4 *>(sstate + cl * 16 + n0);
             float h[4] = {hv.x, hv.y, hv.z, hv.w};
             const float A[4] = {Av[half].x, Av[half].y, Av[half].z, Av[half].w};
             const float x = to_f32(sx[cl]);
-            const float v = to_f32(sdl[cl]) + biasv[half];
-            const float dt = a.softplus ? softplus_f(v) : v;
             const float dx = dt * x;
             const float dtl = dt * kLog2e;
             float acc = 0.0f;
@@ -261,8 +279,21 @@ state_update_stream_kernel(const UpdateArgs a) {
             acc += __shfl_xor_sync(0xffffffffu, acc, 1);
             acc += __shfl_xor_sync(0xffffffffu, acc, 2);
             *reinterpret_cast<float4 *>(sstate + cl * 16 + n0) = make_float4(h[0], h[1], h[2], h[3]);
-            if (q == 0) {
-                float yv = acc + Dv[half] * x;
+            accs[half] = acc;
+            xs[half] = x;
+        }
+        if (q < kHalves) {
+            float acc = accs[0], x = xs[0], Dh = Dv[0];
+#pragma unroll
+            for (int hh = 1; hh < kHalves; ++hh)
+                if (q == hh) {
+                    acc = accs[hh];
+                    x = xs[hh];
+                    Dh = Dv[hh];
+                }
+            const int cl = (threadIdx.x >> 2) + q * (kComputeThreads / 4);
+            if (MS_CHECK(a.status, cl < kTC && d0 + cl < a.dim)) {
+                float yv = acc + Dh * x;
                 if (has_z) yv *= silu_f(to_f32(sz[cl]));
                 Elem<TOut>::store(sy + cl, yv);
             }

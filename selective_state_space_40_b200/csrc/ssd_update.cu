@@ -71,9 +71,11 @@ __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a
                 xv[i] = ldv(xr + p);
             }
         }
+        float part[kRowsPerWarp];
 #pragma unroll
         for (int i = 0; i < kRowsPerWarp; ++i) {
             const int p = p0 + kUW * i;
+            part[i] = 0.0f;
             if (p < P) {
                 float4 s = sv[i];
                 s.x = fmaf(decay, s.x, xv[i] * Bv[0]);
@@ -81,12 +83,36 @@ __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a
                 s.z = fmaf(decay, s.z, xv[i] * Bv[2]);
                 s.w = fmaf(decay, s.w, xv[i] * Bv[3]);
                 *reinterpret_cast<float4 *>(st + (int64_t)p * N) = s;
-                float part = Cv[0] * s.x + Cv[1] * s.y + Cv[2] * s.z + Cv[3] * s.w;
-#pragma unroll
-                for (int off = 16; off >= 1; off >>= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-                if (lane == 0) Elem<TOut>::store(yr + p, part + Dh * xv[i]);
+                part[i] = Cv[0] * s.x + Cv[1] * s.y + Cv[2] * s.z + Cv[3] * s.w;
             }
         }
+        // the rows' readouts summed over the warp by a reduce-scatter: lanes with
+        // bit 4 keep rows 4..7 and pass 0..3 (then bits 3, 2 halve the rest), the
+        // last two levels sum within groups of 4 lanes; lane l ends with the sum
+        // of row r = 4 b4 + 2 b3 + b2 (b = the bits of l)
+        static_assert(kRowsPerWarp == 8, "reduce-scatter of 8 rows over 32 lanes");
+#pragma unroll
+        for (int lvl = 0; lvl < 3; ++lvl) {
+            const int w = 4 >> lvl;                 // values kept after this level
+            const bool hi = (lane >> (4 - lvl)) & 1;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (j < w) {
+                    const float send = hi ? part[j] : part[w + j];
+                    const float keep = hi ? part[w + j] : part[j];
+                    part[j] = keep + __shfl_xor_sync(0xffffffffu, send, 16 >> lvl);
+                }
+            }
+        }
+        part[0] += __shfl_xor_sync(0xffffffffu, part[0], 2);
+        part[0] += __shfl_xor_sync(0xffffffffu, part[0], 1);
+        const int r = ((lane >> 4) & 1) * 4 + ((lane >> 3) & 1) * 2 + ((lane >> 2) & 1);
+        float xr_ = xv[0];
+#pragma unroll
+        for (int i = 1; i < kRowsPerWarp; ++i)
+            if (r == i) xr_ = xv[i];
+        const int pr = p0 + kUW * r;
+        if ((lane & 3) == 0 && pr < P) Elem<TOut>::store(yr + pr, part[0] + Dh * xr_);
     }
 }
 

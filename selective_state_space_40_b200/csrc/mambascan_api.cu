@@ -565,7 +565,7 @@ int mamba_scan_bwd(const void *u, const void *delta, const float *A, const void 
     a.u = u; a.delta = delta; a.z = z; a.B = B; a.C = C;
     a.A = A; a.D = D; a.bias = delta_bias; a.ckpt = ckpt; a.dlast = dlast; a.dout = dout;
     a.du = du; a.ddelta = ddelta; a.dz = z ? dz : nullptr; a.dA = dA; a.dB = dB; a.dC = dC; a.dD = dD;
-    a.dbias = ddelta_bias; a.dh0 = dinitial_state;
+    a.dbias = ddelta_bias; a.dh0 = dinitial_state; a.status = dev_status;
     a.batch = nb; a.dim = nd; a.L = L; a.N = (int)N;
     a.u_sb = dims->u_sb; a.u_sd = dims->u_sd; a.dl_sb = dims->delta_sb; a.dl_sd = dims->delta_sd;
     a.z_sb = dims->z_sb; a.z_sd = dims->z_sd; a.y_sb = dims->y_sb; a.y_sd = dims->y_sd;
@@ -753,7 +753,6 @@ int mamba2_ssd_chunk_cb(const void *B, const void *C, float *cb, const ms_ssd_di
 int mamba2_ssd_state_update(float *state, const void *x, const void *dt, const float *A, const void *B,
                             const void *C, const float *D, const float *dt_bias, int softplus_flag, void *y,
                             const ms_ssd_update_dims *dm, int *dev_status, ms_stream_t stream) {
-    (void)dev_status;
     if (!dm) return MS_ERR_NULL;
     if ((dm->in_dtype != MS_F32 && dm->in_dtype != MS_BF16) || (dm->out_dtype != MS_F32 && dm->out_dtype != MS_BF16))
         return MS_ERR_DTYPE;
@@ -778,6 +777,7 @@ int mamba2_ssd_state_update(float *state, const void *x, const void *dt, const f
         return MS_ERR_SHAPE;
     ms::SsdUpdArgs a{};
     a.state = state; a.x = x; a.dt = dt; a.B = B; a.C = C; a.A = A; a.D = D; a.dt_bias = dt_bias; a.y = y;
+    a.status = dev_status;
     a.batch = dm->batch; a.H = H; a.G = G; a.P = (int)P;
     a.x_sb = dm->x_sb; a.x_sh = dm->x_sh; a.dt_sb = dm->dt_sb; a.B_sb = dm->B_sb; a.B_sg = dm->B_sg;
     a.C_sb = dm->C_sb; a.C_sg = dm->C_sg; a.y_sb = dm->y_sb; a.y_sh = dm->y_sh;

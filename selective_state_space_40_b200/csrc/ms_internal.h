@@ -54,6 +54,7 @@ struct BwdArgs {
     const float *A, *D, *bias, *ckpt, *dlast;
     const void *dout;                   // output dtype, strides y_sb / y_sd
     float *du, *ddelta, *dz, *dA, *dB, *dC, *dD, *dbias, *dh0;
+    int *status;  // device status word of the debug build's bounds checks, or null
     int64_t batch, dim, L;
     int N;
     int64_t u_sb, u_sd, dl_sb, dl_sd, z_sb, z_sd, y_sb, y_sd;
@@ -117,6 +118,7 @@ struct SsdUpdArgs {
     const void *x, *dt, *B, *C;
     const float *A, *D, *dt_bias;
     void *y;
+    int *status;  // device status word of the debug build's bounds checks, or null
     int64_t batch, H, G;
     int P;
     int64_t x_sb, x_sh, dt_sb, B_sb, B_sg, C_sb, C_sg, y_sb, y_sh, st_sb, st_sh;

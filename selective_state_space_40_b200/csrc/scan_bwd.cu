@@ -215,6 +215,9 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
     const int64_t dd = active ? d : 0;
     const int N = a.N;
     const int64_t L = a.L;
+    // debug build: the grid covers exactly batch x ceil(dim / channels per CTA)
+    if (!MS_CHECK(a.status, b < a.batch && N <= 16)) return;
+    [[maybe_unused]] const int64_t grad_elems = a.batch * a.dim * L;  // each dense gradient [batch, dim, L]
     const int n0 = g * 4;
 
     // the lane's 4 states as 2 packed pairs (states n0+2p, n0+2p+1)
@@ -329,7 +332,9 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
             float hv[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-                hv[i] = (active && n0 + i < N) ? __ldg(a.ckpt + ((b * a.dim + d) * nblk + kb) * N + n0 + i) : 0.0f;
+                hv[i] = (active && n0 + i < N && MS_CHECK(a.status, kb >= 0 && kb < nblk))
+                            ? __ldg(a.ckpt + ((b * a.dim + d) * nblk + kb) * N + n0 + i)
+                            : 0.0f;
             h[0] = f2_make(hv[0], hv[1]);
             h[1] = f2_make(hv[2], hv[3]);
         }
@@ -468,7 +473,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                     }
                 }
                 const bool want_dz = has_z && a.dz != nullptr;
-                if (active && t + 1 < L &&
+                if (active && t + 1 < L && MS_CHECK(a.status, t >= 0 && grow + t + 1 < grad_elems) &&
                     ((reinterpret_cast<uintptr_t>(a.ddelta + grow + t) | reinterpret_cast<uintptr_t>(a.du + grow + t) |
                       (want_dz ? reinterpret_cast<uintptr_t>(a.dz + grow + t) : 0)) & 7u) == 0) {
                     *reinterpret_cast<float2 *>(a.ddelta + grow + t) = make_float2(ddv[0], ddv[1]);
@@ -477,7 +482,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 } else if (active) {
 #pragma unroll
                     for (int k = 0; k < 2; ++k) {
-                        if (t + k < L) {
+                        if (t + k < L && MS_CHECK(a.status, t + k >= 0 && grow + t + k < grad_elems)) {
                             a.ddelta[grow + t + k] = ddv[k];
                             a.du[grow + t + k] = duv[k];
                             if (want_dz) a.dz[grow + t + k] = dzv[k];
@@ -504,7 +509,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                     for (int w = 0; w < kBNW; ++w) sum[k] += sm.red[rb][w][j][col];
                 }
                 const int64_t t = ts + 4 * qd;
-                if (n < N) {
+                if (n < N && MS_CHECK(a.status, t >= 0 && b < a.batch)) {
                     float *dst = (isC ? a.dC : a.dB) + (b * N + n) * L + t;
                     if (a.vec_bc && t + 4 <= L) {
                         atomicAdd(reinterpret_cast<float4 *>(dst), make_float4(sum[0], sum[1], sum[2], sum[3]));

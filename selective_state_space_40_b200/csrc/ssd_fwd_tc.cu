@@ -433,10 +433,13 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
             const int pb = it & 1;
             if (it >= 2) ok = bar_wait(bar(kBarParFree + pb), (uint32_t)(((it - 2) >> 1) & 1));
             ok = __all_sync(0xffffffffu, ok && *abort_flag == 0u);
-            const bool valid = ok && T < w.items;
             const int64_t k = T / per_chunk, r0 = T % per_chunk;
             const int64_t b = r0 / (a.G * nhb), g = (r0 / nhb) % a.G, hbk = r0 % nhb;
             const int64_t h0 = g * hpg + hbk * w.hb;
+            // debug build: a ticket below the item count names a chunk of the sequence,
+            // a batch row and a block of its group's heads (an item that fails is dropped)
+            const bool valid = ok && T < w.items &&
+                               MS_CHECK(a.status, k * kQ < L && b < a.batch && g < a.G && hbk * w.hb < hpg);
             const int64_t left = hpg - hbk * w.hb;
             const int nh = valid ? (int)(left < (int64_t)w.hb ? left : (int64_t)w.hb) : 0;
             const int64_t t0 = k * kQ;
@@ -692,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
         // it reads (X' and D x); rows past L are zero-filled
         auto load_x = [&](const ItemDesc &d, int j) {
             const int64_t ts = d.k * kQ + row;
-            const bool in = ts < L;
+            const bool in = ts < L && MS_CHECK(a.status, ts >= 0 && d.b < a.batch && d.h0 + j < a.H);
             const __nv_bfloat16 *src =
                 static_cast<const __nv_bfloat16 *>(a.x) + d.b * a.x_sb + (d.h0 + j) * a.x_sh + (in ? ts : 0) * a.x_sl;
             const uint32_t dst = saddr(X);
@@ -937,7 +940,7 @@ __global__ void __launch_bounds__(kThreads, 1) ssd_fwd_tc_kernel(const SsdArgs a
                         for (int half = 0; half < 2 && ok; ++half) {
                             float ys[32];
                             tmem_ld32(tb + kColSC + (uint32_t)(32 * half), ys);
-                            if (t0 + t < L) {
+                            if (t0 + t < L && MS_CHECK(a.status, b < a.batch && h < a.H)) {
 #pragma unroll
                                 for (int q = 0; q < 4; ++q) {
                                     float yo[8];

@@ -44,6 +44,8 @@ __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a
     const int64_t g = h / (a.H / a.G);
     const int P = a.P;
     constexpr int N = 128;
+    // debug build: the grid covers exactly batch x H, and g names one of the G groups
+    if (!MS_CHECK(a.status, b < a.batch && g < a.G)) return;
     const float v = ldv(static_cast<const TIn *>(a.dt) + b * a.dt_sb + h) + (a.dt_bias ? __ldg(a.dt_bias + h) : 0.0f);
     const float dl = a.softplus ? softplus_f(v) : v;
     const float decay = exp2_mufu(dl * __ldg(a.A + h) * kLog2e);
@@ -112,7 +114,8 @@ __global__ void __launch_bounds__(kUW * 32) ssd_update_kernel(const SsdUpdArgs a
         for (int i = 1; i < kRowsPerWarp; ++i)
             if (r == i) xr_ = xv[i];
         const int pr = p0 + kUW * r;
-        if ((lane & 3) == 0 && pr < P) Elem<TOut>::store(yr + pr, part[0] + Dh * xr_);
+        if ((lane & 3) == 0 && pr < P && MS_CHECK(a.status, r < kRowsPerWarp))
+            Elem<TOut>::store(yr + pr, part[0] + Dh * xr_);
     }
 }
 

@@ -4,9 +4,10 @@ the caller's status word instead of performing an out-of-range access.
 
 * the probe hook: an in-range index writes, an out-of-range one is recorded
   (and skipped), in the debug build; the product build refuses the hook;
-* tiny shapes through every kernel family of the forward path (both scan
-  engines, the sequence split, the conv front-end, the decode step) report
-  no bounds failure and still match the oracle.
+* tiny shapes through every kernel family (both scan engines, the sequence
+  split, the conv front-end, the decode step, the training forward and the
+  backward, the Mamba-2 SSD forward and its decode step) report no bounds
+  failure and still match the oracle.
 """
 import os
 
@@ -17,7 +18,7 @@ import oracle
 from selective_state_space_40_b200 import binding as mb
 from selective_state_space_40_b200 import build as mbuild
 from selective_state_space_40_b200 import synthetic as syn
-from parity_util import check, f64
+from parity_util import check, check_bf16, f64
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -97,3 +98,52 @@ def test_conv_and_decode_clean(debug_lib):
                                   f64(s["C"]), f64(p["D"]), f64(s["z"]), f64(p["delta_bias"]), True)
     check(f64(yd), ydr, torch.float32, "debug decode y")
     check(f64(state), hr, torch.float32, "debug decode state")
+
+
+@pytest.mark.parametrize("L", [128, 130])
+def test_training_forward_and_backward_clean(debug_lib, L):
+    # L = 128: 16-byte dB/dC atomics; L = 130: ragged last block, 4-byte atomics
+    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=L, in_dtype=torch.float32, seed=L)
+    inp = syn.scan_inputs(w)
+    inp["A"] = syn.a_matrix_varied(w.dim, w.dstate, L)
+    gen = torch.Generator().manual_seed(L)
+    dout = torch.randn(w.batch, w.dim, L, generator=gen)
+    dlast = torch.randn(w.batch, w.dim, w.dstate, generator=gen)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    st_fwd, st_bwd = _status(), _status()
+    _, _, ckpt = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                   True, dev_status=st_fwd)
+    gr = mb.scan_bwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True,
+                     dout.to(DEV), dlast=dlast.to(DEV), ckpt=ckpt, dev_status=st_bwd)
+    torch.cuda.synchronize()
+    assert (int(st_fwd.item()), int(st_bwd.item())) == (0, 0)
+    rr = oracle.scan_bwd(*(f64(inp[k]) for k in ("u", "delta", "A", "B", "C", "D", "z", "delta_bias")), True,
+                         f64(dout), dlast=f64(dlast))
+    for k in ("du", "ddelta", "dA", "dB", "dC", "dD", "dz", "ddelta_bias"):
+        check(f64(gr[k]), rr[k], torch.float32, f"debug backward {k}")
+
+
+def test_ssd_forward_and_decode_clean(debug_lib):
+    w = syn.SsdWorkload("dbg", 2, 300, 4, 64, 128, 2, seed=7)
+    inp = syn.ssd_inputs(w)
+    s0 = 0.3 * torch.randn(2, 4, 64, 128, generator=torch.Generator().manual_seed(7))
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    st = _status()
+    y, fs = mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True,
+                       initial_state=s0.to(DEV), dev_status=st)
+    # two decode steps from the forward's final state: tokens 0 and 1 again
+    state = fs.clone()
+    yd = [mb.ssd_state_update(state, g["x"][:, t].contiguous(), g["dt"][:, t].contiguous(), g["A"],
+                              g["B"][:, t].contiguous(), g["C"][:, t].contiguous(), g["D"], g["dt_bias"], True,
+                              dev_status=st) for t in range(2)]
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    A64 = f64(inp["A"])
+    yr, fr = oracle.ssd(f64(inp["x"]), f64(inp["dt"]), A64, f64(inp["B"]), f64(inp["C"]), f64(inp["D"]),
+                        f64(inp["dt_bias"]), True, f64(s0))
+    check_bf16(f64(y), yr, "debug ssd y")
+    check_bf16(f64(fs), fr, "debug ssd final_state")
+    ydr, sr = oracle.ssd(f64(inp["x"])[:, :2], f64(inp["dt"])[:, :2], A64, f64(inp["B"])[:, :2],
+                         f64(inp["C"])[:, :2], f64(inp["D"]), f64(inp["dt_bias"]), True, fr)
+    check_bf16(f64(torch.stack(yd, dim=1)), ydr, "debug ssd decode y")
+    check_bf16(f64(state), sr, "debug ssd decode state")

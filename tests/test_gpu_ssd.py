@@ -135,6 +135,18 @@ def test_many_items_per_cta(b, L, H, G, out_dtype):
     check_bf16(f64(fs), fr, f"b={b} L={L} H={H} G={G} final_state")
 
 
+def test_repeat_is_bitwise_deterministic():
+    """Items go to CTAs by ticket and chunk states pass between them through
+    the workspace, so which CTA computes an item changes from run to run; the
+    arithmetic of each output does not, and two runs agree bit for bit."""
+    _, inp = _case(8, 2048, 9, 1, 77)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    outs = [mb.ssd_fwd(g["x"], g["dt"], g["A"], g["B"], g["C"], g["D"], g["dt_bias"], True) for _ in range(3)]
+    torch.cuda.synchronize()
+    for y, fs in outs[1:]:
+        assert torch.equal(y, outs[0][0]) and torch.equal(fs, outs[0][1])
+
+
 def test_state_in_place_and_in_workspace():
     """initial_state and final_state as one array (updated in place), and no
     final_state (the running state in the workspace): the same y."""
@@ -275,6 +287,27 @@ def test_decode_steps_against_oracle(dtype, P, G):
                             f64(par["D"]), f64(par["dt_bias"]), True, sr)
         check(f64(y), yr[:, 0], dtype, f"ssd decode step {k} y")
     check(f64(sg), sr, dtype, "ssd decode final state")
+
+
+def test_full_decode_b64_every_output():
+    """The decode step at the benchmark's size (64 sequences of the 2.7B-class
+    layer, state [64, 80, 64, 128] fp32, bf16 inputs): three steps from a
+    random state, every y of every step and the whole final state against the
+    oracle's recurrence."""
+    b, H, P, N = 64, 80, 64, 128
+    par = syn.ssd_inputs(syn.SsdWorkload("d", 1, 1, H, P, N, 1))
+    state = 0.1 * torch.randn(b, H, P, N, generator=torch.Generator().manual_seed(11))
+    sg = state.to(DEV)
+    sr = f64(state)
+    for k in range(3):
+        x, dt, B, C = _decode_inputs(b, H, P, 1, 300 + k)
+        y = mb.ssd_state_update(sg, x.to(DEV), dt.to(DEV), par["A"].to(DEV), B.to(DEV), C.to(DEV),
+                                par["D"].to(DEV), par["dt_bias"].to(DEV), True)
+        torch.cuda.synchronize()
+        yr, sr = oracle.ssd(f64(x)[:, None], f64(dt)[:, None], f64(par["A"]), f64(B)[:, None], f64(C)[:, None],
+                            f64(par["D"]), f64(par["dt_bias"]), True, sr)
+        check(f64(y), yr[:, 0], torch.bfloat16, f"b64 decode step {k} y (every element)")
+    check(f64(sg), sr, torch.bfloat16, "b64 decode final state (every element)")
 
 
 def test_decode_steps_equal_chunked_forward():

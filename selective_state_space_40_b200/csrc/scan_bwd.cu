@@ -386,7 +386,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
             }
             // recompute A_bar and h of the sub-chunk, and the pre-gate output q
             f2 hs[2], ab[kSub][2], hh[kSub][2];
-            float dq[kSub], qv[kSub];
+            float dq[kSub], qp[kSub];  // qp: the lane's share of the readout C . h
             hs[0] = f2_make(sm.sub[warp][s][0][lane], sm.sub[warp][s][1][lane]);
             hs[1] = f2_make(sm.sub[warp][s][2][lane], sm.sub[warp][s][3][lane]);
 #pragma unroll
@@ -405,10 +405,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                 }
                 float plo, phi;
                 f2_split(acc, plo, phi);
-                float part = plo + phi;
-                part += __shfl_xor_sync(0xffffffffu, part, 1);
-                part += __shfl_xor_sync(0xffffffffu, part, 2);
-                qv[j] = part + Dd * uv[j];
+                qp[j] = plo + phi;
                 dq[j] = ov[j] * gate[j];
             }
             // adjoint over the sub-chunk, last token first
@@ -452,6 +449,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
             // across the warp's 8 channels)
             reduce_scatter_lanes(ddt, g);
             reduce_scatter_lanes(dus, g);
+            reduce_scatter_lanes(qp, g);  // the readout of tokens 2g, 2g+1 (only dz needs it)
             {
                 // v[2g + k] from compile-time indices
                 auto pick = [&](const float (&v)[kSub], int k) {
@@ -466,7 +464,7 @@ __global__ void __launch_bounds__(kBThreads, 3) scan_bwd_kernel(const BwdArgs a)
                     const float dqk = pick(dq, k);
                     ddv[k] = ddt[k] * tk_sig[j0 + k];
                     duv[k] = fmaf(Dd, dqk, dus[k]);
-                    dzv[k] = pick(ov, k) * pick(qv, k) * tk_gp[j0 + k];
+                    dzv[k] = pick(ov, k) * fmaf(Dd, pick(uv, k), qp[k]) * tk_gp[j0 + k];
                     if (active && t + k < L) {
                         dDacc = fmaf(dqk, pick(uv, k), dDacc);
                         dbacc += ddv[k];

@@ -251,11 +251,6 @@ static bool plan_valid(const ms_scan_plan *p) {
            (q == 0 || q == 2 || q == 4 || q == 8);
 }
 
-// Exponentials on the FMA-pipe polynomial in the tensor-memory kernel, in
-// eighths: bf16 inputs balance the MUFU and FMA pipes; fp32 inputs take every
-// exponential from the polynomial (unbiased near 1, see ms_device.cuh).
-constexpr int kTmemPoly8Bf16 = 0;
-
 // The plan a call without an explicit plan runs: the tensor-memory kernel
 // where it applies (sizes, strides, alignment and outputs), else the
 // register-prefetch kernel with its own heuristic.
@@ -266,7 +261,7 @@ static ms::ScanPlan auto_plan_args(const ms::ScanArgs &a, bool in_bf16, bool out
         pl.engine = MS_ENGINE_TMEM;
         pl.lanes_per_channel = 4;
         pl.chunks_per_lane = 1;
-        pl.poly8 = in_bf16 ? kTmemPoly8Bf16 : 8;
+        pl.poly8 = in_bf16 ? ms::kTmemPoly8Bf16 : 8;
     }
     return pl;
 }

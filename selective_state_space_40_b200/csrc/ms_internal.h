@@ -48,6 +48,12 @@ cudaError_t launch_carry_combine(const float *E, const float *dsum, const float 
 // each block from its saved state).
 constexpr int kCkptTokens = 64;
 
+// The automatic plan of the tensor-memory kernel: exponentials on the FMA-pipe
+// polynomial, in eighths. bf16 inputs take every one on MUFU (the polynomial
+// costs more issue than it frees); fp32 inputs take every one from the
+// polynomial (unbiased near 1, see ms_device.cuh).
+constexpr int kTmemPoly8Bf16 = 0;
+
 // Arguments of the backward kernel (gradients are fp32, dense).
 struct BwdArgs {
     const void *u, *delta, *z, *B, *C;  // input dtype

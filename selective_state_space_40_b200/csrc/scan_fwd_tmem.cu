@@ -381,8 +381,11 @@ __device__ __forceinline__ void store8_in(T *p, bool vec, const float (&v)[8]) {
 
 
 // YOUT false: the first pass of a sequence split (no y; the end state and
-// the sum of Delta over the tokens per channel instead).
-template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false>
+// the sum of Delta over the tokens per channel instead). CKPT: the training
+// forward of a layer wider than the 12-warp instantiation covers (that one
+// saves states whenever it is given a buffer; in the wider ones the store
+// costs the plain forward's state loop spills, so they have their own).
+template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false, bool CKPT = false>
 __global__ void __launch_bounds__(32 * (MAXW + 1), 1)
 scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, const int W, const int S) {
     extern __shared__ __align__(1024) unsigned char smem[];
@@ -805,10 +808,10 @@ scan_fwd_tmem_kernel(const ScanArgs a, const __grid_constant__ TmMaps maps, cons
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
             const int s = k % S, vb = k & 1;
             const int64_t t0 = (int64_t)k * kT;
-            // Training (the 12-warp instantiation only; wider layers' training forwards
-            // take the register engine): the state before this 64-token block, for the
-            // backward's recompute ([batch, dim, ceil(L / 64), 16] fp32; this lane's 4 states)
-            if (MAXW == kMaxWSmall && a.ckpt != nullptr && t0 % kCkptTokens == 0 && active) {
+            // Training (the 12-warp instantiation, and the CKPT instantiations of the
+            // wider ones): the state before this 64-token block, for the backward's
+            // recompute ([batch, dim, ceil(L / 64), 16] fp32; this lane's 4 states)
+            if ((MAXW == kMaxWSmall || CKPT) && a.ckpt != nullptr && t0 % kCkptTokens == 0 && active) {
                 float h0a, h0b, h1a, h1b;
                 f2_split(h[0], h0a, h0b);
                 f2_split(h[1], h1a, h1b);
@@ -1205,12 +1208,12 @@ int choose_w(int64_t batch, int64_t dim, int num_sms, int in_bytes) {
     return (int)w;
 }
 
-template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false>
+template <typename TIn, typename TOut, int POLY8, int MAXW, bool YOUT, bool CONV = false, bool CKPT = false>
 cudaError_t launch_tm(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaStream_t stream) {
     const TmLayout lay{W, S, (int)sizeof(TIn)};
     static SmemOptIn opt_in;
     cudaError_t e = opt_in.ensure(
-        reinterpret_cast<const void *>(scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV>), kSmemLimit);
+        reinterpret_cast<const void *>(scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV, CKPT>), kSmemLimit);
     if (e != cudaSuccess) return e;
     const int64_t blocks = a.batch * ((a.dim + lay.cwc() - 1) / lay.cwc());
     if (blocks <= 0) return cudaSuccess;
@@ -1218,7 +1221,7 @@ cudaError_t launch_tm(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaS
     // At least half of an SM's shared memory: one CTA per SM, so the CTA's
     // 512 tensor-memory columns are always free when it allocates them.
     const int smem = lay.total() > kOneCtaSmem ? lay.total() : kOneCtaSmem;
-    scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV>
+    scan_fwd_tmem_kernel<TIn, TOut, POLY8, MAXW, YOUT, CONV, CKPT>
         <<<(unsigned)blocks, 32 * (W + 1), smem, stream>>>(a, maps, W, S);
     return cudaGetLastError();
 }
@@ -1228,6 +1231,15 @@ cudaError_t launch_w(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaSt
     if (W <= kMaxWSmall) return launch_tm<TIn, TOut, POLY8, kMaxWSmall, YOUT, CONV>(a, maps, W, S, stream);
     if (W <= kMaxWMid) return launch_tm<TIn, TOut, POLY8, kMaxWMid, YOUT, CONV>(a, maps, W, S, stream);
     return launch_tm<TIn, TOut, POLY8, kMaxWLarge, YOUT, CONV>(a, maps, W, S, stream);
+}
+
+// Training forward of a layer wider than the 12-warp instantiation covers
+// (the automatic plan's exponentials only: every one on MUFU for bf16 inputs,
+// on the FMA-pipe polynomial for fp32).
+template <typename TIn, typename TOut, int POLY8>
+cudaError_t launch_ckpt_wide(const ScanArgs &a, const TmMaps &maps, int W, int S, cudaStream_t stream) {
+    if (W <= kMaxWMid) return launch_tm<TIn, TOut, POLY8, kMaxWMid, true, false, true>(a, maps, W, S, stream);
+    return launch_tm<TIn, TOut, POLY8, kMaxWLarge, true, false, true>(a, maps, W, S, stream);
 }
 
 // First pass of a sequence split (no y): the exponentials as for y.
@@ -1262,17 +1274,9 @@ bool scan_tmem_shape_ok(const ScanArgs &a, bool in_bf16, int out_bytes) {
 bool scan_tmem_applies(const ScanArgs &a, bool in_bf16, int out_bytes) {
     if (!scan_tmem_shape_ok(a, in_bf16, out_bytes)) return false;
     // the training forward's saved states: with y, unsplit, no conv front-end, rows
-    // 16-byte aligned, and a layer the 12-warp instantiation covers (the register
-    // engine takes the rest)
+    // 16-byte aligned
     if (a.ckpt) {
         if (MS_TMEM_FUSED || a.y == nullptr || a.dsum != nullptr || a.conv_w != nullptr || !al16(a.ckpt)) return false;
-        int dev = 0, sms = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) {
-            cudaGetLastError();
-            return false;
-        }
-        if (choose_w(a.batch, a.dim, sms, in_bf16 ? 2 : 4) > kMaxWSmall) return false;
     }
     if (a.conv_w && (a.y == nullptr || a.dsum != nullptr)) return false;  // the conv front-end writes y, unsplit
     // either y (and no Delta sums), or the first pass of a split: no y, the
@@ -1290,7 +1294,6 @@ cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool i
                                  cudaStream_t stream) {
     const int es = in_bf16 ? 2 : 4;
     const int W = choose_w(a.batch, a.dim, num_sms, es);
-    if (a.ckpt != nullptr && W > kMaxWSmall) return cudaErrorInvalidConfiguration;  // only that instantiation saves states
     int S = 3;
     while (S > 2 && TmLayout{W, S, es}.total() > kSmemLimit) --S;
     if (TmLayout{W, S, es}.total() > kSmemLimit) return cudaErrorInvalidConfiguration;
@@ -1315,6 +1318,16 @@ cudaError_t launch_scan_fwd_tmem(const ScanArgs &a, const ScanPlan &plan, bool i
         }
         return out_bf16 ? launch_w<float, __nv_bfloat16, 8, true, true>(a, maps, W, S, stream)
                         : launch_w<float, float, 8, true, true>(a, maps, W, S, stream);
+    }
+    if (a.ckpt != nullptr && W > kMaxWSmall) {
+        // the training forward of a wider layer: its own instantiations, the automatic plan
+        if (poly8 != (in_bf16 ? kTmemPoly8Bf16 : 8)) return cudaErrorInvalidValue;
+        if (in_bf16) {
+            return out_bf16 ? launch_ckpt_wide<__nv_bfloat16, __nv_bfloat16, kTmemPoly8Bf16>(a, maps, W, S, stream)
+                            : launch_ckpt_wide<__nv_bfloat16, float, kTmemPoly8Bf16>(a, maps, W, S, stream);
+        }
+        return out_bf16 ? launch_ckpt_wide<float, __nv_bfloat16, 8>(a, maps, W, S, stream)
+                        : launch_ckpt_wide<float, float, 8>(a, maps, W, S, stream);
     }
     if (a.y == nullptr)
         return in_bf16 ? launch_pass1<__nv_bfloat16>(a, maps, W, S, poly8, stream)

@@ -173,6 +173,32 @@ def test_saved_states_are_block_states(L, dtype, with_h0):
         check(f64(ck[:, :, k]), lr, torch.float32, f"saved state {k}")
 
 
+@pytest.mark.parametrize("dim,dtype", [(8192, torch.bfloat16), (10240, torch.bfloat16), (8192, torch.float32)])
+def test_wide_layer_training_forward(dim, dtype):
+    """Layers wider than one 12-warp CTA per SM covers (2 x 8192 channels: 14
+    compute warps per CTA; 2 x 10240: 18) save their states in the wider
+    instantiations of the tensor-memory kernel: y equals the plain forward's
+    bit for bit (the same engine and arithmetic), and every saved state is the
+    oracle's state before its 64-token block."""
+    L = 192
+    w = syn.scaled(syn.M130, batch=2, dim=dim, seqlen=L, in_dtype=dtype, seed=dim)
+    inp = syn.scan_inputs(w)
+    inp["A"] = syn.a_matrix_varied(dim, 16, dim)
+    g = {k: v.to(DEV) for k, v in inp.items()}
+    y, last, ck = mb.scan_fwd_train(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"],
+                                    True)
+    y0, l0 = mb.scan_fwd(g["u"], g["delta"], g["A"], g["B"], g["C"], g["D"], g["z"], g["delta_bias"], True)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y0) and torch.equal(last, l0)
+    assert float(ck[:, :, 0].abs().max()) == 0.0
+    for k in (1, 2):
+        t = 64 * k
+        pre = {n: (v[:, :, :t] if n in ("u", "delta", "z", "B", "C") else v) for n, v in inp.items()}
+        _, lr = oracle.scan(f64(pre["u"]), f64(pre["delta"]), f64(pre["A"]), f64(pre["B"]), f64(pre["C"]),
+                            f64(pre["D"]), f64(pre["z"]), f64(pre["delta_bias"]), True)
+        check(f64(ck[:, :, k]), lr, torch.float32, f"wide layer saved state {k}")
+
+
 def test_no_dinitial_requested():
     w = syn.scaled(syn.M130, batch=1, dim=32, seqlen=70, in_dtype=torch.float32, seed=700)
     inp, dout, dlast, h0 = _grads_inputs(w, 23)

@@ -100,10 +100,12 @@ def test_conv_and_decode_clean(debug_lib):
     check(f64(state), hr, torch.float32, "debug decode state")
 
 
-@pytest.mark.parametrize("L", [128, 130])
-def test_training_forward_and_backward_clean(debug_lib, L):
-    # L = 128: 16-byte dB/dC atomics; L = 130: ragged last block, 4-byte atomics
-    w = syn.scaled(syn.M130, batch=2, dim=40, seqlen=L, in_dtype=torch.float32, seed=L)
+@pytest.mark.parametrize("L,dim", [(128, 40), (130, 40), (128, 10240)])
+def test_training_forward_and_backward_clean(debug_lib, L, dim):
+    # L = 128: 16-byte dB/dC atomics; L = 130: ragged last block, 4-byte atomics;
+    # dim 10240 (2 rows): a wide saved-state instantiation of the forward (more
+    # than 12 warps per CTA)
+    w = syn.scaled(syn.M130, batch=2, dim=dim, seqlen=L, in_dtype=torch.float32, seed=L)
     inp = syn.scan_inputs(w)
     inp["A"] = syn.a_matrix_varied(w.dim, w.dstate, L)
     gen = torch.Generator().manual_seed(L)
